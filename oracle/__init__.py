@@ -1,0 +1,128 @@
+"""fp64 CPU oracle for the bounded-decay gated delta rule.
+
+TEST INFRASTRUCTURE ONLY. The test suite, the smoke check and the benchmark's
+CPU-baseline leg are the only callers. The CUDA library and its Python binding
+never import this package, and the two share no code: inputs reach both sides
+from the seeded generators in ``workloads.py`` and nothing else.
+
+The arithmetic lives in ``kda_oracle.c`` (plain C, double precision, the
+token-by-token recurrence written in the order of the defining equations).
+This module only converts arrays to contiguous fp64 (an exact widening for
+bf16 and fp32 inputs) and calls it.
+
+Functions and the passages they follow:
+
+* :func:`bounded_decay` -- "Kimi K3: Bounded Decay and Delta Memory",
+  Formula and conventions, eq. 5: ``g = g_min * sigmoid(exp(A) * z)``,
+  ``alpha = exp(g)``.
+* :func:`scan` -- same page, eq. 1 (fade, correct, then read the updated
+  state), with the contract table of that page: q, k ``[B,T,H,K]``, v
+  ``[B,T,H,V]``, alpha ``[B,T,H,K]``, beta ``[B,T,H]``, state ``[B,H,K,V]``
+  (key-by-value), omitted initial state means zeros, T = 0 returns the input
+  state. Packed variable-length sequences follow the ``cu_seqlens`` argument
+  of the production kernel call excerpted on the "Kept memory" page.
+
+Parity status: both functions are pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py`` (printed toy outputs, closed forms, the
+independent product form of the "KDA cheat sheet", exact rational brute force
+and the chunkwise form of the same cheat sheet).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        i64 = ctypes.c_int64
+        lib.kda_oracle_bounded_decay.argtypes = [dp, dp, ctypes.c_double, i64, i64, i64, i64, dp, dp]
+        lib.kda_oracle_bounded_decay.restype = None
+        lib.kda_oracle_scan.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.POINTER(i64), i64,
+                                        i64, i64, i64, i64, i64, dp, dp, ctypes.c_int]
+        lib.kda_oracle_scan.restype = ctypes.c_int
+        lib.kda_oracle_max_threads.argtypes = []
+        lib.kda_oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Contiguous fp64 copy of a numpy array or a (CPU or CUDA) torch tensor."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor: widen in torch (bf16 -> fp64 is exact)
+        import torch
+        x = x.detach().to(device="cpu", dtype=torch.float64).contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if a is not None else None
+
+
+def max_threads() -> int:
+    """OpenMP threads the oracle uses by default (``OMP_NUM_THREADS`` or all cores)."""
+    return int(_load().kda_oracle_max_threads())
+
+
+def bounded_decay(z, A_log, g_min: float = -5.0, return_log: bool = False):
+    """alpha (and optionally g) for logits ``z [B,T,H,K]`` and per-head ``A_log [H]``."""
+    lib = _load()
+    z = _f64(z)
+    A = _f64(A_log)
+    if z.ndim != 4 or A.shape != (z.shape[2],):
+        raise ValueError("z must be [B,T,H,K] and A_log [H]")
+    B, T, H, K = z.shape
+    alpha = np.empty_like(z)
+    g = np.empty_like(z)
+    lib.kda_oracle_bounded_decay(_ptr(z), _ptr(A), float(g_min), B, T, H, K, _ptr(alpha), _ptr(g))
+    return (alpha, g) if return_log else alpha
+
+
+def scan(q, k, v, alpha, beta, initial_state=None, cu_seqlens=None, n_threads: int = 0):
+    """Token-by-token scan. Returns ``(o [B,T,H,V], final_state [N,H,K,V])`` in fp64.
+
+    ``N`` is ``B``, or the number of packed sequences when ``cu_seqlens`` (int
+    offsets, length ``N+1``) is given, in which case ``B`` must be 1.
+    """
+    lib = _load()
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    if q.ndim != 4 or k.shape != q.shape or alpha.shape != q.shape:
+        raise ValueError("q, k, alpha must share the shape [B,T,H,K]")
+    B, T, H, K = q.shape
+    if v.ndim != 4 or v.shape[:3] != (B, T, H):
+        raise ValueError("v must be [B,T,H,V]")
+    V = v.shape[3]
+    if beta.shape != (B, T, H):
+        raise ValueError("beta must be [B,T,H]")
+    cu = None
+    N = B
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+        N = cu.shape[0] - 1
+    s0 = None
+    if initial_state is not None:
+        s0 = _f64(initial_state)
+        if s0.shape != (N, H, K, V):
+            raise ValueError(f"initial_state must be [{N},{H},{K},{V}]")
+    o = np.zeros((B, T, H, V), dtype=np.float64)
+    sf = np.zeros((N, H, K, V), dtype=np.float64)
+    cu_ptr = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)) if cu is not None else None
+    rc = lib.kda_oracle_scan(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(s0),
+                             cu_ptr, N if cu is not None else 0, B, T, H, K, V,
+                             _ptr(o), _ptr(sf), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle scan rejected its arguments")
+    return o, sf
