@@ -1,0 +1,501 @@
+"""Benchmark of the KDA hot path on B200: prefill tokens/s and decode state GB/s.
+
+Workloads (H=96, K=V=128, synthetic seeded inputs from ``workloads.py``):
+
+* prefill -- B=1, T=4096, bf16 q/k/v, fp32 decay logits (z ~ N(0,2)), fp32 beta,
+  zero initial state, fp32 final state. One step = the gate kernel (logits ->
+  alpha) plus the chunked prefill (-> o, final_state). ``value`` is tokens/s.
+* decode -- B=64 kept 128x128 fp32 states (402.7 MB), bf16 q/k/v, z ~ N(0,1).
+  One step = the gate kernel plus the in-place decode step. Reported in the
+  ``decode`` object as state GB/s (2*4*K*V*B*H bytes per step) and steps/s.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronise, CUDA events on the stream the kernels are launched on,
+max over ranks. Every input set is larger than the 126 MB L2, so no flush is
+inserted between steps. ``e2e`` repeats the measurement through the public
+API with pinned host buffers: each step copies its inputs host->device and
+reads its results device->host inside the timed region.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload and prints the same line with ``"impl": "reference"``.
+
+Multi-GPU (``torchrun``): every rank runs its own copy of the workload (the
+(sequence, head) units are independent, so there is no collective on the data
+path); ``value`` = units of all ranks / max-over-ranks time, ``scaling`` weak.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "KDA prefill tokens/s & decode state GB/s (H96,K=V=128); % of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------------------------
+# Algorithmic work per launch (the units the roofline fractions are computed from)
+# ------------------------------------------------------------------------------------------------
+
+def prefill_bytes(B, T, H, K, V, n_states_in, n_states_out, es=2):
+    """Minimum HBM bytes of one prefill launch: read q, k (K each), v (V) in the input dtype,
+    alpha (K fp32) and beta (fp32) per token-head, write o (V); read/write the fp32 states."""
+    per_tok_head = 2 * K * es + V * es + 4 * K + 4 + V * es
+    return B * T * H * per_tok_head + (n_states_in + n_states_out) * H * K * V * 4
+
+
+def prefill_flops(B, T, H, K, V, C=64):
+    """Dense chunk-form FLOPs at a fixed C = 64 per token-head: 6CK + 4CV + 6KV + C^2/3."""
+    return B * T * H * (6 * C * K + 4 * C * V + 6 * K * V + C * C / 3.0)
+
+
+def decode_bytes(B, H, K, V, es=2):
+    """Per step: state read + write (8KV), q, k, v, o in the input dtype, alpha fp32, beta fp32."""
+    return B * H * (8 * K * V + (2 * K + 2 * V) * es + 4 * K + 4)
+
+
+def decode_state_bytes(B, H, K, V):
+    return B * H * 2 * 4 * K * V
+
+
+def gate_bytes(n_elems, es_in=4, es_out=4):
+    return n_elems * (es_in + es_out)
+
+
+# ------------------------------------------------------------------------------------------------
+# Environment helpers
+# ------------------------------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    """One process per GPU under torchrun; returns (rank, world, local_rank)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    if n_gpus != world and world > 1 and rank == 0:
+        print(f"warning: --gpus {n_gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, local_ms: float, world: int) -> tuple:
+    """Whole-job throughput of replicated work: every rank processes `units_per_rank` units in
+    `local_ms`; the job takes the slowest rank's time. Returns (units/s, max ms)."""
+    slowest = max_over_ranks(local_ms, world)
+    return units_per_rank * world / (slowest / 1e3), slowest
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+
+def timed_loop(step_fns, steps, warmup, world, stream, sampler=None):
+    """Runs each step fn once per iteration. Returns (total ms over `steps`, per-fn avg ms).
+
+    Each step fn is bracketed by its own events (recorded on `stream`, the stream the
+    kernels are launched on), so the per-kernel averages come from the same timed run."""
+    for _ in range(warmup):
+        for fn in step_fns:
+            fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    n = len(step_fns)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s in range(steps):
+            ev[s][0].record(stream)
+            for i, fn in enumerate(step_fns):
+                fn()
+                ev[s][i + 1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    per_fn = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps for i in range(n)]
+    barrier(world)
+    return total, per_fn
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
+    w = W.PREFILL
+    d = W.make_scan_inputs(w)
+    B, T, H, K, V = w.B, w.T, w.H, w.K, w.V
+    g = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in d.items()}
+    alpha = torch.empty(B, T, H, K, device=dev, dtype=torch.float32)
+    o = torch.empty(B, T, H, V, device=dev, dtype=torch.bfloat16)
+    sf = torch.empty(B, H, K, V, device=dev, dtype=torch.float32)
+    ws_bytes = kda.prefill_workspace_bytes(B, T, H, K, V, 0, torch.bfloat16)
+    ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
+
+    def gate_fn():
+        kda.bounded_decay(g["z"], g["A_log"], w.g_min, out=alpha)
+
+    def prefill_fn():
+        kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], None, out=o, final_state=sf, workspace=ws)
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    total_ms, (gate_ms, pre_ms) = timed_loop([gate_fn, prefill_fn], args.steps, args.warmup, world, stream, sampler)
+    value, total_ms = weak_scaling_value(B * T * args.steps, total_ms, world)
+    ms_per_step = total_ms / args.steps
+    tokens = B * T * world
+    pb = prefill_bytes(B, T, H, K, V, 0, 1)
+    achieved = pb / (pre_ms / 1e3) / 1e9
+    flops = prefill_flops(B, T, H, K, V)
+    tflops = flops / (pre_ms / 1e3) / 1e12
+    res = {
+        "value": value, "ms_per_step": ms_per_step, "workload": w, "clocks": sampler.summary() if sampler else None,
+        "kernels_ms": {"bounded_decay": gate_ms, "prefill": pre_ms},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "kernel": "kda_prefill",
+                     "bytes_per_launch": pb, "ms_per_launch": pre_ms, "peak_source": f"{peak_src} hbm_gbs",
+                     "tensor": {"tflops_at_C64_formula": tflops, "peak": bf16_peak,
+                                "frac": tflops / bf16_peak, "flops_per_launch": flops}},
+        "gpu_launches": 2 * args.steps,
+    }
+    if args.no_e2e:
+        return res
+    # e2e: pinned host inputs -> device, gate + prefill, o and final state -> pinned host
+    host = {n: d[n].pin_memory() for n in ("q", "k", "v", "z", "A_log", "beta")}
+    o_host = torch.empty(B, T, H, V, dtype=torch.bfloat16).pin_memory()
+    sf_host = torch.empty(B, H, K, V, dtype=torch.float32).pin_memory()
+    dev_in = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * sf_host.element_size()
+
+    def e2e_fn():
+        for n, x in host.items():
+            dev_in[n].copy_(x, non_blocking=True)
+        kda.bounded_decay(dev_in["z"], dev_in["A_log"], w.g_min, out=alpha)
+        kda.prefill(dev_in["q"], dev_in["k"], dev_in["v"], alpha, dev_in["beta"], None, out=o,
+                    final_state=sf, workspace=ws)
+        o_host.copy_(o, non_blocking=True)
+        sf_host.copy_(sf, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_total, _ = timed_loop([e2e_fn], e2e_steps, max(1, args.warmup // 2), world, stream)
+    e2e_total = max_over_ranks(e2e_total, world)
+    res["e2e"] = {"value": tokens / (e2e_total / e2e_steps / 1e3), "unit": "tokens/s",
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return res
+
+
+def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
+    dw = W.DECODE
+    prm = W.make_decode_params(dw)
+    state = prm["state"].to(dev)
+    A_dec = prm["A_log"].to(dev)
+    n_sets = 4
+    sets = [{n: x.to(dev) for n, x in W.make_decode_step(dw, s).items()} for s in range(n_sets)]
+    a_dec = torch.empty(dw.B, dw.H, dw.K, device=dev)
+    o_dec = torch.empty(dw.B, dw.H, dw.V, device=dev, dtype=torch.bfloat16)
+    it = {"i": 0}
+
+    def dgate_fn():
+        s = sets[it["i"] % n_sets]
+        kda.bounded_decay(s["z"], A_dec, dw.g_min, out=a_dec)
+
+    def dstep_fn():
+        s = sets[it["i"] % n_sets]
+        kda.decode_step(s["q"], s["k"], s["v"], a_dec, s["beta"], state, out=o_dec)
+        it["i"] += 1
+
+    dsteps = max(args.steps, 20)
+    dsampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    d_total, (dg_ms, dk_ms) = timed_loop([dgate_fn, dstep_fn], dsteps, args.warmup, world, stream, dsampler)
+    sbytes = decode_state_bytes(dw.B, dw.H, dw.K, dw.V)
+    d_bps, d_total = weak_scaling_value(sbytes * dsteps, d_total, world)
+    d_ms = d_total / dsteps
+    dbytes = decode_bytes(dw.B, dw.H, dw.K, dw.V)
+    d_achieved = dbytes / (dk_ms / 1e3) / 1e9
+    res = {
+        "workload": dw.name, "value": d_bps / 1e9, "unit": "GB/s (state)",
+        "steps_per_s": 1e3 / d_ms, "ms_per_step": d_ms, "steps": dsteps, "gpu_launches": 2 * dsteps,
+        "kernels_ms": {"bounded_decay": dg_ms, "decode_step": dk_ms},
+        "roofline": {"bound": "hbm", "achieved": d_achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": d_achieved / hbm, "traffic": None, "kernel": "kda_decode_step",
+                     "bytes_per_launch": dbytes, "ms_per_launch": dk_ms, "peak_source": f"{peak_src} hbm_gbs"},
+        "clocks": dsampler.summary() if dsampler is not None else None,
+    }
+    if args.no_e2e:
+        return res
+    hostd = [{n: x.pin_memory() for n, x in W.make_decode_step(dw, s).items()} for s in range(n_sets)]
+    devd = {n: torch.empty_like(x, device=dev) for n, x in hostd[0].items()}
+    o_dec_host = torch.empty(dw.B, dw.H, dw.V, dtype=torch.bfloat16).pin_memory()
+    dh2d = sum(x.numel() * x.element_size() for x in hostd[0].values())
+    dd2h = o_dec_host.numel() * o_dec_host.element_size()
+
+    def de2e_fn():
+        s = hostd[it["i"] % n_sets]
+        for n, x in s.items():
+            devd[n].copy_(x, non_blocking=True)
+        kda.bounded_decay(devd["z"], A_dec, dw.g_min, out=a_dec)
+        kda.decode_step(devd["q"], devd["k"], devd["v"], a_dec, devd["beta"], state, out=o_dec)
+        o_dec_host.copy_(o_dec, non_blocking=True)
+        it["i"] += 1
+
+    de_total, _ = timed_loop([de2e_fn], dsteps, args.warmup, world, stream)
+    de_total = max_over_ranks(de_total, world)
+    res["e2e"] = {"value": sbytes * world / (de_total / dsteps / 1e3) / 1e9, "unit": "GB/s (state)",
+                  "h2d_bytes_per_step": dh2d, "d2h_bytes_per_step": dd2h}
+    return res
+
+
+def gpu_arm(args, rank, world, local):
+    import gated_delta_rule_bounded_b200 as kda
+    kda.load_library()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    bf16_peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    pre = dec = None
+    if args.workload in ("all", "prefill"):
+        pre = prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src)
+        torch.cuda.empty_cache()
+    if args.workload in ("all", "decode"):
+        dec = decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
+    cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if pre is None:  # decode-only profiling run
+        return {"metric": METRIC, "workload_only": "decode", "decode": dec}
+    w = pre["workload"]
+    line = {
+        "metric": METRIC,
+        "value": pre["value"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": pre["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; no dataset)",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "K": w.K, "V": w.V, "g_min": w.g_min,
+                   "z_std": w.z_std, "initial_state": "zeros", "step": "bounded_decay + prefill",
+                   "l2": "inputs larger than L2 (q/k/v/z/alpha ~ 0.9 GB); no flush",
+                   "parallelism": f"replica per GPU x{world}"},
+        "roofline": pre["roofline"],
+        "kernels_ms": pre["kernels_ms"],
+        "e2e": pre.get("e2e"),
+        "gpu_launches": pre["gpu_launches"],
+        "clocks": pre["clocks"],
+    }
+    if dec is not None:
+        line["decode"] = dec
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_prefill_sample(n_heads, inputs=None, threads=0):
+    """Times the fp64 oracle (gate + scan) on `n_heads` heads of the prefill workload.
+    Returns (seconds, tokens-equivalent of the full workload processed)."""
+    import oracle
+    w = W.PREFILL
+    d = inputs if inputs is not None else W.make_scan_inputs(w)
+    hs = list(range(n_heads))
+    sub = {n: d[n][:, :, hs] for n in ("q", "k", "v", "z", "beta")}
+    t0 = time.perf_counter()
+    alpha = oracle.bounded_decay(sub["z"], d["A_log"][hs], w.g_min)
+    oracle.scan(sub["q"], sub["k"], sub["v"], alpha, sub["beta"], None, None, n_threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, w.B * w.T * n_heads / w.H
+
+
+def cpu_baseline(args):
+    import oracle
+    oracle._load()
+    cores = oracle.max_threads()
+    d = W.make_scan_inputs(W.PREFILL)
+    n_heads = max(1, min(W.PREFILL.H, args.cpu_heads or 4 * cores))
+    dt, tok = oracle_prefill_sample(n_heads, d)
+    return {"value": tok / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"prefill workload, {n_heads} of {W.PREFILL.H} heads, full T={W.PREFILL.T}, "
+                      f"fp64 gate + token-by-token scan; {dt:.2f} s; tokens/s scaled to all heads"}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    oracle._load()
+    cores = oracle.max_threads()
+    d = W.make_scan_inputs(W.PREFILL)
+    n_heads = max(1, min(W.PREFILL.H, args.cpu_heads or cores))
+    for _ in range(args.warmup):
+        oracle_prefill_sample(n_heads, d)
+    times, tok = [], 0.0
+    for _ in range(args.steps):
+        dt, tok = oracle_prefill_sample(n_heads, d)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = tok / (ms / 1e3)
+    sample = (f"each step: prefill workload, {n_heads} of {W.PREFILL.H} heads, full T={W.PREFILL.T}, "
+              f"fp64 gate + token-by-token scan on {cores} threads; tokens/s scaled to all heads")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; no dataset)",
+        "config": {"workload": W.PREFILL.name, "B": W.PREFILL.B, "T": W.PREFILL.T, "H": W.PREFILL.H,
+                   "K": W.PREFILL.K, "V": W.PREFILL.V, "g_min": W.PREFILL.g_min},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--cpu-heads", type=int, default=0, help="heads in the oracle sample (0: auto)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
+                    help="prefill/decode alone (profiling runs); the JSON line needs 'all'")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end legs")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = reference_arm(args, rank, world)
+        else:
+            line = gpu_arm(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

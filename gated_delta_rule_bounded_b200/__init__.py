@@ -1,0 +1,263 @@
+"""Bounded-decay gated delta rule (the Kimi Delta Attention scan) on B200.
+
+A thin ctypes binding over ``libkda.so``, whose C ABI is declared in
+``include/kda.h``. Every step of the computation runs in the library's CUDA
+kernels; this module only allocates outputs with torch, reads strides and
+passes pointers and the current CUDA stream. There is no CPU fallback: the
+functions raise if the library is missing or a tensor is not on a CUDA device.
+
+* :func:`bounded_decay` -- ``alpha = exp(g_min * sigmoid(exp(A) * z))``
+  ("Kimi K3: Bounded Decay and Delta Memory", eq. 5).
+* :func:`prefill` -- the scan over whole sequences, returning ``(o, final_state)``
+  (same page, eq. 1; chunkwise form of the "KDA cheat sheet", eqs. 3-4).
+* :func:`decode_step` -- one token against a kept state, updated in place.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["bounded_decay", "prefill", "decode_step", "prefill_workspace_bytes", "KDAError",
+           "library_path", "load_library"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_F32, KDA_BF16 = 0, 1
+KDA_GATE_ALPHA, KDA_GATE_LOG = 0, 1
+_STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA"}
+
+
+class KDAError(RuntimeError):
+    """A libkda call returned a non-zero status."""
+
+    def __init__(self, fn: str, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{fn} failed with {_STATUS.get(status, status)}: {detail}")
+
+
+class Strides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("t", ctypes.c_int64), ("h", ctypes.c_int64)]
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [(n, Strides) for n in ("q", "k", "v", "gate", "beta", "o")]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load ``libkda.so`` (built by ``python -m gated_delta_rule_bounded_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"{p} is missing; build it with `python -m gated_delta_rule_bounded_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sp = ctypes.POINTER(Strides)
+    lp = ctypes.POINTER(Layout)
+    lib.kda_bounded_decay.argtypes = [vp, sp, i32, vp, ctypes.c_float, i64, i64, i64, i64, vp, sp, i32, vp]
+    lib.kda_prefill_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, i64, i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_prefill.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64,
+                                i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
+    lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, i64, i64, i64, i64, lp, vp, vp]
+    for fn in ("kda_bounded_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_decode_step"):
+        getattr(lib, fn).restype = ctypes.c_int
+    lib.kda_last_error.restype = ctypes.c_char_p
+    lib.kda_last_error.argtypes = []
+    lib.kda_version.restype = ctypes.c_char_p
+    lib.kda_version.argtypes = []
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise KDAError(fn, status, load_library().kda_last_error().decode())
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return KDA_F32
+    if dt == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError(f"unsupported dtype {dt}; use torch.bfloat16 or torch.float32")
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _rowwise(t: torch.Tensor) -> torch.Tensor:
+    """The innermost dim must be contiguous and rows 16-byte aligned; copy otherwise."""
+    if t.dim() == 0:
+        return t
+    if t.stride(-1) != 1 and t.shape[-1] > 1:
+        return t.contiguous()
+    es = t.element_size()
+    aligned = t.data_ptr() % 16 == 0 and all(
+        (s * es) % 16 == 0 or n <= 1 for s, n in zip(t.stride()[:-1], t.shape[:-1]))
+    return t if aligned else t.contiguous()
+
+
+def _strides4(t: torch.Tensor) -> Strides:
+    """B, T, H strides of a [B,T,H,D] tensor."""
+    return Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _strides3(t: torch.Tensor) -> Strides:
+    """B, T, H strides of a [B,T,H] tensor."""
+    return Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def bounded_decay(logits: torch.Tensor, A_log: torch.Tensor, g_min: float = -5.0, *,
+                  log_decay: bool = False, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Retention factors (or log-decays with ``log_decay=True``) for ``logits [B,T,H,K]``."""
+    _cuda(logits, "logits")
+    if logits.dim() == 3:  # decode-shaped [B,H,K]
+        res = bounded_decay(logits.unsqueeze(1), A_log, g_min, log_decay=log_decay,
+                            out=None if out is None else out.unsqueeze(1))
+        return res[:, 0]
+    if logits.dim() != 4:
+        raise ValueError("logits must be [B,T,H,K] or [B,H,K]")
+    B, T, H, K = logits.shape
+    logits = _rowwise(logits)
+    A_log = A_log.to(device=logits.device, dtype=torch.float32).contiguous()
+    if A_log.shape != (H,):
+        raise ValueError("A_log must be [H]")
+    if out is None:
+        out = torch.empty_like(logits, memory_format=torch.contiguous_format)
+    _cuda(out, "out")
+    zs, os_ = _strides4(logits), _strides4(out)
+    lib = load_library()
+    _check("kda_bounded_decay", lib.kda_bounded_decay(
+        logits.data_ptr(), ctypes.byref(zs), _dtype_code(logits.dtype), A_log.data_ptr(),
+        float(g_min), B, T, H, K, out.data_ptr(), ctypes.byref(os_),
+        KDA_GATE_LOG if log_decay else KDA_GATE_ALPHA, _stream(logits.device)))
+    return out
+
+
+def prefill_workspace_bytes(B: int, T: int, H: int, K: int, V: int, n_seq: int = 0,
+                            dtype: torch.dtype = torch.bfloat16) -> int:
+    n = ctypes.c_size_t(0)
+    _check("kda_prefill_workspace_bytes", load_library().kda_prefill_workspace_bytes(
+        B, T, H, K, V, n_seq, _dtype_code(dtype), ctypes.byref(n)))
+    return int(n.value)
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
+            initial_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
+            gate_is_log: bool = False, output_final_state: bool = True,
+            out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Scan whole sequences. Returns ``(o [B,T,H,V], final_state [N,H,K,V] fp32 or None)``.
+
+    q, k ``[B,T,H,K]`` and v ``[B,T,H,V]`` share a dtype (bf16 or fp32); gate ``[B,T,H,K]`` fp32
+    holds alpha (or g = log alpha when ``gate_is_log``); beta ``[B,T,H]`` fp32. With ``cu_seqlens``
+    (int32 ``[N+1]`` on the device) B must be 1 and the states have N rows.
+    ``final_state`` may be ``initial_state`` itself to resume in place.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta")):
+        _cuda(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B,T,H,K] and v [B,T,H,V]")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if gate.shape != q.shape or gate.dtype != torch.float32:
+        raise ValueError("gate must be fp32 [B,T,H,K]")
+    if beta.shape != q.shape[:3] or beta.dtype != torch.float32:
+        raise ValueError("beta must be fp32 [B,T,H]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    q, k, v, gate = map(_rowwise, (q, k, v, gate))
+    dev = q.device
+    cu_ptr, n_seq, N = None, 0, B
+    if cu_seqlens is not None:
+        _cuda(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        cu_seqlens = cu_seqlens.contiguous()
+        n_seq = cu_seqlens.numel() - 1
+        N = n_seq
+        cu_ptr = cu_seqlens.data_ptr()
+    s0_ptr = None
+    if initial_state is not None:
+        _cuda(initial_state, "initial_state")
+        if initial_state.shape != (N, H, K, V) or initial_state.dtype != torch.float32 \
+                or not initial_state.is_contiguous():
+            raise ValueError(f"initial_state must be a contiguous fp32 [{N},{H},{K},{V}] tensor")
+        s0_ptr = initial_state.data_ptr()
+    if output_final_state and final_state is None:
+        final_state = torch.empty((N, H, K, V), device=dev, dtype=torch.float32)
+    sf_ptr = None
+    if final_state is not None:
+        if final_state.shape != (N, H, K, V) or final_state.dtype != torch.float32 \
+                or not final_state.is_contiguous():
+            raise ValueError(f"final_state must be a contiguous fp32 [{N},{H},{K},{V}] tensor")
+        sf_ptr = final_state.data_ptr()
+    if out is None:
+        out = torch.empty((B, T, H, V), device=dev, dtype=q.dtype)
+    ws_need = prefill_workspace_bytes(B, T, H, K, V, n_seq, q.dtype)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, device=dev, dtype=torch.uint8)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    layout = Layout(_strides4(q), _strides4(k), _strides4(v), _strides4(gate), _strides3(beta), _strides4(out))
+    lib = load_library()
+    _check("kda_prefill", lib.kda_prefill(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+        KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), s0_ptr, sf_ptr,
+        cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
+        _stream(dev)))
+    return out, final_state
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
+                state: torch.Tensor, *, gate_is_log: bool = False,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One token against the kept ``state [B,H,K,V]`` (fp32, updated in place). Returns ``o [B,H,V]``.
+
+    q, k ``[B,H,K]`` (or ``[B,1,H,K]``), v ``[B,H,V]``, gate ``[B,H,K]`` fp32, beta ``[B,H]`` fp32.
+    """
+    q, k, v, gate = (x[:, 0] if x.dim() == 4 else x for x in (q, k, v, gate))
+    if beta.dim() == 3:
+        beta = beta[:, 0]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta"), (state, "state")):
+        _cuda(t, n)
+    B, H, K = q.shape
+    V = v.shape[2]
+    if k.shape != q.shape or v.shape[:2] != (B, H) or gate.shape != q.shape or beta.shape != (B, H):
+        raise ValueError("decode shapes: q, k, gate [B,H,K]; v [B,H,V]; beta [B,H]")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if gate.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("gate and beta must be fp32")
+    if state.shape != (B, H, K, V) or state.dtype != torch.float32 or not state.is_contiguous():
+        raise ValueError(f"state must be a contiguous fp32 [{B},{H},{K},{V}] tensor")
+    q, k, v, gate = map(_rowwise, (q, k, v, gate))
+    if out is None:
+        out = torch.empty((B, H, V), device=q.device, dtype=q.dtype)
+    s3 = lambda x: Strides(x.stride(0), 0, x.stride(1))  # noqa: E731
+    layout = Layout(s3(q), s3(k), s3(v), s3(gate), Strides(beta.stride(0), 0, beta.stride(1)), s3(out))
+    lib = load_library()
+    _check("kda_decode_step", lib.kda_decode_step(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+        KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), state.data_ptr(),
+        B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
+    return out

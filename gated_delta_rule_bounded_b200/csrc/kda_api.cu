@@ -1,0 +1,298 @@
+// kda_api.cu -- the C ABI: argument validation, kernel selection, status codes.
+//
+// Every check that can fail happens on the host before anything is launched,
+// so a rejected call leaves the GPU untouched. Only launch failures return
+// KDA_ERR_CUDA.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "kda.h"
+#include "kda_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_err[0] = '\0';
+  return KDA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(KDA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t elem_size(kda_dtype dt) { return dt == KDA_F32 ? 4 : 2; }
+
+bool valid_dtype(int dt) { return dt == KDA_F32 || dt == KDA_BF16; }
+
+bool dim_supported(int64_t d) { return d >= 16 && d <= 256 && d % 16 == 0; }
+
+// Contiguous [B,T,H,D] strides for a NULL strides pointer.
+kda_strides contiguous(int64_t T, int64_t H, int64_t D) {
+  kda_strides s;
+  s.h = D;
+  s.t = H * D;
+  s.b = T * H * D;
+  return s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A token row (D contiguous elements) starts on a 16-byte boundary for every
+// (b, t, h) when the base pointer and all three strides are 16-byte multiples.
+// Dimensions of extent 1 never move the pointer, so their strides do not matter.
+bool rows_aligned(const void* base, const kda_strides& s, size_t esize, int64_t B, int64_t T, int64_t H) {
+  if (!aligned16(base)) return false;
+  if (B > 1 && (s.b * (int64_t)esize) % 16 != 0) return false;
+  if (T > 1 && (s.t * (int64_t)esize) % 16 != 0) return false;
+  if (H > 1 && (s.h * (int64_t)esize) % 16 != 0) return false;
+  return true;
+}
+
+bool strides_valid(const kda_strides& s) { return s.b >= 0 && s.t >= 0 && s.h >= 0; }
+
+void put(int64_t dst[3], const kda_strides& s) {
+  dst[0] = s.b;
+  dst[1] = s.t;
+  dst[2] = s.h;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_last_error(void) { return g_err; }
+
+const char* kda_version(void) { return "kda-b200 0.1 (sm_100a)"; }
+
+int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
+                      const float* A_log, float g_min, int64_t B, int64_t T, int64_t H, int64_t K,
+                      void* out, const kda_strides* out_strides, kda_gate_kind out_kind,
+                      kda_stream_t stream) {
+  if (B < 0 || T < 0 || H < 0 || K < 0) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: negative size");
+  if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: unknown dtype %d", (int)dtype);
+  if (out_kind != KDA_GATE_ALPHA && out_kind != KDA_GATE_LOG)
+    return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: unknown out_kind %d", (int)out_kind);
+  if (!std::isfinite(g_min) || !(g_min < 0.f))
+    return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: g_min must be finite and < 0 (got %g)", (double)g_min);
+  if (B * T * H * K == 0) return ok();
+  if (!logits || !A_log || !out) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: null pointer");
+  if (K % 4 != 0) return fail(KDA_ERR_UNSUPPORTED, "kda_bounded_decay: K must be a multiple of 4 (got %lld)", (long long)K);
+  kda_strides zs = logits_strides ? *logits_strides : contiguous(T, H, K);
+  kda_strides os = out_strides ? *out_strides : contiguous(T, H, K);
+  if (!strides_valid(zs) || !strides_valid(os)) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: negative stride");
+  const size_t es = elem_size(dtype);
+  // bf16 rows are read four channels (8 bytes) at a time, fp32 rows 16 bytes.
+  auto al = [&](const void* p, const kda_strides& s) {
+    const size_t need = dtype == KDA_F32 ? 16 : 8;
+    auto ok_mult = [&](int64_t st, int64_t ext) { return ext <= 1 || (st * (int64_t)es) % (int64_t)need == 0; };
+    return (reinterpret_cast<uintptr_t>(p) % need) == 0 && ok_mult(s.b, B) && ok_mult(s.t, T) && ok_mult(s.h, H);
+  };
+  if (!al(logits, zs) || !al(out, os)) return fail(KDA_ERR_UNSUPPORTED, "kda_bounded_decay: misaligned rows");
+  kda::GateParams p;
+  p.z = logits;
+  p.out = out;
+  p.A_log = A_log;
+  put(p.zs, zs);
+  put(p.os, os);
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.K = K;
+  p.g_min = g_min;
+  p.out_log = out_kind == KDA_GATE_LOG;
+  cudaError_t e = kda::launch_gate(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kda_bounded_decay launch");
+  return ok();
+}
+
+int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                int64_t n_seq, kda_dtype dtype, size_t* bytes) {
+  if (!bytes) return fail(KDA_ERR_INVALID_ARG, "kda_prefill_workspace_bytes: null output");
+  if (B < 0 || T < 0 || H < 0 || K < 0 || V < 0 || n_seq < 0)
+    return fail(KDA_ERR_INVALID_ARG, "kda_prefill_workspace_bytes: negative size");
+  if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "kda_prefill_workspace_bytes: unknown dtype");
+  *bytes = 0;
+  if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype))
+    *bytes = kda::chunk_workspace_bytes(B, T, H, K, V, n_seq > 0 ? n_seq : B);
+  return ok();
+}
+
+static int check_scan_common(const char* fn, kda_dtype dtype, int gate_kind, int64_t H, int64_t K, int64_t V) {
+  if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
+    return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, gate_kind);
+  if (H <= 0) return fail(KDA_ERR_INVALID_ARG, "%s: H must be positive", fn);
+  if (!dim_supported(K) || !dim_supported(V))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: K and V must be multiples of 16 in [16,256] (K=%lld, V=%lld)", fn,
+                (long long)K, (long long)V);
+  return KDA_OK;
+}
+
+int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
+                const float* gate, kda_gate_kind gate_kind, const float* beta,
+                const float* initial_state, float* final_state,
+                const int32_t* cu_seqlens, int64_t n_seq,
+                int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                const kda_layout* layout, void* o,
+                void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const char* fn = "kda_prefill";
+  if (B < 0 || T < 0 || n_seq < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  int rc = check_scan_common(fn, dtype, gate_kind, H, K, V);
+  if (rc != KDA_OK) return rc;
+  int64_t N = B;
+  if (cu_seqlens) {
+    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "%s: cu_seqlens requires B == 1 (got %lld)", fn, (long long)B);
+    N = n_seq;
+  }
+  const int64_t state_elems = N * H * K * V;
+  if (initial_state && final_state && initial_state != final_state) {
+    const float* a0 = initial_state;
+    const float* a1 = initial_state + state_elems;
+    const float* b0 = final_state;
+    const float* b1 = final_state + state_elems;
+    if (a0 < b1 && b0 < a1) return fail(KDA_ERR_INVALID_ARG, "%s: initial_state and final_state overlap partially", fn);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B * T == 0 || N == 0) {
+    // Empty scan: the final state is the initial state (or zeros).
+    if (N > 0 && final_state) {
+      cudaError_t e = kda::launch_state_copy(initial_state, final_state, state_elems, s);
+      if (e != cudaSuccess) return cuda_fail(e, "kda_prefill state copy");
+    }
+    return ok();
+  }
+  if (!q || !k || !v || !gate || !beta || !o) return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  kda_layout L;
+  if (layout) {
+    L = *layout;
+  } else {
+    L.q = contiguous(T, H, K);
+    L.k = contiguous(T, H, K);
+    L.gate = contiguous(T, H, K);
+    L.v = contiguous(T, H, V);
+    L.o = contiguous(T, H, V);
+    L.beta = contiguous(T, H, 1);
+  }
+  const kda_strides* all[6] = {&L.q, &L.k, &L.v, &L.gate, &L.beta, &L.o};
+  for (auto* st : all)
+    if (!strides_valid(*st)) return fail(KDA_ERR_INVALID_ARG, "%s: negative stride", fn);
+  const size_t es = elem_size(dtype);
+  if (!rows_aligned(q, L.q, es, B, T, H) || !rows_aligned(k, L.k, es, B, T, H) ||
+      !rows_aligned(v, L.v, es, B, T, H) || !rows_aligned(o, L.o, es, B, T, H) ||
+      !rows_aligned(gate, L.gate, 4, B, T, H))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: token rows must start on 16-byte boundaries", fn);
+  if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: state pointers must be 16-byte aligned", fn);
+  if (T > INT32_MAX) return fail(KDA_ERR_UNSUPPORTED, "%s: T too large", fn);
+
+  kda::ScanParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.gate = gate;
+  p.beta = beta;
+  p.s0 = initial_state;
+  p.sf = final_state;
+  p.cu = cu_seqlens;
+  p.o = o;
+  put(p.qs, L.q);
+  put(p.ks, L.k);
+  put(p.vs, L.v);
+  put(p.gs, L.gate);
+  put(p.bs, L.beta);
+  put(p.os, L.o);
+  p.T = T;
+  p.B = (int)B;
+  p.H = (int)H;
+  p.K = (int)K;
+  p.V = (int)V;
+  p.N = (int)N;
+  p.gate_log = gate_kind == KDA_GATE_LOG;
+
+  cudaError_t e;
+  if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype)) {
+    size_t need = kda::chunk_workspace_bytes(B, T, H, K, V, N);
+    if (workspace_bytes < need || (need > 0 && !workspace))
+      return fail(KDA_ERR_INVALID_ARG, "%s: workspace of %zu bytes given, %zu needed", fn, workspace_bytes, need);
+    e = kda::launch_chunk(p, workspace, workspace_bytes, s);
+  } else {
+    e = kda::launch_recurrent(p, dtype, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "kda_prefill launch");
+  return ok();
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype,
+                    const float* gate, kda_gate_kind gate_kind, const float* beta,
+                    float* state, int64_t B, int64_t H, int64_t K, int64_t V,
+                    const kda_layout* layout, void* o, kda_stream_t stream) {
+  const char* fn = "kda_decode_step";
+  if (B < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  int rc = check_scan_common(fn, dtype, gate_kind, H, K, V);
+  if (rc != KDA_OK) return rc;
+  if (B == 0) return ok();
+  if (!q || !k || !v || !gate || !beta || !state || !o)
+    return fail(KDA_ERR_INVALID_ARG, "%s: null pointer", fn);
+  kda_layout L;
+  if (layout) {
+    L = *layout;
+  } else {
+    L.q = contiguous(1, H, K);
+    L.k = contiguous(1, H, K);
+    L.gate = contiguous(1, H, K);
+    L.v = contiguous(1, H, V);
+    L.o = contiguous(1, H, V);
+    L.beta = contiguous(1, H, 1);
+  }
+  // Decode tensors have no time axis: the t stride is never used.
+  kda_strides* all[6] = {&L.q, &L.k, &L.v, &L.gate, &L.beta, &L.o};
+  for (auto* st : all) {
+    st->t = 0;
+    if (!strides_valid(*st)) return fail(KDA_ERR_INVALID_ARG, "%s: negative stride", fn);
+  }
+  const size_t es = elem_size(dtype);
+  if (!rows_aligned(q, L.q, es, B, 1, H) || !rows_aligned(k, L.k, es, B, 1, H) ||
+      !rows_aligned(v, L.v, es, B, 1, H) || !rows_aligned(o, L.o, es, B, 1, H) ||
+      !rows_aligned(gate, L.gate, 4, B, 1, H) || !aligned16(state))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: rows and state must start on 16-byte boundaries", fn);
+  kda::ScanParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.gate = gate;
+  p.beta = beta;
+  p.s0 = state;
+  p.sf = state;
+  p.cu = nullptr;
+  p.o = o;
+  put(p.qs, L.q);
+  put(p.ks, L.k);
+  put(p.vs, L.v);
+  put(p.gs, L.gate);
+  put(p.bs, L.beta);
+  put(p.os, L.o);
+  p.T = 1;
+  p.B = (int)B;
+  p.H = (int)H;
+  p.K = (int)K;
+  p.V = (int)V;
+  p.N = (int)B;
+  p.gate_log = gate_kind == KDA_GATE_LOG;
+  cudaError_t e = kda::launch_recurrent(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,51 @@
+// kda_internal.h -- host/device interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// Everything a scan kernel needs, passed by value. Strides are in elements, for
+// the B, T and H dimensions of each token tensor; the innermost dim is contiguous.
+struct ScanParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* gate;  // alpha, or g = log(alpha) when gate_log != 0
+  const float* beta;
+  const float* s0;    // [N,H,K,V] or nullptr (zeros)
+  float* sf;          // [N,H,K,V] or nullptr (not written)
+  const int32_t* cu;  // [N+1] packed offsets or nullptr
+  void* o;
+  int64_t qs[3], ks[3], vs[3], gs[3], bs[3], os[3];
+  int64_t T;
+  int B, H, K, V, N;
+  int gate_log;
+};
+
+struct GateParams {
+  const void* z;
+  void* out;
+  const float* A_log;
+  int64_t zs[3], os[3];
+  int64_t B, T, H, K;
+  float g_min;
+  int out_log;
+};
+
+// Launchers return the launch status (cudaGetLastError after the launch).
+cudaError_t launch_gate(const GateParams& p, kda_dtype dt, cudaStream_t s);
+// Token-by-token kernel: the decode step (T = 1, s0 == sf) and the generic
+// prefill path (fp32 inputs, any supported K and V).
+cudaError_t launch_recurrent(const ScanParams& p, kda_dtype dt, cudaStream_t s);
+// Chunked prefill for bf16 inputs (bounded decay), tensor cores.
+bool chunk_supported(int K, int V, kda_dtype dt);
+size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t N);
+cudaError_t launch_chunk(const ScanParams& p, void* ws, size_t ws_bytes, cudaStream_t s);
+// Copy initial state (or zeros) into final state for T == 0 calls.
+cudaError_t launch_state_copy(const float* s0, float* sf, int64_t n, cudaStream_t s);
+
+}  // namespace kda

@@ -1,0 +1,168 @@
+/*
+ * kda.h -- C ABI of libkda: the bounded-decay gated delta rule (the Kimi Delta
+ * Attention scan) on NVIDIA B200 (sm_100a).
+ *
+ * Operations and the passages that define them:
+ *
+ *   kda_bounded_decay  "Kimi K3: Bounded Decay and Delta Memory", Formula and
+ *                      conventions, eq. 5: g = g_min * sigmoid(e^A * z),
+ *                      alpha = e^g, per channel, with A a per-head log-scale.
+ *   kda_prefill        same page, eq. 1 (fade, correct, read the updated
+ *                      state) over whole sequences, returning every output
+ *                      and the final state; computed in the chunkwise form of
+ *                      the "KDA cheat sheet", Chunkwise parallel form
+ *                      (eqs. 3-4). The argument set follows the chunked kernel
+ *                      call excerpted on the "Kept memory" page (initial
+ *                      state, final state, cu_seqlens).
+ *   kda_decode_step    the same recurrence for one new token against a kept
+ *                      state that is updated in place ("Kept memory": the
+ *                      recurrent form used for one new position with a cache).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every call returns a kda_status. KDA_OK is 0. Nothing is launched when a
+ *   call returns an error other than KDA_ERR_CUDA; kda_last_error() then holds
+ *   a one-line, thread-local description. Nothing throws across the ABI.
+ * - Tensor pointers are DEVICE pointers owned by the caller; the library never
+ *   allocates device or pinned memory and never frees what it is given. Calls
+ *   are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *   stream); the caller keeps every buffer alive until the work has finished.
+ * - Layouts are the contract table's: q, k, alpha/g [B,T,H,K]; v, o [B,T,H,V];
+ *   beta [B,T,H]; states [N,H,K,V] (key-by-value: K rows, V columns, V
+ *   contiguous, the whole state tensor contiguous). The innermost dimension of
+ *   every token tensor is contiguous; its B, T and H dimensions take element
+ *   strides (kda_strides), so non-contiguous views such as slices of a fused
+ *   projection can be passed directly. A NULL strides pointer means contiguous.
+ *   Every row start must be 16-byte aligned (base pointer and strides), else
+ *   the call returns KDA_ERR_UNSUPPORTED.
+ * - Inputs are never written, except the decode state, which is updated in
+ *   place by contract.
+ * - No query scaling happens inside the scan (the PaperLeet contract says the
+ *   scan performs no query scaling or key normalisation); a caller who wants
+ *   D^-1/2 scaling pre-scales q.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kda_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad cu_seqlens size, g_min not < 0 ... */
+  KDA_ERR_UNSUPPORTED = 2, /* K, V, dtype or alignment outside the supported set */
+  KDA_ERR_CUDA = 3         /* a CUDA launch or runtime call failed; see kda_last_error() */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* How a decay tensor is given: retention factors alpha in [0,1], or their
+ * logarithms g = log(alpha) <= 0. */
+typedef enum { KDA_GATE_ALPHA = 0, KDA_GATE_LOG = 1 } kda_gate_kind;
+
+/* Element strides of the B, T and H dimensions of a [B,T,H,D] tensor (or of
+ * a [B,T,H] tensor such as beta). For decode tensors ([B,H,D], [B,H]) the t
+ * member is ignored. */
+typedef struct {
+  int64_t b, t, h;
+} kda_strides;
+
+typedef struct {
+  kda_strides q, k, v, gate, beta, o;
+} kda_layout;
+
+/* ---------------------------------------------------------------------------
+ * kda_bounded_decay: retention factors from decay logits.
+ *
+ *   out[b,t,h,c] = alpha = exp(g)      (out_kind == KDA_GATE_ALPHA), or
+ *   out[b,t,h,c] = g                   (out_kind == KDA_GATE_LOG),
+ *   g = g_min * sigmoid(exp(A_log[h]) * logits[b,t,h,c]).
+ *
+ * logits  [B,T,H,K], dtype `dtype` (KDA_F32 or KDA_BF16); `out` has the same
+ *         shape and dtype (the page: retention matches the logits' dtype).
+ * A_log   [H] fp32, the per-head log-scale A.
+ * g_min   the lower bound of the log-decay; must be finite and < 0.
+ * strides of logits and out: NULL = contiguous.
+ * alpha lies in [exp(g_min), 1]; strictly inside for moderate logits, and at
+ * an end point only where sigmoid rounds to 0 or 1 in fp32.
+ * ------------------------------------------------------------------------- */
+int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
+                      const float* A_log, float g_min, int64_t B, int64_t T, int64_t H, int64_t K,
+                      void* out, const kda_strides* out_strides, kda_gate_kind out_kind,
+                      kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * kda_prefill_workspace_bytes: bytes of device scratch kda_prefill needs for
+ * these sizes (0 when the selected kernels keep everything on chip). The
+ * caller allocates it; a larger buffer is fine.
+ * ------------------------------------------------------------------------- */
+int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                int64_t n_seq, kda_dtype dtype, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * kda_prefill: the scan over whole sequences.
+ *
+ * q, k      [B,T,H,K]  dtype `dtype` (KDA_BF16 or KDA_F32; q, k, v share it)
+ * v         [B,T,H,V]  dtype `dtype`
+ * gate      [B,T,H,K]  fp32 alpha (gate_kind KDA_GATE_ALPHA) or g = log alpha
+ *                      (KDA_GATE_LOG). For bf16 inputs the chunked kernel
+ *                      requires the bounded range alpha >= exp(-5), g >= -5
+ *                      (the bound the "KDA cheat sheet" uses to keep every
+ *                      reciprocal rescale within range); fp32 inputs take any
+ *                      alpha in [0,1].
+ * beta      [B,T,H]    fp32 write strength in [0,1]
+ * initial_state [N,H,K,V] fp32 or NULL (zeros)
+ * final_state   [N,H,K,V] fp32 or NULL (not written). It may be the same
+ *               pointer as initial_state (resume in place); partial overlap is
+ *               not allowed.
+ * cu_seqlens  NULL, or int32 [n_seq+1] device offsets of n_seq packed
+ *             sequences along T (B must be 1; offsets non-decreasing from 0
+ *             to T; zero-length sequences allowed). N = n_seq then, else N = B.
+ * o         [B,T,H,V]  dtype `dtype`, o[t] = S_t^T q_t with S_t the state
+ *                      after token t's update.
+ * workspace, workspace_bytes: device scratch of at least
+ *             kda_prefill_workspace_bytes(...) bytes (may be NULL when that is 0).
+ * T == 0 (or a zero-length packed sequence) copies initial_state (or zeros)
+ * to final_state. Supported: K, V multiples of 16 in [16, 256].
+ * ------------------------------------------------------------------------- */
+int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
+                const float* gate, kda_gate_kind gate_kind, const float* beta,
+                const float* initial_state, float* final_state,
+                const int32_t* cu_seqlens, int64_t n_seq,
+                int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                const kda_layout* layout, void* o,
+                void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * kda_decode_step: one new token per (b, h) against a kept state, in place.
+ *
+ * q, k [B,H,K]; v, o [B,H,V]  dtype `dtype` (a [B,1,H,D] tensor is passed with
+ *                             its b and h strides)
+ * gate [B,H,K] fp32 alpha or g; beta [B,H] fp32
+ * state [B,H,K,V] fp32, contiguous: read as S_{t-1}, overwritten with S_t.
+ *   Sbar = Diag(alpha) S;  delta = v - Sbar^T k;  S = Sbar + beta k delta^T;
+ *   o = S^T q.
+ * Any alpha in [0,1] is accepted. Supported: K, V multiples of 16 in [16,256].
+ * ------------------------------------------------------------------------- */
+int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype,
+                    const float* gate, kda_gate_kind gate_kind, const float* beta,
+                    float* state, int64_t B, int64_t H, int64_t K, int64_t V,
+                    const kda_layout* layout, void* o, kda_stream_t stream);
+
+/* Last error of the calling thread ("" when the last call succeeded). */
+const char* kda_last_error(void);
+
+/* Library version string. */
+const char* kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,384 @@
+"""GPU parity: the CUDA path against the fp64 oracle on the same seeded inputs.
+
+Both sides start from the same raw inputs (q, k, v, decay logits z, A_log,
+beta, initial state) drawn by ``workloads.py``. The GPU side runs its own gate
+kernel and scan kernels through the C ABI; the oracle side runs its own fp64
+gate and token-by-token scan. Tolerances (written in each test):
+
+* fp32 q/k/v: max |gpu - oracle| <= 1e-4 on o and on final_state;
+* bf16 q/k/v: the relative RMS error rms(gpu - oracle) <= 2e-2 * rms(oracle),
+  separately for o and final_state, plus an elementwise guard
+  |gpu - oracle| <= (|oracle| + rms(oracle)) / 8 that any wrong term, index or
+  token fails. The bound is read as an RMS ratio because a max-abs reading is
+  out of reach for a bf16 result: rounding the exact output to bf16 alone
+  gives max|err| / rms = 1.8e-2 at T = 150 and more at larger sizes (the
+  largest outputs are 10-20x the RMS), while bf16 tensor-core arithmetic
+  keeps the RMS ratio near 5e-3;
+* gate: |g - g_ref| <= |g_ref| 2^-22 (1 + |e^A z|) for fp32 output (the fp32
+  rounding of the sigmoid's argument carried through), within one bf16
+  rounding (2^-8 relative) for bf16 output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+FP32_ATOL = 1e-4
+BF16_REL_RMS = 2e-2
+GUARD = 0.125
+
+
+@pytest.fixture(scope="module")
+def kda():
+    from gated_delta_rule_bounded_b200 import build
+    build.build()
+    import gated_delta_rule_bounded_b200 as m
+    m.load_library()
+    return m
+
+
+def check(got, ref, dtype, what):
+    """fp32: max-abs <= 1e-4. bf16: rms(err) <= 2e-2 rms(ref) and |err| <= (|ref| + rms(ref)) / 8.
+    Returns the RMS error ratio (bf16) or the max abs error (fp32)."""
+    got = got.detach().double().cpu().numpy() if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} != {ref.shape}"
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    if ref.size == 0:
+        return 0.0
+    err = np.abs(got - ref)
+    if dtype == "f32":
+        m = float(err.max())
+        assert m <= FP32_ATOL, f"{what}: max abs err {m:.3e} > {FP32_ATOL}"
+        return m
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    ratio = float(np.sqrt(np.mean(err ** 2))) / rms
+    assert ratio <= BF16_REL_RMS, f"{what}: rms error / rms {ratio:.3e} > {BF16_REL_RMS}"
+    worst = float((err / (np.abs(ref) + rms)).max())
+    assert worst <= GUARD, f"{what}: elementwise error {worst:.3e} of (|ref| + rms) > {GUARD}"
+    return ratio
+
+
+def to_dev(d):
+    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def gpu_pipeline(kda, d, **kw):
+    """z -> alpha (gate kernel) -> scan (prefill kernels), all through the C ABI."""
+    g = to_dev(d)
+    alpha = kda.bounded_decay(g["z"], g["A_log"], g["g_min"])
+    o, sf = kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], g["initial_state"], g["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    return o, sf
+
+
+def oracle_pipeline(d, heads=None):
+    """Oracle gate and scan, optionally on a subset of heads."""
+    sel = (lambda x: x) if heads is None else (lambda x: x[:, :, heads])
+    z, q, k, v, beta = (sel(d[n]) for n in ("z", "q", "k", "v", "beta"))
+    A = d["A_log"] if heads is None else d["A_log"][heads]
+    s0 = d["initial_state"]
+    if s0 is not None and heads is not None:
+        s0 = s0[:, heads]
+    alpha = oracle.bounded_decay(z, A, d["g_min"])
+    return oracle.scan(q, k, v, alpha, beta, s0, d["cu_seqlens"])
+
+
+# ---------------------------------------------------------------------------------------------
+# Gate
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 256, 4, 32), (2, 37, 3, 128), (1, 5, 96, 128)])
+def test_gate_matches_oracle(kda, dtype, shape):
+    g = torch.Generator().manual_seed(sum(shape))
+    z = (torch.randn(*shape, generator=g) * 4).to(W.DTYPES[dtype])
+    A = torch.randn(shape[2], generator=g) * 0.5
+    for g_min in (-5.0, -1.5):
+        alpha = kda.bounded_decay(z.to(DEV), A.to(DEV), g_min).double().cpu().numpy()
+        lg = kda.bounded_decay(z.to(DEV), A.to(DEV), g_min, log_decay=True).double().cpu().numpy()
+        ra, rg = oracle.bounded_decay(z, A, g_min, return_log=True)
+        if dtype == "f32":
+            # fp32 evaluation: x = e^A z is itself rounded (relative 2^-24), and sigmoid carries
+            # that into g with a factor of at most |x|, so |dg| <= |g| 2^-22 (1 + |x|).
+            x = np.abs(np.exp(A.double().numpy())[None, None, :, None] * z.double().numpy())
+            tol_g = np.abs(rg) * 2.0 ** -22 * (1 + x)
+            assert np.all(np.abs(lg - rg) <= tol_g), "log-decay outside the fp32 evaluation bound"
+            assert np.all(np.abs(alpha - ra) <= ra * (tol_g + 2.0 ** -22)), "alpha outside the fp32 bound"
+        else:
+            np.testing.assert_allclose(alpha, ra, rtol=2.0 ** -8, atol=0)
+            np.testing.assert_allclose(lg, rg, rtol=2.0 ** -8, atol=1e-30)
+        lo = np.exp(g_min) * (1 - (2.0 ** -8 if dtype == "bf16" else 1e-6))  # one rounding of the output
+        assert np.all(alpha >= lo) and np.all(alpha <= 1.0)
+
+
+def test_gate_strided_logits(kda):
+    g = torch.Generator().manual_seed(3)
+    big = torch.randn(2, 9, 3, 192, generator=g)
+    z = big[..., 32:160]                       # a non-contiguous view, rows 16-byte aligned
+    A = torch.randn(3, generator=g)
+    got = kda.bounded_decay(z.to(DEV), A.to(DEV), -5.0).double().cpu().numpy()
+    np.testing.assert_allclose(got, oracle.bounded_decay(z, A, -5.0), rtol=2e-6)
+
+
+# ---------------------------------------------------------------------------------------------
+# Prefill, small cases that span several chunks and a ragged tail
+# ---------------------------------------------------------------------------------------------
+
+def test_tiny_fp32_workload(kda):
+    """B=1, T=256, H=4, K=V=32, fp32, zero initial state: max-abs <= 1e-4."""
+    d = W.make_scan_inputs(W.TINY_FP32)
+    o, sf = gpu_pipeline(kda, d)
+    ro, rs = oracle_pipeline(d)
+    check(o, ro, "f32", "o")
+    check(sf, rs, "f32", "final_state")
+
+
+@pytest.mark.parametrize("B,T,H,K,V,init", [
+    (1, 200, 3, 128, 128, False),
+    (2, 131, 2, 128, 128, True),
+    (1, 64, 2, 128, 256, True),
+    (2, 77, 2, 128, 64, True),
+    (1, 300, 1, 64, 128, True),
+    (1, 1, 2, 128, 128, True),
+    (3, 16, 2, 32, 48, True),
+])
+def test_prefill_bf16_matches_oracle(kda, B, T, H, K, V, init):
+    d = W.random_scan_case(B, T, H, K, V, seed=T + H + K, dtype="bf16", z_std=2.0,
+                           init_std=0.1 if init else None)
+    o, sf = gpu_pipeline(kda, d)
+    ro, rs = oracle_pipeline(d)
+    check(o, ro, "bf16", "o")
+    check(sf, rs, "bf16", "final_state")
+
+
+@pytest.mark.parametrize("B,T,H,K,V", [(1, 150, 2, 32, 32), (2, 70, 3, 64, 16), (1, 40, 1, 128, 256)])
+def test_prefill_fp32_matches_oracle(kda, B, T, H, K, V):
+    d = W.random_scan_case(B, T, H, K, V, seed=5 + T, dtype="f32", z_std=1.0, init_std=0.1)
+    o, sf = gpu_pipeline(kda, d)
+    ro, rs = oracle_pipeline(d)
+    check(o, ro, "f32", "o")
+    check(sf, rs, "f32", "final_state")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_prefill_varlen_with_empty_segments(kda, dtype):
+    lens = [70, 0, 129, 1, 0, 64, 200]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    d = W.random_scan_case(1, int(cu[-1]), 2, 128, 128, seed=17, dtype=dtype, z_std=2.0, init_std=None)
+    d["cu_seqlens"] = cu
+    d["initial_state"] = torch.randn(len(lens), 2, 128, 128, generator=torch.Generator().manual_seed(1)) * 0.1
+    o, sf = gpu_pipeline(kda, d)
+    ro, rs = oracle_pipeline(d)
+    check(o, ro, dtype, "o")
+    check(sf, rs, dtype, "final_state")
+    # Zero-length sequences return their initial state exactly.
+    for n, L in enumerate(lens):
+        if L == 0:
+            assert torch.equal(sf[n].cpu(), d["initial_state"][n])
+
+
+@pytest.mark.parametrize("with_init", [True, False])
+def test_prefill_empty_sequence(kda, with_init):
+    B, H, K, V = 2, 3, 128, 64
+    s0 = torch.randn(B, H, K, V) if with_init else None
+    z = torch.zeros(B, 0, H, K, device=DEV)
+    q = torch.zeros(B, 0, H, K, device=DEV, dtype=torch.bfloat16)
+    v = torch.zeros(B, 0, H, V, device=DEV, dtype=torch.bfloat16)
+    o, sf = kda.prefill(q, q, v, z, torch.zeros(B, 0, H, device=DEV),
+                        None if s0 is None else s0.to(DEV))
+    torch.cuda.synchronize()
+    assert o.shape == (B, 0, H, V)
+    assert torch.equal(sf.cpu(), s0 if with_init else torch.zeros(B, H, K, V))
+
+
+def test_prefill_strided_views(kda):
+    """q, k, v as slices of one fused projection tensor; gate and o as views too."""
+    B, T, H, K, V = 2, 97, 3, 128, 128
+    g = torch.Generator().manual_seed(8)
+    fused = torch.randn(B, T, H, 2 * K + V, generator=g)
+    q = torch.nn.functional.normalize(fused[..., :K], dim=-1).bfloat16()
+    k = torch.nn.functional.normalize(fused[..., K:2 * K], dim=-1).bfloat16()
+    qkv = torch.cat([q, k, fused[..., 2 * K:].bfloat16()], dim=-1).to(DEV)
+    zbig = (torch.randn(B, T, H, K + 64, generator=g) * 2)
+    A = torch.randn(H, generator=g) * 0.5
+    beta_big = torch.sigmoid(torch.randn(B, T, H, 2, generator=g))
+    s0 = torch.randn(B, H, K, V, generator=g) * 0.1
+    qd, kd, vd = qkv[..., :K], qkv[..., K:2 * K], qkv[..., 2 * K:]
+    assert not qd.is_contiguous()
+    alpha = kda.bounded_decay(zbig[..., 32:32 + K].to(DEV), A.to(DEV), -5.0)
+    o_big = torch.zeros(B, T, H, 2 * V, device=DEV, dtype=torch.bfloat16)
+    o, sf = kda.prefill(qd, kd, vd, alpha, beta_big[..., 0].to(DEV), s0.to(DEV), out=o_big[..., V:])
+    torch.cuda.synchronize()
+    assert o.data_ptr() == o_big[..., V:].data_ptr()
+    ra = oracle.bounded_decay(zbig[..., 32:32 + K], A, -5.0)
+    ro, rs = oracle.scan(q, k, fused[..., 2 * K:].bfloat16(), ra, beta_big[..., 0], s0)
+    check(o, ro, "bf16", "o")
+    check(sf, rs, "bf16", "final_state")
+    assert torch.count_nonzero(o_big[..., :V]) == 0
+
+
+def test_prefill_log_gate_and_inputs_untouched(kda):
+    d = W.random_scan_case(1, 130, 2, 128, 128, seed=23, dtype="bf16", z_std=2.0, init_std=0.1)
+    g = to_dev(d)
+    lg = kda.bounded_decay(g["z"], g["A_log"], -5.0, log_decay=True)
+    copies = {n: g[n].clone() for n in ("q", "k", "v", "beta", "initial_state")}
+    lg_copy = lg.clone()
+    o, sf = kda.prefill(g["q"], g["k"], g["v"], lg, g["beta"], g["initial_state"], gate_is_log=True)
+    torch.cuda.synchronize()
+    for n, c in copies.items():
+        assert torch.equal(g[n], c), f"{n} was modified"
+    assert torch.equal(lg, lg_copy)
+    ro, rs = oracle_pipeline(d)
+    check(o, ro, "bf16", "o")
+    check(sf, rs, "bf16", "final_state")
+
+
+def test_prefill_resume_in_place(kda):
+    """final_state may alias initial_state; splitting and resuming equals one pass."""
+    d = W.random_scan_case(2, 200, 2, 128, 128, seed=31, dtype="bf16", z_std=2.0, init_std=0.1)
+    g = to_dev(d)
+    alpha = kda.bounded_decay(g["z"], g["A_log"], -5.0)
+    o_full, s_full = kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], g["initial_state"])
+    st = g["initial_state"].clone()
+    cut = 77
+    o1, _ = kda.prefill(g["q"][:, :cut], g["k"][:, :cut], g["v"][:, :cut], alpha[:, :cut], g["beta"][:, :cut],
+                        st, final_state=st)
+    o2, _ = kda.prefill(g["q"][:, cut:], g["k"][:, cut:], g["v"][:, cut:], alpha[:, cut:], g["beta"][:, cut:],
+                        st, final_state=st)
+    torch.cuda.synchronize()
+    ro, rs = oracle_pipeline(d)
+    check(torch.cat([o1, o2], 1), ro, "bf16", "o (split)")
+    check(st, rs, "bf16", "final_state (split)")
+    check(o_full, ro, "bf16", "o")
+    check(s_full, rs, "bf16", "final_state")
+
+
+# ---------------------------------------------------------------------------------------------
+# Decode
+# ---------------------------------------------------------------------------------------------
+
+def decode_run(kda, w, steps, heads_sample):
+    """Runs `steps` decode steps on the GPU; returns GPU outputs and final state on sampled
+    heads plus the oracle's (the oracle scans the sampled heads' steps as one sequence)."""
+    prm = W.make_decode_params(w)
+    state = prm["state"].to(DEV)
+    A = prm["A_log"].to(DEV)
+    bsel, hsel = heads_sample
+    outs, ins = [], {n: [] for n in ("q", "k", "v", "z", "beta")}
+    for s in range(steps):
+        st = W.make_decode_step(w, s)
+        gd = to_dev(st)
+        alpha = kda.bounded_decay(gd["z"], A, w.g_min)
+        o = kda.decode_step(gd["q"], gd["k"], gd["v"], alpha, gd["beta"], state)
+        outs.append(o[bsel][:, hsel].cpu())
+        for n in ins:
+            ins[n].append(st[n][bsel][:, hsel])
+    torch.cuda.synchronize()
+    got_o = torch.stack(outs, 1)                        # [b, steps, h, V]
+    got_s = state[bsel][:, hsel].cpu()
+    seq = {n: torch.stack(x, 1) for n, x in ins.items()}  # [b, steps, h, *]
+    alpha = oracle.bounded_decay(seq["z"], prm["A_log"][hsel], w.g_min)
+    ro, rs = oracle.scan(seq["q"], seq["k"], seq["v"], alpha, seq["beta"], prm["state"][bsel][:, hsel])
+    return got_o, got_s, ro, rs
+
+
+def test_decode_small_matches_oracle(kda):
+    w = W.DecodeWorkload("decode_small", 3, 4, 128, 128, steps=40)
+    got_o, got_s, ro, rs = decode_run(kda, w, 40, (torch.arange(3), torch.arange(4)))
+    check(got_o, ro, "bf16", "o")
+    check(got_s, rs, "bf16", "state")
+
+
+@pytest.mark.parametrize("K,V", [(32, 32), (64, 128), (128, 256), (48, 80)])
+def test_decode_shapes_fp32(kda, K, V):
+    w = W.DecodeWorkload("decode_fp32", 2, 3, K, V, steps=25, dtype="f32")
+    got_o, got_s, ro, rs = decode_run(kda, w, 25, (torch.arange(2), torch.arange(3)))
+    check(got_o, ro, "f32", "o")
+    check(got_s, rs, "f32", "state")
+
+
+def test_decode_alpha_zero_and_one(kda):
+    """Gate end points: alpha = 0 wipes the faded state, alpha = 1 with beta = 0 keeps it."""
+    B, H, K, V = 2, 2, 128, 128
+    g = torch.Generator().manual_seed(2)
+    state = (torch.randn(B, H, K, V, generator=g) * 0.1)
+    q = torch.nn.functional.normalize(torch.randn(B, H, K, generator=g), dim=-1).bfloat16()
+    k = torch.nn.functional.normalize(torch.randn(B, H, K, generator=g), dim=-1).bfloat16()
+    v = torch.randn(B, H, V, generator=g).bfloat16()
+    for a_val, b_val in ((0.0, 0.7), (1.0, 0.0)):
+        alpha = torch.full((B, H, K), a_val)
+        beta = torch.full((B, H), b_val)
+        sd = state.clone().to(DEV)
+        o = kda.decode_step(q.to(DEV), k.to(DEV), v.to(DEV), alpha.to(DEV), beta.to(DEV), sd)
+        torch.cuda.synchronize()
+        ro, rs = oracle.scan(q[:, None], k[:, None], v[:, None], alpha[:, None], beta[:, None], state)
+        check(o, ro[:, 0], "bf16", "o")
+        check(sd, rs, "bf16", "state")
+
+
+@pytest.mark.slow
+def test_decode_workload_1000_steps_sampled(kda):
+    """The kept-memory decode workload (B=64, H=96, K=V=128, 1000 steps), every head on the
+    GPU, the oracle on a sample of (batch, head) pairs."""
+    w = W.DECODE
+    bsel = torch.tensor([0, 17, 63])
+    hsel = torch.tensor([0, 41, 95])
+    got_o, got_s, ro, rs = decode_run(kda, w, w.steps, (bsel, hsel))
+    check(got_o, ro, "bf16", "o")
+    check(got_s, rs, "bf16", "state")
+
+
+# ---------------------------------------------------------------------------------------------
+# Full-size prefill workloads, sampled heads
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.slow
+def test_prefill_workload_4096_sampled_heads(kda):
+    d = W.make_scan_inputs(W.PREFILL)
+    o, sf = gpu_pipeline(kda, d)
+    heads = [0, 13, 47, 95]
+    ro, rs = oracle_pipeline(d, heads)
+    check(o[:, :, heads], ro, "bf16", "o")
+    check(sf[:, heads], rs, "bf16", "final_state")
+
+
+@pytest.mark.slow
+def test_varlen_workload_sampled_heads(kda):
+    d = W.make_scan_inputs(W.VARLEN)
+    o, sf = gpu_pipeline(kda, d)
+    heads = [3, 60]
+    ro, rs = oracle_pipeline(d, heads)
+    check(o[:, :, heads], ro, "bf16", "o")
+    check(sf[:, heads], rs, "bf16", "final_state")
+    cu = d["cu_seqlens"].numpy()
+    for n in range(len(cu) - 1):  # per-sequence bound as well
+        s, e = cu[n], cu[n + 1]
+        check(o[:, s:e][:, :, heads], ro[:, s:e], "bf16", f"o seq {n}")
+
+
+@pytest.mark.slow
+def test_long_kv_workload_split_resume_sampled(kda):
+    """B=4, T=16384, H=32, K=128, V=256: one pass, and a split at 8192 resumed from the
+    final state, both against the oracle on sampled heads."""
+    d = W.make_scan_inputs(W.LONG_KV)
+    g = to_dev(d)
+    alpha = kda.bounded_decay(g["z"], g["A_log"], -5.0)
+    o, sf = kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], g["initial_state"])
+    half = 8192
+    o1, s1 = kda.prefill(g["q"][:, :half], g["k"][:, :half], g["v"][:, :half], alpha[:, :half],
+                         g["beta"][:, :half], g["initial_state"])
+    o2, s2 = kda.prefill(g["q"][:, half:], g["k"][:, half:], g["v"][:, half:], alpha[:, half:],
+                         g["beta"][:, half:], s1)
+    torch.cuda.synchronize()
+    heads = [5, 30]
+    ro, rs = oracle_pipeline(d, heads)
+    check(o[:, :, heads], ro, "bf16", "o")
+    check(sf[:, heads], rs, "bf16", "final_state")
+    check(torch.cat([o1, o2], 1)[:, :, heads], ro, "bf16", "o (split)")
+    check(s2[:, heads], rs, "bf16", "final_state (split)")
