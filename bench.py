@@ -51,7 +51,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 def prefill_bytes(B, T, H, K, V, n_states_in, n_states_out, es=2):
     """Minimum HBM bytes of one prefill launch: read q, k (K each), v (V) in the input dtype,
-    alpha (K fp32) and beta (fp32) per token-head, write o (V); read/write the fp32 states."""
+    the decay (alpha or g, K fp32) and beta (fp32) per token-head, write o (V); read/write the
+    fp32 states."""
     per_tok_head = 2 * K * es + V * es + 4 * K + 4 + V * es
     return B * T * H * per_tok_head + (n_states_in + n_states_out) * H * K * V * 4
 
@@ -246,11 +247,14 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     ws_bytes = kda.prefill_workspace_bytes(B, T, H, K, V, 0, torch.bfloat16)
     ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
 
+    # The gate writes the log-decay g = log(alpha) and the prefill takes it directly (the ABI
+    # accepts alpha or g); this skips an exp in the gate and a log in the scan.
     def gate_fn():
-        kda.bounded_decay(g["z"], g["A_log"], w.g_min, out=alpha)
+        kda.bounded_decay(g["z"], g["A_log"], w.g_min, log_decay=True, out=alpha)
 
     def prefill_fn():
-        kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], None, out=o, final_state=sf, workspace=ws)
+        kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], None, gate_is_log=True, out=o, final_state=sf,
+                    workspace=ws)
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
     total_ms, (gate_ms, pre_ms) = timed_loop([gate_fn, prefill_fn], args.steps, args.warmup, world, stream, sampler)
@@ -284,8 +288,8 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     def e2e_fn():
         for n, x in host.items():
             dev_in[n].copy_(x, non_blocking=True)
-        kda.bounded_decay(dev_in["z"], dev_in["A_log"], w.g_min, out=alpha)
-        kda.prefill(dev_in["q"], dev_in["k"], dev_in["v"], alpha, dev_in["beta"], None, out=o,
+        kda.bounded_decay(dev_in["z"], dev_in["A_log"], w.g_min, log_decay=True, out=alpha)
+        kda.prefill(dev_in["q"], dev_in["k"], dev_in["v"], alpha, dev_in["beta"], None, gate_is_log=True, out=o,
                     final_state=sf, workspace=ws)
         o_host.copy_(o, non_blocking=True)
         sf_host.copy_(sf, non_blocking=True)
@@ -392,7 +396,7 @@ def gpu_arm(args, rank, world, local):
         "dtype": "bf16",
         "data": "synthetic (seeded; no dataset)",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "K": w.K, "V": w.V, "g_min": w.g_min,
-                   "z_std": w.z_std, "initial_state": "zeros", "step": "bounded_decay + prefill",
+                   "z_std": w.z_std, "initial_state": "zeros", "step": "bounded_decay (log-decay out) + prefill (log-decay in)",
                    "l2": "inputs larger than L2 (q/k/v/z/alpha ~ 0.9 GB); no flush",
                    "parallelism": f"replica per GPU x{world}"},
         "roofline": pre["roofline"],

@@ -1,7 +1,7 @@
 // gate.cu -- bounded decay gate ("Kimi K3: Bounded Decay and Delta Memory", eq. 5):
 //   g = g_min * sigmoid(exp(A_h) * z),  alpha = exp(g).
-// Elementwise and HBM-bound: each thread handles four consecutive channels of a
-// (b, t, h) row with 16-byte (fp32) or 8-byte (bf16) accesses; the grid is a
+// Elementwise and HBM-bound: a warp owns a (b, t, h) row and each lane four
+// consecutive channels (16-byte fp32 or 8-byte bf16 accesses); the grid is a
 // multiple of the SM count and strides over all rows.
 #include "common.cuh"
 #include "kda_internal.h"
@@ -15,34 +15,37 @@ __device__ __forceinline__ float gate_sigmoid(float x) {
   return e / (1.f + e);
 }
 
+// One warp per (b, t, h) row: the row's coordinates are decomposed once (32-bit
+// arithmetic), A_log is read once, and the lanes stride over its K/4 channel quads.
 template <typename T>
 __global__ void __launch_bounds__(256) bounded_decay_kernel(GateParams p) {
-  const int64_t quads = p.K / 4;
-  const int64_t total = p.B * p.T * p.H * quads;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    int64_t c4 = i % quads;
-    int64_t r = i / quads;
-    int64_t h = r % p.H;
-    r /= p.H;
-    int64_t t = r % p.T;
-    int64_t b = r / p.T;
-    const T* zp = static_cast<const T*>(p.z) + b * p.zs[0] + t * p.zs[1] + h * p.zs[2] + 4 * c4;
-    T* op = static_cast<T*>(p.out) + b * p.os[0] + t * p.os[1] + h * p.os[2] + 4 * c4;
-    float scale = expf(__ldg(p.A_log + h));
-    float4 z = load4(zp);
-    float4 g;
-    g.x = p.g_min * gate_sigmoid(scale * z.x);
-    g.y = p.g_min * gate_sigmoid(scale * z.y);
-    g.z = p.g_min * gate_sigmoid(scale * z.z);
-    g.w = p.g_min * gate_sigmoid(scale * z.w);
-    if (!p.out_log) {
-      g.x = expf(g.x);
-      g.y = expf(g.y);
-      g.z = expf(g.z);
-      g.w = expf(g.w);
+  const int lane = threadIdx.x & 31;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const uint32_t rows = (uint32_t)(p.B * p.T * p.H);
+  const uint32_t H = (uint32_t)p.H, Tn = (uint32_t)p.T;
+  const int quads = (int)(p.K / 4);
+  for (uint32_t r = warp; r < rows; r += nwarps) {
+    const uint32_t h = r % H, bt = r / H;
+    const uint32_t t = bt % Tn, b = bt / Tn;
+    const T* zp = static_cast<const T*>(p.z) + b * p.zs[0] + t * p.zs[1] + h * p.zs[2];
+    T* op = static_cast<T*>(p.out) + b * p.os[0] + t * p.os[1] + h * p.os[2];
+    const float scale = expf(__ldg(p.A_log + h));
+    for (int c4 = lane; c4 < quads; c4 += 32) {
+      const float4 z = load4(zp + 4 * c4);
+      float4 g;
+      g.x = p.g_min * gate_sigmoid(scale * z.x);
+      g.y = p.g_min * gate_sigmoid(scale * z.y);
+      g.z = p.g_min * gate_sigmoid(scale * z.z);
+      g.w = p.g_min * gate_sigmoid(scale * z.w);
+      if (!p.out_log) {
+        g.x = expf(g.x);
+        g.y = expf(g.y);
+        g.z = expf(g.z);
+        g.w = expf(g.w);
+      }
+      store4(op + 4 * c4, g);
     }
-    store4(op, g);
   }
 }
 
@@ -50,9 +53,9 @@ cudaError_t launch_gate(const GateParams& p, kda_dtype dt, cudaStream_t s) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t total = p.B * p.T * p.H * (p.K / 4);
-  int64_t want = (total + 255) / 256;
-  int64_t cap = (int64_t)sms * 8;  // 8 resident 256-thread blocks per SM
+  const int64_t rows = p.B * p.T * p.H;  // one warp per row, 8 warps per block
+  const int64_t want = (rows + 7) / 8;
+  const int64_t cap = (int64_t)sms * 8;   // 8 resident 256-thread blocks per SM
   int grid = (int)(want < cap ? want : cap);
   if (grid < 1) grid = 1;
   if (dt == KDA_F32)

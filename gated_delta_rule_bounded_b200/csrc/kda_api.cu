@@ -89,6 +89,8 @@ int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda
   if (B * T * H * K == 0) return ok();
   if (!logits || !A_log || !out) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: null pointer");
   if (K % 4 != 0) return fail(KDA_ERR_UNSUPPORTED, "kda_bounded_decay: K must be a multiple of 4 (got %lld)", (long long)K);
+  if (B * T * H >= (int64_t)INT32_MAX)
+    return fail(KDA_ERR_UNSUPPORTED, "kda_bounded_decay: B*T*H must be below 2^31 rows");
   kda_strides zs = logits_strides ? *logits_strides : contiguous(T, H, K);
   kda_strides os = out_strides ? *out_strides : contiguous(T, H, K);
   if (!strides_valid(zs) || !strides_valid(os)) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: negative stride");
