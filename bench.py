@@ -90,7 +90,11 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs.
+
+    A reader thread collects the CSV lines. Entering waits for the first sample
+    (so the sampler is running before the timed region starts); leaving waits
+    for one more sample after it ends, so even a short region is covered."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -99,34 +103,53 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
-        self.out = None
+        self.lines = []
+        self.thread = None
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
+    def _wait_lines(self, n, timeout):
+        t_end = time.time() + timeout
+        while len(self.lines) < n and time.time() < t_end:
+            time.sleep(0.01)
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.25)
+            return self
+        self.thread = threading.Thread(target=self._reader, daemon=True)
+        self.thread.start()
+        self._wait_lines(1, 3.0)
+        self.first = len(self.lines)
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            time.sleep(0.15)
-            self.proc.terminate()
-            try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                self.out, _ = self.proc.communicate()
+        if self.proc is None:
+            return False
+        self._wait_lines(len(self.lines) + 1, 1.0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        return False
 
     def summary(self):
-        if not self.out:
+        if not self.lines:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.out.strip().splitlines():
+        # samples from just before the timed region to just after it
+        for line in self.lines[max(0, self.first - 1):]:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue

@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["bounded_decay", "prefill", "decode_step", "prefill_workspace_bytes", "KDAError",
+__all__ = ["bounded_decay", "prefill", "decode_step", "prefill_workspace_bytes", "device_status", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -77,6 +77,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_last_error.argtypes = []
     lib.kda_version.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
+    lib.kda_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+    lib.kda_device_status.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
@@ -261,3 +263,10 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
         KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), state.data_ptr(),
         B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
     return out
+
+
+def device_status(reset: bool = True) -> bool:
+    """Synchronises the device; True if a kernel's bounded wait expired since the last reset."""
+    flag = ctypes.c_int(0)
+    _check("kda_device_status", load_library().kda_device_status(ctypes.byref(flag), int(reset)))
+    return bool(flag.value)

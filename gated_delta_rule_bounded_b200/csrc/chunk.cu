@@ -1,105 +1,123 @@
-// chunk.cu -- chunked prefill of the bounded-decay gated delta rule (bf16 q/k/v).
+// chunk.cu -- chunked prefill of the bounded-decay gated delta rule (bf16 q/k/v) on
+// sm_100a: the per-chunk state products run on tcgen05 tensor cores with the
+// fp32 state held in tensor memory (TMEM).
 //
 // Math ("KDA cheat sheet", Chunkwise parallel form, eqs. 3-4, with the UT
 // transform re-derived from eq. 1 of "Kimi K3: Bounded Decay and Delta
 // Memory"). For a chunk of C = 64 tokens starting from state S0 (K x V), with
-// G the chunk-local inclusive cumulative log-decay per channel and
-// Gamma = exp(G):
+// G the chunk-local inclusive cumulative log-decay per channel and Gamma = exp(G):
 //   A_kk[t,i] = beta_t sum_c k_tc k_ic exp(G_tc - G_ic)        (i < t)
 //   A_qk[t,i] =        sum_c q_tc k_ic exp(G_tc - G_ic)        (i <= t)
-//   T = (I + A_kk)^-1,  W = T Diag(beta)(K*Gamma),  Ut = T Diag(beta) V
-//   U = Ut - W S0
-//   O = (Q*Gamma) S0 + A_qk U
-//   S = Diag(gamma_C) S0 + (K * gamma_C/Gamma)^T U
+//   T' = (I + A_kk)^-1 Diag(beta),  W = T' (K*Gamma),  Ut = T' V
+//   U = Ut - W S0,  O = (Q*Gamma) S0 + A_qk U,  S = Diag(gamma_C) S0 + (K * gamma_C/Gamma)^T U
 //
-// Numerics of the decay ratios. exp(G_t - G_i) <= 1 for i <= t, but the
-// factored form (q exp(G_t)) (k exp(-G_i)) overflows over 64 tokens (G reaches
-// -320). The chunk is split into four 16-token blocks and every factor is
-// taken against a block boundary: with s_a the token before block a and r_b
-// the last token of block b,
+// Decay ratios. exp(G_t - G_i) <= 1 for i <= t, but the factored form
+// (q exp(G_t))(k exp(-G_i)) overflows over 64 tokens (G reaches -320). The
+// chunk is split into four 16-token blocks and every factor is taken against
+// a block boundary: with s_a the token before block a and r_b the last token
+// of block b,
 //   q_t exp(G_t - G_ic) = [q_t exp(G_t - G_{s_a})] exp(G_{s_a} - G_{r_b}) [k_i exp(G_{r_b} - G_i)]
 // for t in block a, i in block b <= a. The bracketed factors are <= 1; the
 // middle per-channel factor is <= 1 off the diagonal and at most the decay of
-// 15 tokens on it, which the lower bound on g (>= -5.5 here) keeps below
-// e^83, inside the bf16/fp32 range ("KDA cheat sheet", Lower-bounded decay:
-// the bound is what lets every tile, the diagonal included, be a dense matmul).
-// Every other operand (Q*Gamma, K*Gamma, K*gamma_C/Gamma) is <= 1 times q or k.
+// 15 tokens on it, which the lower bound on g (clamped at -5.5 here) keeps
+// below e^83, inside the bf16/fp32 range ("KDA cheat sheet", Lower-bounded
+// decay: the bound is what lets every tile, the diagonal included, be a dense
+// matmul). Q*Gamma, K*Gamma and K*gamma_C/Gamma are <= 1 times q or k.
 //
-// Kernel organisation. One CTA owns one (sequence, head, 128-wide V-tile) and
-// walks its chunks in order; 8 warps; K = 128. The fp32 state lives in the
-// accumulator registers of the state-update MMA (warp w owns key rows
-// 16w..16w+15, all 128 value columns) and a bf16 copy in shared memory feeds
-// the W*S and (Q*Gamma)*S products. All contractions are bf16 tensor-core MMAs
-// with fp32 accumulation (mma.sync m16n8k16); the 64x64 triangular inverse is
-// blocked forward substitution in fp32 on 16x16 blocks. The next chunk's q, k,
-// g are fetched with cp.async as soon as the decay pass has consumed them, and
-// its v and beta once the UT products are done, so loads overlap the MMAs.
-// Tokens past the end of a sequence are zero-filled with g = 0 and beta = 0,
-// which leaves the state unchanged.
+// Organisation. One CTA (8 warps) owns one (sequence, head, 128-wide V-tile)
+// and walks its chunks in order; K = 128. The state is kept transposed,
+// S^T (V x K, fp32), in TMEM lanes 0..127 (one lane per value column), so
+// every state product is an M = 128 tcgen05 MMA issued by one thread:
+//   group 1:  W^T = (K*Gamma)^T T'^T,  U^T = V^T T'^T,  O^T = S^T (Q*Gamma)^T
+//   group 2:  U^T += S^T (-W)^T
+//   group 3:  O^T += U^T A_qk^T,       S^T += U^T (K*gamma_C/Gamma)   (S^T pre-scaled by gamma_C)
+// Operands are bf16 tiles in shared memory in the 128-byte-swizzled canonical
+// layouts; accumulators are fp32 in TMEM. Between groups all 8 warps move
+// accumulators out of TMEM (one TMEM lane per thread, one contiguous smem row
+// per thread). The decay pass and the 16x16 A_qk / A_kk tiles (whose operands
+// need a different decay factor per block pair) stay on the SIMT pipes and
+// mma.sync; the 64x64 triangular inverse is blocked forward substitution in
+// fp32. The next chunk's q, k, g are loaded into registers while the MMAs of
+// the current chunk run, and its v tile and beta by cp.async into a second
+// buffer. Every wait on an mbarrier has an iteration limit; on expiry the
+// kernel records the timeout in a device flag, stops, releases TMEM and
+// returns. Tokens past the end of a sequence are zero-filled with g = 0 and
+// beta = 0, which leaves the state unchanged.
 #include <atomic>
 
 #include "common.cuh"
 #include "kda_internal.h"
 
 namespace kda {
+
+// Set to 1 by any chunk-kernel CTA whose bounded wait on an MMA completion expired.
+__device__ int g_chunk_timeout = 0;
+
 namespace {
 
 constexpr int C = 64;     // tokens per chunk
-constexpr int KD = 128;   // key dim (rows of the state)
+constexpr int KD = 128;   // key dim
 constexpr int VT = 128;   // value columns per CTA
 constexpr int NTHREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
-// Lower clamp of the per-token log2-decay: g >= -5.5 (natural log).
-constexpr float G2_MIN = -5.5f * LOG2E;
+constexpr float G2_MIN = -5.5f * LOG2E;  // lower clamp of the per-token log2-decay
 
-// Shared-memory map (bytes). Regions are reused once their first content is dead.
-constexpr int OFF_RAWQ = 0;                  // bf16 [64][128], plain rows
-constexpr int OFF_RAWK = OFF_RAWQ + 16384;   // bf16 [64][128], plain rows
-constexpr int OFF_RAWV = OFF_RAWK + 16384;   // bf16 [64][128], swizzled (ldmatrix source)
-constexpr int OFF_RAWG = OFF_RAWV + 16384;   // f32  [64][128], plain rows
-constexpr int OFF_BETA = OFF_RAWG + 32768;   // f32  [64]
-constexpr int OFF_QE = OFF_BETA + 256;       // bf16 [64][128] q*exp(G_t - G_s)
-constexpr int OFF_KE = OFF_QE + 16384;       // bf16 [64][128] k*exp(G_t - G_s); later U
-constexpr int OFF_KC = OFF_KE + 16384;       // bf16 [64][128] k*exp(G_r - G_t)
-constexpr int OFF_AKK = OFF_KC + 16384;      // f32 [64][64] A_kk; later T as bf16 [64][64]
-constexpr int OFF_TF = OFF_AKK + 16384;      // f32 [64][64] T; later -W bf16 [64][128]; then O staging
-constexpr int OFF_AQK = OFF_TF + 16384;      // bf16 [64][64] A_qk
-constexpr int OFF_S = OFF_AQK + 8192;        // bf16 [128][128] state copy
-constexpr int OFF_VEC = OFF_S + 32768;       // f32 per-channel vectors
-constexpr int VEC_D = 0;                     // [10][128] exp(G_{s_a} - G_{r_b}), pairs a >= b
-constexpr int VEC_GS = VEC_D + 10 * 128;     // [4][128]  exp(G_{s_a}) (Gamma at block starts)
-constexpr int VEC_P = VEC_GS + 4 * 128;      // [4][128]  exp(G_C - G_{r_b})
-constexpr int VEC_GAM = VEC_P + 4 * 128;     // [128]     exp(G_C) = gamma_C
-constexpr int VEC_TOT = VEC_GAM + 128;       // [4][128]  per-block log2-decay sums
-constexpr int VEC_FLOATS = VEC_TOT + 4 * 128;
-constexpr int SMEM_BYTES = OFF_VEC + VEC_FLOATS * 4;
+// Shared-memory map (bytes). Every bf16 operand tile uses 128-byte rows with the
+// 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r & 7)); tiles
+// with 128 columns are two 64-column "atoms" stored one after the other.
+constexpr int OFF_V = 0;          // 2 x 16K  v tile [i][v], two v-halves (MN-major A of U^T)
+constexpr int OFF_QE = 32768;     // 16K  q*exp(G_t - G_s) [t][c]; later T (fp32 [64][64])
+constexpr int OFF_KE = 49152;     // 16K  k*exp(G_t - G_s) [t][c]; later T' (bf16 [t][i], K-major B)
+constexpr int OFF_KC = 65536;     // 16K  k*exp(G_r - G_t) [t][c]
+constexpr int OFF_AKK = 81920;    // 16K  A_kk fp32 [64][64]
+constexpr int OFF_QG = 98304;     // 16K  Q*Gamma [t][c] (K-major B); later -W [c][t] (MN-major B)
+constexpr int OFF_KG = 114688;    // 16K  K*Gamma [i][c] (MN-major A); later U [v][i] (K-major A)
+constexpr int OFF_KT = 131072;    // 16K  K*gamma_C/Gamma [t][c] (MN-major B)
+constexpr int OFF_AQK = 147456;   // 8K   A_qk bf16 [t][i] (K-major B)
+constexpr int OFF_S = 155648;     // 32K  S bf16 [v][c], two c-atoms of [128][64] (K-major A)
+constexpr int OFF_BETA = 188416;  // 2 x 64 fp32
+constexpr int OFF_VEC = 188928;   // fp32 vectors
+constexpr int VEC_D = 0;          // [10][128] exp(G_{s_a} - G_{r_b}), pairs a >= b
+constexpr int VEC_GAM = 1280;     // [128]     gamma_C
+constexpr int VEC_TOT = 1408;     // [4][128]  per-block log2-decay sums
+constexpr int VEC_FLOATS = 1920;
+constexpr int OFF_BAR = OFF_VEC + VEC_FLOATS * 4;  // mbarrier (8 B) + TMEM base (4 B)
+constexpr int SMEM_BYTES = OFF_BAR + 64;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(OFF_S % 1024 == 0 && OFF_AQK % 1024 == 0 && OFF_KT % 1024 == 0, "swizzle atoms need 1 KB alignment");
+
+// TMEM columns (fp32 accumulators; lanes 0..127).
+constexpr uint32_t TM_S = 0;      // S^T [v][c], 128 columns
+constexpr uint32_t TM_U = 128;    // U^T [v][t], 64 columns
+constexpr uint32_t TM_O = 192;    // O^T [v][t], 64 columns
+constexpr uint32_t TM_W = 256;    // W^T [c][t], 64 columns
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t WAIT_LIMIT = 1u << 22;
 
 // ---------------------------------------------------------------------------------------------
-// Small PTX helpers
+// PTX helpers
 // ---------------------------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// 16-byte chunk j of row r in a tile with 256-byte (128 x bf16) or 128-byte rows, XOR-swizzled
-// so that eight consecutive rows at the same chunk fall in distinct bank groups.
-__device__ __forceinline__ uint32_t swz256(int r, int j) { return r * 256 + ((j ^ (r & 7)) << 4); }
-__device__ __forceinline__ uint32_t swz128(int r, int j) { return r * 128 + ((j ^ (r & 7)) << 4); }
-__device__ __forceinline__ uint32_t swz256_e(int r, int c) { return swz256(r, c >> 3) + ((c & 7) << 1); }
-__device__ __forceinline__ uint32_t swz128_e(int r, int c) { return swz128(r, c >> 3) + ((c & 7) << 1); }
+// Byte offset of element (r, c) in a tile of 128-byte rows (64 bf16 per atom); atom_bytes is the
+// distance between the two 64-column atoms of a 128-column tile.
+__device__ __forceinline__ uint32_t sw_e(int r, int c, int atom_bytes) {
+  return (c >> 6) * atom_bytes + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+// Byte offset of the 16-byte chunk holding columns 8j..8j+7 of row r.
+__device__ __forceinline__ uint32_t sw_chunk(int r, int j, int atom_bytes) {
+  return (j >> 3) * atom_bytes + r * 128 + (((j & 7) ^ (r & 7)) << 4);
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
 
-// D += A * B, m16n8k16, bf16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -124,9 +142,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+}
 __device__ __forceinline__ uint32_t scale2(uint32_t u, float s0, float s1) {
-  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
-  float2 f = __bfloat1622float2(v);
+  const float2 f = unpack_bf16(u);
   return pack_bf16(f.x * s0, f.y * s1);
 }
 
@@ -140,6 +160,74 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool va
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: 128-byte swizzle, start address, leading and stride byte offsets.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+               "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tm_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Waits for phase `parity` of the mbarrier with an iteration limit. Returns false (and records
+// the timeout) when the limit expires.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    if (done) return true;
+  }
+  atomicExch(&g_chunk_timeout, 1);
+  return false;
+}
+
+__device__ __forceinline__ uint4 pack8(const uint32_t (&r)[32], int j, float sign) {
+  uint4 w;
+  w.x = pack_bf16(sign * __uint_as_float(r[8 * j + 0]), sign * __uint_as_float(r[8 * j + 1]));
+  w.y = pack_bf16(sign * __uint_as_float(r[8 * j + 2]), sign * __uint_as_float(r[8 * j + 3]));
+  w.z = pack_bf16(sign * __uint_as_float(r[8 * j + 4]), sign * __uint_as_float(r[8 * j + 5]));
+  w.w = pack_bf16(sign * __uint_as_float(r[8 * j + 6]), sign * __uint_as_float(r[8 * j + 7]));
+  return w;
+}
 
 // ---------------------------------------------------------------------------------------------
 // The kernel
@@ -155,49 +243,55 @@ struct ChunkCtx {
   int64_t qst, kst, vst, gst, bst;       // element strides between tokens
 };
 
-// q, k, g of chunk c (tokens tc0 .. tc0+nv-1) into the raw buffers; rows >= nv are zero-filled.
-__device__ __forceinline__ void load_qkg(const ChunkCtx& x, uint32_t sb, int64_t tc0, int nv, int tid) {
+// Registers holding one thread's share of a chunk's q, k, g: channels c0, c0+1 of the 16 tokens
+// of block a (thread = (channel pair, block)).
+struct Prefetch {
+  float2 g[16];
+  uint32_t q[16], k[16];
+};
+
+__device__ __forceinline__ void load_qkg(const ChunkCtx& x, int64_t tc0, int nv, int c0, int a, Prefetch& pf) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int idx = tid + NTHREADS * i;
-    const int row = idx >> 4, piece = idx & 15;
-    const bool ok = row < nv;
-    const int64_t t = tc0 + (ok ? row : 0);
-    cp_async16(sb + OFF_RAWQ + row * 256 + piece * 16, x.q + x.qrow + t * x.qst + piece * 8, ok);
-    cp_async16(sb + OFF_RAWK + row * 256 + piece * 16, x.k + x.krow + t * x.kst + piece * 8, ok);
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int idx = tid + NTHREADS * i;
-    const int row = idx >> 5, piece = idx & 31;
-    const bool ok = row < nv;
-    const int64_t t = tc0 + (ok ? row : 0);
-    cp_async16(sb + OFF_RAWG + row * 512 + piece * 16, x.gate + x.grow + t * x.gst + piece * 4, ok);
+  for (int i = 0; i < 16; ++i) {
+    const int row = 16 * a + i;
+    if (row < nv) {
+      const int64_t t = tc0 + row;
+      pf.g[i] = *reinterpret_cast<const float2*>(x.gate + x.grow + t * x.gst + c0);
+      pf.q[i] = *reinterpret_cast<const uint32_t*>(x.q + x.qrow + t * x.qst + c0);
+      pf.k[i] = *reinterpret_cast<const uint32_t*>(x.k + x.krow + t * x.kst + c0);
+    } else {
+      pf.g[i] = make_float2(0.f, 0.f);
+      pf.q[i] = pf.k[i] = 0u;
+    }
   }
 }
 
-// v tile and beta of chunk c.
-__device__ __forceinline__ void load_vb(const ChunkCtx& x, uint32_t sb, int64_t tc0, int nv, int tid) {
+// v tile (into the MN-major operand layout) and beta of a chunk.
+__device__ __forceinline__ void load_vb(const ChunkCtx& x, uint32_t vbase, uint32_t bbase, int64_t tc0, int nv,
+                                        int tid) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int idx = tid + NTHREADS * i;
     const int row = idx >> 4, piece = idx & 15;
     const bool ok = row < nv;
     const int64_t t = tc0 + (ok ? row : 0);
-    cp_async16(sb + OFF_RAWV + swz256(row, piece), x.v + x.vrow + t * x.vst + piece * 8, ok);
+    cp_async16(vbase + (piece >> 3) * 8192 + row * 128 + (((piece & 7) ^ (row & 7)) << 4),
+               x.v + x.vrow + t * x.vst + piece * 8, ok);
   }
   if (tid < C) {
     const bool ok = tid < nv;
     const int64_t t = tc0 + (ok ? tid : 0);
-    cp_async4(sb + OFF_BETA + tid * 4, x.beta + x.boff + t * x.bst, ok);
+    cp_async4(bbase + tid * 4, x.beta + x.boff + t * x.bst, ok);
   }
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p) {
-  extern __shared__ __align__(128) unsigned char sm[];
+  extern __shared__ __align__(1024) unsigned char sm[];
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
+  const int quad = warp & 3, half = warp >> 2;   // TMEM lane quadrant, column half (epilogues)
+  const int trow = 32 * quad + lane;             // the TMEM lane this thread moves
 
   const int n_vt = p.V / VT;
   int blk = blockIdx.x;
@@ -232,109 +326,137 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
   x.bst = p.bs[1];
 
   float* vec = reinterpret_cast<float*>(sm + OFF_VEC);
-  const float* beta_s = reinterpret_cast<const float*>(sm + OFF_BETA);
+  const uint32_t bar = sb + OFF_BAR;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 8);
 
+  // decay-pass ownership: channel pair (c0, c0+1) of block da
+  const int c0 = 2 * (tid & 63), da = tid >> 6;
+
+  Prefetch pf;
   if (n_chunks > 0) {
-    load_qkg(x, sb, t0, (int)min((int64_t)C, t1 - t0), tid);
-    load_vb(x, sb, t0, (int)min((int64_t)C, t1 - t0), tid);
+    const int nv0 = (int)min((int64_t)C, t1 - t0);
+    load_vb(x, sb + OFF_V, sb + OFF_BETA, t0, nv0, tid);
     cp_async_commit();
+    load_qkg(x, t0, nv0, c0, da, pf);
   }
 
-  // State: warp owns key rows 16*warp + {g, g+8}; n8 tile j covers value columns 8j .. 8j+7.
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(TM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tlane = tmem + ((uint32_t)(32 * quad) << 16);  // this warp's TMEM lane quadrant
+
+  // Initial state: TMEM lane v = trow holds column v of S; this thread moves columns [64*half, +64).
   const size_t sbase = ((size_t)n * p.H + h) * (size_t)KD * p.V + (size_t)vt * VT;
-  const int srow0 = 16 * warp + g, srow1 = srow0 + 8;
-  float S[16][4];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int col = 8 * j + 2 * tq;
-    if (p.s0) {
-      const float2 a = *reinterpret_cast<const float2*>(p.s0 + sbase + (size_t)srow0 * p.V + col);
-      const float2 b = *reinterpret_cast<const float2*>(p.s0 + sbase + (size_t)srow1 * p.V + col);
-      S[j][0] = a.x; S[j][1] = a.y; S[j][2] = b.x; S[j][3] = b.y;
-    } else {
-      S[j][0] = S[j][1] = S[j][2] = S[j][3] = 0.f;
-    }
-    *reinterpret_cast<uint32_t*>(sm + OFF_S + swz256_e(srow0, col)) = pack_bf16(S[j][0], S[j][1]);
-    *reinterpret_cast<uint32_t*>(sm + OFF_S + swz256_e(srow1, col)) = pack_bf16(S[j][2], S[j][3]);
+  for (int part = 0; part < 2; ++part) {
+    const int cb = 64 * half + 32 * part;
+    uint32_t r[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      r[j] = __float_as_uint(p.s0 ? p.s0[sbase + (size_t)(cb + j) * p.V + trow] : 0.f);
+    tm_st32(tlane + TM_S + cb, r);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4*>(sm + OFF_S + sw_chunk(trow, (cb >> 3) + j, 16384)) = pack8(r, j, 1.f);
   }
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 
-  const int m = warp & 3, nh = warp >> 2;  // 16-row block and 64-column half for the 64x128 products
+  uint32_t phase = 0;
+  bool ok = true;
 
-  for (int c = 0; c < n_chunks; ++c) {
+  for (int c = 0; c < n_chunks && ok; ++c) {
     const int64_t tc0 = t0 + (int64_t)c * C;
     const int nv = (int)min((int64_t)C, t1 - tc0);
     const bool has_next = c + 1 < n_chunks;
     const int64_t tn0 = tc0 + C;
     const int nvn = has_next ? (int)min((int64_t)C, t1 - tn0) : 0;
+    const uint32_t vbuf = sb + OFF_V + (c & 1) * 16384;
+    const float* beta_s = reinterpret_cast<const float*>(sm + OFF_BETA + (c & 1) * 256);
 
     cp_async_wait_all();
-    __syncthreads();  // raw inputs of chunk c are in shared memory; the previous state copy is written
-
-    // ---- decay pass: block-local cumulative log2-decay, scaled copies of q and k ----------------
-    {
-      const int ch = tid & 127, half = tid >> 7;
-      const float* rg = reinterpret_cast<const float*>(sm + OFF_RAWG);
-      const __nv_bfloat16* rq = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_RAWQ);
-      const __nv_bfloat16* rk = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_RAWK);
-#pragma unroll
-      for (int bb = 0; bb < 2; ++bb) {
-        const int a = half * 2 + bb;
-        float pre[16];
-        float run = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = a * 16 + i;
-          float g2 = 0.f;
-          if (t < nv) {
-            const float gv = rg[t * 128 + ch];
-            g2 = p.gate_log ? gv * LOG2E : lg2(gv);
-            g2 = fmaxf(g2, G2_MIN);
-          }
-          run += g2;
-          pre[i] = run;
-        }
-        vec[VEC_TOT + a * 128 + ch] = run;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = a * 16 + i;
-          const float E = ex2(pre[i]);        // exp(G_t - G_{s_a}) <= 1
-          const float F = ex2(run - pre[i]);  // exp(G_{r_a} - G_t) <= 1
-          const float qv = __bfloat162float(rq[t * 128 + ch]);
-          const float kv = __bfloat162float(rk[t * 128 + ch]);
-          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_QE + swz256_e(t, ch)) = __float2bfloat16_rn(qv * E);
-          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_KE + swz256_e(t, ch)) = __float2bfloat16_rn(kv * E);
-          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_KC + swz256_e(t, ch)) = __float2bfloat16_rn(kv * F);
-        }
-      }
-    }
-    __syncthreads();  // raw q, k, g consumed; block sums published
-
-    if (has_next) load_qkg(x, sb, tn0, nvn, tid);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // v tile and beta of chunk c landed; the previous chunk is fully retired
+    tc_fence_after();
+    if (has_next) load_vb(x, sb + OFF_V + ((c + 1) & 1) * 16384, sb + OFF_BETA + ((c + 1) & 1) * 256, tn0, nvn, tid);
     cp_async_commit();
 
-    if (tid < 128) {
-      const int ch = tid;
-      const float e0 = vec[VEC_TOT + ch];
-      const float e1 = e0 + vec[VEC_TOT + 128 + ch];
-      const float e2 = e1 + vec[VEC_TOT + 256 + ch];
-      const float e3 = e2 + vec[VEC_TOT + 384 + ch];
-      const float gs[4] = {0.f, e0, e1, e2};  // log2 Gamma at s_a
-      const float ge[4] = {e0, e1, e2, e3};   // log2 Gamma at r_b
-      int idx = 0;
+    // ---- decay pass, step 1: block-local cumulative log2-decay of (c0, c0+1) over block da -----
+    float2 pre[16];
+    {
+      float2 run = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b <= a; ++b) vec[VEC_D + (idx++) * 128 + ch] = ex2(gs[a] - ge[b]);
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        vec[VEC_GS + a * 128 + ch] = ex2(gs[a]);
-        vec[VEC_P + a * 128 + ch] = ex2(e3 - ge[a]);
+      for (int i = 0; i < 16; ++i) {
+        float2 l = make_float2(0.f, 0.f);
+        if (16 * da + i < nv) {
+          l.x = p.gate_log ? pf.g[i].x * LOG2E : lg2(pf.g[i].x);
+          l.y = p.gate_log ? pf.g[i].y * LOG2E : lg2(pf.g[i].y);
+          l.x = fmaxf(l.x, G2_MIN);
+          l.y = fmaxf(l.y, G2_MIN);
+        }
+        run.x += l.x;
+        run.y += l.y;
+        pre[i] = run;
       }
-      vec[VEC_GAM + ch] = ex2(e3);
+      *reinterpret_cast<float2*>(vec + VEC_TOT + da * 128 + c0) = run;
     }
-    __syncthreads();  // decay vectors ready
+    __syncthreads();
+    // ---- step 2: decay factors, scaled operand tiles, per-pair and per-chunk vectors ------------
+    {
+      float2 e[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) e[b] = *reinterpret_cast<const float2*>(vec + VEC_TOT + b * 128 + c0);
+#pragma unroll
+      for (int b = 1; b < 4; ++b) {
+        e[b].x += e[b - 1].x;
+        e[b].y += e[b - 1].y;
+      }
+      // e[b] = log2 Gamma at r_b; log2 Gamma at s_a is e[a-1] (0 for a = 0)
+      const float2 gs = da == 0 ? make_float2(0.f, 0.f) : (da == 1 ? e[0] : (da == 2 ? e[1] : e[2]));
+      const float2 eda = da == 0 ? e[0] : (da == 1 ? e[1] : (da == 2 ? e[2] : e[3]));
+      const float2 tot = pre[15];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        if (b <= da) {
+          const int pair = da * (da + 1) / 2 + b;
+          *reinterpret_cast<float2*>(vec + VEC_D + pair * 128 + c0) = make_float2(ex2(gs.x - e[b].x), ex2(gs.y - e[b].y));
+        }
+      }
+      if (da == 0) *reinterpret_cast<float2*>(vec + VEC_GAM + c0) = make_float2(ex2(e[3].x), ex2(e[3].y));
+      const float2 GS = make_float2(ex2(gs.x), ex2(gs.y));
+      const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * da + i;
+        const float Ex = ex2(pre[i].x), Ey = ex2(pre[i].y);
+        const float Fx = ex2(tot.x - pre[i].x), Fy = ex2(tot.y - pre[i].y);
+        const float2 qf = unpack_bf16(pf.q[i]), kf = unpack_bf16(pf.k[i]);
+        const uint32_t off = sw_e(t, c0, 8192);
+        const float qex = qf.x * Ex, qey = qf.y * Ey, kex = kf.x * Ex, key = kf.y * Ey;
+        const float kfx = kf.x * Fx, kfy = kf.y * Fy;
+        *reinterpret_cast<uint32_t*>(sm + OFF_QE + off) = pack_bf16(qex, qey);
+        *reinterpret_cast<uint32_t*>(sm + OFF_KE + off) = pack_bf16(kex, key);
+        *reinterpret_cast<uint32_t*>(sm + OFF_KC + off) = pack_bf16(kfx, kfy);
+        *reinterpret_cast<uint32_t*>(sm + OFF_QG + off) = pack_bf16(qex * GS.x, qey * GS.y);
+        *reinterpret_cast<uint32_t*>(sm + OFF_KG + off) = pack_bf16(kex * GS.x, key * GS.y);
+        *reinterpret_cast<uint32_t*>(sm + OFF_KT + off) = pack_bf16(kfx * PM.x, kfy * PM.y);
+      }
+    }
+    __syncthreads();  // scaled tiles and vectors ready; the q/k/g registers are free
 
-    // ---- A_qk (warps 0-3) and A_kk (warps 4-7), 16x16 tiles (a, b), a >= b ----------------------
+    if (has_next) load_qkg(x, tn0, nvn, c0, da, pf);
+
+    // ---- A_qk (warps 0-3) and A_kk (warps 4-7) as 16x16 tiles (a, b), a >= b ----------------------
     {
       const int mat = warp >> 2;
       const uint32_t rows = sb + (mat ? OFF_KE : OFF_QE);
@@ -346,14 +468,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-          ldsm_x4(rows + swz256(16 * a + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
-          const int c0 = 16 * kk + 2 * tq;
-          const float d0 = Dv[c0], d1 = Dv[c0 + 1], d8 = Dv[c0 + 8], d9 = Dv[c0 + 9];
-          a0 = scale2(a0, d0, d1);
-          a1 = scale2(a1, d0, d1);
-          a2 = scale2(a2, d8, d9);
-          a3 = scale2(a3, d8, d9);
-          ldsm_x4(sb + OFF_KC + swz256(16 * b + (lane & 7) + (lane >> 4) * 8, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
+          const int ra = 16 * a + (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldsm_x4(rows + sw_chunk(ra, 2 * kk + (lane >> 4), 8192), a0, a1, a2, a3);
+          const int cc = 16 * kk + 2 * tq;
+          const float2 d01 = *reinterpret_cast<const float2*>(Dv + cc);
+          const float2 d89 = *reinterpret_cast<const float2*>(Dv + cc + 8);
+          a0 = scale2(a0, d01.x, d01.y);
+          a1 = scale2(a1, d01.x, d01.y);
+          a2 = scale2(a2, d89.x, d89.y);
+          a3 = scale2(a3, d89.x, d89.y);
+          const int rb = 16 * b + (lane & 7) + (lane >> 4) * 8;
+          ldsm_x4(sb + OFF_KC + sw_chunk(rb, 2 * kk + ((lane >> 3) & 1), 8192), b0, b1, b2, b3);
           mma_bf16(acc[0], a0, a1, a2, a3, b0, b1);
           mma_bf16(acc[1], a0, a1, a2, a3, b2, b3);
         }
@@ -369,7 +494,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
                 v0 = (i0 <= t) ? v0 : 0.f;
                 v1 = (i0 + 1 <= t) ? v1 : 0.f;
               }
-              *reinterpret_cast<uint32_t*>(sm + OFF_AQK + swz128_e(t, i0)) = pack_bf16(v0, v1);
+              *reinterpret_cast<uint32_t*>(sm + OFF_AQK + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
             } else {
               const float bt = beta_s[t];
               v0 = (a > b || i0 < t) ? v0 * bt : 0.f;
@@ -378,13 +503,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
             }
           }
       }
+      // The MMA reads whole rows of A_qk: zero its six blocks above the diagonal.
+      for (int e = tid; e < 6 * 64; e += NTHREADS) {
+        const int pr = e >> 6, r = (e >> 2) & 15, q4 = e & 3;  // block pair, row, group of 4 columns
+        const int a = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
+        const int b = pr < 3 ? pr + 1 : (pr < 5 ? pr - 1 : 3);
+        *reinterpret_cast<uint2*>(sm + OFF_AQK + sw_e(16 * a + r, 16 * b + 4 * q4, 8192)) = make_uint2(0u, 0u);
+      }
     }
-    __syncthreads();  // A_qk, A_kk ready
+    __syncthreads();  // A_qk, A_kk ready; Qe, Ke, Kc are dead
 
-    // ---- T = (I + A_kk)^-1 by blocked forward substitution (fp32) ----------------------------
+    // ---- T' = (I + A_kk)^-1 Diag(beta) by blocked forward substitution (fp32) ---------------------
     {
       const float* L = reinterpret_cast<const float*>(sm + OFF_AKK);
-      float* Tm = reinterpret_cast<float*>(sm + OFF_TF);
+      float* Tm = reinterpret_cast<float*>(sm + OFF_QE);
       if (tid < 64) {
         const int a = tid >> 4, j = tid & 15;
         float xcol[16];
@@ -402,17 +534,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
 #pragma unroll 1
       for (int d = 1; d <= 3; ++d) {
         const int nblk = 4 - d;
-        // P_ab = sum_{j=b}^{a-1} L_aj T_jb, kept in the unused upper block (b, a) of Tm.
         for (int e = tid; e < nblk * 256; e += NTHREADS) {
           const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15, a = b + d;
           float s = 0.f;
           for (int jb = b; jb < a; ++jb)
 #pragma unroll
             for (int l = 0; l < 16; ++l) s += L[(16 * a + r) * 64 + 16 * jb + l] * Tm[(16 * jb + l) * 64 + 16 * b + cc];
-          Tm[(16 * b + r) * 64 + 16 * a + cc] = s;
+          Tm[(16 * b + r) * 64 + 16 * a + cc] = s;  // scratch in the unused upper block (b, a)
         }
         __syncthreads();
-        // T_ab = -T_aa P_ab
         for (int e = tid; e < nblk * 256; e += NTHREADS) {
           const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15, a = b + d;
           float s = 0.f;
@@ -422,188 +552,152 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
         }
         __syncthreads();
       }
-      // T Diag(beta) to bf16 (the A_kk region is dead now): folding beta into T's columns lets
-      // W and Ut take K*Gamma and V without a per-element beta scale. Only blocks on or below
-      // the diagonal are read later.
+      // T' = T Diag(beta) as the K-major B operand [t][i]; entries above the diagonal are zero.
       for (int e = tid; e < 64 * 32; e += NTHREADS) {
         const int r = e >> 5, c2 = (e & 31) * 2;
         const float2 tv = *reinterpret_cast<const float2*>(Tm + r * 64 + c2);
-        *reinterpret_cast<uint32_t*>(sm + OFF_AKK + swz128_e(r, c2)) =
-            pack_bf16(tv.x * beta_s[c2], tv.y * beta_s[c2 + 1]);
+        const float x0 = (c2 <= r) ? tv.x * beta_s[c2] : 0.f;
+        const float x1 = (c2 + 1 <= r) ? tv.y * beta_s[c2 + 1] : 0.f;
+        *reinterpret_cast<uint32_t*>(sm + OFF_KE + sw_e(r, c2, 8192)) = pack_bf16(x0, x1);
       }
     }
-    __syncthreads();  // T (bf16) ready
+    fence_async_smem();
+    __syncthreads();  // every operand of MMA group 1 is in shared memory
 
-    // ---- W = (T Diag(beta)) (K*Gamma) (stored negated), Ut = (T Diag(beta)) V (in registers) ----
-    float accU[8][4];
+    // ---- MMA group 1: W^T, U^T = V^T T'^T, O^T = S^T (Q*Gamma)^T --------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id_w = idesc_bf16(64, 1, 0);   // A MN-major, B K-major, N = 64
+      constexpr uint32_t id_o = idesc_bf16(64, 0, 0);   // A K-major, B K-major, N = 64
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t bt = sdesc(sb + OFF_KE + ks * 32, 16, 1024);
+        tc_mma(tmem + TM_W, sdesc(sb + OFF_KG + ks * 2048, 8192, 1024), bt, id_w, ks > 0);
+        tc_mma(tmem + TM_U, sdesc(vbuf + ks * 2048, 8192, 1024), bt, id_w, ks > 0);
+      }
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        tc_mma(tmem + TM_O, sdesc(sb + OFF_S + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+               sdesc(sb + OFF_QG + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_o, ks > 0);
+      tc_commit(bar);
+    }
+    ok = __syncthreads_and(mbar_wait(bar, phase));  // one decision for the whole CTA
+    phase ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+
+    // ---- epilogue 1: -W to shared memory (MN-major B, row c holds W[0..63][c]); S^T *= gamma_C ----
     {
-      float accW[8][4];
+      uint32_t r[32];
+      tm_ld32(tlane + TM_W + 32 * half, r);
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(sm + OFF_QG + sw_chunk(trow, 4 * half + j, 0)) = pack8(r, j, -1.f);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) accW[j][e] = accU[j][e] = 0.f;
-      for (int kk = 0; kk <= m; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(sb + OFF_AKK + swz128(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
-        const float* gsv = vec + VEC_GS + kk * 128;
-        const int rr = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+      for (int part = 0; part < 2; ++part) {
+        const int cb = 64 * half + 32 * part;
+        tm_ld32(tlane + TM_S + cb, r);
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-          const int col0 = 64 * nh + 16 * pp;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sb + OFF_KE + swz256(rr, (col0 >> 3) + (lane >> 4)), b0, b1, b2, b3);
-          const float gs0 = gsv[col0 + g], gs1 = gsv[col0 + 8 + g];
-          b0 = scale2(b0, gs0, gs0);
-          b1 = scale2(b1, gs0, gs0);
-          b2 = scale2(b2, gs1, gs1);
-          b3 = scale2(b3, gs1, gs1);
-          mma_bf16(accW[2 * pp], a0, a1, a2, a3, b0, b1);
-          mma_bf16(accW[2 * pp + 1], a0, a1, a2, a3, b2, b3);
-          ldsm_x4_t(sb + OFF_RAWV + swz256(rr, (col0 >> 3) + (lane >> 4)), b0, b1, b2, b3);
-          mma_bf16(accU[2 * pp], a0, a1, a2, a3, b0, b1);
-          mma_bf16(accU[2 * pp + 1], a0, a1, a2, a3, b2, b3);
-        }
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * vec[VEC_GAM + cb + j]);
+        tm_st32(tlane + TM_S + cb, r);
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = 64 * nh + 8 * j + 2 * tq;
-        *reinterpret_cast<uint32_t*>(sm + OFF_TF + swz256_e(16 * m + g, col)) = pack_bf16(-accW[j][0], -accW[j][1]);
-        *reinterpret_cast<uint32_t*>(sm + OFF_TF + swz256_e(16 * m + g + 8, col)) = pack_bf16(-accW[j][2], -accW[j][3]);
-      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
-    __syncthreads();  // -W ready; v tile, beta and K*exp(...) are dead
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
 
-    if (has_next) load_vb(x, sb, tn0, nvn, tid);
-    cp_async_commit();
-
-    // ---- U = Ut - W S ---------------------------------------------------------------------------
-#pragma unroll 2
-    for (int kk = 0; kk < 8; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(sb + OFF_TF + swz256(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
-      const int rr = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+    // ---- MMA group 2: U^T += S^T (-W)^T ---------------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id_u = idesc_bf16(64, 0, 1);   // A K-major, B MN-major, N = 64
 #pragma unroll
-      for (int pp = 0; pp < 4; ++pp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sb + OFF_S + swz256(rr, 8 * nh + 2 * pp + (lane >> 4)), b0, b1, b2, b3);
-        mma_bf16(accU[2 * pp], a0, a1, a2, a3, b0, b1);
-        mma_bf16(accU[2 * pp + 1], a0, a1, a2, a3, b2, b3);
-      }
+      for (int ks = 0; ks < 8; ++ks)
+        tc_mma(tmem + TM_U, sdesc(sb + OFF_S + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+               sdesc(sb + OFF_QG + ks * 2048, 8192, 1024), id_u, 1);
+      tc_commit(bar);
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int col = 64 * nh + 8 * j + 2 * tq;
-      *reinterpret_cast<uint32_t*>(sm + OFF_KE + swz256_e(16 * m + g, col)) = pack_bf16(accU[j][0], accU[j][1]);
-      *reinterpret_cast<uint32_t*>(sm + OFF_KE + swz256_e(16 * m + g + 8, col)) = pack_bf16(accU[j][2], accU[j][3]);
-    }
-    __syncthreads();  // U ready
+    ok = __syncthreads_and(mbar_wait(bar, phase));  // one decision for the whole CTA
+    phase ^= 1;
+    tc_fence_after();
+    if (!ok) break;
 
-    // ---- O = (Q*Gamma) S + A_qk U ------------------------------------------------------------
+    // ---- epilogue 2: U to shared memory (K-major A, row v holds U[0..63][v]) ---------------------
     {
-      float accO[8][4];
+      uint32_t r[32];
+      tm_ld32(tlane + TM_U + 32 * half, r);
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) accO[j][e] = 0.f;
-      const float* gsv = vec + VEC_GS + m * 128;
-#pragma unroll 2
-      for (int kk = 0; kk < 8; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(sb + OFF_QE + swz256(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
-        const int c0 = 16 * kk + 2 * tq;
-        const float s0 = gsv[c0], s1 = gsv[c0 + 1], s8 = gsv[c0 + 8], s9 = gsv[c0 + 9];
-        a0 = scale2(a0, s0, s1);
-        a1 = scale2(a1, s0, s1);
-        a2 = scale2(a2, s8, s9);
-        a3 = scale2(a3, s8, s9);
-        const int rr = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sb + OFF_S + swz256(rr, 8 * nh + 2 * pp + (lane >> 4)), b0, b1, b2, b3);
-          mma_bf16(accO[2 * pp], a0, a1, a2, a3, b0, b1);
-          mma_bf16(accO[2 * pp + 1], a0, a1, a2, a3, b2, b3);
-        }
-      }
-      for (int kk = 0; kk <= m; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(sb + OFF_AQK + swz128(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
-        const int rr = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sb + OFF_KE + swz256(rr, 8 * nh + 2 * pp + (lane >> 4)), b0, b1, b2, b3);
-          mma_bf16(accO[2 * pp], a0, a1, a2, a3, b0, b1);
-          mma_bf16(accO[2 * pp + 1], a0, a1, a2, a3, b2, b3);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = 64 * nh + 8 * j + 2 * tq;
-        *reinterpret_cast<uint32_t*>(sm + OFF_TF + swz256_e(16 * m + g, col)) = pack_bf16(accO[j][0], accO[j][1]);
-        *reinterpret_cast<uint32_t*>(sm + OFF_TF + swz256_e(16 * m + g + 8, col)) = pack_bf16(accO[j][2], accO[j][3]);
-      }
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(sm + OFF_KG + sw_chunk(trow, 4 * half + j, 0)) = pack8(r, j, 1.f);
     }
-    __syncthreads();  // O staged; every read of the state copy for this chunk is done
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
 
+    // ---- MMA group 3: O^T += U^T A_qk^T, S^T += U^T (K*gamma_C/Gamma) ----------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id_o = idesc_bf16(64, 0, 0);    // A K-major, B K-major, N = 64
+      constexpr uint32_t id_s = idesc_bf16(128, 0, 1);   // A K-major, B MN-major, N = 128
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t au = sdesc(sb + OFF_KG + ks * 32, 16, 1024);
+        tc_mma(tmem + TM_O, au, sdesc(sb + OFF_AQK + ks * 32, 16, 1024), id_o, 1);
+        tc_mma(tmem + TM_S, au, sdesc(sb + OFF_KT + ks * 2048, 8192, 1024), id_s, 1);
+      }
+      tc_commit(bar);
+    }
+    ok = __syncthreads_and(mbar_wait(bar, phase));  // one decision for the whole CTA
+    phase ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+
+    // ---- epilogue 3: O to global memory, S to its bf16 copy --------------------------------------
     {
+      uint32_t r[32];
+      tm_ld32(tlane + TM_O + 32 * half, r);
       __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o);
-      const int64_t orow = brow * p.os[0] + h * p.os[2] + (int64_t)vt * VT;
+      const int64_t obase = brow * p.os[0] + h * p.os[2] + (int64_t)vt * VT + trow;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int idx = tid + NTHREADS * i;
-        const int row = idx >> 4, piece = idx & 15;
-        if (row < nv) {
-          const uint4 val = *reinterpret_cast<const uint4*>(sm + OFF_TF + swz256(row, piece));
-          *reinterpret_cast<uint4*>(ob + orow + (tc0 + row) * p.os[1] + piece * 8) = val;
-        }
+      for (int j = 0; j < 32; ++j) {
+        const int t = 32 * half + j;
+        if (t < nv) ob[obase + (tc0 + t) * p.os[1]] = __float2bfloat16_rn(__uint_as_float(r[j]));
+      }
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int cb = 64 * half + 32 * part;
+        tm_ld32(tlane + TM_S + cb, r);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(sm + OFF_S + sw_chunk(trow, (cb >> 3) + j, 16384)) = pack8(r, j, 1.f);
       }
     }
-
-    // ---- S = Diag(gamma_C) S + (K * gamma_C/Gamma)^T U ------------------------------------------
-    {
-      const float gm0 = vec[VEC_GAM + srow0], gm1 = vec[VEC_GAM + srow1];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        S[j][0] *= gm0; S[j][1] *= gm0; S[j][2] *= gm1; S[j][3] *= gm1;
-      }
-      const int mi = lane >> 3;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(sb + OFF_KC + swz256(16 * kk + (mi >> 1) * 8 + (lane & 7), 2 * warp + (mi & 1)), a0, a1, a2, a3);
-        const float p0 = vec[VEC_P + kk * 128 + srow0], p1 = vec[VEC_P + kk * 128 + srow1];
-        a0 = scale2(a0, p0, p0);
-        a1 = scale2(a1, p1, p1);
-        a2 = scale2(a2, p0, p0);
-        a3 = scale2(a3, p1, p1);
-        const int rr = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int pp = 0; pp < 8; ++pp) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sb + OFF_KE + swz256(rr, 2 * pp + (lane >> 4)), b0, b1, b2, b3);
-          mma_bf16(S[2 * pp], a0, a1, a2, a3, b0, b1);
-          mma_bf16(S[2 * pp + 1], a0, a1, a2, a3, b2, b3);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int col = 8 * j + 2 * tq;
-        *reinterpret_cast<uint32_t*>(sm + OFF_S + swz256_e(srow0, col)) = pack_bf16(S[j][0], S[j][1]);
-        *reinterpret_cast<uint32_t*>(sm + OFF_S + swz256_e(srow1, col)) = pack_bf16(S[j][2], S[j][3]);
-      }
-    }
+    // (the barrier at the top of the next iteration orders these writes before their readers)
   }
   cp_async_wait_all();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
-  if (p.sf) {
+  if (ok && p.sf) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int col = 8 * j + 2 * tq;
-      *reinterpret_cast<float2*>(p.sf + sbase + (size_t)srow0 * p.V + col) = make_float2(S[j][0], S[j][1]);
-      *reinterpret_cast<float2*>(p.sf + sbase + (size_t)srow1 * p.V + col) = make_float2(S[j][2], S[j][3]);
+    for (int part = 0; part < 2; ++part) {
+      const int cb = 64 * half + 32 * part;
+      uint32_t r[32];
+      tm_ld32(tlane + TM_S + cb, r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) p.sf[sbase + (size_t)(cb + j) * p.V + trow] = __uint_as_float(r[j]);
     }
   }
+  if (!ok) {
+    // A wait expired: give any MMA still in flight one more bounded wait before releasing TMEM.
+    mbar_wait(bar, phase);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TM_COLS));
 }
 
 }  // namespace
@@ -628,6 +722,13 @@ cudaError_t launch_chunk(const ScanParams& p, void*, size_t, cudaStream_t s) {
   if (grid == 0) return cudaSuccess;
   chunk_prefill_kernel<<<(unsigned)grid, NTHREADS, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t chunk_read_timeout(int* flag, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_chunk_timeout, sizeof(int));
+  if (e != cudaSuccess || !reset) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_chunk_timeout, &zero, sizeof(int));
 }
 
 }  // namespace kda

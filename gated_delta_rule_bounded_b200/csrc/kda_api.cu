@@ -74,7 +74,16 @@ extern "C" {
 
 const char* kda_last_error(void) { return g_err; }
 
-const char* kda_version(void) { return "kda-b200 0.1 (sm_100a)"; }
+const char* kda_version(void) { return "kda-b200 0.2 (sm_100a)"; }
+
+int kda_device_status(int* timed_out, int reset) {
+  if (!timed_out) return fail(KDA_ERR_INVALID_ARG, "kda_device_status: null output");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "kda_device_status synchronize");
+  e = kda::chunk_read_timeout(timed_out, reset != 0);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_device_status read");
+  return ok();
+}
 
 int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
                       const float* A_log, float g_min, int64_t B, int64_t T, int64_t H, int64_t K,

@@ -45,6 +45,8 @@ cudaError_t launch_recurrent(const ScanParams& p, kda_dtype dt, cudaStream_t s);
 bool chunk_supported(int K, int V, kda_dtype dt);
 size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t N);
 cudaError_t launch_chunk(const ScanParams& p, void* ws, size_t ws_bytes, cudaStream_t s);
+// Reads (and optionally clears) the chunk kernel's device-side timeout flag. Synchronous.
+cudaError_t chunk_read_timeout(int* flag, bool reset);
 // Copy initial state (or zeros) into final state for T == 0 calls.
 cudaError_t launch_state_copy(const float* s0, float* sf, int64_t n, cudaStream_t s);
 

@@ -155,6 +155,16 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
                     float* state, int64_t B, int64_t H, int64_t K, int64_t V,
                     const kda_layout* layout, void* o, kda_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * kda_device_status: device-side failure flags, for callers that check them
+ * after their work has finished. Every wait inside the library's kernels has
+ * an iteration limit; a kernel whose wait expires stops, records the event in
+ * a device flag and returns instead of hanging. This call synchronises the
+ * current device, writes 1 to *timed_out if any such event has been recorded
+ * since the last reset (0 otherwise), and clears the flag when reset != 0.
+ * ------------------------------------------------------------------------- */
+int kda_device_status(int* timed_out, int reset);
+
 /* Last error of the calling thread ("" when the last call succeeded). */
 const char* kda_last_error(void);
 
