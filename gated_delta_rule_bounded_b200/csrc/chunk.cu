@@ -66,8 +66,10 @@ constexpr float G2_MIN = -5.5f * LOG2E;  // lower clamp of the per-token log2-de
 // 128-byte swizzle (16-byte chunk j of row r stored at chunk j ^ (r & 7)); tiles
 // with 128 columns are two 64-column "atoms" stored one after the other.
 constexpr int OFF_V = 0;          // 2 x 16K  v tile [i][v], two v-halves (MN-major A of U^T)
-constexpr int OFF_QE = 32768;     // 16K  q*exp(G_t - G_s) [t][c]; later T (fp32 [64][64])
-constexpr int OFF_KE = 49152;     // 16K  k*exp(G_t - G_s) [t][c]; later T' (bf16 [t][i], K-major B)
+constexpr int OFF_QE = 32768;     // 16K  q*exp(G_t - G_s) [t][c]
+constexpr int OFF_KE = 49152;     // 16K  k*exp(G_t - G_s) [t][c]; later T' and a bf16 copy of T
+constexpr int OFF_TP = OFF_KE;        // 8K   T' = T Diag(beta), bf16 [t][i] (K-major B)
+constexpr int OFF_TB = OFF_KE + 8192; // 8K   T, bf16 [t][i] (operand of the inverse's products)
 constexpr int OFF_KC = 65536;     // 16K  k*exp(G_r - G_t) [t][c]
 constexpr int OFF_AKK = 81920;    // 16K  A_kk fp32 [64][64]
 constexpr int OFF_QG = 98304;     // 16K  Q*Gamma [t][c] (K-major B); later -W [c][t] (MN-major B)
@@ -77,10 +79,10 @@ constexpr int OFF_AQK = 147456;   // 8K   A_qk bf16 [t][i] (K-major B)
 constexpr int OFF_S = 155648;     // 32K  S bf16 [v][c], two c-atoms of [128][64] (K-major A)
 constexpr int OFF_BETA = 188416;  // 2 x 64 fp32
 constexpr int OFF_VEC = 188928;   // fp32 vectors
-constexpr int VEC_D = 0;          // [10][128] exp(G_{s_a} - G_{r_b}), pairs a >= b
-constexpr int VEC_GAM = 1280;     // [128]     gamma_C
-constexpr int VEC_TOT = 1408;     // [4][128]  per-block log2-decay sums
-constexpr int VEC_FLOATS = 1920;
+constexpr int VEC_D = 0;          // [10][128] bf16 exp(G_{s_a} - G_{r_b}), pairs a >= b (640 floats)
+constexpr int VEC_GAM = 640;      // [128]     gamma_C
+constexpr int VEC_TOT = 768;      // [4][128]  per-block log2-decay sums
+constexpr int VEC_FLOATS = 1280;
 constexpr int OFF_BAR = OFF_VEC + VEC_FLOATS * 4;  // mbarrier (8 B) + TMEM base (4 B)
 constexpr int SMEM_BYTES = OFF_BAR + 64;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -118,6 +120,11 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
 
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -145,9 +152,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
 }
-__device__ __forceinline__ uint32_t scale2(uint32_t u, float s0, float s1) {
-  const float2 f = unpack_bf16(u);
-  return pack_bf16(f.x * s0, f.y * s1);
+// Elementwise bf16x2 product (one rounding of the exact product).
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -251,18 +259,24 @@ struct Prefetch {
 };
 
 __device__ __forceinline__ void load_qkg(const ChunkCtx& x, int64_t tc0, int nv, int c0, int a, Prefetch& pf) {
+  const int64_t t = tc0 + 16 * a;
+  const float* gp = x.gate + x.grow + t * x.gst + c0;
+  const __nv_bfloat16* qp = x.q + x.qrow + t * x.qst + c0;
+  const __nv_bfloat16* kp = x.k + x.krow + t * x.kst + c0;
+  const int imax = nv - 16 * a;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int row = 16 * a + i;
-    if (row < nv) {
-      const int64_t t = tc0 + row;
-      pf.g[i] = *reinterpret_cast<const float2*>(x.gate + x.grow + t * x.gst + c0);
-      pf.q[i] = *reinterpret_cast<const uint32_t*>(x.q + x.qrow + t * x.qst + c0);
-      pf.k[i] = *reinterpret_cast<const uint32_t*>(x.k + x.krow + t * x.kst + c0);
+    if (i < imax) {
+      pf.g[i] = *reinterpret_cast<const float2*>(gp);
+      pf.q[i] = *reinterpret_cast<const uint32_t*>(qp);
+      pf.k[i] = *reinterpret_cast<const uint32_t*>(kp);
     } else {
       pf.g[i] = make_float2(0.f, 0.f);
       pf.q[i] = pf.k[i] = 0u;
     }
+    gp += x.gst;
+    qp += x.qst;
+    kp += x.kst;
   }
 }
 
@@ -282,6 +296,80 @@ __device__ __forceinline__ void load_vb(const ChunkCtx& x, uint32_t vbase, uint3
     const bool ok = tid < nv;
     const int64_t t = tc0 + (ok ? tid : 0);
     cp_async4(bbase + tid * 4, x.beta + x.boff + t * x.bst, ok);
+  }
+}
+
+// 16x16 block pairs (a, b), a >= b, of A_qk (rows from Qe) or A_kk (rows from Ke) against the Kc
+// columns, with the per-pair decay factor D_ab applied to the row operand. The warp takes tiles
+// first, first + stride, ... (nt of them) and runs their k-loops interleaved so the MMA chains
+// overlap. A_qk is stored as a bf16 K-major operand (diagonal blocks masked to i <= t); A_kk as
+// fp32 [64][64] with beta_t applied and diagonal blocks masked to i < t.
+template <int NTMAX>
+__device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const float* vec, int off_rows, int first,
+                                        int stride, int nt, int lane, int g, int tq, const float* beta_s,
+                                        bool is_qk) {
+  int ta[NTMAX], tbk[NTMAX], tid_[NTMAX];
+#pragma unroll
+  for (int n = 0; n < NTMAX; ++n) {
+    const int tile = first + stride * n;
+    tid_[n] = tile;
+    ta[n] = tile >= 6 ? 3 : (tile >= 3 ? 2 : (tile >= 1 ? 1 : 0));
+    tbk[n] = tile - ta[n] * (ta[n] + 1) / 2;
+  }
+  const __nv_bfloat16* D16 = reinterpret_cast<const __nv_bfloat16*>(vec + VEC_D);
+  float acc[NTMAX][2][4];
+#pragma unroll
+  for (int n = 0; n < NTMAX; ++n)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[n][j][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+    for (int n = 0; n < NTMAX; ++n) {
+      if (n < nt) {
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+        const int ra = 16 * ta[n] + (lane & 7) + ((lane >> 3) & 1) * 8;
+        ldsm_x4(sb + off_rows + sw_chunk(ra, 2 * kk + (lane >> 4), 8192), a0, a1, a2, a3);
+        const __nv_bfloat16* Dv = D16 + tid_[n] * 128 + 16 * kk + 2 * tq;
+        const uint32_t d01 = *reinterpret_cast<const uint32_t*>(Dv);
+        const uint32_t d89 = *reinterpret_cast<const uint32_t*>(Dv + 8);
+        a0 = hmul2(a0, d01);
+        a1 = hmul2(a1, d01);
+        a2 = hmul2(a2, d89);
+        a3 = hmul2(a3, d89);
+        const int rb = 16 * tbk[n] + (lane & 7) + (lane >> 4) * 8;
+        ldsm_x4(sb + OFF_KC + sw_chunk(rb, 2 * kk + ((lane >> 3) & 1), 8192), b0, b1, b2, b3);
+        mma_bf16(acc[n][0], a0, a1, a2, a3, b0, b1);
+        mma_bf16(acc[n][1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NTMAX; ++n) {
+    if (n >= nt) continue;
+    const int a = ta[n], b = tbk[n];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int t = 16 * a + g + 8 * hr;
+        const int i0 = 16 * b + 8 * j + 2 * tq;
+        float v0 = acc[n][j][2 * hr], v1 = acc[n][j][2 * hr + 1];
+        if (is_qk) {
+          if (a == b) {
+            v0 = (i0 <= t) ? v0 : 0.f;
+            v1 = (i0 + 1 <= t) ? v1 : 0.f;
+          }
+          *reinterpret_cast<uint32_t*>(sm + OFF_AQK + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
+        } else {
+          const float bt = beta_s[t];
+          v0 = (a > b || i0 < t) ? v0 * bt : 0.f;
+          v1 = (a > b || i0 + 1 < t) ? v1 * bt : 0.f;
+          *reinterpret_cast<float2*>(sm + OFF_AKK + (t * 64 + i0) * 4) = make_float2(v0, v1);
+        }
+      }
   }
 }
 
@@ -391,22 +479,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
     if (has_next) load_vb(x, sb + OFF_V + ((c + 1) & 1) * 16384, sb + OFF_BETA + ((c + 1) & 1) * 256, tn0, nvn, tid);
     cp_async_commit();
 
-    // ---- decay pass, step 1: block-local cumulative log2-decay of (c0, c0+1) over block da -----
-    float2 pre[16];
+    // ---- decay pass, step 1: per-token log2-decay, retention and block sum for (c0, c0+1) ------
+    float2 al[16];  // retention factors of this thread's 16 tokens (1 past the end of a sequence)
     {
       float2 run = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         float2 l = make_float2(0.f, 0.f);
         if (16 * da + i < nv) {
-          l.x = p.gate_log ? pf.g[i].x * LOG2E : lg2(pf.g[i].x);
-          l.y = p.gate_log ? pf.g[i].y * LOG2E : lg2(pf.g[i].y);
-          l.x = fmaxf(l.x, G2_MIN);
-          l.y = fmaxf(l.y, G2_MIN);
+          l.x = fmaxf(p.gate_log ? pf.g[i].x * LOG2E : lg2(pf.g[i].x), G2_MIN);
+          l.y = fmaxf(p.gate_log ? pf.g[i].y * LOG2E : lg2(pf.g[i].y), G2_MIN);
         }
         run.x += l.x;
         run.y += l.y;
-        pre[i] = run;
+        al[i] = make_float2(ex2(l.x), ex2(l.y));
       }
       *reinterpret_cast<float2*>(vec + VEC_TOT + da * 128 + c0) = run;
     }
@@ -424,26 +510,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
       // e[b] = log2 Gamma at r_b; log2 Gamma at s_a is e[a-1] (0 for a = 0)
       const float2 gs = da == 0 ? make_float2(0.f, 0.f) : (da == 1 ? e[0] : (da == 2 ? e[1] : e[2]));
       const float2 eda = da == 0 ? e[0] : (da == 1 ? e[1] : (da == 2 ? e[2] : e[3]));
-      const float2 tot = pre[15];
+      __nv_bfloat16* D16 = reinterpret_cast<__nv_bfloat16*>(vec + VEC_D);
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         if (b <= da) {
           const int pair = da * (da + 1) / 2 + b;
-          *reinterpret_cast<float2*>(vec + VEC_D + pair * 128 + c0) = make_float2(ex2(gs.x - e[b].x), ex2(gs.y - e[b].y));
+          *reinterpret_cast<uint32_t*>(D16 + pair * 128 + c0) = pack_bf16(ex2(gs.x - e[b].x), ex2(gs.y - e[b].y));
         }
       }
       if (da == 0) *reinterpret_cast<float2*>(vec + VEC_GAM + c0) = make_float2(ex2(e[3].x), ex2(e[3].y));
       const float2 GS = make_float2(ex2(gs.x), ex2(gs.y));
       const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));
+      // F_t = prod_{r > t in block} alpha_r (reverse running product), E_t = prod_{r <= t} alpha_r.
+      float2 F[16];
+      F[15] = make_float2(1.f, 1.f);
+#pragma unroll
+      for (int i = 14; i >= 0; --i) F[i] = make_float2(F[i + 1].x * al[i + 1].x, F[i + 1].y * al[i + 1].y);
+      float2 E = make_float2(1.f, 1.f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int t = 16 * da + i;
-        const float Ex = ex2(pre[i].x), Ey = ex2(pre[i].y);
-        const float Fx = ex2(tot.x - pre[i].x), Fy = ex2(tot.y - pre[i].y);
+        E.x *= al[i].x;
+        E.y *= al[i].y;
         const float2 qf = unpack_bf16(pf.q[i]), kf = unpack_bf16(pf.k[i]);
         const uint32_t off = sw_e(t, c0, 8192);
-        const float qex = qf.x * Ex, qey = qf.y * Ey, kex = kf.x * Ex, key = kf.y * Ey;
-        const float kfx = kf.x * Fx, kfy = kf.y * Fy;
+        const float qex = qf.x * E.x, qey = qf.y * E.y, kex = kf.x * E.x, key = kf.y * E.y;
+        const float kfx = kf.x * F[i].x, kfy = kf.y * F[i].y;
         *reinterpret_cast<uint32_t*>(sm + OFF_QE + off) = pack_bf16(qex, qey);
         *reinterpret_cast<uint32_t*>(sm + OFF_KE + off) = pack_bf16(kex, key);
         *reinterpret_cast<uint32_t*>(sm + OFF_KC + off) = pack_bf16(kfx, kfy);
@@ -456,109 +548,89 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
 
     if (has_next) load_qkg(x, tn0, nvn, c0, da, pf);
 
-    // ---- A_qk (warps 0-3) and A_kk (warps 4-7) as 16x16 tiles (a, b), a >= b ----------------------
+    // ---- A_kk on all warps (block pairs (a, b), a >= b), then the inverse on warps 0-3 while
+    //      warps 4-7 form A_qk --------------------------------------------------------------------
     {
-      const int mat = warp >> 2;
-      const uint32_t rows = sb + (mat ? OFF_KE : OFF_QE);
-      for (int tile = warp & 3; tile < 10; tile += 4) {
-        const int a = tile >= 6 ? 3 : (tile >= 3 ? 2 : (tile >= 1 ? 1 : 0));
-        const int b = tile - a * (a + 1) / 2;
-        const float* Dv = vec + VEC_D + tile * 128;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const int nt = warp < 2 ? 2 : 1;
+      a_tiles<2>(sm, sb, vec, OFF_KE, warp, 8, nt, lane, g, tq, beta_s, /*is_qk=*/false);
+    }
+    __syncthreads();  // A_kk ready; Ke is dead
+
+    if (warp < 4) {
+      // T' = (I + A_kk)^-1 Diag(beta): the four 16x16 diagonal inverses by forward substitution in
+      // fp32, then the blocks below the diagonal by distance d = 1, 2, 3 as tensor-core products
+      // T_ab = -sum_{j=b}^{a-1} (T_aa L_aj) T_jb. A bf16 copy of T (second half of the Ke tile)
+      // feeds the products; T' (first half of the Ke tile) is written from the fp32 values.
+      const float* L = reinterpret_cast<const float*>(sm + OFF_AKK);
+      const uint32_t tb = sb + OFF_TB;
+      if (tid < 64) {
+        const int a = tid >> 4, j = tid & 15;
+        float xs[16];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-          const int ra = 16 * a + (lane & 7) + ((lane >> 3) & 1) * 8;
-          ldsm_x4(rows + sw_chunk(ra, 2 * kk + (lane >> 4), 8192), a0, a1, a2, a3);
-          const int cc = 16 * kk + 2 * tq;
-          const float2 d01 = *reinterpret_cast<const float2*>(Dv + cc);
-          const float2 d89 = *reinterpret_cast<const float2*>(Dv + cc + 8);
-          a0 = scale2(a0, d01.x, d01.y);
-          a1 = scale2(a1, d01.x, d01.y);
-          a2 = scale2(a2, d89.x, d89.y);
-          a3 = scale2(a3, d89.x, d89.y);
-          const int rb = 16 * b + (lane & 7) + (lane >> 4) * 8;
-          ldsm_x4(sb + OFF_KC + sw_chunk(rb, 2 * kk + ((lane >> 3) & 1), 8192), b0, b1, b2, b3);
-          mma_bf16(acc[0], a0, a1, a2, a3, b0, b1);
-          mma_bf16(acc[1], a0, a1, a2, a3, b2, b3);
+        for (int i = 0; i < 16; ++i) xs[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l)
+#pragma unroll
+          for (int i = l + 1; i < 16; ++i) xs[i] -= L[(16 * a + i) * 64 + 16 * a + l] * xs[l];
+        const float bj = beta_s[16 * a + j];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t off = sw_e(16 * a + i, 16 * a + j, 8192);
+          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_TB + off) = __float2bfloat16_rn(xs[i]);
+          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_TP + off) = __float2bfloat16_rn(xs[i] * bj);
         }
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            const int t = 16 * a + g + 8 * hr;
-            const int i0 = 16 * b + 8 * j + 2 * tq;
-            float v0 = acc[j][2 * hr], v1 = acc[j][2 * hr + 1];
-            if (mat == 0) {
-              if (a == b) {
-                v0 = (i0 <= t) ? v0 : 0.f;
-                v1 = (i0 + 1 <= t) ? v1 : 0.f;
-              }
-              *reinterpret_cast<uint32_t*>(sm + OFF_AQK + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
-            } else {
-              const float bt = beta_s[t];
-              v0 = (a > b || i0 < t) ? v0 * bt : 0.f;
-              v1 = (a > b || i0 + 1 < t) ? v1 * bt : 0.f;
-              *reinterpret_cast<float2*>(sm + OFF_AKK + (t * 64 + i0) * 4) = make_float2(v0, v1);
-            }
-          }
+      } else {
+        // T' is lower triangular: zero its six blocks above the diagonal.
+        for (int e = tid - 64; e < 6 * 64; e += 64) {
+          const int pr = e >> 6, r = (e >> 2) & 15, q4 = e & 3;
+          const int a = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
+          const int b = pr < 3 ? pr + 1 : (pr < 5 ? pr - 1 : 3);
+          *reinterpret_cast<uint2*>(sm + OFF_TP + sw_e(16 * a + r, 16 * b + 4 * q4, 8192)) = make_uint2(0u, 0u);
+        }
       }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll 1
+      for (int d = 1; d <= 3; ++d) {
+        if (warp < 4 - d) {
+          const int b = warp, a = b + d;
+          float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          uint32_t t0, t1, t2, t3;  // A fragments of T_aa
+          ldsm_x4(tb + sw_chunk(16 * a + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * a + (lane >> 4), 8192), t0, t1, t2, t3);
+          for (int jb = b; jb < a; ++jb) {
+            float P[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // P = T_aa L_{a,jb}; B[k][n] = L[16a + k][16jb + n]
+              const float* lp = L + (16 * a + 2 * tq) * 64 + 16 * jb + 8 * j + g;
+              mma_bf16(P[j], t0, t1, t2, t3, pack_bf16(lp[0], lp[64]), pack_bf16(lp[8 * 64], lp[9 * 64]));
+            }
+            uint32_t b0, b1, b2, b3;  // B = T_{jb,b}
+            ldsm_x4_t(tb + sw_chunk(16 * jb + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * b + (lane >> 4), 8192), b0, b1, b2, b3);
+            const uint32_t p0 = pack_bf16(P[0][0], P[0][1]), p1 = pack_bf16(P[0][2], P[0][3]);
+            const uint32_t p2 = pack_bf16(P[1][0], P[1][1]), p3 = pack_bf16(P[1][2], P[1][3]);
+            mma_bf16(acc[0], p0, p1, p2, p3, b0, b1);
+            mma_bf16(acc[1], p0, p1, p2, p3, b2, b3);
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+              const int row = 16 * a + g + 8 * hr, col = 16 * b + 8 * j + 2 * tq;
+              const float v0 = -acc[j][2 * hr], v1 = -acc[j][2 * hr + 1];
+              const uint32_t off = sw_e(row, col, 8192);
+              *reinterpret_cast<uint32_t*>(sm + OFF_TB + off) = pack_bf16(v0, v1);
+              *reinterpret_cast<uint32_t*>(sm + OFF_TP + off) = pack_bf16(v0 * beta_s[col], v1 * beta_s[col + 1]);
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+    } else {
+      a_tiles<3>(sm, sb, vec, OFF_QE, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
       // The MMA reads whole rows of A_qk: zero its six blocks above the diagonal.
-      for (int e = tid; e < 6 * 64; e += NTHREADS) {
+      for (int e = tid - 128; e < 6 * 64; e += 128) {
         const int pr = e >> 6, r = (e >> 2) & 15, q4 = e & 3;  // block pair, row, group of 4 columns
         const int a = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
         const int b = pr < 3 ? pr + 1 : (pr < 5 ? pr - 1 : 3);
         *reinterpret_cast<uint2*>(sm + OFF_AQK + sw_e(16 * a + r, 16 * b + 4 * q4, 8192)) = make_uint2(0u, 0u);
-      }
-    }
-    __syncthreads();  // A_qk, A_kk ready; Qe, Ke, Kc are dead
-
-    // ---- T' = (I + A_kk)^-1 Diag(beta) by blocked forward substitution (fp32) ---------------------
-    {
-      const float* L = reinterpret_cast<const float*>(sm + OFF_AKK);
-      float* Tm = reinterpret_cast<float*>(sm + OFF_QE);
-      if (tid < 64) {
-        const int a = tid >> 4, j = tid & 15;
-        float xcol[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float s = (i == j) ? 1.f : 0.f;
-#pragma unroll
-          for (int l = 0; l < i; ++l) s -= L[(16 * a + i) * 64 + 16 * a + l] * xcol[l];
-          xcol[i] = s;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Tm[(16 * a + i) * 64 + 16 * a + j] = xcol[i];
-      }
-      __syncthreads();
-#pragma unroll 1
-      for (int d = 1; d <= 3; ++d) {
-        const int nblk = 4 - d;
-        for (int e = tid; e < nblk * 256; e += NTHREADS) {
-          const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15, a = b + d;
-          float s = 0.f;
-          for (int jb = b; jb < a; ++jb)
-#pragma unroll
-            for (int l = 0; l < 16; ++l) s += L[(16 * a + r) * 64 + 16 * jb + l] * Tm[(16 * jb + l) * 64 + 16 * b + cc];
-          Tm[(16 * b + r) * 64 + 16 * a + cc] = s;  // scratch in the unused upper block (b, a)
-        }
-        __syncthreads();
-        for (int e = tid; e < nblk * 256; e += NTHREADS) {
-          const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15, a = b + d;
-          float s = 0.f;
-#pragma unroll
-          for (int l = 0; l < 16; ++l) s += Tm[(16 * a + r) * 64 + 16 * a + l] * Tm[(16 * b + l) * 64 + 16 * a + cc];
-          Tm[(16 * a + r) * 64 + 16 * b + cc] = -s;
-        }
-        __syncthreads();
-      }
-      // T' = T Diag(beta) as the K-major B operand [t][i]; entries above the diagonal are zero.
-      for (int e = tid; e < 64 * 32; e += NTHREADS) {
-        const int r = e >> 5, c2 = (e & 31) * 2;
-        const float2 tv = *reinterpret_cast<const float2*>(Tm + r * 64 + c2);
-        const float x0 = (c2 <= r) ? tv.x * beta_s[c2] : 0.f;
-        const float x1 = (c2 + 1 <= r) ? tv.y * beta_s[c2 + 1] : 0.f;
-        *reinterpret_cast<uint32_t*>(sm + OFF_KE + sw_e(r, c2, 8192)) = pack_bf16(x0, x1);
       }
     }
     fence_async_smem();
@@ -571,7 +643,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
       constexpr uint32_t id_o = idesc_bf16(64, 0, 0);   // A K-major, B K-major, N = 64
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t bt = sdesc(sb + OFF_KE + ks * 32, 16, 1024);
+        const uint64_t bt = sdesc(sb + OFF_TP + ks * 32, 16, 1024);
         tc_mma(tmem + TM_W, sdesc(sb + OFF_KG + ks * 2048, 8192, 1024), bt, id_w, ks > 0);
         tc_mma(tmem + TM_U, sdesc(vbuf + ks * 2048, 8192, 1024), bt, id_w, ks > 0);
       }
@@ -586,28 +658,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
     tc_fence_after();
     if (!ok) break;
 
-    // ---- epilogue 1: -W to shared memory (MN-major B, row c holds W[0..63][c]); S^T *= gamma_C ----
+    // ---- epilogue 1: -W to shared memory (MN-major B, row c holds W[0..63][c]) ---------------------
     {
       uint32_t r[32];
       tm_ld32(tlane + TM_W + 32 * half, r);
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         *reinterpret_cast<uint4*>(sm + OFF_QG + sw_chunk(trow, 4 * half + j, 0)) = pack8(r, j, -1.f);
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int cb = 64 * half + 32 * part;
-        tm_ld32(tlane + TM_S + cb, r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * vec[VEC_GAM + cb + j]);
-        tm_st32(tlane + TM_S + cb, r);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
 
-    // ---- MMA group 2: U^T += S^T (-W)^T ---------------------------------------------------------
+    // ---- MMA group 2: U^T += S^T (-W)^T; meanwhile S^T *= gamma_C in TMEM (group 2 reads the bf16
+    //      copy of S, not TMEM) --------------------------------------------------------------------
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id_u = idesc_bf16(64, 0, 1);   // A K-major, B MN-major, N = 64
@@ -616,6 +680,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
         tc_mma(tmem + TM_U, sdesc(sb + OFF_S + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                sdesc(sb + OFF_QG + ks * 2048, 8192, 1024), id_u, 1);
       tc_commit(bar);
+    }
+    {
+      uint32_t r[32];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int cb = 64 * half + 32 * part;
+        tm_ld32(tlane + TM_S + cb, r);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 gm = *reinterpret_cast<const float4*>(vec + VEC_GAM + cb + 4 * j);
+          r[4 * j + 0] = __float_as_uint(__uint_as_float(r[4 * j + 0]) * gm.x);
+          r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) * gm.y);
+          r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) * gm.z);
+          r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) * gm.w);
+        }
+        tm_st32(tlane + TM_S + cb, r);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
     ok = __syncthreads_and(mbar_wait(bar, phase));  // one decision for the whole CTA
     phase ^= 1;
@@ -656,12 +738,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
     {
       uint32_t r[32];
       tm_ld32(tlane + TM_O + 32 * half, r);
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.o);
-      const int64_t obase = brow * p.os[0] + h * p.os[2] + (int64_t)vt * VT + trow;
+      const int64_t ost = p.os[1];
+      __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + brow * p.os[0] + h * p.os[2] + (int64_t)vt * VT + trow +
+                          (tc0 + 32 * half) * ost;
+      const int jmax = min(32, nv - 32 * half);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const int t = 32 * half + j;
-        if (t < nv) ob[obase + (tc0 + t) * p.os[1]] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        if (j < jmax) *op = __float2bfloat16_rn(__uint_as_float(r[j]));
+        op += ost;
       }
 #pragma unroll
       for (int part = 0; part < 2; ++part) {

@@ -1,0 +1,253 @@
+// decode.cu -- the in-place decode step for K = V = 128, streaming whole head states through
+// shared memory with bulk asynchronous copies.
+//
+// Per head ("Kimi K3: Bounded Decay and Delta Memory", eq. 1, one token):
+//     Sbar = Diag(alpha) S;  delta = v - Sbar^T k;  S = Sbar + beta k delta^T;
+//     o = S^T q = Sbar^T q + beta (k.q) delta
+// The state of one (b, h) is a contiguous 64 KB block, so it moves as one bulk copy
+// (cp.async.bulk, completion counted in bytes on an mbarrier; no multicast). One
+// persistent CTA per SM walks heads blockIdx.x, blockIdx.x + gridDim.x, ... through a
+// 3-stage ring: while head i is computed out of shared memory, head i+1 is loading
+// and head i-1's updated state is being written back by a bulk store. Each thread
+// owns a float4 column group of 16 key rows; the two key reductions are per-thread
+// partial sums plus one shared-memory reduction over the 8 row groups. The state is
+// read from and written to HBM exactly once. Waits are iteration-limited; an expired
+// wait records a device flag and stops the CTA.
+#include <atomic>
+
+#include "common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+// Set to 1 by any decode CTA whose bounded wait on a bulk copy expired.
+__device__ int g_decode_timeout = 0;
+
+namespace {
+
+constexpr int DK = 128, DV = 128, DNT = 256, NSTAGE = 3, ROWS = DK / 8;
+constexpr uint32_t WAIT_LIMIT = 1u << 22;
+
+template <typename TIn>
+struct StageLayout {
+  static constexpr int IN = DK * (int)sizeof(TIn);  // bytes of one q / k / v row
+  static constexpr int STATE = 0;
+  static constexpr int Q = DK * DV * 4;
+  static constexpr int K = Q + IN;
+  static constexpr int V = K + IN;
+  static constexpr int A = V + IN;
+  static constexpr int BYTES = A + DK * 4;          // + alpha row (fp32)
+  static constexpr int RED = NSTAGE * BYTES;        // partial sums [2][8][128] + k.q [8]
+  static constexpr int BAR = RED + (2 * 8 * DV + 8) * 4;
+  static constexpr int SMEM = BAR + NSTAGE * 8;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    if (done) return true;
+  }
+  atomicExch(&g_decode_timeout, 1);
+  return false;
+}
+
+template <typename TIn>
+struct HeadPtrs {
+  const TIn *q, *k, *v;
+  const float *a, *beta;
+  float* state;
+  TIn* o;
+};
+
+template <typename TIn>
+__device__ __forceinline__ HeadPtrs<TIn> head_ptrs(const ScanParams& p, int head) {
+  const int b = head / p.H, h = head % p.H;
+  HeadPtrs<TIn> r;
+  r.q = static_cast<const TIn*>(p.q) + b * p.qs[0] + h * p.qs[2];
+  r.k = static_cast<const TIn*>(p.k) + b * p.ks[0] + h * p.ks[2];
+  r.v = static_cast<const TIn*>(p.v) + b * p.vs[0] + h * p.vs[2];
+  r.a = p.gate + b * p.gs[0] + h * p.gs[2];
+  r.beta = p.beta + b * p.bs[0] + h * p.bs[2];
+  r.state = p.sf + (size_t)head * DK * DV;
+  r.o = static_cast<TIn*>(p.o) + b * p.os[0] + h * p.os[2];
+  return r;
+}
+
+// One thread (tid 0) arms the stage's mbarrier with the byte count and issues the five copies.
+template <typename TIn>
+__device__ __forceinline__ void issue_stage(const ScanParams& p, int head, uint32_t stage_base, uint32_t bar) {
+  using L = StageLayout<TIn>;
+  const HeadPtrs<TIn> hp = head_ptrs<TIn>(p, head);
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"((uint32_t)(L::BYTES))
+               : "memory");
+  bulk_load(stage_base + L::STATE, hp.state, DK * DV * 4, bar);
+  bulk_load(stage_base + L::Q, hp.q, L::IN, bar);
+  bulk_load(stage_base + L::K, hp.k, L::IN, bar);
+  bulk_load(stage_base + L::V, hp.v, L::IN, bar);
+  bulk_load(stage_base + L::A, hp.a, DK * 4, bar);
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
+  using L = StageLayout<TIn>;
+  extern __shared__ __align__(128) unsigned char sm[];
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x;
+  const int tv = tid & 31, tk = tid >> 5;   // column group (4 columns), row group (16 rows)
+  const int row0 = ROWS * tk, col0 = 4 * tv;
+  const int nheads = p.B * p.H;
+  const int n_my = blockIdx.x < nheads ? (nheads - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  float* red_a = reinterpret_cast<float*>(sm + L::RED);
+  float* red_b = red_a + 8 * DV;
+  float* red_kq = red_b + 8 * DV;
+  const uint32_t bar0 = sb + L::BAR;
+
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8 * s));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  int issued = 0;  // heads whose loads have been issued (meaningful in thread 0)
+  if (tid == 0)
+    for (; issued < NSTAGE && issued < n_my; ++issued)
+      issue_stage<TIn>(p, blockIdx.x + issued * gridDim.x, sb + issued * L::BYTES, bar0 + 8 * issued);
+  int done_heads = 0;
+  float beta_next = n_my > 0 ? __ldg(head_ptrs<TIn>(p, blockIdx.x).beta) : 0.f;
+
+  for (int i = 0; i < n_my; ++i) {
+    const int head = blockIdx.x + i * gridDim.x;
+    const int s = i % NSTAGE;
+    unsigned char* st = sm + s * L::BYTES;
+    const float beta = beta_next;
+    if (i + 1 < n_my) beta_next = __ldg(head_ptrs<TIn>(p, head + gridDim.x).beta);
+    if (!__syncthreads_and(mbar_wait(bar0 + 8 * s, (i / NSTAGE) & 1))) break;
+    done_heads = i + 1;
+
+    const TIn* qs = reinterpret_cast<const TIn*>(st + L::Q);
+    const TIn* ks = reinterpret_cast<const TIn*>(st + L::K);
+    const TIn* vs = reinterpret_cast<const TIn*>(st + L::V);
+    const float* as = reinterpret_cast<const float*>(st + L::A);
+    float* S = reinterpret_cast<float*>(st + L::STATE);
+
+    float4 x[ROWS];
+    float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+    float pkq = 0.f;
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      const int row = row0 + r;
+      const float a = p.gate_log ? expf(as[row]) : as[row], kk = to_f32(ks[row]), qq = to_f32(qs[row]);
+      x[r] = *reinterpret_cast<const float4*>(S + row * DV + col0);
+      x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
+      pa.x = fmaf(kk, x[r].x, pa.x); pa.y = fmaf(kk, x[r].y, pa.y);
+      pa.z = fmaf(kk, x[r].z, pa.z); pa.w = fmaf(kk, x[r].w, pa.w);
+      pb.x = fmaf(qq, x[r].x, pb.x); pb.y = fmaf(qq, x[r].y, pb.y);
+      pb.z = fmaf(qq, x[r].z, pb.z); pb.w = fmaf(qq, x[r].w, pb.w);
+      pkq = fmaf(kk, qq, pkq);
+    }
+    *reinterpret_cast<float4*>(red_a + tk * DV + col0) = pa;
+    *reinterpret_cast<float4*>(red_b + tk * DV + col0) = pb;
+    if (tv == 0) red_kq[tk] = pkq;
+    __syncthreads();
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f), Bq = A;
+    float kq = 0.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const float4 ya = *reinterpret_cast<const float4*>(red_a + g * DV + col0);
+      const float4 yb = *reinterpret_cast<const float4*>(red_b + g * DV + col0);
+      A.x += ya.x; A.y += ya.y; A.z += ya.z; A.w += ya.w;
+      Bq.x += yb.x; Bq.y += yb.y; Bq.z += yb.z; Bq.w += yb.w;
+      kq += red_kq[g];
+    }
+    const float4 vv = load4(vs + col0);
+    const float4 d = make_float4(vv.x - A.x, vv.y - A.y, vv.z - A.z, vv.w - A.w);
+    if (tk == 0) {
+      const float bkq = beta * kq;
+      store4(head_ptrs<TIn>(p, head).o + col0, make_float4(fmaf(bkq, d.x, Bq.x), fmaf(bkq, d.y, Bq.y),
+                                                          fmaf(bkq, d.z, Bq.z), fmaf(bkq, d.w, Bq.w)));
+    }
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      const int row = row0 + r;
+      const float bk = beta * to_f32(ks[row]);
+      x[r].x = fmaf(bk, d.x, x[r].x); x[r].y = fmaf(bk, d.y, x[r].y);
+      x[r].z = fmaf(bk, d.z, x[r].z); x[r].w = fmaf(bk, d.w, x[r].w);
+      *reinterpret_cast<float4*>(S + row * DV + col0) = x[r];
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();  // the updated state is in shared memory; the partial sums are consumed
+    if (tid == 0) {
+      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(head_ptrs<TIn>(p, head).state),
+                   "r"(sb + s * L::BYTES + L::STATE), "r"(DK * DV * 4)
+                   : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      // Refill the stage of head i-1 (its write-back was committed one head ago) with head i-1+NSTAGE.
+      const int j = i - 1 + NSTAGE;
+      if (i >= 1 && j < n_my) {
+        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        const int sj = (i - 1) % NSTAGE;
+        issue_stage<TIn>(p, blockIdx.x + j * gridDim.x, sb + sj * L::BYTES, bar0 + 8 * sj);
+        issued = j + 1;
+      }
+    }
+  }
+  if (tid == 0) {
+    // After an expired wait, give every load still in flight a bounded wait before the CTA's shared
+    // memory goes away; then drain the write-backs.
+    for (int j = done_heads; j < issued; ++j) mbar_wait(bar0 + 8 * (j % NSTAGE), (j / NSTAGE) & 1);
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+}
+
+template <typename TIn>
+cudaError_t launch_bulk(const ScanParams& p, cudaStream_t s) {
+  using L = StageLayout<TIn>;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load(std::memory_order_relaxed) & bit)) {
+    e = cudaFuncSetAttribute(decode_bulk_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int nheads = p.B * p.H;
+  const int grid = nheads < sms ? nheads : sms;
+  if (grid == 0) return cudaSuccess;
+  decode_bulk_kernel<TIn><<<grid, DNT, L::SMEM, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_bulk_supported(const ScanParams& p) {
+  // Whole-state bulk copies need K = V = 128 and the state updated in place.
+  return p.K == DK && p.V == DV && p.s0 == p.sf && p.sf != nullptr;
+}
+
+cudaError_t launch_decode_bulk(const ScanParams& p, kda_dtype dt, cudaStream_t s) {
+  return dt == KDA_F32 ? launch_bulk<float>(p, s) : launch_bulk<__nv_bfloat16>(p, s);
+}
+
+cudaError_t decode_read_timeout(int* flag, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_decode_timeout, sizeof(int));
+  if (e != cudaSuccess || !reset) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_decode_timeout, &zero, sizeof(int));
+}
+
+}  // namespace kda

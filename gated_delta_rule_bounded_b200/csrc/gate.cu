@@ -16,7 +16,11 @@ __device__ __forceinline__ float gate_sigmoid(float x) {
 }
 
 // One warp per (b, t, h) row: the row's coordinates are decomposed once (32-bit
-// arithmetic), A_log is read once, and the lanes stride over its K/4 channel quads.
+// arithmetic), A_log is read once, and the lanes stride over its K/4 channel
+// quads. Each warp takes RPW consecutive rows per step and issues all their
+// loads before any arithmetic, so every lane keeps RPW 16-byte loads in flight.
+constexpr int RPW = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(256) bounded_decay_kernel(GateParams p) {
   const int lane = threadIdx.x & 31;
@@ -25,26 +29,40 @@ __global__ void __launch_bounds__(256) bounded_decay_kernel(GateParams p) {
   const uint32_t rows = (uint32_t)(p.B * p.T * p.H);
   const uint32_t H = (uint32_t)p.H, Tn = (uint32_t)p.T;
   const int quads = (int)(p.K / 4);
-  for (uint32_t r = warp; r < rows; r += nwarps) {
-    const uint32_t h = r % H, bt = r / H;
-    const uint32_t t = bt % Tn, b = bt / Tn;
-    const T* zp = static_cast<const T*>(p.z) + b * p.zs[0] + t * p.zs[1] + h * p.zs[2];
-    T* op = static_cast<T*>(p.out) + b * p.os[0] + t * p.os[1] + h * p.os[2];
-    const float scale = expf(__ldg(p.A_log + h));
+  for (uint32_t r0 = warp * RPW; r0 < rows; r0 += nwarps * RPW) {
     for (int c4 = lane; c4 < quads; c4 += 32) {
-      const float4 z = load4(zp + 4 * c4);
-      float4 g;
-      g.x = p.g_min * gate_sigmoid(scale * z.x);
-      g.y = p.g_min * gate_sigmoid(scale * z.y);
-      g.z = p.g_min * gate_sigmoid(scale * z.z);
-      g.w = p.g_min * gate_sigmoid(scale * z.w);
-      if (!p.out_log) {
-        g.x = expf(g.x);
-        g.y = expf(g.y);
-        g.z = expf(g.z);
-        g.w = expf(g.w);
+      float4 z[RPW];
+      const T* zp[RPW];
+      T* op[RPW];
+      float scale[RPW];
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {
+        const uint32_t r = min(r0 + i, rows - 1);  // clamped rows are recomputed, never out of range
+        const uint32_t h = r % H, bt = r / H;
+        const uint32_t t = bt % Tn, b = bt / Tn;
+        zp[i] = static_cast<const T*>(p.z) + b * p.zs[0] + t * p.zs[1] + h * p.zs[2] + 4 * c4;
+        op[i] = static_cast<T*>(p.out) + b * p.os[0] + t * p.os[1] + h * p.os[2] + 4 * c4;
+        scale[i] = __ldg(p.A_log + h);
       }
-      store4(op + 4 * c4, g);
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) z[i] = load4(zp[i]);
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {
+        if (r0 + i >= rows) break;
+        const float sc = expf(scale[i]);
+        float4 g;
+        g.x = p.g_min * gate_sigmoid(sc * z[i].x);
+        g.y = p.g_min * gate_sigmoid(sc * z[i].y);
+        g.z = p.g_min * gate_sigmoid(sc * z[i].z);
+        g.w = p.g_min * gate_sigmoid(sc * z[i].w);
+        if (!p.out_log) {
+          g.x = expf(g.x);
+          g.y = expf(g.y);
+          g.z = expf(g.z);
+          g.w = expf(g.w);
+        }
+        store4(op[i], g);
+      }
     }
   }
 }
@@ -53,8 +71,8 @@ cudaError_t launch_gate(const GateParams& p, kda_dtype dt, cudaStream_t s) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t rows = p.B * p.T * p.H;  // one warp per row, 8 warps per block
-  const int64_t want = (rows + 7) / 8;
+  const int64_t rows = p.B * p.T * p.H;  // RPW rows per warp step, 8 warps per block
+  const int64_t want = (rows + 8 * RPW - 1) / (8 * RPW);
   const int64_t cap = (int64_t)sms * 8;   // 8 resident 256-thread blocks per SM
   int grid = (int)(want < cap ? want : cap);
   if (grid < 1) grid = 1;

@@ -80,8 +80,11 @@ int kda_device_status(int* timed_out, int reset) {
   if (!timed_out) return fail(KDA_ERR_INVALID_ARG, "kda_device_status: null output");
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "kda_device_status synchronize");
-  e = kda::chunk_read_timeout(timed_out, reset != 0);
+  int chunk_flag = 0, decode_flag = 0;
+  e = kda::chunk_read_timeout(&chunk_flag, reset != 0);
+  if (e == cudaSuccess) e = kda::decode_read_timeout(&decode_flag, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "kda_device_status read");
+  *timed_out = (chunk_flag || decode_flag) ? 1 : 0;
   return ok();
 }
 
@@ -301,7 +304,8 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
   p.V = (int)V;
   p.N = (int)B;
   p.gate_log = gate_kind == KDA_GATE_LOG;
-  cudaError_t e = kda::launch_recurrent(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = kda::decode_bulk_supported(p) ? kda::launch_decode_bulk(p, dtype, s) : kda::launch_recurrent(p, dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
   return ok();
 }

@@ -41,6 +41,10 @@ cudaError_t launch_gate(const GateParams& p, kda_dtype dt, cudaStream_t s);
 // Token-by-token kernel: the decode step (T = 1, s0 == sf) and the generic
 // prefill path (fp32 inputs, any supported K and V).
 cudaError_t launch_recurrent(const ScanParams& p, kda_dtype dt, cudaStream_t s);
+// Decode step for K = V = 128 with whole-state bulk copies (persistent, one CTA per SM).
+bool decode_bulk_supported(const ScanParams& p);
+cudaError_t launch_decode_bulk(const ScanParams& p, kda_dtype dt, cudaStream_t s);
+cudaError_t decode_read_timeout(int* flag, bool reset);
 // Chunked prefill for bf16 inputs (bounded decay), tensor cores.
 bool chunk_supported(int K, int V, kda_dtype dt);
 size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t N);

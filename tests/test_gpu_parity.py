@@ -295,7 +295,16 @@ def test_decode_small_matches_oracle(kda):
     check(got_s, rs, "bf16", "state")
 
 
-@pytest.mark.parametrize("K,V", [(32, 32), (64, 128), (128, 256), (48, 80)])
+def test_decode_more_heads_than_sms(kda):
+    """B*H = 600 heads > SM count: each persistent CTA walks several heads through its ring."""
+    w = W.DecodeWorkload("decode_many", 5, 120, 128, 128, steps=6)
+    got_o, got_s, ro, rs = decode_run(kda, w, 6, (torch.tensor([0, 4]), torch.tensor([0, 59, 119])))
+    check(got_o, ro, "bf16", "o")
+    check(got_s, rs, "bf16", "state")
+    assert not kda.device_status()
+
+
+@pytest.mark.parametrize("K,V", [(32, 32), (64, 128), (128, 128), (128, 256), (48, 80)])
 def test_decode_shapes_fp32(kda, K, V):
     w = W.DecodeWorkload("decode_fp32", 2, 3, K, V, steps=25, dtype="f32")
     got_o, got_s, ro, rs = decode_run(kda, w, 25, (torch.arange(2), torch.arange(3)))
