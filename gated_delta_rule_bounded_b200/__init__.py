@@ -167,13 +167,17 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
             initial_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
             gate_is_log: bool = False, output_final_state: bool = True,
             out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
-            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            workspace: Optional[torch.Tensor] = None,
+            use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Scan whole sequences. Returns ``(o [B,T,H,V], final_state [N,H,K,V] fp32 or None)``.
 
     q, k ``[B,T,H,K]`` and v ``[B,T,H,V]`` share a dtype (bf16 or fp32); gate ``[B,T,H,K]`` fp32
     holds alpha (or g = log alpha when ``gate_is_log``); beta ``[B,T,H]`` fp32. With ``cu_seqlens``
     (int32 ``[N+1]`` on the device) B must be 1 and the states have N rows.
-    ``final_state`` may be ``initial_state`` itself to resume in place.
+    ``final_state`` may be ``initial_state`` itself to resume in place. ``workspace`` (uint8, on the
+    device) enables the two-kernel path when large enough; when it is None and ``use_workspace`` is
+    true, one of ``prefill_workspace_bytes`` bytes is allocated; ``use_workspace=False`` runs the
+    single fused kernel.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta")):
         _cuda(t, n)
@@ -216,7 +220,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
     if out is None:
         out = torch.empty((B, T, H, V), device=dev, dtype=q.dtype)
     ws_need = prefill_workspace_bytes(B, T, H, K, V, n_seq, q.dtype)
-    if workspace is None and ws_need > 0:
+    if workspace is None and ws_need > 0 and use_workspace:
         workspace = torch.empty(ws_need, device=dev, dtype=torch.uint8)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0

@@ -1,0 +1,486 @@
+// chunk_common.cuh -- pieces shared by the chunked prefill kernels: PTX helpers for
+// tcgen05/TMEM, ldmatrix/mma.sync and cp.async, the per-chunk decay pass, the 16x16
+// A_qk / A_kk block pairs and the 64x64 triangular inverse. The math they implement is
+// the chunkwise form of the "KDA cheat sheet" (eqs. 3-4) with the UT transform derived
+// from eq. 1 of "Kimi K3: Bounded Decay and Delta Memory"; see chunk.cu for the notation.
+#pragma once
+
+#include "common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+namespace {
+
+constexpr int C = 64;     // tokens per chunk
+constexpr int KD = 128;   // key dim
+constexpr int VT = 128;   // value columns per state tile
+constexpr int NTHREADS = 256;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float G2_MIN = -5.5f * LOG2E;  // lower clamp of the per-token log2-decay
+constexpr uint32_t WAIT_LIMIT = 1u << 22;
+
+// fp32 vector area written by the decay pass (offsets in floats).
+constexpr int VEC_D = 0;          // [10][128] bf16 exp(G_{s_a} - G_{r_b}), pairs a >= b (640 floats)
+constexpr int VEC_GAM = 640;      // [128]     gamma_C
+constexpr int VEC_TOT = 768;      // [4][128]  per-block log2-decay sums
+constexpr int VEC_FLOATS = 1280;
+
+// Shared-memory offsets (bytes) of the tiles the state-independent phases use. Every bf16
+// tile has 128-byte rows with the 128-byte swizzle; 128-column tiles are two 8 KB atoms.
+struct IntraLayout {
+  int qe, ke, kc;   // row operands of A_qk / A_kk and the column operand, [t][c]
+  int qg, kg, kt;   // Q*Gamma, K*Gamma, K*gamma_C/Gamma, [t][c]
+  int akk;          // A_kk, fp32 [64][64]
+  int aqk;          // A_qk, bf16 [t][i] (K-major operand)
+  int tp, tb;       // T' = T Diag(beta) (K-major operand) and a bf16 copy of T, [t][i]
+  int vec;          // fp32 vectors (VEC_*)
+};
+
+// ---------------------------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Byte offset of element (r, c) in a tile of 128-byte rows (64 bf16 per atom); atom_bytes is the
+// distance between the two 64-column atoms of a 128-column tile.
+__device__ __forceinline__ uint32_t sw_e(int r, int c, int atom_bytes) {
+  return (c >> 6) * atom_bytes + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+// Byte offset of the 16-byte chunk holding columns 8j..8j+7 of row r.
+__device__ __forceinline__ uint32_t sw_chunk(int r, int j, int atom_bytes) {
+  return (j >> 3) * atom_bytes + r * 128 + (((j & 7) ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+}
+// Elementwise bf16x2 product (one rounding of the exact product).
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;  // n == 0 zero-fills the destination
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 4 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: 128-byte swizzle, start address, leading and stride byte offsets.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile("{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+               "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tm_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Waits for phase `parity` of the mbarrier with an iteration limit. Returns false (and records
+// the timeout) when the limit expires.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* timeout_flag) {
+  for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    if (done) return true;
+  }
+  atomicExch(timeout_flag, 1);
+  return false;
+}
+
+__device__ __forceinline__ uint4 pack8(const uint32_t (&r)[32], int j, float sign) {
+  uint4 w;
+  w.x = pack_bf16(sign * __uint_as_float(r[8 * j + 0]), sign * __uint_as_float(r[8 * j + 1]));
+  w.y = pack_bf16(sign * __uint_as_float(r[8 * j + 2]), sign * __uint_as_float(r[8 * j + 3]));
+  w.z = pack_bf16(sign * __uint_as_float(r[8 * j + 4]), sign * __uint_as_float(r[8 * j + 5]));
+  w.w = pack_bf16(sign * __uint_as_float(r[8 * j + 6]), sign * __uint_as_float(r[8 * j + 7]));
+  return w;
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// Inputs
+// ---------------------------------------------------------------------------------------------
+
+struct ChunkCtx {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* gate;
+  const float* beta;
+  int64_t qrow, krow, vrow, grow, boff;  // element offsets of token 0 of this (sequence, head)
+  int64_t qst, kst, vst, gst, bst;       // element strides between tokens
+};
+
+// Registers holding one thread's share of a chunk's q, k, g: channels c0, c0+1 of the 16 tokens
+// of block a (thread = (channel pair, block)).
+struct Prefetch {
+  float2 g[16];
+  uint32_t q[16], k[16];
+};
+
+__device__ __forceinline__ void load_qkg(const ChunkCtx& x, int64_t tc0, int nv, int c0, int a, Prefetch& pf) {
+  const int64_t t = tc0 + 16 * a;
+  const float* gp = x.gate + x.grow + t * x.gst + c0;
+  const __nv_bfloat16* qp = x.q + x.qrow + t * x.qst + c0;
+  const __nv_bfloat16* kp = x.k + x.krow + t * x.kst + c0;
+  const int imax = nv - 16 * a;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i < imax) {
+      pf.g[i] = *reinterpret_cast<const float2*>(gp);
+      pf.q[i] = *reinterpret_cast<const uint32_t*>(qp);
+      pf.k[i] = *reinterpret_cast<const uint32_t*>(kp);
+    } else {
+      pf.g[i] = make_float2(0.f, 0.f);
+      pf.q[i] = pf.k[i] = 0u;
+    }
+    gp += x.gst;
+    qp += x.qst;
+    kp += x.kst;
+  }
+}
+
+// v tile of a chunk into the MN-major operand layout ([i][v], two 64-column halves).
+__device__ __forceinline__ void load_v(const ChunkCtx& x, uint32_t vbase, int64_t tc0, int nv, int tid) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = tid + NTHREADS * i;
+    const int row = idx >> 4, piece = idx & 15;
+    const bool ok = row < nv;
+    const int64_t t = tc0 + (ok ? row : 0);
+    cp_async16(vbase + (piece >> 3) * 8192 + row * 128 + (((piece & 7) ^ (row & 7)) << 4),
+               x.v + x.vrow + t * x.vst + piece * 8, ok);
+  }
+}
+
+// v tile and beta of a chunk.
+__device__ __forceinline__ void load_vb(const ChunkCtx& x, uint32_t vbase, uint32_t bbase, int64_t tc0, int nv,
+                                        int tid) {
+  load_v(x, vbase, tc0, nv, tid);
+  if (tid < C) {
+    const bool ok = tid < nv;
+    const int64_t t = tc0 + (ok ? tid : 0);
+    cp_async4(bbase + tid * 4, x.beta + x.boff + t * x.bst, ok);
+  }
+}
+
+// 16x16 block pairs (a, b), a >= b, of A_qk (rows from Qe) or A_kk (rows from Ke) against the Kc
+// columns, with the per-pair decay factor D_ab applied to the row operand. The warp takes tiles
+// first, first + stride, ... (nt of them) and runs their k-loops interleaved so the MMA chains
+// overlap. A_qk is stored as a bf16 K-major operand (diagonal blocks masked to i <= t); A_kk as
+// fp32 [64][64] with beta_t applied and diagonal blocks masked to i < t.
+template <int NTMAX>
+__device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const IntraLayout& L, int off_rows, int first,
+                                        int stride, int nt, int lane, int g, int tq, const float* beta_s,
+                                        bool is_qk) {
+  const float* vec = reinterpret_cast<const float*>(sm + L.vec);
+  int ta[NTMAX], tbk[NTMAX], tid_[NTMAX];
+#pragma unroll
+  for (int n = 0; n < NTMAX; ++n) {
+    const int tile = first + stride * n;
+    tid_[n] = tile;
+    ta[n] = tile >= 6 ? 3 : (tile >= 3 ? 2 : (tile >= 1 ? 1 : 0));
+    tbk[n] = tile - ta[n] * (ta[n] + 1) / 2;
+  }
+  const __nv_bfloat16* D16 = reinterpret_cast<const __nv_bfloat16*>(vec + VEC_D);
+  float acc[NTMAX][2][4];
+#pragma unroll
+  for (int n = 0; n < NTMAX; ++n)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[n][j][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+    for (int n = 0; n < NTMAX; ++n) {
+      if (n < nt) {
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+        const int ra = 16 * ta[n] + (lane & 7) + ((lane >> 3) & 1) * 8;
+        ldsm_x4(sb + off_rows + sw_chunk(ra, 2 * kk + (lane >> 4), 8192), a0, a1, a2, a3);
+        const __nv_bfloat16* Dv = D16 + tid_[n] * 128 + 16 * kk + 2 * tq;
+        const uint32_t d01 = *reinterpret_cast<const uint32_t*>(Dv);
+        const uint32_t d89 = *reinterpret_cast<const uint32_t*>(Dv + 8);
+        a0 = hmul2(a0, d01);
+        a1 = hmul2(a1, d01);
+        a2 = hmul2(a2, d89);
+        a3 = hmul2(a3, d89);
+        const int rb = 16 * tbk[n] + (lane & 7) + (lane >> 4) * 8;
+        ldsm_x4(sb + L.kc + sw_chunk(rb, 2 * kk + ((lane >> 3) & 1), 8192), b0, b1, b2, b3);
+        mma_bf16(acc[n][0], a0, a1, a2, a3, b0, b1);
+        mma_bf16(acc[n][1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NTMAX; ++n) {
+    if (n >= nt) continue;
+    const int a = ta[n], b = tbk[n];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int t = 16 * a + g + 8 * hr;
+        const int i0 = 16 * b + 8 * j + 2 * tq;
+        float v0 = acc[n][j][2 * hr], v1 = acc[n][j][2 * hr + 1];
+        if (is_qk) {
+          if (a == b) {
+            v0 = (i0 <= t) ? v0 : 0.f;
+            v1 = (i0 + 1 <= t) ? v1 : 0.f;
+          }
+          *reinterpret_cast<uint32_t*>(sm + L.aqk + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
+        } else {
+          const float bt = beta_s[t];
+          v0 = (a > b || i0 < t) ? v0 * bt : 0.f;
+          v1 = (a > b || i0 + 1 < t) ? v1 * bt : 0.f;
+          *reinterpret_cast<float2*>(sm + L.akk + (t * 64 + i0) * 4) = make_float2(v0, v1);
+        }
+      }
+  }
+}
+
+
+// Decay pass, step 1: the per-token log2-decay of channels (c0, c0+1) over the 16 tokens of block
+// da (clamped at G2_MIN; 0 past the end of the sequence), their retention factors, and the block
+// sum, published to VEC_TOT.
+__device__ __forceinline__ void decay_step1(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int nv,
+                                            int da, int c0, bool gate_log, float2 (&al)[16]) {
+  float* vec = reinterpret_cast<float*>(sm + L.vec);
+  float2 run = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float2 l = make_float2(0.f, 0.f);
+    if (16 * da + i < nv) {
+      l.x = fmaxf(gate_log ? pf.g[i].x * LOG2E : lg2(pf.g[i].x), G2_MIN);
+      l.y = fmaxf(gate_log ? pf.g[i].y * LOG2E : lg2(pf.g[i].y), G2_MIN);
+    }
+    run.x += l.x;
+    run.y += l.y;
+    al[i] = make_float2(ex2(l.x), ex2(l.y));
+  }
+  *reinterpret_cast<float2*>(vec + VEC_TOT + da * 128 + c0) = run;
+}
+
+// Decay pass, step 2 (after a barrier): block-boundary decay vectors and the six scaled tiles
+// Qe = q E, Ke = k E, Kc = k F, QG = q E GS, KG = k E GS, Kt = k F PM of this thread's elements,
+// with E_t = exp(G_t - G_{s_a}), F_t = exp(G_{r_a} - G_t), GS = exp(G_{s_a}), PM = exp(G_C - G_{r_a}).
+__device__ __forceinline__ void decay_step2(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int da,
+                                            int c0, const float2 (&al)[16]) {
+  float* vec = reinterpret_cast<float*>(sm + L.vec);
+  float2 e[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) e[b] = *reinterpret_cast<const float2*>(vec + VEC_TOT + b * 128 + c0);
+#pragma unroll
+  for (int b = 1; b < 4; ++b) {
+    e[b].x += e[b - 1].x;
+    e[b].y += e[b - 1].y;
+  }
+  // e[b] = log2 Gamma at r_b; log2 Gamma at s_a is e[a-1] (0 for a = 0)
+  const float2 gs = da == 0 ? make_float2(0.f, 0.f) : (da == 1 ? e[0] : (da == 2 ? e[1] : e[2]));
+  const float2 eda = da == 0 ? e[0] : (da == 1 ? e[1] : (da == 2 ? e[2] : e[3]));
+  __nv_bfloat16* D16 = reinterpret_cast<__nv_bfloat16*>(vec + VEC_D);
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    if (b <= da) {
+      const int pair = da * (da + 1) / 2 + b;
+      *reinterpret_cast<uint32_t*>(D16 + pair * 128 + c0) = pack_bf16(ex2(gs.x - e[b].x), ex2(gs.y - e[b].y));
+    }
+  }
+  if (da == 0) *reinterpret_cast<float2*>(vec + VEC_GAM + c0) = make_float2(ex2(e[3].x), ex2(e[3].y));
+  const float2 GS = make_float2(ex2(gs.x), ex2(gs.y));
+  const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));
+  float2 F[16];
+  F[15] = make_float2(1.f, 1.f);
+#pragma unroll
+  for (int i = 14; i >= 0; --i) F[i] = make_float2(F[i + 1].x * al[i + 1].x, F[i + 1].y * al[i + 1].y);
+  float2 E = make_float2(1.f, 1.f);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = 16 * da + i;
+    E.x *= al[i].x;
+    E.y *= al[i].y;
+    const float2 qf = unpack_bf16(pf.q[i]), kf = unpack_bf16(pf.k[i]);
+    const uint32_t off = sw_e(t, c0, 8192);
+    const float qex = qf.x * E.x, qey = qf.y * E.y, kex = kf.x * E.x, key = kf.y * E.y;
+    const float kfx = kf.x * F[i].x, kfy = kf.y * F[i].y;
+    *reinterpret_cast<uint32_t*>(sm + L.qe + off) = pack_bf16(qex, qey);
+    *reinterpret_cast<uint32_t*>(sm + L.ke + off) = pack_bf16(kex, key);
+    *reinterpret_cast<uint32_t*>(sm + L.kc + off) = pack_bf16(kfx, kfy);
+    *reinterpret_cast<uint32_t*>(sm + L.qg + off) = pack_bf16(qex * GS.x, qey * GS.y);
+    *reinterpret_cast<uint32_t*>(sm + L.kg + off) = pack_bf16(kex * GS.x, key * GS.y);
+    *reinterpret_cast<uint32_t*>(sm + L.kt + off) = pack_bf16(kfx * PM.x, kfy * PM.y);
+  }
+}
+
+// Zeroes the six 16x16 blocks above the diagonal of a [64][64] bf16 K-major tile, using the
+// `count` threads with index `idx` in [0, count).
+__device__ __forceinline__ void zero_upper_blocks(unsigned char* sm, int off, int idx, int count) {
+  for (int e = idx; e < 6 * 64; e += count) {
+    const int pr = e >> 6, r = (e >> 2) & 15, q4 = e & 3;  // block pair, row, group of 4 columns
+    const int a = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
+    const int b = pr < 3 ? pr + 1 : (pr < 5 ? pr - 1 : 3);
+    *reinterpret_cast<uint2*>(sm + off + sw_e(16 * a + r, 16 * b + 4 * q4, 8192)) = make_uint2(0u, 0u);
+  }
+}
+
+// T' = (I + A_kk)^-1 Diag(beta), run by warps 0-3 (128 threads, named barrier 1): the four 16x16
+// diagonal inverses by forward substitution in fp32, then the blocks below the diagonal by distance
+// d = 1, 2, 3 as tensor-core products T_ab = -sum_{j=b}^{a-1} (T_aa L_aj) T_jb, reading the bf16
+// copy of T and writing T' from the fp32 values.
+__device__ __forceinline__ void inverse_warps0to3(unsigned char* sm, uint32_t sb, const IntraLayout& Ly,
+                                                  const float* beta_s, int tid, int warp, int lane, int g, int tq) {
+  const float* L = reinterpret_cast<const float*>(sm + Ly.akk);
+  const uint32_t tb = sb + Ly.tb;
+  if (tid < 64) {
+    const int a = tid >> 4, j = tid & 15;
+    float xs[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xs[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int l = 0; l < 16; ++l)
+#pragma unroll
+      for (int i = l + 1; i < 16; ++i) xs[i] -= L[(16 * a + i) * 64 + 16 * a + l] * xs[l];
+    const float bj = beta_s[16 * a + j];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t off = sw_e(16 * a + i, 16 * a + j, 8192);
+      *reinterpret_cast<__nv_bfloat16*>(sm + Ly.tb + off) = __float2bfloat16_rn(xs[i]);
+      *reinterpret_cast<__nv_bfloat16*>(sm + Ly.tp + off) = __float2bfloat16_rn(xs[i] * bj);
+    }
+  } else {
+    zero_upper_blocks(sm, Ly.tp, tid - 64, 64);  // T' is lower triangular
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll 1
+  for (int d = 1; d <= 3; ++d) {
+    if (warp < 4 - d) {
+      const int b = warp, a = b + d;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      uint32_t t0, t1, t2, t3;  // A fragments of T_aa
+      ldsm_x4(tb + sw_chunk(16 * a + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * a + (lane >> 4), 8192), t0, t1, t2, t3);
+      for (int jb = b; jb < a; ++jb) {
+        float P[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {  // P = T_aa L_{a,jb}; B[k][n] = L[16a + k][16jb + n]
+          const float* lp = L + (16 * a + 2 * tq) * 64 + 16 * jb + 8 * j + g;
+          mma_bf16(P[j], t0, t1, t2, t3, pack_bf16(lp[0], lp[64]), pack_bf16(lp[8 * 64], lp[9 * 64]));
+        }
+        uint32_t b0, b1, b2, b3;  // B = T_{jb,b}
+        ldsm_x4_t(tb + sw_chunk(16 * jb + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * b + (lane >> 4), 8192), b0, b1, b2, b3);
+        const uint32_t p0 = pack_bf16(P[0][0], P[0][1]), p1 = pack_bf16(P[0][2], P[0][3]);
+        const uint32_t p2 = pack_bf16(P[1][0], P[1][1]), p3 = pack_bf16(P[1][2], P[1][3]);
+        mma_bf16(acc[0], p0, p1, p2, p3, b0, b1);
+        mma_bf16(acc[1], p0, p1, p2, p3, b2, b3);
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int row = 16 * a + g + 8 * hr, col = 16 * b + 8 * j + 2 * tq;
+          const float v0 = -acc[j][2 * hr], v1 = -acc[j][2 * hr + 1];
+          const uint32_t off = sw_e(row, col, 8192);
+          *reinterpret_cast<uint32_t*>(sm + Ly.tb + off) = pack_bf16(v0, v1);
+          *reinterpret_cast<uint32_t*>(sm + Ly.tp + off) = pack_bf16(v0 * beta_s[col], v1 * beta_s[col + 1]);
+        }
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
+}
+
+// The state-independent phases after the decay pass: A_kk on all warps; then the inverse on warps
+// 0-3 while warps 4-7 form A_qk (and zero its upper blocks). Ends with a CTA-wide barrier.
+__device__ __forceinline__ void intra_phases(unsigned char* sm, uint32_t sb, const IntraLayout& L, const float* beta_s,
+                                             int tid, int warp, int lane, int g, int tq) {
+  a_tiles<2>(sm, sb, L, L.ke, warp, 8, warp < 2 ? 2 : 1, lane, g, tq, beta_s, /*is_qk=*/false);
+  __syncthreads();  // A_kk ready; Ke is dead
+  if (warp < 4) {
+    inverse_warps0to3(sm, sb, L, beta_s, tid, warp, lane, g, tq);
+  } else {
+    a_tiles<3>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
+    zero_upper_blocks(sm, L.aqk, tid - 128, 128);  // the MMAs read whole rows of A_qk
+  }
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace kda

@@ -1,0 +1,476 @@
+// chunk_split.cu -- chunked prefill in two kernels: the state-independent work of every chunk in
+// parallel (kernel P), then the state recurrence (kernel S).
+//
+// The per-chunk quantities of the chunkwise form that do not depend on the carried state --
+// the decay factors, A_qk and A_kk, T' = (I + A_kk)^-1 Diag(beta), W = T' (K*Gamma), Q*Gamma and
+// K*gamma_C/Gamma -- are most of the arithmetic. In the fused kernel (chunk.cu) they sit on the
+// sequential path of one CTA per (sequence, head). Here kernel P computes them for all chunks of all
+// heads at once, one CTA per (chunk, head) over every SM, and writes each chunk's operand set as
+// one 66,048-byte block to a workspace: the block is the exact image of the shared-memory tiles
+// (128-byte swizzle included), so kernel S moves it with a single bulk copy into a 1 KB-aligned
+// buffer and feeds it straight to tcgen05. Kernel S keeps one CTA per (sequence, head, V-tile) with
+// the transposed state S^T in TMEM and runs two MMA groups per chunk:
+//   group A:  O^T = S^T (Q*Gamma)^T,   U^T = V^T T'^T + S^T (-W)^T
+//   group B:  O^T += U^T A_qk^T,       S^T += U^T (K*gamma_C/Gamma)      (S^T pre-scaled by gamma_C)
+// The price is the workspace traffic (one write and one read of ~1 KB per token-head).
+//
+// Workspace slots. Chunk j of sequence n has slot n * ceil(T/64) + j without cu_seqlens, and
+// floor(cu[n]/64) + n + j with them (unique: a sequence's slots end before the next one's begin).
+#include <atomic>
+
+#include "chunk_common.cuh"
+
+namespace kda {
+
+// Set to 1 by any CTA of the split kernels whose bounded wait expired.
+__device__ int g_split_timeout = 0;
+
+namespace {
+
+// One workspace block = the output region of kernel P = the operand buffer of kernel S.
+constexpr int WB_W = 0;          // 16K  -W [c][t], 128 rows (MN-major B of S^T (-W)^T)
+constexpr int WB_QG = 16384;     // 16K  Q*Gamma [t][c], two atoms (K-major B)
+constexpr int WB_KT = 32768;     // 16K  K*gamma_C/Gamma [t][c], two halves (MN-major B)
+constexpr int WB_TP = 49152;     // 8K   T' [t][i] (K-major B)
+constexpr int WB_AQK = 57344;    // 8K   A_qk [t][i] (K-major B)
+constexpr int WB_GAM = 65536;    // 512  gamma_C, fp32 [128]
+constexpr int WB_BYTES = 66048;
+
+// Kernel P shared memory.
+constexpr int P_OUT = 0;                    // the workspace block image
+constexpr int P_QE = 66560;                 // 16K Qe [t][c]
+constexpr int P_KE = P_QE + 16384;          // 16K Ke [t][c]; after A_kk, the bf16 copy of T
+constexpr int P_KC = P_KE + 16384;          // 16K Kc [t][c]
+constexpr int P_KG = P_KC + 16384;          // 16K K*Gamma [i][c]
+constexpr int P_AKK = P_KG + 16384;         // 16K A_kk fp32
+constexpr int P_BETA = P_AKK + 16384;       // 256 beta
+constexpr int P_VEC = P_BETA + 256;         // vectors
+constexpr int P_SMEM = P_VEC + VEC_FLOATS * 4;
+static_assert(P_SMEM <= 227 * 1024, "shared memory budget");
+
+// Kernel S shared memory.
+constexpr int S_OPS = 0;                    // 2 x operand block (66048 B, padded to 66560)
+constexpr int S_OPS_STRIDE = 66560;
+constexpr int S_V = 2 * S_OPS_STRIDE;       // 2 x 16K v tile [i][v], two halves (MN-major A)
+constexpr int S_SBF = S_V + 2 * 16384;      // 32K S bf16 [v][c], two atoms of [128][64] (K-major A)
+constexpr int S_U = S_SBF + 32768;          // 16K U bf16 [v][i] (K-major A)
+constexpr int S_BAR = S_U + 16384;          // mbarriers: ops0, ops1, mma; TMEM base
+constexpr int S_SMEM = S_BAR + 64;
+static_assert(S_SMEM <= 227 * 1024, "shared memory budget");
+static_assert(S_SBF % 1024 == 0 && S_U % 1024 == 0 && S_V % 1024 == 0, "swizzle atoms need 1 KB alignment");
+
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 192, TM_COLS = 256;
+
+__device__ __forceinline__ void seq_range(const ScanParams& p, int n, int64_t& t0, int64_t& t1, int64_t& brow) {
+  t0 = 0;
+  t1 = p.T;
+  brow = n;
+  if (p.cu) {
+    t1 = min((int64_t)p.cu[n + 1], p.T);
+    t0 = max((int64_t)0, min((int64_t)p.cu[n], t1));
+    brow = 0;
+  }
+}
+
+__device__ __forceinline__ int64_t slot_base(const ScanParams& p, int n, int64_t t0) {
+  return p.cu ? (t0 >> 6) + n : (int64_t)n * ((p.T + C - 1) / C);
+}
+
+// Kernel P: slot s -> (sequence, chunk). Without cu_seqlens the slots are dense; with them, the
+// sequence is the last one whose base slot is <= s (base slots increase with n).
+__device__ __forceinline__ bool locate_slot(const ScanParams& p, int64_t s, int& n_out, int& j_out) {
+  if (!p.cu) {
+    const int64_t ncps = (p.T + C - 1) / C;
+    n_out = (int)(s / ncps);
+    j_out = (int)(s % ncps);
+    return n_out < p.N && (int64_t)j_out * C < p.T;
+  }
+  int lo = 0, hi = p.N - 1, n = -1;
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    int64_t t0, t1, br;
+    seq_range(p, mid, t0, t1, br);
+    if (slot_base(p, mid, t0) <= s) {
+      n = mid;
+      lo = mid + 1;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  if (n < 0) return false;
+  int64_t t0, t1, br;
+  seq_range(p, n, t0, t1, br);
+  const int64_t j = s - slot_base(p, n, t0);
+  if (j * C >= t1 - t0) return false;
+  n_out = n;
+  j_out = (int)j;
+  return true;
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) chunk_intra_kernel(ScanParams p, unsigned char* ws) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const uint32_t sb = smem_u32(sm);
+  constexpr IntraLayout LY{P_QE, P_KE, P_KC, P_OUT + WB_QG, P_KG, P_OUT + WB_KT, P_AKK, P_OUT + WB_AQK,
+                           P_OUT + WB_TP, P_KE, P_VEC};
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+  const int h = blockIdx.y;
+  const int64_t slot = blockIdx.x;
+  int n, j;
+  if (!locate_slot(p, slot, n, j)) return;  // uniform across the CTA
+  int64_t t0, t1, brow;
+  seq_range(p, n, t0, t1, brow);
+  const int64_t tc0 = t0 + (int64_t)j * C;
+  const int nv = (int)min((int64_t)C, t1 - tc0);
+
+  ChunkCtx x;
+  x.q = static_cast<const __nv_bfloat16*>(p.q);
+  x.k = static_cast<const __nv_bfloat16*>(p.k);
+  x.v = nullptr;
+  x.gate = p.gate;
+  x.beta = p.beta;
+  x.qrow = brow * p.qs[0] + h * p.qs[2];
+  x.krow = brow * p.ks[0] + h * p.ks[2];
+  x.vrow = 0;
+  x.grow = brow * p.gs[0] + h * p.gs[2];
+  x.boff = brow * p.bs[0] + h * p.bs[2];
+  x.qst = p.qs[1];
+  x.kst = p.ks[1];
+  x.vst = 0;
+  x.gst = p.gs[1];
+  x.bst = p.bs[1];
+
+  const int c0 = 2 * (tid & 63), da = tid >> 6;
+  Prefetch pf;
+  load_qkg(x, tc0, nv, c0, da, pf);
+  float* beta_s = reinterpret_cast<float*>(sm + P_BETA);
+  if (tid < C) beta_s[tid] = tid < nv ? __ldg(x.beta + x.boff + (tc0 + tid) * x.bst) : 0.f;
+
+  {
+    float2 al[16];
+    decay_step1(sm, LY, pf, nv, da, c0, p.gate_log != 0, al);
+    __syncthreads();
+    decay_step2(sm, LY, pf, da, c0, al);
+  }
+  __syncthreads();
+  intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+
+  // W = T' (K*Gamma) on mma.sync; warp (m, nh) owns rows 16m.. and columns 64nh.. . -W is stored
+  // as the MN-major operand of S^T (-W)^T: row c holds W[0..63][c].
+  {
+    const int m = warp & 3, nh = warp >> 2;
+    float acc[8][4];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[jj][e] = 0.f;
+    for (int kk = 0; kk <= m; ++kk) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(sb + P_OUT + WB_TP + sw_chunk(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4), 8192),
+              a0, a1, a2, a3);
+      const int rr = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sb + P_KG + sw_chunk(rr, 8 * nh + 2 * pp + (lane >> 4), 8192), b0, b1, b2, b3);
+        mma_bf16(acc[2 * pp], a0, a1, a2, a3, b0, b1);
+        mma_bf16(acc[2 * pp + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int t = 16 * m + g + 8 * hr, c = 64 * nh + 8 * jj + 2 * tq;
+        *reinterpret_cast<__nv_bfloat16*>(sm + P_OUT + WB_W + sw_e(c, t, 0)) = __float2bfloat16_rn(-acc[jj][2 * hr]);
+        *reinterpret_cast<__nv_bfloat16*>(sm + P_OUT + WB_W + sw_e(c + 1, t, 0)) =
+            __float2bfloat16_rn(-acc[jj][2 * hr + 1]);
+      }
+    if (tid < 32)
+      *reinterpret_cast<float4*>(sm + P_OUT + WB_GAM + 16 * tid) =
+          *reinterpret_cast<const float4*>(sm + P_VEC + 4 * (VEC_GAM + 4 * tid));
+  }
+  fence_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    unsigned char* dst = ws + ((size_t)slot * p.H + h) * WB_BYTES;
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(sb + P_OUT),
+                 "r"(WB_BYTES)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, const unsigned char* ws) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int quad = warp & 3, half = warp >> 2;
+  const int trow = 32 * quad + lane;
+
+  const int n_vt = p.V / VT;
+  int blk = blockIdx.x;
+  const int vt = blk % n_vt;
+  blk /= n_vt;
+  const int h = blk % p.H;
+  const int n = blk / p.H;
+  int64_t t0, t1, brow;
+  seq_range(p, n, t0, t1, brow);
+  const int n_chunks = (int)((t1 - t0 + C - 1) / C);
+  const int64_t sbase_slot = slot_base(p, n, t0);
+
+  ChunkCtx x;
+  x.v = static_cast<const __nv_bfloat16*>(p.v);
+  x.beta = p.beta;
+  x.vrow = brow * p.vs[0] + h * p.vs[2] + (int64_t)vt * VT;
+  x.vst = p.vs[1];
+  x.boff = 0;
+  x.bst = 0;
+
+  const uint32_t bar_ops = sb + S_BAR, bar_mma = sb + S_BAR + 16;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + S_BAR + 24);
+  auto block_src = [&](int c) { return ws + ((size_t)(sbase_slot + c) * p.H + h) * WB_BYTES; };
+
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ops));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ops + 8));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(TM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tlane = tmem + ((uint32_t)(32 * quad) << 16);
+
+  if (n_chunks > 0) {
+    if (tid == 0) {
+      bulk_load(sb + S_OPS, block_src(0), WB_BYTES, bar_ops);
+      if (n_chunks > 1) bulk_load(sb + S_OPS + S_OPS_STRIDE, block_src(1), WB_BYTES, bar_ops + 8);
+    }
+    load_v(x, sb + S_V, t0, (int)min((int64_t)C, t1 - t0), tid);
+    cp_async_commit();
+  }
+
+  // Initial state: TMEM lane v holds column v of S; this thread moves columns [64*half, +64).
+  const size_t sbase = ((size_t)n * p.H + h) * (size_t)KD * p.V + (size_t)vt * VT;
+#pragma unroll
+  for (int part = 0; part < 2; ++part) {
+    const int cb = 64 * half + 32 * part;
+    uint32_t r[32];
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj)
+      r[jj] = __float_as_uint(p.s0 ? p.s0[sbase + (size_t)(cb + jj) * p.V + trow] : 0.f);
+    tm_st32(tlane + TM_S + cb, r);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      *reinterpret_cast<uint4*>(sm + S_SBF + sw_chunk(trow, (cb >> 3) + jj, 16384)) = pack8(r, jj, 1.f);
+  }
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+
+  uint32_t mma_phase = 0;
+  bool ok = true;
+  for (int c = 0; c < n_chunks && ok; ++c) {
+    const int64_t tc0 = t0 + (int64_t)c * C;
+    const int nv = (int)min((int64_t)C, t1 - tc0);
+    const int buf = c & 1;
+    const uint32_t ops = sb + S_OPS + buf * S_OPS_STRIDE;
+    const unsigned char* opsp = sm + S_OPS + buf * S_OPS_STRIDE;
+    const uint32_t vbuf = sb + S_V + buf * 16384;
+
+    cp_async_wait_all();
+    fence_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(mbar_wait(bar_ops + 8 * buf, (c >> 1) & 1, &g_split_timeout));
+    tc_fence_after();
+    if (!ok) break;
+    if (c + 1 < n_chunks)
+      load_v(x, sb + S_V + (buf ^ 1) * 16384, tc0 + C, (int)min((int64_t)C, t1 - tc0 - C), tid);
+    cp_async_commit();
+
+    // ---- group A: O^T = S^T (Q*Gamma)^T; U^T = V^T T'^T + S^T (-W)^T --------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id_kk = idesc_bf16(64, 0, 0), id_mk = idesc_bf16(64, 1, 0), id_km = idesc_bf16(64, 0, 1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t as = sdesc(sb + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+        tc_mma(tmem + TM_O, as, sdesc(ops + WB_QG + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_kk, ks > 0);
+      }
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        tc_mma(tmem + TM_U, sdesc(vbuf + ks * 2048, 8192, 1024), sdesc(ops + WB_TP + ks * 32, 16, 1024), id_mk, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        tc_mma(tmem + TM_U, sdesc(sb + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+               sdesc(ops + WB_W + ks * 2048, 8192, 1024), id_km, 1);
+      tc_commit(bar_mma);
+    }
+    // meanwhile: S^T *= gamma_C in TMEM (group A reads the bf16 copy of S)
+    {
+      const float* gam = reinterpret_cast<const float*>(opsp + WB_GAM);
+      uint32_t r[32];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int cb = 64 * half + 32 * part;
+        tm_ld32(tlane + TM_S + cb, r);
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float4 gm = *reinterpret_cast<const float4*>(gam + cb + 4 * jj);
+          r[4 * jj + 0] = __float_as_uint(__uint_as_float(r[4 * jj + 0]) * gm.x);
+          r[4 * jj + 1] = __float_as_uint(__uint_as_float(r[4 * jj + 1]) * gm.y);
+          r[4 * jj + 2] = __float_as_uint(__uint_as_float(r[4 * jj + 2]) * gm.z);
+          r[4 * jj + 3] = __float_as_uint(__uint_as_float(r[4 * jj + 3]) * gm.w);
+        }
+        tm_st32(tlane + TM_S + cb, r);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase, &g_split_timeout));
+    mma_phase ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+
+    // ---- U to shared memory (K-major A, row v holds U[0..63][v]) -----------------------------------
+    {
+      uint32_t r[32];
+      tm_ld32(tlane + TM_U + 32 * half, r);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        *reinterpret_cast<uint4*>(sm + S_U + sw_chunk(trow, 4 * half + jj, 0)) = pack8(r, jj, 1.f);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- group B: O^T += U^T A_qk^T; S^T += U^T (K*gamma_C/Gamma) -----------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id_o = idesc_bf16(64, 0, 0), id_s = idesc_bf16(128, 0, 1);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t au = sdesc(sb + S_U + ks * 32, 16, 1024);
+        tc_mma(tmem + TM_O, au, sdesc(ops + WB_AQK + ks * 32, 16, 1024), id_o, 1);
+        tc_mma(tmem + TM_S, au, sdesc(ops + WB_KT + ks * 2048, 8192, 1024), id_s, 1);
+      }
+      tc_commit(bar_mma);
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase, &g_split_timeout));
+    mma_phase ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+
+    // ---- O to global memory, S to its bf16 copy ----------------------------------------------------
+    {
+      uint32_t r[32];
+      tm_ld32(tlane + TM_O + 32 * half, r);
+      const int64_t ost = p.os[1];
+      __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + brow * p.os[0] + h * p.os[2] + (int64_t)vt * VT +
+                          trow + (tc0 + 32 * half) * ost;
+      const int jmax = min(32, nv - 32 * half);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        if (jj < jmax) *op = __float2bfloat16_rn(__uint_as_float(r[jj]));
+        op += ost;
+      }
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int cb = 64 * half + 32 * part;
+        tm_ld32(tlane + TM_S + cb, r);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          *reinterpret_cast<uint4*>(sm + S_SBF + sw_chunk(trow, (cb >> 3) + jj, 16384)) = pack8(r, jj, 1.f);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // every read of this chunk's operand block is done
+    if (tid == 0 && c + 2 < n_chunks) bulk_load(ops, block_src(c + 2), WB_BYTES, bar_ops + 8 * buf);
+  }
+  cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && p.sf) {
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      const int cb = 64 * half + 32 * part;
+      uint32_t r[32];
+      tm_ld32(tlane + TM_S + cb, r);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) p.sf[sbase + (size_t)(cb + jj) * p.V + trow] = __uint_as_float(r[jj]);
+    }
+  }
+  if (!ok && tid == 0) {
+    // A wait expired: give the operand loads and MMAs still in flight a bounded wait before exit.
+    mbar_wait(bar_mma, mma_phase, &g_split_timeout);
+    mbar_wait(bar_ops, 0, &g_split_timeout);
+    mbar_wait(bar_ops + 8, 0, &g_split_timeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TM_COLS));
+}
+
+template <typename F>
+cudaError_t set_smem_once(F* fn, int bytes, std::atomic<uint64_t>& configured) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load(std::memory_order_relaxed) & bit)) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+int64_t split_slots(int64_t B, int64_t T, int64_t N, bool varlen) {
+  return varlen ? T / C + N + 1 : B * ((T + C - 1) / C);
+}
+
+size_t split_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, bool varlen) {
+  return (size_t)split_slots(B, T, N, varlen) * (size_t)H * (size_t)WB_BYTES;
+}
+
+cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
+  static std::atomic<uint64_t> cfg_p{0}, cfg_s{0};
+  cudaError_t e = set_smem_once(chunk_intra_kernel, P_SMEM, cfg_p);
+  if (e == cudaSuccess) e = set_smem_once(chunk_state_kernel, S_SMEM, cfg_s);
+  if (e != cudaSuccess) return e;
+  const int64_t slots = split_slots(p.B, p.T, p.N, p.cu != nullptr);
+  if (slots == 0 || p.N == 0) return cudaSuccess;
+  dim3 gp((unsigned)slots, (unsigned)p.H);
+  chunk_intra_kernel<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t grid = (int64_t)p.N * p.H * (p.V / VT);
+  chunk_state_kernel<<<(unsigned)grid, NTHREADS, S_SMEM, s>>>(p, static_cast<const unsigned char*>(ws));
+  return cudaGetLastError();
+}
+
+cudaError_t split_read_timeout(int* flag, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(flag, g_split_timeout, sizeof(int));
+  if (e != cudaSuccess || !reset) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_split_timeout, &zero, sizeof(int));
+}
+
+}  // namespace kda

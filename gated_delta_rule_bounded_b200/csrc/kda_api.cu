@@ -80,11 +80,12 @@ int kda_device_status(int* timed_out, int reset) {
   if (!timed_out) return fail(KDA_ERR_INVALID_ARG, "kda_device_status: null output");
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "kda_device_status synchronize");
-  int chunk_flag = 0, decode_flag = 0;
+  int chunk_flag = 0, split_flag = 0, decode_flag = 0;
   e = kda::chunk_read_timeout(&chunk_flag, reset != 0);
+  if (e == cudaSuccess) e = kda::split_read_timeout(&split_flag, reset != 0);
   if (e == cudaSuccess) e = kda::decode_read_timeout(&decode_flag, reset != 0);
   if (e != cudaSuccess) return cuda_fail(e, "kda_device_status read");
-  *timed_out = (chunk_flag || decode_flag) ? 1 : 0;
+  *timed_out = (chunk_flag || split_flag || decode_flag) ? 1 : 0;
   return ok();
 }
 
@@ -138,8 +139,7 @@ int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int6
     return fail(KDA_ERR_INVALID_ARG, "kda_prefill_workspace_bytes: negative size");
   if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "kda_prefill_workspace_bytes: unknown dtype");
   *bytes = 0;
-  if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype))
-    *bytes = kda::chunk_workspace_bytes(B, T, H, K, V, n_seq > 0 ? n_seq : B);
+  if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype)) *bytes = kda::chunk_workspace_bytes(B, T, H, n_seq);
   return ok();
 }
 
@@ -237,9 +237,7 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
 
   cudaError_t e;
   if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype)) {
-    size_t need = kda::chunk_workspace_bytes(B, T, H, K, V, N);
-    if (workspace_bytes < need || (need > 0 && !workspace))
-      return fail(KDA_ERR_INVALID_ARG, "%s: workspace of %zu bytes given, %zu needed", fn, workspace_bytes, need);
+    if (workspace_bytes > 0 && !workspace) return fail(KDA_ERR_INVALID_ARG, "%s: workspace_bytes > 0 with a null workspace", fn);
     e = kda::launch_chunk(p, workspace, workspace_bytes, s);
   } else {
     e = kda::launch_recurrent(p, dtype, s);

@@ -46,9 +46,14 @@ bool decode_bulk_supported(const ScanParams& p);
 cudaError_t launch_decode_bulk(const ScanParams& p, kda_dtype dt, cudaStream_t s);
 cudaError_t decode_read_timeout(int* flag, bool reset);
 // Chunked prefill for bf16 inputs (bounded decay), tensor cores.
+// With a workspace of chunk_workspace_bytes(...) it runs as two kernels (all chunks' state-independent
+// operands in parallel, then the recurrence); without one, as a single fused kernel.
 bool chunk_supported(int K, int V, kda_dtype dt);
-size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t N);
+size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t n_seq);
 cudaError_t launch_chunk(const ScanParams& p, void* ws, size_t ws_bytes, cudaStream_t s);
+size_t split_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, bool varlen);
+cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s);
+cudaError_t split_read_timeout(int* flag, bool reset);
 // Reads (and optionally clears) the chunk kernel's device-side timeout flag. Synchronous.
 cudaError_t chunk_read_timeout(int* flag, bool reset);
 // Copy initial state (or zeros) into final state for T == 0 calls.

@@ -98,9 +98,15 @@ int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda
                       kda_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * kda_prefill_workspace_bytes: bytes of device scratch kda_prefill needs for
- * these sizes (0 when the selected kernels keep everything on chip). The
- * caller allocates it; a larger buffer is fine.
+ * kda_prefill_workspace_bytes: bytes of device scratch that let kda_prefill
+ * take its two-kernel path for these sizes (0 when no path uses scratch).
+ * With bf16 inputs and K = 128, the two-kernel path first computes every
+ * chunk's state-independent operands in parallel and stores them in the
+ * workspace (about 1 KB per token and head), then runs the recurrence. Given
+ * at least this many bytes kda_prefill uses it; given less (or no workspace),
+ * it runs the single fused kernel instead, with identical results up to
+ * rounding. The caller allocates the workspace; a larger buffer is fine. n_seq
+ * is the number of packed sequences (0 without cu_seqlens).
  * ------------------------------------------------------------------------- */
 int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                                 int64_t n_seq, kda_dtype dtype, size_t* bytes);
@@ -126,8 +132,9 @@ int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int6
  *             to T; zero-length sequences allowed). N = n_seq then, else N = B.
  * o         [B,T,H,V]  dtype `dtype`, o[t] = S_t^T q_t with S_t the state
  *                      after token t's update.
- * workspace, workspace_bytes: device scratch of at least
- *             kda_prefill_workspace_bytes(...) bytes (may be NULL when that is 0).
+ * workspace, workspace_bytes: device scratch (see kda_prefill_workspace_bytes);
+ *             NULL / 0 selects the single-kernel path. Its contents are
+ *             overwritten; concurrent calls must not share one workspace.
  * T == 0 (or a zero-length packed sequence) copies initial_state (or zeros)
  * to final_state. Supported: K, V multiples of 16 in [16, 256].
  * ------------------------------------------------------------------------- */

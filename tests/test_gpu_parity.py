@@ -74,7 +74,13 @@ def gpu_pipeline(kda, d, **kw):
     alpha = kda.bounded_decay(g["z"], g["A_log"], g["g_min"])
     o, sf = kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], g["initial_state"], g["cu_seqlens"], **kw)
     torch.cuda.synchronize()
+    assert not kda.device_status(), "a kernel's bounded wait expired"
     return o, sf
+
+
+# bf16 prefill runs either as two kernels (state-independent chunk operands for all chunks in
+# parallel through a workspace, then the recurrence) or as one fused kernel (no workspace).
+PATHS = pytest.mark.parametrize("use_workspace", [True, False], ids=["split", "fused"])
 
 
 def oracle_pipeline(d, heads=None):
@@ -148,10 +154,11 @@ def test_tiny_fp32_workload(kda):
     (1, 1, 2, 128, 128, True),
     (3, 16, 2, 32, 48, True),
 ])
-def test_prefill_bf16_matches_oracle(kda, B, T, H, K, V, init):
+@PATHS
+def test_prefill_bf16_matches_oracle(kda, B, T, H, K, V, init, use_workspace):
     d = W.random_scan_case(B, T, H, K, V, seed=T + H + K, dtype="bf16", z_std=2.0,
                            init_std=0.1 if init else None)
-    o, sf = gpu_pipeline(kda, d)
+    o, sf = gpu_pipeline(kda, d, use_workspace=use_workspace)
     ro, rs = oracle_pipeline(d)
     check(o, ro, "bf16", "o")
     check(sf, rs, "bf16", "final_state")
@@ -166,14 +173,15 @@ def test_prefill_fp32_matches_oracle(kda, B, T, H, K, V):
     check(sf, rs, "f32", "final_state")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_prefill_varlen_with_empty_segments(kda, dtype):
+@pytest.mark.parametrize("dtype,use_workspace", [("bf16", True), ("bf16", False), ("f32", True)],
+                         ids=["bf16-split", "bf16-fused", "f32"])
+def test_prefill_varlen_with_empty_segments(kda, dtype, use_workspace):
     lens = [70, 0, 129, 1, 0, 64, 200]
     cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
     d = W.random_scan_case(1, int(cu[-1]), 2, 128, 128, seed=17, dtype=dtype, z_std=2.0, init_std=None)
     d["cu_seqlens"] = cu
     d["initial_state"] = torch.randn(len(lens), 2, 128, 128, generator=torch.Generator().manual_seed(1)) * 0.1
-    o, sf = gpu_pipeline(kda, d)
+    o, sf = gpu_pipeline(kda, d, use_workspace=use_workspace)
     ro, rs = oracle_pipeline(d)
     check(o, ro, dtype, "o")
     check(sf, rs, dtype, "final_state")
@@ -197,7 +205,8 @@ def test_prefill_empty_sequence(kda, with_init):
     assert torch.equal(sf.cpu(), s0 if with_init else torch.zeros(B, H, K, V))
 
 
-def test_prefill_strided_views(kda):
+@PATHS
+def test_prefill_strided_views(kda, use_workspace):
     """q, k, v as slices of one fused projection tensor; gate and o as views too."""
     B, T, H, K, V = 2, 97, 3, 128, 128
     g = torch.Generator().manual_seed(8)
@@ -213,7 +222,8 @@ def test_prefill_strided_views(kda):
     assert not qd.is_contiguous()
     alpha = kda.bounded_decay(zbig[..., 32:32 + K].to(DEV), A.to(DEV), -5.0)
     o_big = torch.zeros(B, T, H, 2 * V, device=DEV, dtype=torch.bfloat16)
-    o, sf = kda.prefill(qd, kd, vd, alpha, beta_big[..., 0].to(DEV), s0.to(DEV), out=o_big[..., V:])
+    o, sf = kda.prefill(qd, kd, vd, alpha, beta_big[..., 0].to(DEV), s0.to(DEV), out=o_big[..., V:],
+                        use_workspace=use_workspace)
     torch.cuda.synchronize()
     assert o.data_ptr() == o_big[..., V:].data_ptr()
     ra = oracle.bounded_decay(zbig[..., 32:32 + K], A, -5.0)
@@ -239,18 +249,20 @@ def test_prefill_log_gate_and_inputs_untouched(kda):
     check(sf, rs, "bf16", "final_state")
 
 
-def test_prefill_resume_in_place(kda):
+@PATHS
+def test_prefill_resume_in_place(kda, use_workspace):
     """final_state may alias initial_state; splitting and resuming equals one pass."""
     d = W.random_scan_case(2, 200, 2, 128, 128, seed=31, dtype="bf16", z_std=2.0, init_std=0.1)
     g = to_dev(d)
     alpha = kda.bounded_decay(g["z"], g["A_log"], -5.0)
-    o_full, s_full = kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], g["initial_state"])
+    kw = dict(use_workspace=use_workspace)
+    o_full, s_full = kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], g["initial_state"], **kw)
     st = g["initial_state"].clone()
     cut = 77
     o1, _ = kda.prefill(g["q"][:, :cut], g["k"][:, :cut], g["v"][:, :cut], alpha[:, :cut], g["beta"][:, :cut],
-                        st, final_state=st)
+                        st, final_state=st, **kw)
     o2, _ = kda.prefill(g["q"][:, cut:], g["k"][:, cut:], g["v"][:, cut:], alpha[:, cut:], g["beta"][:, cut:],
-                        st, final_state=st)
+                        st, final_state=st, **kw)
     torch.cuda.synchronize()
     ro, rs = oracle_pipeline(d)
     check(torch.cat([o1, o2], 1), ro, "bf16", "o (split)")
@@ -348,9 +360,10 @@ def test_decode_workload_1000_steps_sampled(kda):
 # ---------------------------------------------------------------------------------------------
 
 @pytest.mark.slow
-def test_prefill_workload_4096_sampled_heads(kda):
+@PATHS
+def test_prefill_workload_4096_sampled_heads(kda, use_workspace):
     d = W.make_scan_inputs(W.PREFILL)
-    o, sf = gpu_pipeline(kda, d)
+    o, sf = gpu_pipeline(kda, d, use_workspace=use_workspace)
     heads = [0, 13, 47, 95]
     ro, rs = oracle_pipeline(d, heads)
     check(o[:, :, heads], ro, "bf16", "o")
@@ -358,9 +371,10 @@ def test_prefill_workload_4096_sampled_heads(kda):
 
 
 @pytest.mark.slow
-def test_varlen_workload_sampled_heads(kda):
+@PATHS
+def test_varlen_workload_sampled_heads(kda, use_workspace):
     d = W.make_scan_inputs(W.VARLEN)
-    o, sf = gpu_pipeline(kda, d)
+    o, sf = gpu_pipeline(kda, d, use_workspace=use_workspace)
     heads = [3, 60]
     ro, rs = oracle_pipeline(d, heads)
     check(o[:, :, heads], ro, "bf16", "o")
