@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["bounded_decay", "prefill", "decode_step", "prefill_workspace_bytes", "device_status", "KDAError",
+__all__ = ["bounded_decay", "prefill", "prefill_noalloc", "decode_step", "prefill_workspace_bytes", "device_status", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -70,8 +70,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_prefill_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, i64, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.kda_prefill.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64,
                                 i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
+    lib.kda_prefill_noalloc.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64,
+                                        i64, i64, i64, i64, i64, lp, vp, vp]
     lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, i64, i64, i64, i64, lp, vp, vp]
-    for fn in ("kda_bounded_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_decode_step"):
+    for fn in ("kda_bounded_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
+               "kda_decode_step"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_last_error.argtypes = []
@@ -232,6 +235,57 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
         cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
         _stream(dev)))
     return out, final_state
+
+
+NOALLOC_SCRATCH_BYTES = 128 << 20  # the library's static scratch (KDA_NOALLOC_SCRATCH_BYTES)
+
+
+def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
+                    out: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
+                    final_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
+                    gate_is_log: bool = False) -> None:
+    """``kda_prefill_noalloc``: the prefill with the library's static scratch as its workspace.
+
+    For callers that must not allocate device memory between steps (cudaMalloc / cudaFree
+    synchronise the device): neither this wrapper nor the call allocates anything, so every
+    tensor, ``out [B,T,H,V]`` and the optional ``final_state [N,H,K,V]`` included, comes from the
+    caller, contiguous in its innermost dim with 16-byte aligned rows. The first call on a device
+    looks up the scratch address (make it before any stream capture); calls that may overlap on
+    the GPU share the scratch and race on it. Sizes needing more than ``NOALLOC_SCRATCH_BYTES``
+    of workspace raise ``KDAError`` (KDA_ERR_UNSUPPORTED).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta"), (out, "out")):
+        _cuda(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3] or out.shape != v.shape:
+        raise ValueError("q, k must be [B,T,H,K]; v and out [B,T,H,V]")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise TypeError("q, k, v and out must share one dtype")
+    if gate.shape != q.shape or gate.dtype != torch.float32:
+        raise ValueError("gate must be fp32 [B,T,H,K]")
+    if beta.shape != q.shape[:3] or beta.dtype != torch.float32:
+        raise ValueError("beta must be fp32 [B,T,H]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    n_seq, N = 0, B
+    if cu_seqlens is not None:
+        _cuda(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+            raise TypeError("cu_seqlens must be a contiguous int32 tensor")
+        n_seq = N = cu_seqlens.numel() - 1
+    for t, n in ((initial_state, "initial_state"), (final_state, "final_state")):
+        if t is not None:
+            _cuda(t, n)
+            if t.shape != (N, H, K, V) or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous fp32 [{N},{H},{K},{V}] tensor")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (out, "out")):
+        if _rowwise(t) is not t:
+            raise ValueError(f"{n}: innermost dim must be contiguous with 16-byte aligned rows")
+    layout = Layout(_strides4(q), _strides4(k), _strides4(v), _strides4(gate), _strides3(beta), _strides4(out))
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    _check("kda_prefill_noalloc", load_library().kda_prefill_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+        KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), ptr(initial_state), ptr(final_state),
+        ptr(cu_seqlens), n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,

@@ -70,6 +70,12 @@ void put(int64_t dst[3], const kda_strides& s) {
 
 }  // namespace
 
+namespace kda {
+
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
+}  // namespace kda
+
 extern "C" {
 
 const char* kda_last_error(void) { return g_err; }

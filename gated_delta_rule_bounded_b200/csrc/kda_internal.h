@@ -56,6 +56,8 @@ cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s);
 cudaError_t split_read_timeout(int* flag, bool reset);
 // Reads (and optionally clears) the chunk kernel's device-side timeout flag. Synchronous.
 cudaError_t chunk_read_timeout(int* flag, bool reset);
+// Records `msg` as the calling thread's kda_last_error() and returns `code`.
+int report_error(int code, const char* msg);
 // Copy initial state (or zeros) into final state for T == 0 calls.
 cudaError_t launch_state_copy(const float* s0, float* sf, int64_t n, cudaStream_t s);
 

@@ -24,7 +24,9 @@
  *   call returns an error other than KDA_ERR_CUDA; kda_last_error() then holds
  *   a one-line, thread-local description. Nothing throws across the ABI.
  * - Tensor pointers are DEVICE pointers owned by the caller; the library never
- *   allocates device or pinned memory and never frees what it is given. Calls
+ *   allocates device or pinned memory and never frees what it is given (the one
+ *   exception is kda_prefill_noalloc's fixed scratch array, which the CUDA
+ *   runtime places on a device when that call first runs there). Calls
  *   are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
  *   stream); the caller keeps every buffer alive until the work has finished.
  * - Layouts are the contract table's: q, k, alpha/g [B,T,H,K]; v, o [B,T,H,V];
@@ -145,6 +147,41 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
                 int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                 const kda_layout* layout, void* o,
                 void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * kda_prefill_noalloc: kda_prefill for callers that cannot allocate device
+ * memory. The pages have no counterpart; it is a library convenience.
+ *
+ * Who needs it: a plain C host that links only libkda and has no CUDA
+ * allocator of its own, and a serving loop that must not call cudaMalloc /
+ * cudaFree between steps (they synchronise the device). Such callers cannot
+ * hand kda_prefill the workspace its two-kernel path wants. This call takes
+ * that workspace from a scratch array compiled into the library, one copy per
+ * device, of KDA_NOALLOC_SCRATCH_BYTES bytes, and allocates nothing itself.
+ *
+ * Arguments, layouts, results and errors are kda_prefill's, without the
+ * workspace pair. Sizes whose workspace (kda_prefill_workspace_bytes) exceeds
+ * KDA_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_UNSUPPORTED and a
+ * message naming both sizes; nothing is launched then. Sizes that need no
+ * workspace (fp32 inputs, K != 128) run as kda_prefill does without one.
+ *
+ * Setup: the first call on a device (the device current at the call) looks
+ * up the scratch's device address once and keeps it; make that first call
+ * before any stream capture on that device.
+ *
+ * Sharing: every call on a device uses the same scratch. Nothing in it has to
+ * start at zero (each call writes all it reads), but calls whose GPU work may
+ * overlap -- on different streams, or from host threads with no ordering
+ * between them -- race on it; order them on one stream.
+ * ------------------------------------------------------------------------- */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)128 << 20) /* 128 MiB: 2,032 chunk-heads of 64 tokens */
+
+int kda_prefill_noalloc(const void* q, const void* k, const void* v, kda_dtype dtype,
+                        const float* gate, kda_gate_kind gate_kind, const float* beta,
+                        const float* initial_state, float* final_state,
+                        const int32_t* cu_seqlens, int64_t n_seq,
+                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                        const kda_layout* layout, void* o, kda_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * kda_decode_step: one new token per (b, h) against a kept state, in place.

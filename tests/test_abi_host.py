@@ -173,3 +173,25 @@ def test_python_binding_refuses_cpu_tensors():
         kda.bounded_decay(x, torch.zeros(1))
     with pytest.raises(ValueError, match="CUDA"):
         kda.prefill(x, x, x, x, torch.zeros(1, 2, 1))
+
+
+def test_noalloc_scratch_limit_matches_binding():
+    m = re.search(r"#define\s+KDA_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", open(HEADER).read())
+    assert m, "KDA_NOALLOC_SCRATCH_BYTES not found in kda.h"
+    assert int(m.group(1)) << int(m.group(2)) == kda.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_rejects_oversize_before_any_device_call(lib):
+    # 4096 tokens x 96 heads need 64 x 96 x 66,048 bytes of workspace, beyond the static scratch;
+    # the call must refuse on the host (the fake pointers are never dereferenced).
+    layout = Layout(*[Strides(4096 * 96 * 128, 96 * 128, 128)] * 3, Strides(4096 * 96 * 128, 96 * 128, 128),
+                    Strides(4096 * 96, 96, 1), Strides(4096 * 96 * 128, 96 * 128, 128))
+    rc = lib.kda_prefill_noalloc(FAKE, FAKE, FAKE, 1, FAKE, 0, FAKE, None, None, None, 0,
+                                 1, 4096, 96, 128, 128, ctypes.byref(layout), FAKE, None)
+    assert rc == UNSUPPORTED
+    msg = lib.kda_last_error().decode()
+    assert "static scratch" in msg and str(64 * 96 * 66048) in msg
+    # Bad sizes are reported by the workspace query it shares with kda_prefill.
+    rc = lib.kda_prefill_noalloc(FAKE, FAKE, FAKE, 1, FAKE, 0, FAKE, None, None, None, 0,
+                                 1, -1, 96, 128, 128, None, FAKE, None)
+    assert rc == INVALID
