@@ -36,30 +36,42 @@ constexpr int WB_AQK = 57344;    // 8K   A_qk [t][i] (K-major B)
 constexpr int WB_GAM = 65536;    // 512  gamma_C, fp32 [128]
 constexpr int WB_BYTES = 66048;
 
-// Kernel P shared memory.
-constexpr int P_OUT = 0;                    // the workspace block image
-constexpr int P_QE = 66560;                 // 16K Qe [t][c]
+// Kernel P shared memory (104,192 bytes: two CTAs fit on an SM). Q*Gamma and K*gamma_C/Gamma
+// never touch it: the decay pass writes them from registers straight into the workspace block.
+constexpr int P_QE = 0;                     // 16K Qe [t][c]; after A_qk, -W (the block's first 16K)
 constexpr int P_KE = P_QE + 16384;          // 16K Ke [t][c]; after A_kk, the bf16 copy of T
 constexpr int P_KC = P_KE + 16384;          // 16K Kc [t][c]
 constexpr int P_KG = P_KC + 16384;          // 16K K*Gamma [i][c]
 constexpr int P_AKK = P_KG + 16384;         // 16K A_kk fp32
-constexpr int P_BETA = P_AKK + 16384;       // 256 beta
+constexpr int P_TP = P_AKK + 16384;         // 8K  T'    } the block's last 16,896 bytes, in
+constexpr int P_AQK = P_TP + 8192;          // 8K  A_qk  } workspace order
+constexpr int P_GAM = P_AQK + 8192;         // 512 gamma_C }
+constexpr int P_BETA = P_GAM + 512;         // 256 beta
 constexpr int P_VEC = P_BETA + 256;         // vectors
 constexpr int P_SMEM = P_VEC + VEC_FLOATS * 4;
-static_assert(P_SMEM <= 227 * 1024, "shared memory budget");
+constexpr int P_TAIL = WB_BYTES - WB_TP;    // 16,896
+static_assert(P_AQK - P_TP == WB_AQK - WB_TP && P_GAM - P_TP == WB_GAM - WB_TP, "tail order matches the block");
+static_assert(P_TP % 1024 == 0 && P_AQK % 1024 == 0, "swizzle atoms need 1 KB alignment");
+static_assert(2 * (P_SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 
-// Kernel S shared memory.
+// Kernel S shared memory: the operand blocks of two chunks and their v tiles.
 constexpr int S_OPS = 0;                    // 2 x operand block (66048 B, padded to 66560)
 constexpr int S_OPS_STRIDE = 66560;
 constexpr int S_V = 2 * S_OPS_STRIDE;       // 2 x 16K v tile [i][v], two halves (MN-major A)
-constexpr int S_SBF = S_V + 2 * 16384;      // 32K S bf16 [v][c], two atoms of [128][64] (K-major A)
-constexpr int S_U = S_SBF + 32768;          // 16K U bf16 [v][i] (K-major A)
-constexpr int S_BAR = S_U + 16384;          // mbarriers: ops0, ops1, mma; TMEM base
+constexpr int S_BAR = S_V + 2 * 16384;      // mbarriers: ops0, ops1, mma; TMEM base
 constexpr int S_SMEM = S_BAR + 64;
 static_assert(S_SMEM <= 227 * 1024, "shared memory budget");
-static_assert(S_SBF % 1024 == 0 && S_U % 1024 == 0 && S_V % 1024 == 0, "swizzle atoms need 1 KB alignment");
+static_assert(S_V % 1024 == 0 && S_OPS_STRIDE % 1024 == 0, "swizzle atoms need 1 KB alignment");
 
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 192, TM_COLS = 256;
+// Kernel S tensor memory (columns; lane = value column v of the tile). S^T and U^T in fp32 are MMA
+// accumulators; their bf16 copies (two values per column) are the A operands of the next products;
+// O^T alternates between two buffers so one chunk's output drains while the next chunk's MMAs run.
+constexpr uint32_t TM_S = 0;      // 128  S^T fp32 [v][c]
+constexpr uint32_t TM_U = 128;    // 64   U^T fp32 [v][t]
+constexpr uint32_t TM_O = 192;    // 2x64 O^T fp32 [v][t]
+constexpr uint32_t TM_SB = 320;   // 64   S^T bf16 (K = c)
+constexpr uint32_t TM_UB = 384;   // 32   U^T bf16 (K = t)
+constexpr uint32_t TM_COLS = 512;
 
 __device__ __forceinline__ void seq_range(const ScanParams& p, int n, int64_t& t0, int64_t& t1, int64_t& brow) {
   t0 = 0;
@@ -107,11 +119,68 @@ __device__ __forceinline__ bool locate_slot(const ScanParams& p, int64_t s, int&
   return true;
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) chunk_intra_kernel(ScanParams p, unsigned char* ws) {
+// Decay pass, step 2 of kernel P: the same tiles as decay_step2 (chunk_common.cuh), with Q*Gamma and
+// K*gamma_C/Gamma stored straight into the workspace block `blk` (a warp's 32 four-byte stores
+// cover one 128-byte swizzled row). Tokens run forward for the E-scaled tiles and backward for the
+// F-scaled ones, so no per-token F array is held in registers.
+__device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch& pf, int da, int c0,
+                                              const float2 (&al)[16], unsigned char* blk) {
+  float* vec = reinterpret_cast<float*>(sm + P_VEC);
+  float2 e[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) e[b] = *reinterpret_cast<const float2*>(vec + VEC_TOT + b * 128 + c0);
+#pragma unroll
+  for (int b = 1; b < 4; ++b) {
+    e[b].x += e[b - 1].x;
+    e[b].y += e[b - 1].y;
+  }
+  // e[b] = log2 Gamma at r_b; log2 Gamma at s_a is e[a-1] (0 for a = 0)
+  const float2 gs = da == 0 ? make_float2(0.f, 0.f) : (da == 1 ? e[0] : (da == 2 ? e[1] : e[2]));
+  const float2 eda = da == 0 ? e[0] : (da == 1 ? e[1] : (da == 2 ? e[2] : e[3]));
+  __nv_bfloat16* D16 = reinterpret_cast<__nv_bfloat16*>(vec + VEC_D);
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    if (b <= da) {
+      const int pair = da * (da + 1) / 2 + b;
+      *reinterpret_cast<uint32_t*>(D16 + pair * 128 + c0) = pack_bf16(ex2(gs.x - e[b].x), ex2(gs.y - e[b].y));
+    }
+  }
+  if (da == 0) *reinterpret_cast<float2*>(sm + P_GAM + 4 * c0) = make_float2(ex2(e[3].x), ex2(e[3].y));
+  const float2 GS = make_float2(ex2(gs.x), ex2(gs.y));
+  const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));
+  float2 E = make_float2(1.f, 1.f);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = 16 * da + i;
+    E.x *= al[i].x;
+    E.y *= al[i].y;
+    const float2 qf = unpack_bf16(pf.q[i]), kf = unpack_bf16(pf.k[i]);
+    const uint32_t off = sw_e(t, c0, 8192);
+    const float qex = qf.x * E.x, qey = qf.y * E.y, kex = kf.x * E.x, key = kf.y * E.y;
+    *reinterpret_cast<uint32_t*>(sm + P_QE + off) = pack_bf16(qex, qey);
+    *reinterpret_cast<uint32_t*>(sm + P_KE + off) = pack_bf16(kex, key);
+    *reinterpret_cast<uint32_t*>(sm + P_KG + off) = pack_bf16(kex * GS.x, key * GS.y);
+    *reinterpret_cast<uint32_t*>(blk + WB_QG + off) = pack_bf16(qex * GS.x, qey * GS.y);
+  }
+  float2 F = make_float2(1.f, 1.f);
+#pragma unroll
+  for (int i = 15; i >= 0; --i) {
+    const int t = 16 * da + i;
+    const float2 kf = unpack_bf16(pf.k[i]);
+    const uint32_t off = sw_e(t, c0, 8192);
+    const float kfx = kf.x * F.x, kfy = kf.y * F.y;
+    *reinterpret_cast<uint32_t*>(sm + P_KC + off) = pack_bf16(kfx, kfy);
+    *reinterpret_cast<uint32_t*>(blk + WB_KT + off) = pack_bf16(kfx * PM.x, kfy * PM.y);
+    F.x *= al[i].x;
+    F.y *= al[i].y;
+  }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, unsigned char* ws) {
   extern __shared__ __align__(1024) unsigned char sm[];
   const uint32_t sb = smem_u32(sm);
-  constexpr IntraLayout LY{P_QE, P_KE, P_KC, P_OUT + WB_QG, P_KG, P_OUT + WB_KT, P_AKK, P_OUT + WB_AQK,
-                           P_OUT + WB_TP, P_KE, P_VEC};
+  // qg and kt are not staged in shared memory by this kernel (p_decay_step2 stores them to the block).
+  constexpr IntraLayout LY{P_QE, P_KE, P_KC, -1, P_KG, -1, P_AKK, P_AQK, P_TP, P_KE, P_VEC};
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int h = blockIdx.y;
@@ -122,6 +191,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_intra_kernel(ScanParams p, 
   seq_range(p, n, t0, t1, brow);
   const int64_t tc0 = t0 + (int64_t)j * C;
   const int nv = (int)min((int64_t)C, t1 - tc0);
+  unsigned char* blk = ws + ((size_t)slot * p.H + h) * WB_BYTES;
 
   ChunkCtx x;
   x.q = static_cast<const __nv_bfloat16*>(p.q);
@@ -141,64 +211,69 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_intra_kernel(ScanParams p, 
   x.bst = p.bs[1];
 
   const int c0 = 2 * (tid & 63), da = tid >> 6;
-  Prefetch pf;
-  load_qkg(x, tc0, nv, c0, da, pf);
   float* beta_s = reinterpret_cast<float*>(sm + P_BETA);
-  if (tid < C) beta_s[tid] = tid < nv ? __ldg(x.beta + x.boff + (tc0 + tid) * x.bst) : 0.f;
-
   {
+    Prefetch pf;
+    load_qkg(x, tc0, nv, c0, da, pf);
+    if (tid < C) beta_s[tid] = tid < nv ? __ldg(x.beta + x.boff + (tc0 + tid) * x.bst) : 0.f;
     float2 al[16];
     decay_step1(sm, LY, pf, nv, da, c0, p.gate_log != 0, al);
     __syncthreads();
-    decay_step2(sm, LY, pf, da, c0, al);
+    p_decay_step2(sm, pf, da, c0, al, blk);
   }
   __syncthreads();
   intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
 
-  // W = T' (K*Gamma) on mma.sync; warp (m, nh) owns rows 16m.. and columns 64nh.. . -W is stored
-  // as the MN-major operand of S^T (-W)^T: row c holds W[0..63][c].
+  // W = T' (K*Gamma) on mma.sync. Warp w owns columns 16w.. of all 64 rows, so every warp does the
+  // same ten block products of the lower-triangular T'. -W is stored (over the dead Qe tile) as the
+  // MN-major operand of S^T (-W)^T: row c holds W[0..63][c].
   {
-    const int m = warp & 3, nh = warp >> 2;
-    float acc[8][4];
+    float acc[4][2][4];
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj)
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[jj][e] = 0.f;
-    for (int kk = 0; kk <= m; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(sb + P_OUT + WB_TP + sw_chunk(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4), 8192),
-              a0, a1, a2, a3);
-      const int rr = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+      for (int jn = 0; jn < 2; ++jn)
 #pragma unroll
-      for (int pp = 0; pp < 4; ++pp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sb + P_KG + sw_chunk(rr, 8 * nh + 2 * pp + (lane >> 4), 8192), b0, b1, b2, b3);
-        mma_bf16(acc[2 * pp], a0, a1, a2, a3, b0, b1);
-        mma_bf16(acc[2 * pp + 1], a0, a1, a2, a3, b2, b3);
+        for (int e = 0; e < 4; ++e) acc[m][jn][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(sb + P_KG + sw_chunk(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * warp + (lane >> 4), 8192), b0, b1,
+                b2, b3);
+#pragma unroll
+      for (int m = kk; m < 4; ++m) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(sb + P_TP + sw_chunk(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4), 8192), a0, a1,
+                a2, a3);
+        mma_bf16(acc[m][0], a0, a1, a2, a3, b0, b1);
+        mma_bf16(acc[m][1], a0, a1, a2, a3, b2, b3);
       }
     }
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj)
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int t = 16 * m + g + 8 * hr, c = 64 * nh + 8 * jj + 2 * tq;
-        *reinterpret_cast<__nv_bfloat16*>(sm + P_OUT + WB_W + sw_e(c, t, 0)) = __float2bfloat16_rn(-acc[jj][2 * hr]);
-        *reinterpret_cast<__nv_bfloat16*>(sm + P_OUT + WB_W + sw_e(c + 1, t, 0)) =
-            __float2bfloat16_rn(-acc[jj][2 * hr + 1]);
-      }
-    if (tid < 32)
-      *reinterpret_cast<float4*>(sm + P_OUT + WB_GAM + 16 * tid) =
-          *reinterpret_cast<const float4*>(sm + P_VEC + 4 * (VEC_GAM + 4 * tid));
+      for (int jn = 0; jn < 2; ++jn)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int t = 16 * m + g + 8 * hr, c = 16 * warp + 8 * jn + 2 * tq;
+          *reinterpret_cast<__nv_bfloat16*>(sm + P_QE + sw_e(c, t, 0)) = __float2bfloat16_rn(-acc[m][jn][2 * hr]);
+          *reinterpret_cast<__nv_bfloat16*>(sm + P_QE + sw_e(c + 1, t, 0)) =
+              __float2bfloat16_rn(-acc[m][jn][2 * hr + 1]);
+        }
   }
   fence_async_smem();
   __syncthreads();
   if (tid == 0) {
-    unsigned char* dst = ws + ((size_t)slot * p.H + h) * WB_BYTES;
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(sb + P_OUT),
-                 "r"(WB_BYTES)
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(blk + WB_W), "r"(sb + P_QE),
+                 "r"(WB_QG - WB_W)
+                 : "memory");
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(blk + WB_TP), "r"(sb + P_TP),
+                 "r"(P_TAIL)
                  : "memory");
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    // Shared memory must stay valid until the copies have read it; their global writes complete
+    // before the kernel does.
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   }
 }
 
@@ -207,6 +282,22 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
+}
+
+// O^T of one chunk (TMEM columns [tm_o, tm_o + 64)) to o: this thread's lane v, tokens 32*half...
+__device__ __forceinline__ void store_o(const ScanParams& p, uint32_t tlane, uint32_t tm_o, int64_t brow, int h, int vt,
+                                       int trow, int half, int64_t tc0, int nv) {
+  uint32_t r[32];
+  tm_ld32(tlane + tm_o + 32 * half, r);
+  const int64_t ost = p.os[1];
+  __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + brow * p.os[0] + h * p.os[2] + (int64_t)vt * VT + trow +
+                      (tc0 + 32 * half) * ost;
+  const int jmax = min(32, nv - 32 * half);
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    if (jj < jmax) *op = __float2bfloat16_rn(__uint_as_float(r[jj]));
+    op += ost;
+  }
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, const unsigned char* ws) {
@@ -257,10 +348,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
   const uint32_t tlane = tmem + ((uint32_t)(32 * quad) << 16);
 
   if (n_chunks > 0) {
-    if (tid == 0) {
-      bulk_load(sb + S_OPS, block_src(0), WB_BYTES, bar_ops);
-      if (n_chunks > 1) bulk_load(sb + S_OPS + S_OPS_STRIDE, block_src(1), WB_BYTES, bar_ops + 8);
-    }
+    if (tid == 0) bulk_load(sb + S_OPS, block_src(0), WB_BYTES, bar_ops);
     load_v(x, sb + S_V, t0, (int)min((int64_t)C, t1 - t0), tid);
     cp_async_commit();
   }
@@ -275,13 +363,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     for (int jj = 0; jj < 32; ++jj)
       r[jj] = __float_as_uint(p.s0 ? p.s0[sbase + (size_t)(cb + jj) * p.V + trow] : 0.f);
     tm_st32(tlane + TM_S + cb, r);
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj)
-      *reinterpret_cast<uint4*>(sm + S_SBF + sw_chunk(trow, (cb >> 3) + jj, 16384)) = pack8(r, jj, 1.f);
   }
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 
-  uint32_t mma_phase = 0;
+  // Each chunk's MMAs complete twice on bar_mma, group A then group B, and every completion is
+  // waited for before the next group is issued: group A always completes phase parity 0, B parity 1.
   bool ok = true;
   for (int c = 0; c < n_chunks && ok; ++c) {
     const int64_t tc0 = t0 + (int64_t)c * C;
@@ -290,43 +376,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     const uint32_t ops = sb + S_OPS + buf * S_OPS_STRIDE;
     const unsigned char* opsp = sm + S_OPS + buf * S_OPS_STRIDE;
     const uint32_t vbuf = sb + S_V + buf * 16384;
+    const uint32_t tm_o = TM_O + 64 * buf;
 
-    cp_async_wait_all();
-    fence_async_smem();
-    tc_fence_before();
-    ok = __syncthreads_and(mbar_wait(bar_ops + 8 * buf, (c >> 1) & 1, &g_split_timeout));
+    // The previous chunk's group B is done (TMEM S^T holds S_{c-1}); this chunk's operands have landed.
+    bool w = c == 0 || mbar_wait(bar_mma, 1, &g_split_timeout);
+    w = w && mbar_wait(bar_ops + 8 * buf, (c >> 1) & 1, &g_split_timeout);
+    ok = __syncthreads_and(w);
     tc_fence_after();
     if (!ok) break;
-    if (c + 1 < n_chunks)
-      load_v(x, sb + S_V + (buf ^ 1) * 16384, tc0 + C, (int)min((int64_t)C, t1 - tc0 - C), tid);
-    cp_async_commit();
 
-    // ---- group A: O^T = S^T (Q*Gamma)^T; U^T = V^T T'^T + S^T (-W)^T --------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id_kk = idesc_bf16(64, 0, 0), id_mk = idesc_bf16(64, 1, 0), id_km = idesc_bf16(64, 0, 1);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t as = sdesc(sb + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-        tc_mma(tmem + TM_O, as, sdesc(ops + WB_QG + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id_kk, ks > 0);
-      }
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        tc_mma(tmem + TM_U, sdesc(vbuf + ks * 2048, 8192, 1024), sdesc(ops + WB_TP + ks * 32, 16, 1024), id_mk, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        tc_mma(tmem + TM_U, sdesc(sb + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-               sdesc(ops + WB_W + ks * 2048, 8192, 1024), id_km, 1);
-      tc_commit(bar_mma);
-    }
-    // meanwhile: S^T *= gamma_C in TMEM (group A reads the bf16 copy of S)
+    // S^T -> its bf16 copy (group A's operand) and S^T *= gamma_C in place (group B accumulates on it).
     {
       const float* gam = reinterpret_cast<const float*>(opsp + WB_GAM);
-      uint32_t r[32];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         const int cb = 64 * half + 32 * part;
+        uint32_t r[32], b16[16];
         tm_ld32(tlane + TM_S + cb, r);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) b16[jj] = pack_bf16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]));
+        tm_st16(tlane + TM_SB + cb / 2, b16);
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const float4 gm = *reinterpret_cast<const float4*>(gam + cb + 4 * jj);
@@ -339,66 +408,73 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
-    ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase, &g_split_timeout));
-    mma_phase ^= 1;
-    tc_fence_after();
-    if (!ok) break;
-
-    // ---- U to shared memory (K-major A, row v holds U[0..63][v]) -----------------------------------
-    {
-      uint32_t r[32];
-      tm_ld32(tlane + TM_U + 32 * half, r);
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        *reinterpret_cast<uint4*>(sm + S_U + sw_chunk(trow, 4 * half + jj, 0)) = pack8(r, jj, 1.f);
-    }
+    cp_async_wait_all();  // this chunk's v tile
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    tc_fence_after();
 
-    // ---- group B: O^T += U^T A_qk^T; S^T += U^T (K*gamma_C/Gamma) -----------------------------------
+    // The other buffers' last readers (chunk c-1's MMAs) are done: prefetch chunk c+1 into them.
+    if (c + 1 < n_chunks) {
+      if (tid == 0) bulk_load(sb + S_OPS + (buf ^ 1) * S_OPS_STRIDE, block_src(c + 1), WB_BYTES, bar_ops + 8 * (buf ^ 1));
+      load_v(x, sb + S_V + (buf ^ 1) * 16384, tc0 + C, (int)min((int64_t)C, t1 - tc0 - C), tid);
+    }
+    cp_async_commit();
+
+    // ---- group A: O^T = S^T (Q*Gamma)^T; U^T = V^T T'^T + S^T (-W)^T --------------------------------
     if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id_o = idesc_bf16(64, 0, 0), id_s = idesc_bf16(128, 0, 1);
+      constexpr uint32_t id_kk = idesc_bf16(64, 0, 0), id_mk = idesc_bf16(64, 1, 0), id_km = idesc_bf16(64, 0, 1);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t au = sdesc(sb + S_U + ks * 32, 16, 1024);
-        tc_mma(tmem + TM_O, au, sdesc(ops + WB_AQK + ks * 32, 16, 1024), id_o, 1);
-        tc_mma(tmem + TM_S, au, sdesc(ops + WB_KT + ks * 2048, 8192, 1024), id_s, 1);
-      }
+      for (int ks = 0; ks < 8; ++ks)
+        tc_mma_ts(tmem + tm_o, tmem + TM_SB + 8 * ks, sdesc(ops + WB_QG + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
+                  id_kk, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        tc_mma(tmem + TM_U, sdesc(vbuf + ks * 2048, 8192, 1024), sdesc(ops + WB_TP + ks * 32, 16, 1024), id_mk, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        tc_mma_ts(tmem + TM_U, tmem + TM_SB + 8 * ks, sdesc(ops + WB_W + ks * 2048, 8192, 1024), id_km, 1);
       tc_commit(bar_mma);
     }
-    ok = __syncthreads_and(mbar_wait(bar_mma, mma_phase, &g_split_timeout));
-    mma_phase ^= 1;
+    // meanwhile: the previous chunk's output
+    if (c > 0) store_o(p, tlane, TM_O + 64 * (buf ^ 1), brow, h, vt, trow, half, tc0 - C, C);
+
+    ok = __syncthreads_and(mbar_wait(bar_mma, 0, &g_split_timeout));
     tc_fence_after();
     if (!ok) break;
 
-    // ---- O to global memory, S to its bf16 copy ----------------------------------------------------
+    // ---- U^T -> its bf16 copy ---------------------------------------------------------------------
     {
-      uint32_t r[32];
-      tm_ld32(tlane + TM_O + 32 * half, r);
-      const int64_t ost = p.os[1];
-      __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + brow * p.os[0] + h * p.os[2] + (int64_t)vt * VT +
-                          trow + (tc0 + 32 * half) * ost;
-      const int jmax = min(32, nv - 32 * half);
+      uint32_t r[32], b16[16];
+      tm_ld32(tlane + TM_U + 32 * half, r);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        if (jj < jmax) *op = __float2bfloat16_rn(__uint_as_float(r[jj]));
-        op += ost;
-      }
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int cb = 64 * half + 32 * part;
-        tm_ld32(tlane + TM_S + cb, r);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          *reinterpret_cast<uint4*>(sm + S_SBF + sw_chunk(trow, (cb >> 3) + jj, 16384)) = pack8(r, jj, 1.f);
-      }
+      for (int jj = 0; jj < 16; ++jj) b16[jj] = pack_bf16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]));
+      tm_st16(tlane + TM_UB + 16 * half, b16);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
-    fence_async_smem();
     tc_fence_before();
-    __syncthreads();  // every read of this chunk's operand block is done
-    if (tid == 0 && c + 2 < n_chunks) bulk_load(ops, block_src(c + 2), WB_BYTES, bar_ops + 8 * buf);
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- group B: O^T += U^T A_qk^T; S^T += U^T (K*gamma_C/Gamma) -----------------------------------
+    if (tid == 0) {
+      constexpr uint32_t id_o = idesc_bf16(64, 0, 0), id_s = idesc_bf16(128, 0, 1);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        tc_mma_ts(tmem + tm_o, tmem + TM_UB + 8 * ks, sdesc(ops + WB_AQK + ks * 32, 16, 1024), id_o, 1);
+        tc_mma_ts(tmem + TM_S, tmem + TM_UB + 8 * ks, sdesc(ops + WB_KT + ks * 2048, 8192, 1024), id_s, 1);
+      }
+      tc_commit(bar_mma);
+    }
+  }
+  // The last chunk's group B, then its output.
+  if (ok && n_chunks > 0) {
+    ok = __syncthreads_and(mbar_wait(bar_mma, 1, &g_split_timeout));
+    tc_fence_after();
+    if (ok) {
+      const int64_t tl = t0 + (int64_t)(n_chunks - 1) * C;
+      store_o(p, tlane, TM_O + 64 * ((n_chunks - 1) & 1), brow, h, vt, trow, half, tl, (int)(t1 - tl));
+    }
   }
   cp_async_wait_all();
   tc_fence_before();
@@ -415,8 +491,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     }
   }
   if (!ok && tid == 0) {
-    // A wait expired: give the operand loads and MMAs still in flight a bounded wait before exit.
-    mbar_wait(bar_mma, mma_phase, &g_split_timeout);
+    // A wait expired: give the MMAs and operand loads that may still be in flight a bounded wait.
+    mbar_wait(bar_mma, 0, &g_split_timeout);
+    mbar_wait(bar_mma, 1, &g_split_timeout);
     mbar_wait(bar_ops, 0, &g_split_timeout);
     mbar_wait(bar_ops + 8, 0, &g_split_timeout);
   }
@@ -434,6 +511,9 @@ cudaError_t set_smem_once(F* fn, int bytes, std::atomic<uint64_t>& configured) {
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_relaxed) & bit)) {
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    // The largest carveout, so that kernel P's two CTAs per SM both fit.
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
