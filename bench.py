@@ -3,11 +3,13 @@
 Workloads (H=96, K=V=128, synthetic seeded inputs from ``workloads.py``):
 
 * prefill -- B=1, T=4096, bf16 q/k/v, fp32 decay logits (z ~ N(0,2)), fp32 beta,
-  zero initial state, fp32 final state. One step = the gate kernel (logits ->
-  alpha) plus the chunked prefill (-> o, final_state). ``value`` is tokens/s.
+  zero initial state, fp32 final state. One step = one ``kda_prefill_logits``
+  call: the chunked prefill evaluates the bounded gate from the logits while it
+  reads them (-> o, final_state). ``value`` is tokens/s.
 * decode -- B=64 kept 128x128 fp32 states (402.7 MB), bf16 q/k/v, z ~ N(0,1).
-  One step = the gate kernel plus the in-place decode step. Reported in the
-  ``decode`` object as state GB/s (2*4*K*V*B*H bytes per step) and steps/s.
+  One step = one in-place ``kda_decode_step_logits`` call (gate inside the
+  step). Reported in the ``decode`` object as state GB/s (2*4*K*V*B*H bytes per
+  step) and steps/s.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronise, CUDA events on the stream the kernels are launched on,
@@ -51,7 +53,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 def prefill_bytes(B, T, H, K, V, n_states_in, n_states_out, es=2):
     """Minimum HBM bytes of one prefill launch: read q, k (K each), v (V) in the input dtype,
-    the decay (alpha or g, K fp32) and beta (fp32) per token-head, write o (V); read/write the
+    the decay input (alpha, g or the logits z; K fp32) and beta (fp32) per token-head, write o (V); read/write the
     fp32 states."""
     per_tok_head = 2 * K * es + V * es + 4 * K + 4 + V * es
     return B * T * H * per_tok_head + (n_states_in + n_states_out) * H * K * V * 4
@@ -63,7 +65,7 @@ def prefill_flops(B, T, H, K, V, C=64):
 
 
 def decode_bytes(B, H, K, V, es=2):
-    """Per step: state read + write (8KV), q, k, v, o in the input dtype, alpha fp32, beta fp32."""
+    """Per step: state read + write (8KV), q, k, v, o in the input dtype, the decay input (K fp32), beta fp32."""
     return B * H * (8 * K * V + (2 * K + 2 * V) * es + 4 * K + 4)
 
 
@@ -264,23 +266,18 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     d = W.make_scan_inputs(w)
     B, T, H, K, V = w.B, w.T, w.H, w.K, w.V
     g = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in d.items()}
-    alpha = torch.empty(B, T, H, K, device=dev, dtype=torch.float32)
     o = torch.empty(B, T, H, V, device=dev, dtype=torch.bfloat16)
     sf = torch.empty(B, H, K, V, device=dev, dtype=torch.float32)
     ws_bytes = kda.prefill_workspace_bytes(B, T, H, K, V, 0, torch.bfloat16)
     ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
 
-    # The gate writes the log-decay g = log(alpha) and the prefill takes it directly (the ABI
-    # accepts alpha or g); this skips an exp in the gate and a log in the scan.
-    def gate_fn():
-        kda.bounded_decay(g["z"], g["A_log"], w.g_min, log_decay=True, out=alpha)
-
+    # One call: the scan kernels read the decay logits z and evaluate the bounded gate themselves.
     def prefill_fn():
-        kda.prefill(g["q"], g["k"], g["v"], alpha, g["beta"], None, gate_is_log=True, out=o, final_state=sf,
-                    workspace=ws)
+        kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], w.g_min, g["beta"], None, out=o,
+                           final_state=sf, workspace=ws)
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
-    total_ms, (gate_ms, pre_ms) = timed_loop([gate_fn, prefill_fn], args.steps, args.warmup, world, stream, sampler)
+    total_ms, (pre_ms,) = timed_loop([prefill_fn], args.steps, args.warmup, world, stream, sampler)
     value, total_ms = weak_scaling_value(B * T * args.steps, total_ms, world)
     ms_per_step = total_ms / args.steps
     tokens = B * T * world
@@ -290,17 +287,17 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     tflops = flops / (pre_ms / 1e3) / 1e12
     res = {
         "value": value, "ms_per_step": ms_per_step, "workload": w, "clocks": sampler.summary() if sampler else None,
-        "kernels_ms": {"bounded_decay": gate_ms, "prefill": pre_ms},
+        "kernels_ms": {"prefill_logits": pre_ms},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "kernel": "kda_prefill",
+                     "frac": achieved / hbm, "traffic": None, "kernel": "kda_prefill_logits",
                      "bytes_per_launch": pb, "ms_per_launch": pre_ms, "peak_source": f"{peak_src} hbm_gbs",
                      "tensor": {"tflops_at_C64_formula": tflops, "peak": bf16_peak,
                                 "frac": tflops / bf16_peak, "flops_per_launch": flops}},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 2 * args.steps,  # the operand kernel and the recurrence kernel per call
     }
     if args.no_e2e:
         return res
-    # e2e: pinned host inputs -> device, gate + prefill, o and final state -> pinned host
+    # e2e: pinned host inputs -> device, prefill from logits, o and final state -> pinned host
     host = {n: d[n].pin_memory() for n in ("q", "k", "v", "z", "A_log", "beta")}
     o_host = torch.empty(B, T, H, V, dtype=torch.bfloat16).pin_memory()
     sf_host = torch.empty(B, H, K, V, dtype=torch.float32).pin_memory()
@@ -311,9 +308,8 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     def e2e_fn():
         for n, x in host.items():
             dev_in[n].copy_(x, non_blocking=True)
-        kda.bounded_decay(dev_in["z"], dev_in["A_log"], w.g_min, log_decay=True, out=alpha)
-        kda.prefill(dev_in["q"], dev_in["k"], dev_in["v"], alpha, dev_in["beta"], None, gate_is_log=True, out=o,
-                    final_state=sf, workspace=ws)
+        kda.prefill_logits(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["z"], dev_in["A_log"], w.g_min,
+                           dev_in["beta"], None, out=o, final_state=sf, workspace=ws)
         o_host.copy_(o, non_blocking=True)
         sf_host.copy_(sf, non_blocking=True)
 
@@ -332,22 +328,18 @@ def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
     A_dec = prm["A_log"].to(dev)
     n_sets = 4
     sets = [{n: x.to(dev) for n, x in W.make_decode_step(dw, s).items()} for s in range(n_sets)]
-    a_dec = torch.empty(dw.B, dw.H, dw.K, device=dev)
     o_dec = torch.empty(dw.B, dw.H, dw.V, device=dev, dtype=torch.bfloat16)
     it = {"i": 0}
 
-    def dgate_fn():
-        s = sets[it["i"] % n_sets]
-        kda.bounded_decay(s["z"], A_dec, dw.g_min, out=a_dec)
-
+    # One call per step: the decode kernel reads the decay logits and evaluates the gate itself.
     def dstep_fn():
         s = sets[it["i"] % n_sets]
-        kda.decode_step(s["q"], s["k"], s["v"], a_dec, s["beta"], state, out=o_dec)
+        kda.decode_step_logits(s["q"], s["k"], s["v"], s["z"], A_dec, dw.g_min, s["beta"], state, out=o_dec)
         it["i"] += 1
 
     dsteps = max(args.steps, 20)
     dsampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
-    d_total, (dg_ms, dk_ms) = timed_loop([dgate_fn, dstep_fn], dsteps, args.warmup, world, stream, dsampler)
+    d_total, (dk_ms,) = timed_loop([dstep_fn], dsteps, args.warmup, world, stream, dsampler)
     sbytes = decode_state_bytes(dw.B, dw.H, dw.K, dw.V)
     d_bps, d_total = weak_scaling_value(sbytes * dsteps, d_total, world)
     d_ms = d_total / dsteps
@@ -355,10 +347,10 @@ def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
     d_achieved = dbytes / (dk_ms / 1e3) / 1e9
     res = {
         "workload": dw.name, "value": d_bps / 1e9, "unit": "GB/s (state)",
-        "steps_per_s": 1e3 / d_ms, "ms_per_step": d_ms, "steps": dsteps, "gpu_launches": 2 * dsteps,
-        "kernels_ms": {"bounded_decay": dg_ms, "decode_step": dk_ms},
+        "steps_per_s": 1e3 / d_ms, "ms_per_step": d_ms, "steps": dsteps, "gpu_launches": dsteps,
+        "kernels_ms": {"decode_step_logits": dk_ms},
         "roofline": {"bound": "hbm", "achieved": d_achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": d_achieved / hbm, "traffic": None, "kernel": "kda_decode_step",
+                     "frac": d_achieved / hbm, "traffic": None, "kernel": "kda_decode_step_logits",
                      "bytes_per_launch": dbytes, "ms_per_launch": dk_ms, "peak_source": f"{peak_src} hbm_gbs"},
         "clocks": dsampler.summary() if dsampler is not None else None,
     }
@@ -374,8 +366,8 @@ def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
         s = hostd[it["i"] % n_sets]
         for n, x in s.items():
             devd[n].copy_(x, non_blocking=True)
-        kda.bounded_decay(devd["z"], A_dec, dw.g_min, out=a_dec)
-        kda.decode_step(devd["q"], devd["k"], devd["v"], a_dec, devd["beta"], state, out=o_dec)
+        kda.decode_step_logits(devd["q"], devd["k"], devd["v"], devd["z"], A_dec, dw.g_min, devd["beta"], state,
+                               out=o_dec)
         o_dec_host.copy_(o_dec, non_blocking=True)
         it["i"] += 1
 
@@ -419,8 +411,8 @@ def gpu_arm(args, rank, world, local):
         "dtype": "bf16",
         "data": "synthetic (seeded; no dataset)",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "K": w.K, "V": w.V, "g_min": w.g_min,
-                   "z_std": w.z_std, "initial_state": "zeros", "step": "bounded_decay (log-decay out) + prefill (log-decay in)",
-                   "l2": "inputs larger than L2 (q/k/v/z/alpha ~ 0.9 GB); no flush",
+                   "z_std": w.z_std, "initial_state": "zeros", "step": "prefill from decay logits z (bounded gate evaluated inside the scan kernels)",
+                   "l2": "inputs larger than L2 (q/k/v/z ~ 0.5 GB, workspace 0.4 GB); no flush",
                    "parallelism": f"replica per GPU x{world}"},
         "roofline": pre["roofline"],
         "kernels_ms": pre["kernels_ms"],

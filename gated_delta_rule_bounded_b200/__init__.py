@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["bounded_decay", "prefill", "prefill_noalloc", "decode_step", "prefill_workspace_bytes", "device_status", "KDAError",
+__all__ = ["bounded_decay", "prefill", "prefill_logits", "prefill_noalloc", "decode_step", "decode_step_logits", "prefill_workspace_bytes", "device_status", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -73,8 +73,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_prefill_noalloc.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64,
                                         i64, i64, i64, i64, i64, lp, vp, vp]
     lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, i64, i64, i64, i64, lp, vp, vp]
+    lib.kda_prefill_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, vp, vp, vp, i64,
+                                       i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
+    lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, vp, i64, i64, i64, i64, lp,
+                                           vp, vp]
     for fn in ("kda_bounded_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
-               "kda_decode_step"):
+               "kda_decode_step", "kda_prefill_logits", "kda_decode_step_logits"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_last_error.argtypes = []
@@ -166,22 +170,8 @@ def prefill_workspace_bytes(B: int, T: int, H: int, K: int, V: int, n_seq: int =
     return int(n.value)
 
 
-def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
-            initial_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
-            gate_is_log: bool = False, output_final_state: bool = True,
-            out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
-            workspace: Optional[torch.Tensor] = None,
-            use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Scan whole sequences. Returns ``(o [B,T,H,V], final_state [N,H,K,V] fp32 or None)``.
-
-    q, k ``[B,T,H,K]`` and v ``[B,T,H,V]`` share a dtype (bf16 or fp32); gate ``[B,T,H,K]`` fp32
-    holds alpha (or g = log alpha when ``gate_is_log``); beta ``[B,T,H]`` fp32. With ``cu_seqlens``
-    (int32 ``[N+1]`` on the device) B must be 1 and the states have N rows.
-    ``final_state`` may be ``initial_state`` itself to resume in place. ``workspace`` (uint8, on the
-    device) enables the two-kernel path when large enough; when it is None and ``use_workspace`` is
-    true, one of ``prefill_workspace_bytes`` bytes is allocated; ``use_workspace=False`` runs the
-    single fused kernel.
-    """
+def _prefill(q, k, v, gate, beta, initial_state, cu_seqlens, gate_is_log, output_final_state, out, final_state,
+             workspace, use_workspace, logits=None, gate_name="gate"):
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta")):
         _cuda(t, n)
     if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
@@ -189,7 +179,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share one dtype")
     if gate.shape != q.shape or gate.dtype != torch.float32:
-        raise ValueError("gate must be fp32 [B,T,H,K]")
+        raise ValueError(f"{gate_name} must be fp32 [B,T,H,K]")
     if beta.shape != q.shape[:3] or beta.dtype != torch.float32:
         raise ValueError("beta must be fp32 [B,T,H]")
     B, T, H, K = q.shape
@@ -229,12 +219,56 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     layout = Layout(_strides4(q), _strides4(k), _strides4(v), _strides4(gate), _strides3(beta), _strides4(out))
     lib = load_library()
-    _check("kda_prefill", lib.kda_prefill(
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
-        KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), s0_ptr, sf_ptr,
-        cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
-        _stream(dev)))
+    if logits is None:
+        _check("kda_prefill", lib.kda_prefill(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+            KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), s0_ptr, sf_ptr,
+            cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
+            _stream(dev)))
+    else:
+        A_log, g_min = logits
+        _check("kda_prefill_logits", lib.kda_prefill_logits(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+            A_log.data_ptr(), g_min, beta.data_ptr(), s0_ptr, sf_ptr,
+            cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
+            _stream(dev)))
     return out, final_state
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
+            initial_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
+            gate_is_log: bool = False, output_final_state: bool = True,
+            out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None,
+            use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Scan whole sequences. Returns ``(o [B,T,H,V], final_state [N,H,K,V] fp32 or None)``.
+
+    q, k ``[B,T,H,K]`` and v ``[B,T,H,V]`` share a dtype (bf16 or fp32); gate ``[B,T,H,K]`` fp32
+    holds alpha (or g = log alpha when ``gate_is_log``); beta ``[B,T,H]`` fp32. With ``cu_seqlens``
+    (int32 ``[N+1]`` on the device) B must be 1 and the states have N rows.
+    ``final_state`` may be ``initial_state`` itself to resume in place. ``workspace`` (uint8, on the
+    device) enables the two-kernel path when large enough; when it is None and ``use_workspace`` is
+    true, one of ``prefill_workspace_bytes`` bytes is allocated; ``use_workspace=False`` runs the
+    single fused kernel.
+    """
+    return _prefill(q, k, v, gate, beta, initial_state, cu_seqlens, gate_is_log, output_final_state, out,
+                    final_state, workspace, use_workspace)
+
+
+def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
+                   g_min: float, beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
+                   cu_seqlens: Optional[torch.Tensor] = None, *, output_final_state: bool = True,
+                   out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``prefill`` fed with the decay logits ``z [B,T,H,K]`` (fp32) instead of alpha: the scan kernels
+    evaluate ``g = g_min * sigmoid(exp(A_log[h]) * z)`` themselves (``kda_prefill_logits``).
+    ``A_log [H]`` fp32 on the device; ``g_min < 0``. Other arguments as in ``prefill``."""
+    _cuda(A_log, "A_log")
+    if A_log.shape != (q.shape[2],) or A_log.dtype != torch.float32:
+        raise ValueError("A_log must be fp32 [H]")
+    return _prefill(q, k, v, z, beta, initial_state, cu_seqlens, False, output_final_state, out, final_state,
+                    workspace, use_workspace, logits=(A_log.contiguous(), float(g_min)), gate_name="z")
 
 
 NOALLOC_SCRATCH_BYTES = 128 << 20  # the library's static scratch (KDA_NOALLOC_SCRATCH_BYTES)
@@ -290,10 +324,11 @@ def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: tor
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
                 state: torch.Tensor, *, gate_is_log: bool = False,
-                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                out: Optional[torch.Tensor] = None, logits=None) -> torch.Tensor:
     """One token against the kept ``state [B,H,K,V]`` (fp32, updated in place). Returns ``o [B,H,V]``.
 
     q, k ``[B,H,K]`` (or ``[B,1,H,K]``), v ``[B,H,V]``, gate ``[B,H,K]`` fp32, beta ``[B,H]`` fp32.
+    ``logits=(A_log, g_min)`` is the internal form of ``decode_step_logits``.
     """
     q, k, v, gate = (x[:, 0] if x.dim() == 4 else x for x in (q, k, v, gate))
     if beta.dim() == 3:
@@ -316,11 +351,29 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
     s3 = lambda x: Strides(x.stride(0), 0, x.stride(1))  # noqa: E731
     layout = Layout(s3(q), s3(k), s3(v), s3(gate), Strides(beta.stride(0), 0, beta.stride(1)), s3(out))
     lib = load_library()
-    _check("kda_decode_step", lib.kda_decode_step(
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
-        KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), state.data_ptr(),
-        B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
+    if logits is None:
+        _check("kda_decode_step", lib.kda_decode_step(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+            KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), state.data_ptr(),
+            B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
+    else:
+        A_log, g_min = logits
+        _check("kda_decode_step_logits", lib.kda_decode_step_logits(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+            A_log.data_ptr(), g_min, beta.data_ptr(), state.data_ptr(),
+            B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
     return out
+
+
+def decode_step_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
+                       g_min: float, beta: torch.Tensor, state: torch.Tensor, *,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``decode_step`` fed with the decay logits ``z [B,H,K]`` (fp32): the step evaluates the bounded gate
+    itself (``kda_decode_step_logits``). ``A_log [H]`` fp32 on the device; ``g_min < 0``."""
+    _cuda(A_log, "A_log")
+    if A_log.shape != (q.shape[-2],) or A_log.dtype != torch.float32:
+        raise ValueError("A_log must be fp32 [H]")
+    return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min)))
 
 
 def device_status(reset: bool = True) -> bool:

@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
   const int vt = blk % n_vt;
   blk /= n_vt;
   const int h = blk % p.H;
+  const float gsc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int n = blk / p.H;
 
   int64_t t0 = 0, t1 = p.T, brow = n;
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
     // ---- decay pass: block-local cumulative decay, scaled operand tiles, decay vectors -------------
     {
       float2 al[16];
-      decay_step1(sm, LY, pf, nv, da, c0, p.gate_log != 0, al);
+      decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
       __syncthreads();
       decay_step2(sm, LY, pf, da, c0, al);
     }

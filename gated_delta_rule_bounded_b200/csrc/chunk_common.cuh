@@ -6,6 +6,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "gate_math.cuh"
 #include "kda_internal.h"
 
 namespace kda {
@@ -264,8 +265,9 @@ __device__ __forceinline__ void load_vb(const ChunkCtx& x, uint32_t vbase, uint3
 // columns, with the per-pair decay factor D_ab applied to the row operand. The warp takes tiles
 // first, first + stride, ... (nt of them) and runs their k-loops interleaved so the MMA chains
 // overlap. A_qk is stored as a bf16 K-major operand (diagonal blocks masked to i <= t); A_kk as
-// fp32 [64][64] with beta_t applied and diagonal blocks masked to i < t.
-template <int NTMAX>
+// fp32 [64][64] with beta_t applied and diagonal blocks masked to i < t. With QK_T, A_qk is stored
+// transposed ([i][t], the MN-major form of the same operand).
+template <int NTMAX, bool QK_T = false>
 __device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const IntraLayout& L, int off_rows, int first,
                                         int stride, int nt, int lane, int g, int tq, const float* beta_s,
                                         bool is_qk) {
@@ -324,7 +326,12 @@ __device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const In
             v0 = (i0 <= t) ? v0 : 0.f;
             v1 = (i0 + 1 <= t) ? v1 : 0.f;
           }
-          *reinterpret_cast<uint32_t*>(sm + L.aqk + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
+          if (QK_T) {
+            *reinterpret_cast<__nv_bfloat16*>(sm + L.aqk + sw_e(i0, t, 8192)) = __float2bfloat16_rn(v0);
+            *reinterpret_cast<__nv_bfloat16*>(sm + L.aqk + sw_e(i0 + 1, t, 8192)) = __float2bfloat16_rn(v1);
+          } else {
+            *reinterpret_cast<uint32_t*>(sm + L.aqk + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
+          }
         } else {
           const float bt = beta_s[t];
           v0 = (a > b || i0 < t) ? v0 * bt : 0.f;
@@ -336,19 +343,25 @@ __device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const In
 }
 
 
+// The log2-decay of one channel from the gate value x in gate mode `mode` (alpha, g = log alpha, or
+// the decay logits z with sc = e^{A_h}).
+__device__ __forceinline__ float log2_decay(int mode, float x, float sc, float g_min) {
+  return mode == GATE_LOGITS ? bounded_log_decay(sc, x, g_min) * LOG2E : (mode == 1 ? x * LOG2E : lg2(x));
+}
+
 // Decay pass, step 1: the per-token log2-decay of channels (c0, c0+1) over the 16 tokens of block
 // da (clamped at G2_MIN; 0 past the end of the sequence), their retention factors, and the block
 // sum, published to VEC_TOT.
 __device__ __forceinline__ void decay_step1(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int nv,
-                                            int da, int c0, bool gate_log, float2 (&al)[16]) {
+                                            int da, int c0, int mode, float sc, float g_min, float2 (&al)[16]) {
   float* vec = reinterpret_cast<float*>(sm + L.vec);
   float2 run = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float2 l = make_float2(0.f, 0.f);
     if (16 * da + i < nv) {
-      l.x = fmaxf(gate_log ? pf.g[i].x * LOG2E : lg2(pf.g[i].x), G2_MIN);
-      l.y = fmaxf(gate_log ? pf.g[i].y * LOG2E : lg2(pf.g[i].y), G2_MIN);
+      l.x = fmaxf(log2_decay(mode, pf.g[i].x, sc, g_min), G2_MIN);
+      l.y = fmaxf(log2_decay(mode, pf.g[i].y, sc, g_min), G2_MIN);
     }
     run.x += l.x;
     run.y += l.y;
@@ -408,14 +421,16 @@ __device__ __forceinline__ void decay_step2(unsigned char* sm, const IntraLayout
   }
 }
 
-// Zeroes the six 16x16 blocks above the diagonal of a [64][64] bf16 K-major tile, using the
-// `count` threads with index `idx` in [0, count).
+// Zeroes the six 16x16 blocks above the diagonal of a [64][64] bf16 K-major tile (below it when
+// TRANSPOSED), using the `count` threads with index `idx` in [0, count).
+template <bool TRANSPOSED = false>
 __device__ __forceinline__ void zero_upper_blocks(unsigned char* sm, int off, int idx, int count) {
   for (int e = idx; e < 6 * 64; e += count) {
     const int pr = e >> 6, r = (e >> 2) & 15, q4 = e & 3;  // block pair, row, group of 4 columns
     const int a = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
     const int b = pr < 3 ? pr + 1 : (pr < 5 ? pr - 1 : 3);
-    *reinterpret_cast<uint2*>(sm + off + sw_e(16 * a + r, 16 * b + 4 * q4, 8192)) = make_uint2(0u, 0u);
+    const int ra = TRANSPOSED ? b : a, cb = TRANSPOSED ? a : b;
+    *reinterpret_cast<uint2*>(sm + off + sw_e(16 * ra + r, 16 * cb + 4 * q4, 8192)) = make_uint2(0u, 0u);
   }
 }
 
@@ -484,7 +499,9 @@ __device__ __forceinline__ void inverse_warps0to3(unsigned char* sm, uint32_t sb
 }
 
 // The state-independent phases after the decay pass: A_kk on all warps; then the inverse on warps
-// 0-3 while warps 4-7 form A_qk (and zero its upper blocks). Ends with a CTA-wide barrier.
+// 0-3 while warps 4-7 form A_qk (and zero its upper blocks; transposed with QK_T). Ends with a
+// CTA-wide barrier.
+template <bool QK_T = false>
 __device__ __forceinline__ void intra_phases(unsigned char* sm, uint32_t sb, const IntraLayout& L, const float* beta_s,
                                              int tid, int warp, int lane, int g, int tq) {
   a_tiles<2>(sm, sb, L, L.ke, warp, 8, warp < 2 ? 2 : 1, lane, g, tq, beta_s, /*is_qk=*/false);
@@ -492,8 +509,8 @@ __device__ __forceinline__ void intra_phases(unsigned char* sm, uint32_t sb, con
   if (warp < 4) {
     inverse_warps0to3(sm, sb, L, beta_s, tid, warp, lane, g, tq);
   } else {
-    a_tiles<3>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
-    zero_upper_blocks(sm, L.aqk, tid - 128, 128);  // the MMAs read whole rows of A_qk
+    a_tiles<3, QK_T>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
+    zero_upper_blocks<QK_T>(sm, L.aqk, tid - 128, 128);  // the MMAs read whole rows of A_qk
   }
   __syncthreads();
 }

@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int h = blockIdx.y;
+  const float gsc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int64_t slot = blockIdx.x;
   int n, j;
   if (!locate_slot(p, slot, n, j)) return;  // uniform across the CTA
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     load_qkg(x, tc0, nv, c0, da, pf);
     if (tid < C) beta_s[tid] = tid < nv ? __ldg(x.beta + x.boff + (tc0 + tid) * x.bst) : 0.f;
     float2 al[16];
-    decay_step1(sm, LY, pf, nv, da, c0, p.gate_log != 0, al);
+    decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
     __syncthreads();
     p_decay_step2(sm, pf, da, c0, al, blk);
   }

@@ -16,6 +16,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "gate_math.cuh"
 #include "kda_internal.h"
 
 namespace kda {
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
 
   for (int i = 0; i < n_my; ++i) {
     const int head = blockIdx.x + i * gridDim.x;
+    const float sc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + head % p.H)) : 0.f;  // e^{A_h}
     const int s = i % NSTAGE;
     unsigned char* st = sm + s * L::BYTES;
     const float beta = beta_next;
@@ -139,7 +141,12 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
     const TIn* qs = reinterpret_cast<const TIn*>(st + L::Q);
     const TIn* ks = reinterpret_cast<const TIn*>(st + L::K);
     const TIn* vs = reinterpret_cast<const TIn*>(st + L::V);
-    const float* as = reinterpret_cast<const float*>(st + L::A);
+    float* as = reinterpret_cast<float*>(st + L::A);
+    // The staged gate row becomes alpha in place, once per head (each row is read by many threads).
+    if (p.gate_mode != KDA_GATE_ALPHA) {
+      for (int c = tid; c < DK; c += blockDim.x) as[c] = gate_alpha(p.gate_mode, as[c], sc, p.g_min);
+      __syncthreads();
+    }
     float* S = reinterpret_cast<float*>(st + L::STATE);
 
     float4 x[ROWS];
@@ -148,7 +155,7 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
       const int row = row0 + r;
-      const float a = p.gate_log ? expf(as[row]) : as[row], kk = to_f32(ks[row]), qq = to_f32(qs[row]);
+      const float a = as[row], kk = to_f32(ks[row]), qq = to_f32(qs[row]);
       x[r] = *reinterpret_cast<const float4*>(S + row * DV + col0);
       x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
       pa.x = fmaf(kk, x[r].x, pa.x); pa.y = fmaf(kk, x[r].y, pa.y);

@@ -4,16 +4,10 @@
 // consecutive channels (16-byte fp32 or 8-byte bf16 accesses); the grid is a
 // multiple of the SM count and strides over all rows.
 #include "common.cuh"
+#include "gate_math.cuh"
 #include "kda_internal.h"
 
 namespace kda {
-
-__device__ __forceinline__ float gate_sigmoid(float x) {
-  // Evaluated without overflow for either sign.
-  if (x >= 0.f) return 1.f / (1.f + expf(-x));
-  float e = expf(x);
-  return e / (1.f + e);
-}
 
 // One warp per (b, t, h) row: the row's coordinates are decomposed once (32-bit
 // arithmetic), A_log is read once, and the lanes stride over its K/4 channel
@@ -51,10 +45,10 @@ __global__ void __launch_bounds__(256) bounded_decay_kernel(GateParams p) {
         if (r0 + i >= rows) break;
         const float sc = expf(scale[i]);
         float4 g;
-        g.x = p.g_min * gate_sigmoid(sc * z[i].x);
-        g.y = p.g_min * gate_sigmoid(sc * z[i].y);
-        g.z = p.g_min * gate_sigmoid(sc * z[i].z);
-        g.w = p.g_min * gate_sigmoid(sc * z[i].w);
+        g.x = bounded_log_decay(sc, z[i].x, p.g_min);
+        g.y = bounded_log_decay(sc, z[i].y, p.g_min);
+        g.z = bounded_log_decay(sc, z[i].z, p.g_min);
+        g.w = bounded_log_decay(sc, z[i].w, p.g_min);
         if (!p.out_log) {
           g.x = expf(g.x);
           g.y = expf(g.y);

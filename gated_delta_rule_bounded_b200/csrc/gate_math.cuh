@@ -1,0 +1,30 @@
+// gate_math.cuh -- the bounded decay gate of "Kimi K3: Bounded Decay and Delta Memory" (Formula and
+// conventions, eq. 5), g = g_min * sigmoid(e^{A_h} z), as one device function shared by the gate
+// kernel and by every scan kernel that reads decay logits directly. Sharing it makes a scan fed
+// with logits bit-identical to the gate kernel followed by a scan fed with its output.
+#pragma once
+
+#include "kda_internal.h"
+
+namespace kda {
+
+// sigmoid(x) = 1 / (1 + e^-x), branch-free and without overflow for either sign: with
+// t = e^-|x| = 2^(-|x| log2 e) in [0, 1], sigmoid is 1 / (1 + t) for x >= 0 and t / (1 + t) for
+// x < 0. The power of two and the reciprocal are the hardware approximations (ex2.approx and
+// rcp.approx, about two and one ulp); 1 + t lies in [1, 2], where rcp.approx is well inside range.
+__device__ __forceinline__ float gate_sigmoid(float x) {
+  float t, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(-fabsf(x) * 1.4426950408889634f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + t));
+  return x >= 0.f ? r : t * r;
+}
+
+// g = g_min * sigmoid(sc * z) with sc = e^{A_h} (computed once per head as expf(A_log[h])).
+__device__ __forceinline__ float bounded_log_decay(float sc, float z, float g_min) { return g_min * gate_sigmoid(sc * z); }
+
+// The retention factor alpha of one channel for a scan in gate mode `mode`.
+__device__ __forceinline__ float gate_alpha(int mode, float x, float sc, float g_min) {
+  return mode == GATE_LOGITS ? expf(bounded_log_decay(sc, x, g_min)) : (mode == 1 ? expf(x) : x);
+}
+
+}  // namespace kda

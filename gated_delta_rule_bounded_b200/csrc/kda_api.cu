@@ -149,10 +149,26 @@ int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int6
   return ok();
 }
 
-static int check_scan_common(const char* fn, kda_dtype dtype, int gate_kind, int64_t H, int64_t K, int64_t V) {
+// The decay input of a scan: alpha, g = log alpha, or the logits z with A_log and g_min.
+struct GateSpec {
+  const float* data;
+  int mode;
+  const float* A_log;
+  float g_min;
+};
+
+static int check_gate(const char* fn, const GateSpec& gs) {
+  if (gs.mode != KDA_GATE_ALPHA && gs.mode != KDA_GATE_LOG && gs.mode != kda::GATE_LOGITS)
+    return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, gs.mode);
+  if (gs.mode == kda::GATE_LOGITS && (!std::isfinite(gs.g_min) || !(gs.g_min < 0.f)))
+    return fail(KDA_ERR_INVALID_ARG, "%s: g_min must be finite and < 0 (got %g)", fn, (double)gs.g_min);
+  return KDA_OK;
+}
+
+static int check_scan_common(const char* fn, kda_dtype dtype, const GateSpec& gs, int64_t H, int64_t K, int64_t V) {
   if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
-  if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
-    return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, gate_kind);
+  int rc = check_gate(fn, gs);
+  if (rc != KDA_OK) return rc;
   if (H <= 0) return fail(KDA_ERR_INVALID_ARG, "%s: H must be positive", fn);
   if (!dim_supported(K) || !dim_supported(V))
     return fail(KDA_ERR_UNSUPPORTED, "%s: K and V must be multiples of 16 in [16,256] (K=%lld, V=%lld)", fn,
@@ -160,16 +176,16 @@ static int check_scan_common(const char* fn, kda_dtype dtype, int gate_kind, int
   return KDA_OK;
 }
 
-int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
-                const float* gate, kda_gate_kind gate_kind, const float* beta,
-                const float* initial_state, float* final_state,
-                const int32_t* cu_seqlens, int64_t n_seq,
-                int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
-                const kda_layout* layout, void* o,
-                void* workspace, size_t workspace_bytes, kda_stream_t stream) {
-  const char* fn = "kda_prefill";
+static int prefill_impl(const char* fn, const void* q, const void* k, const void* v, kda_dtype dtype,
+                        const GateSpec& gs, const float* beta,
+                        const float* initial_state, float* final_state,
+                        const int32_t* cu_seqlens, int64_t n_seq,
+                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                        const kda_layout* layout, void* o,
+                        void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const float* gate = gs.data;
   if (B < 0 || T < 0 || n_seq < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
-  int rc = check_scan_common(fn, dtype, gate_kind, H, K, V);
+  int rc = check_scan_common(fn, dtype, gs, H, K, V);
   if (rc != KDA_OK) return rc;
   int64_t N = B;
   if (cu_seqlens) {
@@ -193,7 +209,8 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
     }
     return ok();
   }
-  if (!q || !k || !v || !gate || !beta || !o) return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (!q || !k || !v || !gate || !beta || !o || (gs.mode == kda::GATE_LOGITS && !gs.A_log))
+    return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
   kda_layout L;
   if (layout) {
     L = *layout;
@@ -239,7 +256,9 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
   p.K = (int)K;
   p.V = (int)V;
   p.N = (int)N;
-  p.gate_log = gate_kind == KDA_GATE_LOG;
+  p.gate_mode = gs.mode;
+  p.A_log = gs.A_log;
+  p.g_min = gs.g_min;
 
   cudaError_t e;
   if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype)) {
@@ -252,16 +271,42 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
   return ok();
 }
 
-int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype,
-                    const float* gate, kda_gate_kind gate_kind, const float* beta,
-                    float* state, int64_t B, int64_t H, int64_t K, int64_t V,
-                    const kda_layout* layout, void* o, kda_stream_t stream) {
-  const char* fn = "kda_decode_step";
+int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
+                const float* gate, kda_gate_kind gate_kind, const float* beta,
+                const float* initial_state, float* final_state,
+                const int32_t* cu_seqlens, int64_t n_seq,
+                int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                const kda_layout* layout, void* o,
+                void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
+    return fail(KDA_ERR_INVALID_ARG, "kda_prefill: unknown gate kind %d", (int)gate_kind);
+  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f};
+  return prefill_impl("kda_prefill", q, k, v, dtype, gs, beta, initial_state, final_state, cu_seqlens, n_seq, B, T, H,
+                      K, V, layout, o, workspace, workspace_bytes, stream);
+}
+
+int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
+                       const float* logits, const float* A_log, float g_min, const float* beta,
+                       const float* initial_state, float* final_state,
+                       const int32_t* cu_seqlens, int64_t n_seq,
+                       int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                       const kda_layout* layout, void* o,
+                       void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min};
+  return prefill_impl("kda_prefill_logits", q, k, v, dtype, gs, beta, initial_state, final_state, cu_seqlens, n_seq, B,
+                      T, H, K, V, layout, o, workspace, workspace_bytes, stream);
+}
+
+static int decode_impl(const char* fn, const void* q, const void* k, const void* v, kda_dtype dtype,
+                       const GateSpec& gs, const float* beta,
+                       float* state, int64_t B, int64_t H, int64_t K, int64_t V,
+                       const kda_layout* layout, void* o, kda_stream_t stream) {
+  const float* gate = gs.data;
   if (B < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
-  int rc = check_scan_common(fn, dtype, gate_kind, H, K, V);
+  int rc = check_scan_common(fn, dtype, gs, H, K, V);
   if (rc != KDA_OK) return rc;
   if (B == 0) return ok();
-  if (!q || !k || !v || !gate || !beta || !state || !o)
+  if (!q || !k || !v || !gate || !beta || !state || !o || (gs.mode == kda::GATE_LOGITS && !gs.A_log))
     return fail(KDA_ERR_INVALID_ARG, "%s: null pointer", fn);
   kda_layout L;
   if (layout) {
@@ -307,11 +352,31 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
   p.K = (int)K;
   p.V = (int)V;
   p.N = (int)B;
-  p.gate_log = gate_kind == KDA_GATE_LOG;
+  p.gate_mode = gs.mode;
+  p.A_log = gs.A_log;
+  p.g_min = gs.g_min;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kda::decode_bulk_supported(p) ? kda::launch_decode_bulk(p, dtype, s) : kda::launch_recurrent(p, dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
   return ok();
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype,
+                    const float* gate, kda_gate_kind gate_kind, const float* beta,
+                    float* state, int64_t B, int64_t H, int64_t K, int64_t V,
+                    const kda_layout* layout, void* o, kda_stream_t stream) {
+  if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
+    return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: unknown gate kind %d", (int)gate_kind);
+  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f};
+  return decode_impl("kda_decode_step", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
+}
+
+int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
+                           const float* logits, const float* A_log, float g_min, const float* beta,
+                           float* state, int64_t B, int64_t H, int64_t K, int64_t V,
+                           const kda_layout* layout, void* o, kda_stream_t stream) {
+  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min};
+  return decode_impl("kda_decode_step_logits", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 
 }  // extern "C"

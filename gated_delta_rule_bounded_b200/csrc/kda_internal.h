@@ -8,13 +8,17 @@
 
 namespace kda {
 
+// Internal gate mode of a scan, next to KDA_GATE_ALPHA (0) and KDA_GATE_LOG (1): the gate tensor
+// holds the decay logits z, and ScanParams::A_log / g_min complete the bounded gate.
+constexpr int GATE_LOGITS = 2;
+
 // Everything a scan kernel needs, passed by value. Strides are in elements, for
 // the B, T and H dimensions of each token tensor; the innermost dim is contiguous.
 struct ScanParams {
   const void* q;
   const void* k;
   const void* v;
-  const float* gate;  // alpha, or g = log(alpha) when gate_log != 0
+  const float* gate;  // alpha, g = log(alpha), or the logits z, per gate_mode
   const float* beta;
   const float* s0;    // [N,H,K,V] or nullptr (zeros)
   float* sf;          // [N,H,K,V] or nullptr (not written)
@@ -23,7 +27,9 @@ struct ScanParams {
   int64_t qs[3], ks[3], vs[3], gs[3], bs[3], os[3];
   int64_t T;
   int B, H, K, V, N;
-  int gate_log;
+  int gate_mode;        // KDA_GATE_ALPHA, KDA_GATE_LOG, or GATE_LOGITS (gate holds decay logits z)
+  const float* A_log;   // [H], GATE_LOGITS only
+  float g_min;          // GATE_LOGITS only
 };
 
 struct GateParams {

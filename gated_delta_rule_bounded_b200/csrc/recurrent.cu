@@ -19,6 +19,7 @@
 // same kernel serves the prefill of fp32 inputs (any supported K, V) with the
 // state kept in registers across the whole sequence.
 #include "common.cuh"
+#include "gate_math.cuh"
 #include "kda_internal.h"
 
 namespace kda {
@@ -47,6 +48,7 @@ recurrent_kernel(ScanParams p) {
   const int vt = blk % n_vt;
   blk /= n_vt;
   const int h = blk % p.H;
+  const float sc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int n = blk / p.H;
   const int K = p.K, V = p.V;
   const int rpt = kExact ? RPT : K / kRowGroups;
@@ -96,8 +98,7 @@ recurrent_kernel(ScanParams p) {
     const int64_t go = brow * p.gs[0] + t * p.gs[1] + h * p.gs[2];
     const int64_t vo = brow * p.vs[0] + t * p.vs[1] + h * p.vs[2];
     for (int i = tid; i < K; i += NT) {
-      float g = __ldg(p.gate + go + i);
-      s_a[i] = p.gate_log ? expf(g) : g;
+      s_a[i] = gate_alpha(p.gate_mode, __ldg(p.gate + go + i), sc, p.g_min);
       s_k[i] = to_f32(kb[ko + i]);
       s_q[i] = to_f32(qb[qo + i]);
     }

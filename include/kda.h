@@ -17,6 +17,9 @@
  *   kda_decode_step    the same recurrence for one new token against a kept
  *                      state that is updated in place ("Kept memory": the
  *                      recurrent form used for one new position with a cache).
+ *   kda_prefill_logits, kda_decode_step_logits
+ *                      the same two scans fed with the decay logits z: eq. 5
+ *                      is evaluated inside the scan kernels.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -149,6 +152,32 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
                 void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * kda_prefill_logits: kda_prefill with the bounded gate applied inside the
+ * scan ("Kimi K3: Bounded Decay and Delta Memory", Formula and conventions,
+ * eq. 5 feeding eq. 1): the decay input is the logits z instead of alpha or g,
+ *   g = g_min * sigmoid(exp(A_log[h]) * z),  alpha = exp(g),
+ * evaluated per element while the scan reads it, so g never travels through
+ * device memory.
+ *
+ * logits   [B,T,H,K] fp32, strides in layout->gate (the slot kda_prefill
+ *          uses for alpha / g).
+ * A_log    [H] fp32 device pointer; g_min finite and < 0
+ *          (else KDA_ERR_INVALID_ARG).
+ * Every other argument, layout, result, workspace rule and error is
+ * kda_prefill's. The result is bit-identical to kda_bounded_decay with
+ * out_kind KDA_GATE_LOG (bf16 inputs) or KDA_GATE_ALPHA (fp32 inputs)
+ * followed by kda_prefill on its output: both evaluate the gate with the same
+ * device code.
+ * ------------------------------------------------------------------------- */
+int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
+                       const float* logits, const float* A_log, float g_min, const float* beta,
+                       const float* initial_state, float* final_state,
+                       const int32_t* cu_seqlens, int64_t n_seq,
+                       int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                       const kda_layout* layout, void* o,
+                       void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * kda_prefill_noalloc: kda_prefill for callers that cannot allocate device
  * memory. The pages have no counterpart; it is a library convenience.
  *
@@ -198,6 +227,18 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
                     const float* gate, kda_gate_kind gate_kind, const float* beta,
                     float* state, int64_t B, int64_t H, int64_t K, int64_t V,
                     const kda_layout* layout, void* o, kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * kda_decode_step_logits: kda_decode_step with the bounded gate (eq. 5)
+ * applied inside the step: logits [B,H,K] fp32 (strides in layout->gate),
+ * A_log [H] fp32, g_min finite and < 0. alpha = exp(g_min * sigmoid(
+ * exp(A_log[h]) * z)). Everything else is kda_decode_step's; the result is
+ * bit-identical to kda_bounded_decay (alpha out) followed by kda_decode_step.
+ * ------------------------------------------------------------------------- */
+int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
+                           const float* logits, const float* A_log, float g_min, const float* beta,
+                           float* state, int64_t B, int64_t H, int64_t K, int64_t V,
+                           const kda_layout* layout, void* o, kda_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * kda_device_status: device-side failure flags, for callers that check them

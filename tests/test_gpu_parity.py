@@ -405,3 +405,57 @@ def test_long_kv_workload_split_resume_sampled(kda):
     check(sf[:, heads], rs, "bf16", "final_state")
     check(torch.cat([o1, o2], 1)[:, :, heads], ro, "bf16", "o (split)")
     check(s2[:, heads], rs, "bf16", "final_state (split)")
+
+
+# ---------------------------------------------------------------------------------------------
+# Gate inside the scan (kda_prefill_logits / kda_decode_step_logits)
+# ---------------------------------------------------------------------------------------------
+# Both evaluate eq. 5 with the gate kernel's own device function, so a scan fed with the logits
+# must equal, bit for bit, the gate kernel followed by the scan on its output (log-decay for the
+# chunked bf16 kernels, which take log2 of it; alpha for the token-by-token kernel).
+
+@pytest.mark.parametrize("dtype,use_workspace,cu", [("bf16", True, False), ("bf16", False, False),
+                                                    ("bf16", True, True), ("f32", True, False)],
+                         ids=["bf16-split", "bf16-fused", "bf16-varlen", "f32"])
+def test_prefill_logits_equals_gate_then_scan(kda, dtype, use_workspace, cu):
+    B, T, H = (1, 333, 3) if cu else (2, 200, 3)
+    d = W.random_scan_case(B, T, H, 128, 128, seed=41, dtype=dtype, z_std=2.0, init_std=0.1)
+    if cu:
+        lens = [100, 0, 64, 169]
+        d["cu_seqlens"] = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+        d["initial_state"] = torch.randn(len(lens), H, 128, 128, generator=torch.Generator().manual_seed(2)) * 0.1
+    g = to_dev(d)
+    use_log = dtype == "bf16"
+    gate = kda.bounded_decay(g["z"], g["A_log"], g["g_min"], log_decay=use_log)
+    o_ref, s_ref = kda.prefill(g["q"], g["k"], g["v"], gate, g["beta"], g["initial_state"], g["cu_seqlens"],
+                               gate_is_log=use_log, use_workspace=use_workspace)
+    o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"],
+                               g["initial_state"], g["cu_seqlens"], use_workspace=use_workspace)
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    assert torch.equal(o, o_ref) and torch.equal(sf, s_ref)
+    ro, rs = oracle_pipeline(d)
+    check(o, ro, dtype, "o")
+    check(sf, rs, dtype, "final_state")
+
+
+@pytest.mark.parametrize("K,V,dtype", [(128, 128, "bf16"), (64, 32, "f32")], ids=["bulk", "token-kernel"])
+def test_decode_logits_equals_gate_then_step(kda, K, V, dtype):
+    B, H = 3, 5
+    gen = torch.Generator().manual_seed(9)
+    dt = W.DTYPES[dtype]
+    q = torch.nn.functional.normalize(torch.randn(B, H, K, generator=gen), dim=-1).to(dt).to(DEV)
+    k = torch.nn.functional.normalize(torch.randn(B, H, K, generator=gen), dim=-1).to(dt).to(DEV)
+    v = torch.randn(B, H, V, generator=gen).to(dt).to(DEV)
+    z = (torch.randn(B, H, K, generator=gen) * 2).to(DEV)
+    A_log = (torch.randn(H, generator=gen) * 0.5).to(DEV)
+    beta = torch.sigmoid(torch.randn(B, H, generator=gen)).to(DEV)
+    s0 = (torch.randn(B, H, K, V, generator=gen) * 0.1).to(DEV)
+    s_ref, s_new = s0.clone(), s0.clone()
+    for _ in range(3):
+        alpha = kda.bounded_decay(z, A_log, -5.0)
+        o_ref = kda.decode_step(q, k, v, alpha, beta, s_ref)
+        o = kda.decode_step_logits(q, k, v, z, A_log, -5.0, beta, s_new)
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    assert torch.equal(o, o_ref) and torch.equal(s_new, s_ref)
