@@ -10,9 +10,13 @@
 // (128-byte swizzle included), so kernel S moves it with a single bulk copy into a 1 KB-aligned
 // buffer and feeds it straight to tcgen05. Kernel S keeps one CTA per (sequence, head, V-tile) with
 // the transposed state S^T in TMEM and runs two MMA groups per chunk:
-//   group A:  O^T = S^T (Q*Gamma)^T,   U^T = V^T T'^T + S^T (-W)^T
-//   group B:  O^T += U^T A_qk^T,       S^T += U^T (K*gamma_C/Gamma)      (S^T pre-scaled by gamma_C)
-// The price is the workspace traffic (one write and one read of ~1 KB per token-head).
+//   group A:  [U^T | O^T] = S^T [-W ; Q*Gamma]^T  (one N = 128 product),  U^T += V^T T'^T
+//   group B:  [O^T | S^T] += U^T [A_qk ; (K*gamma_C/Gamma)^T]^T  (one N = 192 product; S^T pre-scaled)
+// A tcgen05 MMA's time grows much more slowly than its N, so the products that share an A operand
+// are fused along N. The fused accumulators must be adjacent in TMEM -- [U | O] for group A and
+// [O | S] for group B -- so the O and U buffers alternate with the chunk's parity around the fixed
+// S, and kernel P writes each block's operand pairs in the order that chunk's parity needs.
+// The price of the split is the workspace traffic (one write and one read of ~1 KB per token-head).
 //
 // Workspace slots. Chunk j of sequence n has slot n * ceil(T/64) + j without cu_seqlens, and
 // floor(cu[n]/64) + n + j with them (unique: a sequence's slots end before the next one's begin).
@@ -27,30 +31,29 @@ __device__ int g_split_timeout = 0;
 
 namespace {
 
-// One workspace block = the output region of kernel P = the operand buffer of kernel S.
-constexpr int WB_W = 0;          // 16K  -W [c][t], 128 rows (MN-major B of S^T (-W)^T)
-constexpr int WB_QG = 16384;     // 16K  Q*Gamma [t][c], two atoms (K-major B)
-constexpr int WB_KT = 32768;     // 16K  K*gamma_C/Gamma [t][c], two halves (MN-major B)
-constexpr int WB_TP = 49152;     // 8K   T' [t][i] (K-major B)
-constexpr int WB_AQK = 57344;    // 8K   A_qk [t][i] (K-major B)
+// One workspace block = the output region of kernel P = the operand buffer of kernel S. All three
+// operand regions are K-major; a pair (X, Y) is stored in that order for an even chunk index j and
+// as (Y, X) for an odd one.
+constexpr int WB_WQ = 0;         // 32K  two k-atoms (c) of 128 rows: (-W [t][c], Q*Gamma [t][c])
+constexpr int WB_KA = 32768;     // 24K  one k-atom (t) of 192 rows: (A_qk [t'][t], (K*gamma_C/Gamma)^T [c][t])
+constexpr int WB_TP = 57344;     // 8K   T' [t][i]
 constexpr int WB_GAM = 65536;    // 512  gamma_C, fp32 [128]
 constexpr int WB_BYTES = 66048;
 
 // Kernel P shared memory (104,192 bytes: two CTAs fit on an SM). Q*Gamma and K*gamma_C/Gamma
 // never touch it: the decay pass writes them from registers straight into the workspace block.
-constexpr int P_QE = 0;                     // 16K Qe [t][c]; after A_qk, -W (the block's first 16K)
+constexpr int P_QE = 0;                     // 16K Qe [t][c]; after A_qk, -W [t][c] (two 8K atoms)
 constexpr int P_KE = P_QE + 16384;          // 16K Ke [t][c]; after A_kk, the bf16 copy of T
 constexpr int P_KC = P_KE + 16384;          // 16K Kc [t][c]
 constexpr int P_KG = P_KC + 16384;          // 16K K*Gamma [i][c]
 constexpr int P_AKK = P_KG + 16384;         // 16K A_kk fp32
-constexpr int P_TP = P_AKK + 16384;         // 8K  T'    } the block's last 16,896 bytes, in
-constexpr int P_AQK = P_TP + 8192;          // 8K  A_qk  } workspace order
-constexpr int P_GAM = P_AQK + 8192;         // 512 gamma_C }
+constexpr int P_AQK = P_AKK + 16384;        // 8K  A_qk [t'][t]  } in block order for odd chunks, where
+constexpr int P_TP = P_AQK + 8192;          // 8K  T'            } A_qk ends the KA region and T' and
+constexpr int P_GAM = P_TP + 8192;          // 512 gamma_C       } gamma_C follow it
 constexpr int P_BETA = P_GAM + 512;         // 256 beta
 constexpr int P_VEC = P_BETA + 256;         // vectors
 constexpr int P_SMEM = P_VEC + VEC_FLOATS * 4;
-constexpr int P_TAIL = WB_BYTES - WB_TP;    // 16,896
-static_assert(P_AQK - P_TP == WB_AQK - WB_TP && P_GAM - P_TP == WB_GAM - WB_TP, "tail order matches the block");
+static_assert(P_TP - P_AQK == WB_TP - (WB_KA + 16384) && P_GAM - P_TP == WB_GAM - WB_TP, "odd-chunk tail order");
 static_assert(P_TP % 1024 == 0 && P_AQK % 1024 == 0, "swizzle atoms need 1 KB alignment");
 static_assert(2 * (P_SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 
@@ -63,14 +66,17 @@ constexpr int S_SMEM = S_BAR + 64;
 static_assert(S_SMEM <= 227 * 1024, "shared memory budget");
 static_assert(S_V % 1024 == 0 && S_OPS_STRIDE % 1024 == 0, "swizzle atoms need 1 KB alignment");
 
-// Kernel S tensor memory (columns; lane = value column v of the tile). S^T and U^T in fp32 are MMA
-// accumulators; their bf16 copies (two values per column) are the A operands of the next products;
-// O^T alternates between two buffers so one chunk's output drains while the next chunk's MMAs run.
-constexpr uint32_t TM_S = 0;      // 128  S^T fp32 [v][c]
-constexpr uint32_t TM_U = 128;    // 64   U^T fp32 [v][t]
-constexpr uint32_t TM_O = 192;    // 2x64 O^T fp32 [v][t]
-constexpr uint32_t TM_SB = 320;   // 64   S^T bf16 (K = c)
-constexpr uint32_t TM_UB = 384;   // 32   U^T bf16 (K = t)
+// Kernel S tensor memory (columns; lane = value column v of the tile). S^T, U^T and O^T in fp32 are
+// MMA accumulators, laid out [U_e | O_e | S | O_o | U_o] so that [U | O] and [O | S] are adjacent for
+// chunks of either parity (e: even chunk index, o: odd). The bf16 copies of S^T and U^T (two values
+// per column) are the A operands of the next products.
+constexpr uint32_t TM_UE = 0;     // 64   U^T fp32 [v][t], even chunks
+constexpr uint32_t TM_OE = 64;    // 64   O^T fp32 [v][t], even chunks
+constexpr uint32_t TM_S = 128;    // 128  S^T fp32 [v][c]
+constexpr uint32_t TM_OO = 256;   // 64   O^T, odd chunks
+constexpr uint32_t TM_UO = 320;   // 64   U^T, odd chunks
+constexpr uint32_t TM_SB = 384;   // 64   S^T bf16 (K = c)
+constexpr uint32_t TM_UB = 448;   // 32   U^T bf16 (K = t)
 constexpr uint32_t TM_COLS = 512;
 
 __device__ __forceinline__ void seq_range(const ScanParams& p, int n, int64_t& t0, int64_t& t1, int64_t& brow) {
@@ -119,12 +125,18 @@ __device__ __forceinline__ bool locate_slot(const ScanParams& p, int64_t s, int&
   return true;
 }
 
+__device__ __forceinline__ void bulk_store(unsigned char* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes) : "memory");
+}
+
 // Decay pass, step 2 of kernel P: the same tiles as decay_step2 (chunk_common.cuh), with Q*Gamma and
-// K*gamma_C/Gamma stored straight into the workspace block `blk` (a warp's 32 four-byte stores
-// cover one 128-byte swizzled row). Tokens run forward for the E-scaled tiles and backward for the
-// F-scaled ones, so no per-token F array is held in registers.
+// K*gamma_C/Gamma stored straight into their places in the workspace block. Q*Gamma goes to qg_dst
+// as [t][c] rows of 16 KB k-atoms (a warp's 32 four-byte stores cover one 128-byte swizzled row);
+// K*gamma_C/Gamma goes to kt_dst transposed, [c][t], one 16-byte piece per channel and 8 tokens.
+// Tokens run forward for the E-scaled tiles and backward for the F-scaled ones, so no per-token F
+// array is held in registers.
 __device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch& pf, int da, int c0,
-                                              const float2 (&al)[16], unsigned char* blk) {
+                                              const float2 (&al)[16], unsigned char* qg_dst, unsigned char* kt_dst) {
   float* vec = reinterpret_cast<float*>(sm + P_VEC);
   float2 e[4];
 #pragma unroll
@@ -160,17 +172,27 @@ __device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch&
     *reinterpret_cast<uint32_t*>(sm + P_QE + off) = pack_bf16(qex, qey);
     *reinterpret_cast<uint32_t*>(sm + P_KE + off) = pack_bf16(kex, key);
     *reinterpret_cast<uint32_t*>(sm + P_KG + off) = pack_bf16(kex * GS.x, key * GS.y);
-    *reinterpret_cast<uint32_t*>(blk + WB_QG + off) = pack_bf16(qex * GS.x, qey * GS.y);
+    *reinterpret_cast<uint32_t*>(qg_dst + sw_e(t, c0, 16384)) = pack_bf16(qex * GS.x, qey * GS.y);
   }
   float2 F = make_float2(1.f, 1.f);
+  float ktx[8], kty[8];  // K*gamma_C/Gamma of channels c0, c0+1 for the 8 tokens of one 16-byte piece
 #pragma unroll
   for (int i = 15; i >= 0; --i) {
     const int t = 16 * da + i;
     const float2 kf = unpack_bf16(pf.k[i]);
-    const uint32_t off = sw_e(t, c0, 8192);
     const float kfx = kf.x * F.x, kfy = kf.y * F.y;
-    *reinterpret_cast<uint32_t*>(sm + P_KC + off) = pack_bf16(kfx, kfy);
-    *reinterpret_cast<uint32_t*>(blk + WB_KT + off) = pack_bf16(kfx * PM.x, kfy * PM.y);
+    *reinterpret_cast<uint32_t*>(sm + P_KC + sw_e(t, c0, 8192)) = pack_bf16(kfx, kfy);
+    ktx[i & 7] = kfx * PM.x;
+    kty[i & 7] = kfy * PM.y;
+    if ((i & 7) == 0) {  // tokens 16da + i .. +7 complete: piece j = 2da + i/8 of rows c0 and c0 + 1
+      const int j = 2 * da + (i >> 3);
+      const uint4 wx = make_uint4(pack_bf16(ktx[0], ktx[1]), pack_bf16(ktx[2], ktx[3]), pack_bf16(ktx[4], ktx[5]),
+                                  pack_bf16(ktx[6], ktx[7]));
+      const uint4 wy = make_uint4(pack_bf16(kty[0], kty[1]), pack_bf16(kty[2], kty[3]), pack_bf16(kty[4], kty[5]),
+                                  pack_bf16(kty[6], kty[7]));
+      *reinterpret_cast<uint4*>(kt_dst + sw_chunk(c0, j, 0)) = wx;
+      *reinterpret_cast<uint4*>(kt_dst + sw_chunk(c0 + 1, j, 0)) = wy;
+    }
     F.x *= al[i].x;
     F.y *= al[i].y;
   }
@@ -193,6 +215,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   const int64_t tc0 = t0 + (int64_t)j * C;
   const int nv = (int)min((int64_t)C, t1 - tc0);
   unsigned char* blk = ws + ((size_t)slot * p.H + h) * WB_BYTES;
+  const bool even = (j & 1) == 0;  // operand pair order within the block
 
   ChunkCtx x;
   x.q = static_cast<const __nv_bfloat16*>(p.q);
@@ -220,14 +243,14 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     float2 al[16];
     decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
     __syncthreads();
-    p_decay_step2(sm, pf, da, c0, al, blk);
+    p_decay_step2(sm, pf, da, c0, al, blk + WB_WQ + (even ? 8192 : 0), blk + WB_KA + (even ? 8192 : 0));
   }
   __syncthreads();
   intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
 
   // W = T' (K*Gamma) on mma.sync. Warp w owns columns 16w.. of all 64 rows, so every warp does the
-  // same ten block products of the lower-triangular T'. -W is stored (over the dead Qe tile) as the
-  // MN-major operand of S^T (-W)^T: row c holds W[0..63][c].
+  // same ten block products of the lower-triangular T'. -W is stored over the dead Qe tile as
+  // [t][c], two 64-column atoms: the rows it takes in the block's K-major pair with Q*Gamma.
   {
     float acc[4][2][4];
 #pragma unroll
@@ -257,20 +280,22 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
           const int t = 16 * m + g + 8 * hr, c = 16 * warp + 8 * jn + 2 * tq;
-          *reinterpret_cast<__nv_bfloat16*>(sm + P_QE + sw_e(c, t, 0)) = __float2bfloat16_rn(-acc[m][jn][2 * hr]);
-          *reinterpret_cast<__nv_bfloat16*>(sm + P_QE + sw_e(c + 1, t, 0)) =
-              __float2bfloat16_rn(-acc[m][jn][2 * hr + 1]);
+          *reinterpret_cast<uint32_t*>(sm + P_QE + sw_e(t, c, 8192)) =
+              pack_bf16(-acc[m][jn][2 * hr], -acc[m][jn][2 * hr + 1]);
         }
   }
   fence_async_smem();
   __syncthreads();
   if (tid == 0) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(blk + WB_W), "r"(sb + P_QE),
-                 "r"(WB_QG - WB_W)
-                 : "memory");
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(blk + WB_TP), "r"(sb + P_TP),
-                 "r"(P_TAIL)
-                 : "memory");
+    const uint32_t wq = even ? 0 : 8192;
+    bulk_store(blk + WB_WQ + wq, sb + P_QE, 8192);
+    bulk_store(blk + WB_WQ + 16384 + wq, sb + P_QE + 8192, 8192);
+    if (even) {
+      bulk_store(blk + WB_KA, sb + P_AQK, 8192);
+      bulk_store(blk + WB_TP, sb + P_TP, WB_BYTES - WB_TP);
+    } else {
+      bulk_store(blk + WB_KA + 16384, sb + P_AQK, WB_BYTES - (WB_KA + 16384));
+    }
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     // Shared memory must stay valid until the copies have read it; their global writes complete
     // before the kernel does.
@@ -377,7 +402,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     const uint32_t ops = sb + S_OPS + buf * S_OPS_STRIDE;
     const unsigned char* opsp = sm + S_OPS + buf * S_OPS_STRIDE;
     const uint32_t vbuf = sb + S_V + buf * 16384;
-    const uint32_t tm_o = TM_O + 64 * buf;
+    const uint32_t tm_u = buf ? TM_UO : TM_UE;
 
     // The previous chunk's group B is done (TMEM S^T holds S_{c-1}); this chunk's operands have landed.
     bool w = c == 0 || mbar_wait(bar_mma, 1, &g_split_timeout);
@@ -422,23 +447,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     }
     cp_async_commit();
 
-    // ---- group A: O^T = S^T (Q*Gamma)^T; U^T = V^T T'^T + S^T (-W)^T --------------------------------
+    // ---- group A: [U^T | O^T] = S^T [-W ; Q*Gamma]^T, then U^T += V^T T'^T ---------------------------
     if (tid == 0) {
-      constexpr uint32_t id_kk = idesc_bf16(64, 0, 0), id_mk = idesc_bf16(64, 1, 0), id_km = idesc_bf16(64, 0, 1);
+      constexpr uint32_t id_wq = idesc_bf16(128, 0, 0), id_vt = idesc_bf16(64, 1, 0);
+      const uint32_t d_a = buf ? TM_OO : TM_UE;  // [U_e | O_e] or [O_o | U_o]
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        tc_mma_ts(tmem + tm_o, tmem + TM_SB + 8 * ks, sdesc(ops + WB_QG + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
-                  id_kk, ks > 0);
+        tc_mma_ts(tmem + d_a, tmem + TM_SB + 8 * ks, sdesc(ops + WB_WQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                  id_wq, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        tc_mma(tmem + TM_U, sdesc(vbuf + ks * 2048, 8192, 1024), sdesc(ops + WB_TP + ks * 32, 16, 1024), id_mk, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        tc_mma_ts(tmem + TM_U, tmem + TM_SB + 8 * ks, sdesc(ops + WB_W + ks * 2048, 8192, 1024), id_km, 1);
+        tc_mma(tmem + tm_u, sdesc(vbuf + ks * 2048, 8192, 1024), sdesc(ops + WB_TP + ks * 32, 16, 1024), id_vt, 1);
       tc_commit(bar_mma);
     }
     // meanwhile: the previous chunk's output
-    if (c > 0) store_o(p, tlane, TM_O + 64 * (buf ^ 1), brow, h, vt, trow, half, tc0 - C, C);
+    if (c > 0) store_o(p, tlane, buf ? TM_OE : TM_OO, brow, h, vt, trow, half, tc0 - C, C);
 
     ok = __syncthreads_and(mbar_wait(bar_mma, 0, &g_split_timeout));
     tc_fence_after();
@@ -447,7 +470,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     // ---- U^T -> its bf16 copy ---------------------------------------------------------------------
     {
       uint32_t r[32], b16[16];
-      tm_ld32(tlane + TM_U + 32 * half, r);
+      tm_ld32(tlane + tm_u + 32 * half, r);
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) b16[jj] = pack_bf16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]));
       tm_st16(tlane + TM_UB + 16 * half, b16);
@@ -457,14 +480,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     __syncthreads();
     tc_fence_after();
 
-    // ---- group B: O^T += U^T A_qk^T; S^T += U^T (K*gamma_C/Gamma) -----------------------------------
+    // ---- group B: [O^T | S^T] += U^T [A_qk ; (K*gamma_C/Gamma)^T]^T -----------------------------------
     if (tid == 0) {
-      constexpr uint32_t id_o = idesc_bf16(64, 0, 0), id_s = idesc_bf16(128, 0, 1);
+      constexpr uint32_t id_b = idesc_bf16(192, 0, 0);
+      const uint32_t d_b = buf ? TM_S : TM_OE;  // [O_e | S] or [S | O_o]
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        tc_mma_ts(tmem + tm_o, tmem + TM_UB + 8 * ks, sdesc(ops + WB_AQK + ks * 32, 16, 1024), id_o, 1);
-        tc_mma_ts(tmem + TM_S, tmem + TM_UB + 8 * ks, sdesc(ops + WB_KT + ks * 2048, 8192, 1024), id_s, 1);
-      }
+      for (int ks = 0; ks < 4; ++ks)
+        tc_mma_ts(tmem + d_b, tmem + TM_UB + 8 * ks, sdesc(ops + WB_KA + ks * 32, 16, 1024), id_b, 1);
       tc_commit(bar_mma);
     }
   }
@@ -474,7 +496,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     tc_fence_after();
     if (ok) {
       const int64_t tl = t0 + (int64_t)(n_chunks - 1) * C;
-      store_o(p, tlane, TM_O + 64 * ((n_chunks - 1) & 1), brow, h, vt, trow, half, tl, (int)(t1 - tl));
+      store_o(p, tlane, ((n_chunks - 1) & 1) ? TM_OO : TM_OE, brow, h, vt, trow, half, tl, (int)(t1 - tl));
     }
   }
   cp_async_wait_all();
