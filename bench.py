@@ -77,6 +77,32 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
     return n_elems * (es_in + es_out)
 
 
+# DRAM bytes (read + write) per launch of each step, from one ncu capture of its kernels (the summaries in
+# profiles/ give the commands). They hold only for the kernel sources they were taken on, so the sources'
+# sha256 is kept beside them and a mismatch at run time reports null.
+MEASURED_TRAFFIC = {
+    # chunk_intra_kernel 406,194,432 + 361,915,904; chunk_state_kernel 506,586,880 + 88,780,800
+    "prefill": {"bytes": 1363478016, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                "sha256": "bd6ff9ac2b766c5f6fe04b5e68dd96449333a3ad4a9d305d8bb52317cba10ac4"},
+    # decode_bulk_kernel 410,576,384 + 346,768,128
+    "decode": {"bytes": 757344512, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "c610949afd405b658089a364bcc2cff6f7a87367e31ce3b451c06b1d6b8af854"},
+}
+
+
+def measured_traffic(step: str):
+    import hashlib
+    m = MEASURED_TRAFFIC[step]
+    h = hashlib.sha256()
+    try:
+        for f in m["files"]:
+            with open(os.path.join(ROOT, "gated_delta_rule_bounded_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return m["bytes"] if h.hexdigest() == m["sha256"] else None
+
+
 # ------------------------------------------------------------------------------------------------
 # Environment helpers
 # ------------------------------------------------------------------------------------------------
@@ -289,7 +315,7 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
         "value": value, "ms_per_step": ms_per_step, "workload": w, "clocks": sampler.summary() if sampler else None,
         "kernels_ms": {"prefill_logits": pre_ms},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "kernel": "kda_prefill_logits",
+                     "frac": achieved / hbm, "traffic": measured_traffic("prefill"), "kernel": "kda_prefill_logits",
                      "bytes_per_launch": pb, "ms_per_launch": pre_ms, "peak_source": f"{peak_src} hbm_gbs",
                      "tensor": {"tflops_at_C64_formula": tflops, "peak": bf16_peak,
                                 "frac": tflops / bf16_peak, "flops_per_launch": flops}},
@@ -350,7 +376,7 @@ def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
         "steps_per_s": 1e3 / d_ms, "ms_per_step": d_ms, "steps": dsteps, "gpu_launches": dsteps,
         "kernels_ms": {"decode_step_logits": dk_ms},
         "roofline": {"bound": "hbm", "achieved": d_achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": d_achieved / hbm, "traffic": None, "kernel": "kda_decode_step_logits",
+                     "frac": d_achieved / hbm, "traffic": measured_traffic("decode"), "kernel": "kda_decode_step_logits",
                      "bytes_per_launch": dbytes, "ms_per_launch": dk_ms, "peak_source": f"{peak_src} hbm_gbs"},
         "clocks": dsampler.summary() if dsampler is not None else None,
     }

@@ -52,3 +52,13 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.weak_scaling_value(100.0, 50.0, 1) == (2000.0, 50.0)
+
+
+def test_measured_traffic_only_for_the_profiled_sources(monkeypatch):
+    import bench
+    for step in ("prefill", "decode"):
+        v = bench.measured_traffic(step)
+        assert v is None or v == bench.MEASURED_TRAFFIC[step]["bytes"]
+        changed = dict(bench.MEASURED_TRAFFIC[step], sha256="0" * 64)
+        monkeypatch.setitem(bench.MEASURED_TRAFFIC, step, changed)
+        assert bench.measured_traffic(step) is None
