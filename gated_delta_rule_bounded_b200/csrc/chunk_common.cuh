@@ -498,21 +498,31 @@ __device__ __forceinline__ void inverse_warps0to3(unsigned char* sm, uint32_t sb
   }
 }
 
+// Barrier over the 256 threads of warps 0-7: the whole CTA (barrier 0), or named barrier 2 in a
+// kernel whose other warps run different code.
+template <bool NAMED>
+__device__ __forceinline__ void sync_compute() {
+  if (NAMED)
+    asm volatile("bar.sync 2, 256;" ::: "memory");
+  else
+    __syncthreads();
+}
+
 // The state-independent phases after the decay pass: A_kk on all warps; then the inverse on warps
 // 0-3 while warps 4-7 form A_qk (and zero its upper blocks; transposed with QK_T). Ends with a
-// CTA-wide barrier.
-template <bool QK_T = false>
+// barrier over warps 0-7 (named barrier 2 with NAMED, else the CTA barrier).
+template <bool QK_T = false, bool NAMED = false>
 __device__ __forceinline__ void intra_phases(unsigned char* sm, uint32_t sb, const IntraLayout& L, const float* beta_s,
                                              int tid, int warp, int lane, int g, int tq) {
   a_tiles<2>(sm, sb, L, L.ke, warp, 8, warp < 2 ? 2 : 1, lane, g, tq, beta_s, /*is_qk=*/false);
-  __syncthreads();  // A_kk ready; Ke is dead
+  sync_compute<NAMED>();  // A_kk ready; Ke is dead
   if (warp < 4) {
     inverse_warps0to3(sm, sb, L, beta_s, tid, warp, lane, g, tq);
   } else {
     a_tiles<3, QK_T>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
     zero_upper_blocks<QK_T>(sm, L.aqk, tid - 128, 128);  // the MMAs read whole rows of A_qk
   }
-  __syncthreads();
+  sync_compute<NAMED>();
 }
 
 }  // namespace

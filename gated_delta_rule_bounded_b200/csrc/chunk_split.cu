@@ -205,6 +205,9 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   constexpr IntraLayout LY{P_QE, P_KE, P_KC, -1, P_KG, -1, P_AKK, P_AQK, P_TP, P_KE, P_VEC};
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
+  // Kernel S may be scheduled once every CTA of this grid has started; it reads the workspace only
+  // after this whole grid has completed (griddepcontrol.wait).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int h = blockIdx.y;
   const float gsc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int64_t slot = blockIdx.x;
@@ -374,7 +377,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
   const uint32_t tlane = tmem + ((uint32_t)(32 * quad) << 16);
 
   if (n_chunks > 0) {
-    if (tid == 0) bulk_load(sb + S_OPS, block_src(0), WB_BYTES, bar_ops);
     load_v(x, sb + S_V, t0, (int)min((int64_t)C, t1 - t0), tid);
     cp_async_commit();
   }
@@ -391,6 +393,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     tm_st32(tlane + TM_S + cb, r);
   }
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+  // Everything above reads only the scan's inputs; the operand blocks are kernel P's output, so the
+  // first block is fetched once that grid has completed (a no-op when launched without a dependency).
+  if (tid == 0 && n_chunks > 0) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    bulk_load(sb + S_OPS, block_src(0), WB_BYTES, bar_ops);
+  }
 
   // Each chunk's MMAs complete twice on bar_mma, group A then group B, and every completion is
   // waited for before the next group is issued: group A always completes phase parity 0, B parity 1.
@@ -565,7 +573,20 @@ cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t grid = (int64_t)p.N * p.H * (p.V / VT);
-  chunk_state_kernel<<<(unsigned)grid, NTHREADS, S_SMEM, s>>>(p, static_cast<const unsigned char*>(ws));
+  // Programmatic dependent launch: kernel S's CTAs set up (barriers, TMEM, initial state, first v tile)
+  // while kernel P's last CTAs finish.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = S_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, chunk_state_kernel, p, static_cast<const unsigned char*>(ws));
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
