@@ -28,6 +28,7 @@ _LIB_PATH = os.path.join(_PKG, "libkda.so")
 
 KDA_F32, KDA_BF16 = 0, 1
 KDA_GATE_ALPHA, KDA_GATE_LOG = 0, 1
+KDA_QK_L2NORM, KDA_BETA_LOGITS = 1, 2
 _STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA"}
 
 
@@ -73,10 +74,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_prefill_noalloc.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64,
                                         i64, i64, i64, i64, i64, lp, vp, vp]
     lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, i64, i64, i64, i64, lp, vp, vp]
-    lib.kda_prefill_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, vp, vp, vp, i64,
+    u32 = ctypes.c_uint
+    lib.kda_prefill_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, u32, vp, vp, vp, i64,
                                        i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
-    lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, vp, i64, i64, i64, i64, lp,
-                                           vp, vp]
+    lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, u32, vp, i64, i64, i64, i64,
+                                           lp, vp, vp]
     for fn in ("kda_bounded_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
                "kda_decode_step", "kda_prefill_logits", "kda_decode_step_logits"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -226,10 +228,10 @@ def _prefill(q, k, v, gate, beta, initial_state, cu_seqlens, gate_is_log, output
             cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
             _stream(dev)))
     else:
-        A_log, g_min = logits
+        A_log, g_min, flags = logits
         _check("kda_prefill_logits", lib.kda_prefill_logits(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
-            A_log.data_ptr(), g_min, beta.data_ptr(), s0_ptr, sf_ptr,
+            A_log.data_ptr(), g_min, beta.data_ptr(), flags, s0_ptr, sf_ptr,
             cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
             _stream(dev)))
     return out, final_state
@@ -257,18 +259,22 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
 
 def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
                    g_min: float, beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
-                   cu_seqlens: Optional[torch.Tensor] = None, *, output_final_state: bool = True,
+                   cu_seqlens: Optional[torch.Tensor] = None, *, qk_l2norm: bool = False,
+                   beta_logits: bool = False, output_final_state: bool = True,
                    out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None,
                    use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """``prefill`` fed with the decay logits ``z [B,T,H,K]`` (fp32) instead of alpha: the scan kernels
     evaluate ``g = g_min * sigmoid(exp(A_log[h]) * z)`` themselves (``kda_prefill_logits``).
-    ``A_log [H]`` fp32 on the device; ``g_min < 0``. Other arguments as in ``prefill``."""
+    ``A_log [H]`` fp32 on the device; ``g_min < 0``. ``qk_l2norm``: the kernels L2-normalise q and k over
+    K per (token, head); ``beta_logits``: ``beta`` holds logits and the kernels apply the sigmoid.
+    Other arguments as in ``prefill``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
+    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
     return _prefill(q, k, v, z, beta, initial_state, cu_seqlens, False, output_final_state, out, final_state,
-                    workspace, use_workspace, logits=(A_log.contiguous(), float(g_min)), gate_name="z")
+                    workspace, use_workspace, logits=(A_log.contiguous(), float(g_min), flags), gate_name="z")
 
 
 NOALLOC_SCRATCH_BYTES = 128 << 20  # the library's static scratch (KDA_NOALLOC_SCRATCH_BYTES)
@@ -357,23 +363,25 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
             KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), state.data_ptr(),
             B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
     else:
-        A_log, g_min = logits
+        A_log, g_min, flags = logits
         _check("kda_decode_step_logits", lib.kda_decode_step_logits(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
-            A_log.data_ptr(), g_min, beta.data_ptr(), state.data_ptr(),
+            A_log.data_ptr(), g_min, beta.data_ptr(), flags, state.data_ptr(),
             B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
     return out
 
 
 def decode_step_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
-                       g_min: float, beta: torch.Tensor, state: torch.Tensor, *,
-                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                       g_min: float, beta: torch.Tensor, state: torch.Tensor, *, qk_l2norm: bool = False,
+                       beta_logits: bool = False, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """``decode_step`` fed with the decay logits ``z [B,H,K]`` (fp32): the step evaluates the bounded gate
-    itself (``kda_decode_step_logits``). ``A_log [H]`` fp32 on the device; ``g_min < 0``."""
+    itself (``kda_decode_step_logits``). ``A_log [H]`` fp32 on the device; ``g_min < 0``; ``qk_l2norm`` and
+    ``beta_logits`` as in ``prefill_logits``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[-2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
-    return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min)))
+    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
+    return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min), flags))
 
 
 def device_status(reset: bool = True) -> bool:

@@ -190,6 +190,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
     cp_async_commit();
 
     // ---- decay pass: block-local cumulative decay, scaled operand tiles, decay vectors -------------
+    if (p.beta_sigmoid && tid < C) {  // beta of this chunk arrived as logits
+      float* bw = reinterpret_cast<float*>(sm + OFF_BETA + (c & 1) * 256);
+      bw[tid] = beta_value(bw[tid], 1);
+    }
+    if (p.qk_l2norm) l2norm_qk(pf, vec + VEC_D, tid, da);
     {
       float2 al[16];
       decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);

@@ -343,6 +343,48 @@ __device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const In
 }
 
 
+// L2-normalises, in place, the q and k values a decay-pass thread holds (channels c0, c0+1 of the 16
+// tokens of block da; warps 2da and 2da+1 hold the two halves of each token row) over all K = 128
+// channels, rounding the results back to bf16. Each warp sums its half-rows by a reduce-scatter (lane
+// L ends with token L/2), the two halves meet in `red` (256 floats), and one CTA barrier publishes them.
+__device__ __forceinline__ void l2norm_qk(Prefetch& pf, float* red, int tid, int da) {
+  const int lane = tid & 31, half = (tid >> 5) & 1;
+#pragma unroll
+  for (int which = 0; which < 2; ++which) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 x = unpack_bf16(which ? pf.k[i] : pf.q[i]);
+      v[i] = x.x * x.x + x.y * x.y;
+    }
+#pragma unroll
+    for (int step = 0; step < 4; ++step) {  // keep 8, 4, 2, 1 tokens
+      const int w = 8 >> step, bit = 16 >> step;
+      const bool up = (lane & bit) != 0;
+#pragma unroll
+      for (int j = 0; j < w; ++j) {
+        const float send = up ? v[j] : v[j + w];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, bit);
+        v[j] = (up ? v[j + w] : v[j]) + recv;
+      }
+    }
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+    if ((lane & 1) == 0) red[which * 128 + (da * 2 + half) * 16 + (lane >> 1)] = v[0];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int which = 0; which < 2; ++which) {
+    const float* r0 = red + which * 128 + da * 32;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float sc = l2norm_scale(r0[i] + r0[16 + i]);
+      uint32_t& w = which ? pf.k[i] : pf.q[i];
+      const float2 x = unpack_bf16(w);
+      w = pack_bf16(x.x * sc, x.y * sc);
+    }
+  }
+}
+
 // The log2-decay of one channel from the gate value x in gate mode `mode` (alpha, g = log alpha, or
 // the decay logits z with sc = e^{A_h}).
 __device__ __forceinline__ float log2_decay(int mode, float x, float sc, float g_min) {

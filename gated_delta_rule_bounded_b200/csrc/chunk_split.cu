@@ -242,7 +242,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   {
     Prefetch pf;
     load_qkg(x, tc0, nv, c0, da, pf);
-    if (tid < C) beta_s[tid] = tid < nv ? __ldg(x.beta + x.boff + (tc0 + tid) * x.bst) : 0.f;
+    if (tid < C) beta_s[tid] = tid < nv ? beta_value(__ldg(x.beta + x.boff + (tc0 + tid) * x.bst), p.beta_sigmoid) : 0.f;
+    if (p.qk_l2norm) l2norm_qk(pf, reinterpret_cast<float*>(sm + P_VEC) + VEC_D, tid, da);
     float2 al[16];
     decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
     __syncthreads();

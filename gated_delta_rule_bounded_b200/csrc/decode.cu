@@ -38,8 +38,8 @@ struct StageLayout {
   static constexpr int V = K + IN;
   static constexpr int A = V + IN;
   static constexpr int BYTES = A + DK * 4;          // + alpha row (fp32)
-  static constexpr int RED = NSTAGE * BYTES;        // partial sums [2][8][128] + k.q [8]
-  static constexpr int BAR = RED + (2 * 8 * DV + 8) * 4;
+  static constexpr int RED = NSTAGE * BYTES;        // partial sums [2][8][128] + k.q, k.k, q.q [3][8]
+  static constexpr int BAR = RED + (2 * 8 * DV + 24) * 4;
   static constexpr int SMEM = BAR + NSTAGE * 8;
 };
 
@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
   float* red_a = reinterpret_cast<float*>(sm + L::RED);
   float* red_b = red_a + 8 * DV;
   float* red_kq = red_b + 8 * DV;
+  float* red_kk = red_kq + 8;  // sums of k^2 and q^2 (in-kernel L2 normalisation)
+  float* red_qq = red_kk + 8;
   const uint32_t bar0 = sb + L::BAR;
 
   if (tid == 0) {
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
     for (; issued < NSTAGE && issued < n_my; ++issued)
       issue_stage<TIn>(p, blockIdx.x + issued * gridDim.x, sb + issued * L::BYTES, bar0 + 8 * issued);
   int done_heads = 0;
-  float beta_next = n_my > 0 ? __ldg(head_ptrs<TIn>(p, blockIdx.x).beta) : 0.f;
+  float beta_next = n_my > 0 ? beta_value(__ldg(head_ptrs<TIn>(p, blockIdx.x).beta), p.beta_sigmoid) : 0.f;
 
   for (int i = 0; i < n_my; ++i) {
     const int head = blockIdx.x + i * gridDim.x;
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
     const int s = i % NSTAGE;
     unsigned char* st = sm + s * L::BYTES;
     const float beta = beta_next;
-    if (i + 1 < n_my) beta_next = __ldg(head_ptrs<TIn>(p, head + gridDim.x).beta);
+    if (i + 1 < n_my) beta_next = beta_value(__ldg(head_ptrs<TIn>(p, head + gridDim.x).beta), p.beta_sigmoid);
     if (!__syncthreads_and(mbar_wait(bar0 + 8 * s, (i / NSTAGE) & 1))) break;
     done_heads = i + 1;
 
@@ -151,7 +153,7 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
 
     float4 x[ROWS];
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
-    float pkq = 0.f;
+    float pkq = 0.f, pkk = 0.f, pqq = 0.f;
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
       const int row = row0 + r;
@@ -163,13 +165,19 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
       pb.x = fmaf(qq, x[r].x, pb.x); pb.y = fmaf(qq, x[r].y, pb.y);
       pb.z = fmaf(qq, x[r].z, pb.z); pb.w = fmaf(qq, x[r].w, pb.w);
       pkq = fmaf(kk, qq, pkq);
+      pkk = fmaf(kk, kk, pkk);
+      pqq = fmaf(qq, qq, pqq);
     }
     *reinterpret_cast<float4*>(red_a + tk * DV + col0) = pa;
     *reinterpret_cast<float4*>(red_b + tk * DV + col0) = pb;
-    if (tv == 0) red_kq[tk] = pkq;
+    if (tv == 0) {
+      red_kq[tk] = pkq;
+      red_kk[tk] = pkk;
+      red_qq[tk] = pqq;
+    }
     __syncthreads();
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f), Bq = A;
-    float kq = 0.f;
+    float kq = 0.f, kk2 = 0.f, qq2 = 0.f;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
       const float4 ya = *reinterpret_cast<const float4*>(red_a + g * DV + col0);
@@ -177,6 +185,16 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
       A.x += ya.x; A.y += ya.y; A.z += ya.z; A.w += ya.w;
       Bq.x += yb.x; Bq.y += yb.y; Bq.z += yb.z; Bq.w += yb.w;
       kq += red_kq[g];
+      kk2 += red_kk[g];
+      qq2 += red_qq[g];
+    }
+    // In-kernel L2 normalisation of k and q: every term is linear in each, so the scales apply to the
+    // sums (k^T S, q^T S, k^T q) and to the rank-1 update.
+    const float ik = p.qk_l2norm ? l2norm_scale(kk2) : 1.f, iq = p.qk_l2norm ? l2norm_scale(qq2) : 1.f;
+    if (p.qk_l2norm) {
+      A.x *= ik; A.y *= ik; A.z *= ik; A.w *= ik;
+      Bq.x *= iq; Bq.y *= iq; Bq.z *= iq; Bq.w *= iq;
+      kq *= ik * iq;
     }
     const float4 vv = load4(vs + col0);
     const float4 d = make_float4(vv.x - A.x, vv.y - A.y, vv.z - A.z, vv.w - A.w);
@@ -188,7 +206,7 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
       const int row = row0 + r;
-      const float bk = beta * to_f32(ks[row]);
+      const float bk = beta * (to_f32(ks[row]) * ik);
       x[r].x = fmaf(bk, d.x, x[r].x); x[r].y = fmaf(bk, d.y, x[r].y);
       x[r].z = fmaf(bk, d.z, x[r].z); x[r].w = fmaf(bk, d.w, x[r].w);
       *reinterpret_cast<float4*>(S + row * DV + col0) = x[r];

@@ -22,6 +22,12 @@ __device__ __forceinline__ float gate_sigmoid(float x) {
 // g = g_min * sigmoid(sc * z) with sc = e^{A_h} (computed once per head as expf(A_log[h])).
 __device__ __forceinline__ float bounded_log_decay(float sc, float z, float g_min) { return g_min * gate_sigmoid(sc * z); }
 
+// The write strength: beta itself, or sigmoid(beta) when the scan receives its logits.
+__device__ __forceinline__ float beta_value(float b, int from_logits) { return from_logits ? gate_sigmoid(b) : b; }
+
+// Scale that L2-normalises a q or k row with squared norm `ss` (x / sqrt(ss + 1e-6)).
+__device__ __forceinline__ float l2norm_scale(float ss) { return rsqrtf(ss + 1e-6f); }
+
 // The retention factor alpha of one channel for a scan in gate mode `mode`.
 __device__ __forceinline__ float gate_alpha(int mode, float x, float sc, float g_min) {
   return mode == GATE_LOGITS ? expf(bounded_log_decay(sc, x, g_min)) : (mode == 1 ? expf(x) : x);

@@ -155,6 +155,7 @@ struct GateSpec {
   int mode;
   const float* A_log;
   float g_min;
+  unsigned flags;  // KDA_QK_L2NORM | KDA_BETA_LOGITS
 };
 
 static int check_gate(const char* fn, const GateSpec& gs) {
@@ -162,6 +163,8 @@ static int check_gate(const char* fn, const GateSpec& gs) {
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, gs.mode);
   if (gs.mode == kda::GATE_LOGITS && (!std::isfinite(gs.g_min) || !(gs.g_min < 0.f)))
     return fail(KDA_ERR_INVALID_ARG, "%s: g_min must be finite and < 0 (got %g)", fn, (double)gs.g_min);
+  if (gs.flags & ~(KDA_QK_L2NORM | KDA_BETA_LOGITS))
+    return fail(KDA_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, gs.flags);
   return KDA_OK;
 }
 
@@ -259,6 +262,8 @@ static int prefill_impl(const char* fn, const void* q, const void* k, const void
   p.gate_mode = gs.mode;
   p.A_log = gs.A_log;
   p.g_min = gs.g_min;
+  p.qk_l2norm = (gs.flags & KDA_QK_L2NORM) != 0;
+  p.beta_sigmoid = (gs.flags & KDA_BETA_LOGITS) != 0;
 
   cudaError_t e;
   if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype)) {
@@ -280,19 +285,19 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
                 void* workspace, size_t workspace_bytes, kda_stream_t stream) {
   if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
     return fail(KDA_ERR_INVALID_ARG, "kda_prefill: unknown gate kind %d", (int)gate_kind);
-  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f};
+  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f, 0u};
   return prefill_impl("kda_prefill", q, k, v, dtype, gs, beta, initial_state, final_state, cu_seqlens, n_seq, B, T, H,
                       K, V, layout, o, workspace, workspace_bytes, stream);
 }
 
 int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                       const float* logits, const float* A_log, float g_min, const float* beta,
+                       const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
                        const float* initial_state, float* final_state,
                        const int32_t* cu_seqlens, int64_t n_seq,
                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                        const kda_layout* layout, void* o,
                        void* workspace, size_t workspace_bytes, kda_stream_t stream) {
-  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min};
+  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min, flags};
   return prefill_impl("kda_prefill_logits", q, k, v, dtype, gs, beta, initial_state, final_state, cu_seqlens, n_seq, B,
                       T, H, K, V, layout, o, workspace, workspace_bytes, stream);
 }
@@ -355,6 +360,8 @@ static int decode_impl(const char* fn, const void* q, const void* k, const void*
   p.gate_mode = gs.mode;
   p.A_log = gs.A_log;
   p.g_min = gs.g_min;
+  p.qk_l2norm = (gs.flags & KDA_QK_L2NORM) != 0;
+  p.beta_sigmoid = (gs.flags & KDA_BETA_LOGITS) != 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kda::decode_bulk_supported(p) ? kda::launch_decode_bulk(p, dtype, s) : kda::launch_recurrent(p, dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
@@ -367,15 +374,15 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
                     const kda_layout* layout, void* o, kda_stream_t stream) {
   if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
     return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: unknown gate kind %d", (int)gate_kind);
-  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f};
+  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f, 0u};
   return decode_impl("kda_decode_step", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 
 int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                           const float* logits, const float* A_log, float g_min, const float* beta,
+                           const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
                            float* state, int64_t B, int64_t H, int64_t K, int64_t V,
                            const kda_layout* layout, void* o, kda_stream_t stream) {
-  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min};
+  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min, flags};
   return decode_impl("kda_decode_step_logits", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 

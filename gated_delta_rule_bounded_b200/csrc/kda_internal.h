@@ -30,6 +30,8 @@ struct ScanParams {
   int gate_mode;        // KDA_GATE_ALPHA, KDA_GATE_LOG, or GATE_LOGITS (gate holds decay logits z)
   const float* A_log;   // [H], GATE_LOGITS only
   float g_min;          // GATE_LOGITS only
+  int qk_l2norm;        // q, k are L2-normalised over K inside the kernels
+  int beta_sigmoid;     // beta holds logits; the kernels use sigmoid(beta)
 };
 
 struct GateParams {

@@ -31,7 +31,7 @@ constexpr int kRowGroups = 8;
 // Floats of one staging buffer, rounded up to a multiple of four so that both
 // buffers keep their float4 partial-sum arrays 16-byte aligned.
 __host__ __device__ constexpr int stage_floats(int K, int VT) {
-  return (3 * K + VT + 2 * kRowGroups * VT + kRowGroups + 1 + 3) & ~3;
+  return (3 * K + VT + 2 * kRowGroups * VT + 3 * kRowGroups + 1 + 3) & ~3;
 }
 
 // RPT is the (maximum) number of key rows per thread; kExact marks K == 8 * RPT,
@@ -91,7 +91,9 @@ recurrent_kernel(ScanParams p) {
     float* red_a = s_v + VT;
     float* red_b = red_a + kRowGroups * VT;
     float* red_kq = red_b + kRowGroups * VT;
-    float* s_beta = red_kq + kRowGroups;
+    float* red_kk = red_kq + kRowGroups;  // sums of k^2 and q^2 (in-kernel L2 normalisation)
+    float* red_qq = red_kk + kRowGroups;
+    float* s_beta = red_qq + kRowGroups;
 
     const int64_t qo = brow * p.qs[0] + t * p.qs[1] + h * p.qs[2];
     const int64_t ko = brow * p.ks[0] + t * p.ks[1] + h * p.ks[2];
@@ -103,11 +105,11 @@ recurrent_kernel(ScanParams p) {
       s_q[i] = to_f32(qb[qo + i]);
     }
     for (int j = tid; j < VT; j += NT) s_v[j] = to_f32(vb[vo + vt * VT + j]);
-    if (tid == 0) s_beta[0] = __ldg(p.beta + brow * p.bs[0] + t * p.bs[1] + h * p.bs[2]);
+    if (tid == 0) s_beta[0] = beta_value(__ldg(p.beta + brow * p.bs[0] + t * p.bs[1] + h * p.bs[2]), p.beta_sigmoid);
     __syncthreads();
 
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
-    float pkq = 0.f;
+    float pkq = 0.f, pkk = 0.f, pqq = 0.f;
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       if (r < rpt) {
@@ -119,15 +121,21 @@ recurrent_kernel(ScanParams p) {
         pb.x = fmaf(qq, S[r].x, pb.x); pb.y = fmaf(qq, S[r].y, pb.y);
         pb.z = fmaf(qq, S[r].z, pb.z); pb.w = fmaf(qq, S[r].w, pb.w);
         pkq = fmaf(kk, qq, pkq);
+        pkk = fmaf(kk, kk, pkk);
+        pqq = fmaf(qq, qq, pqq);
       }
     }
     *reinterpret_cast<float4*>(red_a + tk * VT + tv * 4) = pa;
     *reinterpret_cast<float4*>(red_b + tk * VT + tv * 4) = pb;
-    if (tv == 0) red_kq[tk] = pkq;
+    if (tv == 0) {
+      red_kq[tk] = pkq;
+      red_kk[tk] = pkk;
+      red_qq[tk] = pqq;
+    }
     __syncthreads();
 
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f), Bq = A;
-    float kq = 0.f;
+    float kq = 0.f, kk2 = 0.f, qq2 = 0.f;
 #pragma unroll
     for (int g = 0; g < kRowGroups; ++g) {
       float4 x = *reinterpret_cast<const float4*>(red_a + g * VT + tv * 4);
@@ -135,6 +143,16 @@ recurrent_kernel(ScanParams p) {
       A.x += x.x; A.y += x.y; A.z += x.z; A.w += x.w;
       Bq.x += y.x; Bq.y += y.y; Bq.z += y.z; Bq.w += y.w;
       kq += red_kq[g];
+      kk2 += red_kk[g];
+      qq2 += red_qq[g];
+    }
+    // In-kernel L2 normalisation of k and q: every term is linear in each, so the scales apply to the
+    // sums (k^T S, q^T S, k^T q) and to the rank-1 update.
+    const float ik = p.qk_l2norm ? l2norm_scale(kk2) : 1.f, iq = p.qk_l2norm ? l2norm_scale(qq2) : 1.f;
+    if (p.qk_l2norm) {
+      A.x *= ik; A.y *= ik; A.z *= ik; A.w *= ik;
+      Bq.x *= iq; Bq.y *= iq; Bq.z *= iq; Bq.w *= iq;
+      kq *= ik * iq;
     }
     const float beta = s_beta[0];
     float4 d;
@@ -151,7 +169,7 @@ recurrent_kernel(ScanParams p) {
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       if (r < rpt) {
-        const float bk = beta * s_k[row0 + r];
+        const float bk = beta * (s_k[row0 + r] * ik);
         S[r].x = fmaf(bk, d.x, S[r].x); S[r].y = fmaf(bk, d.y, S[r].y);
         S[r].z = fmaf(bk, d.z, S[r].z); S[r].w = fmaf(bk, d.w, S[r].w);
       }

@@ -151,6 +151,16 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
                 const kda_layout* layout, void* o,
                 void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
+/* Input preparation the logits entry points can do inside their kernels
+ * (bit flags): the steps the surrounding model applies to q, k and beta
+ * ("KDA cheat sheet", How the inputs are produced: q, k = L2Norm(...),
+ * beta = Sigmoid(W_beta x)).
+ *   KDA_QK_L2NORM    q and k are replaced by x / sqrt(sum_c x_c^2 + 1e-6) over
+ *                    the K channels of each (token, head) before use.
+ *   KDA_BETA_LOGITS  beta holds logits b; the kernels use sigmoid(b). */
+#define KDA_QK_L2NORM 1u
+#define KDA_BETA_LOGITS 2u
+
 /* ---------------------------------------------------------------------------
  * kda_prefill_logits: kda_prefill with the bounded gate applied inside the
  * scan ("Kimi K3: Bounded Decay and Delta Memory", Formula and conventions,
@@ -163,14 +173,18 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  *          uses for alpha / g).
  * A_log    [H] fp32 device pointer; g_min finite and < 0
  *          (else KDA_ERR_INVALID_ARG).
+ * flags    0, or KDA_QK_L2NORM and/or KDA_BETA_LOGITS (unknown bits:
+ *          KDA_ERR_INVALID_ARG). The chunked bf16 kernels round normalised
+ *          q and k to bf16, their operand precision; the fp32 kernel keeps
+ *          them in fp32.
  * Every other argument, layout, result, workspace rule and error is
- * kda_prefill's. The result is bit-identical to kda_bounded_decay with
- * out_kind KDA_GATE_LOG (bf16 inputs) or KDA_GATE_ALPHA (fp32 inputs)
- * followed by kda_prefill on its output: both evaluate the gate with the same
- * device code.
+ * kda_prefill's. With flags 0 the result is bit-identical to
+ * kda_bounded_decay with out_kind KDA_GATE_LOG (bf16 inputs) or
+ * KDA_GATE_ALPHA (fp32 inputs) followed by kda_prefill on its output: both
+ * evaluate the gate with the same device code.
  * ------------------------------------------------------------------------- */
 int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                       const float* logits, const float* A_log, float g_min, const float* beta,
+                       const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
                        const float* initial_state, float* final_state,
                        const int32_t* cu_seqlens, int64_t n_seq,
                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
@@ -232,11 +246,12 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
  * kda_decode_step_logits: kda_decode_step with the bounded gate (eq. 5)
  * applied inside the step: logits [B,H,K] fp32 (strides in layout->gate),
  * A_log [H] fp32, g_min finite and < 0. alpha = exp(g_min * sigmoid(
- * exp(A_log[h]) * z)). Everything else is kda_decode_step's; the result is
+ * exp(A_log[h]) * z)). flags as for kda_prefill_logits (normalised q, k kept
+ * in fp32). Everything else is kda_decode_step's; with flags 0 the result is
  * bit-identical to kda_bounded_decay (alpha out) followed by kda_decode_step.
  * ------------------------------------------------------------------------- */
 int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                           const float* logits, const float* A_log, float g_min, const float* beta,
+                           const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
                            float* state, int64_t B, int64_t H, int64_t K, int64_t V,
                            const kda_layout* layout, void* o, kda_stream_t stream);
 

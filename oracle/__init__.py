@@ -15,6 +15,11 @@ Functions and the passages they follow:
 * :func:`bounded_decay` -- "Kimi K3: Bounded Decay and Delta Memory",
   Formula and conventions, eq. 5: ``g = g_min * sigmoid(exp(A) * z)``,
   ``alpha = exp(g)``.
+* :func:`l2norm`, :func:`sigmoid` -- the input preparation the surrounding
+  model applies ("KDA cheat sheet", How the inputs are produced: q, k =
+  L2Norm(...), beta = Sigmoid(W_beta x)); they check the scan entry points that
+  do this preparation inside their kernels. L2Norm is read as the unit
+  normalisation of the key axis, guarded by an epsilon of 1e-6 under the root.
 * :func:`scan` -- same page, eq. 1 (fade, correct, then read the updated
   state), with the contract table of that page: q, k ``[B,T,H,K]``, v
   ``[B,T,H,V]``, alpha ``[B,T,H,K]``, beta ``[B,T,H]``, state ``[B,H,K,V]``
@@ -74,6 +79,20 @@ def _ptr(a: np.ndarray):
 def max_threads() -> int:
     """OpenMP threads the oracle uses by default (``OMP_NUM_THREADS`` or all cores)."""
     return int(_load().kda_oracle_max_threads())
+
+
+def l2norm(x, eps: float = 1e-6) -> np.ndarray:
+    """Unit normalisation over the last axis (the key channels of each token and head), in fp64:
+    ``x / sqrt(sum(x^2) + eps)``."""
+    x = _f64(x)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+
+
+def sigmoid(x) -> np.ndarray:
+    """The logistic function in fp64, evaluated without overflow for either sign."""
+    x = _f64(x)
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
 
 
 def bounded_decay(z, A_log, g_min: float = -5.0, return_log: bool = False):

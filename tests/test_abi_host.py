@@ -200,15 +200,25 @@ def test_noalloc_rejects_oversize_before_any_device_call(lib):
 def test_logits_entry_points_reject_bad_gate_arguments(lib):
     layout = Layout(*[Strides(0, 128, 128)] * 4, Strides(0, 1, 1), Strides(0, 128, 128))
     for g_min in (0.0, 1.0, float("nan"), float("inf")):
-        rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, g_min, FAKE, None, None, None, 0,
+        rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, g_min, FAKE, 0, None, None, None, 0,
                                     1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
         assert rc == INVALID and "g_min" in lib.kda_last_error().decode()
-        rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, g_min, FAKE, FAKE, 1, 1, 128, 128,
+        rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, g_min, FAKE, 0, FAKE, 1, 1, 128, 128,
                                         ctypes.byref(layout), FAKE, None)
         assert rc == INVALID and "g_min" in lib.kda_last_error().decode()
-    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, None, -5.0, FAKE, None, None, None, 0,
+    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, None, -5.0, FAKE, 0, None, None, None, 0,
                                 1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
     assert rc == INVALID and "null" in lib.kda_last_error().decode()
-    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, None, -5.0, FAKE, FAKE, 1, 1, 128, 128,
+    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, None, -5.0, FAKE, 0, FAKE, 1, 1, 128, 128,
                                     ctypes.byref(layout), FAKE, None)
     assert rc == INVALID and "null" in lib.kda_last_error().decode()
+
+
+def test_logits_entry_points_reject_unknown_flags(lib):
+    layout = Layout(*[Strides(0, 128, 128)] * 4, Strides(0, 1, 1), Strides(0, 128, 128))
+    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 4, None, None, None, 0,
+                                1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
+    assert rc == INVALID and "flags" in lib.kda_last_error().decode()
+    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 8, FAKE, 1, 1, 128, 128,
+                                    ctypes.byref(layout), FAKE, None)
+    assert rc == INVALID and "flags" in lib.kda_last_error().decode()

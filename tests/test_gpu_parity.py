@@ -459,3 +459,57 @@ def test_decode_logits_equals_gate_then_step(kda, K, V, dtype):
     torch.cuda.synchronize()
     assert not kda.device_status()
     assert torch.equal(o, o_ref) and torch.equal(s_new, s_ref)
+
+
+# ---------------------------------------------------------------------------------------------
+# Input preparation inside the kernels (KDA_QK_L2NORM, KDA_BETA_LOGITS)
+# ---------------------------------------------------------------------------------------------
+# The oracle prepares the raw inputs itself (fp64 L2Norm of q and k over K, sigmoid of the beta
+# logits) and scans; the GPU gets the raw q, k and beta logits. Tolerances as everywhere else.
+
+def oracle_prepared(d, heads=None):
+    sel = (lambda x: x) if heads is None else (lambda x: x[:, :, heads])
+    z, q, k, v, b = (sel(d[n]) for n in ("z", "q", "k", "v", "beta"))
+    A = d["A_log"] if heads is None else d["A_log"][heads]
+    s0 = d["initial_state"]
+    if s0 is not None and heads is not None:
+        s0 = s0[:, heads]
+    alpha = oracle.bounded_decay(z, A, d["g_min"])
+    return oracle.scan(oracle.l2norm(q), oracle.l2norm(k), v, alpha, oracle.sigmoid(b), s0, d["cu_seqlens"])
+
+
+@pytest.mark.parametrize("dtype,use_workspace,cu", [("bf16", True, False), ("bf16", False, False),
+                                                    ("bf16", True, True), ("f32", True, False)],
+                         ids=["bf16-split", "bf16-fused", "bf16-varlen", "f32"])
+def test_prefill_logits_prepares_q_k_beta(kda, dtype, use_workspace, cu):
+    B, T, H, K = (1, 333, 3, 128) if cu else ((2, 200, 3, 128) if dtype == "bf16" else (2, 90, 2, 64))
+    d = W.random_scan_case(B, T, H, K, 128, seed=77, dtype=dtype, z_std=2.0, init_std=0.1, raw_inputs=True)
+    if cu:
+        lens = [100, 0, 64, 169]
+        d["cu_seqlens"] = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+        d["initial_state"] = torch.randn(len(lens), H, K, 128, generator=torch.Generator().manual_seed(5)) * 0.1
+    g = to_dev(d)
+    o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"],
+                               g["initial_state"], g["cu_seqlens"], qk_l2norm=True, beta_logits=True,
+                               use_workspace=use_workspace)
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    ro, rs = oracle_prepared(d)
+    check(o, ro, dtype, "o")
+    check(sf, rs, dtype, "final_state")
+
+
+@pytest.mark.parametrize("K,V,dtype", [(128, 128, "bf16"), (64, 32, "f32")], ids=["bulk", "token-kernel"])
+def test_decode_logits_prepares_q_k_beta(kda, K, V, dtype):
+    d = W.random_scan_case(4, 3, 5, K, V, seed=19, dtype=dtype, z_std=1.0, init_std=0.1, raw_inputs=True)
+    g = to_dev(d)
+    state = g["initial_state"].clone()
+    outs = []
+    for t in range(3):
+        outs.append(kda.decode_step_logits(g["q"][:, t], g["k"][:, t], g["v"][:, t], g["z"][:, t], g["A_log"],
+                                           g["g_min"], g["beta"][:, t], state, qk_l2norm=True, beta_logits=True))
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    ro, rs = oracle_prepared(d)
+    check(torch.stack(outs, dim=1), ro, dtype, "o")
+    check(state, rs, dtype, "state")

@@ -339,3 +339,36 @@ def test_gate_contrast_with_unbounded_softplus_gate():
     unbounded = -np.logaddexp(0.0, z.ravel())                # -softplus, numpy's log-add-exp
     assert unbounded.min() < -10.0 and lg.min() > -5.0
     assert np.all(lg >= -5.0) and np.all(lg <= 0.0)
+
+
+# ---------------------------------------------------------------------------------------------
+# Input preparation ("KDA cheat sheet", How the inputs are produced): L2Norm of q, k; beta = Sigmoid
+# ---------------------------------------------------------------------------------------------
+
+def test_l2norm_pythagorean_rows_and_axis():
+    # Rows (3, 4) and (5, 12) have norms 5 and 13; the epsilon under the root is 1e-6.
+    x = np.array([[[3.0, 4.0], [5.0, 12.0]]])
+    y = oracle.l2norm(x)
+    np.testing.assert_allclose(y[0, 0], np.array([3.0, 4.0]) / np.sqrt(25.0 + 1e-6), rtol=1e-15)
+    np.testing.assert_allclose(y[0, 1], np.array([5.0, 12.0]) / np.sqrt(169.0 + 1e-6), rtol=1e-15)
+    # Normalising over the wrong axis would mix the two rows; each row keeps its direction.
+    assert abs(y[0, 0, 0] / y[0, 0, 1] - 0.75) < 1e-15 and abs(y[0, 1, 0] / y[0, 1, 1] - 5 / 12) < 1e-15
+
+
+def test_l2norm_unit_scale_invariance_and_zero_row():
+    rng = np.random.default_rng(3)
+    x = rng.normal(size=(5, 3, 16))
+    y = oracle.l2norm(x)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), 1.0, atol=1e-6)   # unit rows (up to the epsilon)
+    np.testing.assert_allclose(oracle.l2norm(1e3 * x), y, atol=1e-9)           # scale invariant
+    assert np.all(oracle.l2norm(np.zeros((2, 8))) == 0.0)                      # no NaN for a zero row
+
+
+def test_sigmoid_exact_points_symmetry_and_range():
+    assert oracle.sigmoid(0.0) == 0.5
+    np.testing.assert_allclose(oracle.sigmoid(np.log(3.0)), 0.75, rtol=1e-15)
+    np.testing.assert_allclose(oracle.sigmoid(-np.log(3.0)), 0.25, rtol=1e-15)
+    x = np.linspace(-30, 30, 121)
+    np.testing.assert_allclose(oracle.sigmoid(x) + oracle.sigmoid(-x), 1.0, atol=1e-15)
+    with np.errstate(over="raise", invalid="raise", divide="raise"):  # underflow to 0 is the right answer
+        assert oracle.sigmoid(-800.0) == 0.0 and oracle.sigmoid(800.0) == 1.0

@@ -145,8 +145,19 @@ def make_decode_step(w: DecodeWorkload, step: int) -> dict:
 
 def random_scan_case(B: int, T: int, H: int, K: int, V: int, seed: int, dtype: str = "f32",
                      z_std: float = 1.0, init_std: Optional[float] = 0.1, n_seq: Optional[int] = None,
-                     len_lo: int = 0, len_hi: int = 0) -> dict:
-    """A scan case of arbitrary small sizes with the standard distributions."""
+                     len_lo: int = 0, len_hi: int = 0, raw_inputs: bool = False) -> dict:
+    """A scan case of arbitrary small sizes with the standard distributions.
+
+    With ``raw_inputs`` the case holds what the model has *before* its preparation: q and k are
+    N(0, 2) draws that are not L2-normalised, and ``beta`` holds the N(0,1) logits instead of their
+    sigmoid (for the entry points that prepare q, k and beta inside their kernels)."""
     w = ScanWorkload(f"case_{B}_{T}_{H}_{K}_{V}_{seed}", B, T, H, K, V, dtype=dtype, z_std=z_std,
                      init_std=init_std, n_seq=n_seq, len_lo=len_lo, len_hi=len_hi, seed=seed)
-    return make_scan_inputs(w)
+    d = make_scan_inputs(w)
+    if raw_inputs:
+        g = _gen(seed + 7919)
+        dt = DTYPES[dtype]
+        d["q"] = (torch.randn(d["q"].shape, generator=g) * 2.0).to(dt)
+        d["k"] = (torch.randn(d["k"].shape, generator=g) * 2.0).to(dt)
+        d["beta"] = torch.randn(d["beta"].shape, generator=g)
+    return d
