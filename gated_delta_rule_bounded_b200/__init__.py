@@ -28,7 +28,7 @@ _LIB_PATH = os.path.join(_PKG, "libkda.so")
 
 KDA_F32, KDA_BF16 = 0, 1
 KDA_GATE_ALPHA, KDA_GATE_LOG = 0, 1
-KDA_QK_L2NORM, KDA_BETA_LOGITS = 1, 2
+KDA_QK_L2NORM, KDA_BETA_LOGITS, KDA_STATE_VK = 1, 2, 4
 _STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA"}
 
 
@@ -198,19 +198,20 @@ def _prefill(q, k, v, gate, beta, initial_state, cu_seqlens, gate_is_log, output
         N = n_seq
         cu_ptr = cu_seqlens.data_ptr()
     s0_ptr = None
+    sshape = (N, H, V, K) if (logits is not None and logits[2] & KDA_STATE_VK) else (N, H, K, V)
     if initial_state is not None:
         _cuda(initial_state, "initial_state")
-        if initial_state.shape != (N, H, K, V) or initial_state.dtype != torch.float32 \
+        if initial_state.shape != sshape or initial_state.dtype != torch.float32 \
                 or not initial_state.is_contiguous():
-            raise ValueError(f"initial_state must be a contiguous fp32 [{N},{H},{K},{V}] tensor")
+            raise ValueError(f"initial_state must be a contiguous fp32 {list(sshape)} tensor")
         s0_ptr = initial_state.data_ptr()
     if output_final_state and final_state is None:
-        final_state = torch.empty((N, H, K, V), device=dev, dtype=torch.float32)
+        final_state = torch.empty(sshape, device=dev, dtype=torch.float32)
     sf_ptr = None
     if final_state is not None:
-        if final_state.shape != (N, H, K, V) or final_state.dtype != torch.float32 \
+        if final_state.shape != sshape or final_state.dtype != torch.float32 \
                 or not final_state.is_contiguous():
-            raise ValueError(f"final_state must be a contiguous fp32 [{N},{H},{K},{V}] tensor")
+            raise ValueError(f"final_state must be a contiguous fp32 {list(sshape)} tensor")
         sf_ptr = final_state.data_ptr()
     if out is None:
         out = torch.empty((B, T, H, V), device=dev, dtype=q.dtype)
@@ -257,22 +258,29 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
                     final_state, workspace, use_workspace)
 
 
+def _layout_flag(state_layout: str) -> int:
+    if state_layout not in ("kv", "vk"):
+        raise ValueError('state_layout must be "kv" ([N,H,K,V]) or "vk" ([N,H,V,K])')
+    return KDA_STATE_VK if state_layout == "vk" else 0
+
+
 def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
                    g_min: float, beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
                    cu_seqlens: Optional[torch.Tensor] = None, *, qk_l2norm: bool = False,
-                   beta_logits: bool = False, output_final_state: bool = True,
+                   beta_logits: bool = False, state_layout: str = "kv", output_final_state: bool = True,
                    out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None,
                    use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """``prefill`` fed with the decay logits ``z [B,T,H,K]`` (fp32) instead of alpha: the scan kernels
     evaluate ``g = g_min * sigmoid(exp(A_log[h]) * z)`` themselves (``kda_prefill_logits``).
     ``A_log [H]`` fp32 on the device; ``g_min < 0``. ``qk_l2norm``: the kernels L2-normalise q and k over
-    K per (token, head); ``beta_logits``: ``beta`` holds logits and the kernels apply the sigmoid.
+    K per (token, head); ``beta_logits``: ``beta`` holds logits and the kernels apply the sigmoid;
+    ``state_layout="vk"``: the states are ``[N,H,V,K]`` (value-by-key) instead of ``[N,H,K,V]``.
     Other arguments as in ``prefill``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
-    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
+    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0) | _layout_flag(state_layout)
     return _prefill(q, k, v, z, beta, initial_state, cu_seqlens, False, output_final_state, out, final_state,
                     workspace, use_workspace, logits=(A_log.contiguous(), float(g_min), flags), gate_name="z")
 
@@ -349,8 +357,9 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
         raise TypeError("q, k and v must share one dtype")
     if gate.dtype != torch.float32 or beta.dtype != torch.float32:
         raise TypeError("gate and beta must be fp32")
-    if state.shape != (B, H, K, V) or state.dtype != torch.float32 or not state.is_contiguous():
-        raise ValueError(f"state must be a contiguous fp32 [{B},{H},{K},{V}] tensor")
+    sshape = (B, H, V, K) if (logits is not None and logits[2] & KDA_STATE_VK) else (B, H, K, V)
+    if state.shape != sshape or state.dtype != torch.float32 or not state.is_contiguous():
+        raise ValueError(f"state must be a contiguous fp32 {list(sshape)} tensor")
     q, k, v, gate = map(_rowwise, (q, k, v, gate))
     if out is None:
         out = torch.empty((B, H, V), device=q.device, dtype=q.dtype)
@@ -373,14 +382,15 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
 
 def decode_step_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
                        g_min: float, beta: torch.Tensor, state: torch.Tensor, *, qk_l2norm: bool = False,
-                       beta_logits: bool = False, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                       beta_logits: bool = False, state_layout: str = "kv",
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """``decode_step`` fed with the decay logits ``z [B,H,K]`` (fp32): the step evaluates the bounded gate
-    itself (``kda_decode_step_logits``). ``A_log [H]`` fp32 on the device; ``g_min < 0``; ``qk_l2norm`` and
-    ``beta_logits`` as in ``prefill_logits``."""
+    itself (``kda_decode_step_logits``). ``A_log [H]`` fp32 on the device; ``g_min < 0``; ``qk_l2norm``,
+    ``beta_logits`` and ``state_layout`` (``state`` is ``[B,H,V,K]`` for ``"vk"``) as in ``prefill_logits``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[-2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
-    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
+    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0) | _layout_flag(state_layout)
     return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min), flags))
 
 

@@ -154,14 +154,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
   const uint32_t tlane = tmem + ((uint32_t)(32 * quad) << 16);  // this warp's TMEM lane quadrant
 
   // Initial state: TMEM lane v = trow holds column v of S; this thread moves columns [64*half, +64).
-  const size_t sbase = ((size_t)n * p.H + h) * (size_t)KD * p.V + (size_t)vt * VT;
+  const size_t hbase = ((size_t)n * p.H + h) * (size_t)KD * p.V;  // this head's state
 #pragma unroll
   for (int part = 0; part < 2; ++part) {
     const int cb = 64 * half + 32 * part;
     uint32_t r[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      r[j] = __float_as_uint(p.s0 ? p.s0[sbase + (size_t)(cb + j) * p.V + trow] : 0.f);
+      r[j] = __float_as_uint(p.s0 ? p.s0[state_at(p, hbase, cb + j, vt * VT + trow)] : 0.f);
     tm_st32(tlane + TM_S + cb, r);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
       uint32_t r[32];
       tm_ld32(tlane + TM_S + cb, r);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) p.sf[sbase + (size_t)(cb + j) * p.V + trow] = __uint_as_float(r[j]);
+      for (int j = 0; j < 32; ++j) p.sf[state_at(p, hbase, cb + j, vt * VT + trow)] = __uint_as_float(r[j]);
     }
   }
   if (!ok) {

@@ -383,14 +383,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
   }
 
   // Initial state: TMEM lane v holds column v of S; this thread moves columns [64*half, +64).
-  const size_t sbase = ((size_t)n * p.H + h) * (size_t)KD * p.V + (size_t)vt * VT;
+  const size_t hbase = ((size_t)n * p.H + h) * (size_t)KD * p.V;  // this head's state
 #pragma unroll
   for (int part = 0; part < 2; ++part) {
     const int cb = 64 * half + 32 * part;
     uint32_t r[32];
 #pragma unroll
     for (int jj = 0; jj < 32; ++jj)
-      r[jj] = __float_as_uint(p.s0 ? p.s0[sbase + (size_t)(cb + jj) * p.V + trow] : 0.f);
+      r[jj] = __float_as_uint(p.s0 ? p.s0[state_at(p, hbase, cb + jj, vt * VT + trow)] : 0.f);
     tm_st32(tlane + TM_S + cb, r);
   }
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
       uint32_t r[32];
       tm_ld32(tlane + TM_S + cb, r);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) p.sf[sbase + (size_t)(cb + jj) * p.V + trow] = __uint_as_float(r[jj]);
+      for (int jj = 0; jj < 32; ++jj) p.sf[state_at(p, hbase, cb + jj, vt * VT + trow)] = __uint_as_float(r[jj]);
     }
   }
   if (!ok && tid == 0) {

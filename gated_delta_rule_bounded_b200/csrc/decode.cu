@@ -101,7 +101,8 @@ __device__ __forceinline__ void issue_stage(const ScanParams& p, int head, uint3
   bulk_load(stage_base + L::A, hp.a, DK * 4, bar);
 }
 
-template <typename TIn>
+// VK: the states are stored value-by-key ([V][K]) instead of key-by-value.
+template <typename TIn, bool VK>
 __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
   using L = StageLayout<TIn>;
   extern __shared__ __align__(128) unsigned char sm[];
@@ -151,65 +152,122 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
     }
     float* S = reinterpret_cast<float*>(st + L::STATE);
 
-    float4 x[ROWS];
-    float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
-    float pkq = 0.f, pkk = 0.f, pqq = 0.f;
+    if constexpr (!VK) {
+      float4 x[ROWS];
+      float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+      float pkq = 0.f, pkk = 0.f, pqq = 0.f;
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-      const int row = row0 + r;
-      const float a = as[row], kk = to_f32(ks[row]), qq = to_f32(qs[row]);
-      x[r] = *reinterpret_cast<const float4*>(S + row * DV + col0);
-      x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
-      pa.x = fmaf(kk, x[r].x, pa.x); pa.y = fmaf(kk, x[r].y, pa.y);
-      pa.z = fmaf(kk, x[r].z, pa.z); pa.w = fmaf(kk, x[r].w, pa.w);
-      pb.x = fmaf(qq, x[r].x, pb.x); pb.y = fmaf(qq, x[r].y, pb.y);
-      pb.z = fmaf(qq, x[r].z, pb.z); pb.w = fmaf(qq, x[r].w, pb.w);
-      pkq = fmaf(kk, qq, pkq);
-      pkk = fmaf(kk, kk, pkk);
-      pqq = fmaf(qq, qq, pqq);
-    }
-    *reinterpret_cast<float4*>(red_a + tk * DV + col0) = pa;
-    *reinterpret_cast<float4*>(red_b + tk * DV + col0) = pb;
-    if (tv == 0) {
-      red_kq[tk] = pkq;
-      red_kk[tk] = pkk;
-      red_qq[tk] = pqq;
-    }
-    __syncthreads();
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f), Bq = A;
-    float kq = 0.f, kk2 = 0.f, qq2 = 0.f;
+      for (int r = 0; r < ROWS; ++r) {
+        const int row = row0 + r;
+        const float a = as[row], kk = to_f32(ks[row]), qq = to_f32(qs[row]);
+        x[r] = *reinterpret_cast<const float4*>(S + row * DV + col0);
+        x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
+        pa.x = fmaf(kk, x[r].x, pa.x); pa.y = fmaf(kk, x[r].y, pa.y);
+        pa.z = fmaf(kk, x[r].z, pa.z); pa.w = fmaf(kk, x[r].w, pa.w);
+        pb.x = fmaf(qq, x[r].x, pb.x); pb.y = fmaf(qq, x[r].y, pb.y);
+        pb.z = fmaf(qq, x[r].z, pb.z); pb.w = fmaf(qq, x[r].w, pb.w);
+        pkq = fmaf(kk, qq, pkq);
+        pkk = fmaf(kk, kk, pkk);
+        pqq = fmaf(qq, qq, pqq);
+      }
+      *reinterpret_cast<float4*>(red_a + tk * DV + col0) = pa;
+      *reinterpret_cast<float4*>(red_b + tk * DV + col0) = pb;
+      if (tv == 0) {
+        red_kq[tk] = pkq;
+        red_kk[tk] = pkk;
+        red_qq[tk] = pqq;
+      }
+      __syncthreads();
+      float4 A = make_float4(0.f, 0.f, 0.f, 0.f), Bq = A;
+      float kq = 0.f, kk2 = 0.f, qq2 = 0.f;
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      const float4 ya = *reinterpret_cast<const float4*>(red_a + g * DV + col0);
-      const float4 yb = *reinterpret_cast<const float4*>(red_b + g * DV + col0);
-      A.x += ya.x; A.y += ya.y; A.z += ya.z; A.w += ya.w;
-      Bq.x += yb.x; Bq.y += yb.y; Bq.z += yb.z; Bq.w += yb.w;
-      kq += red_kq[g];
-      kk2 += red_kk[g];
-      qq2 += red_qq[g];
-    }
-    // In-kernel L2 normalisation of k and q: every term is linear in each, so the scales apply to the
-    // sums (k^T S, q^T S, k^T q) and to the rank-1 update.
-    const float ik = p.qk_l2norm ? l2norm_scale(kk2) : 1.f, iq = p.qk_l2norm ? l2norm_scale(qq2) : 1.f;
-    if (p.qk_l2norm) {
-      A.x *= ik; A.y *= ik; A.z *= ik; A.w *= ik;
-      Bq.x *= iq; Bq.y *= iq; Bq.z *= iq; Bq.w *= iq;
-      kq *= ik * iq;
-    }
-    const float4 vv = load4(vs + col0);
-    const float4 d = make_float4(vv.x - A.x, vv.y - A.y, vv.z - A.z, vv.w - A.w);
-    if (tk == 0) {
-      const float bkq = beta * kq;
-      store4(head_ptrs<TIn>(p, head).o + col0, make_float4(fmaf(bkq, d.x, Bq.x), fmaf(bkq, d.y, Bq.y),
-                                                          fmaf(bkq, d.z, Bq.z), fmaf(bkq, d.w, Bq.w)));
-    }
+      for (int g = 0; g < 8; ++g) {
+        const float4 ya = *reinterpret_cast<const float4*>(red_a + g * DV + col0);
+        const float4 yb = *reinterpret_cast<const float4*>(red_b + g * DV + col0);
+        A.x += ya.x; A.y += ya.y; A.z += ya.z; A.w += ya.w;
+        Bq.x += yb.x; Bq.y += yb.y; Bq.z += yb.z; Bq.w += yb.w;
+        kq += red_kq[g];
+        kk2 += red_kk[g];
+        qq2 += red_qq[g];
+      }
+      // In-kernel L2 normalisation of k and q: every term is linear in each, so the scales apply to the
+      // sums (k^T S, q^T S, k^T q) and to the rank-1 update.
+      const float ik = p.qk_l2norm ? l2norm_scale(kk2) : 1.f, iq = p.qk_l2norm ? l2norm_scale(qq2) : 1.f;
+      if (p.qk_l2norm) {
+        A.x *= ik; A.y *= ik; A.z *= ik; A.w *= ik;
+        Bq.x *= iq; Bq.y *= iq; Bq.z *= iq; Bq.w *= iq;
+        kq *= ik * iq;
+      }
+      const float4 vv = load4(vs + col0);
+      const float4 d = make_float4(vv.x - A.x, vv.y - A.y, vv.z - A.z, vv.w - A.w);
+      if (tk == 0) {
+        const float bkq = beta * kq;
+        store4(head_ptrs<TIn>(p, head).o + col0, make_float4(fmaf(bkq, d.x, Bq.x), fmaf(bkq, d.y, Bq.y),
+                                                            fmaf(bkq, d.z, Bq.z), fmaf(bkq, d.w, Bq.w)));
+      }
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-      const int row = row0 + r;
-      const float bk = beta * (to_f32(ks[row]) * ik);
-      x[r].x = fmaf(bk, d.x, x[r].x); x[r].y = fmaf(bk, d.y, x[r].y);
-      x[r].z = fmaf(bk, d.z, x[r].z); x[r].w = fmaf(bk, d.w, x[r].w);
-      *reinterpret_cast<float4*>(S + row * DV + col0) = x[r];
+      for (int r = 0; r < ROWS; ++r) {
+        const int row = row0 + r;
+        const float bk = beta * (to_f32(ks[row]) * ik);
+        x[r].x = fmaf(bk, d.x, x[r].x); x[r].y = fmaf(bk, d.y, x[r].y);
+        x[r].z = fmaf(bk, d.z, x[r].z); x[r].w = fmaf(bk, d.w, x[r].w);
+        *reinterpret_cast<float4*>(S + row * DV + col0) = x[r];
+      }
+    } else {
+      // Value-by-key state, S[v][k]: warp w owns value rows 16w .. 16w+15 and lane l the key columns
+      // 4l .. 4l+3, so a warp reads each row as 512 contiguous bytes. The sums over k are warp
+      // reductions: a reduce-scatter leaves lane l with row 16w + l's k^T Sbar (lanes 0-15) or
+      // q^T Sbar (lanes 16-31), and delta goes back to every lane by shuffles.
+      const int w = tid >> 5, l = tid & 31;
+      const float4 a4 = *reinterpret_cast<const float4*>(as + 4 * l);
+      const float4 k4 = load4(ks + 4 * l), q4 = load4(qs + 4 * l);
+      float4 x[16];
+      float red[32];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        x[r] = *reinterpret_cast<const float4*>(S + (16 * w + r) * DK + 4 * l);
+        x[r].x *= a4.x; x[r].y *= a4.y; x[r].z *= a4.z; x[r].w *= a4.w;
+        red[r] = fmaf(k4.x, x[r].x, fmaf(k4.y, x[r].y, fmaf(k4.z, x[r].z, k4.w * x[r].w)));
+        red[16 + r] = fmaf(q4.x, x[r].x, fmaf(q4.y, x[r].y, fmaf(q4.z, x[r].z, q4.w * x[r].w)));
+      }
+#pragma unroll
+      for (int step = 0; step < 5; ++step) {
+        const int wd = 16 >> step;
+        const bool up = (l & wd) != 0;
+#pragma unroll
+        for (int j = 0; j < wd; ++j) {
+          const float send = up ? red[j] : red[j + wd];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, wd);
+          red[j] = (up ? red[j + wd] : red[j]) + recv;
+        }
+      }
+      float kq = fmaf(k4.x, q4.x, fmaf(k4.y, q4.y, fmaf(k4.z, q4.z, k4.w * q4.w)));
+      float kk2 = fmaf(k4.x, k4.x, fmaf(k4.y, k4.y, fmaf(k4.z, k4.z, k4.w * k4.w)));
+      float qq2 = fmaf(q4.x, q4.x, fmaf(q4.y, q4.y, fmaf(q4.z, q4.z, q4.w * q4.w)));
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) {
+        kq += __shfl_xor_sync(0xffffffffu, kq, m);
+        kk2 += __shfl_xor_sync(0xffffffffu, kk2, m);
+        qq2 += __shfl_xor_sync(0xffffffffu, qq2, m);
+      }
+      const float ik = p.qk_l2norm ? l2norm_scale(kk2) : 1.f, iq = p.qk_l2norm ? l2norm_scale(qq2) : 1.f;
+      const float mine = red[0] * (l < 16 ? ik : iq);  // k^T Sbar (l < 16) or q^T Sbar of row 16w + (l & 15)
+      const float qs_row = __shfl_sync(0xffffffffu, mine, (l + 16) & 31);
+      float delta = 0.f;
+      if (l < 16) {
+        const int vrow = 16 * w + l;
+        delta = to_f32(vs[vrow]) - mine;
+        const float o = fmaf(beta * (kq * ik * iq), delta, qs_row);
+        head_ptrs<TIn>(p, head).o[vrow] = from_f32<TIn>(o);
+      }
+      const float bk = beta * ik;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const float d = __shfl_sync(0xffffffffu, delta, r);
+        x[r].x = fmaf(bk * k4.x, d, x[r].x); x[r].y = fmaf(bk * k4.y, d, x[r].y);
+        x[r].z = fmaf(bk * k4.z, d, x[r].z); x[r].w = fmaf(bk * k4.w, d, x[r].w);
+        *reinterpret_cast<float4*>(S + (16 * w + r) * DK + 4 * l) = x[r];
+      }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();  // the updated state is in shared memory; the partial sums are consumed
@@ -245,7 +303,9 @@ cudaError_t launch_bulk(const ScanParams& p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_relaxed) & bit)) {
-    e = cudaFuncSetAttribute(decode_bulk_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+    e = cudaFuncSetAttribute(decode_bulk_kernel<TIn, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_bulk_kernel<TIn, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
@@ -253,7 +313,10 @@ cudaError_t launch_bulk(const ScanParams& p, cudaStream_t s) {
   const int nheads = p.B * p.H;
   const int grid = nheads < sms ? nheads : sms;
   if (grid == 0) return cudaSuccess;
-  decode_bulk_kernel<TIn><<<grid, DNT, L::SMEM, s>>>(p);
+  if (p.state_vk)
+    decode_bulk_kernel<TIn, true><<<grid, DNT, L::SMEM, s>>>(p);
+  else
+    decode_bulk_kernel<TIn, false><<<grid, DNT, L::SMEM, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -163,7 +163,7 @@ static int check_gate(const char* fn, const GateSpec& gs) {
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, gs.mode);
   if (gs.mode == kda::GATE_LOGITS && (!std::isfinite(gs.g_min) || !(gs.g_min < 0.f)))
     return fail(KDA_ERR_INVALID_ARG, "%s: g_min must be finite and < 0 (got %g)", fn, (double)gs.g_min);
-  if (gs.flags & ~(KDA_QK_L2NORM | KDA_BETA_LOGITS))
+  if (gs.flags & ~(KDA_QK_L2NORM | KDA_BETA_LOGITS | KDA_STATE_VK))
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, gs.flags);
   return KDA_OK;
 }
@@ -264,6 +264,7 @@ static int prefill_impl(const char* fn, const void* q, const void* k, const void
   p.g_min = gs.g_min;
   p.qk_l2norm = (gs.flags & KDA_QK_L2NORM) != 0;
   p.beta_sigmoid = (gs.flags & KDA_BETA_LOGITS) != 0;
+  p.state_vk = (gs.flags & KDA_STATE_VK) != 0;
 
   cudaError_t e;
   if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype)) {
@@ -362,6 +363,7 @@ static int decode_impl(const char* fn, const void* q, const void* k, const void*
   p.g_min = gs.g_min;
   p.qk_l2norm = (gs.flags & KDA_QK_L2NORM) != 0;
   p.beta_sigmoid = (gs.flags & KDA_BETA_LOGITS) != 0;
+  p.state_vk = (gs.flags & KDA_STATE_VK) != 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kda::decode_bulk_supported(p) ? kda::launch_decode_bulk(p, dtype, s) : kda::launch_recurrent(p, dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");

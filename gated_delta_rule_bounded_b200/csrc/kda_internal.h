@@ -32,7 +32,13 @@ struct ScanParams {
   float g_min;          // GATE_LOGITS only
   int qk_l2norm;        // q, k are L2-normalised over K inside the kernels
   int beta_sigmoid;     // beta holds logits; the kernels use sigmoid(beta)
+  int state_vk;         // states stored [N,H,V,K] (K contiguous) instead of [N,H,K,V]
 };
+
+// Offset of state element (key row c, value column v) of a head whose state starts at `head_base`.
+__host__ __device__ inline size_t state_at(const ScanParams& p, size_t head_base, int c, int v) {
+  return p.state_vk ? head_base + (size_t)v * p.K + c : head_base + (size_t)c * p.V + v;
+}
 
 struct GateParams {
   const void* z;

@@ -69,7 +69,15 @@ recurrent_kernel(ScanParams p) {
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
     S[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < rpt && p.s0) S[r] = ld_stream(p.s0 + sbase + (size_t)(row0 + r) * V + col0);
+    if (r < rpt && p.s0) {
+      if (p.state_vk) {  // value-by-key: the four columns are K apart
+        const float* s0 = p.s0 + sbase;
+        S[r] = make_float4(s0[state_at(p, 0, row0 + r, col0)], s0[state_at(p, 0, row0 + r, col0 + 1)],
+                           s0[state_at(p, 0, row0 + r, col0 + 2)], s0[state_at(p, 0, row0 + r, col0 + 3)]);
+      } else {
+        S[r] = ld_stream(p.s0 + sbase + (size_t)(row0 + r) * V + col0);
+      }
+    }
   }
 
   // Double-buffered per-token staging: gate, key, query, value tile, then the
@@ -179,7 +187,17 @@ recurrent_kernel(ScanParams p) {
   if (p.sf) {
 #pragma unroll
     for (int r = 0; r < RPT; ++r)
-      if (r < rpt) st_stream(p.sf + sbase + (size_t)(row0 + r) * V + col0, S[r]);
+      if (r < rpt) {
+        if (p.state_vk) {
+          float* sf = p.sf + sbase;
+          sf[state_at(p, 0, row0 + r, col0)] = S[r].x;
+          sf[state_at(p, 0, row0 + r, col0 + 1)] = S[r].y;
+          sf[state_at(p, 0, row0 + r, col0 + 2)] = S[r].z;
+          sf[state_at(p, 0, row0 + r, col0 + 3)] = S[r].w;
+        } else {
+          st_stream(p.sf + sbase + (size_t)(row0 + r) * V + col0, S[r]);
+        }
+      }
   }
 }
 

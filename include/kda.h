@@ -157,9 +157,14 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  * beta = Sigmoid(W_beta x)).
  *   KDA_QK_L2NORM    q and k are replaced by x / sqrt(sum_c x_c^2 + 1e-6) over
  *                    the K channels of each (token, head) before use.
- *   KDA_BETA_LOGITS  beta holds logits b; the kernels use sigmoid(b). */
+ *   KDA_BETA_LOGITS  beta holds logits b; the kernels use sigmoid(b).
+ *   KDA_STATE_VK     the states (initial, final, decode) are stored
+ *                    value-by-key, [N,H,V,K] with K contiguous (the
+ *                    transpose of the default [N,H,K,V]; "Kept memory": the
+ *                    production cache keeps S this way). */
 #define KDA_QK_L2NORM 1u
 #define KDA_BETA_LOGITS 2u
+#define KDA_STATE_VK 4u
 
 /* ---------------------------------------------------------------------------
  * kda_prefill_logits: kda_prefill with the bounded gate applied inside the
@@ -173,8 +178,8 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  *          uses for alpha / g).
  * A_log    [H] fp32 device pointer; g_min finite and < 0
  *          (else KDA_ERR_INVALID_ARG).
- * flags    0, or KDA_QK_L2NORM and/or KDA_BETA_LOGITS (unknown bits:
- *          KDA_ERR_INVALID_ARG). The chunked bf16 kernels round normalised
+ * flags    0, or any of KDA_QK_L2NORM, KDA_BETA_LOGITS, KDA_STATE_VK
+ *          (unknown bits: KDA_ERR_INVALID_ARG). The chunked bf16 kernels round normalised
  *          q and k to bf16, their operand precision; the fp32 kernel keeps
  *          them in fp32.
  * Every other argument, layout, result, workspace rule and error is

@@ -513,3 +513,42 @@ def test_decode_logits_prepares_q_k_beta(kda, K, V, dtype):
     ro, rs = oracle_prepared(d)
     check(torch.stack(outs, dim=1), ro, dtype, "o")
     check(state, rs, dtype, "state")
+
+
+# ---------------------------------------------------------------------------------------------
+# Value-by-key state layout (KDA_STATE_VK): states [N,H,V,K]
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,use_workspace,K,V", [("bf16", True, 128, 256), ("bf16", False, 128, 128),
+                                                      ("f32", True, 64, 32)],
+                         ids=["bf16-split-V256", "bf16-fused", "f32"])
+def test_prefill_logits_value_by_key_states(kda, dtype, use_workspace, K, V):
+    d = W.random_scan_case(2, 150, 3, K, V, seed=23, dtype=dtype, z_std=2.0, init_std=0.1)
+    g = to_dev(d)
+    s0_vk = g["initial_state"].transpose(-1, -2).contiguous()
+    o, sf_vk = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"], s0_vk,
+                                  state_layout="vk", use_workspace=use_workspace)
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    assert sf_vk.shape == (2, 3, V, K)
+    ro, rs = oracle_pipeline(d)
+    check(o, ro, dtype, "o")
+    check(sf_vk.transpose(-1, -2), rs, dtype, "final_state")
+
+
+@pytest.mark.parametrize("K,V,dtype", [(128, 128, "bf16"), (128, 128, "f32"), (64, 32, "f32")],
+                         ids=["bulk-bf16", "bulk-f32", "token-kernel"])
+def test_decode_logits_value_by_key_state(kda, K, V, dtype):
+    d = W.random_scan_case(4, 3, 5, K, V, seed=31, dtype=dtype, z_std=1.0, init_std=0.1, raw_inputs=True)
+    g = to_dev(d)
+    state_vk = g["initial_state"].transpose(-1, -2).contiguous()
+    outs = []
+    for t in range(3):
+        outs.append(kda.decode_step_logits(g["q"][:, t], g["k"][:, t], g["v"][:, t], g["z"][:, t], g["A_log"],
+                                           g["g_min"], g["beta"][:, t], state_vk, qk_l2norm=True, beta_logits=True,
+                                           state_layout="vk"))
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    ro, rs = oracle_prepared(d)
+    check(torch.stack(outs, dim=1), ro, dtype, "o")
+    check(state_vk.transpose(-1, -2), rs, dtype, "state")
