@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["bounded_decay", "prefill", "prefill_logits", "prefill_noalloc", "decode_step", "decode_step_logits", "prefill_workspace_bytes", "device_status", "KDAError",
+__all__ = ["bounded_decay", "softplus_decay", "prefill", "prefill_logits", "prefill_noalloc", "decode_step", "decode_step_logits", "prefill_workspace_bytes", "device_status", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +28,7 @@ _LIB_PATH = os.path.join(_PKG, "libkda.so")
 
 KDA_F32, KDA_BF16 = 0, 1
 KDA_GATE_ALPHA, KDA_GATE_LOG = 0, 1
-KDA_QK_L2NORM, KDA_BETA_LOGITS, KDA_STATE_VK = 1, 2, 4
+KDA_QK_L2NORM, KDA_BETA_LOGITS, KDA_STATE_VK, KDA_GATE_SOFTPLUS = 1, 2, 4, 8
 _STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA"}
 
 
@@ -68,6 +68,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     sp = ctypes.POINTER(Strides)
     lp = ctypes.POINTER(Layout)
     lib.kda_bounded_decay.argtypes = [vp, sp, i32, vp, ctypes.c_float, i64, i64, i64, i64, vp, sp, i32, vp]
+    lib.kda_softplus_decay.argtypes = [vp, sp, i32, vp, i64, i64, i64, i64, vp, sp, i32, vp]
     lib.kda_prefill_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, i64, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.kda_prefill.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64,
                                 i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
@@ -79,7 +80,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                                        i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, u32, vp, i64, i64, i64, i64,
                                            lp, vp, vp]
-    for fn in ("kda_bounded_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
+    for fn in ("kda_bounded_decay", "kda_softplus_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
                "kda_decode_step", "kda_prefill_logits", "kda_decode_step_logits"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.kda_last_error.restype = ctypes.c_char_p
@@ -138,12 +139,13 @@ def _stream(device: torch.device) -> ctypes.c_void_p:
 
 
 def bounded_decay(logits: torch.Tensor, A_log: torch.Tensor, g_min: float = -5.0, *,
-                  log_decay: bool = False, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                  log_decay: bool = False, out: Optional[torch.Tensor] = None,
+                  _softplus: bool = False) -> torch.Tensor:
     """Retention factors (or log-decays with ``log_decay=True``) for ``logits [B,T,H,K]``."""
     _cuda(logits, "logits")
     if logits.dim() == 3:  # decode-shaped [B,H,K]
         res = bounded_decay(logits.unsqueeze(1), A_log, g_min, log_decay=log_decay,
-                            out=None if out is None else out.unsqueeze(1))
+                            out=None if out is None else out.unsqueeze(1), _softplus=_softplus)
         return res[:, 0]
     if logits.dim() != 4:
         raise ValueError("logits must be [B,T,H,K] or [B,H,K]")
@@ -157,11 +159,23 @@ def bounded_decay(logits: torch.Tensor, A_log: torch.Tensor, g_min: float = -5.0
     _cuda(out, "out")
     zs, os_ = _strides4(logits), _strides4(out)
     lib = load_library()
-    _check("kda_bounded_decay", lib.kda_bounded_decay(
-        logits.data_ptr(), ctypes.byref(zs), _dtype_code(logits.dtype), A_log.data_ptr(),
-        float(g_min), B, T, H, K, out.data_ptr(), ctypes.byref(os_),
-        KDA_GATE_LOG if log_decay else KDA_GATE_ALPHA, _stream(logits.device)))
+    kind = KDA_GATE_LOG if log_decay else KDA_GATE_ALPHA
+    if _softplus:
+        _check("kda_softplus_decay", lib.kda_softplus_decay(
+            logits.data_ptr(), ctypes.byref(zs), _dtype_code(logits.dtype), A_log.data_ptr(),
+            B, T, H, K, out.data_ptr(), ctypes.byref(os_), kind, _stream(logits.device)))
+    else:
+        _check("kda_bounded_decay", lib.kda_bounded_decay(
+            logits.data_ptr(), ctypes.byref(zs), _dtype_code(logits.dtype), A_log.data_ptr(),
+            float(g_min), B, T, H, K, out.data_ptr(), ctypes.byref(os_), kind, _stream(logits.device)))
     return out
+
+
+def softplus_decay(logits: torch.Tensor, A_log: torch.Tensor, *, log_decay: bool = False,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Kimi Linear's unbounded gate (``kda_softplus_decay``): ``g = -exp(A_log[h]) * softplus(logits)``,
+    retention factors ``exp(g)`` (or ``g`` with ``log_decay=True``); shapes as in ``bounded_decay``."""
+    return bounded_decay(logits, A_log, log_decay=log_decay, out=out, _softplus=True)
 
 
 def prefill_workspace_bytes(B: int, T: int, H: int, K: int, V: int, n_seq: int = 0,
@@ -258,6 +272,12 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tenso
                     final_state, workspace, use_workspace)
 
 
+def _gate_flag(gate: str) -> int:
+    if gate not in ("bounded", "softplus"):
+        raise ValueError('gate must be "bounded" (g_min sigmoid) or "softplus" (Kimi Linear)')
+    return KDA_GATE_SOFTPLUS if gate == "softplus" else 0
+
+
 def _layout_flag(state_layout: str) -> int:
     if state_layout not in ("kv", "vk"):
         raise ValueError('state_layout must be "kv" ([N,H,K,V]) or "vk" ([N,H,V,K])')
@@ -267,7 +287,8 @@ def _layout_flag(state_layout: str) -> int:
 def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
                    g_min: float, beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
                    cu_seqlens: Optional[torch.Tensor] = None, *, qk_l2norm: bool = False,
-                   beta_logits: bool = False, state_layout: str = "kv", output_final_state: bool = True,
+                   beta_logits: bool = False, state_layout: str = "kv", gate: str = "bounded",
+                   output_final_state: bool = True,
                    out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None,
                    use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -275,12 +296,14 @@ def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.T
     evaluate ``g = g_min * sigmoid(exp(A_log[h]) * z)`` themselves (``kda_prefill_logits``).
     ``A_log [H]`` fp32 on the device; ``g_min < 0``. ``qk_l2norm``: the kernels L2-normalise q and k over
     K per (token, head); ``beta_logits``: ``beta`` holds logits and the kernels apply the sigmoid;
-    ``state_layout="vk"``: the states are ``[N,H,V,K]`` (value-by-key) instead of ``[N,H,K,V]``.
-    Other arguments as in ``prefill``."""
+    ``state_layout="vk"``: the states are ``[N,H,V,K]`` (value-by-key) instead of ``[N,H,K,V]``;
+    ``gate="softplus"``: the logits feed Kimi Linear's unbounded gate ``g = -exp(A_log) softplus(z)``
+    (``g_min`` unused; the scan then runs token by token). Other arguments as in ``prefill``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
-    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0) | _layout_flag(state_layout)
+    flags = ((KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
+             | _layout_flag(state_layout) | _gate_flag(gate))
     return _prefill(q, k, v, z, beta, initial_state, cu_seqlens, False, output_final_state, out, final_state,
                     workspace, use_workspace, logits=(A_log.contiguous(), float(g_min), flags), gate_name="z")
 
@@ -382,15 +405,17 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
 
 def decode_step_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
                        g_min: float, beta: torch.Tensor, state: torch.Tensor, *, qk_l2norm: bool = False,
-                       beta_logits: bool = False, state_layout: str = "kv",
+                       beta_logits: bool = False, state_layout: str = "kv", gate: str = "bounded",
                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """``decode_step`` fed with the decay logits ``z [B,H,K]`` (fp32): the step evaluates the bounded gate
     itself (``kda_decode_step_logits``). ``A_log [H]`` fp32 on the device; ``g_min < 0``; ``qk_l2norm``,
-    ``beta_logits`` and ``state_layout`` (``state`` is ``[B,H,V,K]`` for ``"vk"``) as in ``prefill_logits``."""
+    ``beta_logits``, ``state_layout`` (``state`` is ``[B,H,V,K]`` for ``"vk"``) and ``gate`` as in
+    ``prefill_logits``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[-2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
-    flags = (KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0) | _layout_flag(state_layout)
+    flags = ((KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
+             | _layout_flag(state_layout) | _gate_flag(gate))
     return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min), flags))
 
 

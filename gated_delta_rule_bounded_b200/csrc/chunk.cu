@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
   const int vt = blk % n_vt;
   blk /= n_vt;
   const int h = blk % p.H;
-  const float gsc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
+  const float gsc = p.gate_mode >= GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int n = blk / p.H;
 
   int64_t t0 = 0, t1 = p.T, brow = n;

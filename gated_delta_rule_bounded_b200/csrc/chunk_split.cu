@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   // after this whole grid has completed (griddepcontrol.wait).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int h = blockIdx.y;
-  const float gsc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
+  const float gsc = p.gate_mode >= GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int64_t slot = blockIdx.x;
   int n, j;
   if (!locate_slot(p, slot, n, j)) return;  // uniform across the CTA

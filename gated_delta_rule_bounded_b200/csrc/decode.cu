@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
 
   for (int i = 0; i < n_my; ++i) {
     const int head = blockIdx.x + i * gridDim.x;
-    const float sc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + head % p.H)) : 0.f;  // e^{A_h}
+    const float sc = p.gate_mode >= GATE_LOGITS ? expf(__ldg(p.A_log + head % p.H)) : 0.f;  // e^{A_h}
     const int s = i % NSTAGE;
     unsigned char* st = sm + s * L::BYTES;
     const float beta = beta_next;

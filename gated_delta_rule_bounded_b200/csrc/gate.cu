@@ -45,10 +45,10 @@ __global__ void __launch_bounds__(256) bounded_decay_kernel(GateParams p) {
         if (r0 + i >= rows) break;
         const float sc = expf(scale[i]);
         float4 g;
-        g.x = bounded_log_decay(sc, z[i].x, p.g_min);
-        g.y = bounded_log_decay(sc, z[i].y, p.g_min);
-        g.z = bounded_log_decay(sc, z[i].z, p.g_min);
-        g.w = bounded_log_decay(sc, z[i].w, p.g_min);
+        g.x = p.softplus ? softplus_log_decay(sc, z[i].x) : bounded_log_decay(sc, z[i].x, p.g_min);
+        g.y = p.softplus ? softplus_log_decay(sc, z[i].y) : bounded_log_decay(sc, z[i].y, p.g_min);
+        g.z = p.softplus ? softplus_log_decay(sc, z[i].z) : bounded_log_decay(sc, z[i].z, p.g_min);
+        g.w = p.softplus ? softplus_log_decay(sc, z[i].w) : bounded_log_decay(sc, z[i].w, p.g_min);
         if (!p.out_log) {
           g.x = expf(g.x);
           g.y = expf(g.y);

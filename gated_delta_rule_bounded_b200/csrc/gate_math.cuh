@@ -22,6 +22,12 @@ __device__ __forceinline__ float gate_sigmoid(float x) {
 // g = g_min * sigmoid(sc * z) with sc = e^{A_h} (computed once per head as expf(A_log[h])).
 __device__ __forceinline__ float bounded_log_decay(float sc, float z, float g_min) { return g_min * gate_sigmoid(sc * z); }
 
+// Kimi Linear's unbounded gate, the contrast of the bounded one on the same page (and the "KDA cheat
+// sheet", g_min table): g = -e^{A_h} softplus(z), softplus(z) = max(z, 0) + log(1 + e^{-|z|}).
+__device__ __forceinline__ float softplus_log_decay(float sc, float z) {
+  return -sc * (fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))));
+}
+
 // The write strength: beta itself, or sigmoid(beta) when the scan receives its logits.
 __device__ __forceinline__ float beta_value(float b, int from_logits) { return from_logits ? gate_sigmoid(b) : b; }
 
@@ -30,6 +36,7 @@ __device__ __forceinline__ float l2norm_scale(float ss) { return rsqrtf(ss + 1e-
 
 // The retention factor alpha of one channel for a scan in gate mode `mode`.
 __device__ __forceinline__ float gate_alpha(int mode, float x, float sc, float g_min) {
+  if (mode == GATE_SOFTPLUS) return expf(softplus_log_decay(sc, x));
   return mode == GATE_LOGITS ? expf(bounded_log_decay(sc, x, g_min)) : (mode == 1 ? expf(x) : x);
 }
 

@@ -95,24 +95,23 @@ int kda_device_status(int* timed_out, int reset) {
   return ok();
 }
 
-int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
-                      const float* A_log, float g_min, int64_t B, int64_t T, int64_t H, int64_t K,
-                      void* out, const kda_strides* out_strides, kda_gate_kind out_kind,
-                      kda_stream_t stream) {
-  if (B < 0 || T < 0 || H < 0 || K < 0) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: negative size");
-  if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: unknown dtype %d", (int)dtype);
+static int gate_impl(const char* fn, const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
+                     const float* A_log, float g_min, bool softplus, int64_t B, int64_t T, int64_t H, int64_t K,
+                     void* out, const kda_strides* out_strides, kda_gate_kind out_kind, kda_stream_t stream) {
+  if (B < 0 || T < 0 || H < 0 || K < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
   if (out_kind != KDA_GATE_ALPHA && out_kind != KDA_GATE_LOG)
-    return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: unknown out_kind %d", (int)out_kind);
-  if (!std::isfinite(g_min) || !(g_min < 0.f))
-    return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: g_min must be finite and < 0 (got %g)", (double)g_min);
+    return fail(KDA_ERR_INVALID_ARG, "%s: unknown out_kind %d", fn, (int)out_kind);
+  if (!softplus && (!std::isfinite(g_min) || !(g_min < 0.f)))
+    return fail(KDA_ERR_INVALID_ARG, "%s: g_min must be finite and < 0 (got %g)", fn, (double)g_min);
   if (B * T * H * K == 0) return ok();
-  if (!logits || !A_log || !out) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: null pointer");
-  if (K % 4 != 0) return fail(KDA_ERR_UNSUPPORTED, "kda_bounded_decay: K must be a multiple of 4 (got %lld)", (long long)K);
+  if (!logits || !A_log || !out) return fail(KDA_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (K % 4 != 0) return fail(KDA_ERR_UNSUPPORTED, "%s: K must be a multiple of 4 (got %lld)", fn, (long long)K);
   if (B * T * H >= (int64_t)INT32_MAX)
-    return fail(KDA_ERR_UNSUPPORTED, "kda_bounded_decay: B*T*H must be below 2^31 rows");
+    return fail(KDA_ERR_UNSUPPORTED, "%s: B*T*H must be below 2^31 rows", fn);
   kda_strides zs = logits_strides ? *logits_strides : contiguous(T, H, K);
   kda_strides os = out_strides ? *out_strides : contiguous(T, H, K);
-  if (!strides_valid(zs) || !strides_valid(os)) return fail(KDA_ERR_INVALID_ARG, "kda_bounded_decay: negative stride");
+  if (!strides_valid(zs) || !strides_valid(os)) return fail(KDA_ERR_INVALID_ARG, "%s: negative stride", fn);
   const size_t es = elem_size(dtype);
   // bf16 rows are read four channels (8 bytes) at a time, fp32 rows 16 bytes.
   auto al = [&](const void* p, const kda_strides& s) {
@@ -120,7 +119,7 @@ int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda
     auto ok_mult = [&](int64_t st, int64_t ext) { return ext <= 1 || (st * (int64_t)es) % (int64_t)need == 0; };
     return (reinterpret_cast<uintptr_t>(p) % need) == 0 && ok_mult(s.b, B) && ok_mult(s.t, T) && ok_mult(s.h, H);
   };
-  if (!al(logits, zs) || !al(out, os)) return fail(KDA_ERR_UNSUPPORTED, "kda_bounded_decay: misaligned rows");
+  if (!al(logits, zs) || !al(out, os)) return fail(KDA_ERR_UNSUPPORTED, "%s: misaligned rows", fn);
   kda::GateParams p;
   p.z = logits;
   p.out = out;
@@ -133,9 +132,26 @@ int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda
   p.K = K;
   p.g_min = g_min;
   p.out_log = out_kind == KDA_GATE_LOG;
+  p.softplus = softplus ? 1 : 0;
   cudaError_t e = kda::launch_gate(p, dtype, reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "kda_bounded_decay launch");
+  if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();
+}
+
+int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
+                      const float* A_log, float g_min, int64_t B, int64_t T, int64_t H, int64_t K,
+                      void* out, const kda_strides* out_strides, kda_gate_kind out_kind,
+                      kda_stream_t stream) {
+  return gate_impl("kda_bounded_decay", logits, logits_strides, dtype, A_log, g_min, false, B, T, H, K, out,
+                   out_strides, out_kind, stream);
+}
+
+int kda_softplus_decay(const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
+                       const float* A_log, int64_t B, int64_t T, int64_t H, int64_t K,
+                       void* out, const kda_strides* out_strides, kda_gate_kind out_kind,
+                       kda_stream_t stream) {
+  return gate_impl("kda_softplus_decay", logits, logits_strides, dtype, A_log, 0.f, true, B, T, H, K, out,
+                   out_strides, out_kind, stream);
 }
 
 int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
@@ -159,11 +175,12 @@ struct GateSpec {
 };
 
 static int check_gate(const char* fn, const GateSpec& gs) {
-  if (gs.mode != KDA_GATE_ALPHA && gs.mode != KDA_GATE_LOG && gs.mode != kda::GATE_LOGITS)
+  if (gs.mode != KDA_GATE_ALPHA && gs.mode != KDA_GATE_LOG && gs.mode != kda::GATE_LOGITS &&
+      gs.mode != kda::GATE_SOFTPLUS)
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, gs.mode);
   if (gs.mode == kda::GATE_LOGITS && (!std::isfinite(gs.g_min) || !(gs.g_min < 0.f)))
     return fail(KDA_ERR_INVALID_ARG, "%s: g_min must be finite and < 0 (got %g)", fn, (double)gs.g_min);
-  if (gs.flags & ~(KDA_QK_L2NORM | KDA_BETA_LOGITS | KDA_STATE_VK))
+  if (gs.flags & ~(KDA_QK_L2NORM | KDA_BETA_LOGITS | KDA_STATE_VK | KDA_GATE_SOFTPLUS))
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, gs.flags);
   return KDA_OK;
 }
@@ -212,7 +229,7 @@ static int prefill_impl(const char* fn, const void* q, const void* k, const void
     }
     return ok();
   }
-  if (!q || !k || !v || !gate || !beta || !o || (gs.mode == kda::GATE_LOGITS && !gs.A_log))
+  if (!q || !k || !v || !gate || !beta || !o || ((gs.mode == kda::GATE_LOGITS || gs.mode == kda::GATE_SOFTPLUS) && !gs.A_log))
     return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
   kda_layout L;
   if (layout) {
@@ -267,7 +284,9 @@ static int prefill_impl(const char* fn, const void* q, const void* k, const void
   p.state_vk = (gs.flags & KDA_STATE_VK) != 0;
 
   cudaError_t e;
-  if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype)) {
+  // The chunked kernels rely on the bounded per-token decay; the unbounded gate takes the exact
+  // token-by-token kernel.
+  if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype) && gs.mode != kda::GATE_SOFTPLUS) {
     if (workspace_bytes > 0 && !workspace) return fail(KDA_ERR_INVALID_ARG, "%s: workspace_bytes > 0 with a null workspace", fn);
     e = kda::launch_chunk(p, workspace, workspace_bytes, s);
   } else {
@@ -298,7 +317,7 @@ int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dt
                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                        const kda_layout* layout, void* o,
                        void* workspace, size_t workspace_bytes, kda_stream_t stream) {
-  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min, flags};
+  const GateSpec gs{logits, (flags & KDA_GATE_SOFTPLUS) ? kda::GATE_SOFTPLUS : kda::GATE_LOGITS, A_log, g_min, flags};
   return prefill_impl("kda_prefill_logits", q, k, v, dtype, gs, beta, initial_state, final_state, cu_seqlens, n_seq, B,
                       T, H, K, V, layout, o, workspace, workspace_bytes, stream);
 }
@@ -312,7 +331,7 @@ static int decode_impl(const char* fn, const void* q, const void* k, const void*
   int rc = check_scan_common(fn, dtype, gs, H, K, V);
   if (rc != KDA_OK) return rc;
   if (B == 0) return ok();
-  if (!q || !k || !v || !gate || !beta || !state || !o || (gs.mode == kda::GATE_LOGITS && !gs.A_log))
+  if (!q || !k || !v || !gate || !beta || !state || !o || ((gs.mode == kda::GATE_LOGITS || gs.mode == kda::GATE_SOFTPLUS) && !gs.A_log))
     return fail(KDA_ERR_INVALID_ARG, "%s: null pointer", fn);
   kda_layout L;
   if (layout) {
@@ -384,7 +403,7 @@ int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtyp
                            const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
                            float* state, int64_t B, int64_t H, int64_t K, int64_t V,
                            const kda_layout* layout, void* o, kda_stream_t stream) {
-  const GateSpec gs{logits, kda::GATE_LOGITS, A_log, g_min, flags};
+  const GateSpec gs{logits, (flags & KDA_GATE_SOFTPLUS) ? kda::GATE_SOFTPLUS : kda::GATE_LOGITS, A_log, g_min, flags};
   return decode_impl("kda_decode_step_logits", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 

@@ -11,6 +11,9 @@ namespace kda {
 // Internal gate mode of a scan, next to KDA_GATE_ALPHA (0) and KDA_GATE_LOG (1): the gate tensor
 // holds the decay logits z, and ScanParams::A_log / g_min complete the bounded gate.
 constexpr int GATE_LOGITS = 2;
+// The gate tensor holds logits z of Kimi Linear's unbounded gate, alpha = exp(-e^{A_h} softplus(z)).
+// Per-token decay is then not bounded below, so scans in this mode take the token-by-token kernel.
+constexpr int GATE_SOFTPLUS = 3;  // both logit modes (>= GATE_LOGITS) use the per-head scale e^{A_h}
 
 // Everything a scan kernel needs, passed by value. Strides are in elements, for
 // the B, T and H dimensions of each token tensor; the innermost dim is contiguous.
@@ -48,6 +51,7 @@ struct GateParams {
   int64_t B, T, H, K;
   float g_min;
   int out_log;
+  int softplus;  // Kimi Linear's unbounded gate instead of the bounded one (g_min unused)
 };
 
 // Launchers return the launch status (cudaGetLastError after the launch).

@@ -48,7 +48,7 @@ recurrent_kernel(ScanParams p) {
   const int vt = blk % n_vt;
   blk /= n_vt;
   const int h = blk % p.H;
-  const float sc = p.gate_mode == GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
+  const float sc = p.gate_mode >= GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int n = blk / p.H;
   const int K = p.K, V = p.V;
   const int rpt = kExact ? RPT : K / kRowGroups;

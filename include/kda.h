@@ -103,6 +103,19 @@ int kda_bounded_decay(const void* logits, const kda_strides* logits_strides, kda
                       kda_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * kda_softplus_decay: Kimi Linear's unbounded gate, the contrast the
+ * bounded-decay page draws (Figure 3(a); "KDA cheat sheet", g_min table):
+ *   g = -exp(A_log[h]) * softplus(logits),  softplus(z) = log(1 + e^z),
+ * out = exp(g) or g as for kda_bounded_decay, whose arguments, layouts and
+ * errors it shares (without g_min). g is unbounded below: alpha can be
+ * arbitrarily close to 0.
+ * ------------------------------------------------------------------------- */
+int kda_softplus_decay(const void* logits, const kda_strides* logits_strides, kda_dtype dtype,
+                       const float* A_log, int64_t B, int64_t T, int64_t H, int64_t K,
+                       void* out, const kda_strides* out_strides, kda_gate_kind out_kind,
+                       kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * kda_prefill_workspace_bytes: bytes of device scratch that let kda_prefill
  * take its two-kernel path for these sizes (0 when no path uses scratch).
  * With bf16 inputs and K = 128, the two-kernel path first computes every
@@ -161,10 +174,16 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  *   KDA_STATE_VK     the states (initial, final, decode) are stored
  *                    value-by-key, [N,H,V,K] with K contiguous (the
  *                    transpose of the default [N,H,K,V]; "Kept memory": the
- *                    production cache keeps S this way). */
+ *                    production cache keeps S this way).
+ *   KDA_GATE_SOFTPLUS the logits feed Kimi Linear's unbounded gate,
+ *                    g = -exp(A_log[h]) * softplus(z) (g_min is ignored),
+ *                    instead of the bounded one. Its per-token decay has no
+ *                    lower bound, so the chunked kernels (which rely on it) are
+ *                    not used: the scan runs token by token (exact, slower). */
 #define KDA_QK_L2NORM 1u
 #define KDA_BETA_LOGITS 2u
 #define KDA_STATE_VK 4u
+#define KDA_GATE_SOFTPLUS 8u
 
 /* ---------------------------------------------------------------------------
  * kda_prefill_logits: kda_prefill with the bounded gate applied inside the
@@ -178,8 +197,8 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  *          uses for alpha / g).
  * A_log    [H] fp32 device pointer; g_min finite and < 0
  *          (else KDA_ERR_INVALID_ARG).
- * flags    0, or any of KDA_QK_L2NORM, KDA_BETA_LOGITS, KDA_STATE_VK
- *          (unknown bits: KDA_ERR_INVALID_ARG). The chunked bf16 kernels round normalised
+ * flags    0, or any of KDA_QK_L2NORM, KDA_BETA_LOGITS, KDA_STATE_VK,
+ *          KDA_GATE_SOFTPLUS (unknown bits: KDA_ERR_INVALID_ARG). The chunked bf16 kernels round normalised
  *          q and k to bf16, their operand precision; the fp32 kernel keeps
  *          them in fp32.
  * Every other argument, layout, result, workspace rule and error is

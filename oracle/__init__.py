@@ -15,6 +15,8 @@ Functions and the passages they follow:
 * :func:`bounded_decay` -- "Kimi K3: Bounded Decay and Delta Memory",
   Formula and conventions, eq. 5: ``g = g_min * sigmoid(exp(A) * z)``,
   ``alpha = exp(g)``.
+* :func:`softplus_decay` -- Kimi Linear's unbounded gate, the contrast drawn in
+  Figure 3(a) of the same page: ``g = -exp(A) * softplus(z)``.
 * :func:`l2norm`, :func:`sigmoid` -- the input preparation the surrounding
   model applies ("KDA cheat sheet", How the inputs are produced: q, k =
   L2Norm(...), beta = Sigmoid(W_beta x)); they check the scan entry points that
@@ -93,6 +95,17 @@ def sigmoid(x) -> np.ndarray:
     x = _f64(x)
     e = np.exp(-np.abs(x))
     return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def softplus_decay(z, A_log, return_log: bool = False):
+    """Kimi Linear's unbounded gate in fp64 ("Kimi K3: Bounded Decay and Delta Memory", Figure 3(a)
+    contrast; "KDA cheat sheet", g_min table): ``g = -exp(A_log[h]) * softplus(z)`` with
+    ``softplus(z) = max(z, 0) + log(1 + exp(-|z|))``; ``alpha = exp(g)``. z ``[B,T,H,K]``."""
+    z = _f64(z)
+    sc = np.exp(_f64(A_log))[None, None, :, None]
+    g = -sc * (np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z))))
+    alpha = np.exp(g)
+    return (alpha, g) if return_log else alpha
 
 
 def bounded_decay(z, A_log, g_min: float = -5.0, return_log: bool = False):

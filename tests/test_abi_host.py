@@ -216,9 +216,9 @@ def test_logits_entry_points_reject_bad_gate_arguments(lib):
 
 def test_logits_entry_points_reject_unknown_flags(lib):
     layout = Layout(*[Strides(0, 128, 128)] * 4, Strides(0, 1, 1), Strides(0, 128, 128))
-    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 8, None, None, None, 0,
+    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 16, None, None, None, 0,
                                 1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
     assert rc == INVALID and "flags" in lib.kda_last_error().decode()
-    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 16, FAKE, 1, 1, 128, 128,
+    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 32, FAKE, 1, 1, 128, 128,
                                     ctypes.byref(layout), FAKE, None)
     assert rc == INVALID and "flags" in lib.kda_last_error().decode()

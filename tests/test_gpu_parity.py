@@ -552,3 +552,50 @@ def test_decode_logits_value_by_key_state(kda, K, V, dtype):
     ro, rs = oracle_prepared(d)
     check(torch.stack(outs, dim=1), ro, dtype, "o")
     check(state_vk.transpose(-1, -2), rs, dtype, "state")
+
+
+# ---------------------------------------------------------------------------------------------
+# Kimi Linear's unbounded gate (KDA_GATE_SOFTPLUS, kda_softplus_decay)
+# ---------------------------------------------------------------------------------------------
+# fp32 gate: |g - g_ref| <= |g_ref| 2^-20 (expf, log1pf and the e^A product, each a few ulp; no argument
+# rounding enters since softplus reads z directly). The scans use the tolerances above.
+
+def oracle_softplus_pipeline(d):
+    alpha = oracle.softplus_decay(d["z"], d["A_log"])
+    return oracle.scan(d["q"], d["k"], d["v"], alpha, d["beta"], d["initial_state"], d["cu_seqlens"])
+
+
+def test_softplus_gate_matches_oracle(kda):
+    d = W.random_scan_case(2, 300, 3, 128, 32, seed=13, dtype="f32", z_std=4.0, init_std=None)
+    g = kda.softplus_decay(d["z"].to(DEV), d["A_log"].to(DEV), log_decay=True)
+    torch.cuda.synchronize()
+    _, ref = oracle.softplus_decay(d["z"], d["A_log"], return_log=True)
+    err = np.abs(g.double().cpu().numpy() - ref)
+    assert np.all(err <= np.abs(ref) * 2.0 ** -20), float((err / np.abs(ref)).max())
+    assert ref.min() < -20.0  # the decay is far below what a bounded gate allows
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_prefill_logits_softplus_gate(kda, dtype):
+    d = W.random_scan_case(2, 150, 3, 128, 128, seed=43, dtype=dtype, z_std=2.0, init_std=0.1)
+    g = to_dev(d)
+    o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"],
+                               g["initial_state"], gate="softplus")
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    ro, rs = oracle_softplus_pipeline(d)
+    check(o, ro, dtype, "o")
+    check(sf, rs, dtype, "final_state")
+
+
+def test_decode_logits_softplus_gate(kda):
+    d = W.random_scan_case(4, 3, 5, 128, 128, seed=47, dtype="bf16", z_std=2.0, init_std=0.1)
+    g = to_dev(d)
+    state = g["initial_state"].clone()
+    outs = [kda.decode_step_logits(g["q"][:, t], g["k"][:, t], g["v"][:, t], g["z"][:, t], g["A_log"], g["g_min"],
+                                   g["beta"][:, t], state, gate="softplus") for t in range(3)]
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    ro, rs = oracle_softplus_pipeline(d)
+    check(torch.stack(outs, dim=1), ro, "bf16", "o")
+    check(state, rs, "bf16", "state")

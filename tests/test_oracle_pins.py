@@ -372,3 +372,34 @@ def test_sigmoid_exact_points_symmetry_and_range():
     np.testing.assert_allclose(oracle.sigmoid(x) + oracle.sigmoid(-x), 1.0, atol=1e-15)
     with np.errstate(over="raise", invalid="raise", divide="raise"):  # underflow to 0 is the right answer
         assert oracle.sigmoid(-800.0) == 0.0 and oracle.sigmoid(800.0) == 1.0
+
+
+# ---------------------------------------------------------------------------------------------
+# Kimi Linear's unbounded gate, g = -e^A softplus(z) (Figure 3(a) contrast; cheat sheet g_min table)
+# ---------------------------------------------------------------------------------------------
+
+def _sp(z, A=0.0):
+    z = np.asarray(z, dtype=np.float64).reshape(1, -1, 1, 1)
+    return oracle.softplus_decay(z, np.array([A]), return_log=True)[1].ravel()
+
+
+def test_softplus_gate_exact_point_and_reflection():
+    assert abs(_sp([0.0])[0] + np.log(2.0)) < 1e-16                     # softplus(0) = ln 2
+    z = np.linspace(-40, 40, 161)
+    np.testing.assert_allclose(_sp(z) - _sp(-z), -z, atol=1e-12)         # softplus(z) - softplus(-z) = z
+
+
+def test_softplus_gate_slope_is_minus_sigmoid_and_scale():
+    z = np.linspace(-12, 12, 97)
+    h = 1e-5
+    slope = (_sp(z + h) - _sp(z - h)) / (2 * h)
+    np.testing.assert_allclose(slope, -oracle.sigmoid(z), atol=1e-9)    # d softplus / dz = sigmoid
+    np.testing.assert_allclose(_sp(z, A=0.7), np.exp(0.7) * _sp(z), rtol=1e-14)
+
+
+def test_softplus_gate_is_unbounded_below_and_stable():
+    g = _sp([10.0, 50.0, 800.0, -50.0])
+    assert g[0] < -10.0 and abs(g[1] + 50.0) < 1e-12 and g[2] == -800.0   # no overflow, no lower bound
+    assert -1e-21 < g[3] < 0.0                                             # -softplus(-50) = -e^-50 (1 - ...)
+    alpha = np.exp(g)
+    assert np.all(alpha <= 1.0) and np.all(alpha >= 0.0)
