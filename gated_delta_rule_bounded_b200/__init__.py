@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["bounded_decay", "softplus_decay", "prefill", "prefill_logits", "prefill_noalloc", "decode_step", "decode_step_logits", "prefill_workspace_bytes", "device_status", "KDAError",
+__all__ = ["bounded_decay", "softplus_decay", "prefill", "prefill_logits", "prefill_noalloc", "scan_backward", "bounded_decay_backward", "decode_step", "decode_step_logits", "prefill_workspace_bytes", "device_status", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -80,6 +80,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                                        i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, u32, vp, i64, i64, i64, i64,
                                            lp, vp, vp]
+    lib.kda_scan_backward_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_scan_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64, i64, i64, i64, i64, lp,
+                                      vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.kda_bounded_decay_backward.argtypes = [vp, vp, ctypes.c_float, vp, i64, i64, i64, i64, vp, vp, vp]
+    for fn in ("kda_scan_backward_workspace_bytes", "kda_scan_backward", "kda_bounded_decay_backward"):
+        getattr(lib, fn).restype = ctypes.c_int
     for fn in ("kda_bounded_decay", "kda_softplus_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
                "kda_decode_step", "kda_prefill_logits", "kda_decode_step_logits"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -417,6 +423,63 @@ def decode_step_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: tor
     flags = ((KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
              | _layout_flag(state_layout) | _gate_flag(gate))
     return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min), flags))
+
+
+def scan_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
+                  initial_state: Optional[torch.Tensor], d_o: torch.Tensor, d_final_state: Optional[torch.Tensor] = None,
+                  *, gate_is_log: bool = False) -> dict:
+    """Gradients of the scan (``kda_scan_backward``): returns fp32 ``dq, dk [B,T,H,K]``, ``dv [B,T,H,V]``,
+    ``dgate`` (dL/dalpha, or dL/dg with ``gate_is_log``), ``dbeta [B,T,H]`` and ``d_initial_state [B,H,K,V]``
+    for ``L = <o, d_o> + <S_T, d_final_state>``. Inputs as for ``prefill`` (no cu_seqlens)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta"), (d_o, "d_o")):
+        _cuda(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B,T,H,K] and v [B,T,H,V]")
+    if gate.shape != q.shape or gate.dtype != torch.float32 or beta.shape != q.shape[:3] or beta.dtype != torch.float32:
+        raise ValueError("gate must be fp32 [B,T,H,K] and beta fp32 [B,T,H]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    dev = q.device
+    q, k, v, gate = map(_rowwise, (q, k, v, gate))
+    d_o = d_o.to(torch.float32).contiguous()
+    if d_o.shape != (B, T, H, V):
+        raise ValueError("d_o must be [B,T,H,V]")
+    f32 = lambda t: None if t is None else t.to(device=dev, dtype=torch.float32).contiguous()  # noqa: E731
+    initial_state, d_final_state = f32(initial_state), f32(d_final_state)
+    for t, n in ((initial_state, "initial_state"), (d_final_state, "d_final_state")):
+        if t is not None and t.shape != (B, H, K, V):
+            raise ValueError(f"{n} must be [{B},{H},{K},{V}]")
+    out = {"dq": torch.empty(B, T, H, K, device=dev), "dk": torch.empty(B, T, H, K, device=dev),
+           "dv": torch.empty(B, T, H, V, device=dev), "dgate": torch.empty(B, T, H, K, device=dev),
+           "dbeta": torch.empty(B, T, H, device=dev), "d_initial_state": torch.empty(B, H, K, V, device=dev)}
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    _check("kda_scan_backward_workspace_bytes", lib.kda_scan_backward_workspace_bytes(B, T, H, K, V, ctypes.byref(n)))
+    ws = torch.empty(max(int(n.value), 16), device=dev, dtype=torch.uint8)
+    layout = Layout(_strides4(q), _strides4(k), _strides4(v), _strides4(gate), _strides3(beta), Strides(0, 0, 0))
+    ptr = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
+    _check("kda_scan_backward", lib.kda_scan_backward(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+        KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), ptr(initial_state), d_o.data_ptr(),
+        ptr(d_final_state), B, T, H, K, V, ctypes.byref(layout), out["dq"].data_ptr(), out["dk"].data_ptr(),
+        out["dv"].data_ptr(), out["dgate"].data_ptr(), out["dbeta"].data_ptr(), out["d_initial_state"].data_ptr(),
+        ws.data_ptr(), ws.numel(), _stream(dev)))
+    return out
+
+
+def bounded_decay_backward(logits: torch.Tensor, A_log: torch.Tensor, g_min: float,
+                           d_log_decay: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """``kda_bounded_decay_backward``: ``(dL/dlogits [B,T,H,K], dL/dA_log [H])`` given ``dL/dg`` (all fp32)."""
+    _cuda(logits, "logits")
+    B, T, H, K = logits.shape
+    z = logits.to(torch.float32).contiguous()
+    dg = d_log_decay.to(device=z.device, dtype=torch.float32).contiguous()
+    A = A_log.to(device=z.device, dtype=torch.float32).contiguous()
+    dz, dA = torch.empty_like(z), torch.empty(H, device=z.device)
+    _check("kda_bounded_decay_backward", load_library().kda_bounded_decay_backward(
+        z.data_ptr(), A.data_ptr(), float(g_min), dg.data_ptr(), B, T, H, K, dz.data_ptr(), dA.data_ptr(),
+        _stream(z.device)))
+    return dz, dA
 
 
 def device_status(reset: bool = True) -> bool:

@@ -407,4 +407,112 @@ int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtyp
   return decode_impl("kda_decode_step_logits", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 
+int kda_scan_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes) {
+  if (!bytes) return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_workspace_bytes: null output");
+  if (B < 0 || T < 0 || H < 0 || K < 0 || V < 0)
+    return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_workspace_bytes: negative size");
+  *bytes = kda::backward_workspace_bytes(B, T, H, K, V);
+  return ok();
+}
+
+int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dtype,
+                      const float* gate, kda_gate_kind gate_kind, const float* beta,
+                      const float* initial_state, const float* d_o, const float* d_final_state,
+                      int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
+                      float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
+                      void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const char* fn = "kda_scan_backward";
+  if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
+    return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, (int)gate_kind);
+  if (!kda::backward_supported((int)K, (int)V))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: K and V must be 16, 32, 64 or 128 (K=%lld, V=%lld)", fn, (long long)K,
+                (long long)V);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B * H == 0) return ok();
+  if (T == 0) {  // nothing to differentiate through: dS_0 = dS_T
+    if (d_initial_state) {
+      cudaError_t e = kda::launch_state_copy(d_final_state, d_initial_state, B * H * K * V, s);
+      if (e != cudaSuccess) return cuda_fail(e, fn);
+    }
+    return ok();
+  }
+  if (!q || !k || !v || !gate || !beta || !d_o || !dq || !dk || !dv || !dgate || !dbeta)
+    return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (T > INT32_MAX) return fail(KDA_ERR_UNSUPPORTED, "%s: T too large", fn);
+  const size_t need = kda::backward_workspace_bytes(B, T, H, K, V);
+  if (!workspace || workspace_bytes < need)
+    return fail(KDA_ERR_INVALID_ARG, "%s: the workspace needs %zu bytes (got %zu)", fn, need, workspace_bytes);
+  kda_layout L;
+  if (layout) {
+    L = *layout;
+  } else {
+    L.q = contiguous(T, H, K);
+    L.k = contiguous(T, H, K);
+    L.gate = contiguous(T, H, K);
+    L.v = contiguous(T, H, V);
+    L.o = contiguous(T, H, V);
+    L.beta = contiguous(T, H, 1);
+  }
+  const kda_strides* all[5] = {&L.q, &L.k, &L.v, &L.gate, &L.beta};
+  for (auto* st : all)
+    if (!strides_valid(*st)) return fail(KDA_ERR_INVALID_ARG, "%s: negative stride", fn);
+  const size_t es = elem_size(dtype);
+  if (!rows_aligned(q, L.q, es, B, T, H) || !rows_aligned(k, L.k, es, B, T, H) ||
+      !rows_aligned(v, L.v, es, B, T, H) || !rows_aligned(gate, L.gate, 4, B, T, H) || !aligned16(d_o) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dgate) || !aligned16(workspace) ||
+      (initial_state && !aligned16(initial_state)) || (d_final_state && !aligned16(d_final_state)) ||
+      (d_initial_state && !aligned16(d_initial_state)))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: rows and buffers must start on 16-byte boundaries", fn);
+  kda::BwdParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.gate = gate;
+  p.beta = beta;
+  p.s0 = initial_state;
+  p.d_o = d_o;
+  p.d_sf = d_final_state;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dgate = dgate;
+  p.dbeta = dbeta;
+  p.ds0 = d_initial_state;
+  const int64_t n_seg = (T + 31) / 32;
+  p.ckpt = static_cast<float*>(workspace);
+  p.scratch = p.ckpt + (size_t)B * H * (n_seg + 1) * K * V;
+  put(p.qs, L.q);
+  put(p.ks, L.k);
+  put(p.vs, L.v);
+  put(p.gs, L.gate);
+  put(p.bs, L.beta);
+  p.T = T;
+  p.B = (int)B;
+  p.H = (int)H;
+  p.K = (int)K;
+  p.V = (int)V;
+  p.gate_log = gate_kind == KDA_GATE_LOG;
+  cudaError_t e = kda::launch_scan_backward(p, dtype, s);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
+int kda_bounded_decay_backward(const float* logits, const float* A_log, float g_min, const float* d_log_decay,
+                               int64_t B, int64_t T, int64_t H, int64_t K, float* d_logits, float* d_A_log,
+                               kda_stream_t stream) {
+  const char* fn = "kda_bounded_decay_backward";
+  if (B < 0 || T < 0 || H < 0 || K < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (!std::isfinite(g_min) || !(g_min < 0.f))
+    return fail(KDA_ERR_INVALID_ARG, "%s: g_min must be finite and < 0 (got %g)", fn, (double)g_min);
+  if (H == 0) return ok();
+  if (!A_log || !d_A_log || (B * T * K > 0 && (!logits || !d_log_decay || !d_logits)))
+    return fail(KDA_ERR_INVALID_ARG, "%s: null pointer", fn);
+  cudaError_t e = kda::launch_bounded_decay_backward(logits, A_log, g_min, d_log_decay, B * T * H, (int)H, (int)K,
+                                                     d_logits, d_A_log, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
 }  // extern "C"

@@ -54,6 +54,32 @@ struct GateParams {
   int softplus;  // Kimi Linear's unbounded gate instead of the bounded one (g_min unused)
 };
 
+// Gradients of the scan (backward.cu). Inputs as for the forward scan (per-element strides for B, T,
+// H); d_o [B,T,H,V], d_sf [B,H,K,V] (or null) and every output fp32 and contiguous.
+struct BwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* gate;  // alpha, or g = log(alpha) when gate_log != 0
+  const float* beta;
+  const float* s0;    // [B,H,K,V] or nullptr (zeros)
+  const float* d_o;
+  const float* d_sf;  // or nullptr (zeros)
+  float *dq, *dk, *dv, *dgate, *dbeta;
+  float* ds0;         // or nullptr (not written)
+  float* ckpt;        // workspace: checkpoints, then the per-CTA segment scratch
+  float* scratch;
+  int64_t qs[3], ks[3], vs[3], gs[3], bs[3];
+  int64_t T;
+  int B, H, K, V;
+  int gate_log;
+};
+bool backward_supported(int K, int V);
+size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V);
+cudaError_t launch_scan_backward(const BwdParams& p, kda_dtype dt, cudaStream_t s);
+cudaError_t launch_bounded_decay_backward(const float* z, const float* A_log, float g_min, const float* dg,
+                                          int64_t rows, int H, int K, float* dz, float* dA, cudaStream_t s);
+
 // Launchers return the launch status (cudaGetLastError after the launch).
 cudaError_t launch_gate(const GateParams& p, kda_dtype dt, cudaStream_t s);
 // Token-by-token kernel: the decode step (T = 1, s0 == sf) and the generic

@@ -280,6 +280,43 @@ int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtyp
                            const kda_layout* layout, void* o, kda_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * kda_scan_backward: gradients of kda_prefill's scan (eq. 1 over whole
+ * sequences) with respect to every input. The pages' contract is
+ * differentiable ("Kimi K3: Bounded Decay and Delta Memory", contract table);
+ * this computes, by the adjoint of the token recurrence,
+ *   dq, dk [B,T,H,K], dv [B,T,H,V], dgate [B,T,H,K] (dL/dalpha for
+ *   KDA_GATE_ALPHA, dL/dg for KDA_GATE_LOG), dbeta [B,T,H] and
+ *   d_initial_state [B,H,K,V] (NULL: not written),
+ * given d_o [B,T,H,V] = dL/do and d_final_state [B,H,K,V] = dL/dS_T (NULL:
+ * zeros). All gradient tensors are fp32 and contiguous; q, k, v, gate, beta
+ * and initial_state are the forward call's inputs (layout strides for q, k, v,
+ * gate, beta as in kda_prefill). Supported: K, V in {16, 32, 64, 128}; no
+ * cu_seqlens (one sequence per batch row). The scan is recomputed from
+ * checkpoints every 32 tokens: the caller passes a workspace of
+ * kda_scan_backward_workspace_bytes (KDA_ERR_INVALID_ARG if smaller). This is
+ * the exact token-by-token adjoint, not a chunked kernel.
+ * ------------------------------------------------------------------------- */
+int kda_scan_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes);
+
+int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dtype,
+                      const float* gate, kda_gate_kind gate_kind, const float* beta,
+                      const float* initial_state, const float* d_o, const float* d_final_state,
+                      int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
+                      float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
+                      void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * kda_bounded_decay_backward: gradients of eq. 5's log-decay
+ * g = g_min * sigmoid(exp(A_log[h]) * z) given d_log_decay = dL/dg:
+ *   d_logits = dL/dz [B,T,H,K], d_A_log = dL/dA_log [H] (overwritten).
+ * All fp32 and contiguous. With kda_scan_backward in KDA_GATE_LOG mode this
+ * completes the chain from the logits.
+ * ------------------------------------------------------------------------- */
+int kda_bounded_decay_backward(const float* logits, const float* A_log, float g_min, const float* d_log_decay,
+                               int64_t B, int64_t T, int64_t H, int64_t K, float* d_logits, float* d_A_log,
+                               kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * kda_device_status: device-side failure flags, for callers that check them
  * after their work has finished. Every wait inside the library's kernels has
  * an iteration limit; a kernel whose wait expires stops, records the event in

@@ -15,6 +15,10 @@ Functions and the passages they follow:
 * :func:`bounded_decay` -- "Kimi K3: Bounded Decay and Delta Memory",
   Formula and conventions, eq. 5: ``g = g_min * sigmoid(exp(A) * z)``,
   ``alpha = exp(g)``.
+* :func:`scan_backward`, :func:`bounded_decay_backward` -- gradients of the
+  scan and of the gate: eq. 1 and eq. 5 restated with plain fp64 PyTorch ops
+  (:func:`scan_torch`) and differentiated by autograd. Pinned by the C
+  oracle's forward values and by finite differences (gradcheck).
 * :func:`softplus_decay` -- Kimi Linear's unbounded gate, the contrast drawn in
   Figure 3(a) of the same page: ``g = -exp(A) * softplus(z)``.
 * :func:`l2norm`, :func:`sigmoid` -- the input preparation the surrounding
@@ -158,3 +162,46 @@ def scan(q, k, v, alpha, beta, initial_state=None, cu_seqlens=None, n_threads: i
     if rc != 0:
         raise ValueError("oracle scan rejected its arguments")
     return o, sf
+
+
+def scan_torch(q, k, v, alpha, beta, initial_state=None):
+    """Eq. 1 token by token with fp64 torch tensors (differentiable): fade, correct, then read.
+    Returns ``(o [B,T,H,V], final_state [B,H,K,V])``."""
+    import torch
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    S = initial_state if initial_state is not None else torch.zeros(B, H, K, V, dtype=torch.float64)
+    outs = []
+    for t in range(T):
+        Sb = alpha[:, t][..., None] * S                                    # Diag(alpha) S
+        delta = v[:, t] - torch.einsum("bhk,bhkv->bhv", k[:, t], Sb)      # v - Sbar^T k
+        S = Sb + beta[:, t][..., None, None] * k[:, t][..., None] * delta[..., None, :]
+        outs.append(torch.einsum("bhk,bhkv->bhv", q[:, t], S))             # S^T q
+    return torch.stack(outs, dim=1), S
+
+
+def scan_backward(q, k, v, alpha, beta, initial_state, d_o, d_final_state=None):
+    """Gradients of ``L = <o, d_o> + <S_T, d_final_state>`` with respect to q, k, v, alpha, beta and the
+    initial state, in fp64 (numpy arrays; ``initial_state`` may be None = zeros)."""
+    import torch
+    t64 = lambda x: torch.tensor(_f64(x), requires_grad=True)  # noqa: E731
+    Q, Kk, Vv, A, Bt = (t64(x) for x in (q, k, v, alpha, beta))
+    S0 = t64(initial_state) if initial_state is not None else torch.zeros(
+        Q.shape[0], Q.shape[2], Q.shape[3], Vv.shape[3], dtype=torch.float64, requires_grad=True)
+    o, sf = scan_torch(Q, Kk, Vv, A, Bt, S0)
+    L = (o * torch.tensor(_f64(d_o))).sum()
+    if d_final_state is not None:
+        L = L + (sf * torch.tensor(_f64(d_final_state))).sum()
+    L.backward()
+    return {n: x.grad.numpy() for n, x in (("q", Q), ("k", Kk), ("v", Vv), ("alpha", A), ("beta", Bt),
+                                              ("initial_state", S0))}
+
+
+def bounded_decay_backward(z, A_log, g_min, d_log_decay):
+    """dL/dz and dL/dA_log of eq. 5's log-decay ``g = g_min * sigmoid(exp(A_log) * z)`` given dL/dg."""
+    import torch
+    Z = torch.tensor(_f64(z), requires_grad=True)
+    Al = torch.tensor(_f64(A_log), requires_grad=True)
+    g = g_min * torch.sigmoid(torch.exp(Al)[None, None, :, None] * Z)
+    (g * torch.tensor(_f64(d_log_decay))).sum().backward()
+    return Z.grad.numpy(), Al.grad.numpy()

@@ -599,3 +599,52 @@ def test_decode_logits_softplus_gate(kda):
     ro, rs = oracle_softplus_pipeline(d)
     check(torch.stack(outs, dim=1), ro, "bf16", "o")
     check(state, rs, "bf16", "state")
+
+
+# ---------------------------------------------------------------------------------------------
+# Gradients: kda_scan_backward, kda_bounded_decay_backward against the fp64 autograd oracle
+# ---------------------------------------------------------------------------------------------
+# The backward kernel works in fp32 for either input dtype (bf16 inputs are exact fp32 values), so one
+# bound serves both: |grad - ref| <= 3e-4 (|ref| + rms(ref)) elementwise, per gradient. A single fp32
+# rounding per operation over a few hundred dependent steps stays far inside it; a wrong term or index
+# does not.
+
+def check_grad(got, ref, what):
+    got = got.detach().double().cpu().numpy()
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} != {ref.shape}"
+    rms = float(np.sqrt(np.mean(ref ** 2))) + 1e-30
+    worst = float((np.abs(got - ref) / (np.abs(ref) + rms)).max())
+    assert worst <= 3e-4, f"{what}: elementwise error {worst:.3e} of (|ref| + rms)"
+
+
+@pytest.mark.parametrize("B,T,H,K,V,dtype,log_gate", [(2, 100, 2, 64, 64, "f32", False),
+                                                       (1, 70, 2, 128, 128, "bf16", True),
+                                                       (2, 33, 3, 32, 16, "f32", True)])
+def test_scan_backward_matches_autograd_oracle(kda, B, T, H, K, V, dtype, log_gate):
+    d = W.random_scan_case(B, T, H, K, V, seed=T + K, dtype=dtype, z_std=2.0, init_std=0.1)
+    gen = torch.Generator().manual_seed(T)
+    do = torch.randn(B, T, H, V, generator=gen)
+    dsf = torch.randn(B, H, K, V, generator=gen) * 0.1
+    alpha, lg = oracle.bounded_decay(d["z"], d["A_log"], d["g_min"], return_log=True)
+    gate = torch.tensor(lg if log_gate else alpha, dtype=torch.float32)
+    gd = to_dev(d)
+    out = kda.scan_backward(gd["q"], gd["k"], gd["v"], gate.to(DEV), gd["beta"], gd["initial_state"], do.to(DEV),
+                            dsf.to(DEV), gate_is_log=log_gate)
+    torch.cuda.synchronize()
+    # the oracle sees exactly the gate values the GPU read
+    a_used = np.exp(gate.double().numpy()) if log_gate else gate.double().numpy()
+    ref = oracle.scan_backward(d["q"], d["k"], d["v"], a_used, d["beta"], d["initial_state"], do, dsf)
+    for n, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("beta", "dbeta"), ("initial_state", "d_initial_state")):
+        check_grad(out[key], ref[n], key)
+    check_grad(out["dgate"], ref["alpha"] * a_used if log_gate else ref["alpha"], "dgate")
+
+
+def test_gate_backward_matches_autograd_oracle(kda):
+    d = W.random_scan_case(2, 50, 3, 64, 16, seed=3, dtype="f32", z_std=2.0, init_std=None)
+    dg = torch.randn(2, 50, 3, 64, generator=torch.Generator().manual_seed(4))
+    dz, dA = kda.bounded_decay_backward(d["z"].to(DEV), d["A_log"].to(DEV), d["g_min"], dg.to(DEV))
+    torch.cuda.synchronize()
+    rz, rA = oracle.bounded_decay_backward(d["z"], d["A_log"], d["g_min"], dg)
+    check_grad(dz, rz, "dz")
+    np.testing.assert_allclose(dA.double().cpu().numpy(), rA, rtol=1e-4, atol=1e-4)

@@ -403,3 +403,54 @@ def test_softplus_gate_is_unbounded_below_and_stable():
     assert -1e-21 < g[3] < 0.0                                             # -softplus(-50) = -e^-50 (1 - ...)
     alpha = np.exp(g)
     assert np.all(alpha <= 1.0) and np.all(alpha >= 0.0)
+
+
+# ---------------------------------------------------------------------------------------------
+# Gradients (the contract is differentiable): the fp64 torch restatement and its autograd
+# ---------------------------------------------------------------------------------------------
+
+def test_torch_scan_equals_c_oracle():
+    import torch
+    rng = np.random.default_rng(8)
+    B, T, H, K, V = 2, 9, 2, 5, 3
+    q, k, v = rng.normal(size=(B, T, H, K)), rng.normal(size=(B, T, H, K)), rng.normal(size=(B, T, H, V))
+    a, b, s0 = rng.uniform(0.1, 1, (B, T, H, K)), rng.uniform(0, 1, (B, T, H)), rng.normal(size=(B, H, K, V))
+    o, sf = oracle.scan_torch(*(torch.tensor(x) for x in (q, k, v, a, b, s0)))
+    ro, rs = oracle.scan(q, k, v, a, b, s0)
+    np.testing.assert_allclose(o.numpy(), ro, atol=1e-12)
+    np.testing.assert_allclose(sf.numpy(), rs, atol=1e-12)
+
+
+def test_scan_gradients_match_finite_differences():
+    import torch
+    rng = np.random.default_rng(9)
+    B, T, H, K, V = 1, 4, 1, 3, 2
+    args = [torch.tensor(x, requires_grad=True) for x in (
+        rng.normal(size=(B, T, H, K)), rng.normal(size=(B, T, H, K)), rng.normal(size=(B, T, H, V)),
+        rng.uniform(0.2, 1, (B, T, H, K)), rng.uniform(0.1, 0.9, (B, T, H)), rng.normal(size=(B, H, K, V)))]
+    do, dsf = rng.normal(size=(B, T, H, V)), rng.normal(size=(B, H, K, V))
+
+    def loss(*a):
+        o, sf = oracle.scan_torch(*a)
+        return (o * torch.tensor(do)).sum() + (sf * torch.tensor(dsf)).sum()
+    assert torch.autograd.gradcheck(loss, args, eps=1e-6, atol=1e-8)
+    g = oracle.scan_backward(*(x.detach().numpy() for x in args), do, dsf)
+    auto = torch.autograd.grad(loss(*args), args)
+    for name, ga in zip(("q", "k", "v", "alpha", "beta", "initial_state"), auto):
+        np.testing.assert_allclose(g[name], ga.numpy(), atol=1e-12)
+
+
+def test_gate_gradients_match_finite_differences():
+    import torch
+    rng = np.random.default_rng(10)
+    z, A = rng.normal(size=(1, 3, 2, 4)), rng.normal(size=2) * 0.5
+    dg = rng.normal(size=(1, 3, 2, 4))
+    dz, dA = oracle.bounded_decay_backward(z, A, -5.0, dg)
+    f = lambda zz, aa: (-5.0 * torch.sigmoid(torch.exp(aa)[None, None, :, None] * zz) * torch.tensor(dg)).sum()  # noqa: E731
+    assert torch.autograd.gradcheck(f, (torch.tensor(z, requires_grad=True), torch.tensor(A, requires_grad=True)))
+    h = 1e-6
+    zp, zm = z.copy(), z.copy()
+    zp[0, 1, 1, 2] += h
+    zm[0, 1, 1, 2] -= h
+    num = (f(torch.tensor(zp), torch.tensor(A)) - f(torch.tensor(zm), torch.tensor(A))).item() / (2 * h)
+    assert abs(num - dz[0, 1, 1, 2]) < 1e-7
