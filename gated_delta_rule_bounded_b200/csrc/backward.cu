@@ -9,7 +9,7 @@
 // and dS_0 = G after the first token. One CTA owns one (batch row, head) and, like the forward
 // token kernel, keeps a K x V state slice in registers (a thread: four consecutive value columns
 // of K/8 key rows). Walking backwards needs S_{t-1} at every t: a forward pass stores the state
-// every R tokens (checkpoints), and each R-token segment is recomputed forward from its checkpoint
+// every kSeg tokens (checkpoints), and each segment is recomputed forward from its checkpoint
 // into a per-CTA scratch before the adjoint sweeps it in reverse. Sums over value columns are
 // shuffles among the threads of a row group; sums over key rows go through shared memory.
 #include "common.cuh"
@@ -267,13 +267,14 @@ __global__ void bounded_decay_backward_kernel(const float* __restrict__ z, const
 
 }  // namespace
 
+int64_t backward_segments(int64_t T) { return (T + kSeg - 1) / kSeg; }
+
 bool backward_supported(int K, int V) {
   return (K == 16 || K == 32 || K == 64 || K == 128) && (V == 16 || V == 32 || V == 64 || V == 128);
 }
 
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V) {
-  const int64_t n_seg = (T + kSeg - 1) / kSeg;
-  return (size_t)B * H * (size_t)(n_seg + 1 + kSeg) * (size_t)K * V * sizeof(float);
+  return (size_t)B * H * (size_t)(backward_segments(T) + 1 + kSeg) * (size_t)K * V * sizeof(float);
 }
 
 cudaError_t launch_scan_backward(const BwdParams& p, kda_dtype dt, cudaStream_t s) {

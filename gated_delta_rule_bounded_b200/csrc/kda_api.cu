@@ -480,7 +480,7 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
   p.dgate = dgate;
   p.dbeta = dbeta;
   p.ds0 = d_initial_state;
-  const int64_t n_seg = (T + 31) / 32;
+  const int64_t n_seg = kda::backward_segments(T);
   p.ckpt = static_cast<float*>(workspace);
   p.scratch = p.ckpt + (size_t)B * H * (n_seg + 1) * K * V;
   put(p.qs, L.q);

@@ -75,6 +75,7 @@ struct BwdParams {
   int gate_log;
 };
 bool backward_supported(int K, int V);
+int64_t backward_segments(int64_t T);  // checkpoint segments; the workspace holds segments + 1 checkpoints
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V);
 cudaError_t launch_scan_backward(const BwdParams& p, kda_dtype dt, cudaStream_t s);
 cudaError_t launch_bounded_decay_backward(const float* z, const float* A_log, float g_min, const float* dg,
