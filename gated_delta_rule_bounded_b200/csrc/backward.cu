@@ -10,8 +10,13 @@
 // token kernel, keeps a K x V state slice in registers (a thread: four consecutive value columns
 // of K/8 key rows). Walking backwards needs S_{t-1} at every t: a forward pass stores the state
 // every kSeg tokens (checkpoints), and each segment is recomputed forward from its checkpoint
-// into a per-CTA scratch before the adjoint sweeps it in reverse. Sums over value columns are
-// shuffles among the threads of a row group; sums over key rows go through shared memory.
+// into a per-CTA scratch before the adjoint sweeps it in reverse.
+//
+// The per-token work is short, so latency decides the speed: every segment's inputs (gate, k, v,
+// beta, and q, do for the adjoint) are brought into shared memory with one batch of asynchronous
+// copies, and during the adjoint the state S_{t-2} is copied from the scratch into a shared-memory
+// ring while token t is processed. Sums over key rows go through shared memory; the per-row sums
+// over value columns (dq, dk, dalpha) are warp reduce-scatters, one shuffle per value and level.
 #include "common.cuh"
 #include "gate_math.cuh"
 #include "kda_internal.h"
@@ -23,13 +28,37 @@ namespace {
 constexpr int kGroups = 8;  // key-row groups
 constexpr int kSeg = 32;    // tokens per checkpoint segment
 
-template <int RPT, int VT>
+constexpr int align16(int x) { return (x + 15) & ~15; }
+
+// Dynamic shared memory (byte offsets): one segment's inputs, the key-row partial sums and the
+// two-slot ring of scratch states (slot, row r, thread: float4).
+template <int RPT, int VT, typename TIn>
 struct BwdSmem {
   static constexpr int K = kGroups * RPT;
-  static constexpr int A = 0, KK = A + K, Q = KK + K, V = Q + K, DO = V + VT, BETA = DO + VT;
-  static constexpr int RED = (BETA + 4 + 3) & ~3;        // [kGroups][VT] column partial sums
-  static constexpr int FLOATS = RED + kGroups * VT;
+  static constexpr int NT = kGroups * (VT / 4);
+  static constexpr int GATE = 0;                                                  // float [kSeg][K]
+  static constexpr int KK = GATE + kSeg * K * 4;                                  // TIn [kSeg][K]
+  static constexpr int Q = align16(KK + kSeg * K * (int)sizeof(TIn));             // TIn [kSeg][K]
+  static constexpr int V = align16(Q + kSeg * K * (int)sizeof(TIn));              // TIn [kSeg][VT]
+  static constexpr int DO = align16(V + kSeg * VT * (int)sizeof(TIn));            // float [kSeg][VT]
+  static constexpr int BETA = DO + kSeg * VT * 4;                                 // float [kSeg]
+  static constexpr int RED = align16(BETA + kSeg * 4);                            // float [kGroups][VT]
+  static constexpr int RING = align16(RED + kGroups * VT * 4);                    // float4 [2][RPT][NT]
+  static constexpr int BYTES = RING + 2 * RPT * NT * 16;
 };
+
+__device__ __forceinline__ uint32_t shared_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(shared_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(shared_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Sum over the VT/4 column-group threads of one row group (consecutive lanes).
 template <int VT>
@@ -37,6 +66,36 @@ __device__ __forceinline__ float rowgroup_sum(float x) {
 #pragma unroll
   for (int m = VT / 8; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
   return x;
+}
+
+// Sums v[r] (r < N, one value per key row of this thread) over the CG threads of the row group.
+// Each level exchanges half of the live values with the partner lane, so afterwards this lane
+// holds the totals of NR = max(1, N / CG) consecutive rows starting at `first` in v[0..NR).
+// With N < CG, CG / N lanes hold the same row; the one whose low bits are zero reports it (`own`).
+template <int N, int CG>
+__device__ __forceinline__ void rowgroup_reduce_scatter(float (&v)[N], int tv, int& first, bool& own) {
+  first = 0;
+  int n = N;
+#pragma unroll
+  for (int m = CG / 2; m >= 1; m >>= 1) {
+    if (n > 1) {
+      const bool up = (tv & m) != 0;
+      const int hn = n / 2;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        if (i < hn) {
+          const float send = up ? v[i] : v[i + hn];
+          const float keep = up ? v[i + hn] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+      if (up) first += hn;
+      n = hn;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+    }
+  }
+  own = N >= CG || (tv & (CG / N - 1)) == 0;
 }
 
 template <int RPT, int VT>
@@ -51,16 +110,19 @@ __device__ __forceinline__ float4 colsum(const float* red, int col0) {
 }
 
 template <int RPT, int VT, typename TIn>
-__global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdParams p) {
-  using L = BwdSmem<RPT, VT>;
-  constexpr int K = L::K, CG = VT / 4, NT = kGroups * CG;
-  __shared__ __align__(16) float sm[L::FLOATS];
-  float* sa = sm + L::A;
-  float* sk = sm + L::KK;
-  float* sq = sm + L::Q;
-  float* sv = sm + L::V;
-  float* sdo = sm + L::DO;
-  float* red = sm + L::RED;
+__global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(BwdParams p) {
+  using L = BwdSmem<RPT, VT, TIn>;
+  constexpr int K = L::K, CG = VT / 4, NT = L::NT;
+  constexpr int NR = RPT > CG ? RPT / CG : 1;  // rows per lane after a reduce-scatter
+  extern __shared__ __align__(16) unsigned char smb[];
+  float* sa = reinterpret_cast<float*>(smb + L::GATE);
+  TIn* sk = reinterpret_cast<TIn*>(smb + L::KK);
+  TIn* sq = reinterpret_cast<TIn*>(smb + L::Q);
+  TIn* sv = reinterpret_cast<TIn*>(smb + L::V);
+  float* sdo = reinterpret_cast<float*>(smb + L::DO);
+  float* sbeta = reinterpret_cast<float*>(smb + L::BETA);
+  float* red = reinterpret_cast<float*>(smb + L::RED);
+  float4* ring = reinterpret_cast<float4*>(smb + L::RING);
 
   const int tid = threadIdx.x, tv = tid % CG, tk = tid / CG;
   const int row0 = tk * RPT, col0 = 4 * tv;
@@ -75,31 +137,46 @@ __global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdPa
   const TIn* vb = static_cast<const TIn*>(p.v);
   auto tile = [&](float* base, int r) { return reinterpret_cast<float4*>(base + (size_t)(row0 + r) * VT + col0); };
 
-  // Stages token t's alpha, k, v, beta (and q, do when `adj`).
-  auto stage = [&](int64_t t, bool adj) {
-    const int64_t ko = b * p.ks[0] + t * p.ks[1] + h * p.ks[2];
-    const int64_t go = b * p.gs[0] + t * p.gs[1] + h * p.gs[2];
-    const int64_t qo = b * p.qs[0] + t * p.qs[1] + h * p.qs[2];
-    const int64_t vo = b * p.vs[0] + t * p.vs[1] + h * p.vs[2];
-    for (int i = tid; i < K; i += NT) {
-      const float gv = __ldg(p.gate + go + i);
-      sa[i] = p.gate_log ? expf(gv) : gv;
-      sk[i] = to_f32(kb[ko + i]);
-      if (adj) sq[i] = to_f32(qb[qo + i]);
+  // Brings tokens t0 .. t0+n-1 into shared memory (q and do as well when `adj`) and turns the gate
+  // into alpha. Every row starts on a 16-byte boundary (checked by the host).
+  auto stage_segment = [&](int64_t t0, int n, bool adj) {
+    constexpr int PK = K * (int)sizeof(TIn) / 16, PV = VT * (int)sizeof(TIn) / 16;  // 16-byte pieces per row
+    for (int i = tid; i < n * (K / 4); i += NT) {
+      const int tt = i / (K / 4), c = 4 * (i % (K / 4));
+      cp_async16(sa + tt * K + c, p.gate + b * p.gs[0] + (t0 + tt) * p.gs[1] + h * p.gs[2] + c);
     }
-    for (int j = tid; j < VT; j += NT) {
-      sv[j] = to_f32(vb[vo + j]);
-      if (adj) sdo[j] = p.d_o[((b * T + t) * p.H + h) * (int64_t)VT + j];
+    for (int i = tid; i < n * PK; i += NT) {
+      const int tt = i / PK, c = (i % PK) * (16 / (int)sizeof(TIn));
+      cp_async16(sk + tt * K + c, kb + b * p.ks[0] + (t0 + tt) * p.ks[1] + h * p.ks[2] + c);
+      if (adj) cp_async16(sq + tt * K + c, qb + b * p.qs[0] + (t0 + tt) * p.qs[1] + h * p.qs[2] + c);
     }
-    if (tid == 0) sm[L::BETA] = __ldg(p.beta + b * p.bs[0] + t * p.bs[1] + h * p.bs[2]);
+    for (int i = tid; i < n * PV; i += NT) {
+      const int tt = i / PV, c = (i % PV) * (16 / (int)sizeof(TIn));
+      cp_async16(sv + tt * VT + c, vb + b * p.vs[0] + (t0 + tt) * p.vs[1] + h * p.vs[2] + c);
+    }
+    if (adj) {
+      for (int i = tid; i < n * (VT / 4); i += NT) {
+        const int tt = i / (VT / 4), c = 4 * (i % (VT / 4));
+        cp_async16(sdo + tt * VT + c, p.d_o + ((b * T + t0 + tt) * p.H + h) * (int64_t)VT + c);
+      }
+    }
+    for (int i = tid; i < n; i += NT) cp_async4(sbeta + i, p.beta + b * p.bs[0] + (t0 + i) * p.bs[1] + h * p.bs[2]);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    if (p.gate_log)
+      for (int i = tid; i < n * K; i += NT) sa[i] = expf(sa[i]);
+    __syncthreads();
   };
 
-  // One forward step on the registers x (S_{t-1} -> S_t); token t already staged.
-  auto forward_step = [&](float4 (&x)[RPT]) {
+  // One forward step on the registers x (S_{t-1} -> S_t) for staged token tt.
+  auto forward_step = [&](float4 (&x)[RPT], int tt) {
+    const float* a_ = sa + tt * K;
+    const TIn* k_ = sk + tt * K;
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-      const float a = sa[row0 + r], kk = sk[row0 + r];
+      const float a = a_[row0 + r], kk = to_f32(k_[row0 + r]);
       x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
       pa.x = fmaf(kk, x[r].x, pa.x); pa.y = fmaf(kk, x[r].y, pa.y);
       pa.z = fmaf(kk, x[r].z, pa.z); pa.w = fmaf(kk, x[r].w, pa.w);
@@ -107,15 +184,17 @@ __global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdPa
     *reinterpret_cast<float4*>(red + tk * VT + col0) = pa;
     __syncthreads();
     const float4 A = colsum<RPT, VT>(red, col0);
-    const float beta = sm[L::BETA];
-    const float4 d = make_float4(sv[col0] - A.x, sv[col0 + 1] - A.y, sv[col0 + 2] - A.z, sv[col0 + 3] - A.w);
+    const float beta = sbeta[tt];
+    const TIn* v_ = sv + tt * VT;
+    const float4 d = make_float4(to_f32(v_[col0]) - A.x, to_f32(v_[col0 + 1]) - A.y, to_f32(v_[col0 + 2]) - A.z,
+                                 to_f32(v_[col0 + 3]) - A.w);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-      const float bk = beta * sk[row0 + r];
+      const float bk = beta * to_f32(k_[row0 + r]);
       x[r].x = fmaf(bk, d.x, x[r].x); x[r].y = fmaf(bk, d.y, x[r].y);
       x[r].z = fmaf(bk, d.z, x[r].z); x[r].w = fmaf(bk, d.w, x[r].w);
     }
-    __syncthreads();  // red and the staged token are free again
+    __syncthreads();  // red is free again
   };
 
   // ---- checkpoints: the state before every kSeg-th token --------------------------------------------
@@ -124,14 +203,14 @@ __global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdPa
 #pragma unroll
   for (int r = 0; r < RPT; ++r) x[r] = p.s0 ? *reinterpret_cast<const float4*>(p.s0 + sbase + (size_t)(row0 + r) * VT + col0)
                                             : make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int64_t t = 0; t < T; ++t) {
-    if (t % kSeg == 0) {
+  for (int seg = 0; seg < n_seg; ++seg) {
+    const int64_t t0 = (int64_t)seg * kSeg;
+    const int n = (int)min((int64_t)kSeg, T - t0);
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) *tile(ckpt + (size_t)(t / kSeg) * slice, r) = x[r];
-    }
-    stage(t, false);
-    __syncthreads();
-    forward_step(x);
+    for (int r = 0; r < RPT; ++r) *tile(ckpt + (size_t)seg * slice, r) = x[r];
+    stage_segment(t0, n, false);
+    for (int tt = 0; tt < n; ++tt) forward_step(x, tt);
+    __syncthreads();  // the staged segment is free again
   }
 
   // ---- adjoint, segment by segment from the end -------------------------------------------------------
@@ -139,32 +218,49 @@ __global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdPa
 #pragma unroll
   for (int r = 0; r < RPT; ++r) G[r] = p.d_sf ? *reinterpret_cast<const float4*>(p.d_sf + sbase + (size_t)(row0 + r) * VT + col0)
                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+  // This thread's float4 of row r in ring slot j (consecutive threads, consecutive 16 bytes).
+  auto ring_at = [&](int j, int r) { return ring + (j * RPT + r) * NT + tid; };
+  auto fetch = [&](int tt) {  // S_{t0+tt-1} from the scratch into ring slot tt & 1
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) cp_async16(ring_at(tt & 1, r), tile(scr + (size_t)tt * slice, r));
+    cp_async_commit();
+  };
   for (int seg = n_seg - 1; seg >= 0; --seg) {
-    const int64_t t0 = (int64_t)seg * kSeg, t1 = min(T, t0 + kSeg);
+    const int64_t t0 = (int64_t)seg * kSeg;
+    const int n = (int)min((int64_t)kSeg, T - t0);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) x[r] = *tile(ckpt + (size_t)seg * slice, r);
-    for (int64_t t = t0; t < t1; ++t) {  // recompute: scr[t - t0] = S_{t-1}
+    stage_segment(t0, n, true);
+    for (int tt = 0; tt < n; ++tt) {  // recompute: scr[tt] = S_{t0+tt-1}
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) *tile(scr + (size_t)(t - t0) * slice, r) = x[r];
-      stage(t, false);
-      __syncthreads();
-      forward_step(x);
+      for (int r = 0; r < RPT; ++r) *tile(scr + (size_t)tt * slice, r) = x[r];
+      forward_step(x, tt);
     }
-    for (int64_t t = t1 - 1; t >= t0; --t) {
-      stage(t, true);
+    fetch(n - 1);  // this thread reads back only what it wrote itself
+    for (int tt = n - 1; tt >= 0; --tt) {
+      const int64_t t = t0 + tt;
+      if (tt > 0) {
+        fetch(tt - 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) x[r] = *tile(scr + (size_t)(t - t0) * slice, r);  // S_{t-1}
-      __syncthreads();
-      const float beta = sm[L::BETA];
+      for (int r = 0; r < RPT; ++r) x[r] = *ring_at(tt & 1, r);  // S_{t-1}
+      const float* a_ = sa + tt * K;
+      const TIn* k_ = sk + tt * K;
+      const TIn* q_ = sq + tt * K;
+      const TIn* v_ = sv + tt * VT;
+      const float beta = sbeta[tt];
       // delta from Sbar = Diag(alpha) S_{t-1} (Sbar is recomputed from S_{t-1} where needed)
       auto sbar = [&](int r) {
-        const float a = sa[row0 + r];
+        const float a = a_[row0 + r];
         return make_float4(a * x[r].x, a * x[r].y, a * x[r].z, a * x[r].w);
       };
       float4 pa = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
-        const float kk = sk[row0 + r];
+        const float kk = to_f32(k_[row0 + r]);
         const float4 xb = sbar(r);
         pa.x = fmaf(kk, xb.x, pa.x); pa.y = fmaf(kk, xb.y, pa.y);
         pa.z = fmaf(kk, xb.z, pa.z); pa.w = fmaf(kk, xb.w, pa.w);
@@ -172,24 +268,35 @@ __global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdPa
       *reinterpret_cast<float4*>(red + tk * VT + col0) = pa;
       __syncthreads();
       const float4 A = colsum<RPT, VT>(red, col0);
-      const float4 d = make_float4(sv[col0] - A.x, sv[col0 + 1] - A.y, sv[col0 + 2] - A.z, sv[col0 + 3] - A.w);
-      const float4 dov = *reinterpret_cast<const float4*>(sdo + col0);
+      const float4 d = make_float4(to_f32(v_[col0]) - A.x, to_f32(v_[col0 + 1]) - A.y, to_f32(v_[col0 + 2]) - A.z,
+                                   to_f32(v_[col0 + 3]) - A.w);
+      const float4 dov = *reinterpret_cast<const float4*>(sdo + tt * VT + col0);
       __syncthreads();  // red is reused below
       // G += q do^T (the output's share), dq = S_t do, and c = G^T k
       float4 pc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float rq[RPT];
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
-        const float qq = sq[row0 + r], kk = sk[row0 + r], bk = beta * kk;
+        const float qq = to_f32(q_[row0 + r]), kk = to_f32(k_[row0 + r]), bk = beta * kk;
         G[r].x = fmaf(qq, dov.x, G[r].x); G[r].y = fmaf(qq, dov.y, G[r].y);
         G[r].z = fmaf(qq, dov.z, G[r].z); G[r].w = fmaf(qq, dov.w, G[r].w);
         const float4 xb = sbar(r);
         const float4 st = make_float4(fmaf(bk, d.x, xb.x), fmaf(bk, d.y, xb.y), fmaf(bk, d.z, xb.z), fmaf(bk, d.w, xb.w));
-        const float dq = rowgroup_sum<VT>(st.x * dov.x + st.y * dov.y + st.z * dov.z + st.w * dov.w);
-        if (tv == 0) p.dq[((b * T + t) * p.H + h) * (int64_t)K + row0 + r] = dq;
+        rq[r] = st.x * dov.x + st.y * dov.y + st.z * dov.z + st.w * dov.w;
         pc.x = fmaf(kk, G[r].x, pc.x); pc.y = fmaf(kk, G[r].y, pc.y);
         pc.z = fmaf(kk, G[r].z, pc.z); pc.w = fmaf(kk, G[r].w, pc.w);
       }
       *reinterpret_cast<float4*>(red + tk * VT + col0) = pc;
+      const int64_t orow = ((b * T + t) * p.H + h) * (int64_t)K + row0;
+      {
+        int first;
+        bool own;
+        rowgroup_reduce_scatter<RPT, CG>(rq, tv, first, own);
+        if (own) {
+#pragma unroll
+          for (int i = 0; i < NR; ++i) p.dq[orow + first + i] = rq[i];
+        }
+      }
       __syncthreads();
       const float4 c = colsum<RPT, VT>(red, col0);
       const float4 dd = make_float4(beta * c.x, beta * c.y, beta * c.z, beta * c.w);  // dL/d delta = dv
@@ -199,23 +306,33 @@ __global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdPa
         *reinterpret_cast<float4*>(p.dv + ((b * T + t) * p.H + h) * (int64_t)VT + col0) = dd;
         if (tv == 0) p.dbeta[(b * T + t) * p.H + h] = db;
       }
+      float rk[RPT], ra[RPT];
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
-        const float kk = sk[row0 + r], a = sa[row0 + r];
+        const float kk = to_f32(k_[row0 + r]), a = a_[row0 + r];
         const float4 xb = sbar(r);
-        const float dk = rowgroup_sum<VT>(beta * (G[r].x * d.x + G[r].y * d.y + G[r].z * d.z + G[r].w * d.w) -
-                                          (xb.x * dd.x + xb.y * dd.y + xb.z * dd.z + xb.w * dd.w));
+        rk[r] = beta * (G[r].x * d.x + G[r].y * d.y + G[r].z * d.z + G[r].w * d.w) -
+                (xb.x * dd.x + xb.y * dd.y + xb.z * dd.z + xb.w * dd.w);
         const float4 ds = make_float4(G[r].x - kk * dd.x, G[r].y - kk * dd.y, G[r].z - kk * dd.z, G[r].w - kk * dd.w);
-        const float da = rowgroup_sum<VT>(ds.x * x[r].x + ds.y * x[r].y + ds.z * x[r].z + ds.w * x[r].w);
-        if (tv == 0) {
-          const int64_t o = ((b * T + t) * p.H + h) * (int64_t)K + row0 + r;
-          p.dk[o] = dk;
-          p.dgate[o] = p.gate_log ? da * a : da;  // dL/dg = dL/dalpha * alpha
-        }
+        ra[r] = ds.x * x[r].x + ds.y * x[r].y + ds.z * x[r].z + ds.w * x[r].w;
         G[r] = make_float4(a * ds.x, a * ds.y, a * ds.z, a * ds.w);
       }
-      __syncthreads();  // red and the staged token are free again
+      {
+        int first;
+        bool own;
+        rowgroup_reduce_scatter<RPT, CG>(rk, tv, first, own);
+        rowgroup_reduce_scatter<RPT, CG>(ra, tv, first, own);
+        if (own) {
+#pragma unroll
+          for (int i = 0; i < NR; ++i) {
+            p.dk[orow + first + i] = rk[i];
+            p.dgate[orow + first + i] = p.gate_log ? ra[i] * a_[row0 + first + i] : ra[i];  // dL/dg = dL/dalpha * alpha
+          }
+        }
+      }
+      __syncthreads();  // red is free again
     }
+    __syncthreads();  // the staged segment is free again
   }
   if (p.ds0) {
 #pragma unroll
@@ -225,7 +342,11 @@ __global__ void __launch_bounds__(kGroups * (VT / 4)) scan_backward_kernel(BwdPa
 
 template <int RPT, int VT, typename TIn>
 cudaError_t launch_b(const BwdParams& p, cudaStream_t s) {
-  scan_backward_kernel<RPT, VT, TIn><<<(unsigned)(p.B * p.H), kGroups * (VT / 4), 0, s>>>(p);
+  constexpr int bytes = BwdSmem<RPT, VT, TIn>::BYTES;
+  static_assert(bytes <= 227 * 1024, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(scan_backward_kernel<RPT, VT, TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  scan_backward_kernel<RPT, VT, TIn><<<(unsigned)(p.B * p.H), kGroups * (VT / 4), bytes, s>>>(p);
   return cudaGetLastError();
 }
 
