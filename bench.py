@@ -351,6 +351,67 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     return res
 
 
+def backward_bytes(B, T, H, K, V, es=2):
+    """Minimum HBM bytes of one backward step from the logits, per token-head: the gate (read z, write g:
+    8K), the scan gradients (read q, k, v in the input dtype, g, beta, dL/do in fp32; write dq, dk, dg, dv,
+    dbeta in fp32) and the gate's gradient (read z and dg, write dz: 12K)."""
+    gate = 8 * K
+    scan = (2 * K + V) * es + 4 * K + 4 + 4 * V + 4 * (3 * K + V) + 4
+    gate_bwd = 12 * K
+    return B * T * H * (gate + scan + gate_bwd)
+
+
+def backward_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
+    """Gradients of the prefill from logits: the log-decay gate, kda_scan_backward and
+    kda_bounded_decay_backward, on the prefill workload with dL/do ~ N(0, 1)."""
+    w = W.PREFILL
+    d = W.make_scan_inputs(w)
+    B, T, H, K, V = w.B, w.T, w.H, w.K, w.V
+    g = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in d.items()}
+    d_o = W.make_output_grad(w).to(dev)
+
+    def bwd_fn():
+        lg = kda.bounded_decay(g["z"], g["A_log"], w.g_min, log_decay=True)
+        grads = kda.scan_backward(g["q"], g["k"], g["v"], lg, g["beta"], None, d_o, gate_is_log=True)
+        kda.bounded_decay_backward(g["z"], g["A_log"], w.g_min, grads["dgate"])
+
+    steps = max(3, min(args.steps, 10))
+    total_ms, (ms,) = timed_loop([bwd_fn], steps, args.warmup, world, stream)
+    value, total_ms = weak_scaling_value(B * T * steps, total_ms, world)
+    nb = backward_bytes(B, T, H, K, V)
+    achieved = nb / (ms / 1e3) / 1e9
+    return {
+        "workload": w.name + "_backward", "value": value, "unit": "tokens/s", "ms_per_step": total_ms / steps,
+        "steps": steps, "gpu_launches": 3 * steps,  # gate, scan gradients, gate gradient
+        "kernels_ms": {"backward_from_logits": ms},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "kernel": "kda_scan_backward (+ gate and gate gradient)",
+                     "bytes_per_launch": nb, "ms_per_launch": ms, "peak_source": f"{peak_src} hbm_gbs",
+                     "note": "token-serial adjoint: latency-bound, one CTA per head"},
+    }
+
+
+def cpu_backward_sample(T=1024, n_heads=8):
+    """Times the fp64 oracle's gradients (gate and scan through autograd) on a slice of the prefill workload;
+    returns tokens/s scaled to all heads of the workload."""
+    import time
+    import oracle
+    w = W.PREFILL
+    d = W.make_scan_inputs(w, T=T)
+    hs = list(range(n_heads))
+    d_o = W.make_output_grad(w, T=T)[:, :, hs].numpy()
+    q, k, v = (d[n][:, :, hs] for n in ("q", "k", "v"))
+    z, A_log, beta = d["z"][:, :, hs], d["A_log"][hs], d["beta"][:, :, hs]
+    t = time.perf_counter()
+    alpha = oracle.bounded_decay(z, A_log, w.g_min)
+    r = oracle.scan_backward(q, k, v, alpha, beta, None, d_o)
+    oracle.bounded_decay_backward(z, A_log, w.g_min, r["alpha"] * alpha)
+    dt = time.perf_counter() - t
+    return {"value": T * n_heads / dt / w.H, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"backward of the prefill workload, {n_heads} of {w.H} heads, first {T} tokens, fp64 autograd; "
+                      f"{dt:.2f} s; tokens/s scaled to all heads"}
+
+
 def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
     dw = W.DECODE
     prm = W.make_decode_params(dw)
@@ -423,7 +484,15 @@ def gpu_arm(args, rank, world, local):
         torch.cuda.empty_cache()
     if args.workload in ("all", "decode"):
         dec = decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
+        torch.cuda.empty_cache()
+    bwd = None
+    if args.workload in ("all", "backward"):
+        bwd = backward_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            bwd["cpu_baseline"] = cpu_backward_sample()
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if pre is None and bwd is not None and dec is None:  # backward-only profiling run
+        return {"metric": METRIC, "workload_only": "backward", "backward": bwd}
     if pre is None:  # decode-only profiling run
         return {"metric": METRIC, "workload_only": "decode", "decode": dec}
     w = pre["workload"]
@@ -452,6 +521,8 @@ def gpu_arm(args, rank, world, local):
     }
     if dec is not None:
         line["decode"] = dec
+    if bwd is not None:
+        line["backward"] = bwd
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line
@@ -526,8 +597,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--cpu-heads", type=int, default=0, help="heads in the oracle sample (0: auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
-                    help="prefill/decode alone (profiling runs); the JSON line needs 'all'")
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "backward"], default="all",
+                    help="one leg alone (profiling runs); the JSON line needs 'all'")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end legs")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -371,18 +371,73 @@ cudaError_t launch_bk(const BwdParams& p, cudaStream_t s) {
 }
 
 // Gate backward: dz = dg * g_min * s (1 - s) * e^A and dA_log[h] += dg * g_min * s (1 - s) * x,
-// with x = e^A z and s = sigmoid(x) (the same device sigmoid as the forward gate).
-__global__ void bounded_decay_backward_kernel(const float* __restrict__ z, const float* __restrict__ A_log,
-                                              float g_min, const float* __restrict__ dg, int64_t rows, int H, int K,
-                                              float* __restrict__ dz, float* __restrict__ dA) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * K; i += (int64_t)gridDim.x * blockDim.x) {
-    const int h = (int)((i / K) % H);
-    const float sc = expf(__ldg(A_log + h));
-    const float x = sc * z[i];
-    const float s = gate_sigmoid(x);
-    const float w = dg[i] * g_min * s * (1.f - s);
-    dz[i] = w * sc;
-    atomicAdd(dA + h, w * x);
+// with x = e^A z and s = sigmoid(x) (the same device sigmoid as the forward gate). One block per
+// (head, slice of the rows); the block sums its share of dA_log[h] and adds it with one atomic.
+template <int VW>
+struct VecF;
+template <>
+struct VecF<1> {
+  using T = float;
+};
+template <>
+struct VecF<4> {
+  using T = float4;
+};
+
+template <int VW>
+__global__ void __launch_bounds__(256) bounded_decay_backward_kernel(const float* __restrict__ z,
+                                                                     const float* __restrict__ A_log, float g_min,
+                                                                     const float* __restrict__ dg, int64_t rows_bt,
+                                                                     int H, int K, float* __restrict__ dz,
+                                                                     float* __restrict__ dA) {
+  using VT = typename VecF<VW>::T;
+  constexpr int U = 4;  // independent elements in flight per thread
+  const int h = blockIdx.x;
+  const int tpr = K / VW;  // vectors per (b, t) row of this head
+  const float sc = expf(__ldg(A_log + h));
+  const int64_t n = rows_bt * tpr, stride = (int64_t)gridDim.y * blockDim.x;
+  float acc = 0.f;
+  for (int64_t e0 = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; e0 < n; e0 += U * stride) {
+    VT zv[U], gv[U];
+    int64_t off[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t e = e0 + u * stride;
+      off[u] = -1;
+      if (e < n) {
+        const int64_t r = e / tpr;
+        off[u] = ((r * H + h) * K) / VW + (e - r * tpr);
+        zv[u] = reinterpret_cast<const VT*>(z)[off[u]];
+        gv[u] = reinterpret_cast<const VT*>(dg)[off[u]];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (off[u] < 0) continue;
+      const float* zf = reinterpret_cast<const float*>(&zv[u]);
+      const float* gf = reinterpret_cast<const float*>(&gv[u]);
+      VT out;
+      float* of = reinterpret_cast<float*>(&out);
+#pragma unroll
+      for (int c = 0; c < VW; ++c) {
+        const float x = sc * zf[c];
+        const float s = gate_sigmoid(x);
+        const float w = gf[c] * g_min * s * (1.f - s);
+        of[c] = w * sc;
+        acc = fmaf(w, x, acc);
+      }
+      reinterpret_cast<VT*>(dz)[off[u]] = out;
+    }
+  }
+  __shared__ float part[8];
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += part[w];
+    atomicAdd(dA + h, t);
   }
 }
 
@@ -403,14 +458,22 @@ cudaError_t launch_scan_backward(const BwdParams& p, kda_dtype dt, cudaStream_t 
 }
 
 cudaError_t launch_bounded_decay_backward(const float* z, const float* A_log, float g_min, const float* dg,
-                                          int64_t rows, int H, int K, float* dz, float* dA, cudaStream_t s) {
+                                          int64_t rows_bt, int H, int K, float* dz, float* dA, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(dA, 0, sizeof(float) * H, s);
   if (e != cudaSuccess) return e;
-  const int64_t n = rows * K;
-  if (n == 0) return cudaSuccess;
-  int64_t grid = (n + 255) / 256;
-  if (grid > 148 * 8) grid = 148 * 8;
-  bounded_decay_backward_kernel<<<(unsigned)grid, 256, 0, s>>>(z, A_log, g_min, dg, rows, H, K, dz, dA);
+  if (rows_bt * K == 0) return cudaSuccess;
+  const bool vec = K % 4 == 0 && ((reinterpret_cast<uintptr_t>(z) | reinterpret_cast<uintptr_t>(dg) |
+                                   reinterpret_cast<uintptr_t>(dz)) & 15) == 0;
+  const int64_t per_head = rows_bt * (vec ? K / 4 : K);
+  int64_t ny = (per_head + 255) / 256;
+  const int64_t cap = (148 * 8 + H - 1) / H;
+  if (ny > cap) ny = cap;
+  if (ny > 65535) ny = 65535;
+  const dim3 grid((unsigned)H, (unsigned)ny);
+  if (vec)
+    bounded_decay_backward_kernel<4><<<grid, 256, 0, s>>>(z, A_log, g_min, dg, rows_bt, H, K, dz, dA);
+  else
+    bounded_decay_backward_kernel<1><<<grid, 256, 0, s>>>(z, A_log, g_min, dg, rows_bt, H, K, dz, dA);
   return cudaGetLastError();
 }
 

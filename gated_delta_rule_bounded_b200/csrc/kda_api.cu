@@ -509,7 +509,7 @@ int kda_bounded_decay_backward(const float* logits, const float* A_log, float g_
   if (H == 0) return ok();
   if (!A_log || !d_A_log || (B * T * K > 0 && (!logits || !d_log_decay || !d_logits)))
     return fail(KDA_ERR_INVALID_ARG, "%s: null pointer", fn);
-  cudaError_t e = kda::launch_bounded_decay_backward(logits, A_log, g_min, d_log_decay, B * T * H, (int)H, (int)K,
+  cudaError_t e = kda::launch_bounded_decay_backward(logits, A_log, g_min, d_log_decay, B * T, (int)H, (int)K,
                                                      d_logits, d_A_log, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return ok();

@@ -79,7 +79,7 @@ int64_t backward_segments(int64_t T);  // checkpoint segments; the workspace hol
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V);
 cudaError_t launch_scan_backward(const BwdParams& p, kda_dtype dt, cudaStream_t s);
 cudaError_t launch_bounded_decay_backward(const float* z, const float* A_log, float g_min, const float* dg,
-                                          int64_t rows, int H, int K, float* dz, float* dA, cudaStream_t s);
+                                          int64_t rows_bt, int H, int K, float* dz, float* dA, cudaStream_t s);
 
 // Launchers return the launch status (cudaGetLastError after the launch).
 cudaError_t launch_gate(const GateParams& p, kda_dtype dt, cudaStream_t s);

@@ -119,6 +119,13 @@ def make_scan_inputs(w: ScanWorkload, T: Optional[int] = None, H: Optional[int] 
                 cu_seqlens=cu, g_min=w.g_min)
 
 
+def make_output_grad(w: ScanWorkload, T: Optional[int] = None, H: Optional[int] = None) -> torch.Tensor:
+    """dL/do ``[B,T,H,V]`` fp32 N(0,1) for the gradient workloads (its own seed, so the scan inputs of
+    the same workload are unchanged)."""
+    g = _gen(w.seed + 1)
+    return torch.randn(w.B, w.T if T is None else T, w.H if H is None else H, w.V, generator=g)
+
+
 def make_decode_params(w: DecodeWorkload) -> dict:
     """Per-head log-scale ``A_log [H]`` and the initial kept state ``[B,H,K,V]`` fp32."""
     g = _gen(w.seed)
