@@ -98,6 +98,30 @@ __device__ __forceinline__ void rowgroup_reduce_scatter(float (&v)[N], int tv, i
   own = N >= CG || (tv & (CG / N - 1)) == 0;
 }
 
+// N consecutive per-row values (N = 2 or 4) from shared memory, as fp32: one vector load. All lanes
+// of a warp read the same rows, so the load is a broadcast.
+template <int N>
+__device__ __forceinline__ void lds_rows(const float* p, float (&r)[N]) {
+  if constexpr (N == 4) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    r[0] = x.x; r[1] = x.y; r[2] = x.z; r[3] = x.w;
+  } else {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    r[0] = x.x; r[1] = x.y;
+  }
+}
+template <int N>
+__device__ __forceinline__ void lds_rows(const __nv_bfloat16* p, float (&r)[N]) {
+  if constexpr (N == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    r[0] = __uint_as_float(x.x << 16); r[1] = __uint_as_float(x.x & 0xffff0000u);
+    r[2] = __uint_as_float(x.y << 16); r[3] = __uint_as_float(x.y & 0xffff0000u);
+  } else {
+    const uint32_t x = *reinterpret_cast<const uint32_t*>(p);
+    r[0] = __uint_as_float(x << 16); r[1] = __uint_as_float(x & 0xffff0000u);
+  }
+}
+
 template <int RPT, int VT>
 __device__ __forceinline__ float4 colsum(const float* red, int col0) {
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -114,6 +138,7 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
   using L = BwdSmem<RPT, VT, TIn>;
   constexpr int K = L::K, CG = VT / 4, NT = L::NT;
   constexpr int NR = RPT > CG ? RPT / CG : 1;  // rows per lane after a reduce-scatter
+  constexpr int RG = RPT >= 4 ? 4 : RPT;       // rows per vector load of the per-row values
   extern __shared__ __align__(16) unsigned char smb[];
   float* sa = reinterpret_cast<float*>(smb + L::GATE);
   TIn* sk = reinterpret_cast<TIn*>(smb + L::KK);
@@ -171,15 +196,22 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
 
   // One forward step on the registers x (S_{t-1} -> S_t) for staged token tt.
   auto forward_step = [&](float4 (&x)[RPT], int tt) {
-    const float* a_ = sa + tt * K;
-    const TIn* k_ = sk + tt * K;
+    const float* a_ = sa + tt * K + row0;
+    const TIn* k_ = sk + tt * K + row0;
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const float a = a_[row0 + r], kk = to_f32(k_[row0 + r]);
-      x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
-      pa.x = fmaf(kk, x[r].x, pa.x); pa.y = fmaf(kk, x[r].y, pa.y);
-      pa.z = fmaf(kk, x[r].z, pa.z); pa.w = fmaf(kk, x[r].w, pa.w);
+    for (int rr = 0; rr < RPT; rr += RG) {
+      float av[RG], kv[RG];
+      lds_rows<RG>(a_ + rr, av);
+      lds_rows<RG>(k_ + rr, kv);
+#pragma unroll
+      for (int j = 0; j < RG; ++j) {
+        const int r = rr + j;
+        const float a = av[j], kk = kv[j];
+        x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
+        pa.x = fmaf(kk, x[r].x, pa.x); pa.y = fmaf(kk, x[r].y, pa.y);
+        pa.z = fmaf(kk, x[r].z, pa.z); pa.w = fmaf(kk, x[r].w, pa.w);
+      }
     }
     *reinterpret_cast<float4*>(red + tk * VT + col0) = pa;
     __syncthreads();
@@ -189,10 +221,16 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
     const float4 d = make_float4(to_f32(v_[col0]) - A.x, to_f32(v_[col0 + 1]) - A.y, to_f32(v_[col0 + 2]) - A.z,
                                  to_f32(v_[col0 + 3]) - A.w);
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const float bk = beta * to_f32(k_[row0 + r]);
-      x[r].x = fmaf(bk, d.x, x[r].x); x[r].y = fmaf(bk, d.y, x[r].y);
-      x[r].z = fmaf(bk, d.z, x[r].z); x[r].w = fmaf(bk, d.w, x[r].w);
+    for (int rr = 0; rr < RPT; rr += RG) {
+      float kv[RG];
+      lds_rows<RG>(k_ + rr, kv);
+#pragma unroll
+      for (int j = 0; j < RG; ++j) {
+        const int r = rr + j;
+        const float bk = beta * kv[j];
+        x[r].x = fmaf(bk, d.x, x[r].x); x[r].y = fmaf(bk, d.y, x[r].y);
+        x[r].z = fmaf(bk, d.z, x[r].z); x[r].w = fmaf(bk, d.w, x[r].w);
+      }
     }
     __syncthreads();  // red is free again
   };
@@ -247,23 +285,27 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
       }
 #pragma unroll
       for (int r = 0; r < RPT; ++r) x[r] = *ring_at(tt & 1, r);  // S_{t-1}
-      const float* a_ = sa + tt * K;
-      const TIn* k_ = sk + tt * K;
-      const TIn* q_ = sq + tt * K;
+      const float* a_ = sa + tt * K + row0;
+      const TIn* k_ = sk + tt * K + row0;
+      const TIn* q_ = sq + tt * K + row0;
       const TIn* v_ = sv + tt * VT;
       const float beta = sbeta[tt];
       // delta from Sbar = Diag(alpha) S_{t-1} (Sbar is recomputed from S_{t-1} where needed)
-      auto sbar = [&](int r) {
-        const float a = a_[row0 + r];
-        return make_float4(a * x[r].x, a * x[r].y, a * x[r].z, a * x[r].w);
-      };
+      auto sbar = [&](int r, float a) { return make_float4(a * x[r].x, a * x[r].y, a * x[r].z, a * x[r].w); };
       float4 pa = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        const float kk = to_f32(k_[row0 + r]);
-        const float4 xb = sbar(r);
-        pa.x = fmaf(kk, xb.x, pa.x); pa.y = fmaf(kk, xb.y, pa.y);
-        pa.z = fmaf(kk, xb.z, pa.z); pa.w = fmaf(kk, xb.w, pa.w);
+      for (int rr = 0; rr < RPT; rr += RG) {
+        float av[RG], kv[RG];
+        lds_rows<RG>(a_ + rr, av);
+        lds_rows<RG>(k_ + rr, kv);
+#pragma unroll
+        for (int j = 0; j < RG; ++j) {
+          const int r = rr + j;
+          const float kk = kv[j];
+          const float4 xb = sbar(r, av[j]);
+          pa.x = fmaf(kk, xb.x, pa.x); pa.y = fmaf(kk, xb.y, pa.y);
+          pa.z = fmaf(kk, xb.z, pa.z); pa.w = fmaf(kk, xb.w, pa.w);
+        }
       }
       *reinterpret_cast<float4*>(red + tk * VT + col0) = pa;
       __syncthreads();
@@ -276,15 +318,23 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
       float4 pc = make_float4(0.f, 0.f, 0.f, 0.f);
       float rq[RPT];
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        const float qq = to_f32(q_[row0 + r]), kk = to_f32(k_[row0 + r]), bk = beta * kk;
-        G[r].x = fmaf(qq, dov.x, G[r].x); G[r].y = fmaf(qq, dov.y, G[r].y);
-        G[r].z = fmaf(qq, dov.z, G[r].z); G[r].w = fmaf(qq, dov.w, G[r].w);
-        const float4 xb = sbar(r);
-        const float4 st = make_float4(fmaf(bk, d.x, xb.x), fmaf(bk, d.y, xb.y), fmaf(bk, d.z, xb.z), fmaf(bk, d.w, xb.w));
-        rq[r] = st.x * dov.x + st.y * dov.y + st.z * dov.z + st.w * dov.w;
-        pc.x = fmaf(kk, G[r].x, pc.x); pc.y = fmaf(kk, G[r].y, pc.y);
-        pc.z = fmaf(kk, G[r].z, pc.z); pc.w = fmaf(kk, G[r].w, pc.w);
+      for (int rr = 0; rr < RPT; rr += RG) {
+        float av[RG], kv[RG], qv[RG];
+        lds_rows<RG>(a_ + rr, av);
+        lds_rows<RG>(k_ + rr, kv);
+        lds_rows<RG>(q_ + rr, qv);
+#pragma unroll
+        for (int j = 0; j < RG; ++j) {
+          const int r = rr + j;
+          const float qq = qv[j], kk = kv[j], bk = beta * kk;
+          G[r].x = fmaf(qq, dov.x, G[r].x); G[r].y = fmaf(qq, dov.y, G[r].y);
+          G[r].z = fmaf(qq, dov.z, G[r].z); G[r].w = fmaf(qq, dov.w, G[r].w);
+          const float4 xb = sbar(r, av[j]);
+          const float4 st = make_float4(fmaf(bk, d.x, xb.x), fmaf(bk, d.y, xb.y), fmaf(bk, d.z, xb.z), fmaf(bk, d.w, xb.w));
+          rq[r] = st.x * dov.x + st.y * dov.y + st.z * dov.z + st.w * dov.w;
+          pc.x = fmaf(kk, G[r].x, pc.x); pc.y = fmaf(kk, G[r].y, pc.y);
+          pc.z = fmaf(kk, G[r].z, pc.z); pc.w = fmaf(kk, G[r].w, pc.w);
+        }
       }
       *reinterpret_cast<float4*>(red + tk * VT + col0) = pc;
       const int64_t orow = ((b * T + t) * p.H + h) * (int64_t)K + row0;
@@ -308,14 +358,21 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
       }
       float rk[RPT], ra[RPT];
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        const float kk = to_f32(k_[row0 + r]), a = a_[row0 + r];
-        const float4 xb = sbar(r);
-        rk[r] = beta * (G[r].x * d.x + G[r].y * d.y + G[r].z * d.z + G[r].w * d.w) -
-                (xb.x * dd.x + xb.y * dd.y + xb.z * dd.z + xb.w * dd.w);
-        const float4 ds = make_float4(G[r].x - kk * dd.x, G[r].y - kk * dd.y, G[r].z - kk * dd.z, G[r].w - kk * dd.w);
-        ra[r] = ds.x * x[r].x + ds.y * x[r].y + ds.z * x[r].z + ds.w * x[r].w;
-        G[r] = make_float4(a * ds.x, a * ds.y, a * ds.z, a * ds.w);
+      for (int rr = 0; rr < RPT; rr += RG) {
+        float av[RG], kv[RG];
+        lds_rows<RG>(a_ + rr, av);
+        lds_rows<RG>(k_ + rr, kv);
+#pragma unroll
+        for (int j = 0; j < RG; ++j) {
+          const int r = rr + j;
+          const float kk = kv[j], a = av[j];
+          const float4 xb = sbar(r, a);
+          rk[r] = beta * (G[r].x * d.x + G[r].y * d.y + G[r].z * d.z + G[r].w * d.w) -
+                  (xb.x * dd.x + xb.y * dd.y + xb.z * dd.z + xb.w * dd.w);
+          const float4 ds = make_float4(G[r].x - kk * dd.x, G[r].y - kk * dd.y, G[r].z - kk * dd.z, G[r].w - kk * dd.w);
+          ra[r] = ds.x * x[r].x + ds.y * x[r].y + ds.z * x[r].z + ds.w * x[r].w;
+          G[r] = make_float4(a * ds.x, a * ds.y, a * ds.z, a * ds.w);
+        }
       }
       {
         int first;
@@ -326,7 +383,7 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
 #pragma unroll
           for (int i = 0; i < NR; ++i) {
             p.dk[orow + first + i] = rk[i];
-            p.dgate[orow + first + i] = p.gate_log ? ra[i] * a_[row0 + first + i] : ra[i];  // dL/dg = dL/dalpha * alpha
+            p.dgate[orow + first + i] = p.gate_log ? ra[i] * a_[first + i] : ra[i];  // dL/dg = dL/dalpha * alpha
           }
         }
       }
