@@ -80,8 +80,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                                        i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, u32, vp, i64, i64, i64, i64,
                                            lp, vp, vp]
-    lib.kda_scan_backward_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
-    lib.kda_scan_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64, i64, i64, i64, i64, lp,
+    lib.kda_scan_backward_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_scan_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, lp,
                                       vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_bounded_decay_backward.argtypes = [vp, vp, ctypes.c_float, vp, i64, i64, i64, i64, vp, vp, vp]
     for fn in ("kda_scan_backward_workspace_bytes", "kda_scan_backward", "kda_bounded_decay_backward"):
@@ -427,10 +427,12 @@ def decode_step_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: tor
 
 def scan_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
                   initial_state: Optional[torch.Tensor], d_o: torch.Tensor, d_final_state: Optional[torch.Tensor] = None,
-                  *, gate_is_log: bool = False) -> dict:
+                  cu_seqlens: Optional[torch.Tensor] = None, *, gate_is_log: bool = False) -> dict:
     """Gradients of the scan (``kda_scan_backward``): returns fp32 ``dq, dk [B,T,H,K]``, ``dv [B,T,H,V]``,
-    ``dgate`` (dL/dalpha, or dL/dg with ``gate_is_log``), ``dbeta [B,T,H]`` and ``d_initial_state [B,H,K,V]``
-    for ``L = <o, d_o> + <S_T, d_final_state>``. Inputs as for ``prefill`` (no cu_seqlens)."""
+    ``dgate`` (dL/dalpha, or dL/dg with ``gate_is_log``), ``dbeta [B,T,H]`` and ``d_initial_state [N,H,K,V]``
+    for ``L = <o, d_o> + <S_T, d_final_state>``. Inputs as for ``prefill``: with ``cu_seqlens`` (int32
+    ``[N+1]``, B = 1) the states are per sequence (N = number of sequences, else N = B) and the gradients
+    of tokens outside every sequence are zero."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta"), (d_o, "d_o")):
         _cuda(t, n)
     if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
@@ -444,24 +446,36 @@ def scan_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch
     d_o = d_o.to(torch.float32).contiguous()
     if d_o.shape != (B, T, H, V):
         raise ValueError("d_o must be [B,T,H,V]")
+    N, n_seq, cu_ptr = B, 0, None
+    if cu_seqlens is not None:
+        _cuda(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        if B != 1:
+            raise ValueError("cu_seqlens requires B == 1")
+        cu_seqlens = cu_seqlens.contiguous()
+        N = n_seq = cu_seqlens.numel() - 1
+        cu_ptr = cu_seqlens.data_ptr()
     f32 = lambda t: None if t is None else t.to(device=dev, dtype=torch.float32).contiguous()  # noqa: E731
     initial_state, d_final_state = f32(initial_state), f32(d_final_state)
     for t, n in ((initial_state, "initial_state"), (d_final_state, "d_final_state")):
-        if t is not None and t.shape != (B, H, K, V):
-            raise ValueError(f"{n} must be [{B},{H},{K},{V}]")
-    out = {"dq": torch.empty(B, T, H, K, device=dev), "dk": torch.empty(B, T, H, K, device=dev),
-           "dv": torch.empty(B, T, H, V, device=dev), "dgate": torch.empty(B, T, H, K, device=dev),
-           "dbeta": torch.empty(B, T, H, device=dev), "d_initial_state": torch.empty(B, H, K, V, device=dev)}
+        if t is not None and t.shape != (N, H, K, V):
+            raise ValueError(f"{n} must be [{N},{H},{K},{V}]")
+    new = torch.zeros if cu_seqlens is not None else torch.empty
+    out = {"dq": new(B, T, H, K, device=dev), "dk": new(B, T, H, K, device=dev),
+           "dv": new(B, T, H, V, device=dev), "dgate": new(B, T, H, K, device=dev),
+           "dbeta": new(B, T, H, device=dev), "d_initial_state": torch.empty(N, H, K, V, device=dev)}
     lib = load_library()
     n = ctypes.c_size_t(0)
-    _check("kda_scan_backward_workspace_bytes", lib.kda_scan_backward_workspace_bytes(B, T, H, K, V, ctypes.byref(n)))
+    _check("kda_scan_backward_workspace_bytes",
+           lib.kda_scan_backward_workspace_bytes(B, T, H, K, V, n_seq, ctypes.byref(n)))
     ws = torch.empty(max(int(n.value), 16), device=dev, dtype=torch.uint8)
     layout = Layout(_strides4(q), _strides4(k), _strides4(v), _strides4(gate), _strides3(beta), Strides(0, 0, 0))
     ptr = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
     _check("kda_scan_backward", lib.kda_scan_backward(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
         KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), ptr(initial_state), d_o.data_ptr(),
-        ptr(d_final_state), B, T, H, K, V, ctypes.byref(layout), out["dq"].data_ptr(), out["dk"].data_ptr(),
+        ptr(d_final_state), cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out["dq"].data_ptr(), out["dk"].data_ptr(),
         out["dv"].data_ptr(), out["dgate"].data_ptr(), out["dbeta"].data_ptr(), out["d_initial_state"].data_ptr(),
         ws.data_ptr(), ws.numel(), _stream(dev)))
     return out

@@ -151,12 +151,24 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
 
   const int tid = threadIdx.x, tv = tid % CG, tk = tid / CG;
   const int row0 = tk * RPT, col0 = 4 * tv;
-  const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
-  const int64_t T = p.T;
-  const int n_seg = (int)((T + kSeg - 1) / kSeg);
+  const int bh = blockIdx.x, seq = bh / p.H, h = bh % p.H;  // (sequence or batch row, head)
+  const int64_t T = p.T;  // tokens per batch row (the packed total with cu_seqlens)
   const size_t slice = (size_t)K * VT;
-  float* ckpt = p.ckpt + (size_t)bh * (n_seg + 1) * slice;  // state before token j*kSeg, j = 0..n_seg
-  float* scr = p.scratch + (size_t)bh * kSeg * slice;       // states before each token of a segment
+  // This CTA's tokens are ts .. ts + len - 1 of batch row b.
+  int b = seq;
+  int64_t ts = 0, len = T;
+  float* ckpt;  // state before token ts + j*kSeg, j = 0..n_seg
+  if (p.cu) {
+    const int64_t t1 = min((int64_t)p.cu[seq + 1], T);
+    ts = max((int64_t)0, min((int64_t)p.cu[seq], t1));
+    len = t1 - ts;
+    b = 0;
+    ckpt = p.ckpt + ((size_t)h * p.ckpt_slots + (size_t)(ts / kSeg) + 2 * (size_t)seq) * slice;
+  } else {
+    ckpt = p.ckpt + (size_t)bh * ((T + kSeg - 1) / kSeg + 1) * slice;
+  }
+  const int n_seg = (int)((len + kSeg - 1) / kSeg);
+  float* scr = p.scratch + (size_t)bh * kSeg * slice;  // states before each token of a segment
   const TIn* qb = static_cast<const TIn*>(p.q);
   const TIn* kb = static_cast<const TIn*>(p.k);
   const TIn* vb = static_cast<const TIn*>(p.v);
@@ -242,8 +254,8 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
   for (int r = 0; r < RPT; ++r) x[r] = p.s0 ? *reinterpret_cast<const float4*>(p.s0 + sbase + (size_t)(row0 + r) * VT + col0)
                                             : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int seg = 0; seg < n_seg; ++seg) {
-    const int64_t t0 = (int64_t)seg * kSeg;
-    const int n = (int)min((int64_t)kSeg, T - t0);
+    const int64_t t0 = ts + (int64_t)seg * kSeg;
+    const int n = (int)min((int64_t)kSeg, ts + len - t0);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) *tile(ckpt + (size_t)seg * slice, r) = x[r];
     stage_segment(t0, n, false);
@@ -264,8 +276,8 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
     cp_async_commit();
   };
   for (int seg = n_seg - 1; seg >= 0; --seg) {
-    const int64_t t0 = (int64_t)seg * kSeg;
-    const int n = (int)min((int64_t)kSeg, T - t0);
+    const int64_t t0 = ts + (int64_t)seg * kSeg;
+    const int n = (int)min((int64_t)kSeg, ts + len - t0);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) x[r] = *tile(ckpt + (size_t)seg * slice, r);
     stage_segment(t0, n, true);
@@ -403,7 +415,7 @@ cudaError_t launch_b(const BwdParams& p, cudaStream_t s) {
   static_assert(bytes <= 227 * 1024, "shared memory budget");
   cudaError_t e = cudaFuncSetAttribute(scan_backward_kernel<RPT, VT, TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  scan_backward_kernel<RPT, VT, TIn><<<(unsigned)(p.B * p.H), kGroups * (VT / 4), bytes, s>>>(p);
+  scan_backward_kernel<RPT, VT, TIn><<<(unsigned)(p.N * p.H), kGroups * (VT / 4), bytes, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -500,14 +512,19 @@ __global__ void __launch_bounds__(256) bounded_decay_backward_kernel(const float
 
 }  // namespace
 
-int64_t backward_segments(int64_t T) { return (T + kSeg - 1) / kSeg; }
+int64_t backward_ckpt_slots(int64_t T, int64_t n_seq) {
+  return n_seq > 0 ? T / kSeg + 2 * n_seq + 1 : (T + kSeg - 1) / kSeg + 1;
+}
 
 bool backward_supported(int K, int V) {
   return (K == 16 || K == 32 || K == 64 || K == 128) && (V == 16 || V == 32 || V == 64 || V == 128);
 }
 
-size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V) {
-  return (size_t)B * H * (size_t)(backward_segments(T) + 1 + kSeg) * (size_t)K * V * sizeof(float);
+size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t n_seq) {
+  const size_t slice = (size_t)K * V * sizeof(float);
+  if (n_seq > 0)  // checkpoints shared per head, scratch per (sequence, head)
+    return (size_t)H * backward_ckpt_slots(T, n_seq) * slice + (size_t)n_seq * H * kSeg * slice;
+  return (size_t)B * H * (size_t)(backward_ckpt_slots(T, 0) + kSeg) * slice;
 }
 
 cudaError_t launch_scan_backward(const BwdParams& p, kda_dtype dt, cudaStream_t s) {

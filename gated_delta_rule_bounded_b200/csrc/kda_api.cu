@@ -407,22 +407,29 @@ int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtyp
   return decode_impl("kda_decode_step_logits", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 
-int kda_scan_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes) {
+int kda_scan_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t n_seq,
+                                      size_t* bytes) {
   if (!bytes) return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_workspace_bytes: null output");
-  if (B < 0 || T < 0 || H < 0 || K < 0 || V < 0)
+  if (B < 0 || T < 0 || H < 0 || K < 0 || V < 0 || n_seq < 0)
     return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_workspace_bytes: negative size");
-  *bytes = kda::backward_workspace_bytes(B, T, H, K, V);
+  *bytes = kda::backward_workspace_bytes(B, T, H, K, V, n_seq);
   return ok();
 }
 
 int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dtype,
                       const float* gate, kda_gate_kind gate_kind, const float* beta,
                       const float* initial_state, const float* d_o, const float* d_final_state,
+                      const int32_t* cu_seqlens, int64_t n_seq,
                       int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
                       float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
                       void* workspace, size_t workspace_bytes, kda_stream_t stream) {
   const char* fn = "kda_scan_backward";
-  if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (B < 0 || T < 0 || H < 0 || n_seq < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  int64_t N = B;  // sequences
+  if (cu_seqlens) {
+    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "%s: cu_seqlens requires B == 1 (got %lld)", fn, (long long)B);
+    N = n_seq;
+  }
   if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
   if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, (int)gate_kind);
@@ -430,10 +437,10 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
     return fail(KDA_ERR_UNSUPPORTED, "%s: K and V must be 16, 32, 64 or 128 (K=%lld, V=%lld)", fn, (long long)K,
                 (long long)V);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (B * H == 0) return ok();
+  if (N * H == 0) return ok();
   if (T == 0) {  // nothing to differentiate through: dS_0 = dS_T
     if (d_initial_state) {
-      cudaError_t e = kda::launch_state_copy(d_final_state, d_initial_state, B * H * K * V, s);
+      cudaError_t e = kda::launch_state_copy(d_final_state, d_initial_state, N * H * K * V, s);
       if (e != cudaSuccess) return cuda_fail(e, fn);
     }
     return ok();
@@ -441,7 +448,8 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
   if (!q || !k || !v || !gate || !beta || !d_o || !dq || !dk || !dv || !dgate || !dbeta)
     return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
   if (T > INT32_MAX) return fail(KDA_ERR_UNSUPPORTED, "%s: T too large", fn);
-  const size_t need = kda::backward_workspace_bytes(B, T, H, K, V);
+  const int64_t n_ws = cu_seqlens ? N : 0;
+  const size_t need = kda::backward_workspace_bytes(B, T, H, K, V, n_ws);
   if (!workspace || workspace_bytes < need)
     return fail(KDA_ERR_INVALID_ARG, "%s: the workspace needs %zu bytes (got %zu)", fn, need, workspace_bytes);
   kda_layout L;
@@ -480,9 +488,10 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
   p.dgate = dgate;
   p.dbeta = dbeta;
   p.ds0 = d_initial_state;
-  const int64_t n_seg = kda::backward_segments(T);
+  p.cu = cu_seqlens;
+  p.ckpt_slots = kda::backward_ckpt_slots(T, n_ws);
   p.ckpt = static_cast<float*>(workspace);
-  p.scratch = p.ckpt + (size_t)B * H * (n_seg + 1) * K * V;
+  p.scratch = p.ckpt + (size_t)(cu_seqlens ? H : B * H) * p.ckpt_slots * K * V;
   put(p.qs, L.q);
   put(p.ks, L.k);
   put(p.vs, L.v);
@@ -490,6 +499,7 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
   put(p.bs, L.beta);
   p.T = T;
   p.B = (int)B;
+  p.N = (int)N;
   p.H = (int)H;
   p.K = (int)K;
   p.V = (int)V;

@@ -69,14 +69,19 @@ struct BwdParams {
   float* ds0;         // or nullptr (not written)
   float* ckpt;        // workspace: checkpoints, then the per-CTA segment scratch
   float* scratch;
+  const int32_t* cu;  // [N + 1] sequence offsets (B == 1), or nullptr: one sequence per batch row
+  int64_t ckpt_slots; // with cu: checkpoint slots per head
   int64_t qs[3], ks[3], vs[3], gs[3], bs[3];
   int64_t T;
-  int B, H, K, V;
+  int B, N, H, K, V;  // N: sequences (B without cu)
   int gate_log;
 };
 bool backward_supported(int K, int V);
-int64_t backward_segments(int64_t T);  // checkpoint segments; the workspace holds segments + 1 checkpoints
-size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V);
+// Checkpoint slots per head: (T/32 rounded up + 1) per batch row without cu_seqlens; with n_seq packed
+// sequences, floor(T/32) + 2 n_seq + 1 shared by the sequences of a head (sequence n starts at slot
+// floor(cu[n]/32) + 2n, which keeps them disjoint).
+int64_t backward_ckpt_slots(int64_t T, int64_t n_seq);
+size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t n_seq);
 cudaError_t launch_scan_backward(const BwdParams& p, kda_dtype dt, cudaStream_t s);
 cudaError_t launch_bounded_decay_backward(const float* z, const float* A_log, float g_min, const float* dg,
                                           int64_t rows_bt, int H, int K, float* dz, float* dA, cudaStream_t s);

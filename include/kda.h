@@ -288,19 +288,25 @@ int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtyp
  *   KDA_GATE_ALPHA, dL/dg for KDA_GATE_LOG), dbeta [B,T,H] and
  *   d_initial_state [B,H,K,V] (NULL: not written),
  * given d_o [B,T,H,V] = dL/do and d_final_state [B,H,K,V] = dL/dS_T (NULL:
- * zeros). All gradient tensors are fp32 and contiguous; q, k, v, gate, beta
+ * zeros); with cu_seqlens the states are per sequence (below). All gradient tensors are fp32 and contiguous; q, k, v, gate, beta
  * and initial_state are the forward call's inputs (layout strides for q, k, v,
- * gate, beta as in kda_prefill). Supported: K, V in {16, 32, 64, 128}; no
- * cu_seqlens (one sequence per batch row). The scan is recomputed from
- * checkpoints every 32 tokens: the caller passes a workspace of
- * kda_scan_backward_workspace_bytes (KDA_ERR_INVALID_ARG if smaller). This is
+ * gate, beta as in kda_prefill). cu_seqlens (device int32 [n_seq + 1],
+ * nullable) packs variable-length sequences as in kda_prefill: B must be 1,
+ * the states initial_state, d_final_state and d_initial_state are
+ * [n_seq,H,K,V], and gradients of tokens outside [cu[0], cu[n_seq]) are not
+ * written; without it n_seq is ignored. Supported: K, V in {16, 32, 64, 128}.
+ * The scan is recomputed from checkpoints every 32 tokens: the caller passes
+ * a workspace of kda_scan_backward_workspace_bytes for the same B, T, H, K, V
+ * and n_seq (0 without cu_seqlens; KDA_ERR_INVALID_ARG if smaller). This is
  * the exact token-by-token adjoint, not a chunked kernel.
  * ------------------------------------------------------------------------- */
-int kda_scan_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes);
+int kda_scan_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t n_seq,
+                                      size_t* bytes);
 
 int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dtype,
                       const float* gate, kda_gate_kind gate_kind, const float* beta,
                       const float* initial_state, const float* d_o, const float* d_final_state,
+                      const int32_t* cu_seqlens, int64_t n_seq,
                       int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
                       float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
                       void* workspace, size_t workspace_bytes, kda_stream_t stream);

@@ -159,6 +159,46 @@ def test_workspace_query(lib):
     assert lib.kda_prefill_workspace_bytes(1, 1, 1, 128, 128, 0, 1, None) == INVALID
 
 
+def _backward(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dtype=1, gate=FAKE, gk=1, beta=FAKE, s0=None, do=FAKE, dsf=None, cu=None,
+             n_seq=0, B=1, T=64, H=2, K=128, V=128, layout=None, dq=FAKE, dk=FAKE, dv=FAKE, dg=FAKE, db=FAKE,
+             ds0=None, ws=FAKE, wsb=0, stream=None)
+    a.update(kw)
+    rc = lib.kda_scan_backward(a["q"], a["k"], a["v"], a["dtype"], a["gate"], a["gk"], a["beta"], a["s0"], a["do"],
+                               a["dsf"], a["cu"], a["n_seq"], a["B"], a["T"], a["H"], a["K"], a["V"], a["layout"],
+                               a["dq"], a["dk"], a["dv"], a["dg"], a["db"], a["ds0"], a["ws"], a["wsb"], a["stream"])
+    return rc, lib.kda_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,code,msg", [
+    (dict(B=-1), INVALID, "negative"),
+    (dict(n_seq=-1), INVALID, "negative"),
+    (dict(cu=FAKE, n_seq=3, B=2), INVALID, "B == 1"),
+    (dict(gk=3), INVALID, "gate kind"),
+    (dict(K=48), UNSUPPORTED, "K and V"),
+    (dict(dq=None), INVALID, "null"),
+    (dict(wsb=1024), INVALID, "workspace"),
+    (dict(cu=FAKE, n_seq=4, wsb=1024), INVALID, "workspace"),
+])
+def test_scan_backward_rejects_bad_arguments(lib, kw, code, msg):
+    rc, err = _backward(lib, **kw)
+    assert rc == code and msg in err, (rc, err)
+
+
+def test_scan_backward_workspace_query(lib):
+    def ws(B, T, H, K, V, n_seq):
+        n = ctypes.c_size_t(0)
+        assert lib.kda_scan_backward_workspace_bytes(B, T, H, K, V, n_seq, ctypes.byref(n)) == OK
+        return n.value
+    slice_ = 128 * 128 * 4
+    # one sequence per batch row: (ceil(T/32) + 1) checkpoints and 32 scratch states per (row, head)
+    assert ws(2, 100, 3, 128, 128, 0) == 2 * 3 * (4 + 1 + 32) * slice_
+    # packed sequences: floor(T/32) + 2N + 1 checkpoint slots per head, 32 scratch states per (sequence, head)
+    assert ws(1, 100, 3, 128, 128, 5) == 3 * (3 + 10 + 1) * slice_ + 5 * 3 * 32 * slice_
+    n = ctypes.c_size_t(0)
+    assert lib.kda_scan_backward_workspace_bytes(1, 10, 1, 128, 128, -1, ctypes.byref(n)) == INVALID
+
+
 def test_last_error_cleared_on_success(lib):
     _gate(lib, g_min=0.0)
     assert lib.kda_last_error().decode() != ""

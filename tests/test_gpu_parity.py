@@ -640,6 +640,40 @@ def test_scan_backward_matches_autograd_oracle(kda, B, T, H, K, V, dtype, log_ga
     check_grad(out["dgate"], ref["alpha"] * a_used if log_gate else ref["alpha"], "dgate")
 
 
+@pytest.mark.parametrize("dtype,K,V", [("bf16", 128, 128), ("f32", 64, 32)])
+def test_scan_backward_varlen_matches_oracle_per_sequence(kda, dtype, K, V):
+    # Packed sequences of ragged lengths (one empty, one of a single token, several crossing the 32-token
+    # checkpoint segments), each with its own initial state and dL/dS_T; every sequence must get the
+    # gradients of its own scan, and an empty one dL/dS_0 = dL/dS_T.
+    lens = [70, 0, 129, 1, 64, 33]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    N, T, H = len(lens), int(cu[-1]), 2
+    d = W.random_scan_case(1, T, H, K, V, seed=41, dtype=dtype, z_std=2.0, init_std=None)
+    gen = torch.Generator().manual_seed(42)
+    s0 = torch.randn(N, H, K, V, generator=gen) * 0.1
+    dsf = torch.randn(N, H, K, V, generator=gen) * 0.1
+    do = torch.randn(1, T, H, V, generator=gen)
+    _, lg = oracle.bounded_decay(d["z"], d["A_log"], d["g_min"], return_log=True)
+    gate = torch.tensor(lg, dtype=torch.float32)
+    gd = to_dev(d)
+    out = kda.scan_backward(gd["q"], gd["k"], gd["v"], gate.to(DEV), gd["beta"], s0.to(DEV), do.to(DEV), dsf.to(DEV),
+                            cu_seqlens=torch.tensor(cu).to(DEV), gate_is_log=True)
+    torch.cuda.synchronize()
+    a_used = np.exp(gate.double().numpy())
+    for n in range(N):
+        a, b = int(cu[n]), int(cu[n + 1])
+        if a == b:
+            np.testing.assert_array_equal(out["d_initial_state"][n].cpu().numpy(), dsf[n].numpy())
+            continue
+        sl = lambda x: x[:, a:b]  # noqa: E731
+        ref = oracle.scan_backward(sl(d["q"]), sl(d["k"]), sl(d["v"]), a_used[:, a:b], sl(d["beta"]), s0[n:n + 1],
+                                   do[:, a:b], dsf[n:n + 1])
+        for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("beta", "dbeta")):
+            check_grad(out[key][:, a:b], ref[name], f"{key} of sequence {n}")
+        check_grad(out["dgate"][:, a:b], ref["alpha"] * a_used[:, a:b], f"dgate of sequence {n}")
+        check_grad(out["d_initial_state"][n:n + 1], ref["initial_state"], f"d_initial_state of sequence {n}")
+
+
 def test_gate_backward_matches_autograd_oracle(kda):
     d = W.random_scan_case(2, 50, 3, 64, 16, seed=3, dtype="f32", z_std=2.0, init_std=None)
     dg = torch.randn(2, 50, 3, 64, generator=torch.Generator().manual_seed(4))
