@@ -83,10 +83,14 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 MEASURED_TRAFFIC = {
     # chunk_intra_kernel 404,604,416 + 359,971,072; chunk_state_kernel 506,579,456 + 87,632,128
     "prefill": {"bytes": 1358787072, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "75515deebf2f36e39fdb781925fc16d98ea8037d7b85d8613a5f5e79377970d4"},
+                "sha256": "d7cc6002b08133fbd28a88baae802c511a038cea16d375973c1d46771747fca1"},
     # decode_bulk_kernel 410,578,688 + 346,280,704
     "decode": {"bytes": 756859392, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "bfa67c5dc56d225b3ded53734266d52acbe99bf41188d181eea5539246d78b1f"},
+               "sha256": "221f3c9de7dacd4479d0b46c6dfe6e77dfea3e984ec7bd20c3c8757dfb22bcc3"},
+    # bounded_decay_kernel 201,352,704 + 153,886,720; scan_backward_kernel 19,299,634,688 + 27,350,004,480;
+    # bounded_decay_backward_kernel 402,688,512 + 162,508,288 (one backward step from the logits)
+    "backward": {"bytes": 47570075392, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                 "sha256": "6fbc4cb59dd35e5a50259e40bea1b8bfdaec0df3e3591672ca456c301fd21702"},
 }
 
 
@@ -385,7 +389,7 @@ def backward_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
         "steps": steps, "gpu_launches": 3 * steps,  # gate, scan gradients, gate gradient
         "kernels_ms": {"backward_from_logits": ms},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": None, "kernel": "kda_scan_backward (+ gate and gate gradient)",
+                     "traffic": measured_traffic("backward"), "kernel": "kda_scan_backward (+ gate and gate gradient)",
                      "bytes_per_launch": nb, "ms_per_launch": ms, "peak_source": f"{peak_src} hbm_gbs",
                      "note": "token-serial adjoint: latency-bound, one CTA per head"},
     }
