@@ -77,20 +77,20 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
     return n_elems * (es_in + es_out)
 
 
-# DRAM bytes (read + write) per launch of each step, from one ncu capture of its kernels (the summaries in
-# profiles/ give the commands). They hold only for the kernel sources they were taken on, so the sources'
-# sha256 is kept beside them and a mismatch at run time reports null.
+# DRAM bytes (read + write) per launch of each step, from one ncu capture of its kernels (commands and
+# per-kernel values in profiles/dram_traffic__bench_steps.md). They hold only for the kernel sources they were
+# taken on, so the sources' sha256 is kept beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
-    # chunk_intra_kernel 404,604,416 + 359,971,072; chunk_state_kernel 506,579,456 + 87,632,128
-    "prefill": {"bytes": 1358787072, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "d7cc6002b08133fbd28a88baae802c511a038cea16d375973c1d46771747fca1"},
-    # decode_bulk_kernel 410,578,688 + 346,280,704
-    "decode": {"bytes": 756859392, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "221f3c9de7dacd4479d0b46c6dfe6e77dfea3e984ec7bd20c3c8757dfb22bcc3"},
+    # chunk_intra_kernel 404,795,392 + 359,710,208; chunk_state_kernel 506,546,432 + 84,204,288
+    "prefill": {"bytes": 1355256320, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                "sha256": "2a3c340ba45947bb5c894a4c44d2e7fb398ffe751f3ef1584c72a65f1548ca85"},
+    # decode_bulk_kernel 410,584,832 + 345,193,472
+    "decode": {"bytes": 755778304, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "f0ea99d5bd7f661f413f4c3d98366402d4a4d4fb81de98a6017e64fd316622f2"},
     # bounded_decay_kernel 201,352,704 + 153,886,720; scan_backward_kernel 19,299,634,688 + 27,350,004,480;
     # bounded_decay_backward_kernel 402,688,512 + 162,508,288 (one backward step from the logits)
     "backward": {"bytes": 47570075392, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "6fbc4cb59dd35e5a50259e40bea1b8bfdaec0df3e3591672ca456c301fd21702"},
+                 "sha256": "4193000631bcc6119793735c091255da4542ad2b653c903d95780e375766ad2f"},
 }
 
 

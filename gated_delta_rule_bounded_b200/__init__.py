@@ -84,7 +84,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_scan_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, lp,
                                       vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_bounded_decay_backward.argtypes = [vp, vp, ctypes.c_float, vp, i64, i64, i64, i64, vp, vp, vp]
-    for fn in ("kda_scan_backward_workspace_bytes", "kda_scan_backward", "kda_bounded_decay_backward"):
+    lib.kda_selftest_wait_expiry.argtypes = [vp]
+    for fn in ("kda_scan_backward_workspace_bytes", "kda_scan_backward", "kda_bounded_decay_backward",
+               "kda_selftest_wait_expiry"):
         getattr(lib, fn).restype = ctypes.c_int
     for fn in ("kda_bounded_decay", "kda_softplus_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
                "kda_decode_step", "kda_prefill_logits", "kda_decode_step_logits"):
@@ -494,6 +496,13 @@ def bounded_decay_backward(logits: torch.Tensor, A_log: torch.Tensor, g_min: flo
         z.data_ptr(), A.data_ptr(), float(g_min), dg.data_ptr(), B, T, H, K, dz.data_ptr(), dA.data_ptr(),
         _stream(z.device)))
     return dz, dA
+
+
+def selftest_wait_expiry(device=None) -> None:
+    """``kda_selftest_wait_expiry``: one kernel whose bounded wait runs out (about a second); the next
+    ``device_status()`` then reports True."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check("kda_selftest_wait_expiry", load_library().kda_selftest_wait_expiry(_stream(dev)))
 
 
 def device_status(reset: bool = True) -> bool:

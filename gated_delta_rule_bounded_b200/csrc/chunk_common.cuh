@@ -18,7 +18,6 @@ constexpr int VT = 128;   // value columns per state tile
 constexpr int NTHREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float G2_MIN = -5.5f * LOG2E;  // lower clamp of the per-token log2-decay
-constexpr uint32_t WAIT_LIMIT = 1u << 22;
 
 // fp32 vector area written by the decay pass (offsets in floats).
 constexpr int VEC_D = 0;          // [10][128] bf16 exp(G_{s_a} - G_{r_b}), pairs a >= b (640 floats)
@@ -173,13 +172,7 @@ __device__ __forceinline__ void tm_st16(uint32_t taddr, const uint32_t (&r)[16])
 }
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* timeout_flag) {
-  for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-    if (done) return true;
-  }
+  if (mbar_try_wait_bounded(bar, parity)) return true;
   atomicExch(timeout_flag, 1);
   return false;
 }

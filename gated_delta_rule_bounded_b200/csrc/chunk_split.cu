@@ -591,6 +591,22 @@ cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+namespace {
+// One thread waits on an mbarrier that expects one arrival which never comes: the bounded wait must
+// give up and record the expiry in g_split_timeout.
+__global__ void wait_expiry_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
+  mbar_wait(b, 0, &g_split_timeout);
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(cudaStream_t s) {
+  wait_expiry_selftest_kernel<<<1, 1, 0, s>>>();
+  return cudaGetLastError();
+}
+
 cudaError_t split_read_timeout(int* flag, bool reset) {
   cudaError_t e = cudaMemcpyFromSymbol(flag, g_split_timeout, sizeof(int));
   if (e != cudaSuccess || !reset) return e;

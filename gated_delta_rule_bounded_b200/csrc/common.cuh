@@ -17,6 +17,39 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Bounded wait on phase `parity` of the mbarrier at shared address `bar`. Each poll may suspend the thread
+// for at most WAIT_HINT_NS; the wait gives up after WAIT_NS of %globaltimer time (counted from the first
+// unsuccessful poll) or WAIT_POLLS polls, whichever comes first, and returns false. Callers record the
+// expiry in a device flag that kda_device_status reports, and carry on without the awaited data.
+constexpr uint32_t WAIT_POLLS = 1u << 22;
+constexpr uint32_t WAIT_HINT_NS = 1000u;
+constexpr uint64_t WAIT_NS = 1000000000ull;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool mbar_try_wait_bounded(uint32_t bar, uint32_t parity) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0; it < WAIT_POLLS; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(WAIT_HINT_NS)
+        : "memory");
+    if (done) return true;
+    if (it == 0) {
+      t0 = globaltimer_ns();
+    } else if ((it & 15) == 0 && globaltimer_ns() - t0 > WAIT_NS) {
+      break;
+    }
+  }
+  return false;
+}
+
 // Streaming (evict-first) 16-byte load and store for data touched once per launch.
 __device__ __forceinline__ float4 ld_stream(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ void st_stream(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }

@@ -27,7 +27,6 @@ __device__ int g_decode_timeout = 0;
 namespace {
 
 constexpr int DK = 128, DV = 128, DNT = 256, NSTAGE = 3, ROWS = DK / 8;
-constexpr uint32_t WAIT_LIMIT = 1u << 22;
 
 template <typename TIn>
 struct StageLayout {
@@ -54,13 +53,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 }
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t it = 0; it < WAIT_LIMIT; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-    if (done) return true;
-  }
+  if (mbar_try_wait_bounded(bar, parity)) return true;
   atomicExch(&g_decode_timeout, 1);
   return false;
 }

@@ -82,6 +82,12 @@ const char* kda_last_error(void) { return g_err; }
 
 const char* kda_version(void) { return "kda-b200 0.2 (sm_100a)"; }
 
+int kda_selftest_wait_expiry(kda_stream_t stream) {
+  cudaError_t e = kda::launch_wait_selftest(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_wait_expiry");
+  return ok();
+}
+
 int kda_device_status(int* timed_out, int reset) {
   if (!timed_out) return fail(KDA_ERR_INVALID_ARG, "kda_device_status: null output");
   cudaError_t e = cudaDeviceSynchronize();

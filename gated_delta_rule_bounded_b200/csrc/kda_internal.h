@@ -103,6 +103,7 @@ size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t n_seq);
 cudaError_t launch_chunk(const ScanParams& p, void* ws, size_t ws_bytes, cudaStream_t s);
 size_t split_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, bool varlen);
 cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s);
+cudaError_t launch_wait_selftest(cudaStream_t s);  // one wait that expires (kda_selftest_wait_expiry)
 cudaError_t split_read_timeout(int* flag, bool reset);
 // Reads (and optionally clears) the chunk kernel's device-side timeout flag. Synchronous.
 cudaError_t chunk_read_timeout(int* flag, bool reset);

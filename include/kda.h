@@ -324,13 +324,23 @@ int kda_bounded_decay_backward(const float* logits, const float* A_log, float g_
 
 /* ---------------------------------------------------------------------------
  * kda_device_status: device-side failure flags, for callers that check them
- * after their work has finished. Every wait inside the library's kernels has
- * an iteration limit; a kernel whose wait expires stops, records the event in
- * a device flag and returns instead of hanging. This call synchronises the
- * current device, writes 1 to *timed_out if any such event has been recorded
- * since the last reset (0 otherwise), and clears the flag when reset != 0.
+ * after their work has finished. Every wait inside the library's kernels is
+ * bounded (about one second of device time, at most 2^22 polls); a kernel
+ * whose wait expires records the event in a device flag and returns instead
+ * of hanging. This call synchronises the current device, writes 1 to
+ * *timed_out if any such event has been recorded since the last reset (0
+ * otherwise), and clears the flag when reset != 0.
  * ------------------------------------------------------------------------- */
 int kda_device_status(int* timed_out, int reset);
+
+/* ---------------------------------------------------------------------------
+ * kda_selftest_wait_expiry: diagnostics for the failure path above. Launches
+ * one single-thread kernel on `stream` that waits on an mbarrier nothing ever
+ * arrives on; the wait gives up after its limit (about one second) and
+ * records the expiry, which the next kda_device_status reports. Nothing else
+ * is touched and the context stays usable.
+ * ------------------------------------------------------------------------- */
+int kda_selftest_wait_expiry(kda_stream_t stream);
 
 /* Last error of the calling thread ("" when the last call succeeded). */
 const char* kda_last_error(void);
