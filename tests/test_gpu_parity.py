@@ -674,6 +674,21 @@ def test_scan_backward_varlen_matches_oracle_per_sequence(kda, dtype, K, V):
         check_grad(out["d_initial_state"][n:n + 1], ref["initial_state"], f"d_initial_state of sequence {n}")
 
 
+@pytest.mark.parametrize("B,T,H,K", [(1, 37, 2, 6), (2, 300, 3, 128)])
+def test_gate_backward_paths(kda, B, T, H, K):
+    # K = 6: the scalar path (rows are not whole float4s); 2 x 300 x 3 x 128: many row blocks per head, whose
+    # partial sums of dL/dA_log meet in one atomic each.
+    gen = torch.Generator().manual_seed(K + T)
+    z = torch.randn(B, T, H, K, generator=gen) * 2.0
+    A_log = torch.randn(H, generator=gen) * 0.5
+    dg = torch.randn(B, T, H, K, generator=gen)
+    dz, dA = kda.bounded_decay_backward(z.to(DEV), A_log.to(DEV), -5.0, dg.to(DEV))
+    torch.cuda.synchronize()
+    rz, rA = oracle.bounded_decay_backward(z, A_log, -5.0, dg)
+    check_grad(dz, rz, "dz")
+    np.testing.assert_allclose(dA.double().cpu().numpy(), rA, rtol=1e-4, atol=1e-4 * float(np.abs(rA).max()))
+
+
 def test_gate_backward_matches_autograd_oracle(kda):
     d = W.random_scan_case(2, 50, 3, 64, 16, seed=3, dtype="f32", z_std=2.0, init_std=None)
     dg = torch.randn(2, 50, 3, 64, generator=torch.Generator().manual_seed(4))
