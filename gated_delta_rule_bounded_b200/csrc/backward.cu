@@ -133,7 +133,10 @@ __device__ __forceinline__ float4 colsum(const float* red, int col0) {
   return s;
 }
 
-template <int RPT, int VT, typename TIn>
+// LOGG: the gate is g = log(alpha). Then dL/dg = rowsum(dSbar * Sbar), so the adjoint keeps Sbar itself in
+// the registers of S_{t-1} and never needs S_{t-1} again; with alpha given, dL/dalpha needs S_{t-1} and
+// Sbar is formed where it is used.
+template <int RPT, int VT, typename TIn, bool LOGG>
 __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(BwdParams p) {
   using L = BwdSmem<RPT, VT, TIn>;
   constexpr int K = L::K, CG = VT / 4, NT = L::NT;
@@ -302,8 +305,11 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
       const TIn* q_ = sq + tt * K + row0;
       const TIn* v_ = sv + tt * VT;
       const float beta = sbeta[tt];
-      // delta from Sbar = Diag(alpha) S_{t-1} (Sbar is recomputed from S_{t-1} where needed)
-      auto sbar = [&](int r, float a) { return make_float4(a * x[r].x, a * x[r].y, a * x[r].z, a * x[r].w); };
+      // delta from Sbar = Diag(alpha) S_{t-1}: with LOGG x becomes Sbar here, otherwise Sbar is formed
+      // from S_{t-1} where it is needed
+      auto sbar = [&](int r, float a) {
+        return LOGG ? x[r] : make_float4(a * x[r].x, a * x[r].y, a * x[r].z, a * x[r].w);
+      };
       float4 pa = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int rr = 0; rr < RPT; rr += RG) {
@@ -314,6 +320,10 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
         for (int j = 0; j < RG; ++j) {
           const int r = rr + j;
           const float kk = kv[j];
+          if (LOGG) {
+            const float a = av[j];
+            x[r].x *= a; x[r].y *= a; x[r].z *= a; x[r].w *= a;
+          }
           const float4 xb = sbar(r, av[j]);
           pa.x = fmaf(kk, xb.x, pa.x); pa.y = fmaf(kk, xb.y, pa.y);
           pa.z = fmaf(kk, xb.z, pa.z); pa.w = fmaf(kk, xb.w, pa.w);
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
           rk[r] = beta * (G[r].x * d.x + G[r].y * d.y + G[r].z * d.z + G[r].w * d.w) -
                   (xb.x * dd.x + xb.y * dd.y + xb.z * dd.z + xb.w * dd.w);
           const float4 ds = make_float4(G[r].x - kk * dd.x, G[r].y - kk * dd.y, G[r].z - kk * dd.z, G[r].w - kk * dd.w);
-          ra[r] = ds.x * x[r].x + ds.y * x[r].y + ds.z * x[r].z + ds.w * x[r].w;
+          ra[r] = ds.x * x[r].x + ds.y * x[r].y + ds.z * x[r].z + ds.w * x[r].w;  // LOGG: dL/dg, else dL/dalpha
           G[r] = make_float4(a * ds.x, a * ds.y, a * ds.z, a * ds.w);
         }
       }
@@ -395,7 +405,7 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
 #pragma unroll
           for (int i = 0; i < NR; ++i) {
             p.dk[orow + first + i] = rk[i];
-            p.dgate[orow + first + i] = p.gate_log ? ra[i] * a_[first + i] : ra[i];  // dL/dg = dL/dalpha * alpha
+            p.dgate[orow + first + i] = ra[i];
           }
         }
       }
@@ -409,14 +419,20 @@ __global__ void __launch_bounds__(kGroups * (VT / 4), 1) scan_backward_kernel(Bw
   }
 }
 
-template <int RPT, int VT, typename TIn>
-cudaError_t launch_b(const BwdParams& p, cudaStream_t s) {
+template <int RPT, int VT, typename TIn, bool LOGG>
+cudaError_t launch_bg(const BwdParams& p, cudaStream_t s) {
   constexpr int bytes = BwdSmem<RPT, VT, TIn>::BYTES;
   static_assert(bytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(scan_backward_kernel<RPT, VT, TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  auto kern = scan_backward_kernel<RPT, VT, TIn, LOGG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  scan_backward_kernel<RPT, VT, TIn><<<(unsigned)(p.N * p.H), kGroups * (VT / 4), bytes, s>>>(p);
+  kern<<<(unsigned)(p.N * p.H), kGroups * (VT / 4), bytes, s>>>(p);
   return cudaGetLastError();
+}
+
+template <int RPT, int VT, typename TIn>
+cudaError_t launch_b(const BwdParams& p, cudaStream_t s) {
+  return p.gate_log ? launch_bg<RPT, VT, TIn, true>(p, s) : launch_bg<RPT, VT, TIn, false>(p, s);
 }
 
 template <int RPT, typename TIn>
