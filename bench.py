@@ -87,10 +87,10 @@ MEASURED_TRAFFIC = {
     # decode_bulk_kernel 410,584,832 + 345,193,472
     "decode": {"bytes": 755778304, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                "sha256": "f0ea99d5bd7f661f413f4c3d98366402d4a4d4fb81de98a6017e64fd316622f2"},
-    # bounded_decay_kernel 201,352,704 + 153,886,720; scan_backward_kernel 19,299,634,688 + 27,350,004,480;
-    # bounded_decay_backward_kernel 402,688,512 + 162,508,288 (one backward step from the logits)
-    "backward": {"bytes": 47570075392, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "4193000631bcc6119793735c091255da4542ad2b653c903d95780e375766ad2f"},
+    # bounded_decay_kernel 201,388,032 + 154,186,496; scan_backward_kernel 17,959,960,832 + 27,343,060,992;
+    # bounded_decay_backward_kernel 402,712,832 + 162,471,424 (one backward step from the logits)
+    "backward": {"bytes": 46223780608, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                 "sha256": "4e128306fa88fbe43e6de95d747168e1ba8523f2254c7b9a3a2c8d1c262d07b2"},
 }
 
 
