@@ -697,3 +697,26 @@ def test_gate_backward_matches_autograd_oracle(kda):
     rz, rA = oracle.bounded_decay_backward(d["z"], d["A_log"], d["g_min"], dg)
     check_grad(dz, rz, "dz")
     np.testing.assert_allclose(dA.double().cpu().numpy(), rA, rtol=1e-4, atol=1e-4)
+
+
+def test_usage_example_from_the_design_notes(kda):
+    # The Python usage example of the design notes, at a small size: every call must accept what the
+    # example passes (views included) and return finite values of the documented shapes.
+    B, T, H, K, V = 1, 130, 4, 128, 128
+    gen = torch.Generator().manual_seed(11)
+    q, k = (torch.randn(B, T, H, K, generator=gen).to(DEV, torch.bfloat16) for _ in range(2))
+    v = torch.randn(B, T, H, V, generator=gen).to(DEV, torch.bfloat16)
+    z = torch.randn(B, T, H, K, generator=gen).to(DEV)
+    A_log = torch.zeros(H, device=DEV)
+    beta = torch.rand(B, T, H, generator=gen).to(DEV)
+    o, S = kda.prefill_logits(q, k, v, z, A_log, -5.0, beta, qk_l2norm=True)
+    assert o.shape == (B, T, H, V) and S.shape == (B, H, K, V)
+    o1 = kda.decode_step_logits(q[:, 0], k[:, 0], v[:, 0], z[:, 0], A_log, -5.0, beta[:, 0], S)
+    assert o1.shape == (B, H, V)
+    g = kda.bounded_decay(z, A_log, -5.0, log_decay=True)
+    grads = kda.scan_backward(q, k, v, g, beta, None, torch.randn_like(o, dtype=torch.float32), gate_is_log=True)
+    dz, dA_log = kda.bounded_decay_backward(z, A_log, -5.0, grads["dgate"])
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    for t in (o, S, o1, dz, dA_log, *grads.values()):
+        assert torch.isfinite(t.float()).all()
