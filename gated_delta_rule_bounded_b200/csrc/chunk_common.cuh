@@ -386,7 +386,10 @@ __device__ __forceinline__ float log2_decay(int mode, float x, float sc, float g
 
 // Decay pass, step 1: the per-token log2-decay of channels (c0, c0+1) over the 16 tokens of block
 // da (clamped at G2_MIN; 0 past the end of the sequence), their retention factors, and the block
-// sum, published to VEC_TOT.
+// sum, published to VEC_TOT. With UNBOUNDED the logits feed Kimi Linear's gate g = -e^{A_h} softplus(z)
+// and nothing is clamped: every factor this pass forms is then still <= 1 except the diagonal-block
+// pair factors, which the caller replaces (see softplus_diag_kernel).
+template <bool UNBOUNDED = false>
 __device__ __forceinline__ void decay_step1(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int nv,
                                             int da, int c0, int mode, float sc, float g_min, float2 (&al)[16]) {
   float* vec = reinterpret_cast<float*>(sm + L.vec);
@@ -395,8 +398,13 @@ __device__ __forceinline__ void decay_step1(unsigned char* sm, const IntraLayout
   for (int i = 0; i < 16; ++i) {
     float2 l = make_float2(0.f, 0.f);
     if (16 * da + i < nv) {
-      l.x = fmaxf(log2_decay(mode, pf.g[i].x, sc, g_min), G2_MIN);
-      l.y = fmaxf(log2_decay(mode, pf.g[i].y, sc, g_min), G2_MIN);
+      if (UNBOUNDED) {
+        l.x = softplus_log_decay(sc, pf.g[i].x) * LOG2E;
+        l.y = softplus_log_decay(sc, pf.g[i].y) * LOG2E;
+      } else {
+        l.x = fmaxf(log2_decay(mode, pf.g[i].x, sc, g_min), G2_MIN);
+        l.y = fmaxf(log2_decay(mode, pf.g[i].y, sc, g_min), G2_MIN);
+      }
     }
     run.x += l.x;
     run.y += l.y;

@@ -39,6 +39,10 @@ constexpr int WB_KA = 32768;     // 24K  one k-atom (t) of 192 rows: (A_qk [t'][
 constexpr int WB_TP = 57344;     // 8K   T' [t][i]
 constexpr int WB_GAM = 65536;    // 512  gamma_C, fp32 [128]
 constexpr int WB_BYTES = 66048;
+// Unbounded gate only: the pairwise diagonal blocks of A_kk and A_qk (see softplus_diag_kernel), written
+// into the T' region before kernel P runs; P reads them there before its final bulk store overwrites it.
+constexpr int WB_DIAG = WB_TP;
+static_assert(2 * 4 * 16 * 16 * 4 <= WB_GAM - WB_TP, "the diagonal blocks fit the T' region");
 
 // Kernel P shared memory (104,192 bytes: two CTAs fit on an SM). Q*Gamma and K*gamma_C/Gamma
 // never touch it: the decay pass writes them from registers straight into the workspace block.
@@ -198,6 +202,154 @@ __device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch&
   }
 }
 
+// Kimi Linear's unbounded gate (KDA_GATE_SOFTPLUS), g = -e^{A_h} softplus(z): the diagonal 16x16 blocks
+// of A_kk and A_qk of one (chunk, head), pair by pair. Within a block exp(G_t - G_j) <= 1 for j <= t, but
+// kernel P's block-boundary factorisation splits it as exp(G_t - G_s) exp(G_s - G_j), whose second factor
+// grows with the decay of the whole block, which this gate does not bound. One warp per (block a, column
+// j), lanes over the channels: A_qk[t][j] = sum_c q_tc k_jc exp(G_tc - G_jc) for t >= j and A_kk[t][j] =
+// beta_t sum_c k_tc k_jc exp(G_tc - G_jc) for t > j, with q, k L2-normalised and rounded to bf16 first
+// when the flag asks, and beta from its logits when the flag asks, as kernel P does.
+constexpr int D_Q = 0, D_K = 16384, D_G = 32768, D_BETA = 65536, D_SMEM = D_BETA + 256;
+
+__global__ void __launch_bounds__(NTHREADS) softplus_diag_kernel(ScanParams p, unsigned char* ws) {
+  extern __shared__ __align__(16) unsigned char sm[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.y;
+  const int64_t slot = blockIdx.x;
+  int n, jc;
+  if (!locate_slot(p, slot, n, jc)) return;  // uniform across the CTA
+  int64_t t0, t1, brow;
+  seq_range(p, n, t0, t1, brow);
+  const int64_t tc0 = t0 + (int64_t)jc * C;
+  const int nv = (int)min((int64_t)C, t1 - tc0);
+  float* out = reinterpret_cast<float*>(ws + ((size_t)slot * p.H + h) * WB_BYTES + WB_DIAG);
+  const float sc = expf(__ldg(p.A_log + h));
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k);
+  __nv_bfloat16* sq = reinterpret_cast<__nv_bfloat16*>(sm + D_Q);
+  __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(sm + D_K);
+  float* sg = reinterpret_cast<float*>(sm + D_G);
+  float* sbeta = reinterpret_cast<float*>(sm + D_BETA);
+
+  // Rows: warp w takes tokens w, w + 8, ...; lane l channels 4l .. 4l + 3.
+  for (int r = warp; r < C; r += 8) {
+    const int64_t t = tc0 + r;
+    uint2 qv = make_uint2(0u, 0u), kv = make_uint2(0u, 0u);
+    float4 lg = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < nv) {
+      qv = *reinterpret_cast<const uint2*>(qb + brow * p.qs[0] + t * p.qs[1] + h * p.qs[2] + 4 * lane);
+      kv = *reinterpret_cast<const uint2*>(kb + brow * p.ks[0] + t * p.ks[1] + h * p.ks[2] + 4 * lane);
+      const float4 z = *reinterpret_cast<const float4*>(p.gate + brow * p.gs[0] + t * p.gs[1] + h * p.gs[2] + 4 * lane);
+      lg = make_float4(softplus_log_decay(sc, z.x) * LOG2E, softplus_log_decay(sc, z.y) * LOG2E,
+                       softplus_log_decay(sc, z.z) * LOG2E, softplus_log_decay(sc, z.w) * LOG2E);
+    }
+    if (p.qk_l2norm) {
+      float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y), k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
+      float ssq = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
+      float ssk = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) {
+        ssq += __shfl_xor_sync(0xffffffffu, ssq, m);
+        ssk += __shfl_xor_sync(0xffffffffu, ssk, m);
+      }
+      const float fq = l2norm_scale(ssq), fk = l2norm_scale(ssk);
+      qv = make_uint2(pack_bf16(q01.x * fq, q01.y * fq), pack_bf16(q23.x * fq, q23.y * fq));
+      kv = make_uint2(pack_bf16(k01.x * fk, k01.y * fk), pack_bf16(k23.x * fk, k23.y * fk));
+    }
+    *reinterpret_cast<uint2*>(sq + r * KD + 4 * lane) = qv;
+    *reinterpret_cast<uint2*>(sk + r * KD + 4 * lane) = kv;
+    *reinterpret_cast<float4*>(sg + r * KD + 4 * lane) = lg;
+    if (lane == 0)
+      sbeta[r] = r < nv ? beta_value(__ldg(p.beta + brow * p.bs[0] + t * p.bs[1] + h * p.bs[2]), p.beta_sigmoid) : 0.f;
+  }
+  __syncthreads();
+  // G: the running log2-decay within each 16-token block, one (block, channel) column per thread.
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const int col = tid + NTHREADS * m, a = col >> 7, c = col & (KD - 1);
+    float run = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float* x = sg + (16 * a + i) * KD + c;
+      run += *x;
+      *x = run;
+    }
+  }
+  __syncthreads();
+  for (int item = warp; item < 64; item += 8) {
+    const int a = item >> 4, j = item & 15, rj = 16 * a + j;
+    float kj[4], gj[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      kj[m] = __bfloat162float(sk[rj * KD + lane + 32 * m]);
+      gj[m] = sg[rj * KD + lane + 32 * m];
+    }
+    for (int t = 0; t < 16; ++t) {
+      const int rt = 16 * a + t;
+      float sqk = 0.f, skk = 0.f;
+      if (t >= j) {  // uniform across the warp
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int c = lane + 32 * m;
+          const float w = kj[m] * ex2(sg[rt * KD + c] - gj[m]);
+          sqk = fmaf(__bfloat162float(sq[rt * KD + c]), w, sqk);
+          skk = fmaf(__bfloat162float(sk[rt * KD + c]), w, skk);
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+          sqk += __shfl_xor_sync(0xffffffffu, sqk, m);
+          skk += __shfl_xor_sync(0xffffffffu, skk, m);
+        }
+      }
+      if (lane == 0) {
+        out[(a * 16 + t) * 16 + j] = t > j ? skk * sbeta[rt] : 0.f;
+        out[1024 + (a * 16 + t) * 16 + j] = sqk;
+      }
+    }
+  }
+}
+
+// The four diagonal 16x16 blocks of A_kk and A_qk for the unbounded gate, formed pairwise by
+// softplus_diag_kernel and stored as fp32 [A_kk | A_qk][block a][t][j] (A_kk with beta_t folded in, zero
+// on and above the diagonal; A_qk zero above it) in the T' region of the chunk's workspace block.
+
+// intra_phases (chunk_common.cuh) for the unbounded gate: the tile products run as usual, then the
+// diagonal blocks, whose block-boundary factorisation needs exp(-decay of 16 tokens) and can overflow,
+// are replaced by the pairwise values from `diag` before the inverse and the W phase read them.
+__device__ __forceinline__ void unbounded_intra_phases(unsigned char* sm, uint32_t sb, const IntraLayout& L,
+                                                       const float* beta_s, int tid, int warp, int lane, int g,
+                                                       int tq, const float* diag) {
+  float dk[4], dq[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    dk[r] = __ldg(diag + tid + NTHREADS * r);
+    dq[r] = __ldg(diag + 1024 + tid + NTHREADS * r);
+  }
+  a_tiles<2>(sm, sb, L, L.ke, warp, 8, warp < 2 ? 2 : 1, lane, g, tq, beta_s, /*is_qk=*/false);
+  __syncthreads();
+  float* akk = reinterpret_cast<float*>(sm + L.akk);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int e = tid + NTHREADS * r, a = e >> 8, t = (e >> 4) & 15, j = e & 15;
+    akk[(16 * a + t) * 64 + 16 * a + j] = dk[r];
+  }
+  __syncthreads();  // A_kk ready
+  if (warp < 4) {
+    inverse_warps0to3(sm, sb, L, beta_s, tid, warp, lane, g, tq);
+  } else {
+    a_tiles<3>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
+    zero_upper_blocks(sm, L.aqk, tid - 128, 128);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int e = tid + NTHREADS * r, a = e >> 8, t = (e >> 4) & 15, j = e & 15;
+    *reinterpret_cast<__nv_bfloat16*>(sm + L.aqk + sw_e(16 * a + t, 16 * a + j, 8192)) = __float2bfloat16_rn(dq[r]);
+  }
+  // The W phase does not read A_qk; the barrier before the bulk store publishes these writes.
+}
+
+template <bool UNBOUNDED>
 __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, unsigned char* ws) {
   extern __shared__ __align__(1024) unsigned char sm[];
   const uint32_t sb = smem_u32(sm);
@@ -245,12 +397,16 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     if (tid < C) beta_s[tid] = tid < nv ? beta_value(__ldg(x.beta + x.boff + (tc0 + tid) * x.bst), p.beta_sigmoid) : 0.f;
     if (p.qk_l2norm) l2norm_qk(pf, reinterpret_cast<float*>(sm + P_VEC) + VEC_D, tid, da);
     float2 al[16];
-    decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
+    decay_step1<UNBOUNDED>(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
     __syncthreads();
     p_decay_step2(sm, pf, da, c0, al, blk + WB_WQ + (even ? 8192 : 0), blk + WB_KA + (even ? 8192 : 0));
   }
   __syncthreads();
-  intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+  if constexpr (UNBOUNDED) {
+    unbounded_intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq, reinterpret_cast<const float*>(blk + WB_DIAG));
+  } else {
+    intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+  }
 
   // W = T' (K*Gamma) on mma.sync. Warp w owns columns 16w.. of all 64 rows, so every warp does the
   // same ten block products of the lower-triangular T'. -W is stored over the dead Qe tile as
@@ -563,14 +719,24 @@ size_t split_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, bool va
 }
 
 cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
-  static std::atomic<uint64_t> cfg_p{0}, cfg_s{0};
-  cudaError_t e = set_smem_once(chunk_intra_kernel, P_SMEM, cfg_p);
+  const bool unbounded = p.gate_mode == GATE_SOFTPLUS;
+  static std::atomic<uint64_t> cfg_p{0}, cfg_pu{0}, cfg_d{0}, cfg_s{0};
+  cudaError_t e = unbounded ? set_smem_once(chunk_intra_kernel<true>, P_SMEM, cfg_pu)
+                            : set_smem_once(chunk_intra_kernel<false>, P_SMEM, cfg_p);
+  if (e == cudaSuccess && unbounded) e = set_smem_once(softplus_diag_kernel, D_SMEM, cfg_d);
   if (e == cudaSuccess) e = set_smem_once(chunk_state_kernel, S_SMEM, cfg_s);
   if (e != cudaSuccess) return e;
   const int64_t slots = split_slots(p.B, p.T, p.N, p.cu != nullptr);
   if (slots == 0 || p.N == 0) return cudaSuccess;
   dim3 gp((unsigned)slots, (unsigned)p.H);
-  chunk_intra_kernel<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
+  if (unbounded) {
+    softplus_diag_kernel<<<gp, NTHREADS, D_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    chunk_intra_kernel<true><<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
+  } else {
+    chunk_intra_kernel<false><<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t grid = (int64_t)p.N * p.H * (p.V / VT);

@@ -290,10 +290,12 @@ static int prefill_impl(const char* fn, const void* q, const void* k, const void
   p.state_vk = (gs.flags & KDA_STATE_VK) != 0;
 
   cudaError_t e;
-  // The chunked kernels rely on the bounded per-token decay; the unbounded gate takes the exact
-  // token-by-token kernel.
-  if (dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype) && gs.mode != kda::GATE_SOFTPLUS) {
-    if (workspace_bytes > 0 && !workspace) return fail(KDA_ERR_INVALID_ARG, "%s: workspace_bytes > 0 with a null workspace", fn);
+  if (workspace_bytes > 0 && !workspace) return fail(KDA_ERR_INVALID_ARG, "%s: workspace_bytes > 0 with a null workspace", fn);
+  const bool chunked = dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype);
+  // The unbounded gate runs chunked only on the two-kernel path (its pairwise diagonal blocks live in
+  // the workspace); without a workspace it takes the exact token-by-token kernel.
+  const bool split_ok = workspace && workspace_bytes >= kda::split_workspace_bytes(B, T, H, N, cu_seqlens != nullptr);
+  if (chunked && (gs.mode != kda::GATE_SOFTPLUS || split_ok)) {
     e = kda::launch_chunk(p, workspace, workspace_bytes, s);
   } else {
     e = kda::launch_recurrent(p, dtype, s);

@@ -575,17 +575,43 @@ def test_softplus_gate_matches_oracle(kda):
     assert ref.min() < -20.0  # the decay is far below what a bounded gate allows
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_prefill_logits_softplus_gate(kda, dtype):
+@pytest.mark.parametrize("dtype,use_workspace", [("bf16", True), ("bf16", False), ("f32", True)],
+                         ids=["bf16-chunked", "bf16-token-kernel", "f32"])
+def test_prefill_logits_softplus_gate(kda, dtype, use_workspace):
     d = W.random_scan_case(2, 150, 3, 128, 128, seed=43, dtype=dtype, z_std=2.0, init_std=0.1)
     g = to_dev(d)
     o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"],
-                               g["initial_state"], gate="softplus")
+                               g["initial_state"], gate="softplus", use_workspace=use_workspace)
     torch.cuda.synchronize()
     assert not kda.device_status()
     ro, rs = oracle_softplus_pipeline(d)
     check(o, ro, dtype, "o")
     check(sf, rs, dtype, "final_state")
+
+
+def test_prefill_logits_softplus_chunked_extreme_decay(kda):
+    # The chunked path of the unbounded gate, with heads whose decay within one 16-token block is far past
+    # what the block-boundary factorisation can hold (exp of thousands), packed ragged sequences with their
+    # own initial states, and q, k, beta prepared inside the kernels; against the fp64 oracle.
+    lens = [70, 0, 129, 1, 64, 200]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    T, H, K, V = int(cu[-1]), 4, 128, 128
+    d = W.random_scan_case(1, T, H, K, V, seed=61, dtype="bf16", z_std=4.0, init_std=None, raw_inputs=True)
+    d["A_log"] = torch.tensor([-1.0, 0.5, 2.0, 4.0])
+    d["cu_seqlens"] = cu
+    d["initial_state"] = torch.randn(len(lens), H, K, V, generator=torch.Generator().manual_seed(62)) * 0.1
+    g = to_dev(d)
+    o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"], g["initial_state"],
+                               g["cu_seqlens"], qk_l2norm=True, beta_logits=True, gate="softplus")
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    alpha, lg = oracle.softplus_decay(d["z"], d["A_log"], return_log=True)
+    # the last heads' decay over some 16-token block is beyond the fp32 range of its reciprocal
+    assert float(lg[0, :16, 3].sum(axis=0).min()) < -200.0
+    ro, rs = oracle.scan(oracle.l2norm(d["q"]), oracle.l2norm(d["k"]), d["v"], alpha, oracle.sigmoid(d["beta"]),
+                         d["initial_state"], d["cu_seqlens"])
+    check(o, ro, "bf16", "o")
+    check(sf, rs, "bf16", "final_state")
 
 
 def test_decode_logits_softplus_gate(kda):
