@@ -87,6 +87,8 @@ MEASURED_TRAFFIC = {
     # decode_bulk_kernel 410,584,832 + 345,193,472
     "decode": {"bytes": 755778304, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                "sha256": "f0ea99d5bd7f661f413f4c3d98366402d4a4d4fb81de98a6017e64fd316622f2"},
+    # softplus_diag_kernel, chunk_intra_kernel<true>, chunk_state_kernel: not yet captured
+    "softplus": {"bytes": None, "files": [], "sha256": ""},
     # bounded_decay_kernel 201,388,032 + 154,186,496; scan_backward_kernel 17,959,960,832 + 27,343,060,992;
     # bounded_decay_backward_kernel 402,712,832 + 162,471,424 (one backward step from the logits)
     "backward": {"bytes": 46223780608, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
@@ -355,6 +357,37 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     return res
 
 
+def softplus_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
+    """The prefill workload through Kimi Linear's unbounded gate (gate="softplus"): the pairwise
+    diagonal-block pre-pass, kernel P and kernel S; device-timed only."""
+    w = W.PREFILL
+    d = W.make_scan_inputs(w)
+    B, T, H, K, V = w.B, w.T, w.H, w.K, w.V
+    g = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in d.items()}
+    o = torch.empty(B, T, H, V, device=dev, dtype=torch.bfloat16)
+    sf = torch.empty(B, H, K, V, device=dev, dtype=torch.float32)
+    ws = torch.empty(max(kda.prefill_workspace_bytes(B, T, H, K, V, 0, torch.bfloat16), 1), device=dev,
+                     dtype=torch.uint8)
+
+    def fn():
+        kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], w.g_min, g["beta"], None, gate="softplus",
+                           out=o, final_state=sf, workspace=ws)
+
+    steps = max(3, min(args.steps, 20))
+    total_ms, (ms,) = timed_loop([fn], steps, args.warmup, world, stream)
+    value, total_ms = weak_scaling_value(B * T * steps, total_ms, world)
+    pb = prefill_bytes(B, T, H, K, V, 0, 1)
+    achieved = pb / (ms / 1e3) / 1e9
+    return {
+        "workload": w.name + "_softplus_gate", "value": value, "unit": "tokens/s", "ms_per_step": total_ms / steps,
+        "steps": steps, "gpu_launches": 3 * steps,  # diagonal-block pre-pass, kernel P, kernel S
+        "kernels_ms": {"prefill_logits_softplus": ms},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": measured_traffic("softplus"), "kernel": "kda_prefill_logits (KDA_GATE_SOFTPLUS)",
+                     "bytes_per_launch": pb, "ms_per_launch": ms, "peak_source": f"{peak_src} hbm_gbs"},
+    }
+
+
 def backward_bytes(B, T, H, K, V, es=2):
     """Minimum HBM bytes of one backward step from the logits, per token-head: the gate (read z, write g:
     8K), the scan gradients (read q, k, v in the input dtype, g, beta, dL/do in fp32; write dq, dk, dg, dv,
@@ -489,14 +522,18 @@ def gpu_arm(args, rank, world, local):
     if args.workload in ("all", "decode"):
         dec = decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
         torch.cuda.empty_cache()
+    spl = None
+    if args.workload in ("all", "softplus"):
+        spl = softplus_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
+        torch.cuda.empty_cache()
     bwd = None
     if args.workload in ("all", "backward"):
         bwd = backward_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             bwd["cpu_baseline"] = cpu_backward_sample()
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
-    if pre is None and bwd is not None and dec is None:  # backward-only profiling run
-        return {"metric": METRIC, "workload_only": "backward", "backward": bwd}
+    if pre is None and dec is None:  # single-leg profiling run
+        return {"metric": METRIC, "workload_only": args.workload, "backward": bwd, "softplus": spl}
     if pre is None:  # decode-only profiling run
         return {"metric": METRIC, "workload_only": "decode", "decode": dec}
     w = pre["workload"]
@@ -525,6 +562,8 @@ def gpu_arm(args, rank, world, local):
     }
     if dec is not None:
         line["decode"] = dec
+    if spl is not None:
+        line["softplus"] = spl
     if bwd is not None:
         line["backward"] = bwd
     if cpu is not None:
@@ -601,7 +640,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--cpu-heads", type=int, default=0, help="heads in the oracle sample (0: auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "backward"], default="all",
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "softplus", "backward"], default="all",
                     help="one leg alone (profiling runs); the JSON line needs 'all'")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end legs")
     args = ap.parse_args(argv)

@@ -306,7 +306,8 @@ def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.T
     K per (token, head); ``beta_logits``: ``beta`` holds logits and the kernels apply the sigmoid;
     ``state_layout="vk"``: the states are ``[N,H,V,K]`` (value-by-key) instead of ``[N,H,K,V]``;
     ``gate="softplus"``: the logits feed Kimi Linear's unbounded gate ``g = -exp(A_log) softplus(z)``
-    (``g_min`` unused; the scan then runs token by token). Other arguments as in ``prefill``."""
+    (``g_min`` unused; chunked with its diagonal blocks formed pairwise when a workspace is used, token by
+    token otherwise). Other arguments as in ``prefill``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")

@@ -178,8 +178,10 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  *   KDA_GATE_SOFTPLUS the logits feed Kimi Linear's unbounded gate,
  *                    g = -exp(A_log[h]) * softplus(z) (g_min is ignored),
  *                    instead of the bounded one. Its per-token decay has no
- *                    lower bound, so the chunked kernels (which rely on it) are
- *                    not used: the scan runs token by token (exact, slower). */
+ *                    lower bound, so the diagonal 16x16 blocks of the chunk
+ *                    form are computed pairwise by an extra kernel; this
+ *                    chunked path needs the workspace (bf16, K = 128), and
+ *                    without one the scan runs token by token (exact, slower). */
 #define KDA_QK_L2NORM 1u
 #define KDA_BETA_LOGITS 2u
 #define KDA_STATE_VK 4u
