@@ -18,6 +18,11 @@
 // S, and kernel P writes each block's operand pairs in the order that chunk's parity needs.
 // The price of the split is the workspace traffic (one write and one read of ~1 KB per token-head).
 //
+// With Kimi Linear's unbounded gate (KDA_GATE_SOFTPLUS) a pre-pass, softplus_diag_kernel, first forms the
+// diagonal 16x16 blocks of A_kk and A_qk pair by pair (their block-boundary factorisation would need the
+// reciprocal of a whole block's decay, which that gate does not bound), and chunk_intra_kernel<true> takes
+// them from the workspace in place of its own diagonal tiles; every other factor stays <= 1.
+//
 // Workspace slots. Chunk j of sequence n has slot n * ceil(T/64) + j without cu_seqlens, and
 // floor(cu[n]/64) + n + j with them (unique: a sequence's slots end before the next one's begin).
 #include <atomic>

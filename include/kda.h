@@ -123,7 +123,7 @@ int kda_softplus_decay(const void* logits, const kda_strides* logits_strides, kd
  * workspace (about 1 KB per token and head), then runs the recurrence. Given
  * at least this many bytes kda_prefill uses it; given less (or no workspace),
  * it runs the single fused kernel instead, with identical results up to
- * rounding. The caller allocates the workspace; a larger buffer is fine. n_seq
+ * rounding (with KDA_GATE_SOFTPLUS, the token-by-token kernel instead). The caller allocates the workspace; a larger buffer is fine. n_seq
  * is the number of packed sequences (0 without cu_seqlens).
  * ------------------------------------------------------------------------- */
 int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
