@@ -64,3 +64,42 @@ def chunkwise_scan(q, k, v, alpha, beta, S0, C):
             o[b_, :, h], sf[b_, h] = chunkwise_head(q[b_, :, h], k[b_, :, h], v[b_, :, h],
                                                     alpha[b_, :, h], beta[b_, :, h], s0, C)
     return o, sf
+
+
+def block_factored_a(q, k, G, pairwise_diag=False, blk=16, dtype=np.float32):
+    """A_qk[t,i] = sum_c q_tc k_ic exp(G_tc - G_ic) (i <= t) of one chunk, formed the way the chunked
+    kernels form it, in `dtype` arithmetic: 16-token blocks a, b with the block-boundary references
+    s_a (cumulative log-decay before block a) and r_b (after block b), as
+    (q * exp(G - G_s_a)) * exp(G_s_a - G_r_b) . (k * exp(G_r_b - G))  for a > b,
+    and for the diagonal blocks either the same split with exp(G_s_a - G_r_a) -- the reciprocal of the
+    block's whole decay -- or pairwise (``pairwise_diag``). Returns (A_qk, largest factor applied off the
+    diagonal blocks). G is the inclusive cumulative log-decay [n, K] in fp64."""
+    n, K = q.shape
+    G = np.asarray(G, dtype=np.float64)
+    nb = (n + blk - 1) // blk
+    Gs = [np.zeros(K) if a == 0 else G[blk * a - 1] for a in range(nb)]
+    Gr = [G[min(blk * (a + 1), n) - 1] for a in range(nb)]
+    A = np.zeros((n, n), dtype=dtype)
+    worst = 0.0
+    with np.errstate(over="ignore", invalid="ignore", under="ignore"):
+        for a in range(nb):
+            ta = slice(blk * a, min(blk * (a + 1), n))
+            E = np.exp(G[ta] - Gs[a])
+            for b in range(a + 1):
+                tb = slice(blk * b, min(blk * (b + 1), n))
+                if a == b and pairwise_diag:
+                    d = G[ta][:, None, :] - G[tb][None, :, :]
+                    ratio = np.where(np.tril(np.ones((d.shape[0], d.shape[1]), bool))[:, :, None],
+                                     np.exp(np.minimum(d, 0.0)), 0.0).astype(dtype)
+                    A[ta, tb] = np.einsum("tc,ic,tic->ti", q[ta].astype(dtype), k[tb].astype(dtype), ratio)
+                    continue
+                F = np.exp(Gr[b] - G[tb])
+                D = np.exp(Gs[a] - Gr[b])
+                if a > b:
+                    worst = max(worst, float(E.max()), float(F.max()), float(D.max()))
+                lhs = (q[ta] * E).astype(dtype) * D.astype(dtype)[None, :]
+                blockA = lhs @ (k[tb] * F).astype(dtype).T
+                if a == b:
+                    blockA = np.tril(blockA)
+                A[ta, tb] = blockA
+    return A, worst

@@ -454,3 +454,50 @@ def test_gate_gradients_match_finite_differences():
     zm[0, 1, 1, 2] -= h
     num = (f(torch.tensor(zp), torch.tensor(A)) - f(torch.tensor(zm), torch.tensor(A))).item() / (2 * h)
     assert abs(num - dz[0, 1, 1, 2]) < 1e-7
+
+
+# The unbounded gate on the chunked path ("Kimi K3: Bounded Decay and Delta Memory", Figure 3(a) contrast;
+# "KDA cheat sheet", the BF16 reciprocal-rescale argument): with g = -e^A softplus(z) the reciprocal of a
+# 16-token block's decay leaves the fp32 range, so the diagonal blocks are formed pairwise, while every
+# factor that crosses a block boundary stays <= 1. Checked in fp32 arithmetic against the pairwise
+# definition in fp64.
+
+def _a_qk_exact(q, k, G):
+    d = G[:, None, :] - G[None, :, :]
+    ratio = np.where(np.tril(np.ones((len(q), len(q)), bool))[:, :, None], np.exp(np.minimum(d, 0.0)), 0.0)
+    return np.einsum("tc,ic,tic->ti", q, k, ratio)
+
+
+def _unit(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def test_block_factorisation_needs_pairwise_diagonal_blocks_for_the_unbounded_gate():
+    from tests.chunkwise_fp64 import block_factored_a
+    rng = np.random.default_rng(7)
+    n, K = 64, 32
+    q, k = _unit(rng.standard_normal((n, K))), _unit(rng.standard_normal((n, K)))
+    z = rng.standard_normal((n, K)) * 4.0
+    g = -np.exp(4.0) * (np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z))))   # softplus gate, e^A = e^4
+    G = np.cumsum(g, axis=0)
+    assert (G[15] - 0.0).min() < -1000.0                                      # a block's decay is e^-1000 or less
+    exact = _a_qk_exact(q, k, G)
+    A_split, _ = block_factored_a(q, k, G, pairwise_diag=False)
+    assert not np.all(np.isfinite(A_split))                                   # the split diagonal overflows
+    A_pair, worst = block_factored_a(q, k, G, pairwise_diag=True)
+    assert worst <= 1.0                                                       # every cross-block factor <= 1
+    assert np.all(np.isfinite(A_pair))
+    np.testing.assert_allclose(A_pair, exact, rtol=0, atol=1e-5)
+
+
+def test_block_factorisation_is_safe_for_the_bounded_gate():
+    from tests.chunkwise_fp64 import block_factored_a
+    rng = np.random.default_rng(8)
+    n, K = 64, 32
+    q, k = _unit(rng.standard_normal((n, K))), _unit(rng.standard_normal((n, K)))
+    g = np.full((n, K), -5.0)                                                 # the bound itself, every token
+    G = np.cumsum(g, axis=0)
+    exact = _a_qk_exact(q, k, G)
+    A_split, worst = block_factored_a(q, k, G, pairwise_diag=False)
+    assert worst <= 1.0 and np.all(np.isfinite(A_split))                      # e^80 at most on the diagonal
+    np.testing.assert_allclose(A_split, exact, rtol=0, atol=1e-5)
