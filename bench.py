@@ -83,14 +83,14 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 MEASURED_TRAFFIC = {
     # chunk_intra_kernel 404,795,392 + 359,710,208; chunk_state_kernel 506,546,432 + 84,204,288
     "prefill": {"bytes": 1355256320, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "9b3066076fa5e43a36de3f75ead61a769c8310a7f245025aa41db9ebe0013e48"},
+                "sha256": "8e578cec51f4b2a8c9123e9926752cea1b27036a61725d3b0797108e08b6ffa1"},
     # decode_bulk_kernel 410,584,832 + 345,193,472
     "decode": {"bytes": 755778304, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                "sha256": "f0ea99d5bd7f661f413f4c3d98366402d4a4d4fb81de98a6017e64fd316622f2"},
-    # softplus_diag_kernel 404,593,664 + 42,189,056; chunk_intra_kernel<true> 455,069,184 + 356,146,432;
-    # chunk_state_kernel 506,545,920 + 84,337,152 (the unbounded gate's chunked prefill)
-    "softplus": {"bytes": 1848881408, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "9b3066076fa5e43a36de3f75ead61a769c8310a7f245025aa41db9ebe0013e48"},
+    # softplus_diag_kernel 404,549,888 + 41,925,120; chunk_intra_kernel<true> 455,110,656 + 356,195,840;
+    # chunk_state_kernel 506,546,176 + 84,393,216 (the unbounded gate's chunked prefill)
+    "softplus": {"bytes": 1848720896, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                 "sha256": "8e578cec51f4b2a8c9123e9926752cea1b27036a61725d3b0797108e08b6ffa1"},
     # bounded_decay_kernel 201,388,032 + 154,186,496; scan_backward_kernel 17,959,960,832 + 27,343,060,992;
     # bounded_decay_backward_kernel 402,712,832 + 162,471,424 (one backward step from the logits)
     "backward": {"bytes": 46223780608, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],

@@ -216,7 +216,7 @@ __device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch&
 // when the flag asks, and beta from its logits when the flag asks, as kernel P does.
 constexpr int D_Q = 0, D_K = 16384, D_G = 32768, D_BETA = 65536, D_SMEM = D_BETA + 256;
 
-__global__ void __launch_bounds__(NTHREADS) softplus_diag_kernel(ScanParams p, unsigned char* ws) {
+__global__ void __launch_bounds__(NTHREADS, 3) softplus_diag_kernel(ScanParams p, unsigned char* ws) {
   extern __shared__ __align__(16) unsigned char sm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.y;
@@ -236,36 +236,53 @@ __global__ void __launch_bounds__(NTHREADS) softplus_diag_kernel(ScanParams p, u
   float* sg = reinterpret_cast<float*>(sm + D_G);
   float* sbeta = reinterpret_cast<float*>(sm + D_BETA);
 
-  // Rows: warp w takes tokens w, w + 8, ...; lane l channels 4l .. 4l + 3.
-  for (int r = warp; r < C; r += 8) {
-    const int64_t t = tc0 + r;
-    uint2 qv = make_uint2(0u, 0u), kv = make_uint2(0u, 0u);
-    float4 lg = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < nv) {
-      qv = *reinterpret_cast<const uint2*>(qb + brow * p.qs[0] + t * p.qs[1] + h * p.qs[2] + 4 * lane);
-      kv = *reinterpret_cast<const uint2*>(kb + brow * p.ks[0] + t * p.ks[1] + h * p.ks[2] + 4 * lane);
-      const float4 z = *reinterpret_cast<const float4*>(p.gate + brow * p.gs[0] + t * p.gs[1] + h * p.gs[2] + 4 * lane);
-      lg = make_float4(softplus_log_decay(sc, z.x) * LOG2E, softplus_log_decay(sc, z.y) * LOG2E,
-                       softplus_log_decay(sc, z.z) * LOG2E, softplus_log_decay(sc, z.w) * LOG2E);
-    }
-    if (p.qk_l2norm) {
-      float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y), k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
-      float ssq = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
-      float ssk = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
+  // Rows: warp w takes tokens w, w + 8, ...; lane l channels 4l .. 4l + 3, in two batches of four rows
+  // whose loads are all issued before the first is used.
 #pragma unroll
-      for (int m = 16; m >= 1; m >>= 1) {
-        ssq += __shfl_xor_sync(0xffffffffu, ssq, m);
-        ssk += __shfl_xor_sync(0xffffffffu, ssk, m);
+  for (int half = 0; half < 2; ++half) {
+    uint2 qv[4], kv[4];
+    float4 zv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = warp + 8 * (4 * half + i);
+      const int64_t t = tc0 + r;
+      qv[i] = kv[i] = make_uint2(0u, 0u);
+      zv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nv) {
+        qv[i] = *reinterpret_cast<const uint2*>(qb + brow * p.qs[0] + t * p.qs[1] + h * p.qs[2] + 4 * lane);
+        kv[i] = *reinterpret_cast<const uint2*>(kb + brow * p.ks[0] + t * p.ks[1] + h * p.ks[2] + 4 * lane);
+        zv[i] = *reinterpret_cast<const float4*>(p.gate + brow * p.gs[0] + t * p.gs[1] + h * p.gs[2] + 4 * lane);
       }
-      const float fq = l2norm_scale(ssq), fk = l2norm_scale(ssk);
-      qv = make_uint2(pack_bf16(q01.x * fq, q01.y * fq), pack_bf16(q23.x * fq, q23.y * fq));
-      kv = make_uint2(pack_bf16(k01.x * fk, k01.y * fk), pack_bf16(k23.x * fk, k23.y * fk));
     }
-    *reinterpret_cast<uint2*>(sq + r * KD + 4 * lane) = qv;
-    *reinterpret_cast<uint2*>(sk + r * KD + 4 * lane) = kv;
-    *reinterpret_cast<float4*>(sg + r * KD + 4 * lane) = lg;
-    if (lane == 0)
-      sbeta[r] = r < nv ? beta_value(__ldg(p.beta + brow * p.bs[0] + t * p.bs[1] + h * p.bs[2]), p.beta_sigmoid) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = warp + 8 * (4 * half + i);
+      const float4 z = zv[i];
+      const float4 lg = r < nv ? make_float4(softplus_log_decay(sc, z.x) * LOG2E, softplus_log_decay(sc, z.y) * LOG2E,
+                                             softplus_log_decay(sc, z.z) * LOG2E, softplus_log_decay(sc, z.w) * LOG2E)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      uint2 qr = qv[i], kr = kv[i];
+      if (p.qk_l2norm) {
+        float2 q01 = unpack_bf16(qr.x), q23 = unpack_bf16(qr.y), k01 = unpack_bf16(kr.x), k23 = unpack_bf16(kr.y);
+        float ssq = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
+        float ssk = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+          ssq += __shfl_xor_sync(0xffffffffu, ssq, m);
+          ssk += __shfl_xor_sync(0xffffffffu, ssk, m);
+        }
+        const float fq = l2norm_scale(ssq), fk = l2norm_scale(ssk);
+        qr = make_uint2(pack_bf16(q01.x * fq, q01.y * fq), pack_bf16(q23.x * fq, q23.y * fq));
+        kr = make_uint2(pack_bf16(k01.x * fk, k01.y * fk), pack_bf16(k23.x * fk, k23.y * fk));
+      }
+      *reinterpret_cast<uint2*>(sq + r * KD + 4 * lane) = qr;
+      *reinterpret_cast<uint2*>(sk + r * KD + 4 * lane) = kr;
+      *reinterpret_cast<float4*>(sg + r * KD + 4 * lane) = lg;
+      if (lane == 0) {
+        const int64_t t = tc0 + r;
+        sbeta[r] = r < nv ? beta_value(__ldg(p.beta + brow * p.bs[0] + t * p.bs[1] + h * p.bs[2]), p.beta_sigmoid) : 0.f;
+      }
+    }
   }
   __syncthreads();
   // G: the running log2-decay within each 16-token block, one (block, channel) column per thread.
@@ -281,6 +298,9 @@ __global__ void __launch_bounds__(NTHREADS) softplus_diag_kernel(ScanParams p, u
     }
   }
   __syncthreads();
+  // One warp per (block a, column j): each lane sums its four channels for every row t >= j of the block
+  // (v[t] for A_qk, v[16 + t] for A_kk), then one reduce-scatter over the warp leaves lane l with the
+  // total of entry l: A_qk[t = l][j] for l < 16, A_kk[t = l - 16][j] otherwise.
   for (int item = warp; item < 64; item += 8) {
     const int a = item >> 4, j = item & 15, rj = 16 * a + j;
     float kj[4], gj[4];
@@ -289,10 +309,12 @@ __global__ void __launch_bounds__(NTHREADS) softplus_diag_kernel(ScanParams p, u
       kj[m] = __bfloat162float(sk[rj * KD + lane + 32 * m]);
       gj[m] = sg[rj * KD + lane + 32 * m];
     }
+    float v[32];
+#pragma unroll
     for (int t = 0; t < 16; ++t) {
-      const int rt = 16 * a + t;
       float sqk = 0.f, skk = 0.f;
       if (t >= j) {  // uniform across the warp
+        const int rt = 16 * a + t;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int c = lane + 32 * m;
@@ -300,16 +322,31 @@ __global__ void __launch_bounds__(NTHREADS) softplus_diag_kernel(ScanParams p, u
           sqk = fmaf(__bfloat162float(sq[rt * KD + c]), w, sqk);
           skk = fmaf(__bfloat162float(sk[rt * KD + c]), w, skk);
         }
+      }
+      v[t] = sqk;
+      v[16 + t] = skk;
+    }
+    int first = 0;
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) {
-          sqk += __shfl_xor_sync(0xffffffffu, sqk, m);
-          skk += __shfl_xor_sync(0xffffffffu, skk, m);
+    for (int m = 16, nl = 32; m >= 1; m >>= 1, nl >>= 1) {
+      const bool up = (lane & m) != 0;
+      const int hn = nl / 2;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i < hn) {
+          const float send = up ? v[i] : v[i + hn];
+          const float keep = up ? v[i + hn] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
         }
       }
-      if (lane == 0) {
-        out[(a * 16 + t) * 16 + j] = t > j ? skk * sbeta[rt] : 0.f;
-        out[1024 + (a * 16 + t) * 16 + j] = sqk;
-      }
+      if (up) first += hn;
+    }
+    // first == lane
+    if (first < 16) {
+      out[1024 + (a * 16 + first) * 16 + j] = v[0];
+    } else {
+      const int t = first - 16;
+      out[(a * 16 + t) * 16 + j] = t > j ? v[0] * sbeta[16 * a + t] : 0.f;
     }
   }
 }
