@@ -103,3 +103,111 @@ def block_factored_a(q, k, G, pairwise_diag=False, blk=16, dtype=np.float32):
                     blockA = np.tril(blockA)
                 A[ta, tb] = blockA
     return A, worst
+
+
+def chunkwise_backward_head(q, k, v, alpha, beta, S0, d_o, d_sf, C):
+    """Gradients of one head's scan through the chunkwise form (the derivation a chunked backward kernel
+    follows), in fp64. Inputs as for ``chunkwise_head`` plus d_o [T,V] = dL/do and d_sf [K,V] = dL/dS_T.
+    Returns dq, dk, dv, dalpha, dbeta, dS0.
+
+    Per chunk, with G the chunk-local inclusive cumulative log-decay, R[t,i,c] = exp(G_tc - G_ic) (i <= t),
+    M_q = sum_c q k R (lower, diagonal kept), M_k = sum_c k k R (strictly lower), A_kk = Diag(beta) M_k,
+    T = (I + A_kk)^-1, TB = T Diag(beta), W = TB (K*Gamma), Ut = TB V, U = Ut - W S0,
+    O = (Q*Gamma) S0 + M_q U, S_C = Diag(gamma_C) S0 + (K*gamma_C/Gamma)^T U, the adjoints are
+        dU = M_q^T dO + (K*gamma_C/Gamma) dS_C,  dS0 = (Q*Gamma)^T dO + Diag(gamma_C) dS_C - W^T dU,
+        dTB = dU V^T - dU S0^T (K*Gamma)^T,  dT = dTB Diag(beta),  dA_kk = -T^T dT T^T (strictly lower),
+    and the bilinear forms M_q, M_k and the Gamma factors give dq, dk and dG; dlog(alpha) is the reverse
+    cumulative sum of dG within the chunk. Chunks are walked backwards from the last, each chunk's dS0 being
+    the previous chunk's dS_C; the chunk-start states come from a forward pass."""
+    T_, K = q.shape
+    Vd = v.shape[1]
+    la = np.log(alpha)
+    starts = list(range(0, T_, C))
+    S = np.array(S0, dtype=np.float64, copy=True)
+    S_start = []
+    for start in starts:  # forward: the state at every chunk start
+        S_start.append(S.copy())
+        sl = slice(start, min(start + C, T_))
+        _, S = chunkwise_head(q[sl], k[sl], v[sl], alpha[sl], beta[sl], S, C)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dla, dbeta = np.zeros_like(la), np.zeros_like(beta)
+    dS = np.array(d_sf, dtype=np.float64, copy=True)
+    for ci in range(len(starts) - 1, -1, -1):
+        sl = slice(starts[ci], min(starts[ci] + C, T_))
+        n = sl.stop - sl.start
+        Q, Kc, Vc, b, S0c, dO = q[sl], k[sl], v[sl], beta[sl], S_start[ci], d_o[sl]
+        G = np.cumsum(la[sl], axis=0)
+        Gam = np.exp(G)
+        diff = G[:, None, :] - G[None, :, :]
+        low_incl = np.tril(np.ones((n, n), dtype=bool))
+        low = np.tril(np.ones((n, n), dtype=bool), -1)
+        R = np.where(low_incl[:, :, None], np.exp(np.minimum(diff, 0.0)), 0.0)
+        Mq = np.einsum("tc,ic,tic->ti", Q, Kc, R)
+        Mk = np.where(low, np.einsum("tc,ic,tic->ti", Kc, Kc, R), 0.0)
+        A = b[:, None] * Mk
+        Tm = np.linalg.inv(np.eye(n) + A)
+        TB = Tm * b[None, :]
+        KG = Kc * Gam
+        W = TB @ KG
+        Ut = TB @ Vc
+        U = Ut - W @ S0c
+        QG = Q * Gam
+        gC = np.exp(G[-1])
+        KT = Kc * np.exp(G[-1][None, :] - G)
+        # adjoints
+        dU = Mq.T @ dO + KT @ dS
+        dMq = np.where(low_incl, dO @ U.T, 0.0)
+        dQG = dO @ S0c.T
+        dS0 = QG.T @ dO + gC[:, None] * dS - W.T @ dU
+        dKT = U @ dS.T
+        dgC = np.sum(dS * S0c, axis=1)
+        dW = -dU @ S0c.T
+        dTB = dU @ Vc.T + dW @ KG.T
+        dv[sl] += TB.T @ dU
+        dKG = TB.T @ dW
+        dT = dTB * b[None, :]
+        dbeta[sl] += np.sum(dTB * Tm, axis=0)
+        dA = np.where(low, -Tm.T @ dT @ Tm.T, 0.0)
+        dbeta[sl] += np.sum(dA * Mk, axis=1)
+        dMk = dA * b[:, None]
+        dG = np.zeros_like(G)
+        # M_q[t,i] = sum_c Q_tc K_ic R_tic
+        Pq = dMq[:, :, None] * Q[:, None, :] * Kc[None, :, :] * R
+        dq[sl] += np.einsum("ti,ic,tic->tc", dMq, Kc, R)
+        dk[sl] += np.einsum("ti,tc,tic->ic", dMq, Q, R)
+        dG += Pq.sum(axis=1) - Pq.sum(axis=0)
+        # M_k[t,i] = sum_c K_tc K_ic R_tic (strictly lower)
+        Pk = dMk[:, :, None] * Kc[:, None, :] * Kc[None, :, :] * R
+        dk[sl] += np.einsum("ti,ic,tic->tc", dMk, Kc, R) + np.einsum("ti,tc,tic->ic", dMk, Kc, R)
+        dG += Pk.sum(axis=1) - Pk.sum(axis=0)
+        # the Gamma factors
+        dq[sl] += dQG * Gam
+        dG += dQG * QG
+        dk[sl] += dKG * Gam
+        dG += dKG * KG
+        dk[sl] += dKT * np.exp(G[-1][None, :] - G)
+        dG -= dKT * KT
+        dG[-1] += np.sum(dKT * KT, axis=0) + dgC * gC
+        dla[sl] += np.cumsum(dG[::-1], axis=0)[::-1]
+        dS = dS0
+    return dq, dk, dv, dla / alpha, dbeta, dS
+
+
+def chunkwise_backward(q, k, v, alpha, beta, S0, d_o, d_sf, C):
+    """[B,T,H,*] inputs (S0, d_sf [B,H,K,V] or None). Returns a dict of fp64 gradients keyed like
+    ``oracle.scan_backward``: q, k, v, alpha, beta, initial_state."""
+    q, k, v, alpha, beta, d_o = (np.asarray(x, dtype=np.float64) for x in (q, k, v, alpha, beta, d_o))
+    B, T, H, K = q.shape
+    V = v.shape[-1]
+    out = {n: np.zeros_like(x) for n, x in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta))}
+    out["initial_state"] = np.zeros((B, H, K, V))
+    for b_ in range(B):
+        for h in range(H):
+            s0 = np.zeros((K, V)) if S0 is None else np.asarray(S0[b_, h], dtype=np.float64)
+            dsf = np.zeros((K, V)) if d_sf is None else np.asarray(d_sf[b_, h], dtype=np.float64)
+            r = chunkwise_backward_head(q[b_, :, h], k[b_, :, h], v[b_, :, h], alpha[b_, :, h], beta[b_, :, h],
+                                        s0, d_o[b_, :, h], dsf, C)
+            for name, g in zip(("q", "k", "v", "alpha", "beta"), r[:5]):
+                out[name][b_, :, h] = g
+            out["initial_state"][b_, h] = r[5]
+    return out

@@ -501,3 +501,25 @@ def test_block_factorisation_is_safe_for_the_bounded_gate():
     A_split, worst = block_factored_a(q, k, G, pairwise_diag=False)
     assert worst <= 1.0 and np.all(np.isfinite(A_split))                      # e^80 at most on the diagonal
     np.testing.assert_allclose(A_split, exact, rtol=0, atol=1e-5)
+
+
+@pytest.mark.parametrize("C", [1, 4, 16, 64])
+def test_chunkwise_backward_derivation_matches_the_oracle_gradients(C):
+    # The adjoint of the chunkwise form (tests/chunkwise_fp64.py: dU, dS0, dT through the UT transform's
+    # inverse, the bilinear forms A_qk and A_kk, the Gamma factors, dlog(alpha) as a reverse cumulative sum),
+    # walked chunk by chunk from the end, equals the token-level autograd gradients of eq. 1 for every chunk
+    # length, a ragged last chunk included.
+    from tests.chunkwise_fp64 import chunkwise_backward
+    rng = np.random.default_rng(3)
+    B, T, H, K, V = 1, 37, 2, 6, 5
+    q, k = rng.standard_normal((B, T, H, K)), rng.standard_normal((B, T, H, K)) * 0.5
+    v = rng.standard_normal((B, T, H, V))
+    alpha = np.exp(-rng.uniform(0.01, 2.0, (B, T, H, K)))
+    beta = rng.uniform(0.1, 0.9, (B, T, H))
+    s0 = rng.standard_normal((B, H, K, V)) * 0.3
+    do = rng.standard_normal((B, T, H, V))
+    dsf = rng.standard_normal((B, H, K, V)) * 0.3
+    ref = oracle.scan_backward(q, k, v, alpha, beta, s0, do, dsf)
+    got = chunkwise_backward(q, k, v, alpha, beta, s0, do, dsf, C)
+    for name in ref:
+        np.testing.assert_allclose(got[name], ref[name], rtol=0, atol=1e-12 * float(np.abs(ref[name]).max()))
