@@ -211,3 +211,85 @@ def chunkwise_backward(q, k, v, alpha, beta, S0, d_o, d_sf, C):
                 out[name][b_, :, h] = g
             out["initial_state"][b_, h] = r[5]
     return out
+
+
+def chunkwise_backward_split(q, k, v, alpha, beta, S0, d_o, d_sf, C):
+    """``chunkwise_backward_head`` rearranged into the three passes a chunked backward runs as kernels:
+    (1) per chunk, in parallel, the state-independent operands (the forward's, plus dO); (2) one reverse
+    recurrence over chunks carrying dS, which needs only dU = A_qk^T dO + (K*gamma_C/Gamma) dS_C and
+    dS0 = (Q*Gamma)^T dO + Diag(gamma_C) dS_C - W^T dU, i.e. the affine map
+    dS0 = (Q*Gamma - A_qk W)^T dO + (Diag(gamma_C) - W^T (K*gamma_C/Gamma)) dS_C, and emits dU per chunk;
+    (3) per chunk, in parallel, every other gradient from dU and the chunk-start state S0.
+    One head, inputs as for ``chunkwise_backward_head``; same outputs."""
+    T_, K = q.shape
+    la = np.log(alpha)
+    starts = list(range(0, T_, C))
+    # forward states at chunk starts (the forward's recurrence)
+    S = np.array(S0, dtype=np.float64, copy=True)
+    S_start = []
+    for start in starts:
+        S_start.append(S.copy())
+        sl = slice(start, min(start + C, T_))
+        _, S = chunkwise_head(q[sl], k[sl], v[sl], alpha[sl], beta[sl], S, C)
+    # pass 1: state-independent operands per chunk
+    ops = []
+    for start in starts:
+        sl = slice(start, min(start + C, T_))
+        n = sl.stop - sl.start
+        Q, Kc, b = q[sl], k[sl], beta[sl]
+        G = np.cumsum(la[sl], axis=0)
+        Gam = np.exp(G)
+        diff = G[:, None, :] - G[None, :, :]
+        low_incl = np.tril(np.ones((n, n), dtype=bool))
+        low = np.tril(np.ones((n, n), dtype=bool), -1)
+        R = np.where(low_incl[:, :, None], np.exp(np.minimum(diff, 0.0)), 0.0)
+        Mq = np.einsum("tc,ic,tic->ti", Q, Kc, R)
+        Mk = np.where(low, np.einsum("tc,ic,tic->ti", Kc, Kc, R), 0.0)
+        Tm = np.linalg.inv(np.eye(n) + b[:, None] * Mk)
+        TB = Tm * b[None, :]
+        W = TB @ (Kc * Gam)
+        KT = Kc * np.exp(G[-1][None, :] - G)
+        ops.append(dict(sl=sl, n=n, G=G, Gam=Gam, R=R, Mq=Mq, Mk=Mk, Tm=Tm, TB=TB, W=W, KT=KT, QG=Q * Gam,
+                        gC=np.exp(G[-1])))
+    # pass 2: reverse recurrence over dS, emitting dU and dS_C per chunk
+    dS = np.array(d_sf, dtype=np.float64, copy=True)
+    dU_all, dSC_all = [None] * len(starts), [None] * len(starts)
+    for ci in range(len(starts) - 1, -1, -1):
+        o = ops[ci]
+        dO = d_o[o["sl"]]
+        dU = o["Mq"].T @ dO + o["KT"] @ dS
+        dU_all[ci], dSC_all[ci] = dU, dS
+        dS = o["QG"].T @ dO + o["gC"][:, None] * dS - o["W"].T @ dU
+    # pass 3: the remaining gradients per chunk, from dU, dS_C and S0
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dla, dbeta = np.zeros_like(la), np.zeros_like(beta)
+    for ci, o in enumerate(ops):
+        sl, n = o["sl"], o["n"]
+        Q, Kc, Vc, b, S0c, dO = q[sl], k[sl], v[sl], beta[sl], S_start[ci], d_o[sl]
+        dU, dSC = dU_all[ci], dSC_all[ci]
+        G, Gam, R, Mq, Mk, Tm, TB, KT, gC = (o[x] for x in ("G", "Gam", "R", "Mq", "Mk", "Tm", "TB", "KT", "gC"))
+        KG = Kc * Gam
+        U = TB @ Vc - o["W"] @ S0c
+        low_incl = np.tril(np.ones((n, n), dtype=bool))
+        low = np.tril(np.ones((n, n), dtype=bool), -1)
+        dMq = np.where(low_incl, dO @ U.T, 0.0)
+        dQG = dO @ S0c.T
+        dKT = U @ dSC.T
+        dgC = np.sum(dSC * S0c, axis=1)
+        dW = -dU @ S0c.T
+        dTB = dU @ Vc.T + dW @ KG.T
+        dv[sl] = TB.T @ dU
+        dKG = TB.T @ dW
+        dA = np.where(low, -Tm.T @ (dTB * b[None, :]) @ Tm.T, 0.0)
+        dbeta[sl] = np.sum(dTB * Tm, axis=0) + np.sum(dA * Mk, axis=1)
+        dMk = dA * b[:, None]
+        Pq = dMq[:, :, None] * Q[:, None, :] * Kc[None, :, :] * R
+        Pk = dMk[:, :, None] * Kc[:, None, :] * Kc[None, :, :] * R
+        dq[sl] = np.einsum("ti,ic,tic->tc", dMq, Kc, R) + dQG * Gam
+        dk[sl] = (np.einsum("ti,tc,tic->ic", dMq, Q, R) + np.einsum("ti,ic,tic->tc", dMk, Kc, R)
+                  + np.einsum("ti,tc,tic->ic", dMk, Kc, R) + dKG * Gam + dKT * np.exp(G[-1][None, :] - G))
+        dG = (Pq.sum(axis=1) - Pq.sum(axis=0) + Pk.sum(axis=1) - Pk.sum(axis=0) + dQG * o["QG"] + dKG * KG
+              - dKT * KT)
+        dG[-1] += np.sum(dKT * KT, axis=0) + dgC * gC
+        dla[sl] = np.cumsum(dG[::-1], axis=0)[::-1]
+    return dq, dk, dv, dla / alpha, dbeta, dS

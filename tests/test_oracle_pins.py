@@ -523,3 +523,25 @@ def test_chunkwise_backward_derivation_matches_the_oracle_gradients(C):
     got = chunkwise_backward(q, k, v, alpha, beta, s0, do, dsf, C)
     for name in ref:
         np.testing.assert_allclose(got[name], ref[name], rtol=0, atol=1e-12 * float(np.abs(ref[name]).max()))
+
+
+@pytest.mark.parametrize("C", [4, 16, 64])
+def test_chunkwise_backward_three_pass_split_matches_the_oracle(C):
+    # The same gradients computed as a chunked backward's kernels would: state-independent operands per
+    # chunk, one reverse recurrence over dS that emits dU, then every other gradient per chunk in parallel.
+    from tests.chunkwise_fp64 import chunkwise_backward_split
+    rng = np.random.default_rng(5)
+    T, K, V = 45, 7, 4
+    q, k = rng.standard_normal((T, K)), rng.standard_normal((T, K)) * 0.5
+    v = rng.standard_normal((T, V))
+    alpha = np.exp(-rng.uniform(0.01, 2.0, (T, K)))
+    beta = rng.uniform(0.1, 0.9, T)
+    s0 = rng.standard_normal((K, V)) * 0.3
+    do = rng.standard_normal((T, V))
+    dsf = rng.standard_normal((K, V)) * 0.3
+    ref = oracle.scan_backward(q[None, :, None], k[None, :, None], v[None, :, None], alpha[None, :, None],
+                               beta[None, :, None], s0[None, None], do[None, :, None], dsf[None, None])
+    got = chunkwise_backward_split(q, k, v, alpha, beta, s0, do, dsf, C)
+    for g, name in zip(got, ("q", "k", "v", "alpha", "beta", "initial_state")):
+        r = ref[name][0, :, 0] if name != "initial_state" else ref[name][0, 0]
+        np.testing.assert_allclose(g, r, rtol=0, atol=1e-12 * float(np.abs(r).max()))
