@@ -10,6 +10,13 @@ Workloads (H=96, K=V=128, synthetic seeded inputs from ``workloads.py``):
   One step = one in-place ``kda_decode_step_logits`` call (gate inside the
   step). Reported in the ``decode`` object as state GB/s (2*4*K*V*B*H bytes per
   step) and steps/s.
+* varlen, long_kv -- the 16 packed sequences of 512..8192 tokens (H=96, own
+  initial states) and the long K != V batch (B=4, T=16384, H=32, V=256, initial
+  states), each one ``kda_prefill_logits`` call per step; the ``varlen`` and
+  ``long_kv`` objects carry tokens/s, the HBM roofline of their algorithmic
+  bytes (states included), e2e and the oracle on a sample of heads.
+* softplus, backward -- the prefill workload through Kimi Linear's unbounded
+  gate, and the gradients from the logits (their own objects).
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronise, CUDA events on the stream the kernels are launched on,
@@ -77,8 +84,8 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
     return n_elems * (es_in + es_out)
 
 
-# DRAM bytes (read + write) per launch of each step, from one ncu capture of its kernels (commands and
-# per-kernel values in profiles/dram_traffic__bench_steps.md). They hold only for the kernel sources they were
+# DRAM bytes (read + write) per launch of each step, from one ncu capture of its kernels (dram__bytes_read.sum +
+# dram__bytes_write.sum of every kernel the step launches). They hold only for the kernel sources they were
 # taken on, so the sources' sha256 is kept beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
     # chunk_intra_kernel 404,795,392 + 359,710,208; chunk_state_kernel 506,546,432 + 84,204,288
@@ -360,8 +367,9 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
 
 
 def softplus_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
-    """The prefill workload through Kimi Linear's unbounded gate (gate="softplus"): the pairwise
-    diagonal-block pre-pass, kernel P and kernel S; device-timed only."""
+    """The prefill workload through Kimi Linear's unbounded gate (gate="softplus"): kernel P (with the
+    pairwise diagonal tiles of the blocks whose decay leaves the factorisation's range) and kernel S;
+    device-timed only."""
     w = W.PREFILL
     d = W.make_scan_inputs(w)
     B, T, H, K, V = w.B, w.T, w.H, w.K, w.V
@@ -382,12 +390,88 @@ def softplus_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
     achieved = pb / (ms / 1e3) / 1e9
     return {
         "workload": w.name + "_softplus_gate", "value": value, "unit": "tokens/s", "ms_per_step": total_ms / steps,
-        "steps": steps, "gpu_launches": 3 * steps,  # diagonal-block pre-pass, kernel P, kernel S
+        "steps": steps, "gpu_launches": 2 * steps,  # kernel P, kernel S
         "kernels_ms": {"prefill_logits_softplus": ms},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": measured_traffic("softplus"), "kernel": "kda_prefill_logits (KDA_GATE_SOFTPLUS)",
                      "bytes_per_launch": pb, "ms_per_launch": ms, "peak_source": f"{peak_src} hbm_gbs"},
     }
+
+
+def workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, w, cpu_heads):
+    """Throughput of one more prefill workload through the same call as the headline (kda_prefill_logits,
+    two-kernel path, gate from the logits): the 16 packed variable-length sequences with their own initial
+    states, or the long K != V batch. tokens/s, the HBM roofline of its algorithmic bytes, e2e through
+    pinned host buffers and the oracle on a sample of heads."""
+    d = W.make_scan_inputs(w)
+    cu = d["cu_seqlens"]
+    B, T, H, K, V = d["q"].shape[0], d["q"].shape[1], w.H, w.K, w.V
+    N = B if cu is None else cu.numel() - 1
+    g = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in d.items()}
+    o = torch.empty(B, T, H, V, device=dev, dtype=torch.bfloat16)
+    sf = torch.empty(N, H, K, V, device=dev, dtype=torch.float32)
+    ws = torch.empty(max(kda.prefill_workspace_bytes(B, T, H, K, V, 0 if cu is None else N, torch.bfloat16), 1),
+                     device=dev, dtype=torch.uint8)
+
+    def fn():
+        kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], w.g_min, g["beta"], g["initial_state"],
+                           g["cu_seqlens"], out=o, final_state=sf, workspace=ws)
+
+    steps = max(3, min(args.steps, 20))
+    sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    total_ms, (ms,) = timed_loop([fn], steps, args.warmup, world, stream, sampler)
+    value, total_ms = weak_scaling_value(B * T * steps, total_ms, world)
+    pb = prefill_bytes(B, T, H, K, V, N, N)
+    achieved = pb / (ms / 1e3) / 1e9
+    flops = prefill_flops(B, T, H, K, V)
+    res = {
+        "workload": w.name, "value": value, "unit": "tokens/s", "ms_per_step": total_ms / steps, "steps": steps,
+        "tokens_per_step": B * T, "gpu_launches": 2 * steps,  # kernel P, kernel S
+        "kernels_ms": {"prefill_logits": ms},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "kernel": "kda_prefill_logits", "bytes_per_launch": pb, "ms_per_launch": ms,
+                     "peak_source": f"{peak_src} hbm_gbs",
+                     "tensor": {"tflops_at_C64_formula": flops / (ms / 1e3) / 1e12, "peak": bf16_peak,
+                                "frac": flops / (ms / 1e3) / 1e12 / bf16_peak, "flops_per_launch": flops}},
+        "clocks": sampler.summary() if sampler else None,
+    }
+    if not args.no_e2e:
+        names = ("q", "k", "v", "z", "A_log", "beta", "initial_state")
+        host = {n: d[n].pin_memory() for n in names}
+        o_host = torch.empty(B, T, H, V, dtype=torch.bfloat16).pin_memory()
+        sf_host = torch.empty(N, H, K, V, dtype=torch.float32).pin_memory()
+        dev_in = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
+        h2d = sum(x.numel() * x.element_size() for x in host.values())
+        d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * sf_host.element_size()
+
+        def e2e_fn():
+            for n, x in host.items():
+                dev_in[n].copy_(x, non_blocking=True)
+            kda.prefill_logits(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["z"], dev_in["A_log"], w.g_min,
+                               dev_in["beta"], dev_in["initial_state"], g["cu_seqlens"], out=o, final_state=sf,
+                               workspace=ws)
+            o_host.copy_(o, non_blocking=True)
+            sf_host.copy_(sf, non_blocking=True)
+
+        e2e_steps = 3
+        e2e_total, _ = timed_loop([e2e_fn], e2e_steps, 1, world, stream)
+        e2e_total = max_over_ranks(e2e_total, world)
+        res["e2e"] = {"value": B * T * world / (e2e_total / e2e_steps / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle._load()
+        hs = list(range(cpu_heads))
+        s0 = d["initial_state"][:, hs] if d["initial_state"] is not None else None
+        t_start = time.perf_counter()
+        alpha = oracle.bounded_decay(d["z"][:, :, hs], d["A_log"][hs], w.g_min)
+        oracle.scan(d["q"][:, :, hs], d["k"][:, :, hs], d["v"][:, :, hs], alpha, d["beta"][:, :, hs], s0, cu)
+        dt = time.perf_counter() - t_start
+        res["cpu_baseline"] = {"value": B * T * cpu_heads / H / dt, "unit": "tokens/s", "cores": oracle.max_threads(),
+                               "kind": "oracle",
+                               "sample": f"{w.name}, {cpu_heads} of {H} heads, every token; fp64 gate + "
+                                         f"token-by-token scan; {dt:.2f} s; tokens/s scaled to all heads"}
+    return res
 
 
 def backward_bytes(B, T, H, K, V, es=2):
@@ -528,6 +612,11 @@ def gpu_arm(args, rank, world, local):
     if args.workload in ("all", "softplus"):
         spl = softplus_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
         torch.cuda.empty_cache()
+    more = {}
+    for key, wl, heads in (("varlen", W.VARLEN, 16), ("long_kv", W.LONG_KV, 4)):
+        if args.workload in ("all", key):
+            more[key] = workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, wl, heads)
+            torch.cuda.empty_cache()
     bwd = None
     if args.workload in ("all", "backward"):
         bwd = backward_leg(args, kda, dev, stream, rank, world, hbm, peak_src)
@@ -535,7 +624,7 @@ def gpu_arm(args, rank, world, local):
             bwd["cpu_baseline"] = cpu_backward_sample()
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if pre is None and dec is None:  # single-leg profiling run
-        return {"metric": METRIC, "workload_only": args.workload, "backward": bwd, "softplus": spl}
+        return {"metric": METRIC, "workload_only": args.workload, "backward": bwd, "softplus": spl, **more}
     if pre is None:  # decode-only profiling run
         return {"metric": METRIC, "workload_only": "decode", "decode": dec}
     w = pre["workload"]
@@ -566,6 +655,7 @@ def gpu_arm(args, rank, world, local):
         line["decode"] = dec
     if spl is not None:
         line["softplus"] = spl
+    line.update(more)
     if bwd is not None:
         line["backward"] = bwd
     if cpu is not None:
@@ -642,7 +732,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--cpu-heads", type=int, default=0, help="heads in the oracle sample (0: auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "softplus", "backward"], default="all",
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "softplus", "varlen", "long_kv", "backward"],
+                    default="all",
                     help="one leg alone (profiling runs); the JSON line needs 'all'")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end legs")
     args = ap.parse_args(argv)

@@ -76,10 +76,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                                         i64, i64, i64, i64, i64, lp, vp, vp]
     lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, i64, i64, i64, i64, lp, vp, vp]
     u32 = ctypes.c_uint
-    lib.kda_prefill_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, u32, vp, vp, vp, i64,
+    lib.kda_prefill_logits.argtypes = [vp, vp, vp, i32, vp, vp, vp, ctypes.c_float, vp, u32, vp, vp, vp, i64,
                                        i64, i64, i64, i64, i64, lp, vp, vp, ctypes.c_size_t, vp]
-    lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, ctypes.c_float, vp, u32, vp, i64, i64, i64, i64,
-                                           lp, vp, vp]
+    lib.kda_decode_step_logits.argtypes = [vp, vp, vp, i32, vp, vp, vp, ctypes.c_float, vp, u32, vp, i64, i64, i64,
+                                           i64, lp, vp, vp]
     lib.kda_scan_backward_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
     lib.kda_scan_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, lp,
                                       vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
@@ -251,10 +251,11 @@ def _prefill(q, k, v, gate, beta, initial_state, cu_seqlens, gate_is_log, output
             cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
             _stream(dev)))
     else:
-        A_log, g_min, flags = logits
+        A_log, g_min, flags, dt_bias = logits
         _check("kda_prefill_logits", lib.kda_prefill_logits(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
-            A_log.data_ptr(), g_min, beta.data_ptr(), flags, s0_ptr, sf_ptr,
+            A_log.data_ptr(), None if dt_bias is None else dt_bias.data_ptr(), g_min, beta.data_ptr(), flags,
+            s0_ptr, sf_ptr,
             cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out.data_ptr(), ws_ptr, ws_bytes,
             _stream(dev)))
     return out, final_state
@@ -296,7 +297,7 @@ def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.T
                    g_min: float, beta: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
                    cu_seqlens: Optional[torch.Tensor] = None, *, qk_l2norm: bool = False,
                    beta_logits: bool = False, state_layout: str = "kv", gate: str = "bounded",
-                   output_final_state: bool = True,
+                   dt_bias: Optional[torch.Tensor] = None, output_final_state: bool = True,
                    out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None,
                    use_workspace: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -306,15 +307,25 @@ def prefill_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.T
     K per (token, head); ``beta_logits``: ``beta`` holds logits and the kernels apply the sigmoid;
     ``state_layout="vk"``: the states are ``[N,H,V,K]`` (value-by-key) instead of ``[N,H,K,V]``;
     ``gate="softplus"``: the logits feed Kimi Linear's unbounded gate ``g = -exp(A_log) softplus(z)``
-    (``g_min`` unused; chunked with its diagonal blocks formed pairwise when a workspace is used, token by
-    token otherwise). Other arguments as in ``prefill``."""
+    (``g_min`` unused). ``dt_bias [H,K]`` fp32 (optional) is added to ``z`` before either gate. Other
+    arguments as in ``prefill``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
     flags = ((KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
              | _layout_flag(state_layout) | _gate_flag(gate))
+    bias = _bias(dt_bias, q.shape[2], q.shape[3])
     return _prefill(q, k, v, z, beta, initial_state, cu_seqlens, False, output_final_state, out, final_state,
-                    workspace, use_workspace, logits=(A_log.contiguous(), float(g_min), flags), gate_name="z")
+                    workspace, use_workspace, logits=(A_log.contiguous(), float(g_min), flags, bias), gate_name="z")
+
+
+def _bias(dt_bias: Optional[torch.Tensor], H: int, K: int) -> Optional[torch.Tensor]:
+    if dt_bias is None:
+        return None
+    _cuda(dt_bias, "dt_bias")
+    if dt_bias.shape != (H, K) or dt_bias.dtype != torch.float32:
+        raise ValueError("dt_bias must be fp32 [H,K]")
+    return dt_bias.contiguous()
 
 
 NOALLOC_SCRATCH_BYTES = 128 << 20  # the library's static scratch (KDA_NOALLOC_SCRATCH_BYTES)
@@ -374,7 +385,7 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
     """One token against the kept ``state [B,H,K,V]`` (fp32, updated in place). Returns ``o [B,H,V]``.
 
     q, k ``[B,H,K]`` (or ``[B,1,H,K]``), v ``[B,H,V]``, gate ``[B,H,K]`` fp32, beta ``[B,H]`` fp32.
-    ``logits=(A_log, g_min)`` is the internal form of ``decode_step_logits``.
+    ``logits=(A_log, g_min, flags, dt_bias)`` is the internal form of ``decode_step_logits``.
     """
     q, k, v, gate = (x[:, 0] if x.dim() == 4 else x for x in (q, k, v, gate))
     if beta.dim() == 3:
@@ -404,10 +415,11 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
             KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), state.data_ptr(),
             B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
     else:
-        A_log, g_min, flags = logits
+        A_log, g_min, flags, dt_bias = logits
         _check("kda_decode_step_logits", lib.kda_decode_step_logits(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
-            A_log.data_ptr(), g_min, beta.data_ptr(), flags, state.data_ptr(),
+            A_log.data_ptr(), None if dt_bias is None else dt_bias.data_ptr(), g_min, beta.data_ptr(), flags,
+            state.data_ptr(),
             B, H, K, V, ctypes.byref(layout), out.data_ptr(), _stream(q.device)))
     return out
 
@@ -415,17 +427,18 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.T
 def decode_step_logits(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, z: torch.Tensor, A_log: torch.Tensor,
                        g_min: float, beta: torch.Tensor, state: torch.Tensor, *, qk_l2norm: bool = False,
                        beta_logits: bool = False, state_layout: str = "kv", gate: str = "bounded",
-                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                       dt_bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """``decode_step`` fed with the decay logits ``z [B,H,K]`` (fp32): the step evaluates the bounded gate
     itself (``kda_decode_step_logits``). ``A_log [H]`` fp32 on the device; ``g_min < 0``; ``qk_l2norm``,
-    ``beta_logits``, ``state_layout`` (``state`` is ``[B,H,V,K]`` for ``"vk"``) and ``gate`` as in
-    ``prefill_logits``."""
+    ``beta_logits``, ``state_layout`` (``state`` is ``[B,H,V,K]`` for ``"vk"``), ``gate`` and ``dt_bias`` as
+    in ``prefill_logits``."""
     _cuda(A_log, "A_log")
     if A_log.shape != (q.shape[-2],) or A_log.dtype != torch.float32:
         raise ValueError("A_log must be fp32 [H]")
     flags = ((KDA_QK_L2NORM if qk_l2norm else 0) | (KDA_BETA_LOGITS if beta_logits else 0)
              | _layout_flag(state_layout) | _gate_flag(gate))
-    return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min), flags))
+    bias = _bias(dt_bias, q.shape[-2], q.shape[-1])
+    return decode_step(q, k, v, z, beta, state, out=out, logits=(A_log.contiguous(), float(g_min), flags, bias))
 
 
 def scan_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,

@@ -18,11 +18,14 @@
 // of block b,
 //   q_t exp(G_t - G_ic) = [q_t exp(G_t - G_{s_a})] exp(G_{s_a} - G_{r_b}) [k_i exp(G_{r_b} - G_i)]
 // for t in block a, i in block b <= a. The bracketed factors are <= 1; the
-// middle per-channel factor is <= 1 off the diagonal and at most the decay of
-// 15 tokens on it, which the lower bound on g (clamped at -5.5 here) keeps
-// below e^83, inside the bf16/fp32 range ("KDA cheat sheet", Lower-bounded
-// decay: the bound is what lets every tile, the diagonal included, be a dense
-// matmul). Q*Gamma, K*Gamma and K*gamma_C/Gamma are <= 1 times q or k.
+// middle per-channel factor is <= 1 off the diagonal and the reciprocal of the
+// block's whole decay on it, which a lower bound on g keeps in range (g >= -5
+// gives at most e^80; "KDA cheat sheet", Lower-bounded decay: the bound is what
+// lets every tile, the diagonal included, be a dense matmul). A block whose
+// decay on some channel leaves that range (a steeper or unbounded gate, alpha
+// near 0) gets its diagonal tiles pair by pair instead (diag_pairwise), with
+// running products of alpha that never overflow. Q*Gamma, K*Gamma and
+// K*gamma_C/Gamma are <= 1 times q or k.
 //
 // Organisation. One CTA (8 warps) owns one (sequence, head, 128-wide V-tile)
 // and walks its chunks in order; K = 128. The state is kept transposed,
@@ -129,6 +132,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
 
   // decay-pass ownership: channel pair (c0, c0+1) of block da
   const int c0 = 2 * (tid & 63), da = tid >> 6;
+  const float2 bias2 = load_bias2(p, h, c0);
 
   Prefetch pf;
   if (n_chunks > 0) {
@@ -195,18 +199,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_prefill_kernel(ScanParams p
       bw[tid] = beta_value(bw[tid], 1);
     }
     if (p.qk_l2norm) l2norm_qk(pf, vec + VEC_D, tid, da);
+    int pairwise;  // blocks whose diagonal tiles are formed pair by pair
     {
       float2 al[16];
-      decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
+      decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, bias2, al);
       __syncthreads();
+      pairwise = pairwise_blocks(sm, LY);
       decay_step2(sm, LY, pf, da, c0, al);
+      if (pairwise) diag_pairwise(sm, LY, pf, al, beta_s, da, pairwise);  // CTA-uniform
     }
     __syncthreads();  // scaled tiles and vectors ready; the q/k/g registers are free
 
     if (has_next) load_qkg(x, tn0, nvn, c0, da, pf);
 
     // ---- A_kk, then the inverse (warps 0-3) alongside A_qk (warps 4-7) ----------------------------
-    intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+    intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq, pairwise);
     fence_async_smem();
     __syncthreads();  // every operand of MMA group 1 is in shared memory
 
@@ -367,14 +374,15 @@ size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t n_seq) {
 }
 
 cudaError_t launch_chunk(const ScanParams& p, void* ws, size_t ws_bytes, cudaStream_t s) {
-  if (ws != nullptr && ws_bytes >= split_workspace_bytes(p.B, p.T, p.H, p.N, p.cu != nullptr))
+  if (ws != nullptr && ws_bytes >= split_workspace_bytes(p.B, p.T, p.H, p.N, p.cu != nullptr) && split_maps_ok(p))
     return launch_chunk_split(p, ws, s);
   // The shared-memory opt-in is per device; remember which devices have it.
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;  // one configuration bit per device
+  const uint64_t bit = 1ull << dev;
   if (!(configured.load(std::memory_order_relaxed) & bit)) {
     e = cudaFuncSetAttribute(chunk_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;

@@ -17,13 +17,20 @@ constexpr int KD = 128;   // key dim
 constexpr int VT = 128;   // value columns per state tile
 constexpr int NTHREADS = 256;
 constexpr float LOG2E = 1.4426950408889634f;
-constexpr float G2_MIN = -5.5f * LOG2E;  // lower clamp of the per-token log2-decay
+// Range of the block-boundary factorisation. A per-token log2-decay below L2_FLOOR (alpha = 0 included) is
+// raised to it: alpha < 2^-126 and alpha = 0 differ by less than fp32 resolves next to any other term. A
+// 16-token block whose log2-decay sum on some channel is below BLOCK_SAFE would need a diagonal pair factor
+// above 2^120; such blocks take the pairwise diagonal path (diag_pairwise) instead. A per-token bound of
+// g >= -5 (the bounded gate at g_min = -5) keeps every block sum >= -115.4 in log2, inside the range.
+constexpr float L2_FLOOR = -126.f;
+constexpr float BLOCK_SAFE = -120.f;
 
 // fp32 vector area written by the decay pass (offsets in floats).
 constexpr int VEC_D = 0;          // [10][128] bf16 exp(G_{s_a} - G_{r_b}), pairs a >= b (640 floats)
 constexpr int VEC_GAM = 640;      // [128]     gamma_C
 constexpr int VEC_TOT = 768;      // [4][128]  per-block log2-decay sums
-constexpr int VEC_FLOATS = 1280;
+constexpr int VEC_FLAG = 1280;    // [8] int   per warp: one of its channels' block sums is below BLOCK_SAFE
+constexpr int VEC_FLOATS = 1288;
 
 // Shared-memory offsets (bytes) of the tiles the state-independent phases use. Every bf16
 // tile has 128-byte rows with the 128-byte swizzle; 128-column tiles are two 8 KB atoms.
@@ -201,6 +208,12 @@ struct ChunkCtx {
   int64_t qst, kst, vst, gst, bst;       // element strides between tokens
 };
 
+// The logits' bias of channels (c0, c0 + 1) of head h, or zeros.
+__device__ __forceinline__ float2 load_bias2(const ScanParams& p, int h, int c0) {
+  if (!p.dt_bias || p.gate_mode < GATE_LOGITS) return make_float2(0.f, 0.f);
+  return __ldg(reinterpret_cast<const float2*>(p.dt_bias + (size_t)h * KD + c0));
+}
+
 // Registers holding one thread's share of a chunk's q, k, g: channels c0, c0+1 of the 16 tokens
 // of block a (thread = (channel pair, block)).
 struct Prefetch {
@@ -258,12 +271,12 @@ __device__ __forceinline__ void load_vb(const ChunkCtx& x, uint32_t vbase, uint3
 // columns, with the per-pair decay factor D_ab applied to the row operand. The warp takes tiles
 // first, first + stride, ... (nt of them) and runs their k-loops interleaved so the MMA chains
 // overlap. A_qk is stored as a bf16 K-major operand (diagonal blocks masked to i <= t); A_kk as
-// fp32 [64][64] with beta_t applied and diagonal blocks masked to i < t. With QK_T, A_qk is stored
-// transposed ([i][t], the MN-major form of the same operand).
-template <int NTMAX, bool QK_T = false>
+// fp32 [64][64] with beta_t applied and diagonal blocks masked to i < t. The diagonal blocks of the
+// blocks set in `pairwise` (bit a: block a) are not stored: diag_pairwise has written them.
+template <int NTMAX>
 __device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const IntraLayout& L, int off_rows, int first,
                                         int stride, int nt, int lane, int g, int tq, const float* beta_s,
-                                        bool is_qk) {
+                                        bool is_qk, int pairwise) {
   const float* vec = reinterpret_cast<const float*>(sm + L.vec);
   int ta[NTMAX], tbk[NTMAX], tid_[NTMAX];
 #pragma unroll
@@ -307,6 +320,7 @@ __device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const In
   for (int n = 0; n < NTMAX; ++n) {
     if (n >= nt) continue;
     const int a = ta[n], b = tbk[n];
+    if (a == b && ((pairwise >> a) & 1)) continue;
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -319,12 +333,7 @@ __device__ __forceinline__ void a_tiles(unsigned char* sm, uint32_t sb, const In
             v0 = (i0 <= t) ? v0 : 0.f;
             v1 = (i0 + 1 <= t) ? v1 : 0.f;
           }
-          if (QK_T) {
-            *reinterpret_cast<__nv_bfloat16*>(sm + L.aqk + sw_e(i0, t, 8192)) = __float2bfloat16_rn(v0);
-            *reinterpret_cast<__nv_bfloat16*>(sm + L.aqk + sw_e(i0 + 1, t, 8192)) = __float2bfloat16_rn(v1);
-          } else {
-            *reinterpret_cast<uint32_t*>(sm + L.aqk + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
-          }
+          *reinterpret_cast<uint32_t*>(sm + L.aqk + sw_e(t, i0, 8192)) = pack_bf16(v0, v1);
         } else {
           const float bt = beta_s[t];
           v0 = (a > b || i0 < t) ? v0 * bt : 0.f;
@@ -378,39 +387,126 @@ __device__ __forceinline__ void l2norm_qk(Prefetch& pf, float* red, int tid, int
   }
 }
 
-// The log2-decay of one channel from the gate value x in gate mode `mode` (alpha, g = log alpha, or
-// the decay logits z with sc = e^{A_h}).
+// The log2-decay of one channel from the gate value x in gate mode `mode` (alpha, g = log alpha, the
+// bounded gate's logits z, or the unbounded gate's logits, both with sc = e^{A_h}), raised to L2_FLOOR.
 __device__ __forceinline__ float log2_decay(int mode, float x, float sc, float g_min) {
-  return mode == GATE_LOGITS ? bounded_log_decay(sc, x, g_min) * LOG2E : (mode == 1 ? x * LOG2E : lg2(x));
+  float l;
+  if (mode == GATE_LOGITS)
+    l = bounded_log_decay(sc, x, g_min) * LOG2E;
+  else if (mode == GATE_SOFTPLUS)
+    l = softplus_log_decay(sc, x) * LOG2E;
+  else
+    l = mode == KDA_GATE_LOG ? x * LOG2E : lg2(x);
+  return fmaxf(l, L2_FLOOR);  // fmaxf(-inf, floor) = floor: alpha = 0 stays finite in log space
 }
 
 // Decay pass, step 1: the per-token log2-decay of channels (c0, c0+1) over the 16 tokens of block
-// da (clamped at G2_MIN; 0 past the end of the sequence), their retention factors, and the block
-// sum, published to VEC_TOT. With UNBOUNDED the logits feed Kimi Linear's gate g = -e^{A_h} softplus(z)
-// and nothing is clamped: every factor this pass forms is then still <= 1 except the diagonal-block
-// pair factors, which the caller replaces (see softplus_diag_kernel).
-template <bool UNBOUNDED = false>
+// da (0 past the end of the sequence), their retention factors, and the block sum, published to
+// VEC_TOT. `bias` is the logits' per-channel bias (0 without one). Each warp also records in VEC_FLAG
+// whether one of its channels' block sums lies below BLOCK_SAFE (read back by pairwise_blocks after
+// the caller's barrier).
 __device__ __forceinline__ void decay_step1(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int nv,
-                                            int da, int c0, int mode, float sc, float g_min, float2 (&al)[16]) {
+                                            int da, int c0, int mode, float sc, float g_min, float2 bias,
+                                            float2 (&al)[16]) {
   float* vec = reinterpret_cast<float*>(sm + L.vec);
   float2 run = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float2 l = make_float2(0.f, 0.f);
     if (16 * da + i < nv) {
-      if (UNBOUNDED) {
-        l.x = softplus_log_decay(sc, pf.g[i].x) * LOG2E;
-        l.y = softplus_log_decay(sc, pf.g[i].y) * LOG2E;
-      } else {
-        l.x = fmaxf(log2_decay(mode, pf.g[i].x, sc, g_min), G2_MIN);
-        l.y = fmaxf(log2_decay(mode, pf.g[i].y, sc, g_min), G2_MIN);
-      }
+      l.x = log2_decay(mode, gate_input(mode, pf.g[i].x, bias.x), sc, g_min);
+      l.y = log2_decay(mode, gate_input(mode, pf.g[i].y, bias.y), sc, g_min);
     }
     run.x += l.x;
     run.y += l.y;
     al[i] = make_float2(ex2(l.x), ex2(l.y));
   }
   *reinterpret_cast<float2*>(vec + VEC_TOT + da * 128 + c0) = run;
+  const unsigned out_of_range = __any_sync(0xffffffffu, run.x < BLOCK_SAFE || run.y < BLOCK_SAFE);
+  if ((threadIdx.x & 31) == 0) reinterpret_cast<int*>(vec + VEC_FLAG)[threadIdx.x >> 5] = out_of_range ? 1 : 0;
+}
+
+// After decay_step1 and a barrier: bit a set when block a needs its diagonal blocks pairwise (the
+// two warps 2a, 2a + 1 own its channels).
+__device__ __forceinline__ int pairwise_blocks(const unsigned char* sm, const IntraLayout& L) {
+  const int* f = reinterpret_cast<const int*>(sm + L.vec) + VEC_FLAG;
+  int m = 0;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) m |= (f[2 * a] | f[2 * a + 1]) << a;
+  return m;
+}
+
+// The diagonal 16x16 blocks of A_qk and A_kk of the blocks set in `pairwise`, pair by pair, without the
+// block-boundary factorisation (whose diagonal factor 2^{-block sum} is out of range there):
+//   A_qk[t][j] = sum_c q_tc k_jc w_tjc (j <= t),  A_kk[t][j] = beta_t sum_c k_tc k_jc w_tjc (j < t),
+//   w_tjc = prod_{m = j+1..t} alpha_mc,
+// each w built as a running product (every factor <= 1, so nothing overflows and a decay that underflows
+// gives the right limit, 0). Run by all 256 threads after decay_step2 (a CTA-uniform call): the thread that
+// owns channels (c0, c0 + 1) of block da forms its two channels' share of all 32 entries of each column j
+// (16 of A_qk, 16 of A_kk), a reduce-scatter over the warp leaves lane l with entry l, and the two warps of
+// the block meet through unused (off-diagonal) parts of the A_kk area, written over by a_tiles later. The
+// results go straight to A_kk (fp32) and A_qk (bf16); a_tiles then skips these diagonal blocks.
+__device__ __forceinline__ void diag_pairwise(unsigned char* sm, const IntraLayout& L, const Prefetch& pf,
+                                              const float2 (&al)[16], const float* beta_s, int da, int pairwise) {
+  const int lane = threadIdx.x & 31, hw = (threadIdx.x >> 5) & 1;  // the block's first or second warp
+  const bool mine = (pairwise >> da) & 1;
+  float* akk = reinterpret_cast<float*>(sm + L.akk);
+  // A row of the A_kk area that holds warp 2da + 1's entries of column j: row 16da + j, the columns of
+  // blocks da + 1 and da + 2 (mod 4), never a diagonal block.
+  auto scratch = [&](int j, int l) { return akk + (16 * da + j) * 64 + 16 * ((da + 1 + (l >> 4)) & 3) + (l & 15); };
+  float res[16];
+  if (mine) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float2 kj = unpack_bf16(pf.k[j]);
+      float v[32];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) v[t] = v[16 + t] = 0.f;
+      float2 w = make_float2(kj.x, kj.y);  // k_j * w_tj
+#pragma unroll
+      for (int t = j; t < 16; ++t) {
+        if (t > j) {
+          w.x *= al[t].x;
+          w.y *= al[t].y;
+        }
+        const float2 qt = unpack_bf16(pf.q[t]), kt = unpack_bf16(pf.k[t]);
+        v[t] = fmaf(qt.x, w.x, qt.y * w.y);
+        v[16 + t] = fmaf(kt.x, w.x, kt.y * w.y);
+      }
+      // reduce-scatter: lane l ends with the warp's total of entry l
+#pragma unroll
+      for (int m = 16, nl = 32; m >= 1; m >>= 1, nl >>= 1) {
+        const bool up = (lane & m) != 0;
+        const int hn = nl / 2;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i < hn) {
+            const float send = up ? v[i] : v[i + hn];
+            const float keep = up ? v[i + hn] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+          }
+        }
+      }
+      res[j] = v[0];
+      if (hw) *scratch(j, lane) = v[0];
+    }
+  }
+  __syncthreads();
+  if (mine && !hw) {
+    const int t = lane & 15;
+    const float bt = beta_s[16 * da + t];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float sum = res[j] + *scratch(j, lane);
+      if (lane < 16) {
+        *reinterpret_cast<__nv_bfloat16*>(sm + L.aqk + sw_e(16 * da + t, 16 * da + j, 8192)) =
+            __float2bfloat16_rn(t >= j ? sum : 0.f);
+      } else {
+        akk[(16 * da + t) * 64 + 16 * da + j] = t > j ? sum * bt : 0.f;
+      }
+    }
+  }
+  // The next barrier (the caller's) orders these writes before a_tiles and the inverse.
 }
 
 // Decay pass, step 2 (after a barrier): block-boundary decay vectors and the six scaled tiles
@@ -464,16 +560,14 @@ __device__ __forceinline__ void decay_step2(unsigned char* sm, const IntraLayout
   }
 }
 
-// Zeroes the six 16x16 blocks above the diagonal of a [64][64] bf16 K-major tile (below it when
-// TRANSPOSED), using the `count` threads with index `idx` in [0, count).
-template <bool TRANSPOSED = false>
+// Zeroes the six 16x16 blocks above the diagonal of a [64][64] bf16 K-major tile, using the `count`
+// threads with index `idx` in [0, count).
 __device__ __forceinline__ void zero_upper_blocks(unsigned char* sm, int off, int idx, int count) {
   for (int e = idx; e < 6 * 64; e += count) {
     const int pr = e >> 6, r = (e >> 2) & 15, q4 = e & 3;  // block pair, row, group of 4 columns
     const int a = pr < 3 ? 0 : (pr < 5 ? 1 : 2);
     const int b = pr < 3 ? pr + 1 : (pr < 5 ? pr - 1 : 3);
-    const int ra = TRANSPOSED ? b : a, cb = TRANSPOSED ? a : b;
-    *reinterpret_cast<uint2*>(sm + off + sw_e(16 * ra + r, 16 * cb + 4 * q4, 8192)) = make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(sm + off + sw_e(16 * a + r, 16 * b + 4 * q4, 8192)) = make_uint2(0u, 0u);
   }
 }
 
@@ -541,31 +635,20 @@ __device__ __forceinline__ void inverse_warps0to3(unsigned char* sm, uint32_t sb
   }
 }
 
-// Barrier over the 256 threads of warps 0-7: the whole CTA (barrier 0), or named barrier 2 in a
-// kernel whose other warps run different code.
-template <bool NAMED>
-__device__ __forceinline__ void sync_compute() {
-  if (NAMED)
-    asm volatile("bar.sync 2, 256;" ::: "memory");
-  else
-    __syncthreads();
-}
-
 // The state-independent phases after the decay pass: A_kk on all warps; then the inverse on warps
-// 0-3 while warps 4-7 form A_qk (and zero its upper blocks; transposed with QK_T). Ends with a
-// barrier over warps 0-7 (named barrier 2 with NAMED, else the CTA barrier).
-template <bool QK_T = false, bool NAMED = false>
+// 0-3 while warps 4-7 form A_qk (and zero its upper blocks). Diagonal blocks set in `pairwise` are the
+// ones diag_pairwise wrote. Ends with a CTA barrier.
 __device__ __forceinline__ void intra_phases(unsigned char* sm, uint32_t sb, const IntraLayout& L, const float* beta_s,
-                                             int tid, int warp, int lane, int g, int tq) {
-  a_tiles<2>(sm, sb, L, L.ke, warp, 8, warp < 2 ? 2 : 1, lane, g, tq, beta_s, /*is_qk=*/false);
-  sync_compute<NAMED>();  // A_kk ready; Ke is dead
+                                             int tid, int warp, int lane, int g, int tq, int pairwise) {
+  a_tiles<2>(sm, sb, L, L.ke, warp, 8, warp < 2 ? 2 : 1, lane, g, tq, beta_s, /*is_qk=*/false, pairwise);
+  __syncthreads();  // A_kk ready; Ke is dead
   if (warp < 4) {
     inverse_warps0to3(sm, sb, L, beta_s, tid, warp, lane, g, tq);
   } else {
-    a_tiles<3, QK_T>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
-    zero_upper_blocks<QK_T>(sm, L.aqk, tid - 128, 128);  // the MMAs read whole rows of A_qk
+    a_tiles<3>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true, pairwise);
+    zero_upper_blocks(sm, L.aqk, tid - 128, 128);  // the MMAs read whole rows of A_qk
   }
-  sync_compute<NAMED>();
+  __syncthreads();
 }
 
 }  // namespace

@@ -18,13 +18,15 @@
 // S, and kernel P writes each block's operand pairs in the order that chunk's parity needs.
 // The price of the split is the workspace traffic (one write and one read of ~1 KB per token-head).
 //
-// With Kimi Linear's unbounded gate (KDA_GATE_SOFTPLUS) a pre-pass, softplus_diag_kernel, first forms the
-// diagonal 16x16 blocks of A_kk and A_qk pair by pair (their block-boundary factorisation would need the
-// reciprocal of a whole block's decay, which that gate does not bound), and chunk_intra_kernel<true> takes
-// them from the workspace in place of its own diagonal tiles; every other factor stays <= 1.
+// Decays steep enough to put a 16-token block outside the range of the block-boundary factorisation (any
+// gate: alpha near 0, g_min below about -5.2, Kimi Linear's unbounded gate) are detected per block by the
+// decay pass, and those blocks' diagonal 16x16 tiles are formed pair by pair instead (diag_pairwise in
+// chunk_common.cuh); every other factor stays <= 1 for any decay.
 //
 // Workspace slots. Chunk j of sequence n has slot n * ceil(T/64) + j without cu_seqlens, and
 // floor(cu[n]/64) + n + j with them (unique: a sequence's slots end before the next one's begin).
+#include <cuda.h>
+
 #include <atomic>
 
 #include "chunk_common.cuh"
@@ -36,35 +38,49 @@ __device__ int g_split_timeout = 0;
 
 namespace {
 
-// One workspace block = the output region of kernel P = the operand buffer of kernel S. All three
-// operand regions are K-major; a pair (X, Y) is stored in that order for an even chunk index j and
-// as (Y, X) for an odd one.
+// One workspace block = the output region of kernel P = the operand buffer of kernel S. A pair (X, Y)
+// of operands sharing a product is stored in that order for an even chunk index j and as (Y, X) for an
+// odd one.
 constexpr int WB_WQ = 0;         // 32K  two k-atoms (c) of 128 rows: (-W [t][c], Q*Gamma [t][c])
-constexpr int WB_KA = 32768;     // 24K  one k-atom (t) of 192 rows: (A_qk [t'][t], (K*gamma_C/Gamma)^T [c][t])
+constexpr int WB_KA = 32768;     // 24K  MN-major, three 8K n-atoms of 64 rows (the K index t or i):
+                                 //      (A_qk^T [i][t'], K*gamma_C/Gamma [t][c 0..63], [t][c 64..127])
 constexpr int WB_TP = 57344;     // 8K   T' [t][i]
 constexpr int WB_GAM = 65536;    // 512  gamma_C, fp32 [128]
 constexpr int WB_BYTES = 66048;
-// Unbounded gate only: the pairwise diagonal blocks of A_kk and A_qk (see softplus_diag_kernel), written
-// into the T' region before kernel P runs; P reads them there before its final bulk store overwrites it.
-constexpr int WB_DIAG = WB_TP;
-static_assert(2 * 4 * 16 * 16 * 4 <= WB_GAM - WB_TP, "the diagonal blocks fit the T' region");
 
-// Kernel P shared memory (104,192 bytes: two CTAs fit on an SM). Q*Gamma and K*gamma_C/Gamma
-// never touch it: the decay pass writes them from registers straight into the workspace block.
-constexpr int P_QE = 0;                     // 16K Qe [t][c]; after A_qk, -W [t][c] (two 8K atoms)
-constexpr int P_KE = P_QE + 16384;          // 16K Ke [t][c]; after A_kk, the bf16 copy of T
-constexpr int P_KC = P_KE + 16384;          // 16K Kc [t][c]
-constexpr int P_KG = P_KC + 16384;          // 16K K*Gamma [i][c]
-constexpr int P_AKK = P_KG + 16384;         // 16K A_kk fp32
-constexpr int P_AQK = P_AKK + 16384;        // 8K  A_qk [t'][t]  } in block order for odd chunks, where
-constexpr int P_TP = P_AQK + 8192;          // 8K  T'            } A_qk ends the KA region and T' and
-constexpr int P_GAM = P_TP + 8192;          // 512 gamma_C       } gamma_C follow it
-constexpr int P_BETA = P_GAM + 512;         // 256 beta
-constexpr int P_VEC = P_BETA + 256;         // vectors
-constexpr int P_SMEM = P_VEC + VEC_FLOATS * 4;
-static_assert(P_TP - P_AQK == WB_TP - (WB_KA + 16384) && P_GAM - P_TP == WB_GAM - WB_TP, "odd-chunk tail order");
-static_assert(P_TP % 1024 == 0 && P_AQK % 1024 == 0, "swizzle atoms need 1 KB alignment");
+// Kernel P shared memory (111,968 bytes: two CTAs fit on an SM), in three overlapping phases.
+//  Inputs (TMA): q, k as [64-channel half][64 tokens][128 B] and the gate input as [half][64 tokens][256 B].
+//  Operands (written by the decay pass once every input is in registers): the row operand KQ, the column
+//   views VIEW and K*Gamma, all 128-byte-swizzled K-major tiles of 128-byte rows, two 64-channel halves.
+//  After the A products: A_kk (fp32), A_qk^T, T and T' over the dead KQ and VIEW rows, and -W.
+constexpr int P_QS = 0;                     // 16K q staging
+constexpr int P_KS = 16384;                 // 16K k staging
+constexpr int P_GS = 32768;                 // 32K gate-input staging (fp32)
+constexpr int P_KQ = 0;                     // 32K row operand: [half][128 rows][128 B]
+constexpr int VIEW_ROWS = 176;              // views 3, 0, 2, 1 at rows 0, 64, 80, 144
+constexpr int VIEW_HALF = VIEW_ROWS * 128;  // 22,528
+constexpr int P_VIEW = 32768;               // 44K column views: [half][176 rows][128 B]
+constexpr int P_KG = 81920;                 // 16K K*Gamma [half][64 rows][128 B] (4K after VIEW: the second
+                                            //     A product reads 32 rows past the views' end)
+constexpr int P_DIAG = 98304;               // 8K  pairwise diagonal blocks, fp32 [A_kk | A_qk][block][t][j]
+constexpr int P_VEC = 106496;               // vectors (VEC_*)
+constexpr int P_BETA = P_VEC + VEC_FLOATS * 4;  // 256 beta
+constexpr int P_GAM = P_BETA + 256;         // 512 gamma_C (bulk-stored with T')
+constexpr int P_BAR = P_GAM + 512;          // mbarriers (inputs, MMA) and the TMEM base
+constexpr int P_SMEM = P_BAR + 64;
+constexpr int P_AKK = 0;                    // 16K A_kk fp32 [t][i] (beta_t applied, strictly lower)
+constexpr int P_AQKT = 16384;               // 8K  A_qk^T bf16 [i][t] (zero above the diagonal of A_qk)
+constexpr int P_TB = 24576;                 // 8K  T bf16 [t][i]
+constexpr int P_TP = P_VIEW + 8192;         // 8K  T' bf16 [t][i]; the W product (M = 128) also reads the
+                                            //     next 8K, whose rows it discards
+constexpr int P_W = P_VIEW + VIEW_HALF + 8192;  // 16K -W bf16 [half][64 rows][128 B]
+static_assert(P_GS + 32768 <= P_KG && P_VIEW + 2 * VIEW_HALF + 32 * 128 <= P_KG, "staging and view overrun");
+static_assert(P_TP + 16384 <= P_VIEW + VIEW_HALF + 8192 && P_W >= P_VIEW + VIEW_HALF + 8192 && P_W + 16384 <= P_KG,
+              "post-product tiles must not overlap the K*gamma_C/Gamma rows still being stored");
+static_assert(P_KG % 1024 == 0 && P_VIEW % 1024 == 0 && VIEW_HALF % 1024 == 0 && P_TP % 1024 == 0 &&
+              P_W % 1024 == 0 && P_AQKT % 1024 == 0 && P_TB % 1024 == 0, "swizzle atoms need 1 KB alignment");
 static_assert(2 * (P_SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+constexpr uint32_t P_TM_COLS = 256;         // TMEM: A products at columns 0 and 64, W at 128
 
 // Kernel S shared memory: the operand blocks of two chunks and their v tiles.
 constexpr int S_OPS = 0;                    // 2 x operand block (66048 B, padded to 66560)
@@ -138,15 +154,52 @@ __device__ __forceinline__ void bulk_store(unsigned char* dst, uint32_t src, uin
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes) : "memory");
 }
 
-// Decay pass, step 2 of kernel P: the same tiles as decay_step2 (chunk_common.cuh), with Q*Gamma and
-// K*gamma_C/Gamma stored straight into their places in the workspace block. Q*Gamma goes to qg_dst
-// as [t][c] rows of 16 KB k-atoms (a warp's 32 four-byte stores cover one 128-byte swizzled row);
-// K*gamma_C/Gamma goes to kt_dst transposed, [c][t], one 16-byte piece per channel and 8 tokens.
-// Tokens run forward for the E-scaled tiles and backward for the F-scaled ones, so no per-token F
-// array is held in registers.
-__device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch& pf, int da, int c0,
-                                              const float2 (&al)[16], unsigned char* qg_dst, unsigned char* kt_dst) {
-  float* vec = reinterpret_cast<float*>(sm + P_VEC);
+// ---------------------------------------------------------------------------------------------
+// Kernel P: the state-independent operands of one (chunk, head), tcgen05 products fed by TMA.
+//
+// Decay ratios. With e[a] the log2-decay of the chunk up to the end of block a (e[-1] = 0) and G_t the
+// running log2-decay at token t, the ratio 2^{G_t - G_i} (t in block a, i <= t) is split at a reference
+// point R_a of block a: [x_t 2^{G_t - R_a}] [k_i 2^{R_a - G_i}]. R_a = e[a], the end of block a, puts
+// every factor of the column operand at or below 1 (i <= r_a) and bounds the row factor by the block's
+// own decay (at most 2^120 for blocks within range, the g_min argument of the "KDA cheat sheet"). For a
+// block out of range R_a = e[a - 1], the start: the row factor is then <= 1, the cross-block column
+// factors 2^{e[a-1] - G_i} stay <= 1, and only the block's own diagonal tile is lost -- that one is
+// formed pair by pair (diag_pairwise) and substituted when A_kk and A_qk are read back.
+//
+// Products. View a of the column operand holds k_i 2^{R_a - G_i} for the tokens i <= r_a of blocks
+// 0..a (view 3 with R_3 = e[3] is K*gamma_C/Gamma, an operand of kernel S as well). The row operand KQ
+// holds k_t 2^{G_t - R_a} and q_t 2^{G_t - R_a} for every block a. Two M = 128, N = 64, K = 128 products
+// give every pair: rows [view 3 | view 0] against [K_3 | Q_3 | K_0 | Q_0], and [view 2 | view 1] against
+// [K_2 | Q_2 | K_1 | Q_1] (the cross terms between different blocks are computed and discarded), so the
+// accumulator lane is the column index i of A and the accumulator column the row index t. W = T' (K*Gamma)
+// is a third product (M = 128 with the upper 64 rows discarded, N = 128, K = 64).
+// First row of view a (views 3, 0 form the first product's A operand, 2, 1 the second's), and of block a's
+// k rows in KQ (its q rows follow at +16; blocks 3, 0 form the first product's B operand, 2, 1 the second's).
+__device__ __forceinline__ int view_base(int a) { return a == 3 ? 0 : (a == 0 ? 64 : (a == 2 ? 80 : 144)); }
+__device__ __forceinline__ int kq_base(int a) { return a == 3 ? 0 : (a == 0 ? 32 : (a == 2 ? 64 : 96)); }
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int h, int t, int b,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t), "r"(b), "r"(bar)
+      : "memory");
+}
+
+// Tensor maps of the three token tensors kernel P reads: q and k (bf16 boxes of 64 channels x 64
+// tokens) and the gate input (fp32, same boxes).
+struct PMaps {
+  CUtensorMap q, k, g;
+};
+
+// Decay pass, step 2 of kernel P: the row operand KQ, the column views, K*Gamma (smem), Q*Gamma (straight
+// to its place in the workspace block, qg_dst: [t][c] rows of 16 KB k-atoms) and gamma_C. View 3 is
+// K*gamma_C/Gamma unless block 3 is out of range (its reference is then the block's start); in that case
+// K*gamma_C/Gamma goes straight to the workspace too (kt_dst: [t][c] rows of 8 KB n-atoms).
+__device__ __forceinline__ void p_operands(unsigned char* sm, const Prefetch& pf, int da, int c0, int pairwise,
+                                           const float2 (&al)[16], unsigned char* qg_dst, unsigned char* kt_dst) {
+  const float* vec = reinterpret_cast<const float*>(sm + P_VEC);
   float2 e[4];
 #pragma unroll
   for (int b = 0; b < 4; ++b) e[b] = *reinterpret_cast<const float2*>(vec + VEC_TOT + b * 128 + c0);
@@ -155,20 +208,27 @@ __device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch&
     e[b].x += e[b - 1].x;
     e[b].y += e[b - 1].y;
   }
-  // e[b] = log2 Gamma at r_b; log2 Gamma at s_a is e[a-1] (0 for a = 0)
+  // e[b] = log2 Gamma at the end of block b; the start of block a is e[a-1] (0 for a = 0)
+  float2 R[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const float2 st = a == 0 ? make_float2(0.f, 0.f) : e[a - 1];
+    R[a] = ((pairwise >> a) & 1) ? st : e[a];
+  }
   const float2 gs = da == 0 ? make_float2(0.f, 0.f) : (da == 1 ? e[0] : (da == 2 ? e[1] : e[2]));
   const float2 eda = da == 0 ? e[0] : (da == 1 ? e[1] : (da == 2 ? e[2] : e[3]));
-  __nv_bfloat16* D16 = reinterpret_cast<__nv_bfloat16*>(vec + VEC_D);
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    if (b <= da) {
-      const int pair = da * (da + 1) / 2 + b;
-      *reinterpret_cast<uint32_t*>(D16 + pair * 128 + c0) = pack_bf16(ex2(gs.x - e[b].x), ex2(gs.y - e[b].y));
-    }
-  }
+  const float2 Rd = da == 0 ? R[0] : (da == 1 ? R[1] : (da == 2 ? R[2] : R[3]));
   if (da == 0) *reinterpret_cast<float2*>(sm + P_GAM + 4 * c0) = make_float2(ex2(e[3].x), ex2(e[3].y));
-  const float2 GS = make_float2(ex2(gs.x), ex2(gs.y));
-  const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));
+  const float2 GS = make_float2(ex2(gs.x), ex2(gs.y));               // Gamma at the start of the block
+  const float2 DI = make_float2(ex2(gs.x - Rd.x), ex2(gs.y - Rd.y)); // 2^{G_start - R_da} (>= 1)
+  // Column-view scales of this block's tokens: 2^{R_a - e[da]} for views a > da (<= 1); 1 for a = da, or 0
+  // when this block is out of range (its diagonal tile comes from diag_pairwise).
+  float2 SV[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+    SV[a] = a > da ? make_float2(ex2(R[a].x - eda.x), ex2(R[a].y - eda.y))
+                   : (((pairwise >> da) & 1) ? make_float2(0.f, 0.f) : make_float2(1.f, 1.f));
+  const int rk = kq_base(da);
   float2 E = make_float2(1.f, 1.f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -176,227 +236,94 @@ __device__ __forceinline__ void p_decay_step2(unsigned char* sm, const Prefetch&
     E.x *= al[i].x;
     E.y *= al[i].y;
     const float2 qf = unpack_bf16(pf.q[i]), kf = unpack_bf16(pf.k[i]);
-    const uint32_t off = sw_e(t, c0, 8192);
-    const float qex = qf.x * E.x, qey = qf.y * E.y, kex = kf.x * E.x, key = kf.y * E.y;
-    *reinterpret_cast<uint32_t*>(sm + P_QE + off) = pack_bf16(qex, qey);
-    *reinterpret_cast<uint32_t*>(sm + P_KE + off) = pack_bf16(kex, key);
-    *reinterpret_cast<uint32_t*>(sm + P_KG + off) = pack_bf16(kex * GS.x, key * GS.y);
-    *reinterpret_cast<uint32_t*>(qg_dst + sw_e(t, c0, 16384)) = pack_bf16(qex * GS.x, qey * GS.y);
+    const float rx = E.x * DI.x, ry = E.y * DI.y;      // 2^{G_t - R_da}
+    const float gx = E.x * GS.x, gy = E.y * GS.y;      // Gamma_t
+    *reinterpret_cast<uint32_t*>(sm + P_KQ + sw_e(rk + i, c0, 16384)) = pack_bf16(kf.x * rx, kf.y * ry);
+    *reinterpret_cast<uint32_t*>(sm + P_KQ + sw_e(rk + 16 + i, c0, 16384)) = pack_bf16(qf.x * rx, qf.y * ry);
+    *reinterpret_cast<uint32_t*>(sm + P_KG + sw_e(t, c0, 8192)) = pack_bf16(kf.x * gx, kf.y * gy);
+    *reinterpret_cast<uint32_t*>(qg_dst + sw_e(t, c0, 16384)) = pack_bf16(qf.x * gx, qf.y * gy);
   }
-  float2 F = make_float2(1.f, 1.f);
-  float ktx[8], kty[8];  // K*gamma_C/Gamma of channels c0, c0+1 for the 8 tokens of one 16-byte piece
+  const bool kt_apart = (pairwise >> 3) & 1;
+  const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));  // 2^{e[3] - e[da]}
+  float2 F = make_float2(1.f, 1.f);  // 2^{e[da] - G_i}, tokens after i within the block
 #pragma unroll
   for (int i = 15; i >= 0; --i) {
     const int t = 16 * da + i;
     const float2 kf = unpack_bf16(pf.k[i]);
-    const float kfx = kf.x * F.x, kfy = kf.y * F.y;
-    *reinterpret_cast<uint32_t*>(sm + P_KC + sw_e(t, c0, 8192)) = pack_bf16(kfx, kfy);
-    ktx[i & 7] = kfx * PM.x;
-    kty[i & 7] = kfy * PM.y;
-    if ((i & 7) == 0) {  // tokens 16da + i .. +7 complete: piece j = 2da + i/8 of rows c0 and c0 + 1
-      const int j = 2 * da + (i >> 3);
-      const uint4 wx = make_uint4(pack_bf16(ktx[0], ktx[1]), pack_bf16(ktx[2], ktx[3]), pack_bf16(ktx[4], ktx[5]),
-                                  pack_bf16(ktx[6], ktx[7]));
-      const uint4 wy = make_uint4(pack_bf16(kty[0], kty[1]), pack_bf16(kty[2], kty[3]), pack_bf16(kty[4], kty[5]),
-                                  pack_bf16(kty[6], kty[7]));
-      *reinterpret_cast<uint4*>(kt_dst + sw_chunk(c0, j, 0)) = wx;
-      *reinterpret_cast<uint4*>(kt_dst + sw_chunk(c0 + 1, j, 0)) = wy;
-    }
+    const float kx = kf.x * F.x, ky = kf.y * F.y;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+      if (a >= da)
+        *reinterpret_cast<uint32_t*>(sm + P_VIEW + sw_e(view_base(a) + t, c0, VIEW_HALF)) =
+            pack_bf16(kx * SV[a].x, ky * SV[a].y);
+    if (kt_apart) *reinterpret_cast<uint32_t*>(kt_dst + sw_e(t, c0, 8192)) = pack_bf16(kx * PM.x, ky * PM.y);
     F.x *= al[i].x;
     F.y *= al[i].y;
   }
 }
 
-// Kimi Linear's unbounded gate (KDA_GATE_SOFTPLUS), g = -e^{A_h} softplus(z): the diagonal 16x16 blocks
-// of A_kk and A_qk of one (chunk, head), pair by pair. Within a block exp(G_t - G_j) <= 1 for j <= t, but
-// kernel P's block-boundary factorisation splits it as exp(G_t - G_s) exp(G_s - G_j), whose second factor
-// grows with the decay of the whole block, which this gate does not bound. One warp per (block a, column
-// j), lanes over the channels: A_qk[t][j] = sum_c q_tc k_jc exp(G_tc - G_jc) for t >= j and A_kk[t][j] =
-// beta_t sum_c k_tc k_jc exp(G_tc - G_jc) for t > j, with q, k L2-normalised and rounded to bf16 first
-// when the flag asks, and beta from its logits when the flag asks, as kernel P does.
-constexpr int D_Q = 0, D_K = 16384, D_G = 32768, D_BETA = 65536, D_SMEM = D_BETA + 256;
-
-__global__ void __launch_bounds__(NTHREADS, 3) softplus_diag_kernel(ScanParams p, unsigned char* ws) {
-  extern __shared__ __align__(16) unsigned char sm[];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.y;
-  const int64_t slot = blockIdx.x;
-  int n, jc;
-  if (!locate_slot(p, slot, n, jc)) return;  // uniform across the CTA
-  int64_t t0, t1, brow;
-  seq_range(p, n, t0, t1, brow);
-  const int64_t tc0 = t0 + (int64_t)jc * C;
-  const int nv = (int)min((int64_t)C, t1 - tc0);
-  float* out = reinterpret_cast<float*>(ws + ((size_t)slot * p.H + h) * WB_BYTES + WB_DIAG);
-  const float sc = expf(__ldg(p.A_log + h));
-  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.k);
-  __nv_bfloat16* sq = reinterpret_cast<__nv_bfloat16*>(sm + D_Q);
-  __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(sm + D_K);
-  float* sg = reinterpret_cast<float*>(sm + D_G);
-  float* sbeta = reinterpret_cast<float*>(sm + D_BETA);
-
-  // Rows: warp w takes tokens w, w + 8, ...; lane l channels 4l .. 4l + 3, in two batches of four rows
-  // whose loads are all issued before the first is used.
+// diag_pairwise (chunk_common.cuh) with its results in the fp32 buffer `out` [A_kk | A_qk][block][t][j]
+// (A_kk with beta_t applied and zero for j >= t, A_qk zero for j > t); the block's two warps combine their
+// halves of the channels in place there.
+__device__ __forceinline__ void p_diag_pairwise(float* out, const Prefetch& pf, const float2 (&al)[16],
+                                                const float* beta_s, int da, int pairwise) {
+  const int lane = threadIdx.x & 31, hw = (threadIdx.x >> 5) & 1;
+  const bool mine = (pairwise >> da) & 1;
+  // entry l of column j: A_qk[t = l][j] (l < 16) or A_kk[t = l - 16][j]
+  auto slot = [&](int j, int l) { return out + (l < 16 ? 1024 : 0) + (da * 16 + (l & 15)) * 16 + j; };
+  float res[16];
+  if (mine) {
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint2 qv[4], kv[4];
-    float4 zv[4];
+    for (int j = 0; j < 16; ++j) {
+      const float2 kj = unpack_bf16(pf.k[j]);
+      float v[32];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = warp + 8 * (4 * half + i);
-      const int64_t t = tc0 + r;
-      qv[i] = kv[i] = make_uint2(0u, 0u);
-      zv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < nv) {
-        qv[i] = *reinterpret_cast<const uint2*>(qb + brow * p.qs[0] + t * p.qs[1] + h * p.qs[2] + 4 * lane);
-        kv[i] = *reinterpret_cast<const uint2*>(kb + brow * p.ks[0] + t * p.ks[1] + h * p.ks[2] + 4 * lane);
-        zv[i] = *reinterpret_cast<const float4*>(p.gate + brow * p.gs[0] + t * p.gs[1] + h * p.gs[2] + 4 * lane);
-      }
-    }
+      for (int t = 0; t < 16; ++t) v[t] = v[16 + t] = 0.f;
+      float2 w = make_float2(kj.x, kj.y);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = warp + 8 * (4 * half + i);
-      const float4 z = zv[i];
-      const float4 lg = r < nv ? make_float4(softplus_log_decay(sc, z.x) * LOG2E, softplus_log_decay(sc, z.y) * LOG2E,
-                                             softplus_log_decay(sc, z.z) * LOG2E, softplus_log_decay(sc, z.w) * LOG2E)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-      uint2 qr = qv[i], kr = kv[i];
-      if (p.qk_l2norm) {
-        float2 q01 = unpack_bf16(qr.x), q23 = unpack_bf16(qr.y), k01 = unpack_bf16(kr.x), k23 = unpack_bf16(kr.y);
-        float ssq = q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y;
-        float ssk = k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y;
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) {
-          ssq += __shfl_xor_sync(0xffffffffu, ssq, m);
-          ssk += __shfl_xor_sync(0xffffffffu, ssk, m);
+      for (int t = j; t < 16; ++t) {
+        if (t > j) {
+          w.x *= al[t].x;
+          w.y *= al[t].y;
         }
-        const float fq = l2norm_scale(ssq), fk = l2norm_scale(ssk);
-        qr = make_uint2(pack_bf16(q01.x * fq, q01.y * fq), pack_bf16(q23.x * fq, q23.y * fq));
-        kr = make_uint2(pack_bf16(k01.x * fk, k01.y * fk), pack_bf16(k23.x * fk, k23.y * fk));
+        const float2 qt = unpack_bf16(pf.q[t]), kt = unpack_bf16(pf.k[t]);
+        v[t] = fmaf(qt.x, w.x, qt.y * w.y);
+        v[16 + t] = fmaf(kt.x, w.x, kt.y * w.y);
       }
-      *reinterpret_cast<uint2*>(sq + r * KD + 4 * lane) = qr;
-      *reinterpret_cast<uint2*>(sk + r * KD + 4 * lane) = kr;
-      *reinterpret_cast<float4*>(sg + r * KD + 4 * lane) = lg;
-      if (lane == 0) {
-        const int64_t t = tc0 + r;
-        sbeta[r] = r < nv ? beta_value(__ldg(p.beta + brow * p.bs[0] + t * p.bs[1] + h * p.bs[2]), p.beta_sigmoid) : 0.f;
+#pragma unroll
+      for (int m = 16, nl = 32; m >= 1; m >>= 1, nl >>= 1) {
+        const bool up = (lane & m) != 0;
+        const int hn = nl / 2;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i < hn) {
+            const float send = up ? v[i] : v[i + hn];
+            const float keep = up ? v[i + hn] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+          }
+        }
       }
+      res[j] = v[0];
+      if (hw) *slot(j, lane) = v[0];
     }
   }
   __syncthreads();
-  // G: the running log2-decay within each 16-token block, one (block, channel) column per thread.
+  if (mine && !hw) {
+    const int t = lane & 15;
+    const float bt = beta_s[16 * da + t];
 #pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const int col = tid + NTHREADS * m, a = col >> 7, c = col & (KD - 1);
-    float run = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float* x = sg + (16 * a + i) * KD + c;
-      run += *x;
-      *x = run;
-    }
-  }
-  __syncthreads();
-  // One warp per (block a, column j): each lane sums its four channels for every row t >= j of the block
-  // (v[t] for A_qk, v[16 + t] for A_kk), then one reduce-scatter over the warp leaves lane l with the
-  // total of entry l: A_qk[t = l][j] for l < 16, A_kk[t = l - 16][j] otherwise.
-  for (int item = warp; item < 64; item += 8) {
-    const int a = item >> 4, j = item & 15, rj = 16 * a + j;
-    float kj[4], gj[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      kj[m] = __bfloat162float(sk[rj * KD + lane + 32 * m]);
-      gj[m] = sg[rj * KD + lane + 32 * m];
-    }
-    float v[32];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      float sqk = 0.f, skk = 0.f;
-      if (t >= j) {  // uniform across the warp
-        const int rt = 16 * a + t;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int c = lane + 32 * m;
-          const float w = kj[m] * ex2(sg[rt * KD + c] - gj[m]);
-          sqk = fmaf(__bfloat162float(sq[rt * KD + c]), w, sqk);
-          skk = fmaf(__bfloat162float(sk[rt * KD + c]), w, skk);
-        }
-      }
-      v[t] = sqk;
-      v[16 + t] = skk;
-    }
-    int first = 0;
-#pragma unroll
-    for (int m = 16, nl = 32; m >= 1; m >>= 1, nl >>= 1) {
-      const bool up = (lane & m) != 0;
-      const int hn = nl / 2;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if (i < hn) {
-          const float send = up ? v[i] : v[i + hn];
-          const float keep = up ? v[i + hn] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-        }
-      }
-      if (up) first += hn;
-    }
-    // first == lane
-    if (first < 16) {
-      out[1024 + (a * 16 + first) * 16 + j] = v[0];
-    } else {
-      const int t = first - 16;
-      out[(a * 16 + t) * 16 + j] = t > j ? v[0] * sbeta[16 * a + t] : 0.f;
+    for (int j = 0; j < 16; ++j) {
+      const float sum = res[j] + *slot(j, lane);
+      *slot(j, lane) = lane < 16 ? (t >= j ? sum : 0.f) : (t > j ? sum * bt : 0.f);
     }
   }
 }
 
-// The four diagonal 16x16 blocks of A_kk and A_qk for the unbounded gate, formed pairwise by
-// softplus_diag_kernel and stored as fp32 [A_kk | A_qk][block a][t][j] (A_kk with beta_t folded in, zero
-// on and above the diagonal; A_qk zero above it) in the T' region of the chunk's workspace block.
-
-// intra_phases (chunk_common.cuh) for the unbounded gate: the tile products run as usual, then the
-// diagonal blocks, whose block-boundary factorisation needs exp(-decay of 16 tokens) and can overflow,
-// are replaced by the pairwise values from `diag` before the inverse and the W phase read them.
-__device__ __forceinline__ void unbounded_intra_phases(unsigned char* sm, uint32_t sb, const IntraLayout& L,
-                                                       const float* beta_s, int tid, int warp, int lane, int g,
-                                                       int tq, const float* diag) {
-  float dk[4], dq[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    dk[r] = __ldg(diag + tid + NTHREADS * r);
-    dq[r] = __ldg(diag + 1024 + tid + NTHREADS * r);
-  }
-  a_tiles<2>(sm, sb, L, L.ke, warp, 8, warp < 2 ? 2 : 1, lane, g, tq, beta_s, /*is_qk=*/false);
-  __syncthreads();
-  float* akk = reinterpret_cast<float*>(sm + L.akk);
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int e = tid + NTHREADS * r, a = e >> 8, t = (e >> 4) & 15, j = e & 15;
-    akk[(16 * a + t) * 64 + 16 * a + j] = dk[r];
-  }
-  __syncthreads();  // A_kk ready
-  if (warp < 4) {
-    inverse_warps0to3(sm, sb, L, beta_s, tid, warp, lane, g, tq);
-  } else {
-    a_tiles<3>(sm, sb, L, L.qe, warp - 4, 4, (warp - 4) < 2 ? 3 : 2, lane, g, tq, beta_s, /*is_qk=*/true);
-    zero_upper_blocks(sm, L.aqk, tid - 128, 128);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int e = tid + NTHREADS * r, a = e >> 8, t = (e >> 4) & 15, j = e & 15;
-    *reinterpret_cast<__nv_bfloat16*>(sm + L.aqk + sw_e(16 * a + t, 16 * a + j, 8192)) = __float2bfloat16_rn(dq[r]);
-  }
-  // The W phase does not read A_qk; the barrier before the bulk store publishes these writes.
-}
-
-template <bool UNBOUNDED>
-__global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, unsigned char* ws) {
+__global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, unsigned char* ws,
+                                                                  const __grid_constant__ PMaps maps) {
   extern __shared__ __align__(1024) unsigned char sm[];
   const uint32_t sb = smem_u32(sm);
-  // qg and kt are not staged in shared memory by this kernel (p_decay_step2 stores them to the block).
-  constexpr IntraLayout LY{P_QE, P_KE, P_KC, -1, P_KG, -1, P_AKK, P_AQK, P_TP, P_KE, P_VEC};
+  constexpr IntraLayout LY{-1, -1, -1, -1, -1, -1, P_AKK, -1, P_TP, P_TB, P_VEC};
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
   // Kernel S may be scheduled once every CTA of this grid has started; it reads the workspace only
@@ -412,97 +339,189 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   const int64_t tc0 = t0 + (int64_t)j * C;
   const int nv = (int)min((int64_t)C, t1 - tc0);
   unsigned char* blk = ws + ((size_t)slot * p.H + h) * WB_BYTES;
-  const bool even = (j & 1) == 0;  // operand pair order within the block
+  const bool even = (j & 1) == 0;  // operand order within the block's pairs
 
-  ChunkCtx x;
-  x.q = static_cast<const __nv_bfloat16*>(p.q);
-  x.k = static_cast<const __nv_bfloat16*>(p.k);
-  x.v = nullptr;
-  x.gate = p.gate;
-  x.beta = p.beta;
-  x.qrow = brow * p.qs[0] + h * p.qs[2];
-  x.krow = brow * p.ks[0] + h * p.ks[2];
-  x.vrow = 0;
-  x.grow = brow * p.gs[0] + h * p.gs[2];
-  x.boff = brow * p.bs[0] + h * p.bs[2];
-  x.qst = p.qs[1];
-  x.kst = p.ks[1];
-  x.vst = 0;
-  x.gst = p.gs[1];
-  x.bst = p.bs[1];
+  const uint32_t bar_in = sb + P_BAR, bar_mma = sb + P_BAR + 8;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + P_BAR + 16);
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_in));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // q, k and the gate input of the chunk's 64 tokens (rows past the tensor's end read as zeros; rows past
+    // the sequence's end are zeroed below); 64 KB on one barrier.
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_in), "r"(65536) : "memory");
+    const int tt = (int)tc0, bb = (int)brow;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      tma_load_4d(sb + P_QS + half * 8192, &maps.q, 64 * half, h, tt, bb, bar_in);
+      tma_load_4d(sb + P_KS + half * 8192, &maps.k, 64 * half, h, tt, bb, bar_in);
+      tma_load_4d(sb + P_GS + half * 16384, &maps.g, 64 * half, h, tt, bb, bar_in);
+    }
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(P_TM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  float* beta_s = reinterpret_cast<float*>(sm + P_BETA);
+  if (tid < C) {
+    beta_s[tid] = tid < nv ? beta_value(__ldg(p.beta + brow * p.bs[0] + h * p.bs[2] + (tc0 + tid) * p.bs[1]),
+                                        p.beta_sigmoid)
+                           : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
 
   const int c0 = 2 * (tid & 63), da = tid >> 6;
-  float* beta_s = reinterpret_cast<float*>(sm + P_BETA);
-  {
+  const int hc = c0 >> 6, cc = c0 & 63;
+  bool ok = __syncthreads_and(mbar_wait(bar_in, 0, &g_split_timeout));
+  int pairwise = 0;
+  int mma_groups = 0;  // product groups committed to bar_mma (thread 0)
+  if (ok) {
     Prefetch pf;
-    load_qkg(x, tc0, nv, c0, da, pf);
-    if (tid < C) beta_s[tid] = tid < nv ? beta_value(__ldg(x.beta + x.boff + (tc0 + tid) * x.bst), p.beta_sigmoid) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int t = 16 * da + i;
+      const bool v = t < nv;
+      pf.q[i] = v ? *reinterpret_cast<const uint32_t*>(sm + P_QS + hc * 8192 + t * 128 + cc * 2) : 0u;
+      pf.k[i] = v ? *reinterpret_cast<const uint32_t*>(sm + P_KS + hc * 8192 + t * 128 + cc * 2) : 0u;
+      pf.g[i] = v ? *reinterpret_cast<const float2*>(sm + P_GS + hc * 16384 + t * 256 + cc * 4) : make_float2(0.f, 0.f);
+    }
     if (p.qk_l2norm) l2norm_qk(pf, reinterpret_cast<float*>(sm + P_VEC) + VEC_D, tid, da);
     float2 al[16];
-    decay_step1<UNBOUNDED>(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, al);
+    decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, load_bias2(p, h, c0), al);
+    __syncthreads();  // block sums and flags published; every input is in registers (staging is dead)
+    pairwise = pairwise_blocks(sm, LY);
+    p_operands(sm, pf, da, c0, pairwise, al, blk + WB_WQ + (even ? 8192 : 0), blk + WB_KA + (even ? 8192 : 0));
+    if (pairwise) p_diag_pairwise(reinterpret_cast<float*>(sm + P_DIAG), pf, al, beta_s, da, pairwise);
+    fence_async_smem();
+    tc_fence_before();
     __syncthreads();
-    p_decay_step2(sm, pf, da, c0, al, blk + WB_WQ + (even ? 8192 : 0), blk + WB_KA + (even ? 8192 : 0));
+    tc_fence_after();
+    // ---- the A products: [view 3 | view 0] x [K_3 | Q_3 | K_0 | Q_0], [view 2 | view 1] x [K_2 | Q_2 | K_1 | Q_1]
+    if (tid == 0) {
+      constexpr uint32_t id_a = idesc_bf16(64, 0, 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kv = (ks >> 2) * VIEW_HALF + (ks & 3) * 32, kq = (ks >> 2) * 16384 + (ks & 3) * 32;
+        tc_mma(tmem, sdesc(sb + P_VIEW + kv, 16, 1024), sdesc(sb + P_KQ + kq, 16, 1024), id_a, ks > 0);
+        tc_mma(tmem + 64, sdesc(sb + P_VIEW + 80 * 128 + kv, 16, 1024), sdesc(sb + P_KQ + 64 * 128 + kq, 16, 1024),
+               id_a, ks > 0);
+      }
+      tc_commit(bar_mma);
+      mma_groups = 1;
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma, 0, &g_split_timeout));
+    tc_fence_after();
   }
-  __syncthreads();
-  if constexpr (UNBOUNDED) {
-    unbounded_intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq, reinterpret_cast<const float*>(blk + WB_DIAG));
-  } else {
-    intra_phases(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+  if (ok) {
+    // K*gamma_C/Gamma (view 3) goes to the workspace as kernel S's MN-major operand rows [t][c] (when block 3
+    // is out of range the decay pass has stored it already).
+    if (tid == 0 && !((pairwise >> 3) & 1)) {
+      const uint32_t kt = WB_KA + (even ? 8192 : 0);
+      bulk_store(blk + kt, sb + P_VIEW, 8192);
+      bulk_store(blk + kt + 8192, sb + P_VIEW + VIEW_HALF, 8192);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    // ---- read back: warps 0-3 the first product, 4-7 the second; TMEM lane L = 32 (warp & 3) + lane
+    {
+      const int L = 32 * (warp & 3) + lane, second = warp >> 2;
+      const int a = second ? (L < 64 ? 2 : 1) : (L < 64 ? 3 : 0);
+      const int i = L & 63;
+      uint32_t r[32];
+      tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * second + (L < 64 ? 0 : 32), r);
+      const bool from_pairs = ((pairwise >> a) & 1) && (i >> 4) == a;
+      const float* dg = reinterpret_cast<const float*>(sm + P_DIAG);
+      float* akk = reinterpret_cast<float*>(sm + P_AKK);
+      float vq[16];
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int t = 16 * a + jj;
+        float vk = __uint_as_float(r[jj]);
+        vq[jj] = __uint_as_float(r[16 + jj]);
+        if (from_pairs) {
+          vk = dg[(a * 16 + jj) * 16 + (i & 15)];
+          vq[jj] = dg[1024 + (a * 16 + jj) * 16 + (i & 15)];
+        } else {
+          vk = i < t ? vk * beta_s[t] : 0.f;
+          vq[jj] = i <= t ? vq[jj] : 0.f;
+        }
+        akk[t * 64 + i] = vk;
+      }
+      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a, 0)) =
+          make_uint4(pack_bf16(vq[0], vq[1]), pack_bf16(vq[2], vq[3]), pack_bf16(vq[4], vq[5]), pack_bf16(vq[6], vq[7]));
+      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a + 1, 0)) = make_uint4(
+          pack_bf16(vq[8], vq[9]), pack_bf16(vq[10], vq[11]), pack_bf16(vq[12], vq[13]), pack_bf16(vq[14], vq[15]));
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // A_kk and A_qk^T complete
+    if (tid == 0) {
+      bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    // ---- T' = (I + A_kk)^-1 Diag(beta) on warps 0-3
+    if (warp < 4) inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- W = T' (K*Gamma): A = T' (K-major [t][i], rows 64..127 discarded), B = K*Gamma (MN-major [i][c])
+    if (tid == 0) {
+      constexpr uint32_t id_w = idesc_bf16(128, 0, 1);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        tc_mma(tmem + 128, sdesc(sb + P_TP + ks * 32, 16, 1024), sdesc(sb + P_KG + ks * 2048, 8192, 1024), id_w,
+               ks > 0);
+      tc_commit(bar_mma);
+      mma_groups = 2;
+      bulk_store(blk + WB_TP, sb + P_TP, 8192);
+      bulk_store(blk + WB_GAM, sb + P_GAM, 512);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma, 1, &g_split_timeout));
+    tc_fence_after();
   }
-
-  // W = T' (K*Gamma) on mma.sync. Warp w owns columns 16w.. of all 64 rows, so every warp does the
-  // same ten block products of the lower-triangular T'. -W is stored over the dead Qe tile as
-  // [t][c], two 64-column atoms: the rows it takes in the block's K-major pair with Q*Gamma.
-  {
-    float acc[4][2][4];
+  if (ok) {
+    // ---- -W to [half][t][c] (warps 0, 1: channels 0-63; warps 4, 5: 64-127), then to the workspace
+    if ((warp & 3) < 2) {
+      const int t = 32 * (warp & 3) + lane, half = warp >> 2;
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
+      for (int part = 0; part < 2; ++part) {
+        uint32_t r[32];
+        tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 128 + 64 * half + 32 * part, r);
 #pragma unroll
-      for (int jn = 0; jn < 2; ++jn)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[m][jn][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(sb + P_KG + sw_chunk(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * warp + (lane >> 4), 8192), b0, b1,
-                b2, b3);
-#pragma unroll
-      for (int m = kk; m < 4; ++m) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(sb + P_TP + sw_chunk(16 * m + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * kk + (lane >> 4), 8192), a0, a1,
-                a2, a3);
-        mma_bf16(acc[m][0], a0, a1, a2, a3, b0, b1);
-        mma_bf16(acc[m][1], a0, a1, a2, a3, b2, b3);
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<uint4*>(sm + P_W + half * 8192 + sw_chunk(t, 4 * part + q4, 0)) = pack8(r, q4, -1.f);
       }
     }
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-#pragma unroll
-      for (int jn = 0; jn < 2; ++jn)
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int t = 16 * m + g + 8 * hr, c = 16 * warp + 8 * jn + 2 * tq;
-          *reinterpret_cast<uint32_t*>(sm + P_QE + sw_e(t, c, 8192)) =
-              pack_bf16(-acc[m][jn][2 * hr], -acc[m][jn][2 * hr + 1]);
-        }
-  }
-  fence_async_smem();
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t wq = even ? 0 : 8192;
-    bulk_store(blk + WB_WQ + wq, sb + P_QE, 8192);
-    bulk_store(blk + WB_WQ + 16384 + wq, sb + P_QE + 8192, 8192);
-    if (even) {
-      bulk_store(blk + WB_KA, sb + P_AQK, 8192);
-      bulk_store(blk + WB_TP, sb + P_TP, WB_BYTES - WB_TP);
-    } else {
-      bulk_store(blk + WB_KA + 16384, sb + P_AQK, WB_BYTES - (WB_KA + 16384));
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t wq = even ? 0 : 8192;
+      bulk_store(blk + WB_WQ + wq, sb + P_W, 8192);
+      bulk_store(blk + WB_WQ + 16384 + wq, sb + P_W + 8192, 8192);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    // Shared memory must stay valid until the copies have read it; their global writes complete
-    // before the kernel does.
+  }
+  if (tid == 0) {
+    if (!ok) {
+      // A wait expired: give the loads and products that may still be in flight a bounded wait.
+      mbar_wait(bar_in, 0, &g_split_timeout);
+      if (mma_groups >= 1) mbar_wait(bar_mma, 0, &g_split_timeout);
+      if (mma_groups >= 2) mbar_wait(bar_mma, 1, &g_split_timeout);
+    }
+    // Shared memory must stay valid until the stores have read it; their global writes complete before
+    // the kernel does.
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(P_TM_COLS));
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -687,13 +706,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     __syncthreads();
     tc_fence_after();
 
-    // ---- group B: [O^T | S^T] += U^T [A_qk ; (K*gamma_C/Gamma)^T]^T -----------------------------------
+    // ---- group B: [O^T | S^T] += U^T [A_qk ; (K*gamma_C/Gamma)^T]^T, B MN-major (rows: the K index) ------
     if (tid == 0) {
-      constexpr uint32_t id_b = idesc_bf16(192, 0, 0);
+      constexpr uint32_t id_b = idesc_bf16(192, 0, 1);
       const uint32_t d_b = buf ? TM_S : TM_OE;  // [O_e | S] or [S | O_o]
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        tc_mma_ts(tmem + d_b, tmem + TM_UB + 8 * ks, sdesc(ops + WB_KA + ks * 32, 16, 1024), id_b, 1);
+        tc_mma_ts(tmem + d_b, tmem + TM_UB + 8 * ks, sdesc(ops + WB_KA + ks * 2048, 8192, 1024), id_b, 1);
       tc_commit(bar_mma);
     }
   }
@@ -738,7 +757,8 @@ cudaError_t set_smem_once(F* fn, int bytes, std::atomic<uint64_t>& configured) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;  // one configuration bit per device
+  const uint64_t bit = 1ull << dev;
   if (!(configured.load(std::memory_order_relaxed) & bit)) {
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
@@ -760,25 +780,67 @@ size_t split_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, bool va
   return (size_t)split_slots(B, T, N, varlen) * (size_t)H * (size_t)WB_BYTES;
 }
 
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (no link-time libcuda dependency).
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// A [B,T,H,K] token tensor with element strides s = (b, t, h) as a 4-d tensor map (K, H, T, B) read in
+// boxes of 64 channels x 64 tokens of one head. The stride of an extent-1 dimension never moves the
+// pointer; it is given its contiguous value. Returns false when the driver refuses the layout.
+bool token_map(CUtensorMap* m, const void* base, bool bf16, const int64_t s[3], int64_t B, int64_t T, int64_t H,
+               int64_t K) {
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const int64_t es = bf16 ? 2 : 4;
+  const int64_t sh = H > 1 ? s[2] : K;
+  const int64_t st = T > 1 ? s[1] : H * sh;
+  const int64_t sbt = B > 1 ? s[0] : T * st;
+  const cuuint64_t dims[4] = {(cuuint64_t)K, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)(sh * es), (cuuint64_t)(st * es), (cuuint64_t)(sbt * es)};
+  const cuuint32_t box[4] = {64, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool split_maps_ok(const ScanParams& p) {
+  PMaps m;
+  return token_map(&m.q, p.q, true, p.qs, p.B, p.T, p.H, p.K) && token_map(&m.k, p.k, true, p.ks, p.B, p.T, p.H, p.K) &&
+         token_map(&m.g, p.gate, false, p.gs, p.B, p.T, p.H, p.K);
+}
+
 cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
-  const bool unbounded = p.gate_mode == GATE_SOFTPLUS;
-  static std::atomic<uint64_t> cfg_p{0}, cfg_pu{0}, cfg_d{0}, cfg_s{0};
-  cudaError_t e = unbounded ? set_smem_once(chunk_intra_kernel<true>, P_SMEM, cfg_pu)
-                            : set_smem_once(chunk_intra_kernel<false>, P_SMEM, cfg_p);
-  if (e == cudaSuccess && unbounded) e = set_smem_once(softplus_diag_kernel, D_SMEM, cfg_d);
+  static std::atomic<uint64_t> cfg_p{0}, cfg_s{0};
+  cudaError_t e = set_smem_once(chunk_intra_kernel, P_SMEM, cfg_p);
   if (e == cudaSuccess) e = set_smem_once(chunk_state_kernel, S_SMEM, cfg_s);
   if (e != cudaSuccess) return e;
   const int64_t slots = split_slots(p.B, p.T, p.N, p.cu != nullptr);
   if (slots == 0 || p.N == 0) return cudaSuccess;
+  PMaps maps;
+  if (!token_map(&maps.q, p.q, true, p.qs, p.B, p.T, p.H, p.K) ||
+      !token_map(&maps.k, p.k, true, p.ks, p.B, p.T, p.H, p.K) ||
+      !token_map(&maps.g, p.gate, false, p.gs, p.B, p.T, p.H, p.K))
+    return cudaErrorInvalidValue;  // callers check split_maps_ok first
   dim3 gp((unsigned)slots, (unsigned)p.H);
-  if (unbounded) {
-    softplus_diag_kernel<<<gp, NTHREADS, D_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    chunk_intra_kernel<true><<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
-  } else {
-    chunk_intra_kernel<false><<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws));
-  }
+  chunk_intra_kernel<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws), maps);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t grid = (int64_t)p.N * p.H * (p.V / VT);

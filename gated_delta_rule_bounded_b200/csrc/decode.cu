@@ -140,7 +140,10 @@ __global__ void __launch_bounds__(DNT, 1) decode_bulk_kernel(ScanParams p) {
     float* as = reinterpret_cast<float*>(st + L::A);
     // The staged gate row becomes alpha in place, once per head (each row is read by many threads).
     if (p.gate_mode != KDA_GATE_ALPHA) {
-      for (int c = tid; c < DK; c += blockDim.x) as[c] = gate_alpha(p.gate_mode, as[c], sc, p.g_min);
+      for (int c = tid; c < DK; c += blockDim.x) {
+        const float b = p.dt_bias ? __ldg(p.dt_bias + (size_t)(head % p.H) * DK + c) : 0.f;
+        as[c] = gate_alpha(p.gate_mode, gate_input(p.gate_mode, as[c], b), sc, p.g_min);
+      }
       __syncthreads();
     }
     float* S = reinterpret_cast<float*>(st + L::STATE);
@@ -294,7 +297,8 @@ cudaError_t launch_bulk(const ScanParams& p, cudaStream_t s) {
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;  // one configuration bit per device
+  const uint64_t bit = 1ull << dev;
   if (!(configured.load(std::memory_order_relaxed) & bit)) {
     e = cudaFuncSetAttribute(decode_bulk_kernel<TIn, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
     if (e == cudaSuccess)

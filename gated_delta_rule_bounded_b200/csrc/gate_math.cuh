@@ -34,6 +34,10 @@ __device__ __forceinline__ float beta_value(float b, int from_logits) { return f
 // Scale that L2-normalises a q or k row with squared norm `ss` (x / sqrt(ss + 1e-6)).
 __device__ __forceinline__ float l2norm_scale(float ss) { return rsqrtf(ss + 1e-6f); }
 
+// The gate input of one channel: the logits plus the optional per-(head, channel) bias b ("KDA cheat
+// sheet", How the inputs are produced: z = W_up W_down x + b), or alpha / g unchanged.
+__device__ __forceinline__ float gate_input(int mode, float x, float b) { return mode >= GATE_LOGITS ? x + b : x; }
+
 // The retention factor alpha of one channel for a scan in gate mode `mode`.
 __device__ __forceinline__ float gate_alpha(int mode, float x, float sc, float g_min) {
   if (mode == GATE_SOFTPLUS) return expf(softplus_log_decay(sc, x));

@@ -171,13 +171,15 @@ int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int6
   return ok();
 }
 
-// The decay input of a scan: alpha, g = log alpha, or the logits z with A_log and g_min.
+// The decay input of a scan: alpha, g = log alpha, or the logits z with A_log, g_min and an optional
+// per-(head, channel) bias.
 struct GateSpec {
   const float* data;
   int mode;
   const float* A_log;
   float g_min;
-  unsigned flags;  // KDA_QK_L2NORM | KDA_BETA_LOGITS
+  unsigned flags;  // KDA_QK_L2NORM | KDA_BETA_LOGITS | KDA_STATE_VK | KDA_GATE_SOFTPLUS
+  const float* dt_bias;
 };
 
 static int check_gate(const char* fn, const GateSpec& gs) {
@@ -188,6 +190,8 @@ static int check_gate(const char* fn, const GateSpec& gs) {
     return fail(KDA_ERR_INVALID_ARG, "%s: g_min must be finite and < 0 (got %g)", fn, (double)gs.g_min);
   if (gs.flags & ~(KDA_QK_L2NORM | KDA_BETA_LOGITS | KDA_STATE_VK | KDA_GATE_SOFTPLUS))
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown flags 0x%x", fn, gs.flags);
+  if (gs.dt_bias && !aligned16(gs.dt_bias))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: dt_bias must be 16-byte aligned", fn);
   return KDA_OK;
 }
 
@@ -196,6 +200,7 @@ static int check_scan_common(const char* fn, kda_dtype dtype, const GateSpec& gs
   int rc = check_gate(fn, gs);
   if (rc != KDA_OK) return rc;
   if (H <= 0) return fail(KDA_ERR_INVALID_ARG, "%s: H must be positive", fn);
+  if (H > 65535) return fail(KDA_ERR_UNSUPPORTED, "%s: H must be at most 65535 (got %lld)", fn, (long long)H);
   if (!dim_supported(K) || !dim_supported(V))
     return fail(KDA_ERR_UNSUPPORTED, "%s: K and V must be multiples of 16 in [16,256] (K=%lld, V=%lld)", fn,
                 (long long)K, (long long)V);
@@ -284,6 +289,7 @@ static int prefill_impl(const char* fn, const void* q, const void* k, const void
   p.N = (int)N;
   p.gate_mode = gs.mode;
   p.A_log = gs.A_log;
+  p.dt_bias = gs.dt_bias;
   p.g_min = gs.g_min;
   p.qk_l2norm = (gs.flags & KDA_QK_L2NORM) != 0;
   p.beta_sigmoid = (gs.flags & KDA_BETA_LOGITS) != 0;
@@ -292,10 +298,7 @@ static int prefill_impl(const char* fn, const void* q, const void* k, const void
   cudaError_t e;
   if (workspace_bytes > 0 && !workspace) return fail(KDA_ERR_INVALID_ARG, "%s: workspace_bytes > 0 with a null workspace", fn);
   const bool chunked = dtype == KDA_BF16 && kda::chunk_supported((int)K, (int)V, dtype);
-  // The unbounded gate runs chunked only on the two-kernel path (its pairwise diagonal blocks live in
-  // the workspace); without a workspace it takes the exact token-by-token kernel.
-  const bool split_ok = workspace && workspace_bytes >= kda::split_workspace_bytes(B, T, H, N, cu_seqlens != nullptr);
-  if (chunked && (gs.mode != kda::GATE_SOFTPLUS || split_ok)) {
+  if (chunked) {
     e = kda::launch_chunk(p, workspace, workspace_bytes, s);
   } else {
     e = kda::launch_recurrent(p, dtype, s);
@@ -313,19 +316,21 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
                 void* workspace, size_t workspace_bytes, kda_stream_t stream) {
   if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
     return fail(KDA_ERR_INVALID_ARG, "kda_prefill: unknown gate kind %d", (int)gate_kind);
-  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f, 0u};
+  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f, 0u, nullptr};
   return prefill_impl("kda_prefill", q, k, v, dtype, gs, beta, initial_state, final_state, cu_seqlens, n_seq, B, T, H,
                       K, V, layout, o, workspace, workspace_bytes, stream);
 }
 
 int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                       const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
+                       const float* logits, const float* A_log, const float* dt_bias, float g_min,
+                       const float* beta, unsigned flags,
                        const float* initial_state, float* final_state,
                        const int32_t* cu_seqlens, int64_t n_seq,
                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                        const kda_layout* layout, void* o,
                        void* workspace, size_t workspace_bytes, kda_stream_t stream) {
-  const GateSpec gs{logits, (flags & KDA_GATE_SOFTPLUS) ? kda::GATE_SOFTPLUS : kda::GATE_LOGITS, A_log, g_min, flags};
+  const GateSpec gs{logits, (flags & KDA_GATE_SOFTPLUS) ? kda::GATE_SOFTPLUS : kda::GATE_LOGITS, A_log, g_min, flags,
+                    dt_bias};
   return prefill_impl("kda_prefill_logits", q, k, v, dtype, gs, beta, initial_state, final_state, cu_seqlens, n_seq, B,
                       T, H, K, V, layout, o, workspace, workspace_bytes, stream);
 }
@@ -387,6 +392,7 @@ static int decode_impl(const char* fn, const void* q, const void* k, const void*
   p.N = (int)B;
   p.gate_mode = gs.mode;
   p.A_log = gs.A_log;
+  p.dt_bias = gs.dt_bias;
   p.g_min = gs.g_min;
   p.qk_l2norm = (gs.flags & KDA_QK_L2NORM) != 0;
   p.beta_sigmoid = (gs.flags & KDA_BETA_LOGITS) != 0;
@@ -403,15 +409,17 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
                     const kda_layout* layout, void* o, kda_stream_t stream) {
   if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
     return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: unknown gate kind %d", (int)gate_kind);
-  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f, 0u};
+  const GateSpec gs{gate, (int)gate_kind, nullptr, 0.f, 0u, nullptr};
   return decode_impl("kda_decode_step", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 
 int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                           const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
+                           const float* logits, const float* A_log, const float* dt_bias, float g_min,
+                           const float* beta, unsigned flags,
                            float* state, int64_t B, int64_t H, int64_t K, int64_t V,
                            const kda_layout* layout, void* o, kda_stream_t stream) {
-  const GateSpec gs{logits, (flags & KDA_GATE_SOFTPLUS) ? kda::GATE_SOFTPLUS : kda::GATE_LOGITS, A_log, g_min, flags};
+  const GateSpec gs{logits, (flags & KDA_GATE_SOFTPLUS) ? kda::GATE_SOFTPLUS : kda::GATE_LOGITS, A_log, g_min, flags,
+                    dt_bias};
   return decode_impl("kda_decode_step_logits", q, k, v, dtype, gs, beta, state, B, H, K, V, layout, o, stream);
 }
 

@@ -31,7 +31,8 @@ struct ScanParams {
   int64_t T;
   int B, H, K, V, N;
   int gate_mode;        // KDA_GATE_ALPHA, KDA_GATE_LOG, or GATE_LOGITS (gate holds decay logits z)
-  const float* A_log;   // [H], GATE_LOGITS only
+  const float* A_log;   // [H], logit gate modes only
+  const float* dt_bias; // [H,K] or nullptr, logit gate modes only: added to z before the gate
   float g_min;          // GATE_LOGITS only
   int qk_l2norm;        // q, k are L2-normalised over K inside the kernels
   int beta_sigmoid;     // beta holds logits; the kernels use sigmoid(beta)
@@ -103,6 +104,9 @@ size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t n_seq);
 cudaError_t launch_chunk(const ScanParams& p, void* ws, size_t ws_bytes, cudaStream_t s);
 size_t split_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, bool varlen);
 cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s);
+// Whether the driver accepts tensor maps of this call's q, k and gate layouts (the two-kernel path reads
+// them by TMA); when it does not, the single fused kernel runs instead.
+bool split_maps_ok(const ScanParams& p);
 cudaError_t launch_wait_selftest(cudaStream_t s);  // one wait that expires (kda_selftest_wait_expiry)
 cudaError_t split_read_timeout(int* flag, bool reset);
 // Reads (and optionally clears) the chunk kernel's device-side timeout flag. Synchronous.

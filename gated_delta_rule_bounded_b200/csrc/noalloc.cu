@@ -10,7 +10,9 @@
 //
 // Setup: the first call on a device looks up the scratch's device address with
 // cudaGetSymbolAddress (which also loads this module on that device under lazy loading) and
-// caches it; later calls on that device only read the cache.
+// caches it; later calls on that device only read the cache. The cached address belongs to the
+// device's primary context, so a device reset between calls is not supported. Under eager module
+// loading the array is reserved on every device the library loads on, whether or not this call runs.
 //
 // Sharing: every call on a device uses the same array. The first kernel of a call writes every
 // block the second kernel reads, so nothing in it has to start at zero, but two calls whose work

@@ -108,7 +108,9 @@ recurrent_kernel(ScanParams p) {
     const int64_t go = brow * p.gs[0] + t * p.gs[1] + h * p.gs[2];
     const int64_t vo = brow * p.vs[0] + t * p.vs[1] + h * p.vs[2];
     for (int i = tid; i < K; i += NT) {
-      s_a[i] = gate_alpha(p.gate_mode, __ldg(p.gate + go + i), sc, p.g_min);
+      s_a[i] = gate_alpha(p.gate_mode,
+                         gate_input(p.gate_mode, __ldg(p.gate + go + i), p.dt_bias ? __ldg(p.dt_bias + (size_t)h * K + i) : 0.f),
+                         sc, p.g_min);
       s_k[i] = to_f32(kb[ko + i]);
       s_q[i] = to_f32(qb[qo + i]);
     }

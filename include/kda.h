@@ -123,7 +123,7 @@ int kda_softplus_decay(const void* logits, const kda_strides* logits_strides, kd
  * workspace (about 1 KB per token and head), then runs the recurrence. Given
  * at least this many bytes kda_prefill uses it; given less (or no workspace),
  * it runs the single fused kernel instead, with identical results up to
- * rounding (with KDA_GATE_SOFTPLUS, the token-by-token kernel instead). The caller allocates the workspace; a larger buffer is fine. n_seq
+ * rounding. The caller allocates the workspace; a larger buffer is fine. n_seq
  * is the number of packed sequences (0 without cu_seqlens).
  * ------------------------------------------------------------------------- */
 int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
@@ -135,11 +135,16 @@ int kda_prefill_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int6
  * q, k      [B,T,H,K]  dtype `dtype` (KDA_BF16 or KDA_F32; q, k, v share it)
  * v         [B,T,H,V]  dtype `dtype`
  * gate      [B,T,H,K]  fp32 alpha (gate_kind KDA_GATE_ALPHA) or g = log alpha
- *                      (KDA_GATE_LOG). For bf16 inputs the chunked kernel
- *                      requires the bounded range alpha >= exp(-5), g >= -5
- *                      (the bound the "KDA cheat sheet" uses to keep every
- *                      reciprocal rescale within range); fp32 inputs take any
- *                      alpha in [0,1].
+ *                      (KDA_GATE_LOG), any alpha in [0,1] (g in [-inf, 0]).
+ *                      The chunked bf16 kernels factor decay ratios across
+ *                      16-token blocks, which stays in range while a block's
+ *                      decay on every channel is at least 2^-120 (always so
+ *                      for g >= -5, the bounded gate's "KDA cheat sheet"
+ *                      range); a block that decays further has its diagonal
+ *                      16x16 tiles formed pair by pair from running products
+ *                      of alpha instead (slower, exact). alpha below 2^-126,
+ *                      alpha = 0 included, is taken as 2^-126: what it leaves
+ *                      of the past state is below fp32 resolution.
  * beta      [B,T,H]    fp32 write strength in [0,1]
  * initial_state [N,H,K,V] fp32 or NULL (zeros)
  * final_state   [N,H,K,V] fp32 or NULL (not written). It may be the same
@@ -176,12 +181,11 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  *                    transpose of the default [N,H,K,V]; "Kept memory": the
  *                    production cache keeps S this way).
  *   KDA_GATE_SOFTPLUS the logits feed Kimi Linear's unbounded gate,
- *                    g = -exp(A_log[h]) * softplus(z) (g_min is ignored),
- *                    instead of the bounded one. Its per-token decay has no
- *                    lower bound, so the diagonal 16x16 blocks of the chunk
- *                    form are computed pairwise by an extra kernel; this
- *                    chunked path needs the workspace (bf16, K = 128), and
- *                    without one the scan runs token by token (exact, slower). */
+ *                    g = -exp(A_log[h]) * softplus(z + dt_bias) (g_min is
+ *                    ignored), instead of the bounded one. Its per-token decay
+ *                    has no lower bound; the chunked kernels form the diagonal
+ *                    16x16 blocks of any block it takes out of range pair by
+ *                    pair (see kda_prefill), with or without a workspace. */
 #define KDA_QK_L2NORM 1u
 #define KDA_BETA_LOGITS 2u
 #define KDA_STATE_VK 4u
@@ -199,18 +203,26 @@ int kda_prefill(const void* q, const void* k, const void* v, kda_dtype dtype,
  *          uses for alpha / g).
  * A_log    [H] fp32 device pointer; g_min finite and < 0
  *          (else KDA_ERR_INVALID_ARG).
+ * dt_bias  NULL, or [H,K] fp32 device pointer (contiguous, 16-byte aligned):
+ *          a per-(head, channel) bias added to the logits before the gate,
+ *          g = g_min * sigmoid(exp(A_log[h]) * (z + dt_bias[h,c])) ("KDA cheat
+ *          sheet", How the inputs are produced: z = W_up W_down x + b; the
+ *          chunked kernel call on the "Kept memory" page takes it as dt_bias).
+ *          The sum z + dt_bias is rounded to fp32 once, as a caller adding it
+ *          beforehand would.
  * flags    0, or any of KDA_QK_L2NORM, KDA_BETA_LOGITS, KDA_STATE_VK,
  *          KDA_GATE_SOFTPLUS (unknown bits: KDA_ERR_INVALID_ARG). The chunked bf16 kernels round normalised
  *          q and k to bf16, their operand precision; the fp32 kernel keeps
  *          them in fp32.
  * Every other argument, layout, result, workspace rule and error is
  * kda_prefill's. With flags 0 the result is bit-identical to
- * kda_bounded_decay with out_kind KDA_GATE_LOG (bf16 inputs) or
- * KDA_GATE_ALPHA (fp32 inputs) followed by kda_prefill on its output: both
+ * kda_bounded_decay (on z + dt_bias) with out_kind KDA_GATE_LOG (bf16 inputs)
+ * or KDA_GATE_ALPHA (fp32 inputs) followed by kda_prefill on its output: both
  * evaluate the gate with the same device code.
  * ------------------------------------------------------------------------- */
 int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                       const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
+                       const float* logits, const float* A_log, const float* dt_bias, float g_min,
+                       const float* beta, unsigned flags,
                        const float* initial_state, float* final_state,
                        const int32_t* cu_seqlens, int64_t n_seq,
                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
@@ -236,7 +248,12 @@ int kda_prefill_logits(const void* q, const void* k, const void* v, kda_dtype dt
  *
  * Setup: the first call on a device (the device current at the call) looks
  * up the scratch's device address once and keeps it; make that first call
- * before any stream capture on that device.
+ * before any stream capture on that device. The address stays valid for the
+ * life of the device's primary context: do not reset the device
+ * (cudaDeviceReset) between calls, since the scratch may then sit elsewhere.
+ * With lazy module loading (the CUDA default) the array takes device memory
+ * only on devices where this call has run; with CUDA_MODULE_LOADING=EAGER it
+ * is reserved on every device the library is loaded on.
  *
  * Sharing: every call on a device uses the same scratch. Nothing in it has to
  * start at zero (each call writes all it reads), but calls whose GPU work may
@@ -271,13 +288,15 @@ int kda_decode_step(const void* q, const void* k, const void* v, kda_dtype dtype
 /* ---------------------------------------------------------------------------
  * kda_decode_step_logits: kda_decode_step with the bounded gate (eq. 5)
  * applied inside the step: logits [B,H,K] fp32 (strides in layout->gate),
- * A_log [H] fp32, g_min finite and < 0. alpha = exp(g_min * sigmoid(
- * exp(A_log[h]) * z)). flags as for kda_prefill_logits (normalised q, k kept
+ * A_log [H] fp32, dt_bias NULL or [H,K] fp32 (as for kda_prefill_logits),
+ * g_min finite and < 0. alpha = exp(g_min * sigmoid(exp(A_log[h]) *
+ * (z + dt_bias[h,c]))). flags as for kda_prefill_logits (normalised q, k kept
  * in fp32). Everything else is kda_decode_step's; with flags 0 the result is
  * bit-identical to kda_bounded_decay (alpha out) followed by kda_decode_step.
  * ------------------------------------------------------------------------- */
 int kda_decode_step_logits(const void* q, const void* k, const void* v, kda_dtype dtype,
-                           const float* logits, const float* A_log, float g_min, const float* beta, unsigned flags,
+                           const float* logits, const float* A_log, const float* dt_bias, float g_min,
+                           const float* beta, unsigned flags,
                            float* state, int64_t B, int64_t H, int64_t K, int64_t V,
                            const kda_layout* layout, void* o, kda_stream_t stream);
 

@@ -14,13 +14,17 @@ Functions and the passages they follow:
 
 * :func:`bounded_decay` -- "Kimi K3: Bounded Decay and Delta Memory",
   Formula and conventions, eq. 5: ``g = g_min * sigmoid(exp(A) * z)``,
-  ``alpha = exp(g)``.
+  ``alpha = exp(g)``. An optional per-(head, channel) bias is added to the
+  logits first, in fp64 ("KDA cheat sheet", How the inputs are produced:
+  ``z = W_up W_down x + b``; the chunked kernel call on the "Kept memory" page
+  names it ``dt_bias``).
 * :func:`scan_backward`, :func:`bounded_decay_backward` -- gradients of the
   scan and of the gate: eq. 1 and eq. 5 restated with plain fp64 PyTorch ops
   (:func:`scan_torch`) and differentiated by autograd. Pinned by the C
   oracle's forward values and by finite differences (gradcheck).
 * :func:`softplus_decay` -- Kimi Linear's unbounded gate, the contrast drawn in
-  Figure 3(a) of the same page: ``g = -exp(A) * softplus(z)``.
+  Figure 3(a) of the same page: ``g = -exp(A) * softplus(z)`` (with the same
+  optional bias on z).
 * :func:`l2norm`, :func:`sigmoid` -- the input preparation the surrounding
   model applies ("KDA cheat sheet", How the inputs are produced: q, k =
   L2Norm(...), beta = Sigmoid(W_beta x)); they check the scan entry points that
@@ -101,21 +105,33 @@ def sigmoid(x) -> np.ndarray:
     return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
 
 
-def softplus_decay(z, A_log, return_log: bool = False):
-    """Kimi Linear's unbounded gate in fp64 ("Kimi K3: Bounded Decay and Delta Memory", Figure 3(a)
-    contrast; "KDA cheat sheet", g_min table): ``g = -exp(A_log[h]) * softplus(z)`` with
-    ``softplus(z) = max(z, 0) + log(1 + exp(-|z|))``; ``alpha = exp(g)``. z ``[B,T,H,K]``."""
+def _biased(z, dt_bias):
+    """The gate's input: the logits z ``[B,T,H,K]`` plus the bias ``[H,K]`` (when given), in fp64."""
     z = _f64(z)
+    if dt_bias is None:
+        return z
+    b = _f64(dt_bias)
+    if b.shape != (z.shape[2], z.shape[3]):
+        raise ValueError("dt_bias must be [H,K]")
+    return z + b[None, None]
+
+
+def softplus_decay(z, A_log, return_log: bool = False, dt_bias=None):
+    """Kimi Linear's unbounded gate in fp64 ("Kimi K3: Bounded Decay and Delta Memory", Figure 3(a)
+    contrast; "KDA cheat sheet", g_min table): ``g = -exp(A_log[h]) * softplus(z + dt_bias)`` with
+    ``softplus(x) = max(x, 0) + log(1 + exp(-|x|))``; ``alpha = exp(g)``. z ``[B,T,H,K]``."""
+    z = _biased(z, dt_bias)
     sc = np.exp(_f64(A_log))[None, None, :, None]
     g = -sc * (np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z))))
     alpha = np.exp(g)
     return (alpha, g) if return_log else alpha
 
 
-def bounded_decay(z, A_log, g_min: float = -5.0, return_log: bool = False):
-    """alpha (and optionally g) for logits ``z [B,T,H,K]`` and per-head ``A_log [H]``."""
+def bounded_decay(z, A_log, g_min: float = -5.0, return_log: bool = False, dt_bias=None):
+    """alpha (and optionally g) for logits ``z [B,T,H,K]``, per-head ``A_log [H]`` and the optional bias
+    ``dt_bias [H,K]`` added to z: ``g = g_min * sigmoid(exp(A_log[h]) * (z + dt_bias[h]))``."""
     lib = _load()
-    z = _f64(z)
+    z = _biased(z, dt_bias)
     A = _f64(A_log)
     if z.ndim != 4 or A.shape != (z.shape[2],):
         raise ValueError("z must be [B,T,H,K] and A_log [H]")

@@ -240,25 +240,44 @@ def test_noalloc_rejects_oversize_before_any_device_call(lib):
 def test_logits_entry_points_reject_bad_gate_arguments(lib):
     layout = Layout(*[Strides(0, 128, 128)] * 4, Strides(0, 1, 1), Strides(0, 128, 128))
     for g_min in (0.0, 1.0, float("nan"), float("inf")):
-        rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, g_min, FAKE, 0, None, None, None, 0,
+        rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, None, g_min, FAKE, 0, None, None, None, 0,
                                     1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
         assert rc == INVALID and "g_min" in lib.kda_last_error().decode()
-        rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, g_min, FAKE, 0, FAKE, 1, 1, 128, 128,
+        rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, None, g_min, FAKE, 0, FAKE, 1, 1, 128, 128,
                                         ctypes.byref(layout), FAKE, None)
         assert rc == INVALID and "g_min" in lib.kda_last_error().decode()
-    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, None, -5.0, FAKE, 0, None, None, None, 0,
+    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, None, None, -5.0, FAKE, 0, None, None, None, 0,
                                 1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
     assert rc == INVALID and "null" in lib.kda_last_error().decode()
-    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, None, -5.0, FAKE, 0, FAKE, 1, 1, 128, 128,
+    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, None, None, -5.0, FAKE, 0, FAKE, 1, 1, 128, 128,
                                     ctypes.byref(layout), FAKE, None)
     assert rc == INVALID and "null" in lib.kda_last_error().decode()
 
 
 def test_logits_entry_points_reject_unknown_flags(lib):
     layout = Layout(*[Strides(0, 128, 128)] * 4, Strides(0, 1, 1), Strides(0, 128, 128))
-    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 16, None, None, None, 0,
+    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, None, -5.0, FAKE, 16, None, None, None, 0,
                                 1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
     assert rc == INVALID and "flags" in lib.kda_last_error().decode()
-    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, -5.0, FAKE, 32, FAKE, 1, 1, 128, 128,
+    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, None, -5.0, FAKE, 32, FAKE, 1, 1, 128, 128,
                                     ctypes.byref(layout), FAKE, None)
     assert rc == INVALID and "flags" in lib.kda_last_error().decode()
+
+
+def test_logits_entry_points_reject_a_misaligned_bias(lib):
+    layout = Layout(*[Strides(0, 128, 128)] * 4, Strides(0, 1, 1), Strides(0, 128, 128))
+    rc = lib.kda_prefill_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE + 4, -5.0, FAKE, 0, None, None, None, 0,
+                                1, 4, 1, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
+    assert rc == UNSUPPORTED and "dt_bias" in lib.kda_last_error().decode()
+    rc = lib.kda_decode_step_logits(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE + 8, -5.0, FAKE, 0, FAKE, 1, 1, 128, 128,
+                                    ctypes.byref(layout), FAKE, None)
+    assert rc == UNSUPPORTED and "dt_bias" in lib.kda_last_error().decode()
+
+
+def test_prefill_rejects_more_heads_than_a_grid_dimension_holds(lib):
+    # the operand kernel runs one grid row per head; more than 65535 heads are refused up front
+    H = 65536
+    layout = Layout(*[Strides(0, H * 128, 128)] * 4, Strides(0, H, 1), Strides(0, H * 128, 128))
+    rc = lib.kda_prefill(FAKE, FAKE, FAKE, 1, FAKE, 0, FAKE, None, None, None, 0,
+                         1, 4, H, 128, 128, ctypes.byref(layout), FAKE, None, 0, None)
+    assert rc == UNSUPPORTED and "65535" in lib.kda_last_error().decode()

@@ -3,20 +3,12 @@
 Both sides start from the same raw inputs (q, k, v, decay logits z, A_log,
 beta, initial state) drawn by ``workloads.py``. The GPU side runs its own gate
 kernel and scan kernels through the C ABI; the oracle side runs its own fp64
-gate and token-by-token scan. Tolerances (written in each test):
-
-* fp32 q/k/v: max |gpu - oracle| <= 1e-4 on o and on final_state;
-* bf16 q/k/v: the relative RMS error rms(gpu - oracle) <= 2e-2 * rms(oracle),
-  separately for o and final_state, plus an elementwise guard
-  |gpu - oracle| <= (|oracle| + rms(oracle)) / 8 that any wrong term, index or
-  token fails. The bound is read as an RMS ratio because a max-abs reading is
-  out of reach for a bf16 result: rounding the exact output to bf16 alone
-  gives max|err| / rms = 1.8e-2 at T = 150 and more at larger sizes (the
-  largest outputs are 10-20x the RMS), while bf16 tensor-core arithmetic
-  keeps the RMS ratio near 5e-3;
-* gate: |g - g_ref| <= |g_ref| 2^-22 (1 + |e^A z|) for fp32 output (the fp32
-  rounding of the sigmoid's argument carried through), within one bf16
-  rounding (2^-8 relative) for bf16 output.
+gate and token-by-token scan. The scan tolerances are those of ``tests/parity.py``
+(fp32: max-abs 1e-4; bf16: relative RMS 2e-2 with an elementwise guard, and
+max-abs 2e-2 of the RMS on the fp32 final state). The gate's:
+|g - g_ref| <= |g_ref| 2^-22 (1 + |e^A z|) for fp32 output (the fp32 rounding of
+the sigmoid's argument carried through), within one bf16 rounding (2^-8
+relative) for bf16 output.
 """
 import numpy as np
 import pytest
@@ -24,13 +16,9 @@ import torch
 
 import oracle
 import workloads as W
+from tests.parity import DEV, check, to_dev
 
 pytestmark = pytest.mark.gpu
-
-DEV = "cuda"
-FP32_ATOL = 1e-4
-BF16_REL_RMS = 2e-2
-GUARD = 0.125
 
 
 @pytest.fixture(scope="module")
@@ -40,32 +28,6 @@ def kda():
     import gated_delta_rule_bounded_b200 as m
     m.load_library()
     return m
-
-
-def check(got, ref, dtype, what):
-    """fp32: max-abs <= 1e-4. bf16: rms(err) <= 2e-2 rms(ref) and |err| <= (|ref| + rms(ref)) / 8.
-    Returns the RMS error ratio (bf16) or the max abs error (fp32)."""
-    got = got.detach().double().cpu().numpy() if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    assert got.shape == ref.shape, f"{what}: shape {got.shape} != {ref.shape}"
-    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
-    if ref.size == 0:
-        return 0.0
-    err = np.abs(got - ref)
-    if dtype == "f32":
-        m = float(err.max())
-        assert m <= FP32_ATOL, f"{what}: max abs err {m:.3e} > {FP32_ATOL}"
-        return m
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    ratio = float(np.sqrt(np.mean(err ** 2))) / rms
-    assert ratio <= BF16_REL_RMS, f"{what}: rms error / rms {ratio:.3e} > {BF16_REL_RMS}"
-    worst = float((err / (np.abs(ref) + rms)).max())
-    assert worst <= GUARD, f"{what}: elementwise error {worst:.3e} of (|ref| + rms) > {GUARD}"
-    return ratio
-
-
-def to_dev(d):
-    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
 
 
 def gpu_pipeline(kda, d, **kw):
@@ -462,6 +424,66 @@ def test_decode_logits_equals_gate_then_step(kda, K, V, dtype):
 
 
 # ---------------------------------------------------------------------------------------------
+# The logits' bias (dt_bias [H,K], "KDA cheat sheet", How the inputs are produced: z = W_up W_down x + b)
+# ---------------------------------------------------------------------------------------------
+# The kernels add the bias to z in fp32 before the gate, so a call with the bias must equal, bit for
+# bit, the same call without it on z + dt_bias summed by the caller in fp32; the oracle adds the bias
+# in fp64 before its own gate.
+
+def bias_for(H, K, seed):
+    return torch.randn(H, K, generator=torch.Generator().manual_seed(seed)) * 1.5
+
+
+@pytest.mark.parametrize("dtype,use_workspace,gate", [("bf16", True, "bounded"), ("bf16", False, "bounded"),
+                                                      ("bf16", True, "softplus"), ("f32", True, "bounded")],
+                         ids=["bf16-split", "bf16-fused", "bf16-softplus", "f32"])
+def test_prefill_logits_with_dt_bias(kda, dtype, use_workspace, gate):
+    B, T, H = 2, 150, 3
+    d = W.random_scan_case(B, T, H, 128, 128, seed=51, dtype=dtype, z_std=2.0, init_std=0.1)
+    b = bias_for(H, 128, 52)
+    g = to_dev(d)
+    kw = dict(gate=gate, use_workspace=use_workspace)
+    o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"], g["initial_state"],
+                               dt_bias=b.to(DEV), **kw)
+    zb = (d["z"] + b[None, None]).to(DEV)
+    o2, s2 = kda.prefill_logits(g["q"], g["k"], g["v"], zb, g["A_log"], g["g_min"], g["beta"], g["initial_state"], **kw)
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    assert torch.equal(o, o2) and torch.equal(sf, s2)
+    if gate == "softplus":
+        alpha = oracle.softplus_decay(d["z"], d["A_log"], dt_bias=b)
+    else:
+        alpha = oracle.bounded_decay(d["z"], d["A_log"], d["g_min"], dt_bias=b)
+    ro, rs = oracle.scan(d["q"], d["k"], d["v"], alpha, d["beta"], d["initial_state"])
+    check(o, ro, dtype, "o")
+    check(sf, rs, dtype, "final_state")
+
+
+@pytest.mark.parametrize("K,V,dtype", [(128, 128, "bf16"), (64, 32, "f32")], ids=["bulk", "token-kernel"])
+def test_decode_logits_with_dt_bias(kda, K, V, dtype):
+    B, T, H = 3, 4, 5
+    d = W.random_scan_case(B, T, H, K, V, seed=53, dtype=dtype, z_std=2.0, init_std=0.1)
+    b = bias_for(H, K, 54)
+    g = to_dev(d)
+    st, st2 = g["initial_state"].clone(), g["initial_state"].clone()
+    outs, outs2 = [], []
+    for t in range(T):
+        outs.append(kda.decode_step_logits(g["q"][:, t], g["k"][:, t], g["v"][:, t], g["z"][:, t], g["A_log"],
+                                           g["g_min"], g["beta"][:, t], st, dt_bias=b.to(DEV)))
+        zb = (d["z"][:, t] + b[None]).to(DEV)
+        outs2.append(kda.decode_step_logits(g["q"][:, t], g["k"][:, t], g["v"][:, t], zb, g["A_log"], g["g_min"],
+                                            g["beta"][:, t], st2))
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    o = torch.stack(outs, 1)
+    assert torch.equal(o, torch.stack(outs2, 1)) and torch.equal(st, st2)
+    alpha = oracle.bounded_decay(d["z"], d["A_log"], d["g_min"], dt_bias=b)
+    ro, rs = oracle.scan(d["q"], d["k"], d["v"], alpha, d["beta"], d["initial_state"])
+    check(o, ro, dtype, "o")
+    check(st, rs, dtype, "state")
+
+
+# ---------------------------------------------------------------------------------------------
 # Input preparation inside the kernels (KDA_QK_L2NORM, KDA_BETA_LOGITS)
 # ---------------------------------------------------------------------------------------------
 # The oracle prepares the raw inputs itself (fp64 L2Norm of q and k over K, sigmoid of the beta
@@ -576,7 +598,7 @@ def test_softplus_gate_matches_oracle(kda):
 
 
 @pytest.mark.parametrize("dtype,use_workspace", [("bf16", True), ("bf16", False), ("f32", True)],
-                         ids=["bf16-chunked", "bf16-token-kernel", "f32"])
+                         ids=["bf16-split", "bf16-fused", "f32"])
 def test_prefill_logits_softplus_gate(kda, dtype, use_workspace):
     d = W.random_scan_case(2, 150, 3, 128, 128, seed=43, dtype=dtype, z_std=2.0, init_std=0.1)
     g = to_dev(d)
@@ -725,9 +747,9 @@ def test_gate_backward_matches_autograd_oracle(kda):
     np.testing.assert_allclose(dA.double().cpu().numpy(), rA, rtol=1e-4, atol=1e-4)
 
 
-def test_usage_example_from_the_design_notes(kda):
-    # The Python usage example of the design notes, at a small size: every call must accept what the
-    # example passes (views included) and return finite values of the documented shapes.
+def test_usage_example_calls(kda):
+    # A short tour of the Python API at a small size: every call must accept what is passed (views
+    # included) and return finite values of the documented shapes.
     B, T, H, K, V = 1, 130, 4, 128, 128
     gen = torch.Generator().manual_seed(11)
     q, k = (torch.randn(B, T, H, K, generator=gen).to(DEV, torch.bfloat16) for _ in range(2))

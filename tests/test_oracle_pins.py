@@ -341,6 +341,27 @@ def test_gate_contrast_with_unbounded_softplus_gate():
     assert np.all(lg >= -5.0) and np.all(lg <= 0.0)
 
 
+def test_gate_bias_shifts_the_logits_before_the_scale():
+    """The bias enters as z + b inside the sigmoid's argument, before the e^A scale ("KDA cheat sheet",
+    How the inputs are produced: z = W_up W_down x + b). With z = -b[h, c] on every entry the argument is
+    exactly 0 and g = g_min / 2; a bias added after the scale (e^A z + b), to g, or read transposed
+    ([c, h] for [h, c]) leaves a non-zero argument on some entry."""
+    H, K = 2, 3
+    b = np.array([[0.5, -1.25, 2.0], [3.0, -0.75, 1.5]])
+    z = np.broadcast_to(-b, (1, 4, H, K)).copy()
+    A = np.array([0.7, -0.3])
+    for g_min in (-5.0, -8.0):
+        alpha, lg = oracle.bounded_decay(z, A, g_min, return_log=True, dt_bias=b)
+        assert np.all(lg == g_min / 2) and np.allclose(alpha, math.exp(g_min / 2), rtol=1e-15)
+    # z = 0 and b = ln 3 / e^A: the argument is ln 3, sigmoid(ln 3) = 3/4, g = 0.75 g_min
+    b2 = np.log(3.0) * np.exp(-A)[:, None] * np.ones((H, K))
+    lg2 = oracle.bounded_decay(np.zeros((1, 2, H, K)), A, -5.0, return_log=True, dt_bias=b2)[1]
+    np.testing.assert_allclose(lg2, -3.75, rtol=1e-14)
+    # the unbounded gate takes the same bias: z = -b gives softplus(0) = ln 2, g = -e^A ln 2
+    lgs = oracle.softplus_decay(z, A, return_log=True, dt_bias=b)[1]
+    np.testing.assert_allclose(lgs, -np.exp(A)[None, None, :, None] * np.log(2.0) * np.ones_like(z), rtol=1e-15)
+
+
 # ---------------------------------------------------------------------------------------------
 # Input preparation ("KDA cheat sheet", How the inputs are produced): L2Norm of q, k; beta = Sigmoid
 # ---------------------------------------------------------------------------------------------

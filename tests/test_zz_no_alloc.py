@@ -7,7 +7,7 @@ Each case calls the allocation-free entry point through the C ABI twice in a row
 inputs (and, in the varlen case, a different slot layout), and checks both results against
 kda_prefill given a caller-allocated workspace (the existing entry point), with the bf16
 tolerance of the GPU parity suite: rms(err) <= 2e-2 rms(ref) plus the elementwise guard
-|err| <= (|ref| + rms(ref)) / 8; fp32: max |err| <= 1e-4. One head of each call is also checked
+|err| <= 0.05 (|ref| + rms(ref)); fp32: max |err| <= 1e-4. One head of each call is also checked
 against the fp64 oracle with the same tolerance.
 """
 import numpy as np
@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 BF16_REL_RMS = 2e-2
-GUARD = 0.125
+GUARD = 0.05
 FP32_ATOL = 1e-4
 
 
