@@ -81,6 +81,8 @@ static_assert(P_KG % 1024 == 0 && P_VIEW % 1024 == 0 && VIEW_HALF % 1024 == 0 &&
               P_W % 1024 == 0 && P_AQKT % 1024 == 0 && P_TB % 1024 == 0, "swizzle atoms need 1 KB alignment");
 static_assert(2 * (P_SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 constexpr uint32_t P_TM_COLS = 256;         // TMEM: A products at columns 0 and 64, W at 128
+// The view scales of view_expand take the VEC_D area of the vectors (fp32 [6][128]) in kernel P.
+static_assert(VEC_TOT >= VEC_D + 6 * 128, "view scales fit before the block sums");
 
 // Kernel S shared memory: the operand blocks of two chunks and their v tiles.
 constexpr int S_OPS = 0;                    // 2 x operand block (66048 B, padded to 66560)
@@ -193,13 +195,14 @@ struct PMaps {
   CUtensorMap q, k, g;
 };
 
-// Decay pass, step 2 of kernel P: the row operand KQ, the column views, K*Gamma (smem), Q*Gamma (straight
-// to its place in the workspace block, qg_dst: [t][c] rows of 16 KB k-atoms) and gamma_C. View 3 is
-// K*gamma_C/Gamma unless block 3 is out of range (its reference is then the block's start); in that case
-// K*gamma_C/Gamma goes straight to the workspace too (kt_dst: [t][c] rows of 8 KB n-atoms).
+// Decay pass, step 2 of kernel P: the row operand KQ, K*Gamma (smem), Q*Gamma (straight to its place in the
+// workspace block, qg_dst: [t][c] rows of 16 KB k-atoms), gamma_C, and block da's own rows of view da,
+// k_i 2^{e[da] - G_i}, from which view_expand derives the other views. When block 3 is out of range view 3 is
+// not K*gamma_C/Gamma (its reference is then the block's start), which goes straight to the workspace too
+// (kt_dst: [t][c] rows of 8 KB n-atoms).
 __device__ __forceinline__ void p_operands(unsigned char* sm, const Prefetch& pf, int da, int c0, int pairwise,
                                            const float2 (&al)[16], unsigned char* qg_dst, unsigned char* kt_dst) {
-  const float* vec = reinterpret_cast<const float*>(sm + P_VEC);
+  float* vec = reinterpret_cast<float*>(sm + P_VEC);
   float2 e[4];
 #pragma unroll
   for (int b = 0; b < 4; ++b) e[b] = *reinterpret_cast<const float2*>(vec + VEC_TOT + b * 128 + c0);
@@ -219,15 +222,15 @@ __device__ __forceinline__ void p_operands(unsigned char* sm, const Prefetch& pf
   const float2 eda = da == 0 ? e[0] : (da == 1 ? e[1] : (da == 2 ? e[2] : e[3]));
   const float2 Rd = da == 0 ? R[0] : (da == 1 ? R[1] : (da == 2 ? R[2] : R[3]));
   if (da == 0) *reinterpret_cast<float2*>(sm + P_GAM + 4 * c0) = make_float2(ex2(e[3].x), ex2(e[3].y));
+  // Scales 2^{R_a - e[da]} (<= 1) of this block's rows in the views a > da, for view_expand:
+  // fp32 [pair][128] in the VEC_D area, pair (a, b) at a (a - 1) / 2 + b.
+#pragma unroll
+  for (int a = 1; a < 4; ++a)
+    if (a > da)
+      *reinterpret_cast<float2*>(vec + VEC_D + (a * (a - 1) / 2 + da) * 128 + c0) =
+          make_float2(ex2(R[a].x - eda.x), ex2(R[a].y - eda.y));
   const float2 GS = make_float2(ex2(gs.x), ex2(gs.y));               // Gamma at the start of the block
   const float2 DI = make_float2(ex2(gs.x - Rd.x), ex2(gs.y - Rd.y)); // 2^{G_start - R_da} (>= 1)
-  // Column-view scales of this block's tokens: 2^{R_a - e[da]} for views a > da (<= 1); 1 for a = da, or 0
-  // when this block is out of range (its diagonal tile comes from diag_pairwise).
-  float2 SV[4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-    SV[a] = a > da ? make_float2(ex2(R[a].x - eda.x), ex2(R[a].y - eda.y))
-                   : (((pairwise >> da) & 1) ? make_float2(0.f, 0.f) : make_float2(1.f, 1.f));
   const int rk = kq_base(da);
   float2 E = make_float2(1.f, 1.f);
 #pragma unroll
@@ -245,77 +248,107 @@ __device__ __forceinline__ void p_operands(unsigned char* sm, const Prefetch& pf
   }
   const bool kt_apart = (pairwise >> 3) & 1;
   const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));  // 2^{e[3] - e[da]}
+  const int vrow = view_base(da) + 16 * da;
   float2 F = make_float2(1.f, 1.f);  // 2^{e[da] - G_i}, tokens after i within the block
 #pragma unroll
   for (int i = 15; i >= 0; --i) {
-    const int t = 16 * da + i;
     const float2 kf = unpack_bf16(pf.k[i]);
     const float kx = kf.x * F.x, ky = kf.y * F.y;
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-      if (a >= da)
-        *reinterpret_cast<uint32_t*>(sm + P_VIEW + sw_e(view_base(a) + t, c0, VIEW_HALF)) =
-            pack_bf16(kx * SV[a].x, ky * SV[a].y);
-    if (kt_apart) *reinterpret_cast<uint32_t*>(kt_dst + sw_e(t, c0, 8192)) = pack_bf16(kx * PM.x, ky * PM.y);
+    // block da's rows of view da (for an out-of-range block they are its discarded diagonal tile, and the
+    // source of its rows in the later views)
+    *reinterpret_cast<uint32_t*>(sm + P_VIEW + sw_e(vrow + i, c0, VIEW_HALF)) = pack_bf16(kx, ky);
+    if (kt_apart)
+      *reinterpret_cast<uint32_t*>(kt_dst + sw_e(16 * da + i, c0, 8192)) = pack_bf16(kx * PM.x, ky * PM.y);
     F.x *= al[i].x;
     F.y *= al[i].y;
   }
 }
 
-// diag_pairwise (chunk_common.cuh) with its results in the fp32 buffer `out` [A_kk | A_qk][block][t][j]
-// (A_kk with beta_t applied and zero for j >= t, A_qk zero for j > t); the block's two warps combine their
-// halves of the channels in place there.
-__device__ __forceinline__ void p_diag_pairwise(float* out, const Prefetch& pf, const float2 (&al)[16],
-                                                const float* beta_s, int da, int pairwise) {
-  const int lane = threadIdx.x & 31, hw = (threadIdx.x >> 5) & 1;
-  const bool mine = (pairwise >> da) & 1;
-  // entry l of column j: A_qk[t = l][j] (l < 16) or A_kk[t = l - 16][j]
-  auto slot = [&](int j, int l) { return out + (l < 16 ? 1024 : 0) + (da * 16 + (l & 15)) * 16 + j; };
-  float res[16];
-  if (mine) {
+// After p_operands and a barrier: the rows of block b in view a > b, as block b's rows of view b times the
+// scale 2^{R_a - e[b]} of each channel (six block pairs of 16 rows x 128 channels, one 8-channel 16-byte
+// piece per thread and pair; fp32 products rounded once to bf16).
+__device__ __forceinline__ void view_expand(unsigned char* sm, int tid) {
+  const float* vec = reinterpret_cast<const float*>(sm + P_VEC);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float2 kj = unpack_bf16(pf.k[j]);
-      float v[32];
-#pragma unroll
-      for (int t = 0; t < 16; ++t) v[t] = v[16 + t] = 0.f;
-      float2 w = make_float2(kj.x, kj.y);
-#pragma unroll
-      for (int t = j; t < 16; ++t) {
-        if (t > j) {
-          w.x *= al[t].x;
-          w.y *= al[t].y;
-        }
-        const float2 qt = unpack_bf16(pf.q[t]), kt = unpack_bf16(pf.k[t]);
-        v[t] = fmaf(qt.x, w.x, qt.y * w.y);
-        v[16 + t] = fmaf(kt.x, w.x, kt.y * w.y);
-      }
-#pragma unroll
-      for (int m = 16, nl = 32; m >= 1; m >>= 1, nl >>= 1) {
-        const bool up = (lane & m) != 0;
-        const int hn = nl / 2;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (i < hn) {
-            const float send = up ? v[i] : v[i + hn];
-            const float keep = up ? v[i + hn] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-          }
-        }
-      }
-      res[j] = v[0];
-      if (hw) *slot(j, lane) = v[0];
-    }
+  for (int p = 0; p < 6; ++p) {
+    const int a = p == 0 ? 1 : (p < 3 ? 2 : 3);
+    const int b = p - a * (a - 1) / 2;
+    const int row = tid >> 4, j = tid & 15;  // 16 rows x 16 pieces
+    const uint4 src = *reinterpret_cast<const uint4*>(sm + P_VIEW + sw_chunk(view_base(b) + 16 * b + row, j, VIEW_HALF));
+    const float4 s0 = *reinterpret_cast<const float4*>(vec + VEC_D + p * 128 + 8 * j);
+    const float4 s1 = *reinterpret_cast<const float4*>(vec + VEC_D + p * 128 + 8 * j + 4);
+    const float2 x0 = unpack_bf16(src.x), x1 = unpack_bf16(src.y), x2 = unpack_bf16(src.z), x3 = unpack_bf16(src.w);
+    const uint4 dst = make_uint4(pack_bf16(x0.x * s0.x, x0.y * s0.y), pack_bf16(x1.x * s0.z, x1.y * s0.w),
+                                 pack_bf16(x2.x * s1.x, x2.y * s1.y), pack_bf16(x3.x * s1.z, x3.y * s1.w));
+    *reinterpret_cast<uint4*>(sm + P_VIEW + sw_chunk(view_base(a) + 16 * b + row, j, VIEW_HALF)) = dst;
   }
-  __syncthreads();
-  if (mine && !hw) {
-    const int t = lane & 15;
-    const float bt = beta_s[16 * da + t];
+}
+
+// The diagonal 16x16 tiles of the out-of-range blocks (bit a of `pairwise`), pair by pair, from the values the
+// decay pass left in the staging area: q and k (bf16, prepared) and alpha (fp32, in place of the gate input),
+// zero q, k and alpha = 1 past the sequence's end. One warp per (block, column j): lane l takes channels
+// 2l, 2l + 1 of each 64-channel half, forms its share of A_qk[t][j] = sum_c q_tc k_jc w_tjc (t >= j) and
+// A_kk[t][j] = sum_c k_tc k_jc w_tjc (t > j), w_tjc = prod_{m=j+1..t} alpha_mc, for the 16 rows t of the block,
+// and a reduce-scatter over the warp leaves lane l with entry l. Results go to `out` as fp32
+// [A_kk | A_qk][block][t][j], A_kk with beta_t applied. Kept out of line so that its registers do not
+// weigh on the kernel's main path, which never calls it for chunks within range.
+__device__ __noinline__ void p_diag_pairwise(const unsigned char* sm, int pairwise, const float* beta_s, float* out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int blocks[4], nb = 0;
+  for (int a = 0; a < 4; ++a)
+    if ((pairwise >> a) & 1) blocks[nb++] = a;
+  for (int item = warp; item < 16 * nb; item += NTHREADS / 32) {
+    const int a = blocks[item >> 4], j = item & 15;
+    const int rj = 16 * a + j;
+    float kj[4], w[4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float sum = res[j] + *slot(j, lane);
-      *slot(j, lane) = lane < 16 ? (t >= j ? sum : 0.f) : (t > j ? sum * bt : 0.f);
+    for (int h = 0; h < 2; ++h) {
+      const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + P_KS + h * 8192 + rj * 128 + lane * 4));
+      kj[2 * h] = kv.x;
+      kj[2 * h + 1] = kv.y;
     }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) w[m] = kj[m];
+    float v[32];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      float sq = 0.f, sk = 0.f;
+      if (t >= j) {
+        const int rt = 16 * a + t;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + P_QS + h * 8192 + rt * 128 + lane * 4));
+          const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + P_KS + h * 8192 + rt * 128 + lane * 4));
+          if (t > j) {
+            const float2 al = *reinterpret_cast<const float2*>(sm + P_GS + h * 16384 + rt * 256 + lane * 8);
+            w[2 * h] *= al.x;
+            w[2 * h + 1] *= al.y;
+          }
+          sq = fmaf(qv.x, w[2 * h], fmaf(qv.y, w[2 * h + 1], sq));
+          sk = fmaf(kv.x, w[2 * h], fmaf(kv.y, w[2 * h + 1], sk));
+        }
+      }
+      v[t] = sq;
+      v[16 + t] = sk;
+    }
+#pragma unroll
+    for (int m = 16, nl = 32; m >= 1; m >>= 1, nl >>= 1) {
+      const bool up = (lane & m) != 0;
+      const int hn = nl / 2;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i < hn) {
+          const float send = up ? v[i] : v[i + hn];
+          const float keep = up ? v[i + hn] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+    }
+    const int t = lane & 15;
+    if (lane < 16)
+      out[1024 + (a * 16 + t) * 16 + j] = t >= j ? v[0] : 0.f;
+    else
+      out[(a * 16 + t) * 16 + j] = t > j ? v[0] * beta_s[16 * a + t] : 0.f;
   }
 }
 
@@ -392,10 +425,26 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     if (p.qk_l2norm) l2norm_qk(pf, reinterpret_cast<float*>(sm + P_VEC) + VEC_D, tid, da);
     float2 al[16];
     decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, load_bias2(p, h, c0), al);
-    __syncthreads();  // block sums and flags published; every input is in registers (staging is dead)
+    __syncthreads();  // block sums and flags published; every input is in registers
     pairwise = pairwise_blocks(sm, LY);
+    if (pairwise) {  // CTA-uniform; never taken within range
+      if ((pairwise >> da) & 1) {
+        // the prepared inputs of this out-of-range block back into the staging area, alpha over the gate input
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int t = 16 * da + i;
+          *reinterpret_cast<uint32_t*>(sm + P_QS + hc * 8192 + t * 128 + cc * 2) = pf.q[i];
+          *reinterpret_cast<uint32_t*>(sm + P_KS + hc * 8192 + t * 128 + cc * 2) = pf.k[i];
+          *reinterpret_cast<float2*>(sm + P_GS + hc * 16384 + t * 256 + cc * 4) = al[i];
+        }
+      }
+      __syncthreads();
+      p_diag_pairwise(sm, pairwise, beta_s, reinterpret_cast<float*>(sm + P_DIAG));
+      __syncthreads();  // the staging area is read; the operands overwrite it next
+    }
     p_operands(sm, pf, da, c0, pairwise, al, blk + WB_WQ + (even ? 8192 : 0), blk + WB_KA + (even ? 8192 : 0));
-    if (pairwise) p_diag_pairwise(reinterpret_cast<float*>(sm + P_DIAG), pf, al, beta_s, da, pairwise);
+    __syncthreads();  // every block's own view rows and the view scales
+    view_expand(sm, tid);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
