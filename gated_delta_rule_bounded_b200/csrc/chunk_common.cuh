@@ -91,6 +91,29 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// Two fp32 lanes in one 64-bit register pair, and the packed fp32x2 product (two correctly rounded products,
+// the same values as two scalar multiplies, in one instruction).
+__device__ __forceinline__ uint64_t f2_bits(float2 v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+  return r;
+}
+__device__ __forceinline__ float2 bits_f2(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -156,6 +179,15 @@ __device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tm_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tm_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tm_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -400,30 +432,63 @@ __device__ __forceinline__ float log2_decay(int mode, float x, float sc, float g
   return fmaxf(l, L2_FLOOR);  // fmaxf(-inf, floor) = floor: alpha = 0 stays finite in log space
 }
 
+// log2_decay of two channels. For the bounded gate's logits it evaluates bounded_log_decay (gate_math.cuh)
+// with packed fp32x2 products and sums -- the same operations in the same order, so the same values.
+template <int MODE>
+__device__ __forceinline__ float2 log2_decay2(float2 x, float sc, float g_min) {
+  if constexpr (MODE == GATE_LOGITS) {
+    const float2 xs = mul2(make_float2(sc, sc), x);
+    const float2 a = mul2(make_float2(fabsf(xs.x), fabsf(xs.y)), make_float2(-1.4426950408889634f, -1.4426950408889634f));
+    float2 t, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t.x) : "f"(a.x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t.y) : "f"(a.y));
+    const float2 d = add2(make_float2(1.f, 1.f), t);
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.x) : "f"(d.x));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.y) : "f"(d.y));
+    const float2 tr = mul2(t, r);
+    const float2 sg = make_float2(xs.x >= 0.f ? r.x : tr.x, xs.y >= 0.f ? r.y : tr.y);
+    const float2 l = mul2(mul2(make_float2(g_min, g_min), sg), make_float2(LOG2E, LOG2E));
+    return make_float2(fmaxf(l.x, L2_FLOOR), fmaxf(l.y, L2_FLOOR));
+  } else {
+    return make_float2(log2_decay(MODE, x.x, sc, g_min), log2_decay(MODE, x.y, sc, g_min));
+  }
+}
+
 // Decay pass, step 1: the per-token log2-decay of channels (c0, c0+1) over the 16 tokens of block
 // da (0 past the end of the sequence), their retention factors, and the block sum, published to
 // VEC_TOT. `bias` is the logits' per-channel bias (0 without one). Each warp also records in VEC_FLAG
 // whether one of its channels' block sums lies below BLOCK_SAFE (read back by pairwise_blocks after
-// the caller's barrier).
-__device__ __forceinline__ void decay_step1(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int nv,
-                                            int da, int c0, int mode, float sc, float g_min, float2 bias,
-                                            float2 (&al)[16]) {
+// the caller's barrier). MODE is the gate mode, fixed at compile time.
+template <int MODE>
+__device__ __forceinline__ void decay_step1_t(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int nv,
+                                              int da, float sc, float g_min, float2 bias, float2 (&al)[16], int c0) {
   float* vec = reinterpret_cast<float*>(sm + L.vec);
   float2 run = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float2 l = make_float2(0.f, 0.f);
     if (16 * da + i < nv) {
-      l.x = log2_decay(mode, gate_input(mode, pf.g[i].x, bias.x), sc, g_min);
-      l.y = log2_decay(mode, gate_input(mode, pf.g[i].y, bias.y), sc, g_min);
+      const float2 x = MODE >= GATE_LOGITS ? add2(pf.g[i], bias) : pf.g[i];
+      l = log2_decay2<MODE>(x, sc, g_min);
     }
-    run.x += l.x;
-    run.y += l.y;
+    run = add2(run, l);
     al[i] = make_float2(ex2(l.x), ex2(l.y));
   }
   *reinterpret_cast<float2*>(vec + VEC_TOT + da * 128 + c0) = run;
   const unsigned out_of_range = __any_sync(0xffffffffu, run.x < BLOCK_SAFE || run.y < BLOCK_SAFE);
   if ((threadIdx.x & 31) == 0) reinterpret_cast<int*>(vec + VEC_FLAG)[threadIdx.x >> 5] = out_of_range ? 1 : 0;
+}
+
+// decay_step1_t for a gate mode known only at run time.
+__device__ __forceinline__ void decay_step1(unsigned char* sm, const IntraLayout& L, const Prefetch& pf, int nv,
+                                            int da, int c0, int mode, float sc, float g_min, float2 bias,
+                                            float2 (&al)[16]) {
+  switch (mode) {
+    case GATE_LOGITS: decay_step1_t<GATE_LOGITS>(sm, L, pf, nv, da, sc, g_min, bias, al, c0); break;
+    case GATE_SOFTPLUS: decay_step1_t<GATE_SOFTPLUS>(sm, L, pf, nv, da, sc, g_min, bias, al, c0); break;
+    case KDA_GATE_LOG: decay_step1_t<KDA_GATE_LOG>(sm, L, pf, nv, da, sc, g_min, bias, al, c0); break;
+    default: decay_step1_t<KDA_GATE_ALPHA>(sm, L, pf, nv, da, sc, g_min, bias, al, c0); break;
+  }
 }
 
 // After decay_step1 and a barrier: bit a set when block a needs its diagonal blocks pairwise (the

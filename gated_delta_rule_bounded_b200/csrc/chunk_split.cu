@@ -236,15 +236,15 @@ __device__ __forceinline__ void p_operands(unsigned char* sm, const Prefetch& pf
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int t = 16 * da + i;
-    E.x *= al[i].x;
-    E.y *= al[i].y;
+    E = mul2(E, al[i]);
     const float2 qf = unpack_bf16(pf.q[i]), kf = unpack_bf16(pf.k[i]);
-    const float rx = E.x * DI.x, ry = E.y * DI.y;      // 2^{G_t - R_da}
-    const float gx = E.x * GS.x, gy = E.y * GS.y;      // Gamma_t
-    *reinterpret_cast<uint32_t*>(sm + P_KQ + sw_e(rk + i, c0, 16384)) = pack_bf16(kf.x * rx, kf.y * ry);
-    *reinterpret_cast<uint32_t*>(sm + P_KQ + sw_e(rk + 16 + i, c0, 16384)) = pack_bf16(qf.x * rx, qf.y * ry);
-    *reinterpret_cast<uint32_t*>(sm + P_KG + sw_e(t, c0, 8192)) = pack_bf16(kf.x * gx, kf.y * gy);
-    *reinterpret_cast<uint32_t*>(qg_dst + sw_e(t, c0, 16384)) = pack_bf16(qf.x * gx, qf.y * gy);
+    const float2 rr = mul2(E, DI);   // 2^{G_t - R_da}
+    const float2 gg = mul2(E, GS);   // Gamma_t
+    const float2 kr = mul2(kf, rr), qr = mul2(qf, rr), kg = mul2(kf, gg), qg = mul2(qf, gg);
+    *reinterpret_cast<uint32_t*>(sm + P_KQ + sw_e(rk + i, c0, 16384)) = pack_bf16(kr.x, kr.y);
+    *reinterpret_cast<uint32_t*>(sm + P_KQ + sw_e(rk + 16 + i, c0, 16384)) = pack_bf16(qr.x, qr.y);
+    *reinterpret_cast<uint32_t*>(sm + P_KG + sw_e(t, c0, 8192)) = pack_bf16(kg.x, kg.y);
+    *reinterpret_cast<uint32_t*>(qg_dst + sw_e(t, c0, 16384)) = pack_bf16(qg.x, qg.y);
   }
   const bool kt_apart = (pairwise >> 3) & 1;
   const float2 PM = make_float2(ex2(e[3].x - eda.x), ex2(e[3].y - eda.y));  // 2^{e[3] - e[da]}
@@ -252,15 +252,15 @@ __device__ __forceinline__ void p_operands(unsigned char* sm, const Prefetch& pf
   float2 F = make_float2(1.f, 1.f);  // 2^{e[da] - G_i}, tokens after i within the block
 #pragma unroll
   for (int i = 15; i >= 0; --i) {
-    const float2 kf = unpack_bf16(pf.k[i]);
-    const float kx = kf.x * F.x, ky = kf.y * F.y;
+    const float2 kx = mul2(unpack_bf16(pf.k[i]), F);
     // block da's rows of view da (for an out-of-range block they are its discarded diagonal tile, and the
     // source of its rows in the later views)
-    *reinterpret_cast<uint32_t*>(sm + P_VIEW + sw_e(vrow + i, c0, VIEW_HALF)) = pack_bf16(kx, ky);
-    if (kt_apart)
-      *reinterpret_cast<uint32_t*>(kt_dst + sw_e(16 * da + i, c0, 8192)) = pack_bf16(kx * PM.x, ky * PM.y);
-    F.x *= al[i].x;
-    F.y *= al[i].y;
+    *reinterpret_cast<uint32_t*>(sm + P_VIEW + sw_e(vrow + i, c0, VIEW_HALF)) = pack_bf16(kx.x, kx.y);
+    if (kt_apart) {
+      const float2 kt = mul2(kx, PM);
+      *reinterpret_cast<uint32_t*>(kt_dst + sw_e(16 * da + i, c0, 8192)) = pack_bf16(kt.x, kt.y);
+    }
+    F = mul2(F, al[i]);
   }
 }
 
@@ -277,9 +277,12 @@ __device__ __forceinline__ void view_expand(unsigned char* sm, int tid) {
     const uint4 src = *reinterpret_cast<const uint4*>(sm + P_VIEW + sw_chunk(view_base(b) + 16 * b + row, j, VIEW_HALF));
     const float4 s0 = *reinterpret_cast<const float4*>(vec + VEC_D + p * 128 + 8 * j);
     const float4 s1 = *reinterpret_cast<const float4*>(vec + VEC_D + p * 128 + 8 * j + 4);
-    const float2 x0 = unpack_bf16(src.x), x1 = unpack_bf16(src.y), x2 = unpack_bf16(src.z), x3 = unpack_bf16(src.w);
-    const uint4 dst = make_uint4(pack_bf16(x0.x * s0.x, x0.y * s0.y), pack_bf16(x1.x * s0.z, x1.y * s0.w),
-                                 pack_bf16(x2.x * s1.x, x2.y * s1.y), pack_bf16(x3.x * s1.z, x3.y * s1.w));
+    const float2 y0 = mul2(unpack_bf16(src.x), make_float2(s0.x, s0.y));
+    const float2 y1 = mul2(unpack_bf16(src.y), make_float2(s0.z, s0.w));
+    const float2 y2 = mul2(unpack_bf16(src.z), make_float2(s1.x, s1.y));
+    const float2 y3 = mul2(unpack_bf16(src.w), make_float2(s1.z, s1.w));
+    const uint4 dst = make_uint4(pack_bf16(y0.x, y0.y), pack_bf16(y1.x, y1.y), pack_bf16(y2.x, y2.y),
+                                 pack_bf16(y3.x, y3.y));
     *reinterpret_cast<uint4*>(sm + P_VIEW + sw_chunk(view_base(a) + 16 * b + row, j, VIEW_HALF)) = dst;
   }
 }
@@ -352,6 +355,7 @@ __device__ __noinline__ void p_diag_pairwise(const unsigned char* sm, int pairwi
   }
 }
 
+template <int MODE>  // the gate mode of p (KDA_GATE_ALPHA, KDA_GATE_LOG, GATE_LOGITS, GATE_SOFTPLUS)
 __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, unsigned char* ws,
                                                                   const __grid_constant__ PMaps maps) {
   extern __shared__ __align__(1024) unsigned char sm[];
@@ -363,7 +367,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   // after this whole grid has completed (griddepcontrol.wait).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int h = blockIdx.y;
-  const float gsc = p.gate_mode >= GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
+  const float gsc = MODE >= GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
   const int64_t slot = blockIdx.x;
   int n, j;
   if (!locate_slot(p, slot, n, j)) return;  // uniform across the CTA
@@ -424,7 +428,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     }
     if (p.qk_l2norm) l2norm_qk(pf, reinterpret_cast<float*>(sm + P_VEC) + VEC_D, tid, da);
     float2 al[16];
-    decay_step1(sm, LY, pf, nv, da, c0, p.gate_mode, gsc, p.g_min, load_bias2(p, h, c0), al);
+    decay_step1_t<MODE>(sm, LY, pf, nv, da, gsc, p.g_min, load_bias2(p, h, c0), al, c0);
     __syncthreads();  // block sums and flags published; every input is in registers
     pairwise = pairwise_blocks(sm, LY);
     if (pairwise) {  // CTA-uniform; never taken within range
@@ -474,45 +478,55 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
       bulk_store(blk + kt + 8192, sb + P_VIEW + VIEW_HALF, 8192);
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
-    // ---- read back: warps 0-3 the first product, 4-7 the second; TMEM lane L = 32 (warp & 3) + lane
+    // ---- read back. TMEM lane L = 32 (warp & 3) + lane is column i = L & 63 of A in views (3, 2) for L < 64 and
+    // (0, 1) for L >= 64 (first and second product). Warps 0-3 take the A_kk columns and go on to the inverse;
+    // warps 4-7 meanwhile take A_qk^T and store it.
     {
-      const int L = 32 * (warp & 3) + lane, second = warp >> 2;
-      const int a = second ? (L < 64 ? 2 : 1) : (L < 64 ? 3 : 0);
-      const int i = L & 63;
-      uint32_t r[32];
-      tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * second + (L < 64 ? 0 : 32), r);
-      const bool from_pairs = ((pairwise >> a) & 1) && (i >> 4) == a;
-      const float* dg = reinterpret_cast<const float*>(sm + P_DIAG);
-      float* akk = reinterpret_cast<float*>(sm + P_AKK);
-      float vq[16];
+      const int L = 32 * (warp & 3) + lane, i = L & 63;
+      const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (L < 64 ? 0 : 32) + (warp < 4 ? 0 : 16);
+      uint32_t r1[16], r2[16];
+      tm_ld16(tl, r1);       // first product: view 3 or 0
+      tm_ld16(tl + 64, r2);  // second product: view 2 or 1
+      tm_wait_ld();
+      const float* dg = reinterpret_cast<const float*>(sm + P_DIAG) + (warp < 4 ? 0 : 1024);
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const int t = 16 * a + jj;
-        float vk = __uint_as_float(r[jj]);
-        vq[jj] = __uint_as_float(r[16 + jj]);
-        if (from_pairs) {
-          vk = dg[(a * 16 + jj) * 16 + (i & 15)];
-          vq[jj] = dg[1024 + (a * 16 + jj) * 16 + (i & 15)];
-        } else {
-          vk = i < t ? vk * beta_s[t] : 0.f;
-          vq[jj] = i <= t ? vq[jj] : 0.f;
+      for (int part = 0; part < 2; ++part) {
+        const int a = part == 0 ? (L < 64 ? 3 : 0) : (L < 64 ? 2 : 1);
+        const bool from_pairs = ((pairwise >> a) & 1) && (i >> 4) == a;
+        float v[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int t = 16 * a + jj;
+          const float x = __uint_as_float(part == 0 ? r1[jj] : r2[jj]);
+          if (warp < 4)
+            v[jj] = from_pairs ? dg[(a * 16 + jj) * 16 + (i & 15)] : (i < t ? x * beta_s[t] : 0.f);
+          else
+            v[jj] = from_pairs ? dg[(a * 16 + jj) * 16 + (i & 15)] : (i <= t ? x : 0.f);
         }
-        akk[t * 64 + i] = vk;
+        if (warp < 4) {
+          float* akk = reinterpret_cast<float*>(sm + P_AKK);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) akk[(16 * a + jj) * 64 + i] = v[jj];
+        } else {
+          *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a, 0)) =
+              make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+          *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a + 1, 0)) = make_uint4(
+              pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+        }
       }
-      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a, 0)) =
-          make_uint4(pack_bf16(vq[0], vq[1]), pack_bf16(vq[2], vq[3]), pack_bf16(vq[4], vq[5]), pack_bf16(vq[6], vq[7]));
-      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a + 1, 0)) = make_uint4(
-          pack_bf16(vq[8], vq[9]), pack_bf16(vq[10], vq[11]), pack_bf16(vq[12], vq[13]), pack_bf16(vq[14], vq[15]));
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();  // A_kk and A_qk^T complete
-    if (tid == 0) {
-      bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    if (warp < 4) {
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // A_kk complete
+      // ---- T' = (I + A_kk)^-1 Diag(beta)
+      inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+    } else {
+      fence_async_smem();
+      asm volatile("bar.sync 3, 128;" ::: "memory");  // A_qk^T complete
+      if (tid == 128) {
+        bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
     }
-    // ---- T' = (I + A_kk)^-1 Diag(beta) on warps 0-3
-    if (warp < 4) inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -567,6 +581,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     // the kernel does.
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   }
+  if (tid == 128) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the A_qk^T store
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -877,8 +892,12 @@ bool split_maps_ok(const ScanParams& p) {
 }
 
 cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
-  static std::atomic<uint64_t> cfg_p{0}, cfg_s{0};
-  cudaError_t e = set_smem_once(chunk_intra_kernel, P_SMEM, cfg_p);
+  static std::atomic<uint64_t> cfg_p[4], cfg_s{0};
+  auto intra = p.gate_mode == GATE_LOGITS    ? chunk_intra_kernel<GATE_LOGITS>
+               : p.gate_mode == GATE_SOFTPLUS ? chunk_intra_kernel<GATE_SOFTPLUS>
+               : p.gate_mode == KDA_GATE_LOG  ? chunk_intra_kernel<KDA_GATE_LOG>
+                                              : chunk_intra_kernel<KDA_GATE_ALPHA>;
+  cudaError_t e = set_smem_once(intra, P_SMEM, cfg_p[p.gate_mode & 3]);
   if (e == cudaSuccess) e = set_smem_once(chunk_state_kernel, S_SMEM, cfg_s);
   if (e != cudaSuccess) return e;
   const int64_t slots = split_slots(p.B, p.T, p.N, p.cu != nullptr);
@@ -889,7 +908,7 @@ cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
       !token_map(&maps.g, p.gate, false, p.gs, p.B, p.T, p.H, p.K))
     return cudaErrorInvalidValue;  // callers check split_maps_ok first
   dim3 gp((unsigned)slots, (unsigned)p.H);
-  chunk_intra_kernel<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws), maps);
+  intra<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws), maps);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t grid = (int64_t)p.N * p.H * (p.V / VT);
