@@ -478,55 +478,46 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
       bulk_store(blk + kt + 8192, sb + P_VIEW + VIEW_HALF, 8192);
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
-    // ---- read back. TMEM lane L = 32 (warp & 3) + lane is column i = L & 63 of A in views (3, 2) for L < 64 and
-    // (0, 1) for L >= 64 (first and second product). Warps 0-3 take the A_kk columns and go on to the inverse;
-    // warps 4-7 meanwhile take A_qk^T and store it.
+    // ---- read back: warps 0-3 the first product, 4-7 the second; TMEM lane L = 32 (warp & 3) + lane is
+    // column i = L & 63 of A in view 3 or 0 (first product) and 2 or 1 (second)
     {
-      const int L = 32 * (warp & 3) + lane, i = L & 63;
-      const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (L < 64 ? 0 : 32) + (warp < 4 ? 0 : 16);
-      uint32_t r1[16], r2[16];
-      tm_ld16(tl, r1);       // first product: view 3 or 0
-      tm_ld16(tl + 64, r2);  // second product: view 2 or 1
-      tm_wait_ld();
-      const float* dg = reinterpret_cast<const float*>(sm + P_DIAG) + (warp < 4 ? 0 : 1024);
+      const int L = 32 * (warp & 3) + lane, second = warp >> 2;
+      const int a = second ? (L < 64 ? 2 : 1) : (L < 64 ? 3 : 0);
+      const int i = L & 63;
+      uint32_t r[32];
+      tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * second + (L < 64 ? 0 : 32), r);
+      const bool from_pairs = ((pairwise >> a) & 1) && (i >> 4) == a;
+      const float* dg = reinterpret_cast<const float*>(sm + P_DIAG);
+      float* akk = reinterpret_cast<float*>(sm + P_AKK);
+      float vq[16];
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int a = part == 0 ? (L < 64 ? 3 : 0) : (L < 64 ? 2 : 1);
-        const bool from_pairs = ((pairwise >> a) & 1) && (i >> 4) == a;
-        float v[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int t = 16 * a + jj;
-          const float x = __uint_as_float(part == 0 ? r1[jj] : r2[jj]);
-          if (warp < 4)
-            v[jj] = from_pairs ? dg[(a * 16 + jj) * 16 + (i & 15)] : (i < t ? x * beta_s[t] : 0.f);
-          else
-            v[jj] = from_pairs ? dg[(a * 16 + jj) * 16 + (i & 15)] : (i <= t ? x : 0.f);
-        }
-        if (warp < 4) {
-          float* akk = reinterpret_cast<float*>(sm + P_AKK);
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) akk[(16 * a + jj) * 64 + i] = v[jj];
+      for (int jj = 0; jj < 16; ++jj) {
+        const int t = 16 * a + jj;
+        float vk = __uint_as_float(r[jj]);
+        vq[jj] = __uint_as_float(r[16 + jj]);
+        if (from_pairs) {
+          vk = dg[(a * 16 + jj) * 16 + (i & 15)];
+          vq[jj] = dg[1024 + (a * 16 + jj) * 16 + (i & 15)];
         } else {
-          *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a, 0)) =
-              make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-          *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a + 1, 0)) = make_uint4(
-              pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+          vk = i < t ? vk * beta_s[t] : 0.f;
+          vq[jj] = i <= t ? vq[jj] : 0.f;
         }
+        akk[t * 64 + i] = vk;
       }
+      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a, 0)) =
+          make_uint4(pack_bf16(vq[0], vq[1]), pack_bf16(vq[2], vq[3]), pack_bf16(vq[4], vq[5]), pack_bf16(vq[6], vq[7]));
+      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a + 1, 0)) = make_uint4(
+          pack_bf16(vq[8], vq[9]), pack_bf16(vq[10], vq[11]), pack_bf16(vq[12], vq[13]), pack_bf16(vq[14], vq[15]));
     }
-    if (warp < 4) {
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // A_kk complete
-      // ---- T' = (I + A_kk)^-1 Diag(beta)
-      inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
-    } else {
-      fence_async_smem();
-      asm volatile("bar.sync 3, 128;" ::: "memory");  // A_qk^T complete
-      if (tid == 128) {
-        bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-      }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // A_kk and A_qk^T complete
+    if (tid == 0) {
+      bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
+    // ---- T' = (I + A_kk)^-1 Diag(beta) on warps 0-3
+    if (warp < 4) inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -581,7 +572,6 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     // the kernel does.
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   }
-  if (tid == 128) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the A_qk^T store
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
