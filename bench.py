@@ -88,16 +88,21 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 # dram__bytes_write.sum of every kernel the step launches). They hold only for the kernel sources they were
 # taken on, so the sources' sha256 is kept beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
-    # chunk_intra_kernel 404,795,392 + 359,710,208; chunk_state_kernel 506,546,432 + 84,204,288
-    "prefill": {"bytes": 1355256320, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "8e578cec51f4b2a8c9123e9926752cea1b27036a61725d3b0797108e08b6ffa1"},
-    # decode_bulk_kernel 410,584,832 + 345,193,472
-    "decode": {"bytes": 755778304, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "f0ea99d5bd7f661f413f4c3d98366402d4a4d4fb81de98a6017e64fd316622f2"},
-    # softplus_diag_kernel 404,549,888 + 41,925,120; chunk_intra_kernel<true> 455,110,656 + 356,195,840;
-    # chunk_state_kernel 506,546,176 + 84,393,216 (the unbounded gate's chunked prefill)
-    "softplus": {"bytes": 1848720896, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "8e578cec51f4b2a8c9123e9926752cea1b27036a61725d3b0797108e08b6ffa1"},
+    # chunk_intra_kernel<2> 404.6 + 359.1 MB; chunk_state_kernel 506.5 + 84.7 MB
+    "prefill": {"bytes": 1354900000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
+    # decode_bulk_kernel 410.6 + 345.1 MB
+    "decode": {"bytes": 755700000, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "ef9a4cbaa38adbffc745f72fc725ecb508aa04553436b13be7ca12ae07b738db"},
+    # chunk_intra_kernel<3> 405.0 + 359.0 MB; chunk_state_kernel 506.5 + 84.2 MB (the unbounded gate's prefill)
+    "softplus": {"bytes": 1354700000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                 "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
+    # chunk_intra_kernel<2> 8,102.6 + 7,283.6 MB; chunk_state_kernel 9,227.4 + 1,885.2 MB (16 packed sequences)
+    "varlen": {"bytes": 26498800000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
+    # chunk_intra_kernel<2> 2,407.4 + 2,121.2 MB; chunk_state_kernel 3,254.9 + 1,060.3 MB (4 x 16384 x 32, V = 256)
+    "long_kv": {"bytes": 8843800000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
     # bounded_decay_kernel 201,388,032 + 154,186,496; scan_backward_kernel 17,959,960,832 + 27,343,060,992;
     # bounded_decay_backward_kernel 402,712,832 + 162,471,424 (one backward step from the logits)
     "backward": {"bytes": 46223780608, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
@@ -398,7 +403,7 @@ def softplus_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
     }
 
 
-def workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, w, cpu_heads):
+def workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, w, cpu_heads, key):
     """Throughput of one more prefill workload through the same call as the headline (kda_prefill_logits,
     two-kernel path, gate from the logits): the 16 packed variable-length sequences with their own initial
     states, or the long K != V batch. tokens/s, the HBM roofline of its algorithmic bytes, e2e through
@@ -429,7 +434,8 @@ def workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, 
         "tokens_per_step": B * T, "gpu_launches": 2 * steps,  # kernel P, kernel S
         "kernels_ms": {"prefill_logits": ms},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": None, "kernel": "kda_prefill_logits", "bytes_per_launch": pb, "ms_per_launch": ms,
+                     "traffic": measured_traffic(key), "kernel": "kda_prefill_logits", "bytes_per_launch": pb,
+                     "ms_per_launch": ms,
                      "peak_source": f"{peak_src} hbm_gbs",
                      "tensor": {"tflops_at_C64_formula": flops / (ms / 1e3) / 1e12, "peak": bf16_peak,
                                 "frac": flops / (ms / 1e3) / 1e12 / bf16_peak, "flops_per_launch": flops}},
@@ -615,7 +621,7 @@ def gpu_arm(args, rank, world, local):
     more = {}
     for key, wl, heads in (("varlen", W.VARLEN, 16), ("long_kv", W.LONG_KV, 4)):
         if args.workload in ("all", key):
-            more[key] = workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, wl, heads)
+            more[key] = workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, wl, heads, key)
             torch.cuda.empty_cache()
     bwd = None
     if args.workload in ("all", "backward"):

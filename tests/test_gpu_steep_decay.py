@@ -142,3 +142,46 @@ def test_prefill_logits_softplus_both_paths(kda, use_workspace):
     ro, rs = oracle.scan(d["q"], d["k"], d["v"], alpha, d["beta"], d["initial_state"])
     check(o, ro, "bf16", "o")
     check(sf, rs, "bf16", "final_state")
+
+
+@PATHS
+def test_prefill_logits_every_option_together(kda, use_workspace):
+    # packed ragged sequences with initial states, dt_bias, in-kernel L2Norm and beta sigmoid, value-by-key
+    # states and a bounded gate steep enough (g_min = -7) to put some blocks out of range
+    lens = [64, 1, 0, 150, 77]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    T, H = int(cu[-1]), 3
+    d = W.random_scan_case(1, T, H, 128, 128, seed=81, dtype="bf16", z_std=2.0, init_std=None, raw_inputs=True)
+    d["cu_seqlens"] = cu
+    d["A_log"] = torch.tensor([0.8, -0.3, 0.2])
+    s0 = torch.randn(len(lens), H, 128, 128, generator=torch.Generator().manual_seed(82)) * 0.1
+    b = torch.randn(H, 128, generator=torch.Generator().manual_seed(83))
+    g = to_dev(d)
+    o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], -7.0, g["beta"],
+                               s0.transpose(-1, -2).contiguous().to(DEV), g["cu_seqlens"], qk_l2norm=True,
+                               beta_logits=True, state_layout="vk", dt_bias=b.to(DEV), use_workspace=use_workspace)
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    alpha, lg = oracle.bounded_decay(d["z"], d["A_log"], -7.0, return_log=True, dt_bias=b)
+    assert (block_sums_log2(lg) < SAFE_LOG2).any()
+    ro, rs = oracle.scan(oracle.l2norm(d["q"]), oracle.l2norm(d["k"]), d["v"], alpha, oracle.sigmoid(d["beta"]),
+                         s0, d["cu_seqlens"])
+    check(o, ro, "bf16", "o")
+    check(sf.transpose(-1, -2), rs, "bf16", "final_state")
+
+
+@pytest.mark.slow
+def test_softplus_prefill_workload_sampled_heads(kda):
+    # the bench's unbounded-gate leg: the 4096 x 96 prefill through Kimi Linear's gate on the two-kernel path
+    d = W.make_scan_inputs(W.PREFILL)
+    g = to_dev(d)
+    o, sf = kda.prefill_logits(g["q"], g["k"], g["v"], g["z"], g["A_log"], g["g_min"], g["beta"], None,
+                               gate="softplus")
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    heads = [0, 13, 47, 95]
+    alpha, lg = oracle.softplus_decay(d["z"][:, :, heads], d["A_log"][heads], return_log=True)
+    assert (block_sums_log2(lg) < SAFE_LOG2).any()
+    ro, rs = oracle.scan(d["q"][:, :, heads], d["k"][:, :, heads], d["v"][:, :, heads], alpha, d["beta"][:, :, heads])
+    check(o[:, :, heads], ro, "bf16", "o")
+    check(sf[:, heads], rs, "bf16", "final_state")
