@@ -88,9 +88,10 @@ static_assert(VEC_TOT >= VEC_D + 6 * 128, "view scales fit before the block sums
 constexpr int S_OPS = 0;                    // 2 x operand block (66048 B, padded to 66560)
 constexpr int S_OPS_STRIDE = 66560;
 constexpr int S_V = 2 * S_OPS_STRIDE;       // 2 x 16K v tile [i][v], two halves (MN-major A)
-constexpr int S_BAR = S_V + 2 * 16384;      // mbarriers: ops0, ops1, mma; TMEM base
+constexpr int S_BAR = S_V + 2 * 16384;      // mbarriers: part 1 x2, part 2 x2, mma; TMEM base
 constexpr int S_SMEM = S_BAR + 64;
 static_assert(S_SMEM <= 227 * 1024, "shared memory budget");
+static_assert(WB_KA % 16 == 0 && WB_TP % 16 == 0 && WB_BYTES % 16 == 0, "bulk copies move 16-byte multiples");
 static_assert(S_V % 1024 == 0 && S_OPS_STRIDE % 1024 == 0, "swizzle atoms need 1 KB alignment");
 
 // Kernel S tensor memory (columns; lane = value column v of the tile). S^T, U^T and O^T in fp32 are
@@ -578,8 +579,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(P_TM_COLS));
 }
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+// One bulk copy completing on `bar` (the caller has announced the bytes with expect_tx).
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
@@ -627,13 +628,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
   x.boff = 0;
   x.bst = 0;
 
-  const uint32_t bar_ops = sb + S_BAR, bar_mma = sb + S_BAR + 16;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + S_BAR + 24);
+  // Each operand block arrives in two parts, each with its own mbarrier per buffer: part 1 (-W, Q*Gamma,
+  // T', gamma_C: used by the conversion and group A) and part 2 (A_qk^T, K*gamma_C/Gamma: group B). A buffer's
+  // part 1 is refilled as soon as its chunk's group A is done, part 2 once its group B is, so part 1 and the
+  // v tile are fetched about a chunk and a half ahead.
+  const uint32_t bar_p1 = sb + S_BAR, bar_p2 = sb + S_BAR + 16, bar_mma = sb + S_BAR + 32;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + S_BAR + 40);
   auto block_src = [&](int c) { return ws + ((size_t)(sbase_slot + c) * p.H + h) * WB_BYTES; };
+  auto load_part1 = [&](int c, int b) {  // thread 0
+    const uint32_t dst = sb + S_OPS + b * S_OPS_STRIDE, bar = bar_p1 + 8 * b;
+    const unsigned char* src = block_src(c);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(WB_KA + (WB_BYTES - WB_TP))
+                 : "memory");
+    bulk_copy(dst + WB_WQ, src + WB_WQ, WB_KA - WB_WQ, bar);
+    bulk_copy(dst + WB_TP, src + WB_TP, WB_BYTES - WB_TP, bar);
+  };
+  auto load_part2 = [&](int c, int b) {  // thread 0
+    const uint32_t dst = sb + S_OPS + b * S_OPS_STRIDE, bar = bar_p2 + 8 * b;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(WB_TP - WB_KA) : "memory");
+    bulk_copy(dst + WB_KA, block_src(c) + WB_KA, WB_TP - WB_KA, bar);
+  };
 
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ops));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_ops + 8));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_p1));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_p1 + 8));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_p2));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_p2 + 8));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -648,10 +668,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
   const uint32_t tmem = *tslot;
   const uint32_t tlane = tmem + ((uint32_t)(32 * quad) << 16);
 
-  if (n_chunks > 0) {
-    load_v(x, sb + S_V, t0, (int)min((int64_t)C, t1 - t0), tid);
-    cp_async_commit();
-  }
+  // v tiles of chunks 0 and 1; one cp.async group per chunk from here on (empty past the end), so that at
+  // the top of chunk c only chunk c+1's group may still be pending.
+  if (n_chunks > 0) load_v(x, sb + S_V, t0, (int)min((int64_t)C, t1 - t0), tid);
+  cp_async_commit();
+  if (n_chunks > 1) load_v(x, sb + S_V + 16384, t0 + C, (int)min((int64_t)C, t1 - t0 - C), tid);
+  cp_async_commit();
 
   // Initial state: TMEM lane v holds column v of S; this thread moves columns [64*half, +64).
   const size_t hbase = ((size_t)n * p.H + h) * (size_t)KD * p.V;  // this head's state
@@ -669,7 +691,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
   // first block is fetched once that grid has completed (a no-op when launched without a dependency).
   if (tid == 0 && n_chunks > 0) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    bulk_load(sb + S_OPS, block_src(0), WB_BYTES, bar_ops);
+    load_part1(0, 0);
+    load_part2(0, 0);
+    if (n_chunks > 1) load_part1(1, 1);
   }
 
   // Each chunk's MMAs complete twice on bar_mma, group A then group B, and every completion is
@@ -684,9 +708,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     const uint32_t vbuf = sb + S_V + buf * 16384;
     const uint32_t tm_u = buf ? TM_UO : TM_UE;
 
-    // The previous chunk's group B is done (TMEM S^T holds S_{c-1}); this chunk's operands have landed.
+    // The previous chunk's group B is done (TMEM S^T holds S_{c-1}); this chunk's part 1 and v have landed.
     bool w = c == 0 || mbar_wait(bar_mma, 1, &g_split_timeout);
-    w = w && mbar_wait(bar_ops + 8 * buf, (c >> 1) & 1, &g_split_timeout);
+    w = w && mbar_wait(bar_p1 + 8 * buf, (c >> 1) & 1, &g_split_timeout);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's v tile
+    fence_async_smem();
     ok = __syncthreads_and(w);
     tc_fence_after();
     if (!ok) break;
@@ -714,18 +740,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
-    cp_async_wait_all();  // this chunk's v tile
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    // The other buffers' last readers (chunk c-1's MMAs) are done: prefetch chunk c+1 into them.
-    if (c + 1 < n_chunks) {
-      if (tid == 0) bulk_load(sb + S_OPS + (buf ^ 1) * S_OPS_STRIDE, block_src(c + 1), WB_BYTES, bar_ops + 8 * (buf ^ 1));
-      load_v(x, sb + S_V + (buf ^ 1) * 16384, tc0 + C, (int)min((int64_t)C, t1 - tc0 - C), tid);
-    }
-    cp_async_commit();
+    // Chunk c-1's group B is done: the other buffer's part 2 takes chunk c+1's.
+    if (tid == 0 && c + 1 < n_chunks) load_part2(c + 1, buf ^ 1);
 
     // ---- group A: [U^T | O^T] = S^T [-W ; Q*Gamma]^T, then U^T += V^T T'^T ---------------------------
     if (tid == 0) {
@@ -747,6 +767,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     tc_fence_after();
     if (!ok) break;
 
+    // Group A is done with this buffer's part 1 and v tile: refill them with chunk c+2's.
+    if (c + 2 < n_chunks) {
+      if (tid == 0) load_part1(c + 2, buf);
+      load_v(x, vbuf, tc0 + 2 * C, (int)min((int64_t)C, t1 - tc0 - 2 * C), tid);
+    }
+    cp_async_commit();
+
     // ---- U^T -> its bf16 copy ---------------------------------------------------------------------
     {
       uint32_t r[32], b16[16];
@@ -757,8 +784,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(mbar_wait(bar_p2 + 8 * buf, (c >> 1) & 1, &g_split_timeout));  // and part 2 landed
     tc_fence_after();
+    if (!ok) break;
 
     // ---- group B: [O^T | S^T] += U^T [A_qk ; (K*gamma_C/Gamma)^T]^T, B MN-major (rows: the K index) ------
     if (tid == 0) {
@@ -797,8 +825,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     // A wait expired: give the MMAs and operand loads that may still be in flight a bounded wait.
     mbar_wait(bar_mma, 0, &g_split_timeout);
     mbar_wait(bar_mma, 1, &g_split_timeout);
-    mbar_wait(bar_ops, 0, &g_split_timeout);
-    mbar_wait(bar_ops + 8, 0, &g_split_timeout);
+    for (int b = 0; b < 2; ++b) {
+      mbar_wait(bar_p1 + 8 * b, 0, &g_split_timeout);
+      mbar_wait(bar_p2 + 8 * b, 0, &g_split_timeout);
+    }
   }
   tc_fence_before();
   __syncthreads();
