@@ -27,6 +27,7 @@
 // floor(cu[n]/64) + n + j with them (unique: a sequence's slots end before the next one's begin).
 #include <cuda.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "chunk_common.cuh"
@@ -358,7 +359,7 @@ __device__ __noinline__ void p_diag_pairwise(const unsigned char* sm, int pairwi
 
 template <int MODE>  // the gate mode of p (KDA_GATE_ALPHA, KDA_GATE_LOG, GATE_LOGITS, GATE_SOFTPLUS)
 __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, unsigned char* ws,
-                                                                  const __grid_constant__ PMaps maps) {
+                                                                  const __grid_constant__ PMaps maps, int64_t n_slots) {
   extern __shared__ __align__(1024) unsigned char sm[];
   const uint32_t sb = smem_u32(sm);
   constexpr IntraLayout LY{-1, -1, -1, -1, -1, -1, P_AKK, -1, P_TP, P_TB, P_VEC};
@@ -367,17 +368,6 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
   // Kernel S may be scheduled once every CTA of this grid has started; it reads the workspace only
   // after this whole grid has completed (griddepcontrol.wait).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int h = blockIdx.y;
-  const float gsc = MODE >= GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
-  const int64_t slot = blockIdx.x;
-  int n, j;
-  if (!locate_slot(p, slot, n, j)) return;  // uniform across the CTA
-  int64_t t0, t1, brow;
-  seq_range(p, n, t0, t1, brow);
-  const int64_t tc0 = t0 + (int64_t)j * C;
-  const int nv = (int)min((int64_t)C, t1 - tc0);
-  unsigned char* blk = ws + ((size_t)slot * p.H + h) * WB_BYTES;
-  const bool even = (j & 1) == 0;  // operand order within the block's pairs
 
   const uint32_t bar_in = sb + P_BAR, bar_mma = sb + P_BAR + 8;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + P_BAR + 16);
@@ -385,187 +375,218 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_in));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    // q, k and the gate input of the chunk's 64 tokens (rows past the tensor's end read as zeros; rows past
-    // the sequence's end are zeroed below); 64 KB on one barrier.
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_in), "r"(65536) : "memory");
-    const int tt = (int)tc0, bb = (int)brow;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      tma_load_4d(sb + P_QS + half * 8192, &maps.q, 64 * half, h, tt, bb, bar_in);
-      tma_load_4d(sb + P_KS + half * 8192, &maps.k, 64 * half, h, tt, bb, bar_in);
-      tma_load_4d(sb + P_GS + half * 16384, &maps.g, 64 * half, h, tt, bb, bar_in);
-    }
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
                  "r"(P_TM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  float* beta_s = reinterpret_cast<float*>(sm + P_BETA);
-  if (tid < C) {
-    beta_s[tid] = tid < nv ? beta_value(__ldg(p.beta + brow * p.bs[0] + h * p.bs[2] + (tc0 + tid) * p.bs[1]),
-                                        p.beta_sigmoid)
-                           : 0.f;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-
+  float* beta_s = reinterpret_cast<float*>(sm + P_BETA);
   const int c0 = 2 * (tid & 63), da = tid >> 6;
   const int hc = c0 >> 6, cc = c0 & 63;
-  bool ok = __syncthreads_and(mbar_wait(bar_in, 0, &g_split_timeout));
-  int pairwise = 0;
-  int mma_groups = 0;  // product groups committed to bar_mma (thread 0)
-  if (ok) {
-    Prefetch pf;
+
+  // Persistent: the CTA takes items (chunk slot, head) blockIdx.x, + gridDim.x, ... in head-major order.
+  // bar_in completes once per item (phase parity n_done & 1), bar_mma twice (parity 0, then 1).
+  const int64_t n_items = n_slots * p.H;
+  bool ok = true;
+  int n_done = 0;      // items whose inputs were requested
+  int mma_groups = 0;  // product groups of the current item committed to bar_mma (thread 0)
+  for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    const int h = (int)(item / n_slots);
+    const int64_t slot = item - (int64_t)h * n_slots;
+    int n, j;
+    if (!locate_slot(p, slot, n, j)) continue;  // uniform across the CTA
+    const float gsc = MODE >= GATE_LOGITS ? expf(__ldg(p.A_log + h)) : 0.f;  // e^{A_h}
+    int64_t t0, t1, brow;
+    seq_range(p, n, t0, t1, brow);
+    const int64_t tc0 = t0 + (int64_t)j * C;
+    const int nv = (int)min((int64_t)C, t1 - tc0);
+    unsigned char* blk = ws + ((size_t)slot * p.H + h) * WB_BYTES;
+    const bool even = (j & 1) == 0;  // operand order within the block's pairs
+    if (tid == 0) {
+      // q, k and the gate input of the chunk's 64 tokens (rows past the tensor's end read as zeros; rows past
+      // the sequence's end are zeroed below); 64 KB on one barrier. The previous item's readers of this
+      // shared memory are done (the barrier at the end of the item).
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_in), "r"(65536) : "memory");
+      const int tt = (int)tc0, bb = (int)brow;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int t = 16 * da + i;
-      const bool v = t < nv;
-      pf.q[i] = v ? *reinterpret_cast<const uint32_t*>(sm + P_QS + hc * 8192 + t * 128 + cc * 2) : 0u;
-      pf.k[i] = v ? *reinterpret_cast<const uint32_t*>(sm + P_KS + hc * 8192 + t * 128 + cc * 2) : 0u;
-      pf.g[i] = v ? *reinterpret_cast<const float2*>(sm + P_GS + hc * 16384 + t * 256 + cc * 4) : make_float2(0.f, 0.f);
-    }
-    if (p.qk_l2norm) l2norm_qk(pf, reinterpret_cast<float*>(sm + P_VEC) + VEC_D, tid, da);
-    float2 al[16];
-    decay_step1_t<MODE>(sm, LY, pf, nv, da, gsc, p.g_min, load_bias2(p, h, c0), al, c0);
-    __syncthreads();  // block sums and flags published; every input is in registers
-    pairwise = pairwise_blocks(sm, LY);
-    if (pairwise) {  // CTA-uniform; never taken within range
-      if ((pairwise >> da) & 1) {
-        // the prepared inputs of this out-of-range block back into the staging area, alpha over the gate input
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = 16 * da + i;
-          *reinterpret_cast<uint32_t*>(sm + P_QS + hc * 8192 + t * 128 + cc * 2) = pf.q[i];
-          *reinterpret_cast<uint32_t*>(sm + P_KS + hc * 8192 + t * 128 + cc * 2) = pf.k[i];
-          *reinterpret_cast<float2*>(sm + P_GS + hc * 16384 + t * 256 + cc * 4) = al[i];
-        }
+      for (int half = 0; half < 2; ++half) {
+        tma_load_4d(sb + P_QS + half * 8192, &maps.q, 64 * half, h, tt, bb, bar_in);
+        tma_load_4d(sb + P_KS + half * 8192, &maps.k, 64 * half, h, tt, bb, bar_in);
+        tma_load_4d(sb + P_GS + half * 16384, &maps.g, 64 * half, h, tt, bb, bar_in);
       }
+    }
+    if (tid < C) {
+      beta_s[tid] = tid < nv ? beta_value(__ldg(p.beta + brow * p.bs[0] + h * p.bs[2] + (tc0 + tid) * p.bs[1]),
+                                          p.beta_sigmoid)
+                             : 0.f;
+    }
+    ok = __syncthreads_and(mbar_wait(bar_in, n_done & 1, &g_split_timeout));
+    int pairwise = 0;
+    mma_groups = 0;
+    if (ok) {
+      Prefetch pf;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * da + i;
+        const bool v = t < nv;
+        pf.q[i] = v ? *reinterpret_cast<const uint32_t*>(sm + P_QS + hc * 8192 + t * 128 + cc * 2) : 0u;
+        pf.k[i] = v ? *reinterpret_cast<const uint32_t*>(sm + P_KS + hc * 8192 + t * 128 + cc * 2) : 0u;
+        pf.g[i] = v ? *reinterpret_cast<const float2*>(sm + P_GS + hc * 16384 + t * 256 + cc * 4) : make_float2(0.f, 0.f);
+      }
+      if (p.qk_l2norm) l2norm_qk(pf, reinterpret_cast<float*>(sm + P_VEC) + VEC_D, tid, da);
+      float2 al[16];
+      decay_step1_t<MODE>(sm, LY, pf, nv, da, gsc, p.g_min, load_bias2(p, h, c0), al, c0);
+      __syncthreads();  // block sums and flags published; every input is in registers
+      pairwise = pairwise_blocks(sm, LY);
+      if (pairwise) {  // CTA-uniform; never taken within range
+        if ((pairwise >> da) & 1) {
+          // the prepared inputs of this out-of-range block back into the staging area, alpha over the gate input
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int t = 16 * da + i;
+            *reinterpret_cast<uint32_t*>(sm + P_QS + hc * 8192 + t * 128 + cc * 2) = pf.q[i];
+            *reinterpret_cast<uint32_t*>(sm + P_KS + hc * 8192 + t * 128 + cc * 2) = pf.k[i];
+            *reinterpret_cast<float2*>(sm + P_GS + hc * 16384 + t * 256 + cc * 4) = al[i];
+          }
+        }
+        __syncthreads();
+        p_diag_pairwise(sm, pairwise, beta_s, reinterpret_cast<float*>(sm + P_DIAG));
+        __syncthreads();  // the staging area is read; the operands overwrite it next
+      }
+      p_operands(sm, pf, da, c0, pairwise, al, blk + WB_WQ + (even ? 8192 : 0), blk + WB_KA + (even ? 8192 : 0));
+      __syncthreads();  // every block's own view rows and the view scales
+      view_expand(sm, tid);
+      fence_async_smem();
+      tc_fence_before();
       __syncthreads();
-      p_diag_pairwise(sm, pairwise, beta_s, reinterpret_cast<float*>(sm + P_DIAG));
-      __syncthreads();  // the staging area is read; the operands overwrite it next
-    }
-    p_operands(sm, pf, da, c0, pairwise, al, blk + WB_WQ + (even ? 8192 : 0), blk + WB_KA + (even ? 8192 : 0));
-    __syncthreads();  // every block's own view rows and the view scales
-    view_expand(sm, tid);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // ---- the A products: [view 3 | view 0] x [K_3 | Q_3 | K_0 | Q_0], [view 2 | view 1] x [K_2 | Q_2 | K_1 | Q_1]
-    if (tid == 0) {
-      constexpr uint32_t id_a = idesc_bf16(64, 0, 0);
+      tc_fence_after();
+      // ---- the A products: [view 3 | view 0] x [K_3 | Q_3 | K_0 | Q_0], [view 2 | view 1] x [K_2 | Q_2 | K_1 | Q_1]
+      if (tid == 0) {
+        constexpr uint32_t id_a = idesc_bf16(64, 0, 0);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t kv = (ks >> 2) * VIEW_HALF + (ks & 3) * 32, kq = (ks >> 2) * 16384 + (ks & 3) * 32;
-        tc_mma(tmem, sdesc(sb + P_VIEW + kv, 16, 1024), sdesc(sb + P_KQ + kq, 16, 1024), id_a, ks > 0);
-        tc_mma(tmem + 64, sdesc(sb + P_VIEW + 80 * 128 + kv, 16, 1024), sdesc(sb + P_KQ + 64 * 128 + kq, 16, 1024),
-               id_a, ks > 0);
-      }
-      tc_commit(bar_mma);
-      mma_groups = 1;
-    }
-    ok = __syncthreads_and(mbar_wait(bar_mma, 0, &g_split_timeout));
-    tc_fence_after();
-  }
-  if (ok) {
-    // K*gamma_C/Gamma (view 3) goes to the workspace as kernel S's MN-major operand rows [t][c] (when block 3
-    // is out of range the decay pass has stored it already).
-    if (tid == 0 && !((pairwise >> 3) & 1)) {
-      const uint32_t kt = WB_KA + (even ? 8192 : 0);
-      bulk_store(blk + kt, sb + P_VIEW, 8192);
-      bulk_store(blk + kt + 8192, sb + P_VIEW + VIEW_HALF, 8192);
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    }
-    // ---- read back: warps 0-3 the first product, 4-7 the second; TMEM lane L = 32 (warp & 3) + lane is
-    // column i = L & 63 of A in view 3 or 0 (first product) and 2 or 1 (second)
-    {
-      const int L = 32 * (warp & 3) + lane, second = warp >> 2;
-      const int a = second ? (L < 64 ? 2 : 1) : (L < 64 ? 3 : 0);
-      const int i = L & 63;
-      uint32_t r[32];
-      tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * second + (L < 64 ? 0 : 32), r);
-      const bool from_pairs = ((pairwise >> a) & 1) && (i >> 4) == a;
-      const float* dg = reinterpret_cast<const float*>(sm + P_DIAG);
-      float* akk = reinterpret_cast<float*>(sm + P_AKK);
-      float vq[16];
-#pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const int t = 16 * a + jj;
-        float vk = __uint_as_float(r[jj]);
-        vq[jj] = __uint_as_float(r[16 + jj]);
-        if (from_pairs) {
-          vk = dg[(a * 16 + jj) * 16 + (i & 15)];
-          vq[jj] = dg[1024 + (a * 16 + jj) * 16 + (i & 15)];
-        } else {
-          vk = i < t ? vk * beta_s[t] : 0.f;
-          vq[jj] = i <= t ? vq[jj] : 0.f;
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t kv = (ks >> 2) * VIEW_HALF + (ks & 3) * 32, kq = (ks >> 2) * 16384 + (ks & 3) * 32;
+          tc_mma(tmem, sdesc(sb + P_VIEW + kv, 16, 1024), sdesc(sb + P_KQ + kq, 16, 1024), id_a, ks > 0);
+          tc_mma(tmem + 64, sdesc(sb + P_VIEW + 80 * 128 + kv, 16, 1024), sdesc(sb + P_KQ + 64 * 128 + kq, 16, 1024),
+                 id_a, ks > 0);
         }
-        akk[t * 64 + i] = vk;
+        tc_commit(bar_mma);
+        mma_groups = 1;
       }
-      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a, 0)) =
-          make_uint4(pack_bf16(vq[0], vq[1]), pack_bf16(vq[2], vq[3]), pack_bf16(vq[4], vq[5]), pack_bf16(vq[6], vq[7]));
-      *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a + 1, 0)) = make_uint4(
-          pack_bf16(vq[8], vq[9]), pack_bf16(vq[10], vq[11]), pack_bf16(vq[12], vq[13]), pack_bf16(vq[14], vq[15]));
+      ok = __syncthreads_and(mbar_wait(bar_mma, 0, &g_split_timeout));
+      tc_fence_after();
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();  // A_kk and A_qk^T complete
-    if (tid == 0) {
-      bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    }
-    // ---- T' = (I + A_kk)^-1 Diag(beta) on warps 0-3
-    if (warp < 4) inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // ---- W = T' (K*Gamma): A = T' (K-major [t][i], rows 64..127 discarded), B = K*Gamma (MN-major [i][c])
-    if (tid == 0) {
-      constexpr uint32_t id_w = idesc_bf16(128, 0, 1);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        tc_mma(tmem + 128, sdesc(sb + P_TP + ks * 32, 16, 1024), sdesc(sb + P_KG + ks * 2048, 8192, 1024), id_w,
-               ks > 0);
-      tc_commit(bar_mma);
-      mma_groups = 2;
-      bulk_store(blk + WB_TP, sb + P_TP, 8192);
-      bulk_store(blk + WB_GAM, sb + P_GAM, 512);
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    }
-    ok = __syncthreads_and(mbar_wait(bar_mma, 1, &g_split_timeout));
-    tc_fence_after();
-  }
-  if (ok) {
-    // ---- -W to [half][t][c] (warps 0, 1: channels 0-63; warps 4, 5: 64-127), then to the workspace
-    if ((warp & 3) < 2) {
-      const int t = 32 * (warp & 3) + lane, half = warp >> 2;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
+    if (ok) {
+      // K*gamma_C/Gamma (view 3) goes to the workspace as kernel S's MN-major operand rows [t][c] (when block 3
+      // is out of range the decay pass has stored it already).
+      if (tid == 0 && !((pairwise >> 3) & 1)) {
+        const uint32_t kt = WB_KA + (even ? 8192 : 0);
+        bulk_store(blk + kt, sb + P_VIEW, 8192);
+        bulk_store(blk + kt + 8192, sb + P_VIEW + VIEW_HALF, 8192);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+      // ---- read back: warps 0-3 the first product, 4-7 the second; TMEM lane L = 32 (warp & 3) + lane is
+      // column i = L & 63 of A in view 3 or 0 (first product) and 2 or 1 (second)
+      {
+        const int L = 32 * (warp & 3) + lane, second = warp >> 2;
+        const int a = second ? (L < 64 ? 2 : 1) : (L < 64 ? 3 : 0);
+        const int i = L & 63;
         uint32_t r[32];
-        tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 128 + 64 * half + 32 * part, r);
+        tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * second + (L < 64 ? 0 : 32), r);
+        const bool from_pairs = ((pairwise >> a) & 1) && (i >> 4) == a;
+        const float* dg = reinterpret_cast<const float*>(sm + P_DIAG);
+        float* akk = reinterpret_cast<float*>(sm + P_AKK);
+        float vq[16];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          *reinterpret_cast<uint4*>(sm + P_W + half * 8192 + sw_chunk(t, 4 * part + q4, 0)) = pack8(r, q4, -1.f);
+        for (int jj = 0; jj < 16; ++jj) {
+          const int t = 16 * a + jj;
+          float vk = __uint_as_float(r[jj]);
+          vq[jj] = __uint_as_float(r[16 + jj]);
+          if (from_pairs) {
+            vk = dg[(a * 16 + jj) * 16 + (i & 15)];
+            vq[jj] = dg[1024 + (a * 16 + jj) * 16 + (i & 15)];
+          } else {
+            vk = i < t ? vk * beta_s[t] : 0.f;
+            vq[jj] = i <= t ? vq[jj] : 0.f;
+          }
+          akk[t * 64 + i] = vk;
+        }
+        *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a, 0)) =
+            make_uint4(pack_bf16(vq[0], vq[1]), pack_bf16(vq[2], vq[3]), pack_bf16(vq[4], vq[5]), pack_bf16(vq[6], vq[7]));
+        *reinterpret_cast<uint4*>(sm + P_AQKT + sw_chunk(i, 2 * a + 1, 0)) = make_uint4(
+            pack_bf16(vq[8], vq[9]), pack_bf16(vq[10], vq[11]), pack_bf16(vq[12], vq[13]), pack_bf16(vq[14], vq[15]));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();  // A_kk and A_qk^T complete
+      if (tid == 0) {
+        bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+      // ---- T' = (I + A_kk)^-1 Diag(beta) on warps 0-3
+      if (warp < 4) inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      // ---- W = T' (K*Gamma): A = T' (K-major [t][i], rows 64..127 discarded), B = K*Gamma (MN-major [i][c])
+      if (tid == 0) {
+        constexpr uint32_t id_w = idesc_bf16(128, 0, 1);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          tc_mma(tmem + 128, sdesc(sb + P_TP + ks * 32, 16, 1024), sdesc(sb + P_KG + ks * 2048, 8192, 1024), id_w,
+                 ks > 0);
+        tc_commit(bar_mma);
+        mma_groups = 2;
+        bulk_store(blk + WB_TP, sb + P_TP, 8192);
+        bulk_store(blk + WB_GAM, sb + P_GAM, 512);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+      ok = __syncthreads_and(mbar_wait(bar_mma, 1, &g_split_timeout));
+      tc_fence_after();
+    }
+    if (ok) {
+      // ---- -W to [half][t][c] (warps 0, 1: channels 0-63; warps 4, 5: 64-127), then to the workspace
+      if ((warp & 3) < 2) {
+        const int t = 32 * (warp & 3) + lane, half = warp >> 2;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          uint32_t r[32];
+          tm_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 128 + 64 * half + 32 * part, r);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(sm + P_W + half * 8192 + sw_chunk(t, 4 * part + q4, 0)) = pack8(r, q4, -1.f);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        const uint32_t wq = even ? 0 : 8192;
+        bulk_store(blk + WB_WQ + wq, sb + P_W, 8192);
+        bulk_store(blk + WB_WQ + 16384 + wq, sb + P_W + 8192, 8192);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
     }
+    if (!ok) break;
+    // The stores have read their shared memory, and every thread's generic writes are ordered before the
+    // next item's TMA writes: the shared memory and TMEM are free for the next item.
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-      const uint32_t wq = even ? 0 : 8192;
-      bulk_store(blk + WB_WQ + wq, sb + P_W, 8192);
-      bulk_store(blk + WB_WQ + 16384 + wq, sb + P_W + 8192, 8192);
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    }
+    tc_fence_after();
+    ++n_done;
   }
   if (tid == 0) {
     if (!ok) {
       // A wait expired: give the loads and products that may still be in flight a bounded wait.
-      mbar_wait(bar_in, 0, &g_split_timeout);
+      mbar_wait(bar_in, n_done & 1, &g_split_timeout);
       if (mma_groups >= 1) mbar_wait(bar_mma, 0, &g_split_timeout);
       if (mma_groups >= 2) mbar_wait(bar_mma, 1, &g_split_timeout);
     }
@@ -717,7 +738,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     tc_fence_after();
     if (!ok) break;
 
-    // S^T -> its bf16 copy (group A's operand) and S^T *= gamma_C in place (group B accumulates on it).
+    // U^T = V^T T'^T needs no state: the tensor pipe runs it while the state is converted. (U's buffer was
+    // last read by chunk c-2's conversion.)
+    if (tid == 0) {
+      constexpr uint32_t id_vt = idesc_bf16(64, 1, 0);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        tc_mma(tmem + tm_u, sdesc(vbuf + ks * 2048, 8192, 1024), sdesc(ops + WB_TP + ks * 32, 16, 1024), id_vt, ks > 0);
+    }
+
+    // S^T -> its bf16 copy (group A's operand), S^T *= gamma_C in place (group B accumulates on it), and this
+    // chunk's O^T = 0 (group A accumulates on it; chunk c-2's output was read from that buffer in chunk c-1).
     {
       const float* gam = reinterpret_cast<const float*>(opsp + WB_GAM);
 #pragma unroll
@@ -738,6 +769,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
         }
         tm_st32(tlane + TM_S + cb, r);
       }
+      uint32_t z[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) z[jj] = 0u;
+      tm_st32(tlane + (buf ? TM_OO : TM_OE) + 32 * half, z);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
@@ -747,17 +782,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     // Chunk c-1's group B is done: the other buffer's part 2 takes chunk c+1's.
     if (tid == 0 && c + 1 < n_chunks) load_part2(c + 1, buf ^ 1);
 
-    // ---- group A: [U^T | O^T] = S^T [-W ; Q*Gamma]^T, then U^T += V^T T'^T ---------------------------
+    // ---- group A: [U^T | O^T] += S^T [-W ; Q*Gamma]^T ---------------------------------------------------
     if (tid == 0) {
-      constexpr uint32_t id_wq = idesc_bf16(128, 0, 0), id_vt = idesc_bf16(64, 1, 0);
+      constexpr uint32_t id_wq = idesc_bf16(128, 0, 0);
       const uint32_t d_a = buf ? TM_OO : TM_UE;  // [U_e | O_e] or [O_o | U_o]
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         tc_mma_ts(tmem + d_a, tmem + TM_SB + 8 * ks, sdesc(ops + WB_WQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                  id_wq, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        tc_mma(tmem + tm_u, sdesc(vbuf + ks * 2048, 8192, 1024), sdesc(ops + WB_TP + ks * 32, 16, 1024), id_vt, 1);
+                  id_wq, 1);
       tc_commit(bar_mma);
     }
     // meanwhile: the previous chunk's output
@@ -766,13 +798,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     ok = __syncthreads_and(mbar_wait(bar_mma, 0, &g_split_timeout));
     tc_fence_after();
     if (!ok) break;
-
-    // Group A is done with this buffer's part 1 and v tile: refill them with chunk c+2's.
-    if (c + 2 < n_chunks) {
-      if (tid == 0) load_part1(c + 2, buf);
-      load_v(x, vbuf, tc0 + 2 * C, (int)min((int64_t)C, t1 - tc0 - 2 * C), tid);
-    }
-    cp_async_commit();
 
     // ---- U^T -> its bf16 copy ---------------------------------------------------------------------
     {
@@ -797,6 +822,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
         tc_mma_ts(tmem + d_b, tmem + TM_UB + 8 * ks, sdesc(ops + WB_KA + ks * 2048, 8192, 1024), id_b, 1);
       tc_commit(bar_mma);
     }
+    // Group A was done with this buffer's part 1 and v tile: refill them with chunk c+2's while group B runs.
+    if (c + 2 < n_chunks) {
+      if (tid == 0) load_part1(c + 2, buf);
+      load_v(x, vbuf, tc0 + 2 * C, (int)min((int64_t)C, t1 - tc0 - 2 * C), tid);
+    }
+    cp_async_commit();
   }
   // The last chunk's group B, then its output.
   if (ok && n_chunks > 0) {
@@ -927,8 +958,14 @@ cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
       !token_map(&maps.k, p.k, true, p.ks, p.B, p.T, p.H, p.K) ||
       !token_map(&maps.g, p.gate, false, p.gs, p.B, p.T, p.H, p.K))
     return cudaErrorInvalidValue;  // callers check split_maps_ok first
-  dim3 gp((unsigned)slots, (unsigned)p.H);
-  intra<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws), maps);
+  // Persistent kernel P: two CTAs per SM (its shared memory and registers allow two), each walking the items.
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t items = slots * p.H;
+  const unsigned gp = (unsigned)std::min<int64_t>(items, 2 * (int64_t)std::max(sms, 1));
+  intra<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws), maps, slots);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t grid = (int64_t)p.N * p.H * (p.V / VT);
