@@ -88,21 +88,21 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 # dram__bytes_write.sum of every kernel the step launches). They hold only for the kernel sources they were
 # taken on, so the sources' sha256 is kept beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
-    # chunk_intra_kernel<2> 404.6 + 359.1 MB; chunk_state_kernel 506.5 + 84.7 MB
-    "prefill": {"bytes": 1354900000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
+    # chunk_intra_kernel<2> 404.5 + 356.9 MB; chunk_state_kernel 506.6 + 84.1 MB
+    "prefill": {"bytes": 1352000000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
     # decode_bulk_kernel 410.6 + 345.1 MB
     "decode": {"bytes": 755700000, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                "sha256": "ef9a4cbaa38adbffc745f72fc725ecb508aa04553436b13be7ca12ae07b738db"},
-    # chunk_intra_kernel<3> 405.0 + 359.0 MB; chunk_state_kernel 506.5 + 84.2 MB (the unbounded gate's prefill)
-    "softplus": {"bytes": 1354700000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
-    # chunk_intra_kernel<2> 8,102.6 + 7,283.6 MB; chunk_state_kernel 9,227.4 + 1,885.2 MB (16 packed sequences)
-    "varlen": {"bytes": 26498800000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
-    # chunk_intra_kernel<2> 2,407.4 + 2,121.2 MB; chunk_state_kernel 3,254.9 + 1,060.3 MB (4 x 16384 x 32, V = 256)
-    "long_kv": {"bytes": 8843800000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "a8f2f638fa6f8db09c8ea233d4fd6a53ab47239d6e637e5d924838b2e54363bf"},
+    # chunk_intra_kernel<3> 405.3 + 358.1 MB; chunk_state_kernel 506.6 + 84.3 MB (the unbounded gate's prefill)
+    "softplus": {"bytes": 1354200000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                 "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
+    # chunk_intra_kernel<2> 8,011.5 + 7,279.2 MB; chunk_state_kernel 9,227.4 + 1,885.2 MB (16 packed sequences)
+    "varlen": {"bytes": 26403300000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
+    # chunk_intra_kernel<2> 2,389.6 + 2,118.3 MB; chunk_state_kernel 3,254.9 + 1,059.5 MB (4 x 16384 x 32, V = 256)
+    "long_kv": {"bytes": 8822300000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
     # bounded_decay_kernel 201,388,032 + 154,186,496; scan_backward_kernel 17,959,960,832 + 27,343,060,992;
     # bounded_decay_backward_kernel 402,712,832 + 162,471,424 (one backward step from the logits)
     "backward": {"bytes": 46223780608, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],

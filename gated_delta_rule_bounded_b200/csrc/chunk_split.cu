@@ -29,6 +29,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstring>
 
 #include "chunk_common.cuh"
 
@@ -90,10 +91,11 @@ constexpr int S_OPS = 0;                    // 2 x operand block (66048 B, padde
 constexpr int S_OPS_STRIDE = 66560;
 constexpr int S_V = 2 * S_OPS_STRIDE;       // 2 x 16K v tile [i][v], two halves (MN-major A)
 constexpr int S_BAR = S_V + 2 * 16384;      // mbarriers: part 1 x2, part 2 x2, mma; TMEM base
-constexpr int S_SMEM = S_BAR + 64;
+constexpr int S_OST = S_BAR + 1024;          // 2 x 16K output staging [64 tokens][128 values] bf16 (TMA store)
+constexpr int S_SMEM = S_OST + 2 * 16384;
 static_assert(S_SMEM <= 227 * 1024, "shared memory budget");
 static_assert(WB_KA % 16 == 0 && WB_TP % 16 == 0 && WB_BYTES % 16 == 0, "bulk copies move 16-byte multiples");
-static_assert(S_V % 1024 == 0 && S_OPS_STRIDE % 1024 == 0, "swizzle atoms need 1 KB alignment");
+static_assert(S_V % 1024 == 0 && S_OPS_STRIDE % 1024 == 0 && S_OST % 1024 == 0, "1 KB alignment");
 
 // Kernel S tensor memory (columns; lane = value column v of the tile). S^T, U^T and O^T in fp32 are
 // MMA accumulators, laid out [U_e | O_e | S | O_o | U_o] so that [U | O] and [O | S] are adjacent for
@@ -607,6 +609,25 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int x, int h, int t, int b) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(h), "r"(t), "r"(b), "r"(src)
+               : "memory");
+}
+
+// O^T of one full chunk (TMEM columns [tm_o, tm_o + 64)) into the staging tile [t][v] (bf16, 256-byte rows):
+// this thread's lane v, tokens 32*half... Ends with the proxy fence that orders these writes before the TMA
+// store that reads them (issued after the next barrier).
+__device__ __forceinline__ void stage_o(unsigned char* st, uint32_t tlane, uint32_t tm_o, int trow, int half) {
+  uint32_t r[32];
+  tm_ld32(tlane + tm_o + 32 * half, r);
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(st) + (32 * half) * VT + trow;
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) dst[jj * VT] = __float2bfloat16_rn(__uint_as_float(r[jj]));
+  fence_async_smem();
+}
+
 // O^T of one chunk (TMEM columns [tm_o, tm_o + 64)) to o: this thread's lane v, tokens 32*half...
 __device__ __forceinline__ void store_o(const ScanParams& p, uint32_t tlane, uint32_t tm_o, int64_t brow, int h, int vt,
                                        int trow, int half, int64_t tc0, int nv) {
@@ -623,7 +644,9 @@ __device__ __forceinline__ void store_o(const ScanParams& p, uint32_t tlane, uin
   }
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, const unsigned char* ws) {
+__global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, const unsigned char* ws,
+                                                                  const __grid_constant__ CUtensorMap omap,
+                                                                  int use_omap) {
   extern __shared__ __align__(1024) unsigned char sm[];
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -729,6 +752,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     const uint32_t vbuf = sb + S_V + buf * 16384;
     const uint32_t tm_u = buf ? TM_UO : TM_UE;
 
+    // The output staging buffer this chunk fills was read by the store of chunk c-3 (at most the store of chunk
+    // c-2 stays in flight).
+    if (tid == 0 && use_omap) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
     // The previous chunk's group B is done (TMEM S^T holds S_{c-1}); this chunk's part 1 and v have landed.
     bool w = c == 0 || mbar_wait(bar_mma, 1, &g_split_timeout);
     w = w && mbar_wait(bar_p1 + 8 * buf, (c >> 1) & 1, &g_split_timeout);
@@ -792,12 +818,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
                   id_wq, 1);
       tc_commit(bar_mma);
     }
-    // meanwhile: the previous chunk's output
-    if (c > 0) store_o(p, tlane, buf ? TM_OE : TM_OO, brow, h, vt, trow, half, tc0 - C, C);
+    // meanwhile: the previous chunk's output, staged in shared memory for one TMA store (or stored directly)
+    if (c > 0) {
+      if (use_omap)
+        stage_o(sm + S_OST + ((c - 1) & 1) * 16384, tlane, buf ? TM_OE : TM_OO, trow, half);
+      else
+        store_o(p, tlane, buf ? TM_OE : TM_OO, brow, h, vt, trow, half, tc0 - C, C);
+    }
 
     ok = __syncthreads_and(mbar_wait(bar_mma, 0, &g_split_timeout));
     tc_fence_after();
     if (!ok) break;
+    if (tid == 0 && use_omap && c > 0) {  // the staged output of chunk c-1: [64 tokens][128 values] bf16
+      tma_store_4d(&omap, sb + S_OST + ((c - 1) & 1) * 16384, vt * VT, h, (int)(tc0 - C), (int)brow);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
 
     // ---- U^T -> its bf16 copy ---------------------------------------------------------------------
     {
@@ -839,6 +874,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
     }
   }
   cp_async_wait_all();
+  if (tid == 0 && use_omap) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -934,6 +970,24 @@ bool token_map(CUtensorMap* m, const void* base, bool bf16, const int64_t s[3], 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The bf16 output o [B,T,H,V] (element strides s = (b, t, h)) as a 4-d tensor map (V, H, T, B) written in
+// boxes of 128 values x 64 tokens of one head (kernel S's tile of one chunk). False when the driver refuses the
+// layout (kernel S then stores o directly).
+bool out_map(CUtensorMap* m, void* base, const int64_t s[3], int64_t B, int64_t T, int64_t H, int64_t V) {
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const int64_t sh = H > 1 ? s[2] : V;
+  const int64_t st = T > 1 ? s[1] : H * sh;
+  const int64_t sbt = B > 1 ? s[0] : T * st;
+  const cuuint64_t dims[4] = {(cuuint64_t)V, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(st * 2), (cuuint64_t)(sbt * 2)};
+  const cuuint32_t box[4] = {(cuuint32_t)VT, 1, (cuuint32_t)C, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool split_maps_ok(const ScanParams& p) {
@@ -958,13 +1012,18 @@ cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
       !token_map(&maps.k, p.k, true, p.ks, p.B, p.T, p.H, p.K) ||
       !token_map(&maps.g, p.gate, false, p.gs, p.B, p.T, p.H, p.K))
     return cudaErrorInvalidValue;  // callers check split_maps_ok first
-  // Persistent kernel P: two CTAs per SM (its shared memory and registers allow two), each walking the items.
+  // Kernel P persistent: two CTAs per SM (its shared memory and registers allow two), each walking the items
+  // with a fixed stride. The unbounded gate's items differ in cost (pairwise diagonal tiles where the decay is
+  // steep, which depends on the head), so there each CTA takes one item and the hardware balances the load.
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int64_t items = slots * p.H;
-  const unsigned gp = (unsigned)std::min<int64_t>(items, 2 * (int64_t)std::max(sms, 1));
+  if (items > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  const unsigned gp = p.gate_mode == GATE_SOFTPLUS
+                          ? (unsigned)items
+                          : (unsigned)std::min<int64_t>(items, 2 * (int64_t)std::max(sms, 1));
   intra<<<gp, NTHREADS, P_SMEM, s>>>(p, static_cast<unsigned char*>(ws), maps, slots);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -981,7 +1040,10 @@ cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, chunk_state_kernel, p, static_cast<const unsigned char*>(ws));
+  CUtensorMap omap;
+  std::memset(&omap, 0, sizeof(omap));
+  const int use_omap = out_map(&omap, p.o, p.os, p.B, p.T, p.H, p.V) ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, chunk_state_kernel, p, static_cast<const unsigned char*>(ws), omap, use_omap);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
