@@ -103,10 +103,10 @@ MEASURED_TRAFFIC = {
     # chunk_intra_kernel<2> 2,389.6 + 2,118.3 MB; chunk_state_kernel 3,254.9 + 1,059.5 MB (4 x 16384 x 32, V = 256)
     "long_kv": {"bytes": 8822300000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                 "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
-    # bounded_decay_kernel 201,388,032 + 154,186,496; scan_backward_kernel 17,959,960,832 + 27,343,060,992;
-    # bounded_decay_backward_kernel 402,712,832 + 162,471,424 (one backward step from the logits)
-    "backward": {"bytes": 46223780608, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "4e128306fa88fbe43e6de95d747168e1ba8523f2254c7b9a3a2c8d1c262d07b2"},
+    # bounded_decay_kernel 201,369,600 + 154,498,560; scan_backward_kernel 17,579,054,336 + 27,342,757,376;
+    # bounded_decay_backward_kernel 402,670,080 + 162,126,848 (one backward step from the logits)
+    "backward": {"bytes": 45842476800, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                 "sha256": "973813a4f2667f3e3d31825a179fb55c0a23896f4225ad466630a1dc660d4422"},
 }
 
 
