@@ -88,21 +88,21 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 # dram__bytes_write.sum of every kernel the step launches). They hold only for the kernel sources they were
 # taken on, so the sources' sha256 is kept beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
-    # chunk_intra_kernel<2> 404.5 + 356.9 MB; chunk_state_kernel 506.6 + 84.1 MB
-    "prefill": {"bytes": 1352000000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
+    # chunk_intra_kernel<2> 404.4 + 356.9 MB; chunk_state_kernel 506.6 + 84.2 MB
+    "prefill": {"bytes": 1352100000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+              "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
     # decode_bulk_kernel 410.6 + 345.1 MB
     "decode": {"bytes": 755700000, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                "sha256": "ef9a4cbaa38adbffc745f72fc725ecb508aa04553436b13be7ca12ae07b738db"},
-    # chunk_intra_kernel<3> 405.3 + 358.1 MB; chunk_state_kernel 506.6 + 84.3 MB (the unbounded gate's prefill)
-    "softplus": {"bytes": 1354200000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
-    # chunk_intra_kernel<2> 8,011.5 + 7,279.2 MB; chunk_state_kernel 9,227.4 + 1,885.2 MB (16 packed sequences)
-    "varlen": {"bytes": 26403300000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
-    # chunk_intra_kernel<2> 2,389.6 + 2,118.3 MB; chunk_state_kernel 3,254.9 + 1,059.5 MB (4 x 16384 x 32, V = 256)
-    "long_kv": {"bytes": 8822300000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                "sha256": "965ded3181a24593e11e8d42503c95887a0f29d39888b73290457b33a26326c8"},
+    # chunk_intra_kernel<3> 404.9 + 357.6 MB; chunk_state_kernel 506.6 + 83.6 MB (the unbounded gate's prefill)
+    "softplus": {"bytes": 1352700000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
+    # chunk_intra_kernel<2> 8,000.5 + 7,279.4 MB; chunk_state_kernel 9,227.3 + 1,884.0 MB (16 packed sequences)
+    "varlen": {"bytes": 26391200000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+             "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
+    # chunk_intra_kernel<2> 2,391.2 + 2,118.9 MB; chunk_state_kernel 3,261.1 + 1,060.8 MB (4 x 16384 x 32, V = 256)
+    "long_kv": {"bytes": 8832000000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+              "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
     # bounded_decay_kernel 201,369,600 + 154,498,560; scan_backward_kernel 17,579,054,336 + 27,342,757,376;
     # bounded_decay_backward_kernel 402,670,080 + 162,126,848 (one backward step from the logits)
     "backward": {"bytes": 45842476800, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
@@ -303,6 +303,52 @@ def timed_loop(step_fns, steps, warmup, world, stream, sampler=None):
     return total, per_fn
 
 
+def pipelined_e2e(host_in, dev_in, host_out, dev_out, run_fn, steps, warmup, world):
+    """End-to-end steps through the public API, as a serving loop runs them: each step copies its inputs from
+    pinned host memory to the device, calls the library and copies its results back to pinned host memory,
+    with the three stages of consecutive steps overlapped on three streams (step i's inputs come in while step
+    i-1 computes and step i-2's results go out). Inputs and outputs are double-buffered: dev_in and dev_out are
+    two dicts each; run_fn(inputs, outputs) launches on the current stream (the computes run in order on one
+    stream). host_in is a dict of pinned tensors, or a list of such dicts taken in turn. Returns the total ms
+    over `steps` (first input copy to last result copy, CUDA events)."""
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    n = warmup + steps
+    ev = {k: [torch.cuda.Event() for _ in range(n)] for k in ("in", "cmp", "out")}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(n):
+        if i == warmup:
+            torch.cuda.synchronize()
+            start.record(s_in)
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev["cmp"][i - 2])  # step i-2 has read these input buffers
+            src = host_in[i % len(host_in)] if isinstance(host_in, list) else host_in
+            for name, x in src.items():
+                dev_in[b][name].copy_(x, non_blocking=True)
+            ev["in"][i].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev["in"][i])
+            if i >= 2:
+                s_cmp.wait_event(ev["out"][i - 2])  # step i-2's results have left these output buffers
+            run_fn(dev_in[b], dev_out[b])
+            ev["cmp"][i].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["cmp"][i])
+            for name, x in host_out.items():
+                x.copy_(dev_out[b][name], non_blocking=True)
+            ev["out"][i].record(s_out)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cmp)
+    end.record(s_out)
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end)
+
+
 class _Null:
     def __enter__(self):
         return self
@@ -347,24 +393,22 @@ def prefill_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src):
     }
     if args.no_e2e:
         return res
-    # e2e: pinned host inputs -> device, prefill from logits, o and final state -> pinned host
+    # e2e: pinned host inputs -> device, prefill from logits, o and final state -> pinned host, consecutive
+    # steps overlapped (the inputs of one step copy in while the previous step computes)
     host = {n: d[n].pin_memory() for n in ("q", "k", "v", "z", "A_log", "beta")}
-    o_host = torch.empty(B, T, H, V, dtype=torch.bfloat16).pin_memory()
-    sf_host = torch.empty(B, H, K, V, dtype=torch.float32).pin_memory()
-    dev_in = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
+    host_out = {"o": torch.empty(B, T, H, V, dtype=torch.bfloat16).pin_memory(),
+                "sf": torch.empty(B, H, K, V, dtype=torch.float32).pin_memory()}
+    dev_in = [{n: torch.empty_like(x, device=dev) for n, x in host.items()} for _ in range(2)]
+    dev_out = [{"o": o, "sf": sf}, {"o": torch.empty_like(o), "sf": torch.empty_like(sf)}]
     h2d = sum(x.numel() * x.element_size() for x in host.values())
-    d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * sf_host.element_size()
+    d2h = sum(x.numel() * x.element_size() for x in host_out.values())
 
-    def e2e_fn():
-        for n, x in host.items():
-            dev_in[n].copy_(x, non_blocking=True)
-        kda.prefill_logits(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["z"], dev_in["A_log"], w.g_min,
-                           dev_in["beta"], None, out=o, final_state=sf, workspace=ws)
-        o_host.copy_(o, non_blocking=True)
-        sf_host.copy_(sf, non_blocking=True)
+    def run(i, out):
+        kda.prefill_logits(i["q"], i["k"], i["v"], i["z"], i["A_log"], w.g_min, i["beta"], None, out=out["o"],
+                           final_state=out["sf"], workspace=ws)  # computes run in order on one stream
 
     e2e_steps = max(3, min(args.steps, 10))
-    e2e_total, _ = timed_loop([e2e_fn], e2e_steps, max(1, args.warmup // 2), world, stream)
+    e2e_total = pipelined_e2e(host, dev_in, host_out, dev_out, run, e2e_steps, max(1, args.warmup // 2), world)
     e2e_total = max_over_ranks(e2e_total, world)
     res["e2e"] = {"value": tokens / (e2e_total / e2e_steps / 1e3), "unit": "tokens/s",
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
@@ -444,23 +488,19 @@ def workload_leg(args, kda, dev, stream, rank, world, hbm, bf16_peak, peak_src, 
     if not args.no_e2e:
         names = ("q", "k", "v", "z", "A_log", "beta", "initial_state")
         host = {n: d[n].pin_memory() for n in names}
-        o_host = torch.empty(B, T, H, V, dtype=torch.bfloat16).pin_memory()
-        sf_host = torch.empty(N, H, K, V, dtype=torch.float32).pin_memory()
-        dev_in = {n: torch.empty_like(x, device=dev) for n, x in host.items()}
+        host_out = {"o": torch.empty(B, T, H, V, dtype=torch.bfloat16).pin_memory(),
+                    "sf": torch.empty(N, H, K, V, dtype=torch.float32).pin_memory()}
+        dev_in = [{n: torch.empty_like(x, device=dev) for n, x in host.items()} for _ in range(2)]
+        dev_out = [{"o": o, "sf": sf}, {"o": torch.empty_like(o), "sf": torch.empty_like(sf)}]
         h2d = sum(x.numel() * x.element_size() for x in host.values())
-        d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * sf_host.element_size()
+        d2h = sum(x.numel() * x.element_size() for x in host_out.values())
 
-        def e2e_fn():
-            for n, x in host.items():
-                dev_in[n].copy_(x, non_blocking=True)
-            kda.prefill_logits(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["z"], dev_in["A_log"], w.g_min,
-                               dev_in["beta"], dev_in["initial_state"], g["cu_seqlens"], out=o, final_state=sf,
-                               workspace=ws)
-            o_host.copy_(o, non_blocking=True)
-            sf_host.copy_(sf, non_blocking=True)
+        def run(i, out):
+            kda.prefill_logits(i["q"], i["k"], i["v"], i["z"], i["A_log"], w.g_min, i["beta"], i["initial_state"],
+                               g["cu_seqlens"], out=out["o"], final_state=out["sf"], workspace=ws)
 
         e2e_steps = 3
-        e2e_total, _ = timed_loop([e2e_fn], e2e_steps, 1, world, stream)
+        e2e_total = pipelined_e2e(host, dev_in, host_out, dev_out, run, e2e_steps, 1, world)
         e2e_total = max_over_ranks(e2e_total, world)
         res["e2e"] = {"value": B * T * world / (e2e_total / e2e_steps / 1e3), "unit": "tokens/s",
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
@@ -576,22 +616,19 @@ def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
     }
     if args.no_e2e:
         return res
+    # e2e: each step's q, k, v, z, beta from pinned host memory, the step on the kept state, o back to the host;
+    # consecutive steps overlapped (the state update itself stays in order on one stream)
     hostd = [{n: x.pin_memory() for n, x in W.make_decode_step(dw, s).items()} for s in range(n_sets)]
-    devd = {n: torch.empty_like(x, device=dev) for n, x in hostd[0].items()}
-    o_dec_host = torch.empty(dw.B, dw.H, dw.V, dtype=torch.bfloat16).pin_memory()
+    devd = [{n: torch.empty_like(x, device=dev) for n, x in hostd[0].items()} for _ in range(2)]
+    host_out = {"o": torch.empty(dw.B, dw.H, dw.V, dtype=torch.bfloat16).pin_memory()}
+    dev_out = [{"o": o_dec}, {"o": torch.empty_like(o_dec)}]
     dh2d = sum(x.numel() * x.element_size() for x in hostd[0].values())
-    dd2h = o_dec_host.numel() * o_dec_host.element_size()
+    dd2h = host_out["o"].numel() * host_out["o"].element_size()
 
-    def de2e_fn():
-        s = hostd[it["i"] % n_sets]
-        for n, x in s.items():
-            devd[n].copy_(x, non_blocking=True)
-        kda.decode_step_logits(devd["q"], devd["k"], devd["v"], devd["z"], A_dec, dw.g_min, devd["beta"], state,
-                               out=o_dec)
-        o_dec_host.copy_(o_dec, non_blocking=True)
-        it["i"] += 1
+    def drun(i, out):
+        kda.decode_step_logits(i["q"], i["k"], i["v"], i["z"], A_dec, dw.g_min, i["beta"], state, out=out["o"])
 
-    de_total, _ = timed_loop([de2e_fn], dsteps, args.warmup, world, stream)
+    de_total = pipelined_e2e(hostd, devd, host_out, dev_out, drun, dsteps, args.warmup, world)
     de_total = max_over_ranks(de_total, world)
     res["e2e"] = {"value": sbytes * world / (de_total / dsteps / 1e3) / 1e9, "unit": "GB/s (state)",
                   "h2d_bytes_per_step": dh2d, "d2h_bytes_per_step": dd2h}
