@@ -86,41 +86,54 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 
 # DRAM bytes (read + write) per launch of each step, from one ncu capture of its kernels (dram__bytes_read.sum +
 # dram__bytes_write.sum of every kernel the step launches). They hold only for the kernel sources they were
-# taken on, so the sources' sha256 is kept beside them and a mismatch at run time reports null.
+# taken on, so a sha256 of those sources (comments and blank space left out, see source_digest) is kept
+# beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
     # chunk_intra_kernel<2> 404.4 + 356.9 MB; chunk_state_kernel 506.6 + 84.2 MB
     "prefill": {"bytes": 1352100000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-              "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
+              "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
     # decode_bulk_kernel 410.6 + 345.1 MB
     "decode": {"bytes": 755700000, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "ef9a4cbaa38adbffc745f72fc725ecb508aa04553436b13be7ca12ae07b738db"},
+               "sha256": "dfbe3ca4ed44294f1662b85f4506abe22c32c93ea6d7e42319af3c3e7838c5a7"},
     # chunk_intra_kernel<3> 404.9 + 357.6 MB; chunk_state_kernel 506.6 + 83.6 MB (the unbounded gate's prefill)
     "softplus": {"bytes": 1352700000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
+               "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
     # chunk_intra_kernel<2> 8,000.5 + 7,279.4 MB; chunk_state_kernel 9,227.3 + 1,884.0 MB (16 packed sequences)
     "varlen": {"bytes": 26391200000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-             "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
+             "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
     # chunk_intra_kernel<2> 2,391.2 + 2,118.9 MB; chunk_state_kernel 3,261.1 + 1,060.8 MB (4 x 16384 x 32, V = 256)
     "long_kv": {"bytes": 8832000000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-              "sha256": "7e0fc0ddaeba0356a00d2a766b48aadd8176c264008ff97c11e17388a1517651"},
+              "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
     # bounded_decay_kernel 201,369,600 + 154,498,560; scan_backward_kernel 17,579,054,336 + 27,342,757,376;
     # bounded_decay_backward_kernel 402,670,080 + 162,126,848 (one backward step from the logits)
     "backward": {"bytes": 45842476800, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "973813a4f2667f3e3d31825a179fb55c0a23896f4225ad466630a1dc660d4422"},
+                 "sha256": "ed75416944f1f8207064b753d2b529c5b25435b1d8b265a27c5ae9c9afbf9d23"},
 }
 
 
-def measured_traffic(step: str):
+def source_digest(files) -> str:
+    """sha256 of the kernel sources with their comments and blank space removed, so that a change of comments
+    alone keeps a measurement taken on the same code."""
     import hashlib
-    m = MEASURED_TRAFFIC[step]
+    import re
     h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "gated_delta_rule_bounded_b200", "csrc", f), "rb") as fh:
+            text = fh.read().decode()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = (" ".join(line.split()) for line in text.splitlines())
+        h.update("\n".join(line for line in lines if line).encode())
+    return h.hexdigest()
+
+
+def measured_traffic(step: str):
+    m = MEASURED_TRAFFIC[step]
     try:
-        for f in m["files"]:
-            with open(os.path.join(ROOT, "gated_delta_rule_bounded_b200", "csrc", f), "rb") as fh:
-                h.update(fh.read())
+        digest = source_digest(m["files"])
     except OSError:
         return None
-    return m["bytes"] if h.hexdigest() == m["sha256"] else None
+    return m["bytes"] if digest == m["sha256"] else None
 
 
 # ------------------------------------------------------------------------------------------------

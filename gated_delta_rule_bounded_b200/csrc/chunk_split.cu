@@ -5,15 +5,16 @@
 // the decay factors, A_qk and A_kk, T' = (I + A_kk)^-1 Diag(beta), W = T' (K*Gamma), Q*Gamma and
 // K*gamma_C/Gamma -- are most of the arithmetic. In the fused kernel (chunk.cu) they sit on the
 // sequential path of one CTA per (sequence, head). Here kernel P computes them for all chunks of all
-// heads at once, one CTA per (chunk, head) over every SM, and writes each chunk's operand set as
-// one 66,048-byte block to a workspace: the block is the exact image of the shared-memory tiles
-// (128-byte swizzle included), so kernel S moves it with a single bulk copy into a 1 KB-aligned
-// buffer and feeds it straight to tcgen05. Kernel S keeps one CTA per (sequence, head, V-tile) with
-// the transposed state S^T in TMEM and runs two MMA groups per chunk:
-//   group A:  [U^T | O^T] = S^T [-W ; Q*Gamma]^T  (one N = 128 product),  U^T += V^T T'^T
+// heads at once -- a persistent grid of two CTAs per SM walking the (chunk, head) items -- and writes
+// each chunk's operand set as one 66,048-byte block to a workspace: the block is the exact image of the
+// shared-memory tiles (128-byte swizzle included), so kernel S moves it with bulk copies (in two parts,
+// fetched ahead) into a 1 KB-aligned buffer and feeds it straight to tcgen05. Kernel S keeps one CTA per
+// (sequence, head, V-tile) with the transposed state S^T in TMEM and, per chunk:
+//   U^T = V^T T'^T (no state needed: runs while the state is converted to bf16 and rescaled)
+//   group A:  [U^T | O^T] += S^T [-W ; Q*Gamma]^T  (one N = 128 product)
 //   group B:  [O^T | S^T] += U^T [A_qk ; (K*gamma_C/Gamma)^T]^T  (one N = 192 product; S^T pre-scaled)
-// A tcgen05 MMA's time grows much more slowly than its N, so the products that share an A operand
-// are fused along N. The fused accumulators must be adjacent in TMEM -- [U | O] for group A and
+// and writes each full chunk's O with one TMA tensor store. One thread issues a tcgen05 MMA only every
+// ~100-180 cycles, nearly whatever its N, so the products that share an A operand are fused along N. The fused accumulators must be adjacent in TMEM -- [U | O] for group A and
 // [O | S] for group B -- so the O and U buffers alternate with the chunk's parity around the fixed
 // S, and kernel P writes each block's operand pairs in the order that chunk's parity needs.
 // The price of the split is the workspace traffic (one write and one read of ~1 KB per token-head).
