@@ -269,6 +269,108 @@ __device__ __forceinline__ void p_operands(unsigned char* sm, const Prefetch& pf
   }
 }
 
+// T' = (I + A_kk)^-1 Diag(beta) on all eight warps of kernel P. The four 16 x 16 diagonal inverses by forward
+// substitution in fp32 (warps 0-1; warps 2-3 zero T' above the diagonal), then the blocks below the diagonal
+// from the 2 x 2 split into 32 x 32 halves, (I + A)^-1 = [[T1, 0], [-T2 A21 T1, T2]]: level 1 the blocks
+// (1,0) and (3,2) of T1 and T2, T_ab = -T_aa A_ab T_bb; level 2 Y = A21 T1 into a bf16 scratch tile
+// [32][32]; level 3 the lower-left quadrant -T2 Y. Each warp of a level takes one 16 x 8 half of a block
+// (mma.sync, bf16 operands, fp32 sums); T (bf16) is the operand of the later levels, T' the output.
+__device__ __forceinline__ void p_inverse(unsigned char* sm, uint32_t sb, const IntraLayout& Ly, const float* beta_s,
+                                          int tid, int warp, int lane, int g, int tq, uint32_t yscr) {
+  const float* L = reinterpret_cast<const float*>(sm + Ly.akk);
+  const uint32_t tb = sb + Ly.tb;
+  if (tid < 64) {
+    const int a = tid >> 4, j = tid & 15;
+    float xs[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xs[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int l = 0; l < 16; ++l)
+#pragma unroll
+      for (int i = l + 1; i < 16; ++i) xs[i] -= L[(16 * a + i) * 64 + 16 * a + l] * xs[l];
+    const float bj = beta_s[16 * a + j];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t off = sw_e(16 * a + i, 16 * a + j, 8192);
+      *reinterpret_cast<__nv_bfloat16*>(sm + Ly.tb + off) = __float2bfloat16_rn(xs[i]);
+      *reinterpret_cast<__nv_bfloat16*>(sm + Ly.tp + off) = __float2bfloat16_rn(xs[i] * bj);
+    }
+  } else if (tid < 128) {
+    zero_upper_blocks(sm, Ly.tp, tid - 64, 64);  // T' is lower triangular
+  }
+  __syncthreads();
+  const int jh = warp & 1;  // this warp's 8-column half of its block
+  // the B fragment (16 x 8, this warp's half) of a 16 x 16 bf16 block of T at block row r, block column b
+  auto t_bfrag = [&](int r, int b, uint32_t& b0, uint32_t& b1) {
+    uint32_t x0, x1, x2, x3;
+    ldsm_x4_t(tb + sw_chunk(16 * r + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * b + (lane >> 4), 8192), x0, x1, x2, x3);
+    b0 = jh ? x2 : x0;
+    b1 = jh ? x3 : x1;
+  };
+  // -acc to T and T' at block (a, b), this warp's half
+  auto store_t = [&](int a, int b, const float (&acc)[4]) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = 16 * a + g + 8 * hr, col = 16 * b + 8 * jh + 2 * tq;
+      const float v0 = -acc[2 * hr], v1 = -acc[2 * hr + 1];
+      const uint32_t off = sw_e(row, col, 8192);
+      *reinterpret_cast<uint32_t*>(sm + Ly.tb + off) = pack_bf16(v0, v1);
+      *reinterpret_cast<uint32_t*>(sm + Ly.tp + off) = pack_bf16(v0 * beta_s[col], v1 * beta_s[col + 1]);
+    }
+  };
+  if (warp < 4) {  // level 1: T_10 (warps 0, 1) and T_32 (warps 2, 3)
+    const int a = warp < 2 ? 1 : 3, b = a - 1;
+    uint32_t t0, t1, t2, t3;  // A fragments of T_aa
+    ldsm_x4(tb + sw_chunk(16 * a + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * a + (lane >> 4), 8192), t0, t1, t2, t3);
+    float P[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {  // P = T_aa A_ab; B[k][n] = A[16a + k][16b + n]
+      const float* lp = L + (16 * a + 2 * tq) * 64 + 16 * b + 8 * j + g;
+      mma_bf16(P[j], t0, t1, t2, t3, pack_bf16(lp[0], lp[64]), pack_bf16(lp[8 * 64], lp[9 * 64]));
+    }
+    uint32_t b0, b1;
+    t_bfrag(b, b, b0, b1);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_bf16(acc, pack_bf16(P[0][0], P[0][1]), pack_bf16(P[0][2], P[0][3]), pack_bf16(P[1][0], P[1][1]),
+             pack_bf16(P[1][2], P[1][3]), b0, b1);
+    store_t(a, b, acc);
+  }
+  __syncthreads();
+  const int a = 2 + (warp >> 2), b = (warp >> 1) & 1;  // levels 2 and 3: block (a, b) of the lower-left quadrant
+  {  // level 2: Y_ab = sum_{j=b}^{1} A_aj T_jb
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (j < b) continue;
+      const float* la = L + (16 * a + g) * 64 + 16 * j + 2 * tq;
+      uint32_t b0, b1;
+      t_bfrag(j, b, b0, b1);
+      mma_bf16(acc, pack_bf16(la[0], la[1]), pack_bf16(la[8 * 64], la[8 * 64 + 1]), pack_bf16(la[8], la[9]),
+               pack_bf16(la[8 * 64 + 8], la[8 * 64 + 9]), b0, b1);
+    }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = 16 * (a - 2) + g + 8 * hr, col = 16 * b + 8 * jh + 2 * tq;
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(yscr + row * 64 + col * 2), "r"(pack_bf16(acc[2 * hr], acc[2 * hr + 1]))
+                   : "memory");
+    }
+  }
+  __syncthreads();
+  {  // level 3: T_ab = -sum_{j=2}^{a} T_aj Y_jb
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 2; j < 4; ++j) {
+      if (j > a) continue;
+      uint32_t t0, t1, t2, t3, x0, x1, x2, x3;
+      ldsm_x4(tb + sw_chunk(16 * a + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * j + (lane >> 4), 8192), t0, t1, t2, t3);
+      ldsm_x4_t(yscr + (16 * (j - 2) + (lane & 7) + ((lane >> 3) & 1) * 8) * 64 + (16 * b + 8 * (lane >> 4)) * 2, x0, x1,
+                x2, x3);
+      mma_bf16(acc, t0, t1, t2, t3, jh ? x2 : x0, jh ? x3 : x1);
+    }
+    store_t(a, b, acc);
+  }
+}
+
 // After p_operands and a barrier: the rows of block b in view a > b, as block b's rows of view b times the
 // scale 2^{R_a - e[b]} of each channel (six block pairs of 16 rows x 128 channels, one 8-channel 16-byte
 // piece per thread and pair; fp32 products rounded once to bf16).
@@ -531,8 +633,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) chunk_intra_kernel(ScanParams p, 
         bulk_store(blk + WB_KA + (even ? 0 : 16384), sb + P_AQKT, 8192);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
-      // ---- T' = (I + A_kk)^-1 Diag(beta) on warps 0-3
-      if (warp < 4) inverse_warps0to3(sm, sb, LY, beta_s, tid, warp, lane, g, tq);
+      // ---- T' = (I + A_kk)^-1 Diag(beta) (the pairwise tiles' area is free again: scratch for the inverse)
+      p_inverse(sm, sb, LY, beta_s, tid, warp, lane, g, tq, sb + P_DIAG);
       fence_async_smem();
       tc_fence_before();
       __syncthreads();
