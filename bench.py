@@ -89,21 +89,21 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 # taken on, so a sha256 of those sources (comments and blank space left out, see source_digest) is kept
 # beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
-    # chunk_intra_kernel<2> 404.4 + 356.9 MB; chunk_state_kernel 506.6 + 84.2 MB
-    "prefill": {"bytes": 1352100000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-              "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
+    # chunk_intra_kernel<2> 404.5 + 357.3 MB; chunk_state_kernel 506.6 + 83.9 MB
+    "prefill": {"bytes": 1352200000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+              "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
     # decode_bulk_kernel 410.6 + 345.1 MB
     "decode": {"bytes": 755700000, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                "sha256": "dfbe3ca4ed44294f1662b85f4506abe22c32c93ea6d7e42319af3c3e7838c5a7"},
-    # chunk_intra_kernel<3> 404.9 + 357.6 MB; chunk_state_kernel 506.6 + 83.6 MB (the unbounded gate's prefill)
-    "softplus": {"bytes": 1352700000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
-    # chunk_intra_kernel<2> 8,000.5 + 7,279.4 MB; chunk_state_kernel 9,227.3 + 1,884.0 MB (16 packed sequences)
-    "varlen": {"bytes": 26391200000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-             "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
-    # chunk_intra_kernel<2> 2,391.2 + 2,118.9 MB; chunk_state_kernel 3,261.1 + 1,060.8 MB (4 x 16384 x 32, V = 256)
-    "long_kv": {"bytes": 8832000000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-              "sha256": "07a08d32a73887753be06a4371a6c314a4c7acff4006bb67e106299746d316bb"},
+    # chunk_intra_kernel<3> 405.1 + 357.6 MB; chunk_state_kernel 506.6 + 84.1 MB (the unbounded gate's prefill)
+    "softplus": {"bytes": 1353400000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
+    # chunk_intra_kernel<2> 7,911.6 + 7,282.1 MB; chunk_state_kernel 9,227.4 + 1,884.3 MB (16 packed sequences)
+    "varlen": {"bytes": 26305300000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+             "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
+    # chunk_intra_kernel<2> 2,339.6 + 2,120.8 MB; chunk_state_kernel 3,255.0 + 1,060.0 MB (4 x 16384 x 32, V = 256)
+    "long_kv": {"bytes": 8775400000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+              "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
     # bounded_decay_kernel 201,369,600 + 154,498,560; scan_backward_kernel 17,579,054,336 + 27,342,757,376;
     # bounded_decay_backward_kernel 402,670,080 + 162,126,848 (one backward step from the logits)
     "backward": {"bytes": 45842476800, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
