@@ -62,3 +62,18 @@ def test_measured_traffic_only_for_the_profiled_sources(monkeypatch):
         changed = dict(bench.MEASURED_TRAFFIC[step], sha256="0" * 64)
         monkeypatch.setitem(bench.MEASURED_TRAFFIC, step, changed)
         assert bench.measured_traffic(step) is None
+
+
+def test_source_digest_ignores_comments_not_code(tmp_path, monkeypatch):
+    # the traffic records stay valid across a change of comments or blank space, not across a change of code
+    import bench
+    csrc = tmp_path / "gated_delta_rule_bounded_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f = csrc / "k.cu"
+    f.write_text("// kernel\nint f(int x) {\n  return x + 1;  /* one */\n}\n")
+    d0 = bench.source_digest(["k.cu"])
+    f.write_text("/* a longer\n   comment */\nint f(int x) {\n\n    return x + 1;   // one more\n}\n")
+    assert bench.source_digest(["k.cu"]) == d0
+    f.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.source_digest(["k.cu"]) != d0
