@@ -631,11 +631,27 @@ def decode_leg(args, kda, dev, stream, rank, world, hbm, peak_src):
         return res
     # e2e: each step's q, k, v, z, beta from pinned host memory, the step on the kept state, o back to the host;
     # consecutive steps overlapped (the state update itself stays in order on one stream)
-    hostd = [{n: x.pin_memory() for n, x in W.make_decode_step(dw, s).items()} for s in range(n_sets)]
-    devd = [{n: torch.empty_like(x, device=dev) for n, x in hostd[0].items()} for _ in range(2)]
+    # A step's five small inputs travel as one copy: packed into one pinned buffer per input set (256-byte
+    # aligned pieces), unpacked on the device as views of one buffer.
+    steps_in = [W.make_decode_step(dw, s) for s in range(n_sets)]
+    layout, total = {}, 0
+    for n, x in steps_in[0].items():
+        layout[n] = (total, x.numel() * x.element_size(), x.dtype, tuple(x.shape))
+        total += (layout[n][1] + 255) // 256 * 256
+    hostd = []
+    for st in steps_in:
+        buf = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        for n, (off, nb, dt, shp) in layout.items():
+            buf[off:off + nb].copy_(st[n].contiguous().view(torch.uint8).reshape(-1))
+        hostd.append({"buf": buf})
+    devd = []
+    for _ in range(2):
+        dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+        devd.append({"buf": dbuf, **{n: dbuf[off:off + nb].view(dt).view(shp)
+                                     for n, (off, nb, dt, shp) in layout.items()}})
     host_out = {"o": torch.empty(dw.B, dw.H, dw.V, dtype=torch.bfloat16).pin_memory()}
     dev_out = [{"o": o_dec}, {"o": torch.empty_like(o_dec)}]
-    dh2d = sum(x.numel() * x.element_size() for x in hostd[0].values())
+    dh2d = sum(nb for _, nb, _, _ in layout.values())
     dd2h = host_out["o"].numel() * host_out["o"].element_size()
 
     def drun(i, out):
