@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["bounded_decay", "softplus_decay", "prefill", "prefill_logits", "prefill_noalloc", "scan_backward", "bounded_decay_backward", "decode_step", "decode_step_logits", "prefill_workspace_bytes", "device_status", "KDAError",
+__all__ = ["bounded_decay", "softplus_decay", "prefill", "prefill_logits", "prefill_noalloc", "scan_backward", "scan_backward_chunked", "chunked_backward_workspace_bytes", "bounded_decay_backward", "decode_step", "decode_step_logits", "prefill_workspace_bytes", "device_status", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -84,9 +84,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_scan_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, lp,
                                       vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_bounded_decay_backward.argtypes = [vp, vp, ctypes.c_float, vp, i64, i64, i64, i64, vp, vp, vp]
+    lib.kda_scan_backward_chunked_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_scan_backward_chunked.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64, i64, i64, i64, i64, lp,
+                                              vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_selftest_wait_expiry.argtypes = [vp]
     for fn in ("kda_scan_backward_workspace_bytes", "kda_scan_backward", "kda_bounded_decay_backward",
-               "kda_selftest_wait_expiry"):
+               "kda_selftest_wait_expiry", "kda_scan_backward_chunked_workspace_bytes", "kda_scan_backward_chunked"):
         getattr(lib, fn).restype = ctypes.c_int
     for fn in ("kda_bounded_decay", "kda_softplus_decay", "kda_prefill_workspace_bytes", "kda_prefill", "kda_prefill_noalloc",
                "kda_decode_step", "kda_prefill_logits", "kda_decode_step_logits"):
@@ -495,6 +498,57 @@ def scan_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch
         out["dv"].data_ptr(), out["dgate"].data_ptr(), out["dbeta"].data_ptr(), out["d_initial_state"].data_ptr(),
         ws.data_ptr(), ws.numel(), _stream(dev)))
     return out
+
+
+def scan_backward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
+                          initial_state: Optional[torch.Tensor], d_o: torch.Tensor,
+                          d_final_state: Optional[torch.Tensor] = None, *, gate_is_log: bool = False,
+                          workspace: Optional[torch.Tensor] = None) -> dict:
+    """The gradients of ``scan_backward`` through the chunkwise form in parallel over 64-token chunks
+    (``kda_scan_backward_chunked``): bf16 ``q, k, v`` with K = V = 128, dense batch rows. Same outputs.
+    ``workspace``: optional uint8 device tensor of at least ``chunked_backward_workspace_bytes`` bytes."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta"), (d_o, "d_o")):
+        _cuda(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k must be [B,T,H,K] and v [B,T,H,V]")
+    if gate.shape != q.shape or gate.dtype != torch.float32 or beta.shape != q.shape[:3] or beta.dtype != torch.float32:
+        raise ValueError("gate must be fp32 [B,T,H,K] and beta fp32 [B,T,H]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    dev = q.device
+    q, k, v, gate = map(_rowwise, (q, k, v, gate))
+    d_o = d_o.to(torch.float32).contiguous()
+    if d_o.shape != (B, T, H, V):
+        raise ValueError("d_o must be [B,T,H,V]")
+    f32 = lambda t: None if t is None else t.to(device=dev, dtype=torch.float32).contiguous()  # noqa: E731
+    initial_state, d_final_state = f32(initial_state), f32(d_final_state)
+    for t, n in ((initial_state, "initial_state"), (d_final_state, "d_final_state")):
+        if t is not None and t.shape != (B, H, K, V):
+            raise ValueError(f"{n} must be [{B},{H},{K},{V}]")
+    out = {"dq": torch.empty(B, T, H, K, device=dev), "dk": torch.empty(B, T, H, K, device=dev),
+           "dv": torch.empty(B, T, H, V, device=dev), "dgate": torch.empty(B, T, H, K, device=dev),
+           "dbeta": torch.empty(B, T, H, device=dev), "d_initial_state": torch.empty(B, H, K, V, device=dev)}
+    lib = load_library()
+    need = chunked_backward_workspace_bytes(B, T, H, K, V)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
+    layout = Layout(_strides4(q), _strides4(k), _strides4(v), _strides4(gate), _strides3(beta), Strides(0, 0, 0))
+    ptr = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
+    _check("kda_scan_backward_chunked", lib.kda_scan_backward_chunked(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
+        KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), ptr(initial_state), d_o.data_ptr(),
+        ptr(d_final_state), B, T, H, K, V, ctypes.byref(layout), out["dq"].data_ptr(), out["dk"].data_ptr(),
+        out["dv"].data_ptr(), out["dgate"].data_ptr(), out["dbeta"].data_ptr(), out["d_initial_state"].data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(dev)))
+    return out
+
+
+def chunked_backward_workspace_bytes(B: int, T: int, H: int, K: int = 128, V: int = 128) -> int:
+    """Workspace bytes of ``scan_backward_chunked`` (``kda_scan_backward_chunked_workspace_bytes``)."""
+    n = ctypes.c_size_t(0)
+    _check("kda_scan_backward_chunked_workspace_bytes",
+           load_library().kda_scan_backward_chunked_workspace_bytes(B, T, H, K, V, ctypes.byref(n)))
+    return int(n.value)
 
 
 def bounded_decay_backward(logits: torch.Tensor, A_log: torch.Tensor, g_min: float,

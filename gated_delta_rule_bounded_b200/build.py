@@ -2,7 +2,8 @@
 
 Each ``csrc/*.cu`` file is compiled with nvcc for ``sm_100a`` only and linked
 into one shared library next to this file, with the CUDA runtime linked
-statically so the library has no dependency on a particular libcudart.
+statically so the library has no dependency on a particular libcudart (cuBLAS,
+used by the chunked gradients' plain batched products, is linked dynamically).
 Objects are cached under ``_build/`` and rebuilt when a source or header is
 newer. Run ``python -m gated_delta_rule_bounded_b200.build``.
 """
@@ -66,7 +67,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
     newest = max(os.path.getmtime(o) for o in objs)
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
-        cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", LIB + ".tmp", *objs]
+        cuda_lib = os.path.join(os.path.dirname(os.path.dirname(nvcc())), "lib64")
+        cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", LIB + ".tmp", *objs, "-lcublas",
+               "-Xlinker", "-rpath", "-Xlinker", cuda_lib]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -885,6 +885,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) chunk_state_kernel(ScanParams p, 
         const int cb = 64 * half + 32 * part;
         uint32_t r[32], b16[16];
         tm_ld32(tlane + TM_S + cb, r);
+        if (p.s_dump) {  // the chunk's start state, for the chunked gradients
+          float* dst = p.s_dump + ((size_t)(sbase_slot + c) * p.H + h) * KD * p.V + (size_t)cb * p.V + vt * VT + trow;
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) dst[(size_t)jj * p.V] = __uint_as_float(r[jj]);
+        }
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) b16[jj] = pack_bf16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]));
         tm_st16(tlane + TM_SB + cb / 2, b16);

@@ -525,6 +525,101 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
   return ok();
 }
 
+int kda_scan_backward_chunked_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes) {
+  if (!bytes) return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_chunked_workspace_bytes: null output");
+  if (B < 0 || T < 0 || H < 0 || K < 0 || V < 0)
+    return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_chunked_workspace_bytes: negative size");
+  if (K != 128 || V != 128)
+    return fail(KDA_ERR_UNSUPPORTED, "kda_scan_backward_chunked_workspace_bytes: K and V must be 128");
+  *bytes = (B * T * H == 0) ? 0 : kda::chunked_backward_workspace_bytes(B, T, H);
+  return ok();
+}
+
+int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_dtype dtype,
+                              const float* gate, kda_gate_kind gate_kind, const float* beta,
+                              const float* initial_state, const float* d_o, const float* d_final_state,
+                              int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
+                              float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
+                              void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const char* fn = "kda_scan_backward_chunked";
+  if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+  if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
+    return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, (int)gate_kind);
+  if (dtype != KDA_BF16 || K != 128 || V != 128)
+    return fail(KDA_ERR_UNSUPPORTED, "%s: bf16 q, k, v with K = V = 128 only", fn);
+  if (H > 65535) return fail(KDA_ERR_UNSUPPORTED, "%s: H must be at most 65535", fn);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B * H == 0) return ok();
+  if (T == 0) {  // nothing to differentiate through: dS_0 = dS_T
+    if (d_initial_state) {
+      cudaError_t e = kda::launch_state_copy(d_final_state, d_initial_state, B * H * K * V, s);
+      if (e != cudaSuccess) return cuda_fail(e, fn);
+    }
+    return ok();
+  }
+  if (!q || !k || !v || !gate || !beta || !d_o || !dq || !dk || !dv || !dgate || !dbeta)
+    return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (T > INT32_MAX || (T + 63) / 64 * B * H > INT32_MAX) return fail(KDA_ERR_UNSUPPORTED, "%s: T too large", fn);
+  const size_t need = kda::chunked_backward_workspace_bytes(B, T, H);
+  if (!workspace || workspace_bytes < need)
+    return fail(KDA_ERR_INVALID_ARG, "%s: the workspace needs %zu bytes (got %zu)", fn, need, workspace_bytes);
+  kda_layout L;
+  if (layout) {
+    L = *layout;
+  } else {
+    L.q = contiguous(T, H, K);
+    L.k = contiguous(T, H, K);
+    L.gate = contiguous(T, H, K);
+    L.v = contiguous(T, H, V);
+    L.o = contiguous(T, H, V);
+    L.beta = contiguous(T, H, 1);
+  }
+  const kda_strides* all[5] = {&L.q, &L.k, &L.v, &L.gate, &L.beta};
+  for (auto* st : all)
+    if (!strides_valid(*st)) return fail(KDA_ERR_INVALID_ARG, "%s: negative stride", fn);
+  if (!rows_aligned(q, L.q, 2, B, T, H) || !rows_aligned(k, L.k, 2, B, T, H) || !rows_aligned(v, L.v, 2, B, T, H) ||
+      !rows_aligned(gate, L.gate, 4, B, T, H) || !aligned16(d_o) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || !aligned16(dgate) || !aligned16(workspace) || (initial_state && !aligned16(initial_state)) ||
+      (d_final_state && !aligned16(d_final_state)) || (d_initial_state && !aligned16(d_initial_state)))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: rows and buffers must start on 16-byte boundaries", fn);
+  kda::ScanParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.gate = gate;
+  p.beta = beta;
+  p.s0 = initial_state;
+  p.sf = nullptr;
+  p.cu = nullptr;
+  p.o = nullptr;
+  put(p.qs, L.q);
+  put(p.ks, L.k);
+  put(p.vs, L.v);
+  put(p.gs, L.gate);
+  put(p.bs, L.beta);
+  p.T = T;
+  p.B = (int)B;
+  p.H = (int)H;
+  p.K = (int)K;
+  p.V = (int)V;
+  p.N = (int)B;
+  p.gate_mode = (int)gate_kind;
+  p.A_log = nullptr;
+  p.dt_bias = nullptr;
+  p.g_min = 0.f;
+  p.qk_l2norm = 0;
+  p.beta_sigmoid = 0;
+  p.state_vk = 0;
+  if (!kda::split_maps_ok(p)) return fail(KDA_ERR_UNSUPPORTED, "%s: the q, k or gate layout admits no tensor map", fn);
+  int cublas_status = 0;
+  cudaError_t e = kda::launch_chunked_backward(p, d_o, d_final_state, dq, dk, dv, dgate, dbeta, d_initial_state,
+                                               workspace, s, &cublas_status);
+  if (cublas_status != 0) return fail(KDA_ERR_CUDA, "%s: cuBLAS status %d", fn, cublas_status);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
 int kda_bounded_decay_backward(const float* logits, const float* A_log, float g_min, const float* d_log_decay,
                                int64_t B, int64_t T, int64_t H, int64_t K, float* d_logits, float* d_A_log,
                                kda_stream_t stream) {

@@ -37,6 +37,7 @@ struct ScanParams {
   int qk_l2norm;        // q, k are L2-normalised over K inside the kernels
   int beta_sigmoid;     // beta holds logits; the kernels use sigmoid(beta)
   int state_vk;         // states stored [N,H,V,K] (K contiguous) instead of [N,H,K,V]
+  float* s_dump = nullptr;  // split path only: the state at every chunk start, fp32 [slot][H][K][V] (or null)
 };
 
 // Offset of state element (key row c, value column v) of a head whose state starts at `head_base`.
@@ -104,6 +105,11 @@ size_t chunk_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t n_seq);
 cudaError_t launch_chunk(const ScanParams& p, void* ws, size_t ws_bytes, cudaStream_t s);
 size_t split_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, bool varlen);
 cudaError_t launch_chunk_split(const ScanParams& p, void* ws, cudaStream_t s);
+// Gradients through the chunkwise form (backward_chunked.cu): bf16 q/k/v, K = V = 128, dense batch rows.
+size_t chunked_backward_workspace_bytes(int64_t B, int64_t T, int64_t H);
+cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, const float* d_sf, float* dq, float* dk,
+                                    float* dv, float* dgate, float* dbeta, float* ds0, void* ws, cudaStream_t s,
+                                    int* cublas_status);
 // Whether the driver accepts tensor maps of this call's q, k and gate layouts (the two-kernel path reads
 // them by TMA); when it does not, the single fused kernel runs instead.
 bool split_maps_ok(const ScanParams& p);

@@ -333,6 +333,32 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
                       void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * kda_scan_backward_chunked: the same gradients as kda_scan_backward, computed
+ * through the chunkwise form ("KDA cheat sheet", chunkwise form, eqs. 3-4) in
+ * parallel over 64-token chunks: the forward's split kernels keep the state at
+ * every chunk start, one reverse recurrence over chunks gives the gradient of
+ * the state at every chunk end, and every other gradient is formed per chunk
+ * (per-pair decay ratios, triangular inverse, plain batched products through
+ * cuBLAS in fp32 with TF32 tensor cores). Arguments, layouts and outputs as for
+ * kda_scan_backward without cu_seqlens. Supported: bf16 q, k, v with K = V = 128
+ * (KDA_ERR_UNSUPPORTED otherwise). The chunk-start states come from the bf16
+ * tensor-core forward, so the gradients carry its rounding (relative RMS errors
+ * near 1e-3) where kda_scan_backward's token-level adjoint is exact fp32. The
+ * workspace (kda_scan_backward_chunked_workspace_bytes; about 880 KB per chunk
+ * and head) holds every intermediate; cuBLAS creates its handle (device memory)
+ * on the first call on each device and is given a part of the workspace for
+ * its own scratch.
+ * ------------------------------------------------------------------------- */
+int kda_scan_backward_chunked_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes);
+
+int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_dtype dtype,
+                              const float* gate, kda_gate_kind gate_kind, const float* beta,
+                              const float* initial_state, const float* d_o, const float* d_final_state,
+                              int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
+                              float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
+                              void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * kda_bounded_decay_backward: gradients of eq. 5's log-decay
  * g = g_min * sigmoid(exp(A_log[h]) * z) given d_log_decay = dL/dg:
  *   d_logits = dL/dz [B,T,H,K], d_A_log = dL/dA_log [H] (overwritten).
