@@ -42,7 +42,6 @@ namespace {
 
 constexpr int CC = 64;    // tokens per chunk
 constexpr int D = 128;    // K = V
-constexpr int PAD = 129;  // padded row length of the shared-memory [64][128] tiles (no bank conflicts)
 constexpr float LOG2E_F = 1.4426950408889634f;
 constexpr float FLOOR2 = -126.f;  // per-token log2-decay floor (alpha = 0 included), as in the forward
 
@@ -86,8 +85,8 @@ __device__ __forceinline__ void chunk_of(const BwdC& a, int b, int& n, int& j, i
 
 // fp32 copies of the chunk's q, k, v, dO (zero past the end), the log2 cumulative decay (per-token floor at
 // -126, zero past the end: alpha = 1), Q*Gamma, K*Gamma, K*gamma_C/Gamma, gamma_C and beta (zero past the end).
+// Threads 0-127 walk the tokens for channel c (the cumulative sum), threads 128-255 copy v and dO.
 __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
-  __shared__ float Gs[CC][D];
   const int b = blockIdx.x, tid = threadIdx.x;
   int n, j, h, t0, nv;
   chunk_of(a, b, n, j, h, t0, nv);
@@ -95,6 +94,7 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
   if (tid < D) {
     const int c = tid;
     float run = 0.f;
+#pragma unroll 8
     for (int t = 0; t < CC; ++t) {
       const bool in = t < nv;
       const int64_t tt = t0 + t;
@@ -106,7 +106,6 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
         kv = __bfloat162float(static_cast<const __nv_bfloat16*>(a.k)[n * a.ks[0] + tt * a.ks[1] + h * a.ks[2] + c]);
       }
       run += l;
-      Gs[t][c] = run;
       const float gm = ex2f(run);
       w.G2[mat + t * D + c] = run;
       w.Qf[mat + t * D + c] = qv;
@@ -115,9 +114,11 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
       w.KG[mat + t * D + c] = kv * gm;
     }
     w.gam[(size_t)b * D + c] = ex2f(run);
-    for (int t = 0; t < CC; ++t) w.KT[mat + t * D + c] = w.Kf[mat + t * D + c] * ex2f(run - Gs[t][c]);
+#pragma unroll 8
+    for (int t = 0; t < CC; ++t) w.KT[mat + t * D + c] = w.Kf[mat + t * D + c] * ex2f(run - w.G2[mat + t * D + c]);
   } else {
     const int c = tid - D;
+#pragma unroll 8
     for (int t = 0; t < CC; ++t) {
       const bool in = t < nv;
       const int64_t tt = t0 + t;
@@ -137,40 +138,61 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
 }
 
 // Mq and Mk of one chunk, every pair (t, i <= t) summed over the channels with its decay ratio
-// 2^{G2_tc - G2_ic} <= 1 formed directly (no range limit). A warp takes one row t and 32 columns i.
-__global__ void __launch_bounds__(256) pair_kernel(Bufs w) {
-  extern __shared__ float sp[];
+// 2^{G2_tc - G2_ic} <= 1 formed directly (no range limit). A warp takes 4 rows t and 32 columns i (a lane per
+// i), channels 4 at a time from rows padded to 132 floats (the row-t operands are warp-uniform float4 loads).
+constexpr int PAIR_SMEM = 3 * CC * 132 * 4;
+__global__ void __launch_bounds__(256, 2) pair_kernel(Bufs w) {
+  constexpr int PR = 132;
+  extern __shared__ __align__(16) float sp[];
   float* Qs = sp;
-  float* Ks = Qs + CC * PAD;
-  float* Gs = Ks + CC * PAD;
+  float* Ks = Qs + CC * PR;
+  float* Gs = Ks + CC * PR;
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t mat = (size_t)b * CC * D;
-  for (int e = tid; e < CC * D; e += 256) {
-    const int t = e / D, c = e % D;
-    Qs[t * PAD + c] = w.Qf[mat + e];
-    Ks[t * PAD + c] = w.Kf[mat + e];
-    Gs[t * PAD + c] = w.G2[mat + e];
+  for (int e = tid; e < CC * D / 4; e += 256) {
+    const int t = e >> 5, c4 = e & 31;
+    *reinterpret_cast<float4*>(Qs + t * PR + 4 * c4) = reinterpret_cast<const float4*>(w.Qf + mat)[e];
+    *reinterpret_cast<float4*>(Ks + t * PR + 4 * c4) = reinterpret_cast<const float4*>(w.Kf + mat)[e];
+    *reinterpret_cast<float4*>(Gs + t * PR + 4 * c4) = reinterpret_cast<const float4*>(w.G2 + mat)[e];
   }
   __syncthreads();
   const size_t sq = (size_t)b * CC * CC;
-  for (int u = warp; u < 2 * CC; u += 8) {
-    const int t = u >> 1, i = (u & 1) * 32 + lane;
-    float mq = 0.f, mk = 0.f;
-    if (i <= t) {
-      const float* qt = Qs + t * PAD;
-      const float* kt = Ks + t * PAD;
-      const float* gt = Gs + t * PAD;
-      const float* ki = Ks + i * PAD;
-      const float* gi = Gs + i * PAD;
-#pragma unroll 4
-      for (int c = 0; c < D; ++c) {
-        const float r = ex2f(gt[c] - gi[c]) * ki[c];
-        mq = fmaf(qt[c], r, mq);
-        mk = fmaf(kt[c], r, mk);
+  // units (4 rows from 4q, columns from 32 hf): warp w takes q = w, w + 8 with hf = 0 and q = w + 8 with
+  // hf = 1; (q = w, hf = 1) lies above the diagonal and is all zero
+#pragma unroll 1
+  for (int k = 0; k < 4; ++k) {
+    const int u = warp + 8 * k, q = u & 15, hf = u >> 4;
+    const int i = 32 * hf + lane, tq = 4 * q;
+    float mq[4] = {0.f, 0.f, 0.f, 0.f}, mk[4] = {0.f, 0.f, 0.f, 0.f};
+    if (32 * hf <= tq + 3) {
+      const float* ki_ = Ks + i * PR;
+      const float* gi_ = Gs + i * PR;
+#pragma unroll 2
+      for (int c = 0; c < D; c += 4) {
+        const float4 kv = *reinterpret_cast<const float4*>(ki_ + c);
+        const float4 gv = *reinterpret_cast<const float4*>(gi_ + c);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float4 qv = *reinterpret_cast<const float4*>(Qs + (tq + r) * PR + c);
+          const float4 kt = *reinterpret_cast<const float4*>(Ks + (tq + r) * PR + c);
+          const float4 gt = *reinterpret_cast<const float4*>(Gs + (tq + r) * PR + c);
+          float x = ex2f(gt.x - gv.x) * kv.x;
+          mq[r] = fmaf(qv.x, x, mq[r]); mk[r] = fmaf(kt.x, x, mk[r]);
+          x = ex2f(gt.y - gv.y) * kv.y;
+          mq[r] = fmaf(qv.y, x, mq[r]); mk[r] = fmaf(kt.y, x, mk[r]);
+          x = ex2f(gt.z - gv.z) * kv.z;
+          mq[r] = fmaf(qv.z, x, mq[r]); mk[r] = fmaf(kt.z, x, mk[r]);
+          x = ex2f(gt.w - gv.w) * kv.w;
+          mq[r] = fmaf(qv.w, x, mq[r]); mk[r] = fmaf(kt.w, x, mk[r]);
+        }
       }
     }
-    w.Mq[sq + t * CC + i] = mq;
-    w.Mk[sq + t * CC + i] = i < t ? mk : 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int t = tq + r;
+      w.Mq[sq + t * CC + i] = i <= t ? mq[r] : 0.f;
+      w.Mk[sq + t * CC + i] = i < t ? mk[r] : 0.f;
+    }
   }
 }
 
@@ -201,78 +223,120 @@ __global__ void __launch_bounds__(64) inverse_kernel(Bufs w) {
   }
 }
 
-// The reverse recurrence for dS over the chunks of one (batch row, head), value columns [32 s, 32 s + 32):
-// dS_C of every chunk to dSC, dS0 of the first to ds0. A thread holds dS[c][16 columns].
+// 16-byte asynchronous global -> shared copies (the operand prefetch of the dS recurrence).
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The reverse recurrence for dS over the chunks of one (batch row, head), value columns [32 s, 32 s + 32).
+// The dO terms are independent of the recurrence and come in precomputed: X1 = Mq^T dO in dU and
+// Y = QG^T dO - W^T X1 in dS_C's place. Per chunk, from the last:
+//   dS_C = dS;  dU = X1 + KT dS;  dS <- Diag(gamma_C) dS + Y - W^T (KT dS),
+// with dS_C and dU written over Y and X1 and dS0 of the first chunk to ds0. A thread holds dS[c][16 columns];
+// KT and W of the next chunk are prefetched (cp.async) into the other half of a double buffer, rows padded to
+// 132 floats (16-byte aligned, rows 4 banks apart).
 constexpr int VS = 32;
+constexpr int P4 = 132;
+constexpr int DS_OPS = 2 * CC * P4;  // KT and W of one chunk
+constexpr int DSTATE_SMEM = (2 * DS_OPS + D * VS + CC * VS + D) * 4;
+
+__device__ __forceinline__ void dstate_prefetch(const Bufs& w, size_t mat, float* dst, int tid) {
+  const float* kt = w.KT + mat;
+  const float* wm = w.W + mat;
+#pragma unroll
+  for (int e = tid; e < CC * D / 4; e += 256) {
+    const int t = e >> 5, c4 = e & 31;
+    cp_async16(dst + t * P4 + 4 * c4, kt + 4 * e);
+    cp_async16(dst + CC * P4 + t * P4 + 4 * c4, wm + 4 * e);
+  }
+  cp_async_commit();
+}
+
 __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
-  extern __shared__ float sd[];
-  float* Mq = sd;                 // [64][65]
-  float* KT = Mq + CC * (CC + 1); // [64][129]
-  float* QG = KT + CC * PAD;      // [64][129]
-  float* Wm = QG + CC * PAD;      // [64][129]
-  float* dOs = Wm + CC * PAD;     // [64][VS]
-  float* dSs = dOs + CC * VS;     // [128][VS]
-  float* dUs = dSs + D * VS;      // [64][VS]
+  extern __shared__ __align__(16) float sd[];
+  float* dSs = sd + 2 * DS_OPS;   // [128][VS]
+  float* dUs = dSs + D * VS;      // [64][VS]: KT dS
   float* gm = dUs + CC * VS;      // [128]
   const int tid = threadIdx.x;
   const int nh = blockIdx.x, vsl = blockIdx.y;
   const int n = nh / a.H, h = nh % a.H;
   const int c = tid >> 1, v0 = (tid & 1) * 16;   // this thread's dS[c][v0 .. v0 + 15] of the slice
   const int vg = vsl * VS + v0;                  // global value column of v0
+  const int i = tid >> 2, vq = (tid & 3) * 8;    // this thread's dU[i][vq .. vq + 7] of the slice
   float dS[16];
   const size_t shead = ((size_t)n * a.H + h) * D * D;
 #pragma unroll
   for (int u = 0; u < 16; ++u) dS[u] = a.d_sf ? a.d_sf[shead + (size_t)c * D + vg + u] : 0.f;
+  dstate_prefetch(w, (size_t)((n * a.ncps + a.ncps - 1) * a.H + h) * CC * D, sd + ((a.ncps - 1) & 1) * DS_OPS, tid);
   for (int j = a.ncps - 1; j >= 0; --j) {
     const int b = (n * a.ncps + j) * a.H + h;
-    const size_t mat = (size_t)b * CC * D, sq = (size_t)b * CC * CC, st = (size_t)b * D * D;
+    const size_t mat = (size_t)b * CC * D, st = (size_t)b * D * D;
+    const float* KTs = sd + (j & 1) * DS_OPS;
+    const float* Ws = KTs + CC * P4;
+    float y[16];
+    float* dsc = w.dSC + st + (size_t)c * D + vg;
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      w.dSC[st + (size_t)c * D + vg + u] = dS[u];
-      dSs[c * VS + v0 + u] = dS[u];
+    for (int u = 0; u < 16; u += 4) {
+      const float4 t4 = *reinterpret_cast<const float4*>(dsc + u);
+      y[u] = t4.x; y[u + 1] = t4.y; y[u + 2] = t4.z; y[u + 3] = t4.w;
+      const float4 x = make_float4(dS[u], dS[u + 1], dS[u + 2], dS[u + 3]);
+      *reinterpret_cast<float4*>(dsc + u) = x;
+      *reinterpret_cast<float4*>(dSs + c * VS + v0 + u) = x;
     }
-    for (int e = tid; e < CC * CC; e += 256) Mq[(e / CC) * (CC + 1) + e % CC] = w.Mq[sq + e];
-    for (int e = tid; e < CC * D; e += 256) {
-      const int t = e / D, cc = e % D;
-      KT[t * PAD + cc] = w.KT[mat + e];
-      QG[t * PAD + cc] = w.QG[mat + e];
-      Wm[t * PAD + cc] = w.W[mat + e];
-    }
-    for (int e = tid; e < CC * VS; e += 256) dOs[e] = w.dOf[mat + (e / VS) * D + vsl * VS + e % VS];
+    float* du = w.dU + mat + (size_t)i * D + vsl * VS + vq;
+    const float4 x1a = *reinterpret_cast<const float4*>(du);
+    const float4 x1b = *reinterpret_cast<const float4*>(du + 4);
     if (tid < D) gm[tid] = w.gam[(size_t)b * D + tid];
+    if (j > 0) {
+      dstate_prefetch(w, (size_t)((n * a.ncps + j - 1) * a.H + h) * CC * D, sd + ((j - 1) & 1) * DS_OPS, tid);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
-    // dU[i][v] = sum_t Mq[t][i] dO[t][v] + sum_c KT[i][c] dS[c][v]: a thread takes row i, 8 columns
+    // KT dS: a thread takes row i, 8 columns
     {
-      const int i = tid >> 2, vq = (tid & 3) * 8;
       float acc[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-      for (int t = i; t < CC; ++t) {  // Mq[t][i] = 0 for t < i
-        const float m = Mq[t * (CC + 1) + i];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = fmaf(m, dOs[t * VS + vq + u], acc[u]);
-      }
+#pragma unroll 4
       for (int cc = 0; cc < D; ++cc) {
-        const float kt = KT[i * PAD + cc];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = fmaf(kt, dSs[cc * VS + vq + u], acc[u]);
+        const float kt = KTs[i * P4 + cc];
+        const float4 s0 = *reinterpret_cast<const float4*>(dSs + cc * VS + vq);
+        const float4 s1 = *reinterpret_cast<const float4*>(dSs + cc * VS + vq + 4);
+        acc[0] = fmaf(kt, s0.x, acc[0]); acc[1] = fmaf(kt, s0.y, acc[1]); acc[2] = fmaf(kt, s0.z, acc[2]);
+        acc[3] = fmaf(kt, s0.w, acc[3]); acc[4] = fmaf(kt, s1.x, acc[4]); acc[5] = fmaf(kt, s1.y, acc[5]);
+        acc[6] = fmaf(kt, s1.z, acc[6]); acc[7] = fmaf(kt, s1.w, acc[7]);
       }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) dUs[i * VS + vq + u] = acc[u];
+      *reinterpret_cast<float4*>(dUs + i * VS + vq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float4*>(dUs + i * VS + vq + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      *reinterpret_cast<float4*>(du) = make_float4(x1a.x + acc[0], x1a.y + acc[1], x1a.z + acc[2], x1a.w + acc[3]);
+      *reinterpret_cast<float4*>(du + 4) = make_float4(x1b.x + acc[4], x1b.y + acc[5], x1b.z + acc[6], x1b.w + acc[7]);
     }
     __syncthreads();
-    // dS0[c][v] = gamma_C[c] dS[c][v] + sum_t QG[t][c] dO[t][v] - sum_t W[t][c] dU[t][v]
+    // dS <- gamma_C[c] dS[c][v] + Y[c][v] - sum_t W[t][c] (KT dS)[t][v]
     {
       const float g = gm[c];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) dS[u] *= g;
+      for (int u = 0; u < 16; ++u) dS[u] = fmaf(g, dS[u], y[u]);
+#pragma unroll 4
       for (int t = 0; t < CC; ++t) {
-        const float qg = QG[t * PAD + c], wv = Wm[t * PAD + c];
+        const float wv = Ws[t * P4 + c];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) dS[u] = fmaf(qg, dOs[t * VS + v0 + u], fmaf(-wv, dUs[t * VS + v0 + u], dS[u]));
+        for (int u = 0; u < 16; u += 4) {
+          const float4 e = *reinterpret_cast<const float4*>(dUs + t * VS + v0 + u);
+          dS[u] = fmaf(-wv, e.x, dS[u]);
+          dS[u + 1] = fmaf(-wv, e.y, dS[u + 1]);
+          dS[u + 2] = fmaf(-wv, e.z, dS[u + 2]);
+          dS[u + 3] = fmaf(-wv, e.w, dS[u + 3]);
+        }
       }
     }
-    __syncthreads();
+    __syncthreads();  // the buffer just read is the next prefetch's target
   }
   if (a.ds0) {
 #pragma unroll
@@ -280,16 +344,19 @@ __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
   }
 }
 
-// dMq = tril(dMq) (diagonal kept); dgamma_C[c] = sum_v dS_C[c][v] S0[c][v].
+// dMq = tril(dMq) (diagonal kept); dgamma_C[c] = sum_v dS_C[c][v] S0[c][v] (a warp per row c).
 __global__ void __launch_bounds__(256) mask_dgc_kernel(Bufs w) {
-  const int b = blockIdx.x, tid = threadIdx.x;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t sq = (size_t)b * CC * CC, st = (size_t)b * D * D;
   for (int e = tid; e < CC * CC; e += 256)
     if (e % CC > e / CC) w.dMq[sq + e] = 0.f;
-  if (tid < D) {
-    float s = 0.f;
-    for (int v = 0; v < D; ++v) s = fmaf(w.dSC[st + (size_t)tid * D + v], w.S0[st + (size_t)tid * D + v], s);
-    w.dgC[(size_t)b * D + tid] = s;
+  for (int c = warp; c < D; c += 8) {
+    const float4 x = *reinterpret_cast<const float4*>(w.dSC + st + (size_t)c * D + 4 * lane);
+    const float4 y = *reinterpret_cast<const float4*>(w.S0 + st + (size_t)c * D + 4 * lane);
+    float s = x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+    if (lane == 0) w.dgC[(size_t)b * D + c] = s;
   }
 }
 
@@ -309,83 +376,177 @@ __global__ void __launch_bounds__(64) dt_kernel(Bufs w, float* dbeta_part) {
 }
 
 // dA = strict_tril(dA) in place; dbeta = colsum(dTB * T) + rowsum(dA * Mk); dMk = Diag(beta) dA (into dA).
-__global__ void __launch_bounds__(64) da_kernel(Bufs w, float* dbeta_part) {
-  const int b = blockIdx.x, t = threadIdx.x;
+// A warp per row t (lanes over i).
+__global__ void __launch_bounds__(256) da_kernel(Bufs w, float* dbeta_part) {
+  const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t sq = (size_t)b * CC * CC;
-  float s = 0.f;
-  const float bt = w.bet[(size_t)b * CC + t];
-  for (int i = 0; i < CC; ++i) {
-    const float d = i < t ? w.dA[sq + t * CC + i] : 0.f;
-    s = fmaf(d, w.Mk[sq + t * CC + i], s);
-    w.dA[sq + t * CC + i] = d * bt;
+  for (int t = warp; t < CC; t += 8) {
+    const float bt = w.bet[(size_t)b * CC + t];
+    float s = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = lane + 32 * hh;
+      const float d = i < t ? w.dA[sq + t * CC + i] : 0.f;
+      s = fmaf(d, w.Mk[sq + t * CC + i], s);
+      w.dA[sq + t * CC + i] = d * bt;
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+    if (lane == 0) dbeta_part[(size_t)b * CC + t] += s;
   }
-  dbeta_part[(size_t)b * CC + t] += s;
 }
 
 // Per chunk: the gradients of the bilinear forms Mq, Mk (every decay ratio formed per pair and channel), then
-// dq, dk, dv, dbeta and dG -> dlog(alpha) (reverse cumulative sum) for the chunk's real rows. Thread c < 128
-// owns channel c: the row forms as it walks t, the column forms accumulated in shared memory by column i.
+// dq, dk, dv, dbeta and dG -> dlog(alpha) (reverse cumulative sum) for the chunk's real rows.
+// For channel c and the pairs (t, i <= t) with R = 2^{G2_tc - G2_ic}:
+//   row forms (by t):    rq[t] = sum_i dMq[t][i] k_ic R,  rk[t] = sum_i dMk[t][i] k_ic R
+//   column form (by i):  cs[i] = sum_t (dMq[t][i] q_tc + dMk[t][i] k_tc) R
+// Threads 0-127 (one per channel) take the row forms, threads 128-255 the column form, each over 8x8 tiles of
+// pairs with the tile's operands in registers. The per-channel columns of G, K and Q sit transposed in shared
+// memory ([c][t], 16-byte groups XOR-swizzled by c so that a quarter warp's float4 loads hit distinct banks).
+constexpr int ASM_T = D * CC;                             // one transposed [128][64] tile
+constexpr int ASSEMBLE_SMEM = (3 * ASM_T + 2 * CC * CC + CC * D) * 4;
+
+__device__ __forceinline__ int swz(int c, int t) { return c * CC + ((((t >> 2) ^ (c & 7))) << 2) + (t & 3); }
+__device__ __forceinline__ void ld8(const float* X, int c, int t0, float v[8]) {
+  const float4 x = *reinterpret_cast<const float4*>(X + swz(c, t0));
+  const float4 y = *reinterpret_cast<const float4*>(X + swz(c, t0 + 4));
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+__device__ __forceinline__ void ld8r(const float* row, float v[8]) {  // 8 consecutive floats (warp-uniform)
+  const float4 x = *reinterpret_cast<const float4*>(row);
+  const float4 y = *reinterpret_cast<const float4*>(row + 4);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+
+// Row forms of tile (rows 8T.., columns 8I..); DIAG: the tile on the diagonal (pairs i > t skipped).
+template <bool DIAG>
+__device__ __forceinline__ void row_tile(const float* Gt_, const float* Kt_, const float* dMq, const float* dMk, int c,
+                                         int T, int I, const float gt[8], float rq[8], float rk[8]) {
+  float gi[8], ki[8];
+  ld8(Gt_, c, 8 * I, gi);
+  ld8(Kt_, c, 8 * I, ki);
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    float mq[8], mk[8];
+    ld8r(dMq + (8 * T + tt) * CC + 8 * I, mq);
+    ld8r(dMk + (8 * T + tt) * CC + 8 * I, mk);
+#pragma unroll
+    for (int ii = 0; ii < 8; ++ii) {
+      if (DIAG && ii > tt) continue;
+      const float x = ex2f(gt[tt] - gi[ii]) * ki[ii];
+      rq[tt] = fmaf(mq[ii], x, rq[tt]);
+      rk[tt] = fmaf(mk[ii], x, rk[tt]);
+    }
+  }
+}
+
+// Column form of tile (rows 8T.., columns 8I..).
+template <bool DIAG>
+__device__ __forceinline__ void col_tile(const float* Gt_, const float* Kt_, const float* Qt_, const float* dMq,
+                                         const float* dMk, int c, int T, int I, const float gi[8], float cs[8]) {
+  float gt[8], qt[8], kt[8];
+  ld8(Gt_, c, 8 * T, gt);
+  ld8(Qt_, c, 8 * T, qt);
+  ld8(Kt_, c, 8 * T, kt);
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    float mq[8], mk[8];
+    ld8r(dMq + (8 * T + tt) * CC + 8 * I, mq);
+    ld8r(dMk + (8 * T + tt) * CC + 8 * I, mk);
+#pragma unroll
+    for (int ii = 0; ii < 8; ++ii) {
+      if (DIAG && ii > tt) continue;
+      const float wv = fmaf(mq[ii], qt[tt], mk[ii] * kt[tt]);
+      cs[ii] = fmaf(ex2f(gt[tt] - gi[ii]), wv, cs[ii]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const float* dbeta_part) {
-  extern __shared__ float sa[];
-  float* Qs = sa;                   // [64][129]
-  float* Ks = Qs + CC * PAD;        // [64][129]
-  float* Gs = Ks + CC * PAD;        // [64][129]
-  float* dMq = Gs + CC * PAD;       // [64][65]
-  float* dMk = dMq + CC * (CC + 1); // [64][65] (Diag(beta) dA)
-  float* Cq = dMk + CC * (CC + 1);  // [64][129]: sum_t dMq[t][i] q_tc R
-  float* Ck = Cq + CC * PAD;        // [64][129]: sum_t dMk[t][i] k_tc R
+  extern __shared__ __align__(16) float sa[];
+  float* Gt_ = sa;                  // [128][64] swizzled: G2 by channel
+  float* Kt_ = Gt_ + ASM_T;         // [128][64] swizzled: k
+  float* Qt_ = Kt_ + ASM_T;         // [128][64] swizzled: q
+  float* dMq = Qt_ + ASM_T;         // [64][64]
+  float* dMk = dMq + CC * CC;       // [64][64] (Diag(beta) dA)
+  float* Cs = dMk + CC * CC;        // [64][128]: the column form
   const int b = blockIdx.x, tid = threadIdx.x;
   int n, j, h, t0, nv;
   chunk_of(a, b, n, j, h, t0, nv);
   const size_t mat = (size_t)b * CC * D, sq = (size_t)b * CC * CC;
-  for (int e = tid; e < CC * D; e += 256) {
-    const int t = e / D, c = e % D;
-    Qs[t * PAD + c] = w.Qf[mat + e];
-    Ks[t * PAD + c] = w.Kf[mat + e];
-    Gs[t * PAD + c] = w.G2[mat + e];
-    Cq[t * PAD + c] = 0.f;
-    Ck[t * PAD + c] = 0.f;
+  // transposed loads: a thread takes 4 consecutive tokens of one channel (coalesced over the channel)
+  for (int e = tid; e < (CC / 4) * D; e += 256) {
+    const int c = e % D, t4 = (e / D) * 4;
+    float g[4], k[4], q[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      g[u] = w.G2[mat + (t4 + u) * D + c];
+      k[u] = w.Kf[mat + (t4 + u) * D + c];
+      q[u] = w.Qf[mat + (t4 + u) * D + c];
+    }
+    *reinterpret_cast<float4*>(Gt_ + swz(c, t4)) = make_float4(g[0], g[1], g[2], g[3]);
+    *reinterpret_cast<float4*>(Kt_ + swz(c, t4)) = make_float4(k[0], k[1], k[2], k[3]);
+    *reinterpret_cast<float4*>(Qt_ + swz(c, t4)) = make_float4(q[0], q[1], q[2], q[3]);
   }
-  for (int e = tid; e < CC * CC; e += 256) {
-    dMq[(e / CC) * (CC + 1) + e % CC] = w.dMq[sq + e];
-    dMk[(e / CC) * (CC + 1) + e % CC] = w.dA[sq + e];
+  for (int e = tid; e < CC * CC / 4; e += 256) {
+    reinterpret_cast<float4*>(dMq)[e] = reinterpret_cast<const float4*>(w.dMq + sq)[e];
+    reinterpret_cast<float4*>(dMk)[e] = reinterpret_cast<const float4*>(w.dA + sq)[e];
+  }
+  __syncthreads();
+  float dkt_kt = 0.f;  // row threads: sum_t dKT * KT, the share of G_last
+  if (tid < D) {
+    const int c = tid;
+    float gl[8];
+    ld8(Gt_, c, CC - 8, gl);
+    for (int T = 0; T < CC / 8; ++T) {
+      float gt[8], rq[8], rk[8];
+      ld8(Gt_, c, 8 * T, gt);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) rq[u] = rk[u] = 0.f;
+      for (int I = 0; I < T; ++I) row_tile<false>(Gt_, Kt_, dMq, dMk, c, T, I, gt, rq, rk);
+      row_tile<true>(Gt_, Kt_, dMq, dMk, c, T, T, gt, rq, rk);
+      float qt[8], kt[8];
+      ld8(Qt_, c, 8 * T, qt);
+      ld8(Kt_, c, 8 * T, kt);
+#pragma unroll
+      for (int tt = 0; tt < 8; ++tt) {
+        const int t = 8 * T + tt;
+        const size_t e = mat + t * D + c;
+        const float gam_t = ex2f(gt[tt]), kts = ex2f(gl[7] - gt[tt]);
+        const float dqg = w.dQG[e], dkg = w.dKG[e], dkt = w.dKT[e];
+        // dk's and dG's row shares, completed by the column form below
+        w.dKG[e] = rk[tt] + dkg * gam_t + dkt * kts;
+        const float ktv = kt[tt] * kts;
+        w.dQG[e] = qt[tt] * rq[tt] + kt[tt] * rk[tt] + dqg * qt[tt] * gam_t + dkg * kt[tt] * gam_t - dkt * ktv;
+        dkt_kt = fmaf(dkt, ktv, dkt_kt);
+        if (t < nv) a.dq[((n * a.T + t0 + t) * a.H + h) * D + c] = rq[tt] + dqg * gam_t;
+      }
+    }
+  } else {
+    const int c = tid - D;
+    for (int I = 0; I < CC / 8; ++I) {
+      float gi[8], cs[8];
+      ld8(Gt_, c, 8 * I, gi);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) cs[u] = 0.f;
+      col_tile<true>(Gt_, Kt_, Qt_, dMq, dMk, c, I, I, gi, cs);
+      for (int T = I + 1; T < CC / 8; ++T) col_tile<false>(Gt_, Kt_, Qt_, dMq, dMk, c, T, I, gi, cs);
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) Cs[(8 * I + ii) * D + c] = cs[ii];
+    }
   }
   __syncthreads();
   if (tid < D) {
+    // the column form into dk and dG, then dG -> dlog(alpha) by a reverse cumulative sum
     const int c = tid;
-    const float gl = Gs[(CC - 1) * PAD + c];
-    float dkt_kt = 0.f;  // sum_t dKT * KT, the share of G_last
-    for (int t = 0; t < CC; ++t) {
-      const float gt = Gs[t * PAD + c], qt = Qs[t * PAD + c], kt = Ks[t * PAD + c];
-      float rq = 0.f, rk = 0.f;
-      for (int i = 0; i <= t; ++i) {
-        const float r = ex2f(gt - Gs[i * PAD + c]);  // e^{G_t - G_i} <= 1 (G is non-increasing)
-        const float ki = Ks[i * PAD + c];
-        const float mq = dMq[t * (CC + 1) + i], mk = dMk[t * (CC + 1) + i];
-        rq = fmaf(mq * ki, r, rq);
-        rk = fmaf(mk * ki, r, rk);
-        Cq[i * PAD + c] = fmaf(mq * qt, r, Cq[i * PAD + c]);
-        Ck[i * PAD + c] = fmaf(mk * kt, r, Ck[i * PAD + c]);
-      }
-      const size_t e = mat + t * D + c;
-      const float gam_t = ex2f(gt), kts = ex2f(gl - gt);
-      const float dqg = w.dQG[e], dkg = w.dKG[e], dkt = w.dKT[e];
-      const float dq = rq + dqg * gam_t;
-      // dk's row share and dG's row share, completed by the column shares below
-      w.dKG[e] = rk + dkg * gam_t + dkt * kts;
-      const float ktv = kt * kts;
-      w.dQG[e] = qt * rq + kt * rk + dqg * qt * gam_t + dkg * kt * gam_t - dkt * ktv;
-      dkt_kt = fmaf(dkt, ktv, dkt_kt);
-      if (t < nv) a.dq[((n * a.T + t0 + t) * a.H + h) * D + c] = dq;
-    }
-    // column shares, dk, and dG -> dlog(alpha) by a reverse cumulative sum
     float acc = dkt_kt + w.dgC[(size_t)b * D + c] * w.gam[(size_t)b * D + c];  // only G_last's share
+#pragma unroll 4
     for (int t = CC - 1; t >= 0; --t) {
       const size_t e = mat + t * D + c;
-      const float kt = Ks[t * PAD + c], cq = Cq[t * PAD + c], ck = Ck[t * PAD + c];
-      const float dk = w.dKG[e] + cq + ck;
-      const float dg = w.dQG[e] - kt * cq - kt * ck;
-      acc += dg;  // sum_{r >= t} dG[r]
+      const float kt = Kt_[swz(c, t)], cs = Cs[t * D + c];
+      const float dk = w.dKG[e] + cs;
+      acc += w.dQG[e] - kt * cs;  // sum_{r >= t} dG[r]
       if (t < nv) {
         const size_t o = ((n * a.T + t0 + t) * a.H + h) * D + c;
         a.dk[o] = dk;
@@ -503,15 +664,15 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
 
   // 2. per-chunk preparation, Mq and Mk, T and TB
   prep_kernel<<<NB, 256, 0, s>>>(a, w);
-  const int pair_smem = 3 * CC * PAD * 4;
+  const int pair_smem = PAIR_SMEM;
   {
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(configured.load() & (1ull << dev))) {
-      const int dsm = (CC * (CC + 1) + 3 * CC * PAD + CC * VS + D * VS + CC * VS + D) * 4;
-      const int asm_ = (3 * CC * PAD + 2 * CC * (CC + 1) + 2 * CC * PAD) * 4;
+      const int dsm = DSTATE_SMEM;
+      const int asm_ = ASSEMBLE_SMEM;
       if ((e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pair_smem)) != cudaSuccess ||
           (e = cudaFuncSetAttribute(dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm)) != cudaSuccess ||
           (e = cudaFuncSetAttribute(assemble_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, asm_)) != cudaSuccess)
@@ -547,16 +708,21 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
     *cublas_status = (int)cs;
     return cudaErrorUnknown;
   }
-  // 4. the reverse recurrence over chunks for dS
+  // 4. the dO terms of the recurrence (X1 = Mq^T dO into dU, Y = QG^T dO - W^T X1 into dS_C), then the
+  //    reverse recurrence over chunks for dS (completing dU = X1 + KT dS_C)
+  G(true, false, CC, D, CC, 1.f, w.Mq, CC, s64, w.dOf, D, s128, 0.f, w.dU, D, s128);
+  G(true, false, D, D, CC, 1.f, w.QG, D, s128, w.dOf, D, s128, 0.f, w.dSC, D, sst);
+  G(true, false, D, D, CC, -1.f, w.W, D, s128, w.dU, D, s128, 1.f, w.dSC, D, sst);
+  if (cs != CUBLAS_STATUS_SUCCESS) {
+    *cublas_status = (int)cs;
+    return cudaErrorUnknown;
+  }
   {
-    const int dsm = (CC * (CC + 1) + 3 * CC * PAD + CC * VS + D * VS + CC * VS + D) * 4;
-    dstate_kernel<<<dim3((unsigned)(B * H), D / VS), 256, dsm, s>>>(a, w);
+    dstate_kernel<<<dim3((unsigned)(B * H), D / VS), 256, DSTATE_SMEM, s>>>(a, w);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // 5. dU = Mq^T dO + KT dS_C; dMq = dO U^T; dQG = dO S0^T; dKT = U dS_C^T; dW = -dU S0^T;
-  //    dTB = dU V^T + dW KG^T; dV = TB^T dU; dKG = TB^T dW; X = T^T dT; dA = -X T^T
-  G(true, false, CC, D, CC, 1.f, w.Mq, CC, s64, w.dOf, D, s128, 0.f, w.dU, D, s128);
-  G(false, false, CC, D, D, 1.f, w.KT, D, s128, w.dSC, D, sst, 1.f, w.dU, D, s128);
+  // 5. dMq = dO U^T; dQG = dO S0^T; dKT = U dS_C^T; dW = -dU S0^T; dTB = dU V^T + dW KG^T; dV = TB^T dU;
+  //    dKG = TB^T dW; X = T^T dT; dA = -X T^T
   G(false, true, CC, CC, D, 1.f, w.dOf, D, s128, w.U, D, s128, 0.f, w.dMq, CC, s64);
   G(false, true, CC, D, D, 1.f, w.dOf, D, s128, w.S0, D, sst, 0.f, w.dQG, D, s128);
   G(false, true, CC, D, D, 1.f, w.U, D, s128, w.dSC, D, sst, 0.f, w.dKT, D, s128);
@@ -579,11 +745,8 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
     return cudaErrorUnknown;
   }
   std::swap(w.dA, w.X);  // dA now names the result
-  da_kernel<<<NB, 64, 0, s>>>(w, dbeta_part);
-  {
-    const int asm_ = (3 * CC * PAD + 2 * CC * (CC + 1) + 2 * CC * PAD) * 4;
-    assemble_kernel<<<NB, 256, asm_, s>>>(a, w, dbeta_part);
-  }
+  da_kernel<<<NB, 256, 0, s>>>(w, dbeta_part);
+  assemble_kernel<<<NB, 256, ASSEMBLE_SMEM, s>>>(a, w, dbeta_part);
   return cudaGetLastError();
 }
 
