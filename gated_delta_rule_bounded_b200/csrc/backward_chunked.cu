@@ -52,7 +52,8 @@ __device__ __forceinline__ float ex2f(float x) {
 }
 
 struct Bufs {
-  float *Qf, *Kf, *Vf, *dOf, *G2, *QG, *KG, *KT, *gam, *bet;  // [NB][64][128] (gam [NB][128], bet [NB][64])
+  float *Qf, *Kf, *Vf, *dOf, *G2, *QG, *KG, *KT, *gam, *bet;  // [NB][64][128] (KT [NB][128][64], gam [NB][128],
+                                                              // bet [NB][64])
   float *Mq, *Mk, *Tm, *TB;                                   // [NB][64][64]
   float *W, *U, *dU, *dQG, *dKT, *dW, *dKG, *dV;              // [NB][64][128]
   float *S0, *dSC;                                            // [NB][128][128]
@@ -84,8 +85,10 @@ __device__ __forceinline__ void chunk_of(const BwdC& a, int b, int& n, int& j, i
 }
 
 // fp32 copies of the chunk's q, k, v, dO (zero past the end), the log2 cumulative decay (per-token floor at
-// -126, zero past the end: alpha = 1), Q*Gamma, K*Gamma, K*gamma_C/Gamma, gamma_C and beta (zero past the end).
-// Threads 0-127 walk the tokens for channel c (the cumulative sum), threads 128-255 copy v and dO.
+// -126, zero past the end: alpha = 1), Q*Gamma, K*Gamma, K*gamma_C/Gamma (transposed, [c][t]), gamma_C and beta
+// (zero past the end).
+// Threads 0-127 walk the tokens for channel c (the cumulative sum), threads 128-255 copy v and dO; each takes
+// 8 tokens' loads ahead of their stores.
 __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
   const int b = blockIdx.x, tid = threadIdx.x;
   int n, j, h, t0, nv;
@@ -94,41 +97,57 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
   if (tid < D) {
     const int c = tid;
     float run = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < CC; ++t) {
-      const bool in = t < nv;
-      const int64_t tt = t0 + t;
-      float l = 0.f, qv = 0.f, kv = 0.f;
-      if (in) {
-        const float x = a.gate[n * a.gs[0] + tt * a.gs[1] + h * a.gs[2] + c];
-        l = fmaxf(a.gate_log ? x * LOG2E_F : log2f(x), FLOOR2);
-        qv = __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[n * a.qs[0] + tt * a.qs[1] + h * a.qs[2] + c]);
-        kv = __bfloat162float(static_cast<const __nv_bfloat16*>(a.k)[n * a.ks[0] + tt * a.ks[1] + h * a.ks[2] + c]);
+    for (int t8 = 0; t8 < CC; t8 += 8) {
+      float x[8], qv[8], kv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t tt = t0 + t8 + u;
+        const bool in = t8 + u < nv;
+        x[u] = in ? a.gate[n * a.gs[0] + tt * a.gs[1] + h * a.gs[2] + c] : 0.f;
+        qv[u] = in ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[n * a.qs[0] + tt * a.qs[1] + h * a.qs[2] + c]) : 0.f;
+        kv[u] = in ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.k)[n * a.ks[0] + tt * a.ks[1] + h * a.ks[2] + c]) : 0.f;
       }
-      run += l;
-      const float gm = ex2f(run);
-      w.G2[mat + t * D + c] = run;
-      w.Qf[mat + t * D + c] = qv;
-      w.Kf[mat + t * D + c] = kv;
-      w.QG[mat + t * D + c] = qv * gm;
-      w.KG[mat + t * D + c] = kv * gm;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const size_t e = mat + (t8 + u) * D + c;
+        run += t8 + u < nv ? fmaxf(a.gate_log ? x[u] * LOG2E_F : log2f(x[u]), FLOOR2) : 0.f;
+        const float gm = ex2f(run);
+        w.G2[e] = run;
+        w.Qf[e] = qv[u];
+        w.Kf[e] = kv[u];
+        w.QG[e] = qv[u] * gm;
+        w.KG[e] = kv[u] * gm;
+      }
     }
     w.gam[(size_t)b * D + c] = ex2f(run);
-#pragma unroll 8
-    for (int t = 0; t < CC; ++t) w.KT[mat + t * D + c] = w.Kf[mat + t * D + c] * ex2f(run - w.G2[mat + t * D + c]);
+    for (int t8 = 0; t8 < CC; t8 += 8) {  // KT transposed: [c][t]
+      float kf[8], g2[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        kf[u] = w.Kf[mat + (t8 + u) * D + c];
+        g2[u] = w.G2[mat + (t8 + u) * D + c];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) kf[u] *= ex2f(run - g2[u]);
+      *reinterpret_cast<float4*>(w.KT + mat + c * CC + t8) = make_float4(kf[0], kf[1], kf[2], kf[3]);
+      *reinterpret_cast<float4*>(w.KT + mat + c * CC + t8 + 4) = make_float4(kf[4], kf[5], kf[6], kf[7]);
+    }
   } else {
     const int c = tid - D;
-#pragma unroll 8
-    for (int t = 0; t < CC; ++t) {
-      const bool in = t < nv;
-      const int64_t tt = t0 + t;
-      float vv = 0.f, dov = 0.f;
-      if (in) {
-        vv = __bfloat162float(static_cast<const __nv_bfloat16*>(a.v)[n * a.vs[0] + tt * a.vs[1] + h * a.vs[2] + c]);
-        dov = a.d_o[((n * a.T + tt) * a.H + h) * D + c];
+    for (int t8 = 0; t8 < CC; t8 += 8) {
+      float vv[8], dov[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t tt = t0 + t8 + u;
+        const bool in = t8 + u < nv;
+        vv[u] = in ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.v)[n * a.vs[0] + tt * a.vs[1] + h * a.vs[2] + c]) : 0.f;
+        dov[u] = in ? a.d_o[((n * a.T + tt) * a.H + h) * D + c] : 0.f;
       }
-      w.Vf[mat + t * D + c] = vv;
-      w.dOf[mat + t * D + c] = dov;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        w.Vf[mat + (t8 + u) * D + c] = vv[u];
+        w.dOf[mat + (t8 + u) * D + c] = dov[u];
+      }
     }
   }
   if (tid < CC) {
@@ -236,111 +255,140 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // The dO terms are independent of the recurrence and come in precomputed: X1 = Mq^T dO in dU and
 // Y = QG^T dO - W^T X1 in dS_C's place. Per chunk, from the last:
 //   dS_C = dS;  dU = X1 + KT dS;  dS <- Diag(gamma_C) dS + Y - W^T (KT dS),
-// with dS_C and dU written over Y and X1 and dS0 of the first chunk to ds0. A thread holds dS[c][16 columns];
-// KT and W of the next chunk are prefetched (cp.async) into the other half of a double buffer, rows padded to
-// 132 floats (16-byte aligned, rows 4 banks apart).
+// with dS_C and dU written over Y and X1 and dS0 of the first chunk to ds0. A thread holds a 4x4 block of dS;
+// KT dS is split over the channel index between the two halves of the CTA (4x4 blocks each), so that every
+// 16 FMAs take two 16-byte shared loads. Every operand of the next chunk (KT^T, W, the slices of Y and X1,
+// gamma_C) is prefetched with cp.async into the other half of a double buffer.
 constexpr int VS = 32;
-constexpr int P4 = 132;
-constexpr int DS_OPS = 2 * CC * P4;  // KT and W of one chunk
-constexpr int DSTATE_SMEM = (2 * DS_OPS + D * VS + CC * VS + D) * 4;
+constexpr int DS_KT = 0, DS_W = D * CC, DS_Y = 2 * D * CC, DS_X1 = DS_Y + D * VS, DS_G = DS_X1 + CC * VS;
+constexpr int DS_OPS = DS_G + D;  // one chunk's operands
+constexpr int DSTATE_SMEM = (2 * DS_OPS + D * VS + 2 * CC * VS) * 4;
 
-__device__ __forceinline__ void dstate_prefetch(const Bufs& w, size_t mat, float* dst, int tid) {
-  const float* kt = w.KT + mat;
-  const float* wm = w.W + mat;
+__device__ __forceinline__ void dstate_prefetch(const Bufs& w, int b, int vsl, float* dst, int tid) {
+  const size_t mat = (size_t)b * CC * D, st = (size_t)b * D * D;
+  const float* kt = w.KT + mat;  // [128][64]
+  const float* wm = w.W + mat;   // [64][128]
 #pragma unroll
   for (int e = tid; e < CC * D / 4; e += 256) {
-    const int t = e >> 5, c4 = e & 31;
-    cp_async16(dst + t * P4 + 4 * c4, kt + 4 * e);
-    cp_async16(dst + CC * P4 + t * P4 + 4 * c4, wm + 4 * e);
+    cp_async16(dst + DS_KT + 4 * e, kt + 4 * e);
+    cp_async16(dst + DS_W + 4 * e, wm + 4 * e);
   }
+#pragma unroll
+  for (int e = tid; e < D * VS / 4; e += 256) {  // Y[c][32 s ..]
+    const int c = e >> 3, q = e & 7;
+    cp_async16(dst + DS_Y + 4 * e, w.dSC + st + (size_t)c * D + vsl * VS + 4 * q);
+  }
+#pragma unroll
+  for (int e = tid; e < CC * VS / 4; e += 256) {  // X1[i][32 s ..]
+    const int i = e >> 3, q = e & 7;
+    cp_async16(dst + DS_X1 + 4 * e, w.dU + mat + (size_t)i * D + vsl * VS + 4 * q);
+  }
+  if (tid < D / 4) cp_async16(dst + DS_G + 4 * tid, w.gam + (size_t)b * D + 4 * tid);
   cp_async_commit();
+}
+
+__device__ __forceinline__ void unpack4(const float4 v, float o[4]) {
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
 }
 
 __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
   extern __shared__ __align__(16) float sd[];
   float* dSs = sd + 2 * DS_OPS;   // [128][VS]
-  float* dUs = dSs + D * VS;      // [64][VS]: KT dS
-  float* gm = dUs + CC * VS;      // [128]
+  float* dUa = dSs + D * VS;      // [64][VS]: KT dS (channels 0-63, then the sum)
+  float* dUb = dUa + CC * VS;     // [64][VS]: KT dS (channels 64-127)
   const int tid = threadIdx.x;
   const int nh = blockIdx.x, vsl = blockIdx.y;
   const int n = nh / a.H, h = nh % a.H;
-  const int c = tid >> 1, v0 = (tid & 1) * 16;   // this thread's dS[c][v0 .. v0 + 15] of the slice
-  const int vg = vsl * VS + v0;                  // global value column of v0
-  const int i = tid >> 2, vq = (tid & 3) * 8;    // this thread's dU[i][vq .. vq + 7] of the slice
-  float dS[16];
+  const int c0 = 4 * (tid >> 3), v0 = 4 * (tid & 7);   // this thread's dS[c0 .. c0 + 3][v0 .. v0 + 3] of the slice
+  const int half = tid >> 7, i0 = 4 * ((tid & 127) >> 3);  // KT dS: rows i0 .. i0 + 3, channels of this half
+  const int vg = vsl * VS + v0;
+  float dS[4][4];
   const size_t shead = ((size_t)n * a.H + h) * D * D;
 #pragma unroll
-  for (int u = 0; u < 16; ++u) dS[u] = a.d_sf ? a.d_sf[shead + (size_t)c * D + vg + u] : 0.f;
-  dstate_prefetch(w, (size_t)((n * a.ncps + a.ncps - 1) * a.H + h) * CC * D, sd + ((a.ncps - 1) & 1) * DS_OPS, tid);
+  for (int r = 0; r < 4; ++r) {
+    const float4 x = a.d_sf ? *reinterpret_cast<const float4*>(a.d_sf + shead + (size_t)(c0 + r) * D + vg)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    unpack4(x, dS[r]);
+  }
+  dstate_prefetch(w, (n * a.ncps + a.ncps - 1) * a.H + h, vsl, sd + ((a.ncps - 1) & 1) * DS_OPS, tid);
   for (int j = a.ncps - 1; j >= 0; --j) {
     const int b = (n * a.ncps + j) * a.H + h;
     const size_t mat = (size_t)b * CC * D, st = (size_t)b * D * D;
-    const float* KTs = sd + (j & 1) * DS_OPS;
-    const float* Ws = KTs + CC * P4;
-    float y[16];
-    float* dsc = w.dSC + st + (size_t)c * D + vg;
+    const float* buf = sd + (j & 1) * DS_OPS;
 #pragma unroll
-    for (int u = 0; u < 16; u += 4) {
-      const float4 t4 = *reinterpret_cast<const float4*>(dsc + u);
-      y[u] = t4.x; y[u + 1] = t4.y; y[u + 2] = t4.z; y[u + 3] = t4.w;
-      const float4 x = make_float4(dS[u], dS[u + 1], dS[u + 2], dS[u + 3]);
-      *reinterpret_cast<float4*>(dsc + u) = x;
-      *reinterpret_cast<float4*>(dSs + c * VS + v0 + u) = x;
-    }
-    float* du = w.dU + mat + (size_t)i * D + vsl * VS + vq;
-    const float4 x1a = *reinterpret_cast<const float4*>(du);
-    const float4 x1b = *reinterpret_cast<const float4*>(du + 4);
-    if (tid < D) gm[tid] = w.gam[(size_t)b * D + tid];
+    for (int r = 0; r < 4; ++r)
+      *reinterpret_cast<float4*>(dSs + (c0 + r) * VS + v0) = make_float4(dS[r][0], dS[r][1], dS[r][2], dS[r][3]);
     if (j > 0) {
-      dstate_prefetch(w, (size_t)((n * a.ncps + j - 1) * a.H + h) * CC * D, sd + ((j - 1) & 1) * DS_OPS, tid);
+      dstate_prefetch(w, b - a.H, vsl, sd + ((j - 1) & 1) * DS_OPS, tid);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
-    __syncthreads();
-    // KT dS: a thread takes row i, 8 columns
-    {
-      float acc[8];
+    __syncthreads();  // this chunk's operands have landed (Y and X1 among them: their places may be written)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-#pragma unroll 4
-      for (int cc = 0; cc < D; ++cc) {
-        const float kt = KTs[i * P4 + cc];
-        const float4 s0 = *reinterpret_cast<const float4*>(dSs + cc * VS + vq);
-        const float4 s1 = *reinterpret_cast<const float4*>(dSs + cc * VS + vq + 4);
-        acc[0] = fmaf(kt, s0.x, acc[0]); acc[1] = fmaf(kt, s0.y, acc[1]); acc[2] = fmaf(kt, s0.z, acc[2]);
-        acc[3] = fmaf(kt, s0.w, acc[3]); acc[4] = fmaf(kt, s1.x, acc[4]); acc[5] = fmaf(kt, s1.y, acc[5]);
-        acc[6] = fmaf(kt, s1.z, acc[6]); acc[7] = fmaf(kt, s1.w, acc[7]);
+    for (int r = 0; r < 4; ++r)
+      *reinterpret_cast<float4*>(w.dSC + st + (size_t)(c0 + r) * D + vg) =
+          make_float4(dS[r][0], dS[r][1], dS[r][2], dS[r][3]);
+    {  // KT dS over this half's 64 channels
+      const float* KTs = buf + DS_KT;
+      float acc[4][4] = {};
+#pragma unroll 8
+      for (int cc = 64 * half; cc < 64 * half + 64; ++cc) {
+        float kv[4], sv[4];
+        unpack4(*reinterpret_cast<const float4*>(KTs + cc * CC + i0), kv);
+        unpack4(*reinterpret_cast<const float4*>(dSs + cc * VS + v0), sv);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[r][u] = fmaf(kv[r], sv[u], acc[r][u]);
       }
-      *reinterpret_cast<float4*>(dUs + i * VS + vq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      *reinterpret_cast<float4*>(dUs + i * VS + vq + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-      *reinterpret_cast<float4*>(du) = make_float4(x1a.x + acc[0], x1a.y + acc[1], x1a.z + acc[2], x1a.w + acc[3]);
-      *reinterpret_cast<float4*>(du + 4) = make_float4(x1b.x + acc[4], x1b.y + acc[5], x1b.z + acc[6], x1b.w + acc[7]);
+      float* dst = half ? dUb : dUa;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        *reinterpret_cast<float4*>(dst + (i0 + r) * VS + v0) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
     }
     __syncthreads();
-    // dS <- gamma_C[c] dS[c][v] + Y[c][v] - sum_t W[t][c] (KT dS)[t][v]
-    {
-      const float g = gm[c];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) dS[u] = fmaf(g, dS[u], y[u]);
-#pragma unroll 4
+    for (int q = tid; q < CC * VS / 4; q += 256) {  // the two halves summed; dU = X1 + KT dS
+      const int i = q >> 3, v = 4 * (q & 7);
+      const float4 x = *reinterpret_cast<const float4*>(dUa + i * VS + v);
+      const float4 y = *reinterpret_cast<const float4*>(dUb + i * VS + v);
+      const float4 z = make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
+      *reinterpret_cast<float4*>(dUa + i * VS + v) = z;
+      const float4 x1 = *reinterpret_cast<const float4*>(buf + DS_X1 + i * VS + v);
+      *reinterpret_cast<float4*>(w.dU + mat + (size_t)i * D + vsl * VS + v) =
+          make_float4(x1.x + z.x, x1.y + z.y, x1.z + z.z, x1.w + z.w);
+    }
+    __syncthreads();
+    {  // dS <- gamma_C[c] dS[c][v] + Y[c][v] - sum_t W[t][c] (KT dS)[t][v]
+      const float* Ws = buf + DS_W;
+      float g[4];
+      unpack4(*reinterpret_cast<const float4*>(buf + DS_G + c0), g);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float y[4];
+        unpack4(*reinterpret_cast<const float4*>(buf + DS_Y + (c0 + r) * VS + v0), y);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dS[r][u] = fmaf(g[r], dS[r][u], y[u]);
+      }
+#pragma unroll 8
       for (int t = 0; t < CC; ++t) {
-        const float wv = Ws[t * P4 + c];
+        float wv[4], ev[4];
+        unpack4(*reinterpret_cast<const float4*>(Ws + t * D + c0), wv);
+        unpack4(*reinterpret_cast<const float4*>(dUa + t * VS + v0), ev);
 #pragma unroll
-        for (int u = 0; u < 16; u += 4) {
-          const float4 e = *reinterpret_cast<const float4*>(dUs + t * VS + v0 + u);
-          dS[u] = fmaf(-wv, e.x, dS[u]);
-          dS[u + 1] = fmaf(-wv, e.y, dS[u + 1]);
-          dS[u + 2] = fmaf(-wv, e.z, dS[u + 2]);
-          dS[u + 3] = fmaf(-wv, e.w, dS[u + 3]);
-        }
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dS[r][u] = fmaf(-wv[r], ev[u], dS[r][u]);
       }
     }
     __syncthreads();  // the buffer just read is the next prefetch's target
   }
   if (a.ds0) {
 #pragma unroll
-    for (int u = 0; u < 16; ++u) a.ds0[shead + (size_t)c * D + vg + u] = dS[u];
+    for (int r = 0; r < 4; ++r)
+      *reinterpret_cast<float4*>(a.ds0 + shead + (size_t)(c0 + r) * D + vg) =
+          make_float4(dS[r][0], dS[r][1], dS[r][2], dS[r][3]);
   }
 }
 
@@ -419,46 +467,94 @@ __device__ __forceinline__ void ld8r(const float* row, float v[8]) {  // 8 conse
   v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
 }
 
-// Row forms of tile (rows 8T.., columns 8I..); DIAG: the tile on the diagonal (pairs i > t skipped).
-template <bool DIAG>
-__device__ __forceinline__ void row_tile(const float* Gt_, const float* Kt_, const float* dMq, const float* dMk, int c,
-                                         int T, int I, const float gt[8], float rq[8], float rk[8]) {
-  float gi[8], ki[8];
+// Tiles below the diagonal (I < T) put every row t after every column i, so with the reference G_ref = G2 at
+// the block's last column, 2^{G_t - G_i} = 2^{G_t - G_ref} 2^{G_ref - G_i} with both factors <= 1 (a factor
+// that flushes to zero bounds the exact ratio, which is then below 2^-126 as well): 16 exponentials per tile and
+// channel instead of 64. The diagonal tiles form every ratio directly.
+
+// Row forms of tile (rows 8T.., columns 8I..), I < T.
+__device__ __forceinline__ void row_tile_off(const float* Gt_, const float* Kt_, const float* dMq, const float* dMk,
+                                             int c, int T, int I, const float gt[8], float rq[8], float rk[8]) {
+  float gi[8], kb[8];
   ld8(Gt_, c, 8 * I, gi);
-  ld8(Kt_, c, 8 * I, ki);
+  ld8(Kt_, c, 8 * I, kb);
+  const float gref = gi[7];
+#pragma unroll
+  for (int ii = 0; ii < 8; ++ii) kb[ii] *= ex2f(gref - gi[ii]);
 #pragma unroll
   for (int tt = 0; tt < 8; ++tt) {
     float mq[8], mk[8];
     ld8r(dMq + (8 * T + tt) * CC + 8 * I, mq);
     ld8r(dMk + (8 * T + tt) * CC + 8 * I, mk);
+    float sq = 0.f, sk = 0.f;
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
-      if (DIAG && ii > tt) continue;
-      const float x = ex2f(gt[tt] - gi[ii]) * ki[ii];
+      sq = fmaf(mq[ii], kb[ii], sq);
+      sk = fmaf(mk[ii], kb[ii], sk);
+    }
+    const float at = ex2f(gt[tt] - gref);
+    rq[tt] = fmaf(at, sq, rq[tt]);
+    rk[tt] = fmaf(at, sk, rk[tt]);
+  }
+}
+
+// Row forms of the diagonal tile T.
+__device__ __forceinline__ void row_tile_diag(const float* Gt_, const float* Kt_, const float* dMq, const float* dMk,
+                                              int c, int T, const float gt[8], float rq[8], float rk[8]) {
+  float ki[8];
+  ld8(Kt_, c, 8 * T, ki);
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    float mq[8], mk[8];
+    ld8r(dMq + (8 * T + tt) * CC + 8 * T, mq);
+    ld8r(dMk + (8 * T + tt) * CC + 8 * T, mk);
+#pragma unroll
+    for (int ii = 0; ii <= tt; ++ii) {
+      const float x = ex2f(gt[tt] - gt[ii]) * ki[ii];
       rq[tt] = fmaf(mq[ii], x, rq[tt]);
       rk[tt] = fmaf(mk[ii], x, rk[tt]);
     }
   }
 }
 
-// Column form of tile (rows 8T.., columns 8I..).
-template <bool DIAG>
-__device__ __forceinline__ void col_tile(const float* Gt_, const float* Kt_, const float* Qt_, const float* dMq,
-                                         const float* dMk, int c, int T, int I, const float gi[8], float cs[8]) {
-  float gt[8], qt[8], kt[8];
+// Column form of tile (rows 8T.., columns 8I..), I < T, without the column factor 2^{G_ref - G_i}.
+__device__ __forceinline__ void col_tile_off(const float* Gt_, const float* Kt_, const float* Qt_, const float* dMq,
+                                             const float* dMk, int c, int T, int I, float gref, float cs[8]) {
+  float gt[8], aq[8], ak[8];
   ld8(Gt_, c, 8 * T, gt);
-  ld8(Qt_, c, 8 * T, qt);
-  ld8(Kt_, c, 8 * T, kt);
+  ld8(Qt_, c, 8 * T, aq);
+  ld8(Kt_, c, 8 * T, ak);
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    const float e = ex2f(gt[tt] - gref);
+    aq[tt] *= e;
+    ak[tt] *= e;
+  }
 #pragma unroll
   for (int tt = 0; tt < 8; ++tt) {
     float mq[8], mk[8];
     ld8r(dMq + (8 * T + tt) * CC + 8 * I, mq);
     ld8r(dMk + (8 * T + tt) * CC + 8 * I, mk);
 #pragma unroll
-    for (int ii = 0; ii < 8; ++ii) {
-      if (DIAG && ii > tt) continue;
+    for (int ii = 0; ii < 8; ++ii) cs[ii] = fmaf(mq[ii], aq[tt], fmaf(mk[ii], ak[tt], cs[ii]));
+  }
+}
+
+// Column form of the diagonal tile I.
+__device__ __forceinline__ void col_tile_diag(const float* Kt_, const float* Qt_, const float* dMq, const float* dMk,
+                                              int c, int I, const float gi[8], float cs[8]) {
+  float qt[8], kt[8];
+  ld8(Qt_, c, 8 * I, qt);
+  ld8(Kt_, c, 8 * I, kt);
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    float mq[8], mk[8];
+    ld8r(dMq + (8 * I + tt) * CC + 8 * I, mq);
+    ld8r(dMk + (8 * I + tt) * CC + 8 * I, mk);
+#pragma unroll
+    for (int ii = 0; ii <= tt; ++ii) {
       const float wv = fmaf(mq[ii], qt[tt], mk[ii] * kt[tt]);
-      cs[ii] = fmaf(ex2f(gt[tt] - gi[ii]), wv, cs[ii]);
+      cs[ii] = fmaf(ex2f(gi[tt] - gi[ii]), wv, cs[ii]);
     }
   }
 }
@@ -476,6 +572,7 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
   chunk_of(a, b, n, j, h, t0, nv);
   const size_t mat = (size_t)b * CC * D, sq = (size_t)b * CC * CC;
   // transposed loads: a thread takes 4 consecutive tokens of one channel (coalesced over the channel)
+#pragma unroll 2
   for (int e = tid; e < (CC / 4) * D; e += 256) {
     const int c = e % D, t4 = (e / D) * 4;
     float g[4], k[4], q[4];
@@ -500,12 +597,18 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
     float gl[8];
     ld8(Gt_, c, CC - 8, gl);
     for (int T = 0; T < CC / 8; ++T) {
-      float gt[8], rq[8], rk[8];
+      float gt[8], rq[8], rk[8], dqg[8], dkg[8], dkt[8];
       ld8(Gt_, c, 8 * T, gt);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) rq[u] = rk[u] = 0.f;
-      for (int I = 0; I < T; ++I) row_tile<false>(Gt_, Kt_, dMq, dMk, c, T, I, gt, rq, rk);
-      row_tile<true>(Gt_, Kt_, dMq, dMk, c, T, T, gt, rq, rk);
+      for (int u = 0; u < 8; ++u) {  // the epilogue's operands, loaded ahead of the tiles
+        const size_t e = mat + (8 * T + u) * D + c;
+        dqg[u] = w.dQG[e];
+        dkg[u] = w.dKG[e];
+        dkt[u] = w.dKT[e];
+        rq[u] = rk[u] = 0.f;
+      }
+      for (int I = 0; I < T; ++I) row_tile_off(Gt_, Kt_, dMq, dMk, c, T, I, gt, rq, rk);
+      row_tile_diag(Gt_, Kt_, dMq, dMk, c, T, gt, rq, rk);
       float qt[8], kt[8];
       ld8(Qt_, c, 8 * T, qt);
       ld8(Kt_, c, 8 * T, kt);
@@ -514,26 +617,26 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
         const int t = 8 * T + tt;
         const size_t e = mat + t * D + c;
         const float gam_t = ex2f(gt[tt]), kts = ex2f(gl[7] - gt[tt]);
-        const float dqg = w.dQG[e], dkg = w.dKG[e], dkt = w.dKT[e];
         // dk's and dG's row shares, completed by the column form below
-        w.dKG[e] = rk[tt] + dkg * gam_t + dkt * kts;
+        w.dKG[e] = rk[tt] + dkg[tt] * gam_t + dkt[tt] * kts;
         const float ktv = kt[tt] * kts;
-        w.dQG[e] = qt[tt] * rq[tt] + kt[tt] * rk[tt] + dqg * qt[tt] * gam_t + dkg * kt[tt] * gam_t - dkt * ktv;
-        dkt_kt = fmaf(dkt, ktv, dkt_kt);
-        if (t < nv) a.dq[((n * a.T + t0 + t) * a.H + h) * D + c] = rq[tt] + dqg * gam_t;
+        w.dQG[e] = qt[tt] * rq[tt] + kt[tt] * rk[tt] + dqg[tt] * qt[tt] * gam_t + dkg[tt] * kt[tt] * gam_t -
+                   dkt[tt] * ktv;
+        dkt_kt = fmaf(dkt[tt], ktv, dkt_kt);
+        if (t < nv) a.dq[((n * a.T + t0 + t) * a.H + h) * D + c] = rq[tt] + dqg[tt] * gam_t;
       }
     }
   } else {
     const int c = tid - D;
     for (int I = 0; I < CC / 8; ++I) {
-      float gi[8], cs[8];
+      float gi[8], cs[8], cd[8];
       ld8(Gt_, c, 8 * I, gi);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) cs[u] = 0.f;
-      col_tile<true>(Gt_, Kt_, Qt_, dMq, dMk, c, I, I, gi, cs);
-      for (int T = I + 1; T < CC / 8; ++T) col_tile<false>(Gt_, Kt_, Qt_, dMq, dMk, c, T, I, gi, cs);
+      for (int u = 0; u < 8; ++u) cs[u] = cd[u] = 0.f;
+      col_tile_diag(Kt_, Qt_, dMq, dMk, c, I, gi, cd);
+      for (int T = I + 1; T < CC / 8; ++T) col_tile_off(Gt_, Kt_, Qt_, dMq, dMk, c, T, I, gi[7], cs);
 #pragma unroll
-      for (int ii = 0; ii < 8; ++ii) Cs[(8 * I + ii) * D + c] = cs[ii];
+      for (int ii = 0; ii < 8; ++ii) Cs[(8 * I + ii) * D + c] = fmaf(ex2f(gi[7] - gi[ii]), cs[ii], cd[ii]);
     }
   }
   __syncthreads();
@@ -541,27 +644,41 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
     // the column form into dk and dG, then dG -> dlog(alpha) by a reverse cumulative sum
     const int c = tid;
     float acc = dkt_kt + w.dgC[(size_t)b * D + c] * w.gam[(size_t)b * D + c];  // only G_last's share
-#pragma unroll 4
-    for (int t = CC - 1; t >= 0; --t) {
-      const size_t e = mat + t * D + c;
-      const float kt = Kt_[swz(c, t)], cs = Cs[t * D + c];
-      const float dk = w.dKG[e] + cs;
-      acc += w.dQG[e] - kt * cs;  // sum_{r >= t} dG[r]
-      if (t < nv) {
-        const size_t o = ((n * a.T + t0 + t) * a.H + h) * D + c;
-        a.dk[o] = dk;
-        float dl = acc;
-        if (!a.gate_log) {  // dL/dalpha = dL/dlog(alpha) / alpha
-          const float x = a.gate[n * a.gs[0] + (t0 + t) * a.gs[1] + h * a.gs[2] + c];
-          dl = x > 0.f ? acc / x : 0.f;
+    for (int t8 = CC - 8; t8 >= 0; t8 -= 8) {
+      float kg[8], qg[8], x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const size_t e = mat + (t8 + u) * D + c;
+        kg[u] = w.dKG[e];
+        qg[u] = w.dQG[e];
+        x[u] = !a.gate_log && t8 + u < nv ? a.gate[n * a.gs[0] + (t0 + t8 + u) * a.gs[1] + h * a.gs[2] + c] : 1.f;
+      }
+#pragma unroll
+      for (int u = 7; u >= 0; --u) {
+        const int t = t8 + u;
+        const float kt = Kt_[swz(c, t)], cs = Cs[t * D + c];
+        acc += qg[u] - kt * cs;  // sum_{r >= t} dG[r]
+        if (t < nv) {
+          const size_t o = ((n * a.T + t0 + t) * a.H + h) * D + c;
+          a.dk[o] = kg[u] + cs;
+          // dL/dalpha = dL/dlog(alpha) / alpha when alpha itself is the input
+          a.dgate[o] = a.gate_log ? acc : (x[u] > 0.f ? acc / x[u] : 0.f);
         }
-        a.dgate[o] = dl;
       }
     }
   } else {
-    const int c = tid - D;
-    for (int t = 0; t < nv; ++t) a.dv[((n * a.T + t0 + t) * a.H + h) * D + c] = w.dV[mat + t * D + c];
-    if (c < nv) a.dbeta[(n * a.T + t0 + c) * a.H + h] = dbeta_part[(size_t)b * CC + c];
+    const int l = tid - D;  // dv: 16-byte pieces, 8 loads ahead of their stores
+    for (int p0 = 0; p0 < CC * D / 4; p0 += 8 * D) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = reinterpret_cast<const float4*>(w.dV + mat)[p0 + u * D + l];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int pc = p0 + u * D + l, t = pc >> 5, c4 = pc & 31;
+        if (t < nv) *reinterpret_cast<float4*>(a.dv + ((n * a.T + t0 + t) * a.H + h) * D + 4 * c4) = v[u];
+      }
+    }
+    if (l < nv) a.dbeta[(n * a.T + t0 + l) * a.H + h] = dbeta_part[(size_t)b * CC + l];
   }
 }
 
