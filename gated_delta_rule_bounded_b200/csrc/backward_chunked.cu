@@ -84,6 +84,10 @@ __device__ __forceinline__ void chunk_of(const BwdC& a, int b, int& n, int& j, i
   nv = (int)min((int64_t)CC, a.T - t0);
 }
 
+__device__ __forceinline__ void unpack4(const float4 v, float o[4]) {
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+
 // fp32 copies of the chunk's q, k, v, dO (zero past the end), the log2 cumulative decay (per-token floor at
 // -126, zero past the end: alpha = 1), Q*Gamma, K*Gamma, K*gamma_C/Gamma (transposed, [c][t]), gamma_C and beta
 // (zero past the end).
@@ -156,61 +160,118 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
   }
 }
 
-// Mq and Mk of one chunk, every pair (t, i <= t) summed over the channels with its decay ratio
-// 2^{G2_tc - G2_ic} <= 1 formed directly (no range limit). A warp takes 4 rows t and 32 columns i (a lane per
-// i), channels 4 at a time from rows padded to 132 floats (the row-t operands are warp-uniform float4 loads).
-constexpr int PAIR_SMEM = 3 * CC * 132 * 4;
-__global__ void __launch_bounds__(256, 2) pair_kernel(Bufs w) {
+// Mq and Mk of one chunk. A warp takes 4 rows t from 4q and 32 columns i (a lane per i), channels 4 at a time.
+// For the columns before the rows' quad (i < 4q <= t) the decay ratio factors at the reference r = 4q - 1:
+// 2^{G_t - G_i} = 2^{G_t - G_r} 2^{G_r - G_i}, both factors <= 1 (a factor that flushes to zero bounds the
+// exact ratio, which is then below 2^-126 as well); q_t and k_t come pre-scaled by the first factor (QA, KA),
+// so a pair costs two FMAs and a lane one exponential per channel. The 4x4 blocks on the diagonal form every
+// ratio directly. Rows of k and G are padded to 132 floats (lane-indexed float4 loads hit distinct banks).
+constexpr int PAIR_SMEM = (2 * CC * 132 + 2 * CC * D) * 4;
+__global__ void __launch_bounds__(256, 1) pair_kernel(Bufs w) {
   constexpr int PR = 132;
   extern __shared__ __align__(16) float sp[];
-  float* Qs = sp;
-  float* Ks = Qs + CC * PR;
-  float* Gs = Ks + CC * PR;
+  float* Ks = sp;              // [64][132]
+  float* Gs = Ks + CC * PR;    // [64][132]
+  float* QA = Gs + CC * PR;    // [64][128]: q_t, then q_t 2^{G_t - G_r(t)}
+  float* KA = QA + CC * D;     // [64][128]: k_t 2^{G_t - G_r(t)}
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t mat = (size_t)b * CC * D;
-  for (int e = tid; e < CC * D / 4; e += 256) {
-    const int t = e >> 5, c4 = e & 31;
-    *reinterpret_cast<float4*>(Qs + t * PR + 4 * c4) = reinterpret_cast<const float4*>(w.Qf + mat)[e];
-    *reinterpret_cast<float4*>(Ks + t * PR + 4 * c4) = reinterpret_cast<const float4*>(w.Kf + mat)[e];
-    *reinterpret_cast<float4*>(Gs + t * PR + 4 * c4) = reinterpret_cast<const float4*>(w.G2 + mat)[e];
+  const size_t mat = (size_t)b * CC * D, sq = (size_t)b * CC * CC;
+  {
+    float4 kv[8], gv[8], qv[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      kv[m] = reinterpret_cast<const float4*>(w.Kf + mat)[tid + 256 * m];
+      gv[m] = reinterpret_cast<const float4*>(w.G2 + mat)[tid + 256 * m];
+      qv[m] = reinterpret_cast<const float4*>(w.Qf + mat)[tid + 256 * m];
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int e = tid + 256 * m, t = e >> 5, c = 4 * (e & 31);
+      *reinterpret_cast<float4*>(Ks + t * PR + c) = kv[m];
+      *reinterpret_cast<float4*>(Gs + t * PR + c) = gv[m];
+      *reinterpret_cast<float4*>(QA + t * D + c) = qv[m];
+    }
   }
   __syncthreads();
-  const size_t sq = (size_t)b * CC * CC;
-  // units (4 rows from 4q, columns from 32 hf): warp w takes q = w, w + 8 with hf = 0 and q = w + 8 with
-  // hf = 1; (q = w, hf = 1) lies above the diagonal and is all zero
+  // the 4x4 diagonal blocks: warp w takes quads 2w and 2w + 1, a lane one pair (t, i) of them
+  {
+    const int q = 2 * warp + (lane >> 4), r = (lane >> 2) & 3, ii = lane & 3;
+    const int t = 4 * q + r, i = 4 * q + ii;
+    float mq = 0.f, mk = 0.f;
+    if (ii <= r) {
+#pragma unroll 4
+      for (int c = 0; c < D; c += 4) {
+        const float4 qv = *reinterpret_cast<const float4*>(QA + t * D + c);
+        const float4 kt = *reinterpret_cast<const float4*>(Ks + t * PR + c);
+        const float4 gt = *reinterpret_cast<const float4*>(Gs + t * PR + c);
+        const float4 kv = *reinterpret_cast<const float4*>(Ks + i * PR + c);
+        const float4 gv = *reinterpret_cast<const float4*>(Gs + i * PR + c);
+        float x = ex2f(gt.x - gv.x) * kv.x;
+        mq = fmaf(qv.x, x, mq); mk = fmaf(kt.x, x, mk);
+        x = ex2f(gt.y - gv.y) * kv.y;
+        mq = fmaf(qv.y, x, mq); mk = fmaf(kt.y, x, mk);
+        x = ex2f(gt.z - gv.z) * kv.z;
+        mq = fmaf(qv.z, x, mq); mk = fmaf(kt.z, x, mk);
+        x = ex2f(gt.w - gv.w) * kv.w;
+        mq = fmaf(qv.w, x, mq); mk = fmaf(kt.w, x, mk);
+      }
+    }
+    w.Mq[sq + t * CC + i] = ii <= r ? mq : 0.f;
+    w.Mk[sq + t * CC + i] = ii < r ? mk : 0.f;
+  }
+  __syncthreads();  // raw q read; scale in place
+#pragma unroll 2
+  for (int e = tid; e < CC * D / 4; e += 256) {
+    const int t = e >> 5, c = 4 * (e & 31);
+    float4 qa = make_float4(0.f, 0.f, 0.f, 0.f), ka = qa;
+    if (t >= 4) {
+      const int r = (t & ~3) - 1;
+      const float4 g = *reinterpret_cast<const float4*>(Gs + t * PR + c);
+      const float4 gr = *reinterpret_cast<const float4*>(Gs + r * PR + c);
+      const float4 qv = *reinterpret_cast<const float4*>(QA + t * D + c);
+      const float4 kv = *reinterpret_cast<const float4*>(Ks + t * PR + c);
+      const float ax = ex2f(g.x - gr.x), ay = ex2f(g.y - gr.y), az = ex2f(g.z - gr.z), aw = ex2f(g.w - gr.w);
+      qa = make_float4(qv.x * ax, qv.y * ay, qv.z * az, qv.w * aw);
+      ka = make_float4(kv.x * ax, kv.y * ay, kv.z * az, kv.w * aw);
+    }
+    *reinterpret_cast<float4*>(QA + t * D + c) = qa;
+    *reinterpret_cast<float4*>(KA + t * D + c) = ka;
+  }
+  __syncthreads();
+  // units (rows 4q.., columns 32 hf..): warp w takes q = w and w + 8 with hf = 0, q = w + 8 with hf = 1
+  // ((q = w, hf = 1) lies above the diagonal: zeros)
 #pragma unroll 1
   for (int k = 0; k < 4; ++k) {
     const int u = warp + 8 * k, q = u & 15, hf = u >> 4;
     const int i = 32 * hf + lane, tq = 4 * q;
     float mq[4] = {0.f, 0.f, 0.f, 0.f}, mk[4] = {0.f, 0.f, 0.f, 0.f};
-    if (32 * hf <= tq + 3) {
+    if (32 * hf < tq) {  // some column before the quad
       const float* ki_ = Ks + i * PR;
       const float* gi_ = Gs + i * PR;
+      const float* gr_ = Gs + (tq - 1) * PR;
 #pragma unroll 2
       for (int c = 0; c < D; c += 4) {
         const float4 kv = *reinterpret_cast<const float4*>(ki_ + c);
         const float4 gv = *reinterpret_cast<const float4*>(gi_ + c);
+        const float4 gr = *reinterpret_cast<const float4*>(gr_ + c);
+        const float kb0 = kv.x * ex2f(gr.x - gv.x), kb1 = kv.y * ex2f(gr.y - gv.y);
+        const float kb2 = kv.z * ex2f(gr.z - gv.z), kb3 = kv.w * ex2f(gr.w - gv.w);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const float4 qv = *reinterpret_cast<const float4*>(Qs + (tq + r) * PR + c);
-          const float4 kt = *reinterpret_cast<const float4*>(Ks + (tq + r) * PR + c);
-          const float4 gt = *reinterpret_cast<const float4*>(Gs + (tq + r) * PR + c);
-          float x = ex2f(gt.x - gv.x) * kv.x;
-          mq[r] = fmaf(qv.x, x, mq[r]); mk[r] = fmaf(kt.x, x, mk[r]);
-          x = ex2f(gt.y - gv.y) * kv.y;
-          mq[r] = fmaf(qv.y, x, mq[r]); mk[r] = fmaf(kt.y, x, mk[r]);
-          x = ex2f(gt.z - gv.z) * kv.z;
-          mq[r] = fmaf(qv.z, x, mq[r]); mk[r] = fmaf(kt.z, x, mk[r]);
-          x = ex2f(gt.w - gv.w) * kv.w;
-          mq[r] = fmaf(qv.w, x, mq[r]); mk[r] = fmaf(kt.w, x, mk[r]);
+          const float4 qa = *reinterpret_cast<const float4*>(QA + (tq + r) * D + c);
+          const float4 ka = *reinterpret_cast<const float4*>(KA + (tq + r) * D + c);
+          mq[r] = fmaf(qa.x, kb0, fmaf(qa.y, kb1, fmaf(qa.z, kb2, fmaf(qa.w, kb3, mq[r]))));
+          mk[r] = fmaf(ka.x, kb0, fmaf(ka.y, kb1, fmaf(ka.z, kb2, fmaf(ka.w, kb3, mk[r]))));
         }
       }
     }
+    if (i < tq || i > tq + 3) {  // the quad's own columns are the diagonal pass's
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int t = tq + r;
-      w.Mq[sq + t * CC + i] = i <= t ? mq[r] : 0.f;
-      w.Mk[sq + t * CC + i] = i < t ? mk[r] : 0.f;
+      for (int r = 0; r < 4; ++r) {
+        const int t = tq + r;
+        w.Mq[sq + t * CC + i] = i < tq ? mq[r] : 0.f;
+        w.Mk[sq + t * CC + i] = i < tq ? mk[r] : 0.f;
+      }
     }
   }
 }
@@ -287,9 +348,6 @@ __device__ __forceinline__ void dstate_prefetch(const Bufs& w, int b, int vsl, f
   cp_async_commit();
 }
 
-__device__ __forceinline__ void unpack4(const float4 v, float o[4]) {
-  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-}
 
 __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
   extern __shared__ __align__(16) float sd[];
@@ -392,10 +450,16 @@ __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
   }
 }
 
-// dMq = tril(dMq) (diagonal kept); dgamma_C[c] = sum_v dS_C[c][v] S0[c][v] (a warp per row c).
-__global__ void __launch_bounds__(256) mask_dgc_kernel(Bufs w) {
+// dMq = tril(dMq) (diagonal kept); dgamma_C[c] = sum_v dS_C[c][v] S0[c][v] (a warp per row c); dv of the chunk's
+// real rows (dV = TB^T dU, 8 loads ahead of their stores).
+__global__ void __launch_bounds__(256) mask_dgc_kernel(BwdC a, Bufs w) {
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t sq = (size_t)b * CC * CC, st = (size_t)b * D * D;
+  int n, j, h, t0, nv;
+  chunk_of(a, b, n, j, h, t0, nv);
+  const size_t sq = (size_t)b * CC * CC, st = (size_t)b * D * D, mat = (size_t)b * CC * D;
+  float4 v[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) v[u] = reinterpret_cast<const float4*>(w.dV + mat)[tid + 256 * u];
   for (int e = tid; e < CC * CC; e += 256)
     if (e % CC > e / CC) w.dMq[sq + e] = 0.f;
   for (int c = warp; c < D; c += 8) {
@@ -405,6 +469,11 @@ __global__ void __launch_bounds__(256) mask_dgc_kernel(Bufs w) {
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
     if (lane == 0) w.dgC[(size_t)b * D + c] = s;
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int pc = tid + 256 * u, t = pc >> 5, c4 = pc & 31;
+    if (t < nv) *reinterpret_cast<float4*>(a.dv + ((n * a.T + t0 + t) * a.H + h) * D + 4 * c4) = v[u];
   }
 }
 
@@ -423,10 +492,12 @@ __global__ void __launch_bounds__(64) dt_kernel(Bufs w, float* dbeta_part) {
   dbeta_part[(size_t)b * CC + j] = s;
 }
 
-// dA = strict_tril(dA) in place; dbeta = colsum(dTB * T) + rowsum(dA * Mk); dMk = Diag(beta) dA (into dA).
-// A warp per row t (lanes over i).
-__global__ void __launch_bounds__(256) da_kernel(Bufs w, float* dbeta_part) {
+// dA = strict_tril(dA) in place; dbeta = colsum(dTB * T) + rowsum(dA * Mk) written for the chunk's real rows;
+// dMk = Diag(beta) dA (into dA). A warp per row t (lanes over i).
+__global__ void __launch_bounds__(256) da_kernel(BwdC a, Bufs w, const float* dbeta_part) {
   const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int n, j, h, t0, nv;
+  chunk_of(a, b, n, j, h, t0, nv);
   const size_t sq = (size_t)b * CC * CC;
   for (int t = warp; t < CC; t += 8) {
     const float bt = w.bet[(size_t)b * CC + t];
@@ -440,20 +511,21 @@ __global__ void __launch_bounds__(256) da_kernel(Bufs w, float* dbeta_part) {
     }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
-    if (lane == 0) dbeta_part[(size_t)b * CC + t] += s;
+    if (lane == 0 && t < nv) a.dbeta[(n * a.T + t0 + t) * a.H + h] = dbeta_part[(size_t)b * CC + t] + s;
   }
 }
 
-// Per chunk: the gradients of the bilinear forms Mq, Mk (every decay ratio formed per pair and channel), then
-// dq, dk, dv, dbeta and dG -> dlog(alpha) (reverse cumulative sum) for the chunk's real rows.
+// Per chunk: the gradients of the bilinear forms Mq, Mk, then dq, dk and dG -> dlog(alpha) (reverse cumulative
+// sum) for the chunk's real rows.
 // For channel c and the pairs (t, i <= t) with R = 2^{G2_tc - G2_ic}:
 //   row forms (by t):    rq[t] = sum_i dMq[t][i] k_ic R,  rk[t] = sum_i dMk[t][i] k_ic R
 //   column form (by i):  cs[i] = sum_t (dMq[t][i] q_tc + dMk[t][i] k_tc) R
 // Threads 0-127 (one per channel) take the row forms, threads 128-255 the column form, each over 8x8 tiles of
-// pairs with the tile's operands in registers. The per-channel columns of G, K and Q sit transposed in shared
-// memory ([c][t], 16-byte groups XOR-swizzled by c so that a quarter warp's float4 loads hit distinct banks).
+// pairs with the tile's operands in registers; the row shares of dk and dG wait in shared memory for the column
+// form. The per-channel columns of G, K and Q sit transposed in shared memory ([c][t], 16-byte groups
+// XOR-swizzled by c so that a quarter warp's float4 loads hit distinct banks).
 constexpr int ASM_T = D * CC;                             // one transposed [128][64] tile
-constexpr int ASSEMBLE_SMEM = (3 * ASM_T + 2 * CC * CC + CC * D) * 4;
+constexpr int ASSEMBLE_SMEM = (3 * ASM_T + 2 * CC * CC + 3 * CC * D) * 4;
 
 __device__ __forceinline__ int swz(int c, int t) { return c * CC + ((((t >> 2) ^ (c & 7))) << 2) + (t & 3); }
 __device__ __forceinline__ void ld8(const float* X, int c, int t0, float v[8]) {
@@ -559,7 +631,7 @@ __device__ __forceinline__ void col_tile_diag(const float* Kt_, const float* Qt_
   }
 }
 
-__global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const float* dbeta_part) {
+__global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w) {
   extern __shared__ __align__(16) float sa[];
   float* Gt_ = sa;                  // [128][64] swizzled: G2 by channel
   float* Kt_ = Gt_ + ASM_T;         // [128][64] swizzled: k
@@ -567,29 +639,47 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
   float* dMq = Qt_ + ASM_T;         // [64][64]
   float* dMk = dMq + CC * CC;       // [64][64] (Diag(beta) dA)
   float* Cs = dMk + CC * CC;        // [64][128]: the column form
+  float* DKr = Cs + CC * D;         // [64][128]: dk's row share
+  float* DGr = DKr + CC * D;        // [64][128]: dG's row share
   const int b = blockIdx.x, tid = threadIdx.x;
   int n, j, h, t0, nv;
   chunk_of(a, b, n, j, h, t0, nv);
   const size_t mat = (size_t)b * CC * D, sq = (size_t)b * CC * CC;
-  // transposed loads: a thread takes 4 consecutive tokens of one channel (coalesced over the channel)
-#pragma unroll 2
-  for (int e = tid; e < (CC / 4) * D; e += 256) {
-    const int c = e % D, t4 = (e / D) * 4;
-    float g[4], k[4], q[4];
+  // dMq and dMk with cp.async; G2, k, q transposed through registers (a thread takes 4 consecutive tokens of
+  // one channel, coalesced over the channel; every load in flight at once)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      g[u] = w.G2[mat + (t4 + u) * D + c];
-      k[u] = w.Kf[mat + (t4 + u) * D + c];
-      q[u] = w.Qf[mat + (t4 + u) * D + c];
-    }
-    *reinterpret_cast<float4*>(Gt_ + swz(c, t4)) = make_float4(g[0], g[1], g[2], g[3]);
-    *reinterpret_cast<float4*>(Kt_ + swz(c, t4)) = make_float4(k[0], k[1], k[2], k[3]);
-    *reinterpret_cast<float4*>(Qt_ + swz(c, t4)) = make_float4(q[0], q[1], q[2], q[3]);
-  }
   for (int e = tid; e < CC * CC / 4; e += 256) {
-    reinterpret_cast<float4*>(dMq)[e] = reinterpret_cast<const float4*>(w.dMq + sq)[e];
-    reinterpret_cast<float4*>(dMk)[e] = reinterpret_cast<const float4*>(w.dA + sq)[e];
+    cp_async16(dMq + 4 * e, w.dMq + sq + 4 * e);
+    cp_async16(dMk + 4 * e, w.dA + sq + 4 * e);
   }
+  {
+    float g[8][4], k[8][4], q[8][4];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int e = tid + 256 * m, c = e & 127, t4 = (e >> 7) * 4;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        g[m][u] = w.G2[mat + (t4 + u) * D + c];
+        k[m][u] = w.Kf[mat + (t4 + u) * D + c];
+        q[m][u] = w.Qf[mat + (t4 + u) * D + c];
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int e = tid + 256 * m, c = e & 127, t4 = (e >> 7) * 4;
+      *reinterpret_cast<float4*>(Gt_ + swz(c, t4)) = make_float4(g[m][0], g[m][1], g[m][2], g[m][3]);
+      *reinterpret_cast<float4*>(Kt_ + swz(c, t4)) = make_float4(k[m][0], k[m][1], k[m][2], k[m][3]);
+      *reinterpret_cast<float4*>(Qt_ + swz(c, t4)) = make_float4(q[m][0], q[m][1], q[m][2], q[m][3]);
+    }
+  }
+  // dQG and dKG into the row-share buffers (each row thread reads its element, then writes its share over it)
+#pragma unroll
+  for (int e = tid; e < CC * D / 4; e += 256) {
+    cp_async16(DGr + 4 * e, w.dQG + mat + 4 * e);
+    cp_async16(DKr + 4 * e, w.dKG + mat + 4 * e);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
   float dkt_kt = 0.f;  // row threads: sum_t dKT * KT, the share of G_last
   if (tid < D) {
@@ -597,14 +687,11 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
     float gl[8];
     ld8(Gt_, c, CC - 8, gl);
     for (int T = 0; T < CC / 8; ++T) {
-      float gt[8], rq[8], rk[8], dqg[8], dkg[8], dkt[8];
+      float gt[8], rq[8], rk[8], dkt[8];
       ld8(Gt_, c, 8 * T, gt);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // the epilogue's operands, loaded ahead of the tiles
-        const size_t e = mat + (8 * T + u) * D + c;
-        dqg[u] = w.dQG[e];
-        dkg[u] = w.dKG[e];
-        dkt[u] = w.dKT[e];
+      for (int u = 0; u < 8; ++u) {  // dKT of the epilogue, loaded ahead of the tiles
+        dkt[u] = w.dKT[mat + (8 * T + u) * D + c];
         rq[u] = rk[u] = 0.f;
       }
       for (int I = 0; I < T; ++I) row_tile_off(Gt_, Kt_, dMq, dMk, c, T, I, gt, rq, rk);
@@ -615,15 +702,15 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
 #pragma unroll
       for (int tt = 0; tt < 8; ++tt) {
         const int t = 8 * T + tt;
-        const size_t e = mat + t * D + c;
         const float gam_t = ex2f(gt[tt]), kts = ex2f(gl[7] - gt[tt]);
+        const float dqg = DGr[t * D + c], dkg = DKr[t * D + c];
         // dk's and dG's row shares, completed by the column form below
-        w.dKG[e] = rk[tt] + dkg[tt] * gam_t + dkt[tt] * kts;
+        DKr[t * D + c] = rk[tt] + dkg * gam_t + dkt[tt] * kts;
         const float ktv = kt[tt] * kts;
-        w.dQG[e] = qt[tt] * rq[tt] + kt[tt] * rk[tt] + dqg[tt] * qt[tt] * gam_t + dkg[tt] * kt[tt] * gam_t -
-                   dkt[tt] * ktv;
+        DGr[t * D + c] = qt[tt] * rq[tt] + kt[tt] * rk[tt] + dqg * qt[tt] * gam_t + dkg * kt[tt] * gam_t -
+                         dkt[tt] * ktv;
         dkt_kt = fmaf(dkt[tt], ktv, dkt_kt);
-        if (t < nv) a.dq[((n * a.T + t0 + t) * a.H + h) * D + c] = rq[tt] + dqg[tt] * gam_t;
+        if (t < nv) a.dq[((n * a.T + t0 + t) * a.H + h) * D + c] = rq[tt] + dqg * gam_t;
       }
     }
   } else {
@@ -645,40 +732,23 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w, const 
     const int c = tid;
     float acc = dkt_kt + w.dgC[(size_t)b * D + c] * w.gam[(size_t)b * D + c];  // only G_last's share
     for (int t8 = CC - 8; t8 >= 0; t8 -= 8) {
-      float kg[8], qg[8], x[8];
+      float x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const size_t e = mat + (t8 + u) * D + c;
-        kg[u] = w.dKG[e];
-        qg[u] = w.dQG[e];
+      for (int u = 0; u < 8; ++u)
         x[u] = !a.gate_log && t8 + u < nv ? a.gate[n * a.gs[0] + (t0 + t8 + u) * a.gs[1] + h * a.gs[2] + c] : 1.f;
-      }
 #pragma unroll
       for (int u = 7; u >= 0; --u) {
         const int t = t8 + u;
         const float kt = Kt_[swz(c, t)], cs = Cs[t * D + c];
-        acc += qg[u] - kt * cs;  // sum_{r >= t} dG[r]
+        acc += DGr[t * D + c] - kt * cs;  // sum_{r >= t} dG[r]
         if (t < nv) {
           const size_t o = ((n * a.T + t0 + t) * a.H + h) * D + c;
-          a.dk[o] = kg[u] + cs;
+          a.dk[o] = DKr[t * D + c] + cs;
           // dL/dalpha = dL/dlog(alpha) / alpha when alpha itself is the input
           a.dgate[o] = a.gate_log ? acc : (x[u] > 0.f ? acc / x[u] : 0.f);
         }
       }
     }
-  } else {
-    const int l = tid - D;  // dv: 16-byte pieces, 8 loads ahead of their stores
-    for (int p0 = 0; p0 < CC * D / 4; p0 += 8 * D) {
-      float4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = reinterpret_cast<const float4*>(w.dV + mat)[p0 + u * D + l];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int pc = p0 + u * D + l, t = pc >> 5, c4 = pc & 31;
-        if (t < nv) *reinterpret_cast<float4*>(a.dv + ((n * a.T + t0 + t) * a.H + h) * D + 4 * c4) = v[u];
-      }
-    }
-    if (l < nv) a.dbeta[(n * a.T + t0 + l) * a.H + h] = dbeta_part[(size_t)b * CC + l];
   }
 }
 
@@ -852,7 +922,7 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
     *cublas_status = (int)cs;
     return cudaErrorUnknown;
   }
-  mask_dgc_kernel<<<NB, 256, 0, s>>>(w);
+  mask_dgc_kernel<<<NB, 256, 0, s>>>(a, w);
   dt_kernel<<<NB, 64, 0, s>>>(w, dbeta_part);  // X = dT = dTB Diag(beta); dbeta_part = colsum(dTB * T)
   // dA = -(T^T dT) T^T: the product T^T dT into dA, then -dA T^T into X (two products, reusing the buffers)
   G(true, false, CC, CC, CC, 1.f, w.Tm, CC, s64, w.X, CC, s64, 0.f, w.dA, CC, s64);
@@ -862,8 +932,8 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
     return cudaErrorUnknown;
   }
   std::swap(w.dA, w.X);  // dA now names the result
-  da_kernel<<<NB, 256, 0, s>>>(w, dbeta_part);
-  assemble_kernel<<<NB, 256, ASSEMBLE_SMEM, s>>>(a, w, dbeta_part);
+  da_kernel<<<NB, 256, 0, s>>>(a, w, dbeta_part);
+  assemble_kernel<<<NB, 256, ASSEMBLE_SMEM, s>>>(a, w);
   return cudaGetLastError();
 }
 
