@@ -84,9 +84,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_scan_backward.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, lp,
                                       vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_bounded_decay_backward.argtypes = [vp, vp, ctypes.c_float, vp, i64, i64, i64, i64, vp, vp, vp]
-    lib.kda_scan_backward_chunked_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
-    lib.kda_scan_backward_chunked.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, i64, i64, i64, i64, i64, lp,
-                                              vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.kda_scan_backward_chunked_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, i64,
+                                                              ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_scan_backward_chunked.argtypes = [vp, vp, vp, i32, vp, i32, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                              i64, lp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_selftest_wait_expiry.argtypes = [vp]
     for fn in ("kda_scan_backward_workspace_bytes", "kda_scan_backward", "kda_bounded_decay_backward",
                "kda_selftest_wait_expiry", "kda_scan_backward_chunked_workspace_bytes", "kda_scan_backward_chunked"):
@@ -502,10 +503,11 @@ def scan_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch
 
 def scan_backward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: torch.Tensor, beta: torch.Tensor,
                           initial_state: Optional[torch.Tensor], d_o: torch.Tensor,
-                          d_final_state: Optional[torch.Tensor] = None, *, gate_is_log: bool = False,
-                          workspace: Optional[torch.Tensor] = None) -> dict:
+                          d_final_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None, *,
+                          gate_is_log: bool = False, workspace: Optional[torch.Tensor] = None) -> dict:
     """The gradients of ``scan_backward`` through the chunkwise form in parallel over 64-token chunks
-    (``kda_scan_backward_chunked``): bf16 ``q, k, v`` with K = V = 128, dense batch rows. Same outputs.
+    (``kda_scan_backward_chunked``): bf16 ``q, k, v`` with K = V = 128; dense batch rows or packed sequences
+    (``cu_seqlens`` int32 ``[N+1]``, B = 1, states per sequence). Same outputs as ``scan_backward``.
     ``workspace``: optional uint8 device tensor of at least ``chunked_backward_workspace_bytes`` bytes."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (beta, "beta"), (d_o, "d_o")):
         _cuda(t, n)
@@ -520,16 +522,27 @@ def scan_backward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gat
     d_o = d_o.to(torch.float32).contiguous()
     if d_o.shape != (B, T, H, V):
         raise ValueError("d_o must be [B,T,H,V]")
+    N, n_seq, cu_ptr = B, 0, None
+    if cu_seqlens is not None:
+        _cuda(cu_seqlens, "cu_seqlens")
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        if B != 1:
+            raise ValueError("cu_seqlens requires B == 1")
+        cu_seqlens = cu_seqlens.contiguous()
+        N = n_seq = cu_seqlens.numel() - 1
+        cu_ptr = cu_seqlens.data_ptr()
     f32 = lambda t: None if t is None else t.to(device=dev, dtype=torch.float32).contiguous()  # noqa: E731
     initial_state, d_final_state = f32(initial_state), f32(d_final_state)
     for t, n in ((initial_state, "initial_state"), (d_final_state, "d_final_state")):
-        if t is not None and t.shape != (B, H, K, V):
-            raise ValueError(f"{n} must be [{B},{H},{K},{V}]")
-    out = {"dq": torch.empty(B, T, H, K, device=dev), "dk": torch.empty(B, T, H, K, device=dev),
-           "dv": torch.empty(B, T, H, V, device=dev), "dgate": torch.empty(B, T, H, K, device=dev),
-           "dbeta": torch.empty(B, T, H, device=dev), "d_initial_state": torch.empty(B, H, K, V, device=dev)}
+        if t is not None and t.shape != (N, H, K, V):
+            raise ValueError(f"{n} must be [{N},{H},{K},{V}]")
+    new = torch.zeros if cu_seqlens is not None else torch.empty  # tokens outside every sequence: zero
+    out = {"dq": new(B, T, H, K, device=dev), "dk": new(B, T, H, K, device=dev),
+           "dv": new(B, T, H, V, device=dev), "dgate": new(B, T, H, K, device=dev),
+           "dbeta": new(B, T, H, device=dev), "d_initial_state": torch.empty(N, H, K, V, device=dev)}
     lib = load_library()
-    need = chunked_backward_workspace_bytes(B, T, H, K, V)
+    need = chunked_backward_workspace_bytes(B, T, H, K, V, n_seq)
     if workspace is None:
         workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
     layout = Layout(_strides4(q), _strides4(k), _strides4(v), _strides4(gate), _strides3(beta), Strides(0, 0, 0))
@@ -537,17 +550,18 @@ def scan_backward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gat
     _check("kda_scan_backward_chunked", lib.kda_scan_backward_chunked(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q.dtype), gate.data_ptr(),
         KDA_GATE_LOG if gate_is_log else KDA_GATE_ALPHA, beta.data_ptr(), ptr(initial_state), d_o.data_ptr(),
-        ptr(d_final_state), B, T, H, K, V, ctypes.byref(layout), out["dq"].data_ptr(), out["dk"].data_ptr(),
-        out["dv"].data_ptr(), out["dgate"].data_ptr(), out["dbeta"].data_ptr(), out["d_initial_state"].data_ptr(),
-        workspace.data_ptr(), workspace.numel(), _stream(dev)))
+        ptr(d_final_state), cu_ptr, n_seq, B, T, H, K, V, ctypes.byref(layout), out["dq"].data_ptr(),
+        out["dk"].data_ptr(), out["dv"].data_ptr(), out["dgate"].data_ptr(), out["dbeta"].data_ptr(),
+        out["d_initial_state"].data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(dev)))
     return out
 
 
-def chunked_backward_workspace_bytes(B: int, T: int, H: int, K: int = 128, V: int = 128) -> int:
-    """Workspace bytes of ``scan_backward_chunked`` (``kda_scan_backward_chunked_workspace_bytes``)."""
+def chunked_backward_workspace_bytes(B: int, T: int, H: int, K: int = 128, V: int = 128, n_seq: int = 0) -> int:
+    """Workspace bytes of ``scan_backward_chunked`` (``kda_scan_backward_chunked_workspace_bytes``; ``n_seq``:
+    the number of packed sequences, 0 without ``cu_seqlens``)."""
     n = ctypes.c_size_t(0)
     _check("kda_scan_backward_chunked_workspace_bytes",
-           load_library().kda_scan_backward_chunked_workspace_bytes(B, T, H, K, V, ctypes.byref(n)))
+           load_library().kda_scan_backward_chunked_workspace_bytes(B, T, H, K, V, n_seq, ctypes.byref(n)))
     return int(n.value)
 
 

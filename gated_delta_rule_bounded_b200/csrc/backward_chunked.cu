@@ -71,17 +71,56 @@ struct BwdC {
   const float* d_sf;
   float *dq, *dk, *dv, *dgate, *dbeta, *ds0;
   int64_t qs[3], ks[3], vs[3], gs[3], bs[3];
+  const int* cu;  // packed sequences (B = 1), or null
   int64_t T;
-  int B, H, ncps;
+  int B, H, N, ncps;  // N sequences; ncps chunks per batch row without cu
   int gate_log;
 };
 
+// The clamped token range [c0, c1) of packed sequence s.
+__device__ __forceinline__ void seq_tokens(const BwdC& a, int s, int64_t& c0, int64_t& c1) {
+  c1 = min((int64_t)a.cu[s + 1], a.T);
+  c0 = max((int64_t)0, min((int64_t)a.cu[s], c1));
+}
+
+// Chunk-head b -> batch row n (the row of the token tensors), chunk j of its sequence, head h, first token t0
+// within the row and its number of real tokens nv. The chunks are in the forward split kernels' workspace
+// order, b = slot * H + h: without cu_seqlens slot = n * ceil(T / 64) + j; with them, chunk j of sequence s
+// sits at slot floor(c0 / 64) + s + j, and a slot between two sequences' runs has no tokens (nv = 0).
 __device__ __forceinline__ void chunk_of(const BwdC& a, int b, int& n, int& j, int& h, int& t0, int& nv) {
   h = b % a.H;
-  j = (b / a.H) % a.ncps;
-  n = b / (a.H * a.ncps);
-  t0 = j * CC;
-  nv = (int)min((int64_t)CC, a.T - t0);
+  const int slot = b / a.H;
+  if (!a.cu) {
+    j = slot % a.ncps;
+    n = slot / a.ncps;
+    t0 = j * CC;
+    nv = (int)min((int64_t)CC, a.T - t0);
+    return;
+  }
+  n = 0;
+  j = 0;
+  t0 = 0;
+  nv = 0;
+  int lo = 0, hi = a.N - 1, sq = -1;  // the last sequence whose first slot is <= slot
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    int64_t c0, c1;
+    seq_tokens(a, mid, c0, c1);
+    if ((c0 >> 6) + mid <= slot) {
+      sq = mid;
+      lo = mid + 1;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  if (sq < 0) return;
+  int64_t c0, c1;
+  seq_tokens(a, sq, c0, c1);
+  const int64_t jj = slot - ((c0 >> 6) + sq);
+  if (jj * CC >= c1 - c0) return;
+  j = (int)jj;
+  t0 = (int)(c0 + jj * CC);
+  nv = (int)min((int64_t)CC, c1 - t0);
 }
 
 __device__ __forceinline__ void unpack4(const float4 v, float o[4]) {
@@ -157,6 +196,10 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
   if (tid < CC) {
     const int64_t tt = t0 + tid;
     w.bet[(size_t)b * CC + tid] = tid < nv ? a.beta[n * a.bs[0] + tt * a.bs[1] + h * a.bs[2]] : 0.f;
+  }
+  if (nv == 0) {  // a slot without tokens: no forward state was written there
+    for (int e = tid; e < D * D / 4; e += 256)
+      reinterpret_cast<float4*>(w.S0 + (size_t)b * D * D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -356,7 +399,17 @@ __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
   float* dUb = dUa + CC * VS;     // [64][VS]: KT dS (channels 64-127)
   const int tid = threadIdx.x;
   const int nh = blockIdx.x, vsl = blockIdx.y;
-  const int n = nh / a.H, h = nh % a.H;
+  const int n = nh / a.H, h = nh % a.H;  // sequence, head
+  int base, nch;                          // the sequence's first slot and its number of chunks
+  if (a.cu) {
+    int64_t s0, s1;
+    seq_tokens(a, n, s0, s1);
+    base = (int)((s0 >> 6) + n);
+    nch = (int)((s1 - s0 + CC - 1) / CC);
+  } else {
+    base = n * a.ncps;
+    nch = a.ncps;
+  }
   const int c0 = 4 * (tid >> 3), v0 = 4 * (tid & 7);   // this thread's dS[c0 .. c0 + 3][v0 .. v0 + 3] of the slice
   const int half = tid >> 7, i0 = 4 * ((tid & 127) >> 3);  // KT dS: rows i0 .. i0 + 3, channels of this half
   const int vg = vsl * VS + v0;
@@ -368,9 +421,9 @@ __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
                             : make_float4(0.f, 0.f, 0.f, 0.f);
     unpack4(x, dS[r]);
   }
-  dstate_prefetch(w, (n * a.ncps + a.ncps - 1) * a.H + h, vsl, sd + ((a.ncps - 1) & 1) * DS_OPS, tid);
-  for (int j = a.ncps - 1; j >= 0; --j) {
-    const int b = (n * a.ncps + j) * a.H + h;
+  if (nch > 0) dstate_prefetch(w, (base + nch - 1) * a.H + h, vsl, sd + ((nch - 1) & 1) * DS_OPS, tid);
+  for (int j = nch - 1; j >= 0; --j) {
+    const int b = (base + j) * a.H + h;
     const size_t mat = (size_t)b * CC * D, st = (size_t)b * D * D;
     const float* buf = sd + (j & 1) * DS_OPS;
 #pragma unroll
@@ -814,8 +867,10 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
   *cublas_status = 0;
   const int64_t B = fwd.B, T = fwd.T, H = fwd.H;
   const int ncps = (int)((T + CC - 1) / CC);
-  const int NB = (int)(B * ncps * H);
-  const Layout L = carve(B, T, H);
+  // packed sequences: the forward's slot count; the layout is that of one row of n_slots full chunks
+  const int64_t n_slots = fwd.cu ? T / CC + fwd.N + 1 : B * ncps;
+  const int NB = (int)(n_slots * H);
+  const Layout L = fwd.cu ? carve(1, n_slots * CC, H) : carve(B, T, H);
   unsigned char* base = static_cast<unsigned char*>(ws);
   auto F = [&](int i) { return reinterpret_cast<float*>(base + L.off[i]); };
   Bufs w;
@@ -846,7 +901,8 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
   for (int i = 0; i < 3; ++i) {
     a.qs[i] = fwd.qs[i]; a.ks[i] = fwd.ks[i]; a.vs[i] = fwd.vs[i]; a.gs[i] = fwd.gs[i]; a.bs[i] = fwd.bs[i];
   }
-  a.T = T; a.B = (int)B; a.H = (int)H; a.ncps = ncps;
+  a.cu = fwd.cu;
+  a.T = T; a.B = (int)B; a.H = (int)H; a.N = fwd.N; a.ncps = ncps;
   a.gate_log = fwd.gate_mode == KDA_GATE_LOG;
 
   // 2. per-chunk preparation, Mq and Mk, T and TB
@@ -905,7 +961,7 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
     return cudaErrorUnknown;
   }
   {
-    dstate_kernel<<<dim3((unsigned)(B * H), D / VS), 256, DSTATE_SMEM, s>>>(a, w);
+    dstate_kernel<<<dim3((unsigned)((int64_t)fwd.N * H), D / VS), 256, DSTATE_SMEM, s>>>(a, w);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // 5. dMq = dO U^T; dQG = dO S0^T; dKT = U dS_C^T; dW = -dU S0^T; dTB = dU V^T + dW KG^T; dV = TB^T dU;

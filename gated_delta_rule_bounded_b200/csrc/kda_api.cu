@@ -525,24 +525,40 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
   return ok();
 }
 
-int kda_scan_backward_chunked_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes) {
+namespace {
+// Workspace of the chunked backward: with packed sequences the forward's slots (T / 64 + n_seq + 1 per head)
+// are laid out as one row of that many full chunks.
+size_t chunked_bwd_bytes(int64_t B, int64_t T, int64_t H, int64_t n_seq) {
+  if (n_seq > 0) return T * H == 0 ? 0 : kda::chunked_backward_workspace_bytes(1, 64 * (T / 64 + n_seq + 1), H);
+  return B * T * H == 0 ? 0 : kda::chunked_backward_workspace_bytes(B, T, H);
+}
+}  // namespace
+
+int kda_scan_backward_chunked_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, int64_t n_seq,
+                                              size_t* bytes) {
   if (!bytes) return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_chunked_workspace_bytes: null output");
-  if (B < 0 || T < 0 || H < 0 || K < 0 || V < 0)
+  if (B < 0 || T < 0 || H < 0 || K < 0 || V < 0 || n_seq < 0)
     return fail(KDA_ERR_INVALID_ARG, "kda_scan_backward_chunked_workspace_bytes: negative size");
   if (K != 128 || V != 128)
     return fail(KDA_ERR_UNSUPPORTED, "kda_scan_backward_chunked_workspace_bytes: K and V must be 128");
-  *bytes = (B * T * H == 0) ? 0 : kda::chunked_backward_workspace_bytes(B, T, H);
+  *bytes = chunked_bwd_bytes(B, T, H, n_seq);
   return ok();
 }
 
 int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_dtype dtype,
                               const float* gate, kda_gate_kind gate_kind, const float* beta,
                               const float* initial_state, const float* d_o, const float* d_final_state,
+                              const int32_t* cu_seqlens, int64_t n_seq,
                               int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
                               float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
                               void* workspace, size_t workspace_bytes, kda_stream_t stream) {
   const char* fn = "kda_scan_backward_chunked";
-  if (B < 0 || T < 0 || H < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (B < 0 || T < 0 || H < 0 || n_seq < 0) return fail(KDA_ERR_INVALID_ARG, "%s: negative size", fn);
+  int64_t N = B;  // sequences
+  if (cu_seqlens) {
+    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "%s: cu_seqlens requires B == 1 (got %lld)", fn, (long long)B);
+    N = n_seq;
+  }
   if (!valid_dtype(dtype)) return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
   if (gate_kind != KDA_GATE_ALPHA && gate_kind != KDA_GATE_LOG)
     return fail(KDA_ERR_INVALID_ARG, "%s: unknown gate kind %d", fn, (int)gate_kind);
@@ -550,18 +566,20 @@ int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_d
     return fail(KDA_ERR_UNSUPPORTED, "%s: bf16 q, k, v with K = V = 128 only", fn);
   if (H > 65535) return fail(KDA_ERR_UNSUPPORTED, "%s: H must be at most 65535", fn);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (B * H == 0) return ok();
+  if (N * H == 0) return ok();
   if (T == 0) {  // nothing to differentiate through: dS_0 = dS_T
     if (d_initial_state) {
-      cudaError_t e = kda::launch_state_copy(d_final_state, d_initial_state, B * H * K * V, s);
+      cudaError_t e = kda::launch_state_copy(d_final_state, d_initial_state, N * H * K * V, s);
       if (e != cudaSuccess) return cuda_fail(e, fn);
     }
     return ok();
   }
   if (!q || !k || !v || !gate || !beta || !d_o || !dq || !dk || !dv || !dgate || !dbeta)
     return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
-  if (T > INT32_MAX || (T + 63) / 64 * B * H > INT32_MAX) return fail(KDA_ERR_UNSUPPORTED, "%s: T too large", fn);
-  const size_t need = kda::chunked_backward_workspace_bytes(B, T, H);
+  const int64_t n_slots = cu_seqlens ? T / 64 + N + 1 : (T + 63) / 64 * B;
+  if (T > INT32_MAX || n_slots * H > INT32_MAX || N > INT32_MAX)
+    return fail(KDA_ERR_UNSUPPORTED, "%s: T too large", fn);
+  const size_t need = chunked_bwd_bytes(B, T, H, cu_seqlens ? N : 0);
   if (!workspace || workspace_bytes < need)
     return fail(KDA_ERR_INVALID_ARG, "%s: the workspace needs %zu bytes (got %zu)", fn, need, workspace_bytes);
   kda_layout L;
@@ -591,7 +609,7 @@ int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_d
   p.beta = beta;
   p.s0 = initial_state;
   p.sf = nullptr;
-  p.cu = nullptr;
+  p.cu = cu_seqlens;
   p.o = nullptr;
   put(p.qs, L.q);
   put(p.ks, L.k);
@@ -603,7 +621,7 @@ int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_d
   p.H = (int)H;
   p.K = (int)K;
   p.V = (int)V;
-  p.N = (int)B;
+  p.N = (int)N;
   p.gate_mode = (int)gate_kind;
   p.A_log = nullptr;
   p.dt_bias = nullptr;

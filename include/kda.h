@@ -340,20 +340,24 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
  * the state at every chunk end, and every other gradient is formed per chunk
  * (per-pair decay ratios, triangular inverse, plain batched products through
  * cuBLAS in fp32 with TF32 tensor cores). Arguments, layouts and outputs as for
- * kda_scan_backward without cu_seqlens. Supported: bf16 q, k, v with K = V = 128
+ * kda_scan_backward, packed sequences (cu_seqlens, n_seq; B = 1; states per
+ * sequence) included. Supported: bf16 q, k, v with K = V = 128
  * (KDA_ERR_UNSUPPORTED otherwise). The chunk-start states come from the bf16
  * tensor-core forward, so the gradients carry its rounding (relative RMS errors
  * near 1e-3) where kda_scan_backward's token-level adjoint is exact fp32. The
- * workspace (kda_scan_backward_chunked_workspace_bytes; about 880 KB per chunk
- * and head) holds every intermediate; cuBLAS creates its handle (device memory)
+ * workspace (kda_scan_backward_chunked_workspace_bytes for the same B, T, H, K, V
+ * and n_seq, 0 without cu_seqlens; about 880 KB per chunk and head, plus n_seq + 1
+ * chunks per head with cu_seqlens; KDA_ERR_INVALID_ARG if smaller) holds every intermediate; cuBLAS creates its handle (device memory)
  * on the first call on each device and is given a part of the workspace for
  * its own scratch.
  * ------------------------------------------------------------------------- */
-int kda_scan_backward_chunked_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, size_t* bytes);
+int kda_scan_backward_chunked_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                              int64_t n_seq, size_t* bytes);
 
 int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_dtype dtype,
                               const float* gate, kda_gate_kind gate_kind, const float* beta,
                               const float* initial_state, const float* d_o, const float* d_final_state,
+                              const int32_t* cu_seqlens, int64_t n_seq,
                               int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, const kda_layout* layout,
                               float* dq, float* dk, float* dv, float* dgate, float* dbeta, float* d_initial_state,
                               void* workspace, size_t workspace_bytes, kda_stream_t stream);

@@ -284,18 +284,18 @@ def test_prefill_rejects_more_heads_than_a_grid_dimension_holds(lib):
 
 
 def _backward_chunked(lib, **kw):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, dtype=1, gate=FAKE, gk=1, beta=FAKE, s0=None, do=FAKE, dsf=None,
-             B=1, T=64, H=2, K=128, V=128, layout=None, dq=FAKE, dk=FAKE, dv=FAKE, dg=FAKE, db=FAKE,
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dtype=1, gate=FAKE, gk=1, beta=FAKE, s0=None, do=FAKE, dsf=None, cu=None,
+             n_seq=0, B=1, T=64, H=2, K=128, V=128, layout=None, dq=FAKE, dk=FAKE, dv=FAKE, dg=FAKE, db=FAKE,
              ds0=None, ws=FAKE, wsb=0, stream=None)
     a.update(kw)
     f = lib.kda_scan_backward_chunked
     f.restype = ctypes.c_int
     vp, i64 = ctypes.c_void_p, ctypes.c_int64
-    f.argtypes = [vp, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, vp, vp, i64, i64, i64, i64, i64, vp,
+    f.argtypes = [vp, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, vp,
                   vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
-    rc = f(a["q"], a["k"], a["v"], a["dtype"], a["gate"], a["gk"], a["beta"], a["s0"], a["do"], a["dsf"], a["B"], a["T"],
-           a["H"], a["K"], a["V"], a["layout"], a["dq"], a["dk"], a["dv"], a["dg"], a["db"], a["ds0"], a["ws"], a["wsb"],
-           a["stream"])
+    rc = f(a["q"], a["k"], a["v"], a["dtype"], a["gate"], a["gk"], a["beta"], a["s0"], a["do"], a["dsf"], a["cu"],
+           a["n_seq"], a["B"], a["T"], a["H"], a["K"], a["V"], a["layout"], a["dq"], a["dk"], a["dv"], a["dg"], a["db"],
+           a["ds0"], a["ws"], a["wsb"], a["stream"])
     return rc, lib.kda_last_error().decode()
 
 
@@ -306,6 +306,9 @@ def _backward_chunked(lib, **kw):
     (dict(dtype=0), UNSUPPORTED, "bf16"),
     (dict(dq=None), INVALID, "null"),
     (dict(wsb=1024), INVALID, "workspace"),
+    (dict(cu=FAKE, n_seq=2, B=2), INVALID, "B == 1"),
+    (dict(n_seq=-1), INVALID, "negative"),
+    (dict(cu=FAKE, n_seq=3, wsb=1 << 20), INVALID, "workspace"),
 ])
 def test_scan_backward_chunked_rejects_bad_arguments(lib, kw, code, msg):
     # every check runs on the host before any launch
@@ -316,10 +319,16 @@ def test_scan_backward_chunked_rejects_bad_arguments(lib, kw, code, msg):
 def test_scan_backward_chunked_workspace_query(lib):
     f = lib.kda_scan_backward_chunked_workspace_bytes
     f.restype = ctypes.c_int
-    f.argtypes = [ctypes.c_int64] * 5 + [ctypes.POINTER(ctypes.c_size_t)]
+    f.argtypes = [ctypes.c_int64] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
     n = ctypes.c_size_t(0)
-    assert f(1, 4096, 96, 128, 128, ctypes.byref(n)) == OK
-    per_chunk_head = n.value / (64 * 96)
+    assert f(1, 4096, 96, 128, 128, 0, ctypes.byref(n)) == OK
+    dense = n.value
+    per_chunk_head = dense / (64 * 96)
     assert 800e3 < per_chunk_head < 1000e3  # the chunk buffers (~880 KB per chunk and head) plus fixed parts
-    assert f(1, 4096, 96, 64, 128, ctypes.byref(n)) == UNSUPPORTED
-    assert f(0, 4096, 96, 128, 128, ctypes.byref(n)) == OK and n.value == 0
+    # packed sequences: the forward's slots, T / 64 + n_seq + 1 chunks per head
+    assert f(1, 4096, 96, 128, 128, 16, ctypes.byref(n)) == OK
+    assert 16 * 96 * 800e3 < n.value - dense < 18 * 96 * 1000e3
+    assert f(1, 4096, 96, 64, 128, 0, ctypes.byref(n)) == UNSUPPORTED
+    assert f(0, 4096, 96, 128, 128, 0, ctypes.byref(n)) == OK and n.value == 0
+    assert f(1, 0, 96, 128, 128, 4, ctypes.byref(n)) == OK and n.value == 0
+    assert f(1, 64, 2, 128, 128, -1, ctypes.byref(n)) == INVALID

@@ -82,3 +82,41 @@ def test_chunked_backward_empty_and_errors(kda):
         kda.scan_backward_chunked(d["q"].to(DEV), d["k"].to(DEV), d["v"].to(DEV), torch.tensor(lg).float().to(DEV),
                                   d["beta"].to(DEV), None, torch.zeros(1, 70, 2, 128, device=DEV), None,
                                   gate_is_log=True, workspace=small)
+
+
+def test_chunked_backward_packed_sequences_match_oracle_per_sequence(kda):
+    # Packed sequences of ragged lengths starting anywhere inside a 64-token chunk (one empty, one of a single
+    # token, one exactly a chunk long, several crossing chunk boundaries), each with its own initial state and
+    # dL/dS_T; tokens before the first and after the last sequence belong to none. Every sequence must get the
+    # gradients of its own scan, an empty one dL/dS_0 = dL/dS_T, and the tokens outside every sequence zero.
+    lens = [70, 0, 129, 1, 64, 33, 200]
+    cu = np.concatenate([[3], 3 + np.cumsum(lens)]).astype(np.int32)
+    N, T, H = len(lens), int(cu[-1]) + 5, 2
+    d = W.random_scan_case(1, T, H, 128, 128, seed=43, dtype="bf16", z_std=2.0, init_std=None)
+    gen = torch.Generator().manual_seed(44)
+    s0 = torch.randn(N, H, 128, 128, generator=gen) * 0.1
+    dsf = torch.randn(N, H, 128, 128, generator=gen) * 0.1
+    do = torch.randn(1, T, H, 128, generator=gen)
+    _, lg = oracle.bounded_decay(d["z"], d["A_log"], d["g_min"], return_log=True)
+    gate = torch.tensor(lg, dtype=torch.float32)
+    out = kda.scan_backward_chunked(d["q"].to(DEV), d["k"].to(DEV), d["v"].to(DEV), gate.to(DEV), d["beta"].to(DEV),
+                                    s0.to(DEV), do.to(DEV), dsf.to(DEV), cu_seqlens=torch.tensor(cu).to(DEV),
+                                    gate_is_log=True)
+    torch.cuda.synchronize()
+    assert not kda.device_status()
+    a_used = np.exp(gate.double().numpy())
+    for n in range(N):
+        a, b = int(cu[n]), int(cu[n + 1])
+        if a == b:
+            np.testing.assert_array_equal(out["d_initial_state"][n].cpu().numpy(), dsf[n].numpy())
+            continue
+        sl = lambda x: x[:, a:b]  # noqa: E731
+        ref = oracle.scan_backward(sl(d["q"]), sl(d["k"]), sl(d["v"]), a_used[:, a:b], sl(d["beta"]), s0[n:n + 1],
+                                   do[:, a:b], dsf[n:n + 1])
+        for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("beta", "dbeta")):
+            check(out[key][:, a:b], ref[name], f"{key} of sequence {n}")
+        check(out["dgate"][:, a:b], ref["alpha"] * a_used[:, a:b], f"dgate of sequence {n}")
+        check(out["d_initial_state"][n:n + 1], ref["initial_state"], f"d_initial_state of sequence {n}")
+    outside = torch.cat([torch.arange(0, int(cu[0])), torch.arange(int(cu[-1]), T)])
+    for key in ("dq", "dk", "dv", "dgate", "dbeta"):
+        assert torch.count_nonzero(out[key][:, outside]) == 0, key
