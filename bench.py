@@ -89,25 +89,25 @@ def gate_bytes(n_elems, es_in=4, es_out=4):
 # taken on, so a sha256 of those sources (comments and blank space left out, see source_digest) is kept
 # beside them and a mismatch at run time reports null.
 MEASURED_TRAFFIC = {
-    # chunk_intra_kernel<2> 404.5 + 357.3 MB; chunk_state_kernel 506.6 + 83.9 MB
-    "prefill": {"bytes": 1352200000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-              "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
-    # decode_bulk_kernel 410.6 + 345.1 MB
-    "decode": {"bytes": 755700000, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "dfbe3ca4ed44294f1662b85f4506abe22c32c93ea6d7e42319af3c3e7838c5a7"},
-    # chunk_intra_kernel<3> 405.1 + 357.6 MB; chunk_state_kernel 506.6 + 84.1 MB (the unbounded gate's prefill)
-    "softplus": {"bytes": 1353400000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-               "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
-    # chunk_intra_kernel<2> 7,911.6 + 7,282.1 MB; chunk_state_kernel 9,227.4 + 1,884.3 MB (16 packed sequences)
-    "varlen": {"bytes": 26305300000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-             "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
-    # chunk_intra_kernel<2> 2,339.6 + 2,120.8 MB; chunk_state_kernel 3,255.0 + 1,060.0 MB (4 x 16384 x 32, V = 256)
-    "long_kv": {"bytes": 8775400000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-              "sha256": "795744c07e2c89b5d70a872352d3a52935fd5f3a53d501fe45e19a140dd9447b"},
-    # bounded_decay_kernel 201,369,600 + 154,498,560; scan_backward_kernel 17,579,054,336 + 27,342,757,376;
-    # bounded_decay_backward_kernel 402,670,080 + 162,126,848 (one backward step from the logits)
-    "backward": {"bytes": 45842476800, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
-                 "sha256": "ed75416944f1f8207064b753d2b529c5b25435b1d8b265a27c5ae9c9afbf9d23"},
+    # chunk_intra_kernel<2> 404.5 + 357.0 MB; chunk_state_kernel 506.6 + 83.7 MB
+    "prefill": {"bytes": 1351800000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+              "sha256": "93945c09b373a8da39759aa9cdf609f006a5ce122ed041363d97f5658609f158"},
+    # decode_bulk_kernel 410.6 + 342.6 MB
+    "decode": {"bytes": 753100000, "files": ['decode.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "734d2492590f985a4aad384a7233e845473b4b9a545a6749e1a2ccec3f938b83"},
+    # chunk_intra_kernel<3> 405.0 + 357.7 MB; chunk_state_kernel 506.6 + 83.8 MB (the unbounded gate's prefill)
+    "softplus": {"bytes": 1353000000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+               "sha256": "93945c09b373a8da39759aa9cdf609f006a5ce122ed041363d97f5658609f158"},
+    # chunk_intra_kernel<2> 7,937.8 + 7,282.0 MB; chunk_state_kernel 9,227.2 + 1,884.4 MB (16 packed sequences)
+    "varlen": {"bytes": 26331400000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+             "sha256": "93945c09b373a8da39759aa9cdf609f006a5ce122ed041363d97f5658609f158"},
+    # chunk_intra_kernel<2> 2,335.6 + 2,120.8 MB; chunk_state_kernel 3,254.9 + 1,059.7 MB (4 x 16384 x 32, V = 256)
+    "long_kv": {"bytes": 8771000000, "files": ['chunk_split.cu', 'chunk_common.cuh', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+              "sha256": "93945c09b373a8da39759aa9cdf609f006a5ce122ed041363d97f5658609f158"},
+    # bounded_decay_kernel 201.4 + 153.4 MB; scan_backward_kernel 19,322.0 + 27,321.0 MB;
+    # bounded_decay_backward_kernel 402.7 + 163.3 MB (one backward step from the logits, exact token adjoint)
+    "backward": {"bytes": 47563800000, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
+                 "sha256": "7a7ad8f22444f39b7918104ba5cb3bc16be94cd42d9be45876612e744271116e"},
 }
 
 
