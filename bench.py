@@ -106,6 +106,12 @@ MEASURED_TRAFFIC = {
               "sha256": "93945c09b373a8da39759aa9cdf609f006a5ce122ed041363d97f5658609f158"},
     # bounded_decay_kernel 201.4 + 153.4 MB; scan_backward_kernel 19,322.0 + 27,321.0 MB;
     # bounded_decay_backward_kernel 402.7 + 163.3 MB (one backward step from the logits, exact token adjoint)
+    # the chunked backward step (gate, forward kernels P and S, prep, pair, inverse, 16 cuBLAS products, dstate,
+    # mask_dgc, dt, da, assemble, gate gradient): 14,731.0 MB read + 6,852.6 MB written
+    "backward_chunked": {"bytes": 21583700000,
+                         "files": ['backward_chunked.cu', 'chunk_split.cu', 'chunk_common.cuh', 'gate.cu', 'gate_math.cuh',
+                                   'common.cuh', 'kda_internal.h'],
+                         "sha256": "bb2e9d9d537528831321cbbdb646a2cd347d8007ac8c0ba271df77dd13d1ae9f"},
     "backward": {"bytes": 47563800000, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                  "sha256": "7a7ad8f22444f39b7918104ba5cb3bc16be94cd42d9be45876612e744271116e"},
 }

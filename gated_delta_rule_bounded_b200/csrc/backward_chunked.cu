@@ -87,16 +87,18 @@ __device__ __forceinline__ void seq_tokens(const BwdC& a, int s, int64_t& c0, in
 // within the row and its number of real tokens nv. The chunks are in the forward split kernels' workspace
 // order, b = slot * H + h: without cu_seqlens slot = n * ceil(T / 64) + j; with them, chunk j of sequence s
 // sits at slot floor(c0 / 64) + s + j, and a slot between two sequences' runs has no tokens (nv = 0).
+// PACKED (cu_seqlens given) is a template argument, so that the dense kernels carry no trace of the search.
+template <bool PACKED>
 __device__ __forceinline__ void chunk_of(const BwdC& a, int b, int& n, int& j, int& h, int& t0, int& nv) {
   h = b % a.H;
-  const int slot = b / a.H;
-  if (!a.cu) {
-    j = slot % a.ncps;
-    n = slot / a.ncps;
+  if constexpr (!PACKED) {
+    j = (b / a.H) % a.ncps;
+    n = b / (a.H * a.ncps);
     t0 = j * CC;
     nv = (int)min((int64_t)CC, a.T - t0);
     return;
   }
+  const int slot = b / a.H;
   n = 0;
   j = 0;
   t0 = 0;
@@ -132,10 +134,11 @@ __device__ __forceinline__ void unpack4(const float4 v, float o[4]) {
 // (zero past the end).
 // Threads 0-127 walk the tokens for channel c (the cumulative sum), threads 128-255 copy v and dO; each takes
 // 8 tokens' loads ahead of their stores.
+template <bool PACKED>
 __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
   const int b = blockIdx.x, tid = threadIdx.x;
   int n, j, h, t0, nv;
-  chunk_of(a, b, n, j, h, t0, nv);
+  chunk_of<PACKED>(a, b, n, j, h, t0, nv);
   const size_t mat = (size_t)b * CC * D;
   if (tid < D) {
     const int c = tid;
@@ -197,10 +200,17 @@ __global__ void __launch_bounds__(256) prep_kernel(BwdC a, Bufs w) {
     const int64_t tt = t0 + tid;
     w.bet[(size_t)b * CC + tid] = tid < nv ? a.beta[n * a.bs[0] + tt * a.bs[1] + h * a.bs[2]] : 0.f;
   }
-  if (nv == 0) {  // a slot without tokens: no forward state was written there
-    for (int e = tid; e < D * D / 4; e += 256)
-      reinterpret_cast<float4*>(w.S0 + (size_t)b * D * D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+}
+
+// Packed sequences: the start state of a slot without tokens (between two sequences' runs), which the forward
+// never writes, is zeroed so that every product stays finite there.
+__global__ void __launch_bounds__(256) zero_empty_slots_kernel(BwdC a, Bufs w) {
+  const int b = blockIdx.x;
+  int n, j, h, t0, nv;
+  chunk_of<true>(a, b, n, j, h, t0, nv);
+  if (nv != 0) return;
+  for (int e = threadIdx.x; e < D * D / 4; e += 256)
+    reinterpret_cast<float4*>(w.S0 + (size_t)b * D * D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // Mq and Mk of one chunk. A warp takes 4 rows t from 4q and 32 columns i (a lane per i), channels 4 at a time.
@@ -505,10 +515,11 @@ __global__ void __launch_bounds__(256, 1) dstate_kernel(BwdC a, Bufs w) {
 
 // dMq = tril(dMq) (diagonal kept); dgamma_C[c] = sum_v dS_C[c][v] S0[c][v] (a warp per row c); dv of the chunk's
 // real rows (dV = TB^T dU, 8 loads ahead of their stores).
+template <bool PACKED>
 __global__ void __launch_bounds__(256) mask_dgc_kernel(BwdC a, Bufs w) {
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int n, j, h, t0, nv;
-  chunk_of(a, b, n, j, h, t0, nv);
+  chunk_of<PACKED>(a, b, n, j, h, t0, nv);
   const size_t sq = (size_t)b * CC * CC, st = (size_t)b * D * D, mat = (size_t)b * CC * D;
   float4 v[8];
 #pragma unroll
@@ -547,10 +558,11 @@ __global__ void __launch_bounds__(64) dt_kernel(Bufs w, float* dbeta_part) {
 
 // dA = strict_tril(dA) in place; dbeta = colsum(dTB * T) + rowsum(dA * Mk) written for the chunk's real rows;
 // dMk = Diag(beta) dA (into dA). A warp per row t (lanes over i).
+template <bool PACKED>
 __global__ void __launch_bounds__(256) da_kernel(BwdC a, Bufs w, const float* dbeta_part) {
   const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int n, j, h, t0, nv;
-  chunk_of(a, b, n, j, h, t0, nv);
+  chunk_of<PACKED>(a, b, n, j, h, t0, nv);
   const size_t sq = (size_t)b * CC * CC;
   for (int t = warp; t < CC; t += 8) {
     const float bt = w.bet[(size_t)b * CC + t];
@@ -684,6 +696,7 @@ __device__ __forceinline__ void col_tile_diag(const float* Kt_, const float* Qt_
   }
 }
 
+template <bool PACKED>
 __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w) {
   extern __shared__ __align__(16) float sa[];
   float* Gt_ = sa;                  // [128][64] swizzled: G2 by channel
@@ -696,7 +709,7 @@ __global__ void __launch_bounds__(256, 1) assemble_kernel(BwdC a, Bufs w) {
   float* DGr = DKr + CC * D;        // [64][128]: dG's row share
   const int b = blockIdx.x, tid = threadIdx.x;
   int n, j, h, t0, nv;
-  chunk_of(a, b, n, j, h, t0, nv);
+  chunk_of<PACKED>(a, b, n, j, h, t0, nv);
   const size_t mat = (size_t)b * CC * D, sq = (size_t)b * CC * CC;
   // dMq and dMk with cp.async; G2, k, q transposed through registers (a thread takes 4 consecutive tokens of
   // one channel, coalesced over the channel; every load in flight at once)
@@ -906,7 +919,12 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
   a.gate_log = fwd.gate_mode == KDA_GATE_LOG;
 
   // 2. per-chunk preparation, Mq and Mk, T and TB
-  prep_kernel<<<NB, 256, 0, s>>>(a, w);
+  if (fwd.cu) {
+    prep_kernel<true><<<NB, 256, 0, s>>>(a, w);
+    zero_empty_slots_kernel<<<NB, 256, 0, s>>>(a, w);
+  } else {
+    prep_kernel<false><<<NB, 256, 0, s>>>(a, w);
+  }
   const int pair_smem = PAIR_SMEM;
   {
     static std::atomic<uint64_t> configured{0};
@@ -918,7 +936,10 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
       const int asm_ = ASSEMBLE_SMEM;
       if ((e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pair_smem)) != cudaSuccess ||
           (e = cudaFuncSetAttribute(dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm)) != cudaSuccess ||
-          (e = cudaFuncSetAttribute(assemble_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, asm_)) != cudaSuccess)
+          (e = cudaFuncSetAttribute(assemble_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, asm_)) !=
+              cudaSuccess ||
+          (e = cudaFuncSetAttribute(assemble_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, asm_)) !=
+              cudaSuccess)
         return e;
       configured.fetch_or(1ull << dev);
     }
@@ -978,7 +999,10 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
     *cublas_status = (int)cs;
     return cudaErrorUnknown;
   }
-  mask_dgc_kernel<<<NB, 256, 0, s>>>(a, w);
+  if (fwd.cu)
+    mask_dgc_kernel<true><<<NB, 256, 0, s>>>(a, w);
+  else
+    mask_dgc_kernel<false><<<NB, 256, 0, s>>>(a, w);
   dt_kernel<<<NB, 64, 0, s>>>(w, dbeta_part);  // X = dT = dTB Diag(beta); dbeta_part = colsum(dTB * T)
   // dA = -(T^T dT) T^T: the product T^T dT into dA, then -dA T^T into X (two products, reusing the buffers)
   G(true, false, CC, CC, CC, 1.f, w.Tm, CC, s64, w.X, CC, s64, 0.f, w.dA, CC, s64);
@@ -988,8 +1012,13 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
     return cudaErrorUnknown;
   }
   std::swap(w.dA, w.X);  // dA now names the result
-  da_kernel<<<NB, 256, 0, s>>>(a, w, dbeta_part);
-  assemble_kernel<<<NB, 256, ASSEMBLE_SMEM, s>>>(a, w);
+  if (fwd.cu) {
+    da_kernel<true><<<NB, 256, 0, s>>>(a, w, dbeta_part);
+    assemble_kernel<true><<<NB, 256, ASSEMBLE_SMEM, s>>>(a, w);
+  } else {
+    da_kernel<false><<<NB, 256, 0, s>>>(a, w, dbeta_part);
+    assemble_kernel<false><<<NB, 256, ASSEMBLE_SMEM, s>>>(a, w);
+  }
   return cudaGetLastError();
 }
 
