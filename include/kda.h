@@ -342,7 +342,10 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
  * cuBLAS in fp32 with TF32 tensor cores). Arguments, layouts and outputs as for
  * kda_scan_backward, packed sequences (cu_seqlens, n_seq; B = 1; states per
  * sequence) included. Supported: bf16 q, k, v with K = V = 128
- * (KDA_ERR_UNSUPPORTED otherwise). The chunk-start states come from the bf16
+ * (KDA_ERR_UNSUPPORTED otherwise). With KDA_GATE_ALPHA the gate's gradient is
+ * formed as dL/dalpha = (dL/dlog alpha) / alpha: its absolute error grows like
+ * 1/alpha for small alpha, and it is 0 where alpha = 0; gates near zero take
+ * KDA_GATE_LOG or kda_scan_backward. The chunk-start states come from the bf16
  * tensor-core forward, so the gradients carry its rounding (relative RMS errors
  * near 1e-3) where kda_scan_backward's token-level adjoint is exact fp32. The
  * workspace (kda_scan_backward_chunked_workspace_bytes for the same B, T, H, K, V
