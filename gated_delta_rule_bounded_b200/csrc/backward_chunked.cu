@@ -213,48 +213,61 @@ __global__ void __launch_bounds__(256) zero_empty_slots_kernel(BwdC a, Bufs w) {
     reinterpret_cast<float4*>(w.S0 + (size_t)b * D * D)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// Mq and Mk of one chunk. A warp takes 4 rows t from 4q and 32 columns i (a lane per i), channels 4 at a time.
-// For the columns before the rows' quad (i < 4q <= t) the decay ratio factors at the reference r = 4q - 1:
+// Mq and Mk of one chunk, split over two CTAs by row quad (rows 4q .. 4q + 3; CTA `half` takes the quads of
+// its parity). A warp takes one quad and 32 columns i at a time (a lane per i), channels 4 at a time. For the
+// columns before the quad (i < 4q <= t) the decay ratio factors at the reference r = 4q - 1:
 // 2^{G_t - G_i} = 2^{G_t - G_r} 2^{G_r - G_i}, both factors <= 1 (a factor that flushes to zero bounds the
 // exact ratio, which is then below 2^-126 as well); q_t and k_t come pre-scaled by the first factor (QA, KA),
 // so a pair costs two FMAs and a lane one exponential per channel. The 4x4 blocks on the diagonal form every
 // ratio directly. Rows of k and G are padded to 132 floats (lane-indexed float4 loads hit distinct banks).
-constexpr int PAIR_SMEM = (2 * CC * 132 + 2 * CC * D) * 4;
-__global__ void __launch_bounds__(256, 1) pair_kernel(Bufs w) {
+// About 100 KB of shared memory: two CTAs per SM.
+constexpr int PAIR_SMEM = (2 * CC * 132 + 2 * (CC / 2) * D) * 4;
+__global__ void __launch_bounds__(256, 2) pair_kernel(Bufs w) {
   constexpr int PR = 132;
   extern __shared__ __align__(16) float sp[];
   float* Ks = sp;              // [64][132]
   float* Gs = Ks + CC * PR;    // [64][132]
-  float* QA = Gs + CC * PR;    // [64][128]: q_t, then q_t 2^{G_t - G_r(t)}
-  float* KA = QA + CC * D;     // [64][128]: k_t 2^{G_t - G_r(t)}
-  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* QA = Gs + CC * PR;    // [32][128], the CTA's quads in order: q_t, then q_t 2^{G_t - G_r(t)}
+  float* KA = QA + CC / 2 * D; // [32][128]: k_t 2^{G_t - G_r(t)}
+  const int b = blockIdx.x >> 1, half = blockIdx.x & 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t mat = (size_t)b * CC * D, sq = (size_t)b * CC * CC;
+  auto row_of = [&](int lr) { return 4 * (2 * (lr >> 2) + half) + (lr & 3); };  // local row -> token row
   {
-    float4 kv[8], gv[8], qv[8];
+    float4 kv[8], gv[8], qv[4];
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       kv[m] = reinterpret_cast<const float4*>(w.Kf + mat)[tid + 256 * m];
       gv[m] = reinterpret_cast<const float4*>(w.G2 + mat)[tid + 256 * m];
-      qv[m] = reinterpret_cast<const float4*>(w.Qf + mat)[tid + 256 * m];
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int e = tid + 256 * m, lr = e >> 5, c4 = e & 31;
+      qv[m] = reinterpret_cast<const float4*>(w.Qf + mat + (size_t)row_of(lr) * D)[c4];
     }
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       const int e = tid + 256 * m, t = e >> 5, c = 4 * (e & 31);
       *reinterpret_cast<float4*>(Ks + t * PR + c) = kv[m];
       *reinterpret_cast<float4*>(Gs + t * PR + c) = gv[m];
-      *reinterpret_cast<float4*>(QA + t * D + c) = qv[m];
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int e = tid + 256 * m;
+      reinterpret_cast<float4*>(QA)[e] = qv[m];
     }
   }
   __syncthreads();
-  // the 4x4 diagonal blocks: warp w takes quads 2w and 2w + 1, a lane one pair (t, i) of them
-  {
-    const int q = 2 * warp + (lane >> 4), r = (lane >> 2) & 3, ii = lane & 3;
-    const int t = 4 * q + r, i = 4 * q + ii;
+  // the 4x4 diagonal blocks of the CTA's quads: warps 0-3, two quads a warp, a lane one pair (t, i)
+  if (warp < 4) {
+    const int qi = 2 * warp + (lane >> 4), r = (lane >> 2) & 3, ii = lane & 3;
+    const int q = 2 * qi + half, t = 4 * q + r, i = 4 * q + ii;
+    const float* qrow = QA + (4 * qi + r) * D;
     float mq = 0.f, mk = 0.f;
     if (ii <= r) {
 #pragma unroll 4
       for (int c = 0; c < D; c += 4) {
-        const float4 qv = *reinterpret_cast<const float4*>(QA + t * D + c);
+        const float4 qv = *reinterpret_cast<const float4*>(qrow + c);
         const float4 kt = *reinterpret_cast<const float4*>(Ks + t * PR + c);
         const float4 gt = *reinterpret_cast<const float4*>(Gs + t * PR + c);
         const float4 kv = *reinterpret_cast<const float4*>(Ks + i * PR + c);
@@ -274,29 +287,30 @@ __global__ void __launch_bounds__(256, 1) pair_kernel(Bufs w) {
   }
   __syncthreads();  // raw q read; scale in place
 #pragma unroll 2
-  for (int e = tid; e < CC * D / 4; e += 256) {
-    const int t = e >> 5, c = 4 * (e & 31);
+  for (int e = tid; e < CC / 2 * D / 4; e += 256) {
+    const int lr = e >> 5, c = 4 * (e & 31), t = row_of(lr);
     float4 qa = make_float4(0.f, 0.f, 0.f, 0.f), ka = qa;
     if (t >= 4) {
       const int r = (t & ~3) - 1;
       const float4 g = *reinterpret_cast<const float4*>(Gs + t * PR + c);
       const float4 gr = *reinterpret_cast<const float4*>(Gs + r * PR + c);
-      const float4 qv = *reinterpret_cast<const float4*>(QA + t * D + c);
+      const float4 qv = *reinterpret_cast<const float4*>(QA + lr * D + c);
       const float4 kv = *reinterpret_cast<const float4*>(Ks + t * PR + c);
       const float ax = ex2f(g.x - gr.x), ay = ex2f(g.y - gr.y), az = ex2f(g.z - gr.z), aw = ex2f(g.w - gr.w);
       qa = make_float4(qv.x * ax, qv.y * ay, qv.z * az, qv.w * aw);
       ka = make_float4(kv.x * ax, kv.y * ay, kv.z * az, kv.w * aw);
     }
-    *reinterpret_cast<float4*>(QA + t * D + c) = qa;
-    *reinterpret_cast<float4*>(KA + t * D + c) = ka;
+    *reinterpret_cast<float4*>(QA + lr * D + c) = qa;
+    *reinterpret_cast<float4*>(KA + lr * D + c) = ka;
   }
   __syncthreads();
-  // units (rows 4q.., columns 32 hf..): warp w takes q = w and w + 8 with hf = 0, q = w + 8 with hf = 1
-  // ((q = w, hf = 1) lies above the diagonal: zeros)
+  // warp w: quad q = 2w + half, columns 32 hf .. 32 hf + 31 for hf = 0, 1
+  const int q = 2 * warp + half, tq = 4 * q;
+  const float* qa_ = QA + 4 * warp * D;
+  const float* ka_ = KA + 4 * warp * D;
 #pragma unroll 1
-  for (int k = 0; k < 4; ++k) {
-    const int u = warp + 8 * k, q = u & 15, hf = u >> 4;
-    const int i = 32 * hf + lane, tq = 4 * q;
+  for (int hf = 0; hf < 2; ++hf) {
+    const int i = 32 * hf + lane;
     float mq[4] = {0.f, 0.f, 0.f, 0.f}, mk[4] = {0.f, 0.f, 0.f, 0.f};
     if (32 * hf < tq) {  // some column before the quad
       const float* ki_ = Ks + i * PR;
@@ -311,8 +325,8 @@ __global__ void __launch_bounds__(256, 1) pair_kernel(Bufs w) {
         const float kb2 = kv.z * ex2f(gr.z - gv.z), kb3 = kv.w * ex2f(gr.w - gv.w);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const float4 qa = *reinterpret_cast<const float4*>(QA + (tq + r) * D + c);
-          const float4 ka = *reinterpret_cast<const float4*>(KA + (tq + r) * D + c);
+          const float4 qa = *reinterpret_cast<const float4*>(qa_ + r * D + c);
+          const float4 ka = *reinterpret_cast<const float4*>(ka_ + r * D + c);
           mq[r] = fmaf(qa.x, kb0, fmaf(qa.y, kb1, fmaf(qa.z, kb2, fmaf(qa.w, kb3, mq[r]))));
           mk[r] = fmaf(ka.x, kb0, fmaf(ka.y, kb1, fmaf(ka.z, kb2, fmaf(ka.w, kb3, mk[r]))));
         }
@@ -944,7 +958,7 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
       configured.fetch_or(1ull << dev);
     }
   }
-  pair_kernel<<<NB, 256, pair_smem, s>>>(w);
+  pair_kernel<<<2 * NB, 256, pair_smem, s>>>(w);
   inverse_kernel<<<NB, 64, 0, s>>>(w);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 

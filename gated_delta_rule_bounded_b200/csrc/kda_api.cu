@@ -577,7 +577,7 @@ int kda_scan_backward_chunked(const void* q, const void* k, const void* v, kda_d
   if (!q || !k || !v || !gate || !beta || !d_o || !dq || !dk || !dv || !dgate || !dbeta)
     return fail(KDA_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
   const int64_t n_slots = cu_seqlens ? T / 64 + N + 1 : (T + 63) / 64 * B;
-  if (T > INT32_MAX || n_slots * H > INT32_MAX || N > INT32_MAX)
+  if (T > INT32_MAX || n_slots * H > INT32_MAX / 2 || N > INT32_MAX)  // two CTAs per chunk-head in one kernel
     return fail(KDA_ERR_UNSUPPORTED, "%s: T too large", fn);
   const size_t need = chunked_bwd_bytes(B, T, H, cu_seqlens ? N : 0);
   if (!workspace || workspace_bytes < need)
