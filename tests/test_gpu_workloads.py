@@ -1,7 +1,9 @@
 """Full-size parity of the calls the benchmark times: kda_prefill_logits on the three prefill
-workloads, and kda_scan_backward_chunked on the 4096-token workload (sampled heads). The prefill workloads are the single 4096-token sequence (H = 96, K = V = 128, zero initial state), the 16 packed
-sequences of 512..8192 tokens with their own initial states, and the long K != V case (B = 4,
-T = 16384, H = 32, V = 256) run whole and split at T = 8192 and resumed from the final state.
+workloads, and kda_scan_backward_chunked on the 4096-token workload (sampled heads). The prefill
+workloads are the single 4096-token sequence (H = 96, K = V = 128, zero initial state), the 16
+packed sequences of 512..8192 tokens with their own initial states, and the long K != V case
+(B = 4, T = 16384, H = 32, V = 256) run whole and split at T = 8192 and resumed from the final
+state.
 
 The GPU computes every head with the same launch configuration as the benchmark (the two-kernel
 path, the gate evaluated from the logits inside the kernels); the fp64 oracle runs on a sample of
