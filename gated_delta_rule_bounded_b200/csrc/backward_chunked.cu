@@ -842,14 +842,22 @@ cublasStatus_t rm_gemm(cublasHandle_t hd, bool ta, bool tb, int M, int N, int K,
                                     CUBLAS_COMPUTE_32F_FAST_TF32, CUBLAS_GEMM_DEFAULT);
 }
 
-cublasHandle_t handle_for_device() {
+// One cuBLAS handle per device, created on first use, and a per-device lock that a call holds from setting the
+// handle's stream and workspace until its last product is enqueued (host threads sharing a device take turns;
+// enqueueing does not wait for the GPU).
+struct DeviceBlas {
+  std::mutex use;
+  cublasHandle_t handle = nullptr;
+};
+
+DeviceBlas* blas_for_device() {
   static std::mutex mu;
-  static cublasHandle_t handles[64] = {};
+  static DeviceBlas blas[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!handles[dev] && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
-  return handles[dev];
+  if (!blas[dev].handle && cublasCreate(&blas[dev].handle) != CUBLAS_STATUS_SUCCESS) blas[dev].handle = nullptr;
+  return blas[dev].handle ? &blas[dev] : nullptr;
 }
 
 constexpr size_t CUBLAS_WS = 32u << 20;  // handed to cuBLAS, so that its products allocate nothing per call
@@ -962,11 +970,13 @@ cudaError_t launch_chunked_backward(const ScanParams& fwd, const float* d_o, con
   inverse_kernel<<<NB, 64, 0, s>>>(w);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  cublasHandle_t hd = handle_for_device();
-  if (!hd) {
+  DeviceBlas* blas = blas_for_device();
+  if (!blas) {
     *cublas_status = -1;
     return cudaErrorUnknown;
   }
+  std::lock_guard<std::mutex> in_use(blas->use);
+  cublasHandle_t hd = blas->handle;
   if (cublasSetStream(hd, s) != CUBLAS_STATUS_SUCCESS ||
       cublasSetWorkspace(hd, base + L.off[32], CUBLAS_WS) != CUBLAS_STATUS_SUCCESS) {
     *cublas_status = -2;

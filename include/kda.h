@@ -348,11 +348,13 @@ int kda_scan_backward(const void* q, const void* k, const void* v, kda_dtype dty
  * KDA_GATE_LOG or kda_scan_backward. The chunk-start states come from the bf16
  * tensor-core forward, so the gradients carry its rounding (relative RMS errors
  * near 1e-3) where kda_scan_backward's token-level adjoint is exact fp32. The
- * workspace (kda_scan_backward_chunked_workspace_bytes for the same B, T, H, K, V
- * and n_seq, 0 without cu_seqlens; about 880 KB per chunk and head, plus n_seq + 1
- * chunks per head with cu_seqlens; KDA_ERR_INVALID_ARG if smaller) holds every intermediate; cuBLAS creates its handle (device memory)
- * on the first call on each device and is given a part of the workspace for
- * its own scratch.
+ * workspace (kda_scan_backward_chunked_workspace_bytes for the same B, T, H, K,
+ * V and n_seq, 0 without cu_seqlens; about 880 KB per chunk and head, plus
+ * n_seq + 1 chunks per head with cu_seqlens; KDA_ERR_INVALID_ARG if smaller)
+ * holds every intermediate. cuBLAS creates its handle (device memory) on the
+ * first call on each device and is given a part of the workspace for its own
+ * scratch; host threads calling on the same device take turns while a call
+ * enqueues its work (the call does not wait for the GPU).
  * ------------------------------------------------------------------------- */
 int kda_scan_backward_chunked_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                                               int64_t n_seq, size_t* bytes);
