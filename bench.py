@@ -107,11 +107,11 @@ MEASURED_TRAFFIC = {
     # bounded_decay_kernel 201.4 + 153.4 MB; scan_backward_kernel 19,322.0 + 27,321.0 MB;
     # bounded_decay_backward_kernel 402.7 + 163.3 MB (one backward step from the logits, exact token adjoint)
     # the chunked backward step (gate, forward kernels P and S, prep, pair, inverse, 16 cuBLAS products, dstate,
-    # mask_dgc, dt, da, assemble, gate gradient): 14,727.8 MB read + 6,850.8 MB written
-    "backward_chunked": {"bytes": 21578600000,
+    # mask_dgc, dt, da, assemble, gate gradient): 14,730.3 MB read + 6,846.4 MB written
+    "backward_chunked": {"bytes": 21576700000,
                          "files": ['backward_chunked.cu', 'chunk_split.cu', 'chunk_common.cuh', 'gate.cu', 'gate_math.cuh',
                                    'common.cuh', 'kda_internal.h'],
-                         "sha256": "4775726f6924576d30098c92145cc28d9957420572f8a89165e6b28f4d6ce3cb"},
+                         "sha256": "d699bdefb43595a5b8f949e9df41d52f4a85e740593fda122b6cdf073a328ee6"},
     "backward": {"bytes": 47563800000, "files": ['backward.cu', 'gate.cu', 'gate_math.cuh', 'common.cuh', 'kda_internal.h'],
                  "sha256": "7a7ad8f22444f39b7918104ba5cb3bc16be94cd42d9be45876612e744271116e"},
 }
